@@ -1,0 +1,235 @@
+/*
+ * switch_oracle.c -- plain fp64 CPU oracle for the Switch Transformer sparse
+ * FFN layer forward pass.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file; only the test-suite, the smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header or helper with the CUDA
+ * library.
+ *
+ * Every step is the plain definition, in the order the sources give it, in
+ * double precision, with no blocking, fusion or reordering:
+ *
+ *   logits     h(x) = W_r . x                       (llm-papers-study
+ *              "精读 06 | Switch Transformers", §3.1, router logits; Incredible.AI
+ *              "Switch Transformer - Scaling to Trillion Parameter Models",
+ *              section "Router Implementation")
+ *   gate       p_i(x) = exp(h_i) / sum_j exp(h_j)   (llm-papers-study §3.1,
+ *              softmax formula), evaluated with the row maximum subtracted,
+ *              which leaves every p_i unchanged in exact arithmetic
+ *   top-1      i* = argmax_i p_i(x), lowest index on ties (llm-papers-study
+ *              §3.2; the tie rule is not stated by the sources)
+ *   capacity   C = ceil(T / N * c)                  (llm-papers-study §3.4
+ *              expert-capacity formula; rounding reading: ceil)
+ *   overflow   tokens beyond the first C routed to an expert, in token order,
+ *              are dropped (Incredible.AI "MoE Layer"; kasblo "Expert
+ *              Capacityはtokenの受付上限"; byhand.ai "Switch Transformer by
+ *              Hand", walkthrough step 7)
+ *   aux        N * sum_i f_i P_i, f_i = count_i / T before capacity,
+ *              P_i = mean over all T tokens of p_i  (llm-papers-study §3.3)
+ *   output     y = p_{i*}(x) * E_{i*}(x),  E(x) = W_out . ReLU(W_in . x);
+ *              y = 0 for a dropped token (llm-papers-study §3.2 and §3.4)
+ *
+ * Element types: activations and expert weights are read either as IEEE
+ * binary32 (dtype 0) or as bfloat16 bit patterns (dtype 1); both convert to
+ * double exactly.  The router weight and the optional logit bias are binary32.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+
+/* Exact conversion of element i of a binary32 or bfloat16 array to double. */
+static double load_elem(const void *base, int dtype, int64_t i)
+{
+    if (dtype == ORACLE_BF16) {
+        uint16_t bits = ((const uint16_t *)base)[i];
+        uint32_t wide = (uint32_t)bits << 16;
+        float f;
+        memcpy(&f, &wide, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float *)base)[i];
+}
+
+/* Expert capacity C = ceil(T / N * c).  A product within 1e-9 of an integer is
+ * taken as that integer, so that e.g. 512/8*1.5 gives 96 whatever the binary
+ * rounding of c.  At least 1.  Returns -1 for arguments without meaning. */
+int64_t oracle_capacity(int64_t T, int32_t N, double c)
+{
+    if (T < 0 || N < 1 || !(c > 0.0) || !isfinite(c))
+        return -1;
+    double exact = (double)T / (double)N * c;
+    double nearest = floor(exact + 0.5);
+    double cap = fabs(exact - nearest) <= 1e-9 ? nearest : ceil(exact);
+    if (cap < 1.0)
+        cap = 1.0;
+    return (int64_t)cap;
+}
+
+/* Router logits h[t,i] = sum_k x[t,k] * W_r[i,k] (+ bias[i]), all in double.
+ * x is [T,d] row-major, W_r is [N,d] row-major, h is [T,N]. */
+void oracle_router_logits(int64_t T, int32_t d, int32_t N, const void *x, int x_dtype,
+                          const float *w_r, const float *bias, double *h)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t i = 0; i < N; ++i) {
+            double acc = 0.0;
+            for (int32_t k = 0; k < d; ++k)
+                acc += load_elem(x, x_dtype, t * (int64_t)d + k) * (double)w_r[(int64_t)i * d + k];
+            if (bias)
+                acc += (double)bias[i];
+            h[t * (int64_t)N + i] = acc;
+        }
+    }
+}
+
+/* Softmax, top-1 and gate for every row of h[T,N].
+ *   expert[t] = lowest i with h[t,i] equal to the row maximum
+ *   gate[t]   = p[t, expert[t]]
+ *   margin[t] = row maximum minus the largest logit of any other expert
+ *               (+inf when N == 1)
+ *   prob_sum[i] = sum over t of p[t,i], accumulated in token order
+ *   probs (optional, [T,N]) receives every p[t,i]. */
+void oracle_softmax_top1(int64_t T, int32_t N, const double *h, int32_t *expert, double *gate,
+                         double *margin, double *prob_sum, double *probs)
+{
+    double *p = probs ? probs : (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * (size_t)N);
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const double *row = h + t * (int64_t)N;
+        double m = row[0];
+        int32_t arg = 0;
+        for (int32_t i = 1; i < N; ++i) {
+            if (row[i] > m) {
+                m = row[i];
+                arg = i;
+            }
+        }
+        double runner_up = -INFINITY;
+        for (int32_t i = 0; i < N; ++i)
+            if (i != arg && row[i] > runner_up)
+                runner_up = row[i];
+        double denom = 0.0;
+        for (int32_t i = 0; i < N; ++i)
+            denom += exp(row[i] - m);
+        for (int32_t i = 0; i < N; ++i)
+            p[t * (int64_t)N + i] = exp(row[i] - m) / denom;
+        expert[t] = arg;
+        gate[t] = p[t * (int64_t)N + arg];
+        margin[t] = (N == 1) ? INFINITY : m - runner_up;
+    }
+    for (int32_t i = 0; i < N; ++i)
+        prob_sum[i] = 0.0;
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t i = 0; i < N; ++i)
+            prob_sum[i] += p[t * (int64_t)N + i];
+    if (!probs)
+        free(p);
+}
+
+/* Capacity assignment in token order.
+ *   counts[i]         = number of tokens routed to expert i (before capacity)
+ *   slot[t]           = number of earlier tokens routed to the same expert,
+ *                       or -1 when that number is >= C (dropped)
+ *   slot_token[i*C+s] = the token holding slot s of expert i, -1 if empty. */
+void oracle_assign(int64_t T, int32_t N, int64_t C, const int32_t *expert, int32_t *slot,
+                   int32_t *counts, int32_t *slot_token)
+{
+    for (int32_t i = 0; i < N; ++i)
+        counts[i] = 0;
+    for (int64_t s = 0; s < (int64_t)N * C; ++s)
+        slot_token[s] = -1;
+    for (int64_t t = 0; t < T; ++t) {
+        int32_t e = expert[t];
+        int32_t position = counts[e];
+        counts[e] = position + 1;
+        if (position < C) {
+            slot[t] = position;
+            slot_token[(int64_t)e * C + position] = (int32_t)t;
+        } else {
+            slot[t] = -1;
+        }
+    }
+}
+
+/* Load-balancing loss without the alpha weight: N * sum_i f_i * P_i with
+ * f_i = counts[i] / T and P_i = prob_sum[i] / T. */
+double oracle_aux(int64_t T, int32_t N, const int32_t *counts, const double *prob_sum)
+{
+    double total = 0.0;
+    for (int32_t i = 0; i < N; ++i) {
+        double f = (double)counts[i] / (double)T;
+        double P = prob_sum[i] / (double)T;
+        total += f * P;
+    }
+    return (double)N * total;
+}
+
+/* One expert FFN applied to one token and scaled by its gate:
+ *   u[j] = max(0, sum_k W_in[j,k] * x[k]),   j < F
+ *   y[k] = gate * sum_j W_out[k,j] * u[j],   k < d
+ * W_in is [F,d] and W_out is [d,F], both row-major (nn.Linear layout). */
+void oracle_expert_row(int32_t d, int32_t F, const void *x_row, int x_dtype, const void *w_in,
+                       const void *w_out, int w_dtype, double gate, double *y_row)
+{
+    double *x = (double *)malloc(sizeof(double) * (size_t)d);
+    double *u = (double *)malloc(sizeof(double) * (size_t)F);
+    for (int32_t k = 0; k < d; ++k)
+        x[k] = load_elem(x_row, x_dtype, k);
+    for (int32_t j = 0; j < F; ++j) {
+        double acc = 0.0;
+        for (int32_t k = 0; k < d; ++k)
+            acc += load_elem(w_in, w_dtype, (int64_t)j * d + k) * x[k];
+        u[j] = acc > 0.0 ? acc : 0.0;
+    }
+    for (int32_t k = 0; k < d; ++k) {
+        double acc = 0.0;
+        for (int32_t j = 0; j < F; ++j)
+            acc += load_elem(w_out, w_dtype, (int64_t)k * F + j) * u[j];
+        y_row[k] = gate * acc;
+    }
+    free(x);
+    free(u);
+}
+
+/* Layer outputs for a list of tokens: row r of y (shape [n_rows, d]) is the
+ * output of token rows[r].  Kept tokens go through their expert and are
+ * scaled by their gate; dropped tokens (slot -1) get an all-zero row.
+ * w_in is [N,F,d] and w_out is [N,d,F]. */
+void oracle_output_rows(int32_t d, int32_t F, int64_t n_rows, const int64_t *rows, const void *x,
+                        int x_dtype, const void *w_in, const void *w_out, int w_dtype,
+                        const int32_t *expert, const int32_t *slot, const double *gate, double *y)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        int64_t t = rows[r];
+        double *out = y + r * (int64_t)d;
+        if (slot[t] < 0) {
+            for (int32_t k = 0; k < d; ++k)
+                out[k] = 0.0;
+            continue;
+        }
+        int64_t e = expert[t];
+        size_t esize = (w_dtype == ORACLE_BF16) ? 2 : 4;
+        const char *win_e = (const char *)w_in + (size_t)e * (size_t)F * (size_t)d * esize;
+        const char *wout_e = (const char *)w_out + (size_t)e * (size_t)d * (size_t)F * esize;
+        const char *x_t = (const char *)x + (size_t)t * (size_t)d * (x_dtype == ORACLE_BF16 ? 2 : 4);
+        oracle_expert_row(d, F, x_t, x_dtype, win_e, wout_e, w_dtype, gate[t], out);
+    }
+}
+
+/* Number of OpenMP threads the parallel loops above use (1 without OpenMP). */
+int oracle_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

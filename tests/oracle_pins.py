@@ -1,0 +1,349 @@
+"""Checks that pin the fp64 oracle to facts fixed outside the oracle itself.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError
+when the oracle disagrees with a worked example printed by the sources, a
+closed form, an invariant, a special case that reduces to a library routine,
+or brute force on tiny inputs.  The same functions run against the real
+oracle (``test_oracle_pins.py``) and against deliberately broken copies of it
+(``test_oracle_mutants.py``), which shows that each plausible mistake is
+caught by at least one pin.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+from pathlib import Path
+
+import numpy as np
+import scipy.special
+
+GOLDEN = Path(__file__).resolve().parent / "golden"
+
+
+def golden(name: str) -> dict:
+    return json.loads((GOLDEN / name).read_text())
+
+
+def _one_hot_routing(assignment, N, scale=4.0):
+    """Inputs whose router logits are scale * one_hot(assignment[t]): x[t] = e_(a_t), W_r = scale * I."""
+    T = len(assignment)
+    x = np.zeros((T, N), dtype=np.float32)
+    x[np.arange(T), assignment] = 1.0
+    w_r = (scale * np.eye(N)).astype(np.float32)
+    return x, w_r
+
+
+def _identity_experts(N, d):
+    """Experts with W_in = W_out = I, so that E(x) = ReLU(x)."""
+    eye = np.eye(d, dtype=np.float32)
+    return np.stack([eye] * N), np.stack([eye] * N)
+
+
+def _random_problem(rng, T, d, F, N, with_bias=True):
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    w_r = (rng.standard_normal((N, d)) * 0.5).astype(np.float32)
+    bias = (rng.standard_normal(N) * 0.3).astype(np.float32) if with_bias else None
+    w_in = (rng.standard_normal((N, F, d)) / np.sqrt(d)).astype(np.float32)
+    w_out = (rng.standard_normal((N, d, F)) / np.sqrt(F)).astype(np.float32)
+    return x, w_r, bias, w_in, w_out
+
+
+# --------------------------------------------------------------------------
+# Worked examples printed by the sources
+# --------------------------------------------------------------------------
+
+def pin_capacity_examples(o):
+    for case in golden("capacity_examples.json")["cases"]:
+        got = o.capacity(case["T"], case["N"], case["c"])
+        assert got == case["C"], (case, got)
+
+
+def pin_workload_capacities(o):
+    # C = ceil(T / N * c) at the five workload shapes (all exact integers).
+    for T, N, c, C in [(64, 4, 1.0, 16), (8192, 8, 1.25, 1280), (65536, 128, 1.0, 512),
+                       (131072, 128, 1.25, 1280), (32768, 64, 0.5, 256), (32768, 64, 1.0, 512),
+                       (32768, 64, 1.25, 640), (32768, 64, 2.0, 1024)]:
+        assert o.capacity(T, N, c) == C, (T, N, c)
+    # Non-integer quotients round up: 10 / 3 -> 4, 7 / 2 * 1.1 = 3.85 -> 4.
+    assert o.capacity(10, 3, 1.0) == 4
+    assert o.capacity(7, 2, 1.1) == 4
+    assert o.capacity(1, 64, 0.5) == 1
+
+
+def pin_overflow_16tok(o):
+    g = golden("overflow_16tok.json")
+    expert = np.array(g["expert"], dtype=np.int32)
+    a = o.assign(expert, g["N"], o.capacity(len(expert), g["N"], g["c"]))
+    assert a["counts"].tolist() == g["counts"]
+    dropped = np.flatnonzero(a["slot"] < 0).tolist()
+    assert dropped == g["dropped_tokens"], dropped
+    assert int((a["slot"] >= 0).sum()) == g["kept"]
+
+
+def pin_overflow_16tok_routed(o):
+    # The same example driven through the router: one-hot inputs make the
+    # logits select the listed experts.
+    g = golden("overflow_16tok.json")
+    x, w_r = _one_hot_routing(g["expert"], g["N"])
+    r = o.route(x, w_r, capacity_factor=g["c"])
+    assert r["capacity"] == g["capacity"]
+    assert r["expert"].tolist() == g["expert"]
+    assert np.flatnonzero(r["slot"] < 0).tolist() == g["dropped_tokens"]
+
+
+def pin_p1_moe_layer_example(o):
+    g = golden("p1_moe_layer_example.json")
+    a = o.assign(np.array(g["expert"], dtype=np.int32), g["N"], g["capacity"])
+    for e, kept in enumerate(g["kept_by_expert"]):
+        assert a["slot_token"][e].tolist() == kept, (e, a["slot_token"][e])
+
+
+def pin_byhand_overflow(o):
+    g = golden("byhand_5tok.json")
+    rows = g["switch_matrix_rows"]
+    w_r = np.array([rows["A"], rows["B"], rows["C"]], dtype=np.float32)
+    z = np.array(g["Z"], dtype=np.float32)
+    h = o.router_logits(z, w_r)
+    assert h[4].tolist() == g["gate_values_Z5"]
+    w_in, w_out = _identity_experts(3, 3)
+    r = o.layer_fwd(z, w_r, w_in, w_out, capacity=g["capacity"])
+    assert r["expert"].tolist() == g["expert"]
+    assert r["slot"].tolist() == g["slot"]
+    assert r["counts"].tolist() == g["counts"]
+    # The dropped feature gets a zero layer output, so x + y passes it through unchanged.
+    for t in g["dropped"]:
+        assert np.all(r["y"][t] == 0.0)
+        assert np.array_equal(z[t] + r["y"][t], z[t])
+    kept = [t for t in range(5) if t not in g["dropped"]]
+    assert all(np.any(r["y"][t] != 0.0) for t in kept)
+
+
+def pin_p1_softmax_table(o):
+    g = golden("p1_softmax_table.json")
+    p = np.array(g["probs"], dtype=np.float64)
+    # Logits whose softmax is the printed row: h = ln p (a zero probability
+    # becomes a logit so low that its exponential underflows to 0).
+    h = np.where(p > 0, np.log(np.where(p > 0, p, 1.0)), -1000.0)
+    r = o.softmax_top1(h, want_probs=True)
+    assert r["expert"].tolist() == g["selected"]
+    assert np.allclose(r["probs"], p, rtol=0, atol=1e-15)
+    counts = np.bincount(r["expert"], minlength=4).astype(np.int32)
+    assert np.allclose(counts / 5.0, g["derived_f"], atol=0)
+    assert np.allclose(r["prob_sum"] / 5.0, g["derived_P"], atol=1e-15)
+    assert abs(o.aux(5, counts, r["prob_sum"]) - g["derived_aux"]) < 1e-12
+
+
+def pin_p1_aux_tables(o):
+    for case in golden("p1_aux_tables.json")["cases"]:
+        got = o.aux(case["T"], np.array(case["counts"], np.int32), np.array(case["prob_sum"], np.float64))
+        assert abs(got - case["aux"]) < 1e-12, (case["name"], got)
+        assert abs(got / 4 - case["sum_fP"]) < 1e-12
+
+
+def pin_kasblo_gate(o):
+    g = golden("kasblo_gate_063.json")
+    p = np.array(g["probs"], dtype=np.float64)
+    # One token, d = N = 4; x = e_0 and W_r[:, 0] = ln p gives logits ln p.
+    x = np.zeros((1, 4), dtype=np.float32)
+    x[0, 0] = 1.0
+    w_r = np.zeros((4, 4), dtype=np.float32)
+    w_r[:, 0] = np.log(p).astype(np.float32)
+    w_in, w_out = _identity_experts(4, 4)
+    r = o.layer_fwd(x, w_r, w_in, w_out, capacity=1)
+    assert r["expert"][0] == g["selected"]
+    assert abs(r["gate"][0] - g["gate"]) < 1e-6
+    # E(x) = ReLU(e_0) = e_0, so y = 0.63 * e_0.
+    assert np.allclose(r["y"][0], [r["gate"][0], 0, 0, 0], atol=0)
+    assert abs(r["y"][0][0] - 0.63) < 1e-6
+
+
+# --------------------------------------------------------------------------
+# Closed forms, special cases and invariants
+# --------------------------------------------------------------------------
+
+def pin_zero_router_uniform(o):
+    # W_r = 0: every p_i = 1/N so P is uniform and aux = 1; all logits tie and
+    # the lowest index wins, so every token goes to expert 0, C are kept.
+    T, d, N = 40, 8, 5
+    x = np.random.default_rng(1).standard_normal((T, d)).astype(np.float32)
+    r = o.route(x, np.zeros((N, d), np.float32), capacity_factor=1.0)
+    C = r["capacity"]
+    assert C == 8
+    assert r["expert"].tolist() == [0] * T
+    assert r["counts"].tolist() == [T] + [0] * (N - 1)
+    assert int((r["slot"] >= 0).sum()) == C and int((r["slot"] < 0).sum()) == T - C
+    assert r["slot"][:C].tolist() == list(range(C))
+    assert np.allclose(r["gate"], 1.0 / N, rtol=0, atol=1e-15)
+    assert abs(r["aux"] - 1.0) < 1e-12
+
+
+def pin_balanced_routing_aux_one(o):
+    # Each expert receives exactly T/N tokens: f is uniform, so aux = 1 for any P.
+    N, m = 4, 6
+    assignment = np.tile(np.arange(N), m)
+    np.random.default_rng(2).shuffle(assignment)
+    x, w_r = _one_hot_routing(assignment, N, scale=3.0)
+    w_r[0, 0] += 1.0  # make P non-uniform
+    r = o.route(x, w_r, capacity_factor=1.0)
+    assert r["counts"].tolist() == [m] * N
+    assert not np.allclose(r["prob_sum"], r["prob_sum"][0])
+    assert abs(r["aux"] - 1.0) < 1e-12
+
+
+def pin_single_expert_is_dense_ffn(o):
+    # N = 1: p = 1, gate = 1, C = ceil(T * c) = T at c = 1, nothing dropped,
+    # so the layer is the dense FFN ReLU(x W_in^T) W_out^T (numpy reference).
+    rng = np.random.default_rng(3)
+    x, w_r, bias, w_in, w_out = _random_problem(rng, 20, 12, 24, 1)
+    r = o.layer_fwd(x, w_r, w_in, w_out, bias=bias, capacity_factor=1.0)
+    dense = np.maximum(x.astype(np.float64) @ w_in[0].astype(np.float64).T, 0.0) @ w_out[0].astype(np.float64).T
+    assert r["capacity"] == 20
+    assert np.all(r["gate"] == 1.0) and np.all(r["slot"] == np.arange(20))
+    assert np.allclose(r["y"], dense, rtol=1e-12, atol=1e-12)
+    assert abs(r["aux"] - 1.0) < 1e-12
+
+
+def pin_logits_match_numpy(o):
+    # h = x W_r^T + b, against numpy's float64 matrix product.
+    rng = np.random.default_rng(4)
+    x, w_r, bias, _, _ = _random_problem(rng, 33, 17, 4, 5)
+    h = o.router_logits(x, w_r, bias)
+    ref = x.astype(np.float64) @ w_r.astype(np.float64).T + bias.astype(np.float64)
+    assert np.allclose(h, ref, rtol=1e-13, atol=1e-13)
+
+
+def pin_bf16_loads_exact(o):
+    # bfloat16 inputs convert exactly: the same values given as float32 and as
+    # bf16 bit patterns give bit-identical logits.
+    rng = np.random.default_rng(5)
+    vals = rng.standard_normal((9, 16)).astype(np.float32)
+    bits = vals.view(np.uint32) >> np.uint32(16)
+    as_f32 = (bits << np.uint32(16)).view(np.float32)
+    as_bf16 = bits.astype(np.uint16)
+    w_r = rng.standard_normal((3, 16)).astype(np.float32)
+    assert np.array_equal(o.router_logits(as_f32, w_r), o.router_logits(as_bf16, w_r))
+
+
+def pin_softmax_matches_scipy(o):
+    rng = np.random.default_rng(6)
+    h = rng.standard_normal((50, 7)) * 3.0
+    r = o.softmax_top1(h, want_probs=True)
+    ref = scipy.special.softmax(h, axis=1)
+    assert np.allclose(r["probs"], ref, rtol=1e-13, atol=1e-15)
+    assert np.array_equal(r["expert"], np.argmax(h, axis=1))
+    assert np.allclose(r["gate"], ref[np.arange(50), r["expert"]], rtol=1e-13)
+    assert np.allclose(r["prob_sum"], ref.sum(axis=0), rtol=1e-13)
+    srt = np.sort(h, axis=1)
+    assert np.allclose(r["margin"], srt[:, -1] - srt[:, -2], rtol=0, atol=1e-15)
+
+
+def pin_ties_lowest_index(o):
+    h = np.array([[1.0, 3.0, 3.0, 0.0], [2.0, 2.0, 2.0, 2.0], [0.0, 0.0, 5.0, 5.0]])
+    r = o.softmax_top1(h)
+    assert r["expert"].tolist() == [1, 0, 2]
+    assert r["margin"].tolist() == [0.0, 0.0, 0.0]
+
+
+def pin_dense_masked_formulation(o):
+    # A second formulation, in numpy: run every expert on every token, then
+    # keep, per expert, the first C tokens (in token order) whose argmax is
+    # that expert, and scale by the selected probability.
+    for seed, (T, d, F, N, C) in enumerate([(40, 8, 16, 3, 10), (64, 6, 10, 5, 9), (17, 4, 8, 2, 17)]):
+        rng = np.random.default_rng(100 + seed)
+        x, w_r, bias, w_in, w_out = _random_problem(rng, T, d, F, N)
+        r = o.layer_fwd(x, w_r, w_in, w_out, bias=bias, capacity=C)
+        x64 = x.astype(np.float64)
+        h = x64 @ w_r.astype(np.float64).T + bias.astype(np.float64)
+        p = scipy.special.softmax(h, axis=1)
+        ids = np.argmax(p, axis=1)
+        every = np.stack([np.maximum(x64 @ w_in[i].astype(np.float64).T, 0) @ w_out[i].astype(np.float64).T
+                          for i in range(N)])
+        y = np.zeros((T, d))
+        for i in range(N):
+            chosen = np.flatnonzero(ids == i)[:C]
+            y[chosen] = p[chosen, i][:, None] * every[i, chosen]
+        assert np.array_equal(r["expert"], ids)
+        assert np.allclose(r["y"], y, rtol=1e-12, atol=1e-13), np.abs(r["y"] - y).max()
+        f = np.bincount(ids, minlength=N) / T
+        assert abs(r["aux"] - N * np.dot(f, p.mean(axis=0))) < 1e-12
+
+
+def pin_brute_force_assignment(o):
+    # Every assignment of T tokens to N experts, every capacity: the kept
+    # tokens of each expert are exactly its first C tokens in token order.
+    for T, N in [(6, 3), (8, 2), (4, 4)]:
+        for assignment in itertools.product(range(N), repeat=T):
+            expert = np.array(assignment, dtype=np.int32)
+            for C in range(1, T + 1):
+                a = o.assign(expert, N, C)
+                for e in range(N):
+                    mine = [t for t in range(T) if assignment[t] == e]
+                    assert a["counts"][e] == len(mine)
+                    kept = mine[:C]
+                    assert a["slot_token"][e].tolist() == kept + [-1] * (C - len(kept))
+                    for s, t in enumerate(mine):
+                        assert a["slot"][t] == (s if s < C else -1)
+
+
+def pin_invariants_random(o):
+    rng = np.random.default_rng(7)
+    T, d, F, N = 300, 16, 32, 6
+    x, w_r, bias, w_in, w_out = _random_problem(rng, T, d, F, N)
+    r = o.layer_fwd(x, w_r, w_in, w_out, bias=bias, capacity_factor=0.8, want_probs=True)
+    C = r["capacity"]
+    assert C == 40
+    assert int(r["counts"].sum()) == T
+    assert np.allclose(r["probs"].sum(axis=1), 1.0, atol=1e-14)
+    assert np.all(r["gate"] >= 1.0 / N - 1e-15) and np.all(r["gate"] <= 1.0)
+    kept = np.minimum(r["counts"], C)
+    for e in range(N):
+        toks = np.flatnonzero((r["expert"] == e) & (r["slot"] >= 0))
+        assert len(toks) == kept[e]
+        assert r["slot"][toks].tolist() == list(range(kept[e]))
+    assert int((r["slot"] < 0).sum()) == int(np.maximum(r["counts"] - C, 0).sum())
+    assert np.all(r["y"][r["slot"] < 0] == 0.0)
+
+
+def pin_permutation_equivariance(o):
+    # With no drops, permuting the tokens permutes ids, gates and outputs and
+    # leaves counts and aux unchanged.
+    rng = np.random.default_rng(8)
+    T, d, F, N = 48, 8, 12, 4
+    x, w_r, bias, w_in, w_out = _random_problem(rng, T, d, F, N)
+    perm = rng.permutation(T)
+    a = o.layer_fwd(x, w_r, w_in, w_out, bias=bias, capacity=T)
+    b = o.layer_fwd(x[perm], w_r, w_in, w_out, bias=bias, capacity=T)
+    assert np.array_equal(a["expert"][perm], b["expert"])
+    assert np.array_equal(a["counts"], b["counts"])
+    assert np.allclose(a["gate"][perm], b["gate"], rtol=1e-15, atol=0)
+    assert np.allclose(a["y"][perm], b["y"], rtol=1e-13, atol=1e-15)
+    assert abs(a["aux"] - b["aux"]) < 1e-12
+
+
+def pin_relu_and_gate_closed_form(o):
+    # Identity experts: y = gate * ReLU(x) exactly, for kept tokens.
+    rng = np.random.default_rng(9)
+    T, N = 12, 3
+    x = rng.standard_normal((T, N)).astype(np.float32)
+    w_r = (rng.standard_normal((N, N))).astype(np.float32)
+    w_in, w_out = _identity_experts(N, N)
+    r = o.layer_fwd(x, w_r, w_in, w_out, capacity=T)
+    ref = r["gate"][:, None] * np.maximum(x.astype(np.float64), 0.0)
+    assert np.array_equal(r["y"], ref)
+
+
+def pin_expert_weight_layout(o):
+    # W_in[e] is [F, d] (row j feeds hidden unit j) and W_out[e] is [d, F]
+    # (row k produces output k): a single nonzero entry in each shows where
+    # the product goes.
+    d, F = 3, 5
+    x = np.array([[0.0, 2.0, 0.0]], dtype=np.float32)
+    w_in = np.zeros((1, F, d), np.float32)
+    w_out = np.zeros((1, d, F), np.float32)
+    w_in[0, 4, 1] = 3.0   # hidden unit 4 = 3 * x[1] = 6
+    w_out[0, 0, 4] = 0.5  # output 0 = 0.5 * hidden 4 = 3
+    r = o.layer_fwd(x, np.zeros((1, d), np.float32), w_in, w_out, capacity=1)
+    assert r["y"][0].tolist() == [3.0, 0.0, 0.0]
+
+
+PINS = {name: fn for name, fn in sorted(globals().items()) if name.startswith("pin_") and callable(fn)}

@@ -1,0 +1,70 @@
+"""Plant plausible mistakes in copies of the oracle and check that the pins catch each.
+
+Each mutant is a textual edit of ``oracle/switch_oracle.c`` (the original is
+never touched), compiled with gcc into a temporary shared object and run
+through every pin in ``oracle_pins.py``.  A mutant that no pin rejects means
+the pins leave that part of the oracle unchecked.  Every edit keeps memory
+accesses in bounds, so a mutant can give wrong answers but cannot crash.
+"""
+from pathlib import Path
+
+import pytest
+
+import oracle
+from oracle_pins import PINS
+
+SRC = Path(oracle.__file__).resolve().parent / "switch_oracle.c"
+
+MUTANTS = {
+    # router: transposed W_r operand (k < d, i < N keeps k*N+i < N*d)
+    "router_transposed_weight": ("(double)w_r[(int64_t)i * d + k]", "(double)w_r[(int64_t)k * N + i]"),
+    "router_bias_dropped": ("acc += (double)bias[i];", "acc += 0.0;"),
+    "router_bias_sign": ("acc += (double)bias[i];", "acc -= (double)bias[i];"),
+    # top-1: ties resolved to the highest index instead of the lowest
+    "argmax_last_on_ties": ("if (row[i] > m) {", "if (row[i] >= m) {"),
+    # softmax: numerator not shifted by the row maximum while the denominator is
+    "softmax_unshifted_numerator": ("p[t * (int64_t)N + i] = exp(row[i] - m) / denom;",
+                                    "p[t * (int64_t)N + i] = exp(row[i]) / denom;"),
+    "softmax_denominator_missing_term": ("for (int32_t i = 0; i < N; ++i)\n            denom += exp(row[i] - m);",
+                                         "for (int32_t i = 1; i < N; ++i)\n            denom += exp(row[i] - m);"),
+    "gate_is_first_prob": ("gate[t] = p[t * (int64_t)N + arg];", "gate[t] = p[t * (int64_t)N + 0];"),
+    # capacity: floor instead of ceil, or no rounding snap
+    "capacity_floor": ("double cap = fabs(exact - nearest) <= 1e-9 ? nearest : ceil(exact);",
+                       "double cap = floor(exact);"),
+    "capacity_off_by_one": ("double cap = fabs(exact - nearest) <= 1e-9 ? nearest : ceil(exact);",
+                            "double cap = (fabs(exact - nearest) <= 1e-9 ? nearest : ceil(exact)) + 1.0;"),
+    # assignment: slot numbering starts at 1; keeps C+... ; reverse token order
+    "slot_one_based": ("slot[t] = position;", "slot[t] = position + 1;"),
+    "assign_reverse_order": ("for (int64_t t = 0; t < T; ++t) {\n        int32_t e = expert[t];",
+                             "for (int64_t t = T - 1; t >= 0; --t) {\n        int32_t e = expert[t];"),
+    # aux: N factor dropped; f and P not normalised by T
+    "aux_missing_N": ("return (double)N * total;", "return total;"),
+    "aux_P_not_averaged": ("double P = prob_sum[i] / (double)T;", "double P = prob_sum[i];"),
+    # expert FFN: ReLU dropped, wrong activation side, transposed W_out, gate not applied
+    "ffn_no_relu": ("u[j] = acc > 0.0 ? acc : 0.0;", "u[j] = acc;"),
+    "ffn_relu_inverted": ("u[j] = acc > 0.0 ? acc : 0.0;", "u[j] = acc < 0.0 ? acc : 0.0;"),
+    "ffn_w_out_transposed": ("load_elem(w_out, w_dtype, (int64_t)k * F + j)", "load_elem(w_out, w_dtype, (int64_t)j * d + k)"),
+    "ffn_w_in_transposed": ("load_elem(w_in, w_dtype, (int64_t)j * d + k)", "load_elem(w_in, w_dtype, (int64_t)k * F + j)"),
+    "ffn_gate_missing": ("y_row[k] = gate * acc;", "y_row[k] = acc;"),
+    "dropped_token_not_zeroed": ("if (slot[t] < 0) {", "if (slot[t] < -1) {"),
+    # bf16 loads: wrong half of the 32-bit pattern
+    "bf16_wrong_shift": ("uint32_t wide = (uint32_t)bits << 16;", "uint32_t wide = (uint32_t)bits << 15;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(tmp_path, name):
+    old, new = MUTANTS[name]
+    text = SRC.read_text()
+    assert text.count(old) == 1, f"mutation site for {name} not found exactly once"
+    src = tmp_path / "mutant.c"
+    src.write_text(text.replace(old, new))
+    so = oracle.build(force=True, source=src, out=tmp_path / f"lib_{name}.so")
+    mutant = oracle.Oracle(oracle.load(so))
+    failed = []
+    for pin_name, pin in PINS.items():
+        try:
+            pin(mutant)
+        except AssertionError:
+            failed.append(pin_name)
+    assert failed, f"no pin rejects mutant {name}"
