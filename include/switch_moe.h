@@ -1,0 +1,197 @@
+/*
+ * switch_moe.h -- C ABI of the B200 (sm_100a) Switch Transformer sparse FFN
+ * layer forward pass.
+ *
+ * The layer (Switch routing, top-1): for every token x of a group of T tokens
+ *   h = W_r . x (+ b)             router logits, float32
+ *   p_i = softmax(h)_i            gate probabilities
+ *   i* = argmax_i p_i             one expert per token, lowest index on ties
+ *   C  = ceil(T / N * c)          expert capacity (slots per expert)
+ *   the first C tokens of each expert, in token order, are kept; the others
+ *   are dropped and get a zero layer output (they pass on through the
+ *   residual connection, which is the caller's)
+ *   y  = p_i*(x) * W_out[i*] . ReLU(W_in[i*] . x)
+ *   aux = N * sum_i f_i * P_i     load-balancing loss without its alpha weight
+ * Sources: llm-papers-study "精读 06 | Switch Transformers" §3.1 (router
+ * logits and softmax), §3.2 (top-1 routing, y = p_i* E_i*), §3.3 (load
+ * balancing loss), §3.4 (expert capacity, dropped tokens); Incredible.AI
+ * "Switch Transformer - Scaling to Trillion Parameter Models with Simple and
+ * Efficient Sparsity", sections "Router Implementation" and "MoE Layer";
+ * kasblo "Switch Transformerとは？" section "Routerだけfloat32で計算する
+ * Selective Precision" (router in float32, experts in bfloat16).
+ *
+ * Conventions shared by every entry point:
+ *  - Ownership: the caller allocates and frees every buffer.  All array
+ *    arguments are DEVICE pointers to contiguous row-major memory, 16-byte
+ *    aligned, unless marked otherwise.  The library never allocates, frees or
+ *    synchronises, except switch_check() (which synchronises the stream).
+ *  - Streams: every compute call is asynchronous on `stream` (a cudaStream_t;
+ *    NULL means the legacy default stream) and launches only kernels of this
+ *    library on it.
+ *  - Errors: argument errors are detected on the host before anything is
+ *    launched and leave every output untouched.  A failed launch returns
+ *    SWITCH_ERR_CUDA.  A kernel that gives up a bounded wait records
+ *    SWITCH_ERR_DEVICE_TIMEOUT in the workspace status word, which
+ *    switch_check() reports.
+ *  - Token order: token t is row t of x (a [batch, seq, d] tensor flattened
+ *    row-major, t = b * seq + s).
+ */
+#ifndef SWITCH_MOE_H
+#define SWITCH_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *switch_stream_t;
+
+typedef enum {
+    SWITCH_OK = 0,
+    SWITCH_ERR_NULL = 1,           /* a required pointer is NULL */
+    SWITCH_ERR_SHAPE = 2,          /* a size is out of range or violates a divisibility rule */
+    SWITCH_ERR_DTYPE = 3,          /* unknown dtype code */
+    SWITCH_ERR_ALIGN = 4,          /* a pointer is not 16-byte aligned */
+    SWITCH_ERR_WORKSPACE = 5,      /* workspace smaller than switch_workspace_size() */
+    SWITCH_ERR_UNSUPPORTED = 6,    /* valid request this build cannot run (e.g. no sm_100 device) */
+    SWITCH_ERR_CUDA = 7,           /* a CUDA runtime call or kernel launch failed */
+    SWITCH_ERR_DEVICE_TIMEOUT = 8  /* a kernel gave up a bounded wait (reported by switch_check) */
+} switch_status_t;
+
+/* Storage type of activations (x, y, xbuf, ybuf) and expert weights (W_in,
+ * W_out).  The router weight, the logit bias and the gates are always float32. */
+typedef enum {
+    SWITCH_F32 = 0,  /* IEEE binary32 */
+    SWITCH_BF16 = 1  /* bfloat16 */
+} switch_dtype_t;
+
+/* Diagnostic switches for switch_dims_t.flags. */
+enum {
+    SWITCH_FLAG_NONE = 0,
+    /* Run the expert FFN on CUDA cores instead of tcgen05 tensor cores (bf16). */
+    SWITCH_FLAG_SIMT_FFN = 1,
+    /* Compute router logits on CUDA cores (FFMA) even where a tensor-core
+     * router exists. */
+    SWITCH_FLAG_SIMT_ROUTER = 2
+};
+
+typedef struct {
+    int64_t T;            /* tokens in the group; 0 <= T < 2^31 */
+    int32_t d_model;      /* d, 1..8192 */
+    int32_t d_ff;         /* F, 1..32768 */
+    int32_t num_experts;  /* N, 1..256 */
+    int32_t capacity;     /* C, slots per expert, >= 1 (see switch_capacity) */
+    int32_t dtype;        /* switch_dtype_t */
+    int32_t flags;        /* SWITCH_FLAG_* (0 for the default path) */
+} switch_dims_t;
+/* Shape rules: bfloat16 requires d_model % 64 == 0 and d_ff % 64 == 0;
+ * float32 accepts any d_model, d_ff >= 1.  N * C must fit in int32. */
+
+/* Expert capacity C = ceil(T / N * c), at least 1 (llm-papers-study §3.4,
+ * expert capacity = tokens per batch / number of experts x capacity factor;
+ * the sources leave the rounding open and this library rounds up).  A
+ * product within 1e-9 of an integer counts as that integer.  Host only.
+ * Returns -1 if T < 0, N < 1 or c is not a positive finite number. */
+int64_t switch_capacity(int64_t T, int32_t num_experts, double capacity_factor);
+
+/* Bytes of device workspace that every entry point below needs for `dims`
+ * (scan state, per-tile partial sums, the hidden activations H[N, C, F], the
+ * layer's internal [N, C, d] buffers and the status word).  Host only.
+ * Errors: SWITCH_ERR_NULL, SWITCH_ERR_SHAPE, SWITCH_ERR_DTYPE. */
+switch_status_t switch_workspace_size(const switch_dims_t *dims, size_t *bytes);
+
+/* Router, top-1, capacity assignment, per-expert counts and the aux loss
+ * (llm-papers-study §3.1-§3.4; Incredible.AI "Router Implementation").
+ *   x          [T, d]   activation dtype
+ *   w_r        [N, d]   float32 router weight (row i produces logit i)
+ *   logit_bias [N]      float32 added to the logits, or NULL for none
+ * Outputs (all written):
+ *   expert     [T]      int32, argmax expert of each token (lowest index on ties)
+ *   gate       [T]      float32, p_expert(x) = softmax(h)[expert]
+ *   slot       [T]      int32, position of the token in its expert's buffer,
+ *                       in token order, or -1 when it overflowed capacity
+ *   counts     [N]      int32, tokens routed to each expert BEFORE capacity
+ *   slot_token [N * C]  int32, token held by slot s of expert i at [i*C+s],
+ *                       -1 for an empty slot
+ *   aux        [1]      float32, N * sum_i (counts_i / T) * (mean_t p_i);
+ *                       0 when T == 0
+ * Deterministic: identical inputs give identical bytes. */
+switch_status_t switch_route(const switch_dims_t *dims, const void *x, const float *w_r,
+                             const float *logit_bias, int32_t *expert, float *gate, int32_t *slot,
+                             int32_t *counts, int32_t *slot_token, float *aux, void *workspace,
+                             size_t workspace_bytes, switch_stream_t stream);
+
+/* Dispatch: gather the kept tokens into per-expert buffers
+ * (Incredible.AI "MoE Layer", x_flat[expert_indices]; kasblo "tokenを
+ * Expertへ送って戻すforward pass", single-device gather).
+ *   xbuf[i, s, :] = x[slot_token[i*C+s], :]   for s < min(counts[i], C)
+ *   x [T, d], slot_token [N*C], counts [N]  ->  xbuf [N, C, d] (activation dtype)
+ * Rows s >= min(counts[i], C) of xbuf are not written. */
+switch_status_t switch_dispatch(const switch_dims_t *dims, const void *x, const int32_t *slot_token,
+                                const int32_t *counts, void *xbuf, switch_stream_t stream);
+
+/* Expert FFN on the kept rows of every expert:
+ *   ybuf[i, s, :] = W_out[i] . ReLU(W_in[i] . xbuf[i, s, :])   for s < min(counts[i], C)
+ *   xbuf  [N, C, d]   activation dtype
+ *   w_in  [N, F, d]   expert dtype (nn.Linear layout: row j feeds hidden unit j)
+ *   w_out [N, d, F]   expert dtype
+ *   ybuf  [N, C, d]   activation dtype; other rows are not written
+ * bfloat16: tcgen05 tensor cores, float32 accumulation, the hidden
+ * activations rounded to bfloat16 in the workspace.  float32: CUDA cores.
+ * (Switch FFN experts: llm-papers-study §3.2; two-layer ReLU experts without
+ * biases, the sources leave the body open.) */
+switch_status_t switch_expert_ffn(const switch_dims_t *dims, const void *xbuf, const void *w_in,
+                                  const void *w_out, const int32_t *counts, void *ybuf, void *workspace,
+                                  size_t workspace_bytes, switch_stream_t stream);
+
+/* Combine: scatter back to token order, scaled by the gate
+ * (llm-papers-study §3.2, y = p_i*(x) E_i*(x); §3.4, dropped tokens skip the
+ * expert):
+ *   y[t, :] = gate[t] * ybuf[expert[t], slot[t], :]   if slot[t] >= 0
+ *   y[t, :] = 0                                       if slot[t] == -1
+ * The product is formed in float32 and rounded once to the activation dtype.
+ *   ybuf [N, C, d], expert [T], slot [T], gate [T]  ->  y [T, d] */
+switch_status_t switch_combine(const switch_dims_t *dims, const void *ybuf, const int32_t *expert,
+                               const int32_t *slot, const float *gate, void *y, switch_stream_t stream);
+
+/* The whole layer: switch_route, then dispatch, expert FFN and combine, with
+ * the [N, C, d] buffers and slot_token kept in the workspace.  Arguments as
+ * above; y [T, d] is the layer output WITHOUT the residual. */
+switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const float *w_r,
+                                 const float *logit_bias, const void *w_in, const void *w_out, void *y,
+                                 int32_t *expert, float *gate, int32_t *slot, int32_t *counts, float *aux,
+                                 void *workspace, size_t workspace_bytes, switch_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the device status word kept in
+ * `workspace`.  Returns SWITCH_OK, SWITCH_ERR_DEVICE_TIMEOUT, or
+ * SWITCH_ERR_CUDA if the stream reports an error. */
+switch_status_t switch_check(void *workspace, size_t workspace_bytes, switch_stream_t stream);
+
+/* Static description of a status code. */
+const char *switch_status_string(switch_status_t status);
+
+/* ---- instrumentation -------------------------------------------------- */
+
+/* Number of kernels this library has launched in this process. */
+int64_t switch_launch_count(void);
+
+/* Per-launch tracing.  While tracing is on, every kernel launch is bracketed
+ * by two CUDA events recorded on its stream; at most `max_launches` launches
+ * are kept.  switch_trace_read() synchronises those events and fills
+ * kernel_id[k] and ms[k] (elapsed milliseconds of launch k), returning the
+ * number of launches traced.  Host only; not thread-safe. */
+switch_status_t switch_trace_start(int32_t max_launches);
+int32_t switch_trace_read(int32_t *kernel_id, float *ms, int32_t capacity);
+void switch_trace_stop(void);
+/* Name of a traced kernel id, or "?" if unknown. */
+const char *switch_kernel_name(int32_t kernel_id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWITCH_MOE_H */

@@ -1,0 +1,318 @@
+// Expert FFN on the 5th-generation tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+//
+//   GEMM1: H[i, s, :]    = ReLU(xbuf[i, s, :] . W_in[i]^T)    (K = d, Nout = F)
+//   GEMM2: ybuf[i, s, :] = H[i, s, :] . W_out[i]^T            (K = F, Nout = d)
+// over the kept rows s < min(counts[i], C) of every expert i.  Both GEMMs
+// are the same grouped "A . B^T" kernel with both operands K-major (the
+// nn.Linear weight layout), bf16 inputs and fp32 accumulation in tensor
+// memory; the epilogue applies ReLU (GEMM1), rounds to bf16 and stores rows
+// below the expert's kept count.  (Expert FFN: llm-papers-study "精读 06 |
+// Switch Transformers" §3.2; bfloat16 experts with float32 accumulation:
+// kasblo section "Routerだけfloat32で計算するSelective Precision".)
+//
+// Kernel structure (one CTA per SM, persistent over a tile list that every
+// CTA derives on the device from `counts`, so no host synchronisation):
+//   warp 0      one lane issues TMA loads of 128 x 64 A and BN x 64 B tiles
+//               (128-byte swizzle) into a STAGES-deep shared-memory ring
+//   warp 1      allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN,
+//               K=16) into one of two TMEM accumulators and commits to
+//               mbarriers that free ring slots / publish the accumulator
+//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes, ReLU, bf16,
+//               16-byte stores; then release the accumulator
+// Every mbarrier wait is bounded (about 1 s); on a timeout the kernel records
+// SWITCH_ERR_DEVICE_TIMEOUT in the status word, waits (bounded) for its own
+// TMA loads and MMAs in flight, frees TMEM and returns.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace switchmoe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
+constexpr int kThreads = 192;
+constexpr int kEpilogueThreads = 128;
+
+template <int BN, int STAGES>
+struct TcLayout {
+    static constexpr size_t a_bytes = (size_t)BM * BK * 2;
+    static constexpr size_t b_bytes = (size_t)BN * BK * 2;
+    static constexpr size_t ring = STAGES * (a_bytes + b_bytes);
+    static constexpr size_t barriers = (2 * STAGES + 2 + 2 + 1) * 8 + 16;
+    static size_t bytes(int experts) { return 1024 + ring + barriers + (size_t)(experts + 1) * 4; }
+};
+
+__device__ __forceinline__ void locate_tile(const int32_t *tile_start, int E, int n_tiles_n, int tile, int &e,
+                                            int &m, int &n) {
+    int lo = 0, hi = E - 1;  // largest e with tile_start[e] <= tile
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tile_start[mid] <= tile) lo = mid;
+        else hi = mid - 1;
+    }
+    e = lo;
+    const int local = tile - tile_start[e];
+    m = local / n_tiles_n;
+    n = local % n_tiles_n;
+}
+
+template <int BN, int STAGES, bool RELU>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_grouped_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                    __nv_bfloat16 *__restrict__ out, const int32_t *__restrict__ counts, int E, int C, int K,
+                    int Nout, DeviceStatus *status) {
+    using L = TcLayout<BN, STAGES>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;
+    uint8_t *sB = sA + STAGES * L::a_bytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(base + L::ring);
+    uint64_t *empty = full + STAGES;
+    uint64_t *acc_full = empty + STAGES;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *drain = acc_empty + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    int32_t *tile_start = reinterpret_cast<int32_t *>(tmem_holder + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles_n = (Nout + BN - 1) / BN;
+    const int k_blocks = K / BK;
+    constexpr uint32_t kTmemCols = 2 * BN;
+
+    // Tile list: expert e owns tiles [tile_start[e], tile_start[e+1]), laid
+    // out m-major with the BN-wide column tiles innermost.
+    if (warp == 0) {
+        int running = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int kept = e < E ? min(counts[e], C) : 0;
+            const int mine = (kept + BM - 1) / BM * n_tiles_n;
+            int incl = mine;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += u;
+            }
+            if (e < E) tile_start[e] = running + incl - mine;
+            running += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) tile_start[E] = running;
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], 1);
+            }
+            for (int a = 0; a < 2; ++a) {
+                mbar_init(&acc_full[a], 1);
+                mbar_init(&acc_empty[a], kEpilogueThreads);
+            }
+            mbar_init(drain, 1);
+            fence_barrier_init();
+        }
+        __syncwarp();
+        tmem_alloc(tmem_holder, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    const int total_tiles = tile_start[E];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tmap_a);
+            prefetch_tmap(&tmap_b);
+            uint32_t issued = 0, parity_of = 0;  // per ring slot: load issued, parity of its phase
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+                int e, m, n;
+                locate_tile(tile_start, E, n_tiles_n, tile, e, m, n);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, status, 1)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(L::a_bytes + L::b_bytes));
+                    tma_load_3d(sA + stage * L::a_bytes, &tmap_a, &full[stage], kb * BK, m * BM, e);
+                    tma_load_3d(sB + stage * L::b_bytes, &tmap_b, &full[stage], kb * BK, n * BN, e);
+                    issued |= 1u << stage;
+                    parity_of = (parity_of & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // Wind-down: the last load into every slot must have landed
+            // before the CTA may exit (already true unless a wait timed out).
+            for (int s = 0; s < STAGES; ++s)
+                if (issued & (1u << s)) mbar_wait(&full[s], (parity_of >> s) & 1u, status, 6);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, status, 2)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, status, 3)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t a_desc = smem_desc_sw128(sA + stage * L::a_bytes);
+                    const uint64_t b_desc = smem_desc_sw128(sB + stage * L::b_bytes);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        // advance 16 bf16 = 32 bytes along K inside the swizzled row
+                        tc_mma_bf16(d_tmem, a_desc + (uint64_t)(2 * k), b_desc + (uint64_t)(2 * k), idesc,
+                                    (kb | k) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&acc_full[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            // Wind-down: every MMA issued above has completed once `drain` flips.
+            tc_commit(drain);
+            mbar_wait(drain, 0, status, 4);
+        }
+    } else {
+        const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter+32) belong to this warp
+        const int row_in_tile = quarter * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+            int e, m, n;
+            locate_tile(tile_start, E, n_tiles_n, tile, e, m, n);
+            if (!mbar_wait(&acc_full[acc], acc_phase, status, 5)) break;
+            tc_fence_after();
+            const int kept = min(counts[e], C);
+            const int row = m * BM + row_in_tile;
+            const bool row_ok = row < kept;
+            __nv_bfloat16 *orow = out + ((int64_t)e * C + row) * Nout;
+            const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 32) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
+                tmem_ld_wait();
+                const int col0 = n * BN + c;
+                if (row_ok && col0 < Nout) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + col0);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float v[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            v[i] = __uint_as_float(r[8 * q + i]);
+                            if (RELU) v[i] = fmaxf(v[i], 0.f);
+                        }
+                        dst[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launches
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 3-D bf16 tensor [E][rows][K] (K contiguous), box = box_rows x 64, 128-byte swizzle.
+bool make_tmap(CUtensorMap *map, const void *ptr, int E, int rows, int K, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)rows, (cuuint64_t)E};
+    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)rows * K * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)BK, (cuuint32_t)box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, bool RELU>
+cudaError_t launch_gemm(int32_t kernel_id, const void *a, const void *b, void *out, const int32_t *counts, int E,
+                        int C, int K, int Nout, int64_t T, DeviceStatus *status, cudaStream_t stream) {
+    CUtensorMap ta, tb;
+    if (!make_tmap(&ta, a, E, C, K, BM) || !make_tmap(&tb, b, E, Nout, K, BN)) return cudaErrorInvalidValue;
+    const size_t smem = TcLayout<BN, STAGES>::bytes(E);
+    auto kern = tc_grouped_gemm<BN, STAGES, RELU>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    // Upper bound on the number of tiles, from host-known sizes only.
+    const int64_t m_tiles = std::min<int64_t>((int64_t)E * ((C + BM - 1) / BM), (T + BM - 1) / BM + E);
+    const int64_t tiles = m_tiles * ((Nout + BN - 1) / BN);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count(), tiles));
+    launch_begin(kernel_id, stream);
+    kern<<<grid, kThreads, smem, stream>>>(ta, tb, static_cast<__nv_bfloat16 *>(out), counts, E, C, K, Nout, status);
+    err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
+                          const int32_t *counts, void *ybuf, const Workspace &ws, cudaStream_t stream) {
+    const int N = dims.num_experts, C = dims.capacity, d = dims.d_model, F = dims.d_ff;
+    DeviceStatus *st = static_cast<DeviceStatus *>(ws.status);
+    cudaError_t err = launch_gemm<256, 4, true>(K_FFN_TC_GEMM1, xbuf, w_in, ws.hidden, counts, N, C, d, F, dims.T,
+                                                st, stream);
+    if (err != cudaSuccess) return err;
+    return launch_gemm<128, 6, false>(K_FFN_TC_GEMM2, ws.hidden, w_out, ybuf, counts, N, C, F, d, dims.T, st,
+                                      stream);
+}
+
+}  // namespace switchmoe

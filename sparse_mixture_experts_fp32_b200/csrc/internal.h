@@ -1,0 +1,67 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "switch_moe.h"
+
+namespace switchmoe {
+
+// Tokens per routing tile: the granularity of the per-tile expert histograms,
+// of the probability partial sums and of the slot-assignment blocks.
+constexpr int kTileT = 64;
+
+// Kernel ids reported by the tracer.
+enum KernelId : int32_t {
+    K_ROUTER_WARP = 1,
+    K_ROUTER_TILED = 2,
+    K_SCAN = 3,
+    K_ASSIGN = 4,
+    K_DISPATCH = 5,
+    K_FFN_TC_GEMM1 = 6,
+    K_FFN_TC_GEMM2 = 7,
+    K_FFN_SIMT_GEMM1 = 8,
+    K_FFN_SIMT_GEMM2 = 9,
+    K_COMBINE = 10,
+};
+
+struct Workspace {
+    void *status;        // DeviceStatus
+    uint32_t *ticket;    // last-block ticket of the scan kernel
+    int32_t *hist;       // [N][tiles] tokens of each expert in each tile
+    float *psum;         // [N][tiles] sum of p_i over each tile
+    int32_t *tile_off;   // [N][tiles] exclusive prefix of hist over tiles
+    double *prob_total;  // [N] sum of p_i over all tokens
+    int32_t *slot_token; // [N*C] (layer_fwd only)
+    void *xbuf;          // [N][C][d] (layer_fwd only)
+    void *ybuf;          // [N][C][d] (layer_fwd only)
+    void *hidden;        // [N][C][F] expert hidden activations
+    int64_t tiles;
+};
+
+size_t workspace_bytes(const switch_dims_t &dims);
+Workspace carve_workspace(const switch_dims_t &dims, void *base);
+
+// Launch bookkeeping (tracing + launch counter).
+void launch_begin(int32_t kernel_id, cudaStream_t stream);
+void launch_end(cudaStream_t stream);
+
+// Launchers.  Each returns the cudaError_t of its launch.
+cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
+                         int32_t *expert, float *gate, int32_t *slot, int32_t *counts, int32_t *slot_token,
+                         float *aux, const Workspace &ws, cudaStream_t stream);
+cudaError_t launch_dispatch(const switch_dims_t &dims, const void *x, const int32_t *slot_token,
+                            const int32_t *counts, void *xbuf, cudaStream_t stream);
+cudaError_t launch_combine(const switch_dims_t &dims, const void *ybuf, const int32_t *expert,
+                           const int32_t *slot, const float *gate, void *y, cudaStream_t stream);
+cudaError_t launch_ffn_simt(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
+                            const int32_t *counts, void *ybuf, const Workspace &ws, cudaStream_t stream);
+cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
+                          const int32_t *counts, void *ybuf, const Workspace &ws, cudaStream_t stream);
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace switchmoe

@@ -1,0 +1,159 @@
+// Dispatch (gather kept tokens into per-expert buffers) and combine (gated
+// scatter back to token order), sm_100a.
+//
+// Dispatch: xbuf[i, s, :] = x[slot_token[i*C+s], :] for s < min(counts[i], C)
+//   (Incredible.AI "MoE Layer", x_flat[expert_indices]; kasblo section
+//   "tokenをExpertへ送って戻すforward pass": on one device the exchange is a
+//   gather/scatter in memory).
+// Combine:  y[t, :] = gate[t] * ybuf[expert[t], slot[t], :], or 0 for a
+//   dropped token (llm-papers-study "精读 06 | Switch Transformers" §3.2,
+//   y = p_i*(x) E_i*(x); §3.4, dropped tokens skip the expert).
+//
+// Both are pure HBM streams: one warp per row, 16-byte vector accesses, all of
+// a lane's loads issued before its stores.
+#include "common.cuh"
+#include "internal.h"
+
+namespace switchmoe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRowsPerBlock = kThreads / 32;
+constexpr int kUnroll = 4;
+
+// Row copy of `words` 16-byte words by one warp.
+__device__ __forceinline__ void warp_copy_row16(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int words) {
+    const int lane = threadIdx.x & 31;
+    int w = lane;
+    for (; w + 32 * (kUnroll - 1) < words; w += 32 * kUnroll) {
+        uint4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) v[u] = __ldcs(src + w + 32 * u);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) dst[w + 32 * u] = v[u];
+    }
+    for (; w < words; w += 32) dst[w] = __ldcs(src + w);
+}
+
+__global__ void __launch_bounds__(kThreads) dispatch_kernel16(const uint4 *__restrict__ x,
+                                                             const int32_t *__restrict__ slot_token,
+                                                             const int32_t *__restrict__ counts, int N, int C,
+                                                             int words, uint4 *__restrict__ xbuf) {
+    const int64_t row = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
+    if (row >= (int64_t)N * C) return;
+    const int e = (int)(row / C), s = (int)(row % C);
+    if (s >= min(counts[e], C)) return;
+    const int64_t t = slot_token[row];
+    warp_copy_row16(x + t * words, xbuf + row * words, words);
+}
+
+// Rows whose byte size is not a multiple of 16 (float32 with d % 4 != 0).
+__global__ void __launch_bounds__(kThreads) dispatch_kernel4(const uint32_t *__restrict__ x,
+                                                            const int32_t *__restrict__ slot_token,
+                                                            const int32_t *__restrict__ counts, int N, int C,
+                                                            int words, uint32_t *__restrict__ xbuf) {
+    const int64_t row = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
+    if (row >= (int64_t)N * C) return;
+    const int e = (int)(row / C), s = (int)(row % C);
+    if (s >= min(counts[e], C)) return;
+    const int64_t t = slot_token[row];
+    for (int w = threadIdx.x & 31; w < words; w += 32) xbuf[row * words + w] = x[t * words + w];
+}
+
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float g) {
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(w[i] << 16) * g;
+        const float hi = __uint_as_float(w[i] & 0xffff0000u) * g;
+        w[i] = pack_bf16x2(lo, hi);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void __launch_bounds__(kThreads) combine_kernel_bf16(const uint4 *__restrict__ ybuf,
+                                                               const int32_t *__restrict__ expert,
+                                                               const int32_t *__restrict__ slot,
+                                                               const float *__restrict__ gate, int64_t T, int C,
+                                                               int words, uint4 *__restrict__ y) {
+    const int64_t t = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const int lane = threadIdx.x & 31;
+    const int s = slot[t];
+    uint4 *dst = y + t * words;
+    if (s < 0) {
+        for (int w = lane; w < words; w += 32) dst[w] = make_uint4(0u, 0u, 0u, 0u);
+        return;
+    }
+    const float g = gate[t];
+    const uint4 *src = ybuf + ((int64_t)expert[t] * C + s) * words;
+    int w = lane;
+    for (; w + 32 * (kUnroll - 1) < words; w += 32 * kUnroll) {
+        uint4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) v[u] = __ldcs(src + w + 32 * u);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) __stcs(dst + w + 32 * u, scale_bf16x8(v[u], g));
+    }
+    for (; w < words; w += 32) __stcs(dst + w, scale_bf16x8(__ldcs(src + w), g));
+}
+
+__global__ void __launch_bounds__(kThreads) combine_kernel_f32(const float *__restrict__ ybuf,
+                                                              const int32_t *__restrict__ expert,
+                                                              const int32_t *__restrict__ slot,
+                                                              const float *__restrict__ gate, int64_t T, int C, int d,
+                                                              float *__restrict__ y) {
+    const int64_t t = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const int lane = threadIdx.x & 31;
+    const int s = slot[t];
+    float *dst = y + t * d;
+    if (s < 0) {
+        for (int k = lane; k < d; k += 32) dst[k] = 0.f;
+        return;
+    }
+    const float g = gate[t];
+    const float *src = ybuf + ((int64_t)expert[t] * C + s) * d;
+    for (int k = lane; k < d; k += 32) dst[k] = g * src[k];
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const switch_dims_t &dims, const void *x, const int32_t *slot_token,
+                            const int32_t *counts, void *xbuf, cudaStream_t stream) {
+    const int N = dims.num_experts, C = dims.capacity;
+    const int64_t rows = (int64_t)N * C;
+    const int64_t row_bytes = (int64_t)dims.d_model * (dims.dtype == SWITCH_BF16 ? 2 : 4);
+    const unsigned grid = (unsigned)((rows + kRowsPerBlock - 1) / kRowsPerBlock);
+    if (dims.T == 0) return cudaSuccess;
+    launch_begin(K_DISPATCH, stream);
+    if (row_bytes % 16 == 0)
+        dispatch_kernel16<<<grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(x), slot_token, counts, N, C,
+                                                         (int)(row_bytes / 16), static_cast<uint4 *>(xbuf));
+    else
+        dispatch_kernel4<<<grid, kThreads, 0, stream>>>(static_cast<const uint32_t *>(x), slot_token, counts, N, C,
+                                                        (int)(row_bytes / 4), static_cast<uint32_t *>(xbuf));
+    cudaError_t err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
+
+cudaError_t launch_combine(const switch_dims_t &dims, const void *ybuf, const int32_t *expert, const int32_t *slot,
+                           const float *gate, void *y, cudaStream_t stream) {
+    const int64_t T = dims.T;
+    if (T == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((T + kRowsPerBlock - 1) / kRowsPerBlock);
+    launch_begin(K_COMBINE, stream);
+    if (dims.dtype == SWITCH_BF16)
+        combine_kernel_bf16<<<grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(ybuf), expert, slot, gate, T,
+                                                           dims.capacity, dims.d_model / 8,
+                                                           static_cast<uint4 *>(y));
+    else
+        combine_kernel_f32<<<grid, kThreads, 0, stream>>>(static_cast<const float *>(ybuf), expert, slot, gate, T,
+                                                          dims.capacity, dims.d_model, static_cast<float *>(y));
+    cudaError_t err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
+
+}  // namespace switchmoe

@@ -1,0 +1,531 @@
+// Router, top-1, capacity scan and slot assignment (sm_100a).
+//
+//   router  h = W_r . x (+ b) in float32; p = softmax(h); expert = argmax
+//           (lowest index on ties); gate = p[expert]; per 64-token tile:
+//           tokens per expert and sum of p_i.
+//           (llm-papers-study "精读 06 | Switch Transformers" §3.1-§3.2;
+//           kasblo "Switch Transformerとは？" section "Routerだけfloat32で
+//           計算するSelective Precision": router arithmetic in float32.)
+//   scan    per expert, exclusive prefix of the tile counts -> each tile's
+//           first slot; totals -> counts; fp64 sum of p_i -> aux loss
+//           N * sum_i (counts_i / T) * (P_i / T)   (llm-papers-study §3.3).
+//   assign  slot of a token = its tile's first slot for its expert + its
+//           rank among the tile's tokens of that expert; kept iff slot < C
+//           (llm-papers-study §3.4; Incredible.AI "MoE Layer": the first C
+//           tokens of each expert in token order are kept).
+#include <float.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace switchmoe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+__device__ __forceinline__ int lanemask_lt() {
+    int m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Per-token softmax / top-1 bookkeeping, done by one warp.  Each lane holds
+// up to J logits: value v[j] for expert idx[j] (idx < 0: not held).  Every
+// expert is held by exactly one "owner" lane (own[j] true); other lanes may
+// hold copies, which take part in the max but not in the sums.
+template <int J>
+__device__ __forceinline__ void token_epilogue(const float (&v)[J], const int (&idx)[J], const bool (&own)[J],
+                                               int64_t t, float *warp_psum, int32_t *warp_hist, int32_t *expert,
+                                               float *gate) {
+    const int lane = threadIdx.x & 31;
+    float m = -FLT_MAX;
+    int arg = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        if (idx[j] >= 0 && (v[j] > m || (v[j] == m && idx[j] < arg))) {
+            m = v[j];
+            arg = idx[j];
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float om = __shfl_xor_sync(0xffffffffu, m, off);
+        const int oa = __shfl_xor_sync(0xffffffffu, arg, off);
+        if (om > m || (om == m && oa < arg)) {
+            m = om;
+            arg = oa;
+        }
+    }
+    float ex[J];
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        ex[j] = (idx[j] >= 0 && own[j]) ? expf(v[j] - m) : 0.f;
+        s += ex[j];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+        if (idx[j] >= 0 && own[j]) warp_psum[idx[j]] += ex[j] / s;
+    if (lane == 0) {
+        warp_hist[arg] += 1;
+        expert[t] = arg;
+        gate[t] = 1.0f / s;  // p at the argmax: exp(0) / s
+    }
+}
+
+// Sum the per-warp partials of a tile in fixed warp order and publish them
+// expert-major ([N][tiles]) for the scan.
+__device__ __forceinline__ void publish_tile(const float *psum_w, const int32_t *hist_w, int N, int tiles,
+                                             int tile, int32_t *hist, float *psum) {
+    for (int i = threadIdx.x; i < N; i += kThreads) {
+        int32_t c = 0;
+        float p = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            c += hist_w[w * N + i];
+            p += psum_w[w * N + i];
+        }
+        hist[(int64_t)i * tiles + tile] = c;
+        psum[(int64_t)i * tiles + tile] = p;
+    }
+}
+
+template <typename XT>
+struct XLoad;
+template <>
+struct XLoad<__nv_bfloat16> {
+    static constexpr int V = 8;  // elements per 16-byte vector
+    static __device__ __forceinline__ void vec(const __nv_bfloat16 *p, float (&o)[V]) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(p));
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            o[2 * i] = __uint_as_float(w[i] << 16);
+            o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    static __device__ __forceinline__ float one(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+};
+template <>
+struct XLoad<float> {
+    static constexpr int V = 4;
+    static __device__ __forceinline__ void vec(const float *p, float (&o)[V]) {
+        const float4 raw = __ldg(reinterpret_cast<const float4 *>(p));
+        o[0] = raw.x;
+        o[1] = raw.y;
+        o[2] = raw.z;
+        o[3] = raw.w;
+    }
+    static __device__ __forceinline__ float one(const float *p) { return *p; }
+};
+
+// ---------------------------------------------------------------------------
+// Router for N <= 32: one warp per token, W_r resident in shared memory as
+// [d][NP] (NP = N rounded up to a power of two >= 8).  Each lane accumulates
+// NP partial dot products over its share of d; a halving exchange then
+// leaves lane L with the full logit of expert L >> (5 - log2 NP).
+// ---------------------------------------------------------------------------
+template <typename XT, int NP>
+__global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restrict__ x, const float *__restrict__ w_r,
+                                                               const float *__restrict__ bias, int64_t T, int d,
+                                                               int N, int tiles, int32_t *__restrict__ expert,
+                                                               float *__restrict__ gate, int32_t *__restrict__ hist,
+                                                               float *__restrict__ psum, uint32_t *ticket) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    float *wsm = reinterpret_cast<float *>(smem_raw);  // [d][NP]
+    float *psum_w = wsm + (size_t)d * NP;               // [kWarps][N]
+    int32_t *hist_w = reinterpret_cast<int32_t *>(psum_w + kWarps * N);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tile = blockIdx.x;
+
+    if (tile == 0 && tid == 0) *ticket = 0u;
+    for (int i = tid; i < d * NP; i += kThreads) {
+        const int k = i / NP, e = i % NP;
+        wsm[i] = e < N ? w_r[(int64_t)e * d + k] : 0.f;
+    }
+    for (int i = tid; i < kWarps * N; i += kThreads) {
+        psum_w[i] = 0.f;
+        hist_w[i] = 0;
+    }
+    __syncthreads();
+
+    constexpr int LOG_NP = NP == 8 ? 3 : NP == 16 ? 4 : 5;
+    constexpr int SHIFT = 5 - LOG_NP;
+    const int my_e = lane >> SHIFT;
+    const bool valid_e = my_e < N;
+    const float my_bias = (bias && valid_e) ? bias[my_e] : 0.f;
+    constexpr int V = XLoad<XT>::V;
+    const bool vec_ok = (d % V) == 0;
+
+    for (int r = warp; r < kTileT; r += kWarps) {
+        const int64_t t = (int64_t)tile * kTileT + r;
+        if (t >= T) break;
+        const XT *xr = x + t * d;
+        float acc[NP];
+#pragma unroll
+        for (int e = 0; e < NP; ++e) acc[e] = 0.f;
+        if (vec_ok) {
+            for (int k = lane * V; k < d; k += 32 * V) {
+                float xv[V];
+                XLoad<XT>::vec(xr + k, xv);
+#pragma unroll
+                for (int u = 0; u < V; ++u) {
+                    const float4 *wrow = reinterpret_cast<const float4 *>(wsm + (size_t)(k + u) * NP);
+#pragma unroll
+                    for (int q = 0; q < NP / 4; ++q) {
+                        const float4 w4 = wrow[q];
+                        acc[4 * q + 0] = fmaf(xv[u], w4.x, acc[4 * q + 0]);
+                        acc[4 * q + 1] = fmaf(xv[u], w4.y, acc[4 * q + 1]);
+                        acc[4 * q + 2] = fmaf(xv[u], w4.z, acc[4 * q + 2]);
+                        acc[4 * q + 3] = fmaf(xv[u], w4.w, acc[4 * q + 3]);
+                    }
+                }
+            }
+        } else {
+            for (int k = lane; k < d; k += 32) {
+                const float xv = XLoad<XT>::one(xr + k);
+#pragma unroll
+                for (int e = 0; e < NP; ++e) acc[e] = fmaf(xv, wsm[(size_t)k * NP + e], acc[e]);
+            }
+        }
+        // Halving exchange: after step s, a lane keeps the half of its
+        // remaining values selected by lane bit (4 - s) and adds the
+        // partner's copy of that half.
+#pragma unroll
+        for (int step = 0; step < 5; ++step) {
+            const int off = 16 >> step;
+            const int n = NP >> step;  // values still held per lane
+            if (n > 1) {
+                const bool upper = (lane & off) != 0;
+                const int half = n / 2;
+#pragma unroll
+                for (int i = 0; i < NP / 2; ++i) {
+                    if (i < half) {
+                        const float send = upper ? acc[i] : acc[i + half];
+                        const float keep = upper ? acc[i + half] : acc[i];
+                        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                    }
+                }
+            } else {
+                acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], off);
+            }
+        }
+        float v[1] = {acc[0] + my_bias};
+        int idx[1] = {valid_e ? my_e : -1};
+        bool own[1] = {(lane & ((1 << SHIFT) - 1)) == 0};
+        token_epilogue<1>(v, idx, own, t, psum_w + warp * N, hist_w + warp * N, expert, gate);
+    }
+    __syncthreads();
+    publish_tile(psum_w, hist_w, N, tiles, tile, hist, psum);
+}
+
+// ---------------------------------------------------------------------------
+// Router for any N <= 256: a 64-token x EC-expert SIMT tile GEMM over
+// 32-wide chunks of d, logits collected in shared memory, then one warp per
+// token for the softmax / top-1.
+// ---------------------------------------------------------------------------
+constexpr int kKC = 32;
+
+template <typename XT, int EC>
+__global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__restrict__ x, const float *__restrict__ w_r,
+                                                                const float *__restrict__ bias, int64_t T, int d,
+                                                                int N, int tiles, int32_t *__restrict__ expert,
+                                                                float *__restrict__ gate, int32_t *__restrict__ hist,
+                                                                float *__restrict__ psum, uint32_t *ticket) {
+    constexpr int TE = EC / 16;  // experts per thread
+    constexpr int TT = 4;        // tokens per thread
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int NL = N + 1;
+    float *xs = reinterpret_cast<float *>(smem_raw);  // [kKC][kTileT]
+    float *ws = xs + kKC * kTileT;                     // [kKC][EC]
+    float *logits = ws + kKC * EC;                     // [kTileT][NL]
+    float *psum_w = logits + kTileT * NL;              // [kWarps][N]
+    int32_t *hist_w = reinterpret_cast<int32_t *>(psum_w + kWarps * N);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tx = tid % 16, ty = tid / 16;
+    const int tile = blockIdx.x;
+    const int64_t t0 = (int64_t)tile * kTileT;
+
+    if (tile == 0 && tid == 0) *ticket = 0u;
+    for (int i = tid; i < kWarps * N; i += kThreads) {
+        psum_w[i] = 0.f;
+        hist_w[i] = 0;
+    }
+
+    for (int e0 = 0; e0 < N; e0 += EC) {
+        float acc[TT][TE];
+#pragma unroll
+        for (int i = 0; i < TT; ++i)
+#pragma unroll
+            for (int j = 0; j < TE; ++j) acc[i][j] = 0.f;
+        for (int k0 = 0; k0 < d; k0 += kKC) {
+            __syncthreads();
+            for (int i = tid; i < kTileT * kKC; i += kThreads) {
+                const int r = i / kKC, kk = i % kKC;
+                const int64_t t = t0 + r;
+                const int k = k0 + kk;
+                xs[kk * kTileT + r] = (t < T && k < d) ? XLoad<XT>::one(x + t * d + k) : 0.f;
+            }
+            for (int i = tid; i < EC * kKC; i += kThreads) {
+                const int e = i / kKC, kk = i % kKC;
+                const int k = k0 + kk;
+                ws[kk * EC + e] = (e0 + e < N && k < d) ? w_r[(int64_t)(e0 + e) * d + k] : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 8
+            for (int kk = 0; kk < kKC; ++kk) {
+                float a[TT], b[TE];
+#pragma unroll
+                for (int i = 0; i < TT; ++i) a[i] = xs[kk * kTileT + ty + 16 * i];
+#pragma unroll
+                for (int j = 0; j < TE; ++j) b[j] = ws[kk * EC + tx + 16 * j];
+#pragma unroll
+                for (int i = 0; i < TT; ++i)
+#pragma unroll
+                    for (int j = 0; j < TE; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < TT; ++i)
+#pragma unroll
+            for (int j = 0; j < TE; ++j) {
+                const int e = e0 + tx + 16 * j;
+                if (e < N) logits[(ty + 16 * i) * NL + e] = acc[i][j];
+            }
+    }
+    __syncthreads();
+
+    constexpr int J = 8;  // up to 256 experts, 8 per lane
+    for (int r = warp; r < kTileT; r += kWarps) {
+        const int64_t t = t0 + r;
+        if (t >= T) break;
+        float v[J];
+        int idx[J];
+        bool own[J];
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int e = lane + 32 * j;
+            idx[j] = e < N ? e : -1;
+            own[j] = true;
+            v[j] = e < N ? logits[r * NL + e] + (bias ? bias[e] : 0.f) : 0.f;
+        }
+        token_epilogue<J>(v, idx, own, t, psum_w + warp * N, hist_w + warp * N, expert, gate);
+    }
+    __syncthreads();
+    publish_tile(psum_w, hist_w, N, tiles, tile, hist, psum);
+}
+
+// ---------------------------------------------------------------------------
+// Scan: one block per expert.
+// ---------------------------------------------------------------------------
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t *__restrict__ hist,
+                                                            const float *__restrict__ psum, int tiles, int N,
+                                                            int64_t T, int32_t *__restrict__ tile_off,
+                                                            int32_t *__restrict__ counts, double *prob_total,
+                                                            float *aux, uint32_t *ticket) {
+    __shared__ int32_t warp_cnt[kScanThreads / 32];
+    __shared__ double warp_p[kScanThreads / 32];
+    __shared__ bool is_last;
+    const int e = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int chunk = (tiles + kScanThreads - 1) / kScanThreads;
+    const int begin = min(tiles, tid * chunk), end = min(tiles, begin + chunk);
+    const int32_t *h = hist + (int64_t)e * tiles;
+    const float *ps = psum + (int64_t)e * tiles;
+
+    int32_t mine = 0;
+    double pmine = 0.0;
+    for (int i = begin; i < end; ++i) {
+        mine += h[i];
+        pmine += (double)ps[i];
+    }
+    // inclusive warp scan of the chunk totals
+    int32_t incl = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int32_t u = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += u;
+    }
+    double pw = pmine;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) pw += __shfl_xor_sync(0xffffffffu, pw, off);
+    if (lane == 31) warp_cnt[warp] = incl;
+    if (lane == 0) warp_p[warp] = pw;
+    __syncthreads();
+    if (warp == 0) {
+        int32_t c = warp_cnt[lane];
+        int32_t ci = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int32_t u = __shfl_up_sync(0xffffffffu, ci, off);
+            if (lane >= off) ci += u;
+        }
+        warp_cnt[lane] = ci - c;  // exclusive prefix of warp totals
+        if (lane == 31) counts[e] = ci;
+        if (lane == 0) {
+            double p = 0.0;
+            for (int w = 0; w < kScanThreads / 32; ++w) p += warp_p[w];
+            prob_total[e] = p;
+        }
+    }
+    __syncthreads();
+    int32_t run = warp_cnt[warp] + incl - mine;
+    for (int i = begin; i < end; ++i) {
+        tile_off[(int64_t)e * tiles + i] = run;
+        run += h[i];
+    }
+
+    // The last expert block to finish forms the aux loss, in fixed expert order.
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = atomicAdd(ticket, 1u) == (uint32_t)(N - 1);
+    __syncthreads();
+    if (is_last && tid == 0) {
+        __threadfence();
+        double total = 0.0;
+        if (T > 0) {
+            for (int i = 0; i < N; ++i) {
+                const double f = (double)((volatile int32_t *)counts)[i] / (double)T;
+                const double P = ((volatile double *)prob_total)[i] / (double)T;
+                total += f * P;
+            }
+        }
+        *aux = (float)((double)N * total);
+        *ticket = 0u;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Assignment: blocks [0, tiles) take one 64-token tile each (2 warps); every
+// block also clears a share of the empty slots of slot_token.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kTileT) assign_kernel(const int32_t *__restrict__ expert,
+                                                        const int32_t *__restrict__ tile_off,
+                                                        const int32_t *__restrict__ counts, int64_t T, int N, int C,
+                                                        int tiles, int32_t *__restrict__ slot,
+                                                        int32_t *__restrict__ slot_token) {
+    static_assert(kTileT == 64, "assignment assumes two warps per tile");
+    __shared__ int32_t first_warp_count[256];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tile = blockIdx.x;
+    if (tile < tiles) {
+        const int64_t t = (int64_t)tile * kTileT + tid;
+        const bool valid = t < T;
+        const int e = valid ? expert[t] : -1 - lane;  // distinct keys for absent tokens
+        for (int i = tid; i < N; i += kTileT) first_warp_count[i] = 0;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        int rank = __popc(same & (unsigned)lanemask_lt());
+        __syncthreads();
+        if (warp == 0 && valid && rank == 0) first_warp_count[e] = __popc(same);
+        __syncthreads();
+        if (valid) {
+            if (warp == 1) rank += first_warp_count[e];
+            const int s = tile_off[(int64_t)e * tiles + tile] + rank;
+            if (s < C) {
+                slot[t] = s;
+                slot_token[(int64_t)e * C + s] = (int32_t)t;
+            } else {
+                slot[t] = -1;
+            }
+        }
+    }
+    const int64_t total = (int64_t)N * C;
+    for (int64_t i = (int64_t)blockIdx.x * kTileT + tid; i < total; i += (int64_t)gridDim.x * kTileT) {
+        const int e = (int)(i / C);
+        const int s = (int)(i % C);
+        if (s >= min(counts[e], C)) slot_token[i] = -1;
+    }
+}
+
+template <typename XT, int NP>
+cudaError_t launch_router_warp(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
+                               int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
+    const int N = dims.num_experts, d = dims.d_model;
+    const size_t smem = (size_t)d * NP * sizeof(float) + (size_t)kWarps * N * (sizeof(float) + sizeof(int32_t));
+    auto kern = router_warp_kernel<XT, NP>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    launch_begin(K_ROUTER_WARP, stream);
+    kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
+                                                         ws.hist, ws.psum, ws.ticket);
+    err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
+
+template <typename XT, int EC>
+cudaError_t launch_router_tiled(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
+                                int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
+    const int N = dims.num_experts, d = dims.d_model;
+    const size_t smem = (size_t)(kKC * kTileT + kKC * EC + kTileT * (N + 1)) * sizeof(float) +
+                        (size_t)kWarps * N * (sizeof(float) + sizeof(int32_t));
+    auto kern = router_tiled_kernel<XT, EC>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    launch_begin(K_ROUTER_TILED, stream);
+    kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
+                                                         ws.hist, ws.psum, ws.ticket);
+    err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
+
+// Largest d for which the warp router keeps W_r in shared memory.
+constexpr size_t kWarpRouterSmemLimit = 160 * 1024;
+
+template <typename XT>
+cudaError_t launch_router(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
+                          int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
+    const int N = dims.num_experts;
+    const int NP = N <= 8 ? 8 : N <= 16 ? 16 : 32;
+    const bool fits = N <= 32 && (size_t)dims.d_model * NP * sizeof(float) + 2048 * 8 <= kWarpRouterSmemLimit;
+    if (fits) {
+        if (NP == 8) return launch_router_warp<XT, 8>(dims, x, w_r, bias, expert, gate, ws, stream);
+        if (NP == 16) return launch_router_warp<XT, 16>(dims, x, w_r, bias, expert, gate, ws, stream);
+        return launch_router_warp<XT, 32>(dims, x, w_r, bias, expert, gate, ws, stream);
+    }
+    if (N <= 32) return launch_router_tiled<XT, 32>(dims, x, w_r, bias, expert, gate, ws, stream);
+    if (N <= 64) return launch_router_tiled<XT, 64>(dims, x, w_r, bias, expert, gate, ws, stream);
+    return launch_router_tiled<XT, 128>(dims, x, w_r, bias, expert, gate, ws, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
+                         int32_t *expert, float *gate, int32_t *slot, int32_t *counts, int32_t *slot_token,
+                         float *aux, const Workspace &ws, cudaStream_t stream) {
+    cudaError_t err = cudaSuccess;
+    const int N = dims.num_experts, C = dims.capacity;
+    if (ws.tiles > 0) {
+        err = dims.dtype == SWITCH_BF16
+                  ? launch_router<__nv_bfloat16>(dims, static_cast<const __nv_bfloat16 *>(x), w_r, bias, expert,
+                                                 gate, ws, stream)
+                  : launch_router<float>(dims, static_cast<const float *>(x), w_r, bias, expert, gate, ws, stream);
+        if (err != cudaSuccess) return err;
+    } else {
+        // No router launch to reset the scan ticket: do it here.
+        err = cudaMemsetAsync(ws.ticket, 0, sizeof(uint32_t), stream);
+        if (err != cudaSuccess) return err;
+    }
+    launch_begin(K_SCAN, stream);
+    scan_kernel<<<N, kScanThreads, 0, stream>>>(ws.hist, ws.psum, (int)ws.tiles, N, dims.T, ws.tile_off, counts,
+                                                ws.prob_total, aux, ws.ticket);
+    err = cudaGetLastError();
+    launch_end(stream);
+    if (err != cudaSuccess) return err;
+    const int64_t fill_blocks = ((int64_t)N * C + kTileT * 16 - 1) / (kTileT * 16);
+    const int64_t grid = ws.tiles > fill_blocks ? ws.tiles : fill_blocks;
+    launch_begin(K_ASSIGN, stream);
+    assign_kernel<<<(unsigned)grid, kTileT, 0, stream>>>(expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles,
+                                                         slot, slot_token);
+    err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
+
+}  // namespace switchmoe

@@ -1,0 +1,114 @@
+"""GPU-vs-oracle comparison protocol for the Switch layer.
+
+* expert ids must equal the oracle's on every token whose top-2 logit margin
+  (oracle fp64 logits, bias included) exceeds 1e-5; near-tie tokens are
+  counted and their flips reported;
+* slot, counts and slot_token must equal, bit for bit, the oracle's
+  capacity step run on the GPU's own ids (this checks the scan whatever the
+  router did on near ties), and the oracle's own assignment when nothing
+  flipped;
+* aux within 1e-5 relative, gates within 1e-5 absolute of the oracle's p at
+  the GPU's expert;
+* outputs: max-abs error over kept rows <= 2e-2 x RMS(oracle kept rows) for
+  bf16 experts, <= 1e-4 x RMS for float32; dropped rows exactly 0.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as oracle_mod
+from sparse_mixture_experts_fp32_b200 import synth
+
+MARGIN = 1e-5
+TOL_BF16 = 2e-2
+TOL_F32 = 1e-4
+AUX_RTOL = 1e-5
+GATE_ATOL = 1e-5
+
+
+def to_device(a: np.ndarray | None, dev="cuda"):
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def y_to_numpy(y: torch.Tensor) -> np.ndarray:
+    return y.float().cpu().numpy().astype(np.float64)
+
+
+class Report(dict):
+    pass
+
+
+def check_routing(o: dict, g: dict, orc: oracle_mod.Oracle, N: int, C: int, T: int, check_slot_token=True) -> Report:
+    """o: oracle route() result (with probs); g: numpy copies of the GPU outputs."""
+    rep = Report()
+    near = o["margin"] <= MARGIN
+    far = ~near
+    mism = np.flatnonzero((g["expert"] != o["expert"]) & far)
+    assert mism.size == 0, f"{mism.size} expert ids differ on tokens with margin > {MARGIN}: {mism[:10]}"
+    flips = int(((g["expert"] != o["expert"]) & near).sum())
+    rep["near_ties"] = int(near.sum())
+    rep["flips"] = flips
+    a = orc.assign(g["expert"], N, C)
+    assert np.array_equal(g["counts"], a["counts"]), "counts differ from the oracle's count of the GPU ids"
+    bad = np.flatnonzero(g["slot"] != a["slot"])
+    assert bad.size == 0, f"{bad.size} slots differ from the oracle's assignment of the GPU ids: {bad[:10]}"
+    if check_slot_token:
+        assert np.array_equal(g["slot_token"].reshape(N, C), a["slot_token"]), "slot_token differs"
+    if flips == 0:
+        assert np.array_equal(g["slot"], o["slot"]) and np.array_equal(g["counts"], o["counts"])
+    # aux with the GPU's counts (identical to the oracle's when nothing flipped)
+    aux_ref = orc.aux(T, a["counts"], o["prob_sum"]) if T > 0 else 0.0
+    if T > 0:
+        rel = abs(float(g["aux"]) - aux_ref) / abs(aux_ref)
+        assert rel <= AUX_RTOL, f"aux {float(g['aux'])} vs {aux_ref} (rel {rel:.3e})"
+        rep["aux_rel_err"] = rel
+        p_at = o["probs"][np.arange(T), g["expert"]]
+        gerr = float(np.abs(g["gate"].astype(np.float64) - p_at).max())
+        assert gerr <= GATE_ATOL, f"gate error {gerr}"
+        rep["gate_max_err"] = gerr
+    rep["assign"] = a
+    rep["drops"] = int((a["slot"] < 0).sum())
+    return rep
+
+
+def check_outputs(y_gpu: np.ndarray, rows: np.ndarray, o: dict, rep: Report, orc, x, w_in, w_out, g_expert,
+                  fp32: bool) -> None:
+    """Compare GPU output rows (y_gpu[r] is token rows[r]) with the oracle's, using the GPU's ids."""
+    slot = rep["assign"]["slot"]
+    T = slot.shape[0]
+    gate = o["probs"][np.arange(T), g_expert]
+    ref = orc.output_rows(rows, x, w_in, w_out, g_expert, slot, gate)
+    got = y_gpu
+    kept = slot[rows] >= 0
+    if (~kept).any():
+        assert np.all(got[~kept] == 0.0), "a dropped token has a nonzero output row"
+    if kept.any():
+        rms = float(np.sqrt(np.mean(ref[kept] ** 2)))
+        err = float(np.abs(got[kept] - ref[kept]).max())
+        tol = (TOL_F32 if fp32 else TOL_BF16) * rms
+        rep["y_rms"] = rms
+        rep["y_max_abs_err"] = err
+        rep["y_err_over_rms"] = err / rms if rms > 0 else 0.0
+        assert err <= tol, f"max-abs output error {err:.4e} > {tol:.4e} (RMS {rms:.4e})"
+
+
+def oracle_route(orc, inp, C):
+    return orc.route(inp["x"], inp["w_r"], inp["bias"], capacity=C, want_probs=True)
+
+
+def workload_inputs(wl: synth.Workload, T=None, oracle_route_first=None, orc=None, C=None):
+    """Inputs for a workload; expert weights only for experts that the oracle
+    routes kept tokens to (other experts are zeros and are never read)."""
+    x = synth.activations(wl, T=T)
+    w_r = synth.router_weight(wl)
+    bias = synth.router_bias(wl)
+    inp = dict(x=x, w_r=w_r, bias=bias)
+    o = orc.route(x, w_r, bias, capacity=C, want_probs=True)
+    used = np.flatnonzero(np.minimum(o["counts"], C) > 0)
+    inp["w_in"], inp["w_out"] = synth.all_expert_weights(wl, experts=used)
+    return inp, o

@@ -1,0 +1,350 @@
+"""CUDA path (through the C ABI) against the fp64 oracle, element by element.
+
+Small cases run the whole layer for every token at sizes the oracle finishes
+in seconds (several tiles and a ragged tail); full-size cases run the five
+workloads exactly as the benchmark times them, comparing routing on every
+token and outputs on sampled rows.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_mixture_experts_fp32_b200 as sm
+from sparse_mixture_experts_fp32_b200 import synth
+from parity import (check_outputs, check_routing, oracle_route, to_device, workload_inputs, y_to_numpy)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.Oracle()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return sm.lib()
+
+
+def run_layer(inp, C, flags=0):
+    x = to_device(inp["x"])
+    out = sm.layer_fwd(x, to_device(inp["w_r"]), to_device(inp["w_in"]), to_device(inp["w_out"]), capacity=C,
+                       logit_bias=to_device(inp["bias"]), flags=flags)
+    assert sm.switch_check(out["workspace"]) == 0
+    g = {k: out[k].cpu().numpy() for k in ("expert", "gate", "slot", "counts", "aux")}
+    g["aux"] = g["aux"][0]
+    return g, y_to_numpy(out["y"]), out
+
+
+def full_check(orc, wl, T, C=None, flags=0, seed_rows=0):
+    C = C if C is not None else synth_capacity(wl, T)
+    inp, o = workload_inputs(wl, T=T, orc=orc, C=C)
+    g, y, _ = run_layer(inp, C, flags)
+    T = inp["x"].shape[0]
+    rep = check_routing(o, g, orc, wl.num_experts, C, T, check_slot_token=False)
+    rows = np.arange(T, dtype=np.int64)
+    check_outputs(y, rows, o, rep, orc, inp["x"], inp["w_in"], inp["w_out"], g["expert"], wl.dtype == synth.F32)
+    return rep
+
+
+def synth_capacity(wl, T):
+    return sm.switch_capacity(T, wl.num_experts, wl.capacity_factor)
+
+
+# ---------------------------------------------------------------------------
+# small cases: every token, every output element
+# ---------------------------------------------------------------------------
+SMALL = [("tiny_fp32", 64), ("base8", 1000), ("base128_skew", 4000), ("large128", 1500), ("bigexpert64", 300)]
+
+
+@pytest.mark.parametrize("name,T", SMALL, ids=[n for n, _ in SMALL])
+def test_layer_small_all_rows(orc, name, T, record_property):
+    rep = full_check(orc, synth.WORKLOADS[name], T)
+    for k in ("near_ties", "flips", "drops", "aux_rel_err", "y_err_over_rms"):
+        record_property(k, rep.get(k))
+
+
+@pytest.mark.parametrize("name,T", [("base8", 1000), ("large128", 700)])
+def test_layer_small_simt_ffn(orc, name, T):
+    full_check(orc, synth.WORKLOADS[name], T, flags=sm.SWITCH_FLAG_SIMT_FFN)
+
+
+def test_route_entry_point_slot_token(orc):
+    wl = synth.WORKLOADS["base128_skew"]
+    T = 5000
+    C = synth_capacity(wl, T)
+    x, w_r, bias = synth.activations(wl, T=T), synth.router_weight(wl), synth.router_bias(wl)
+    r = sm.route(to_device(x), to_device(w_r), capacity=C, logit_bias=to_device(bias), d_ff=wl.d_ff)
+    assert sm.switch_check(r["workspace"]) == 0
+    g = {k: r[k].cpu().numpy() for k in ("expert", "gate", "slot", "counts", "slot_token", "aux")}
+    g["aux"] = g["aux"][0]
+    o = orc.route(x, w_r, bias, capacity=C, want_probs=True)
+    check_routing(o, g, orc, wl.num_experts, C, T, check_slot_token=True)
+
+
+def test_entry_points_compose_to_layer(orc):
+    """route -> dispatch -> expert_ffn -> combine gives the same bytes as layer_fwd."""
+    wl = synth.WORKLOADS["base8"]
+    T = 2000
+    C = synth_capacity(wl, T)
+    inp = synth.inputs(wl, T=T)
+    dev = {k: to_device(v) for k, v in inp.items()}
+    ref = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C)
+    d = sm.layer_dims(dev["x"], dev["w_in"], capacity=C)
+    ws = sm.workspace(d, "cuda")
+    N, dm = wl.num_experts, wl.d_model
+    expert = torch.empty(T, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, dtype=torch.float32, device="cuda")
+    slot = torch.empty(T, dtype=torch.int32, device="cuda")
+    counts = torch.empty(N, dtype=torch.int32, device="cuda")
+    slot_token = torch.empty(N * C, dtype=torch.int32, device="cuda")
+    aux = torch.empty(1, dtype=torch.float32, device="cuda")
+    xbuf = torch.empty(N * C * dm, dtype=torch.bfloat16, device="cuda")
+    ybuf = torch.empty(N * C * dm, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty_like(dev["x"])
+    sm.switch_route(d, dev["x"], dev["w_r"], None, expert, gate, slot, counts, slot_token, aux, ws)
+    sm.switch_dispatch(d, dev["x"], slot_token, counts, xbuf)
+    sm.switch_expert_ffn(d, xbuf, dev["w_in"], dev["w_out"], counts, ybuf, ws)
+    sm.switch_combine(d, ybuf, expert, slot, gate, y)
+    assert sm.switch_check(ws) == 0
+    assert torch.equal(expert, ref["expert"]) and torch.equal(slot, ref["slot"])
+    assert torch.equal(counts, ref["counts"]) and torch.equal(aux, ref["aux"])
+    assert torch.equal(y.view(torch.int16), ref["y"].view(torch.int16))
+    # dispatch wrote exactly the kept tokens' rows
+    kept = torch.clamp(counts, max=C).cpu().numpy()
+    st = slot_token.view(N, C).cpu().numpy()
+    xb = xbuf.view(N, C, dm).cpu()
+    for e in range(N):
+        if kept[e]:
+            assert torch.equal(xb[e, :kept[e]].view(torch.int16),
+                               dev["x"][torch.from_numpy(st[e, :kept[e]]).long().cuda()].cpu().view(torch.int16))
+
+
+def test_deterministic_bytes(orc):
+    wl = synth.WORKLOADS["base128_skew"]
+    inp = synth.inputs(wl, T=6000, experts=range(8))
+    dev = {k: to_device(v) for k, v in inp.items()}
+    C = synth_capacity(wl, 6000)
+    a = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, logit_bias=dev["bias"])
+    b = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, logit_bias=dev["bias"])
+    for k in ("expert", "gate", "slot", "counts", "aux"):
+        assert torch.equal(a[k], b[k]), k
+    assert torch.equal(a["y"].view(torch.int16), b["y"].view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# edge cases
+# ---------------------------------------------------------------------------
+def _random_inputs(rng, T, d, F, N, dtype, w_scale=1.0, bias=True):
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    w_r = (rng.standard_normal((N, d)) * w_scale / np.sqrt(d)).astype(np.float32)
+    b = (rng.standard_normal(N) * 0.2).astype(np.float32) if bias else None
+    w_in = (rng.standard_normal((N, F, d)) / np.sqrt(d)).astype(np.float32)
+    w_out = (rng.standard_normal((N, d, F)) / np.sqrt(F)).astype(np.float32)
+    if dtype == "bf16":
+        x, w_in, w_out = synth.to_bf16_bits(x), synth.to_bf16_bits(w_in), synth.to_bf16_bits(w_out)
+    return dict(x=x, w_r=w_r, bias=b, w_in=w_in, w_out=w_out)
+
+
+EDGE = [
+    # name, T, d, F, N, C, dtype
+    ("one_token", 1, 64, 64, 4, 1, "bf16"),
+    ("ragged_tail", 1000, 128, 192, 6, 120, "bf16"),
+    ("capacity_one", 500, 64, 128, 5, 1, "bf16"),
+    ("no_drops", 700, 64, 64, 3, 700, "bf16"),
+    ("big_capacity_few_tokens", 100, 64, 64, 4, 4096, "bf16"),
+    ("partial_column_tile", 400, 192, 320, 4, 150, "bf16"),
+    ("max_experts", 3000, 64, 128, 256, 12, "bf16"),
+    ("experts_33", 2000, 128, 128, 33, 70, "bf16"),
+    ("d_model_4096", 300, 4096, 128, 2, 160, "bf16"),
+    ("f32_odd_shapes", 77, 33, 17, 3, 30, "f32"),
+    ("f32_many_experts", 900, 48, 40, 70, 16, "f32"),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[c[0] for c in EDGE])
+def test_edge_cases(orc, case):
+    name, T, d, F, N, C, dt = case
+    inp = _random_inputs(np.random.default_rng(zlib.crc32(name.encode())), T, d, F, N, dt)
+    g, y, _ = run_layer(inp, C)
+    o = oracle_route(orc, inp, C)
+    rep = check_routing(o, g, orc, N, C, T, check_slot_token=False)
+    check_outputs(y, np.arange(T), o, rep, orc, inp["x"], inp["w_in"], inp["w_out"], g["expert"], dt == "f32")
+
+
+def test_single_expert_is_dense_ffn(orc):
+    rng = np.random.default_rng(11)
+    inp = _random_inputs(rng, 640, 256, 512, 1, "bf16")
+    g, y, _ = run_layer(inp, C=640)
+    assert np.all(g["expert"] == 0) and np.all(g["gate"] == 1.0) and np.all(g["slot"] == np.arange(640))
+    assert g["aux"] == 1.0
+    x = synth.bf16_bits_to_f32(inp["x"]).astype(np.float64)
+    wi = synth.bf16_bits_to_f32(inp["w_in"][0]).astype(np.float64)
+    wo = synth.bf16_bits_to_f32(inp["w_out"][0]).astype(np.float64)
+    dense = np.maximum(x @ wi.T, 0) @ wo.T
+    rms = np.sqrt(np.mean(dense ** 2))
+    assert np.abs(y - dense).max() <= 2e-2 * rms
+
+
+def test_zero_router_all_ties(orc):
+    rng = np.random.default_rng(12)
+    inp = _random_inputs(rng, 300, 64, 64, 8, "bf16", bias=False)
+    inp["w_r"][:] = 0.0
+    g, y, _ = run_layer(inp, C=40)
+    assert np.all(g["expert"] == 0)
+    assert g["counts"].tolist() == [300] + [0] * 7
+    assert np.array_equal(g["slot"], np.where(np.arange(300) < 40, np.arange(300), -1))
+    assert abs(g["aux"] - 1.0) <= 1e-6
+    assert np.all(g["gate"] == np.float32(1.0 / 8))
+    assert np.all(y[40:] == 0)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_empty_input(dt):
+    d = 64
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    x = torch.empty(0, d, dtype=tdt, device="cuda")
+    w_r = torch.randn(4, d, device="cuda")
+    w_in = torch.randn(4, 64, d, device="cuda").to(tdt)
+    w_out = torch.randn(4, d, 64, device="cuda").to(tdt)
+    out = sm.layer_fwd(x, w_r, w_in, w_out, capacity=3)
+    assert sm.switch_check(out["workspace"]) == 0
+    assert out["counts"].tolist() == [0, 0, 0, 0]
+    assert out["aux"].item() == 0.0
+    r = sm.route(x, w_r, capacity=3)
+    assert torch.all(r["slot_token"] == -1)
+
+
+def test_outputs_stay_in_bounds(orc):
+    """Every output is a window of a larger sentinel-filled buffer; nothing
+    outside the windows may change."""
+    rng = np.random.default_rng(13)
+    T, d, F, N, C = 777, 128, 256, 5, 100
+    inp = _random_inputs(rng, T, d, F, N, "bf16")
+    dev = {k: to_device(v) for k, v in inp.items()}
+    pad = 4096
+
+    def guarded(n, dtype):
+        big = torch.full((n + 2 * pad,), -7, dtype=dtype, device="cuda")
+        return big, big[pad:pad + n]
+
+    yb, y = guarded(T * d, torch.int16)
+    eb, e = guarded(T, torch.int32)
+    gb, gt = guarded(T, torch.float32)
+    sb, s = guarded(T, torch.int32)
+    cb, c = guarded(N, torch.int32)
+    ab, a = guarded(1, torch.float32)
+    dims = sm.dims(T, d, F, N, C, sm.SWITCH_BF16)
+    wsz = sm.switch_workspace_size(dims)
+    wb, ws = guarded(wsz, torch.uint8)
+    sm.switch_layer_fwd(dims, dev["x"], dev["w_r"], dev["bias"], dev["w_in"], dev["w_out"], y, e, gt, s, c, a, ws)
+    assert sm.switch_check(ws) == 0
+    for big in (yb, eb, gb, sb, cb, ab, wb):
+        head, tail = big[:pad], big[-pad:]
+        assert torch.all(head == -7) and torch.all(tail == -7)
+    o = oracle_route(orc, inp, C)
+    g = dict(expert=e.cpu().numpy(), gate=gt.cpu().numpy(), slot=s.cpu().numpy(), counts=c.cpu().numpy(),
+             aux=a.cpu().numpy()[0])
+    rep = check_routing(o, g, orc, N, C, T, check_slot_token=False)
+    yy = y.view(torch.bfloat16).view(T, d).float().cpu().numpy().astype(np.float64)
+    check_outputs(yy, np.arange(T), o, rep, orc, inp["x"], inp["w_in"], inp["w_out"], g["expert"], False)
+
+
+def test_errors_leave_outputs_untouched():
+    T, d, F, N, C = 64, 64, 64, 4, 16
+    x = torch.randn(T, d, device="cuda").bfloat16()
+    w_r = torch.randn(N, d, device="cuda")
+    w_in = torch.randn(N, F, d, device="cuda").bfloat16()
+    w_out = torch.randn(N, d, F, device="cuda").bfloat16()
+    y = torch.full((T, d), 3.0, device="cuda").bfloat16()
+    dims = sm.dims(T, d, F, N, C, sm.SWITCH_BF16)
+    ws_small = torch.empty(64, dtype=torch.uint8, device="cuda")
+    counts = torch.full((N,), 9, dtype=torch.int32, device="cuda")
+    other = [torch.full((T,), 5, dtype=torch.int32, device="cuda") for _ in range(3)]
+    aux = torch.full((1,), 2.0, device="cuda")
+    with pytest.raises(sm.SwitchError) as ei:
+        sm.switch_layer_fwd(dims, x, w_r, None, w_in, w_out, y, other[0], other[1].float(), other[2], counts, aux,
+                            ws_small)
+    assert ei.value.status == 5
+    torch.cuda.synchronize()
+    assert torch.all(y.float() == 3.0) and torch.all(counts == 9) and aux.item() == 2.0
+
+
+def test_tracer_and_launch_counter():
+    wl = synth.WORKLOADS["base8"]
+    inp = synth.inputs(wl, T=512)
+    dev = {k: to_device(v) for k, v in inp.items()}
+    before = sm.launch_count()
+    sm.trace_start(64)
+    out = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity_factor=1.25)
+    torch.cuda.synchronize()
+    trace = sm.trace_read()
+    sm.trace_stop()
+    names = [n for n, _ in trace]
+    assert names == ["router_warp", "capacity_scan", "slot_assign", "dispatch", "ffn_tc_gemm1_relu",
+                     "ffn_tc_gemm2", "combine"]
+    assert all(ms >= 0 for _, ms in trace)
+    assert sm.launch_count() - before == len(names)
+    assert sm.switch_check(out["workspace"]) == 0
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, as timed by the benchmark
+# ---------------------------------------------------------------------------
+def _sample_rows(slot, n_kept=256, n_any=64, seed=0):
+    rng = np.random.default_rng(seed)
+    kept = np.flatnonzero(slot >= 0)
+    pick = rng.choice(kept, size=min(n_kept, kept.size), replace=False) if kept.size else np.array([], np.int64)
+    extra = rng.choice(slot.shape[0], size=min(n_any, slot.shape[0]), replace=False)
+    return np.unique(np.concatenate([pick, extra]).astype(np.int64))
+
+
+def _full_size(orc, wl, cs, record_property):
+    x = synth.activations(wl)
+    w_r = synth.router_weight(wl)
+    bias = synth.router_bias(wl)
+    T, N = x.shape[0], wl.num_experts
+    h = orc.router_logits(x, w_r, bias)
+    sm_ = orc.softmax_top1(h, want_probs=True)
+    Cs = [sm.switch_capacity(T, N, c) for c in cs]
+    used = set()
+    for C in Cs:
+        used |= set(np.flatnonzero(np.minimum(np.bincount(sm_["expert"], minlength=N), C) > 0).tolist())
+    w_in, w_out = synth.all_expert_weights(wl, experts=sorted(used))
+    dx, dwr, db = to_device(x), to_device(w_r), to_device(bias)
+    dwi, dwo = to_device(w_in), to_device(w_out)
+    for c, C in zip(cs, Cs):
+        o = dict(sm_)
+        o.update(orc.assign(sm_["expert"], N, C))
+        o["aux"] = orc.aux(T, o["counts"], o["prob_sum"])
+        out = sm.layer_fwd(dx, dwr, dwi, dwo, capacity=C, logit_bias=db)
+        assert sm.switch_check(out["workspace"]) == 0
+        g = {k: out[k].cpu().numpy() for k in ("expert", "gate", "slot", "counts", "aux")}
+        g["aux"] = g["aux"][0]
+        rep = check_routing(o, g, orc, N, C, T, check_slot_token=False)
+        # every dropped row is exactly zero, checked on the device
+        dropped = torch.from_numpy(rep["assign"]["slot"] < 0).cuda()
+        assert torch.all(out["y"][dropped] == 0)
+        rows = _sample_rows(rep["assign"]["slot"])
+        y_rows = out["y"][torch.from_numpy(rows).cuda()].float().cpu().numpy().astype(np.float64)
+        check_outputs(y_rows, rows, o, rep, orc, x, w_in, w_out, g["expert"], wl.dtype == synth.F32)
+        record_property(f"c={c}", {k: rep.get(k) for k in ("near_ties", "flips", "drops", "aux_rel_err",
+                                                             "y_err_over_rms")})
+        del out
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "base8", "base128_skew", "large128"])
+def test_full_size(orc, name, record_property):
+    wl = synth.WORKLOADS[name]
+    _full_size(orc, wl, [wl.capacity_factor], record_property)
+
+
+def test_full_size_bigexpert_capacity_sweep(orc, record_property):
+    wl = synth.WORKLOADS["bigexpert64"]
+    _full_size(orc, wl, list(wl.sweep), record_property)
