@@ -62,8 +62,11 @@ typedef enum {
     SWITCH_ERR_DEVICE_TIMEOUT = 8  /* a kernel gave up a bounded wait (reported by switch_check) */
 } switch_status_t;
 
-/* Storage type of activations (x, y, xbuf, ybuf) and expert weights (W_in,
- * W_out).  The router weight, the logit bias and the gates are always float32. */
+/* Storage type of the input activations (x, xbuf) and of the expert weights
+ * (W_in, W_out).  The router weight, the logit bias, the gates, the expert
+ * outputs (ybuf) and the layer output (y) are always float32: the expert
+ * output stays in the float32 accumulator precision until it is scaled by
+ * its gate, and the result is rounded once. */
 typedef enum {
     SWITCH_F32 = 0,  /* IEEE binary32 */
     SWITCH_BF16 = 1  /* bfloat16 */
@@ -139,7 +142,7 @@ switch_status_t switch_dispatch(const switch_dims_t *dims, const void *x, const 
  *   xbuf  [N, C, d]   activation dtype
  *   w_in  [N, F, d]   expert dtype (nn.Linear layout: row j feeds hidden unit j)
  *   w_out [N, d, F]   expert dtype
- *   ybuf  [N, C, d]   activation dtype; other rows are not written
+ *   ybuf  [N, C, d]   float32; other rows are not written
  * bfloat16: tcgen05 tensor cores, float32 accumulation, the hidden
  * activations rounded to bfloat16 in the workspace.  float32: CUDA cores.
  * (Switch FFN experts: llm-papers-study §3.2; two-layer ReLU experts without
@@ -153,22 +156,28 @@ switch_status_t switch_expert_ffn(const switch_dims_t *dims, const void *xbuf, c
  * expert):
  *   y[t, :] = gate[t] * ybuf[expert[t], slot[t], :]   if slot[t] >= 0
  *   y[t, :] = 0                                       if slot[t] == -1
- * The product is formed in float32 and rounded once to the activation dtype.
- *   ybuf [N, C, d], expert [T], slot [T], gate [T]  ->  y [T, d] */
+ * The product is formed in float32.
+ *   ybuf [N, C, d] float32, expert [T], slot [T], gate [T]  ->  y [T, d] float32 */
 switch_status_t switch_combine(const switch_dims_t *dims, const void *ybuf, const int32_t *expert,
                                const int32_t *slot, const float *gate, void *y, switch_stream_t stream);
 
 /* The whole layer: switch_route, then dispatch, expert FFN and combine, with
  * the [N, C, d] buffers and slot_token kept in the workspace.  Arguments as
- * above; y [T, d] is the layer output WITHOUT the residual. */
+ * above; y [T, d] float32 is the layer output WITHOUT the residual.  On the
+ * bfloat16 tensor-core path the dispatch is fused into the slot assignment
+ * and the combine into the second expert GEMM; the result is bit-identical
+ * to calling the four steps one by one. */
 switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const float *w_r,
                                  const float *logit_bias, const void *w_in, const void *w_out, void *y,
                                  int32_t *expert, float *gate, int32_t *slot, int32_t *counts, float *aux,
                                  void *workspace, size_t workspace_bytes, switch_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the device status word kept in
- * `workspace`.  Returns SWITCH_OK, SWITCH_ERR_DEVICE_TIMEOUT, or
- * SWITCH_ERR_CUDA if the stream reports an error. */
+ * `workspace`.  switch_route, switch_expert_ffn and switch_layer_fwd clear
+ * that word before their first kernel runs, so the workspace needs no
+ * initialisation; switch_check reports the first failure recorded since.
+ * Returns SWITCH_OK, SWITCH_ERR_DEVICE_TIMEOUT, or SWITCH_ERR_CUDA if the
+ * stream reports an error. */
 switch_status_t switch_check(void *workspace, size_t workspace_bytes, switch_stream_t stream);
 
 /* Static description of a status code. */

@@ -251,13 +251,13 @@ def layer_dims(x, w_in, capacity=None, capacity_factor=None, flags: int = 0) -> 
 
 def layer_fwd(x, w_r, w_in, w_out, capacity=None, capacity_factor=None, logit_bias=None, flags: int = 0,
               ws=None, out=None, stream=None):
-    """The Switch layer forward pass.  Returns a dict with y [T, d] (no
-    residual), aux (1-element float32), expert, gate, slot, counts."""
+    """The Switch layer forward pass.  Returns a dict with y [T, d] float32
+    (no residual), aux (1-element float32), expert, gate, slot, counts."""
     import torch
     d = layer_dims(x, w_in, capacity, capacity_factor, flags)
     T, dev = x.shape[0], x.device
     if out is None:
-        out = dict(y=torch.empty_like(x), expert=torch.empty(T, dtype=torch.int32, device=dev),
+        out = dict(y=torch.empty(x.shape, dtype=torch.float32, device=dev), expert=torch.empty(T, dtype=torch.int32, device=dev),
                    gate=torch.empty(T, dtype=torch.float32, device=dev),
                    slot=torch.empty(T, dtype=torch.int32, device=dev),
                    counts=torch.empty(d.num_experts, dtype=torch.int32, device=dev),

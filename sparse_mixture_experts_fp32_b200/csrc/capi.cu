@@ -45,7 +45,7 @@ Sections layout(const switch_dims_t &d) {
     s.prob_total = take(N * 8);
     s.slot_token = take(N * C * 4);
     s.xbuf = take(N * C * (size_t)d.d_model * elem_size(d));
-    s.ybuf = take(N * C * (size_t)d.d_model * elem_size(d));
+    s.ybuf = take(N * C * (size_t)d.d_model * sizeof(float));
     s.hidden = take(N * C * (size_t)d.d_ff * elem_size(d));
     s.total = off;
     return s;
@@ -144,7 +144,7 @@ Workspace carve_workspace(const switch_dims_t &dims, void *base) {
     w.prob_total = reinterpret_cast<double *>(b + s.prob_total);
     w.slot_token = reinterpret_cast<int32_t *>(b + s.slot_token);
     w.xbuf = b + s.xbuf;
-    w.ybuf = b + s.ybuf;
+    w.ybuf = reinterpret_cast<float *>(b + s.ybuf);
     w.hidden = b + s.hidden;
     w.tiles = tiles_of(dims);
     return w;
@@ -235,8 +235,10 @@ switch_status_t switch_expert_ffn(const switch_dims_t *dims, const void *xbuf, c
     const Workspace ws = carve_workspace(*dims, workspace);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool tensor_cores = dims->dtype == SWITCH_BF16 && !(dims->flags & SWITCH_FLAG_SIMT_FFN);
-    return from_cuda(tensor_cores ? launch_ffn_tc(*dims, xbuf, w_in, w_out, counts, ybuf, ws, st)
-                                  : launch_ffn_simt(*dims, xbuf, w_in, w_out, counts, ybuf, ws, st));
+    float *yb = static_cast<float *>(ybuf);
+    if (cudaMemsetAsync(ws.status, 0, sizeof(DeviceStatus), st) != cudaSuccess) return SWITCH_ERR_CUDA;
+    return from_cuda(tensor_cores ? launch_ffn_tc(*dims, xbuf, w_in, w_out, counts, yb, nullptr, nullptr, nullptr, ws, st)
+                                  : launch_ffn_simt(*dims, xbuf, w_in, w_out, counts, yb, ws, st));
 }
 
 switch_status_t switch_combine(const switch_dims_t *dims, const void *ybuf, const int32_t *expert,
@@ -248,7 +250,8 @@ switch_status_t switch_combine(const switch_dims_t *dims, const void *ybuf, cons
         if (s != SWITCH_OK) return s;
     }
     if ((s = check_device()) != SWITCH_OK) return s;
-    return from_cuda(launch_combine(*dims, ybuf, expert, slot, gate, y, reinterpret_cast<cudaStream_t>(stream)));
+    return from_cuda(launch_combine(*dims, static_cast<const float *>(ybuf), expert, slot, gate,
+                                    static_cast<float *>(y), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const float *w_r, const float *logit_bias,
@@ -267,14 +270,24 @@ switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const
     if ((s = check_device()) != SWITCH_OK) return s;
     const Workspace ws = carve_workspace(*dims, workspace);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t err = launch_route(*dims, x, w_r, logit_bias, expert, gate, slot, counts, ws.slot_token, aux, ws, st);
-    if (err == cudaSuccess) err = launch_dispatch(*dims, x, ws.slot_token, counts, ws.xbuf, st);
-    if (err == cudaSuccess) {
-        const bool tensor_cores = dims->dtype == SWITCH_BF16 && !(dims->flags & SWITCH_FLAG_SIMT_FFN);
-        err = tensor_cores ? launch_ffn_tc(*dims, ws.xbuf, w_in, w_out, counts, ws.ybuf, ws, st)
-                           : launch_ffn_simt(*dims, ws.xbuf, w_in, w_out, counts, ws.ybuf, ws, st);
+    float *yf = static_cast<float *>(y);
+    const bool tensor_cores = dims->dtype == SWITCH_BF16 && !(dims->flags & SWITCH_FLAG_SIMT_FFN);
+    const bool rows16 = ((int64_t)dims->d_model * (int64_t)elem_size(*dims)) % 16 == 0;
+    cudaError_t err;
+    if (tensor_cores) {
+        // route + scatter-dispatch (zeroing dropped rows of y), GEMM1, GEMM2 with
+        // the gate and the token-order scatter fused into its epilogue
+        err = launch_route(*dims, x, w_r, logit_bias, expert, gate, slot, counts, ws.slot_token, aux, ws, st,
+                           ws.xbuf, yf);
+        if (err == cudaSuccess)
+            err = launch_ffn_tc(*dims, ws.xbuf, w_in, w_out, counts, nullptr, ws.slot_token, gate, yf, ws, st);
+    } else {
+        err = launch_route(*dims, x, w_r, logit_bias, expert, gate, slot, counts, ws.slot_token, aux, ws, st,
+                           rows16 ? ws.xbuf : nullptr, nullptr);
+        if (err == cudaSuccess && !rows16) err = launch_dispatch(*dims, x, ws.slot_token, counts, ws.xbuf, st);
+        if (err == cudaSuccess) err = launch_ffn_simt(*dims, ws.xbuf, w_in, w_out, counts, ws.ybuf, ws, st);
+        if (err == cudaSuccess) err = launch_combine(*dims, ws.ybuf, expert, slot, gate, yf, st);
     }
-    if (err == cudaSuccess) err = launch_combine(*dims, ws.ybuf, expert, slot, gate, y, st);
     return from_cuda(err);
 }
 
@@ -360,6 +373,8 @@ const char *switch_kernel_name(int32_t id) {
         case K_FFN_SIMT_GEMM1: return "ffn_simt_gemm1_relu";
         case K_FFN_SIMT_GEMM2: return "ffn_simt_gemm2";
         case K_COMBINE: return "combine";
+        case K_FFN_TC_GEMM2_GATED: return "ffn_tc_gemm2_gated_scatter";
+        case K_ASSIGN_SCATTER: return "slot_assign_scatter";
     }
     return "?";
 }

@@ -5,10 +5,16 @@
 // over the kept rows s < min(counts[i], C) of every expert i.  Both GEMMs
 // are the same grouped "A . B^T" kernel with both operands K-major (the
 // nn.Linear weight layout), bf16 inputs and fp32 accumulation in tensor
-// memory; the epilogue applies ReLU (GEMM1), rounds to bf16 and stores rows
-// below the expert's kept count.  (Expert FFN: llm-papers-study "精读 06 |
-// Switch Transformers" §3.2; bfloat16 experts with float32 accumulation:
-// kasblo section "Routerだけfloat32で計算するSelective Precision".)
+// memory.  Epilogues (rows below the expert's kept count only):
+//   kEpiHiddenRelu   ReLU, round to bf16, store H[i, s, :]
+//   kEpiExpertOut    store the fp32 accumulator as ybuf[i, s, :]
+//   kEpiGatedScatter y[t, :] = gate[t] * acc in fp32, t = slot_token[i*C+s]
+//                    (the combine step fused into GEMM2: the expert output
+//                    goes straight to token order, scaled by its gate, and
+//                    is rounded once, to float32)
+// (Expert FFN and y = p_i* E_i*(x): llm-papers-study "精读 06 | Switch
+// Transformers" §3.2; bfloat16 experts with float32 accumulation: kasblo
+// section "Routerだけfloat32で計算するSelective Precision".)
 //
 // Kernel structure (one CTA per SM, persistent over a tile list that every
 // CTA derives on the device from `counts`, so no host synchronisation):
@@ -17,8 +23,9 @@
 //   warp 1      allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN,
 //               K=16) into one of two TMEM accumulators and commits to
 //               mbarriers that free ring slots / publish the accumulator
-//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes, ReLU, bf16,
-//               16-byte stores; then release the accumulator
+//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes (one thread per
+//               row), then one of the epilogues above with 16-byte
+//               stores; then release the accumulator
 // Every mbarrier wait is bounded (about 1 s); on a timeout the kernel records
 // SWITCH_ERR_DEVICE_TIMEOUT in the status word, waits (bounded) for its own
 // TMA loads and MMAs in flight, frees TMEM and returns.
@@ -58,11 +65,13 @@ __device__ __forceinline__ void locate_tile(const int32_t *tile_start, int E, in
     n = local % n_tiles_n;
 }
 
-template <int BN, int STAGES, bool RELU>
+enum Epilogue { kEpiHiddenRelu = 0, kEpiExpertOut = 1, kEpiGatedScatter = 2 };
+
+template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_grouped_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                    __nv_bfloat16 *__restrict__ out, const int32_t *__restrict__ counts, int E, int C, int K,
-                    int Nout, DeviceStatus *status) {
+                    void *__restrict__ out, const int32_t *__restrict__ counts, int E, int C, int K, int Nout,
+                    const int32_t *__restrict__ slot_token, const float *__restrict__ gate, DeviceStatus *status) {
     using L = TcLayout<BN, STAGES>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -210,7 +219,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kept = min(counts[e], C);
             const int row = m * BM + row_in_tile;
             const bool row_ok = row < kept;
-            __nv_bfloat16 *orow = out + ((int64_t)e * C + row) * Nout;
+            // destination row of this thread (a token row for the gated scatter)
+            int64_t out_row = (int64_t)e * C + row;
+            float g = 1.f;
+            if (EPI == kEpiGatedScatter && row_ok) {
+                out_row = slot_token[(int64_t)e * C + row];
+                g = gate[out_row];
+            }
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
 #pragma unroll 1
             for (int c = 0; c < BN; c += 32) {
@@ -219,17 +234,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_wait();
                 const int col0 = n * BN + c;
                 if (row_ok && col0 < Nout) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + col0);
+                    if (EPI == kEpiHiddenRelu) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + out_row * Nout + col0);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float v[8];
+                        for (int q = 0; q < 4; ++q) {
+                            float v[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            v[i] = __uint_as_float(r[8 * q + i]);
-                            if (RELU) v[i] = fmaxf(v[i], 0.f);
+                            for (int i = 0; i < 8; ++i) v[i] = fmaxf(__uint_as_float(r[8 * q + i]), 0.f);
+                            dst[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                                pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
                         }
-                        dst[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                    } else {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + out_row * Nout + col0);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            dst[q] = make_float4(g * __uint_as_float(r[4 * q + 0]), g * __uint_as_float(r[4 * q + 1]),
+                                                 g * __uint_as_float(r[4 * q + 2]), g * __uint_as_float(r[4 * q + 3]));
                     }
                 }
             }
@@ -282,13 +302,14 @@ bool make_tmap(CUtensorMap *map, const void *ptr, int E, int rows, int K, int bo
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, bool RELU>
+template <int BN, int STAGES, int EPI>
 cudaError_t launch_gemm(int32_t kernel_id, const void *a, const void *b, void *out, const int32_t *counts, int E,
-                        int C, int K, int Nout, int64_t T, DeviceStatus *status, cudaStream_t stream) {
+                        int C, int K, int Nout, int64_t T, const int32_t *slot_token, const float *gate,
+                        DeviceStatus *status, cudaStream_t stream) {
     CUtensorMap ta, tb;
     if (!make_tmap(&ta, a, E, C, K, BM) || !make_tmap(&tb, b, E, Nout, K, BN)) return cudaErrorInvalidValue;
     const size_t smem = TcLayout<BN, STAGES>::bytes(E);
-    auto kern = tc_grouped_gemm<BN, STAGES, RELU>;
+    auto kern = tc_grouped_gemm<BN, STAGES, EPI>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     // Upper bound on the number of tiles, from host-known sizes only.
@@ -296,7 +317,7 @@ cudaError_t launch_gemm(int32_t kernel_id, const void *a, const void *b, void *o
     const int64_t tiles = m_tiles * ((Nout + BN - 1) / BN);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count(), tiles));
     launch_begin(kernel_id, stream);
-    kern<<<grid, kThreads, smem, stream>>>(ta, tb, static_cast<__nv_bfloat16 *>(out), counts, E, C, K, Nout, status);
+    kern<<<grid, kThreads, smem, stream>>>(ta, tb, out, counts, E, C, K, Nout, slot_token, gate, status);
     err = cudaGetLastError();
     launch_end(stream);
     return err;
@@ -305,14 +326,18 @@ cudaError_t launch_gemm(int32_t kernel_id, const void *a, const void *b, void *o
 }  // namespace
 
 cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
-                          const int32_t *counts, void *ybuf, const Workspace &ws, cudaStream_t stream) {
+                          const int32_t *counts, void *ybuf, const int32_t *slot_token, const float *gate, float *y,
+                          const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts, C = dims.capacity, d = dims.d_model, F = dims.d_ff;
     DeviceStatus *st = static_cast<DeviceStatus *>(ws.status);
-    cudaError_t err = launch_gemm<256, 4, true>(K_FFN_TC_GEMM1, xbuf, w_in, ws.hidden, counts, N, C, d, F, dims.T,
-                                                st, stream);
+    cudaError_t err = launch_gemm<256, 4, kEpiHiddenRelu>(K_FFN_TC_GEMM1, xbuf, w_in, ws.hidden, counts, N, C, d, F,
+                                                          dims.T, nullptr, nullptr, st, stream);
     if (err != cudaSuccess) return err;
-    return launch_gemm<128, 6, false>(K_FFN_TC_GEMM2, ws.hidden, w_out, ybuf, counts, N, C, F, d, dims.T, st,
-                                      stream);
+    if (y)
+        return launch_gemm<128, 6, kEpiGatedScatter>(K_FFN_TC_GEMM2_GATED, ws.hidden, w_out, y, counts, N, C, F, d,
+                                                     dims.T, slot_token, gate, st, stream);
+    return launch_gemm<128, 6, kEpiExpertOut>(K_FFN_TC_GEMM2, ws.hidden, w_out, ybuf, counts, N, C, F, d, dims.T,
+                                              nullptr, nullptr, st, stream);
 }
 
 }  // namespace switchmoe

@@ -25,6 +25,8 @@ enum KernelId : int32_t {
     K_FFN_SIMT_GEMM1 = 8,
     K_FFN_SIMT_GEMM2 = 9,
     K_COMBINE = 10,
+    K_FFN_TC_GEMM2_GATED = 11,
+    K_ASSIGN_SCATTER = 12,
 };
 
 struct Workspace {
@@ -36,7 +38,7 @@ struct Workspace {
     double *prob_total;  // [N] sum of p_i over all tokens
     int32_t *slot_token; // [N*C] (layer_fwd only)
     void *xbuf;          // [N][C][d] (layer_fwd only)
-    void *ybuf;          // [N][C][d] (layer_fwd only)
+    float *ybuf;         // [N][C][d] float32 (layer_fwd only)
     void *hidden;        // [N][C][F] expert hidden activations
     int64_t tiles;
 };
@@ -49,17 +51,25 @@ void launch_begin(int32_t kernel_id, cudaStream_t stream);
 void launch_end(cudaStream_t stream);
 
 // Launchers.  Each returns the cudaError_t of its launch.
+// With `x_scatter` set, the slot assignment also copies every kept token's
+// row of x into xbuf[expert, slot] (scatter form of the dispatch) and, with
+// `y_zero` set, writes the zero output row of every dropped token.
 cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
                          int32_t *expert, float *gate, int32_t *slot, int32_t *counts, int32_t *slot_token,
-                         float *aux, const Workspace &ws, cudaStream_t stream);
+                         float *aux, const Workspace &ws, cudaStream_t stream, void *xbuf_scatter = nullptr,
+                         float *y_zero = nullptr);
 cudaError_t launch_dispatch(const switch_dims_t &dims, const void *x, const int32_t *slot_token,
                             const int32_t *counts, void *xbuf, cudaStream_t stream);
-cudaError_t launch_combine(const switch_dims_t &dims, const void *ybuf, const int32_t *expert,
-                           const int32_t *slot, const float *gate, void *y, cudaStream_t stream);
+cudaError_t launch_combine(const switch_dims_t &dims, const float *ybuf, const int32_t *expert,
+                           const int32_t *slot, const float *gate, float *y, cudaStream_t stream);
+// Expert FFN; ybuf is float32 [N][C][d].
 cudaError_t launch_ffn_simt(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
-                            const int32_t *counts, void *ybuf, const Workspace &ws, cudaStream_t stream);
+                            const int32_t *counts, float *ybuf, const Workspace &ws, cudaStream_t stream);
+// Tensor-core expert FFN.  With `y` set, GEMM2 writes y[t] = gate[t] * acc
+// straight to token order (t = slot_token[i*C+s]) instead of ybuf.
 cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
-                          const int32_t *counts, void *ybuf, const Workspace &ws, cudaStream_t stream);
+                          const int32_t *counts, void *ybuf, const int32_t *slot_token, const float *gate, float *y,
+                          const Workspace &ws, cudaStream_t stream);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();

@@ -5,8 +5,8 @@
 //   (Incredible.AI "MoE Layer", x_flat[expert_indices]; kasblo section
 //   "tokenをExpertへ送って戻すforward pass": on one device the exchange is a
 //   gather/scatter in memory).
-// Combine:  y[t, :] = gate[t] * ybuf[expert[t], slot[t], :], or 0 for a
-//   dropped token (llm-papers-study "精读 06 | Switch Transformers" §3.2,
+// Combine:  y[t, :] = gate[t] * ybuf[expert[t], slot[t], :] in float32, or
+//   0 for a dropped token (llm-papers-study "精读 06 | Switch Transformers" §3.2,
 //   y = p_i*(x) E_i*(x); §3.4, dropped tokens skip the expert).
 //
 // Both are pure HBM streams: one warp per row, 16-byte vector accesses, all of
@@ -60,49 +60,44 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel4(const uint32_t *__r
     for (int w = threadIdx.x & 31; w < words; w += 32) xbuf[row * words + w] = x[t * words + w];
 }
 
-__device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float g) {
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float lo = __uint_as_float(w[i] << 16) * g;
-        const float hi = __uint_as_float(w[i] & 0xffff0000u) * g;
-        w[i] = pack_bf16x2(lo, hi);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-__global__ void __launch_bounds__(kThreads) combine_kernel_bf16(const uint4 *__restrict__ ybuf,
-                                                               const int32_t *__restrict__ expert,
-                                                               const int32_t *__restrict__ slot,
-                                                               const float *__restrict__ gate, int64_t T, int C,
-                                                               int words, uint4 *__restrict__ y) {
+// y[t] = gate[t] * ybuf[expert[t], slot[t]] (float32, one rounding), or 0.
+__global__ void __launch_bounds__(kThreads) combine_kernel_vec(const float4 *__restrict__ ybuf,
+                                                              const int32_t *__restrict__ expert,
+                                                              const int32_t *__restrict__ slot,
+                                                              const float *__restrict__ gate, int64_t T, int C,
+                                                              int words, float4 *__restrict__ y) {
     const int64_t t = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
     if (t >= T) return;
     const int lane = threadIdx.x & 31;
     const int s = slot[t];
-    uint4 *dst = y + t * words;
+    float4 *dst = y + t * words;
     if (s < 0) {
-        for (int w = lane; w < words; w += 32) dst[w] = make_uint4(0u, 0u, 0u, 0u);
+        for (int w = lane; w < words; w += 32) __stcs(dst + w, make_float4(0.f, 0.f, 0.f, 0.f));
         return;
     }
     const float g = gate[t];
-    const uint4 *src = ybuf + ((int64_t)expert[t] * C + s) * words;
+    const float4 *src = ybuf + ((int64_t)expert[t] * C + s) * words;
     int w = lane;
     for (; w + 32 * (kUnroll - 1) < words; w += 32 * kUnroll) {
-        uint4 v[kUnroll];
+        float4 v[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) v[u] = __ldcs(src + w + 32 * u);
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) __stcs(dst + w + 32 * u, scale_bf16x8(v[u], g));
+        for (int u = 0; u < kUnroll; ++u)
+            __stcs(dst + w + 32 * u, make_float4(g * v[u].x, g * v[u].y, g * v[u].z, g * v[u].w));
     }
-    for (; w < words; w += 32) __stcs(dst + w, scale_bf16x8(__ldcs(src + w), g));
+    for (; w < words; w += 32) {
+        const float4 v = __ldcs(src + w);
+        __stcs(dst + w, make_float4(g * v.x, g * v.y, g * v.z, g * v.w));
+    }
 }
 
-__global__ void __launch_bounds__(kThreads) combine_kernel_f32(const float *__restrict__ ybuf,
-                                                              const int32_t *__restrict__ expert,
-                                                              const int32_t *__restrict__ slot,
-                                                              const float *__restrict__ gate, int64_t T, int C, int d,
-                                                              float *__restrict__ y) {
+// Rows of d % 4 != 0 floats.
+__global__ void __launch_bounds__(kThreads) combine_kernel_scalar(const float *__restrict__ ybuf,
+                                                                 const int32_t *__restrict__ expert,
+                                                                 const int32_t *__restrict__ slot,
+                                                                 const float *__restrict__ gate, int64_t T, int C,
+                                                                 int d, float *__restrict__ y) {
     const int64_t t = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
     if (t >= T) return;
     const int lane = threadIdx.x & 31;
@@ -138,19 +133,19 @@ cudaError_t launch_dispatch(const switch_dims_t &dims, const void *x, const int3
     return err;
 }
 
-cudaError_t launch_combine(const switch_dims_t &dims, const void *ybuf, const int32_t *expert, const int32_t *slot,
-                           const float *gate, void *y, cudaStream_t stream) {
+cudaError_t launch_combine(const switch_dims_t &dims, const float *ybuf, const int32_t *expert, const int32_t *slot,
+                           const float *gate, float *y, cudaStream_t stream) {
     const int64_t T = dims.T;
     if (T == 0) return cudaSuccess;
     const unsigned grid = (unsigned)((T + kRowsPerBlock - 1) / kRowsPerBlock);
     launch_begin(K_COMBINE, stream);
-    if (dims.dtype == SWITCH_BF16)
-        combine_kernel_bf16<<<grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(ybuf), expert, slot, gate, T,
-                                                           dims.capacity, dims.d_model / 8,
-                                                           static_cast<uint4 *>(y));
+    if (dims.d_model % 4 == 0)
+        combine_kernel_vec<<<grid, kThreads, 0, stream>>>(reinterpret_cast<const float4 *>(ybuf), expert, slot, gate,
+                                                          T, dims.capacity, dims.d_model / 4,
+                                                          reinterpret_cast<float4 *>(y));
     else
-        combine_kernel_f32<<<grid, kThreads, 0, stream>>>(static_cast<const float *>(ybuf), expert, slot, gate, T,
-                                                          dims.capacity, dims.d_model, static_cast<float *>(y));
+        combine_kernel_scalar<<<grid, kThreads, 0, stream>>>(ybuf, expert, slot, gate, T, dims.capacity,
+                                                             dims.d_model, y);
     cudaError_t err = cudaGetLastError();
     launch_end(stream);
     return err;

@@ -93,6 +93,16 @@ __device__ __forceinline__ void publish_tile(const float *psum_w, const int32_t 
     }
 }
 
+// The first block of a routing call resets the scan ticket and the status
+// word of the workspace (which the caller may hand over uninitialised).
+__device__ __forceinline__ void reset_call_state(uint32_t *ticket, DeviceStatus *status) {
+    *ticket = 0u;
+    status->code = 0;
+    status->where = 0;
+    status->block = 0;
+    status->reserved = 0;
+}
+
 template <typename XT>
 struct XLoad;
 template <>
@@ -133,7 +143,8 @@ __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restr
                                                                const float *__restrict__ bias, int64_t T, int d,
                                                                int N, int tiles, int32_t *__restrict__ expert,
                                                                float *__restrict__ gate, int32_t *__restrict__ hist,
-                                                               float *__restrict__ psum, uint32_t *ticket) {
+                                                               float *__restrict__ psum, uint32_t *ticket,
+                                                               DeviceStatus *status) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *wsm = reinterpret_cast<float *>(smem_raw);  // [d][NP]
     float *psum_w = wsm + (size_t)d * NP;               // [kWarps][N]
@@ -141,7 +152,7 @@ __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restr
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x;
 
-    if (tile == 0 && tid == 0) *ticket = 0u;
+    if (tile == 0 && tid == 0) reset_call_state(ticket, status);
     for (int i = tid; i < d * NP; i += kThreads) {
         const int k = i / NP, e = i % NP;
         wsm[i] = e < N ? w_r[(int64_t)e * d + k] : 0.f;
@@ -234,7 +245,8 @@ __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__rest
                                                                 const float *__restrict__ bias, int64_t T, int d,
                                                                 int N, int tiles, int32_t *__restrict__ expert,
                                                                 float *__restrict__ gate, int32_t *__restrict__ hist,
-                                                                float *__restrict__ psum, uint32_t *ticket) {
+                                                                float *__restrict__ psum, uint32_t *ticket,
+                                                                DeviceStatus *status) {
     constexpr int TE = EC / 16;  // experts per thread
     constexpr int TT = 4;        // tokens per thread
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -249,7 +261,7 @@ __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__rest
     const int tile = blockIdx.x;
     const int64_t t0 = (int64_t)tile * kTileT;
 
-    if (tile == 0 && tid == 0) *ticket = 0u;
+    if (tile == 0 && tid == 0) reset_call_state(ticket, status);
     for (int i = tid; i < kWarps * N; i += kThreads) {
         psum_w[i] = 0.f;
         hist_w[i] = 0;
@@ -401,41 +413,85 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t *__res
 }
 
 // ---------------------------------------------------------------------------
-// Assignment: blocks [0, tiles) take one 64-token tile each (2 warps); every
-// block also clears a share of the empty slots of slot_token.
+// Assignment: blocks [0, tiles) take one 64-token tile each; warps 0 and 1
+// rank the tile's tokens within their experts, and with SCATTER all eight
+// warps then move rows: a kept token's row of x goes to xbuf[expert, slot]
+// (the dispatch, in scatter form), a dropped token's output row is zeroed.
+// Every block also clears a share of the empty slots of slot_token.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kTileT) assign_kernel(const int32_t *__restrict__ expert,
-                                                        const int32_t *__restrict__ tile_off,
-                                                        const int32_t *__restrict__ counts, int64_t T, int N, int C,
-                                                        int tiles, int32_t *__restrict__ slot,
-                                                        int32_t *__restrict__ slot_token) {
-    static_assert(kTileT == 64, "assignment assumes two warps per tile");
+constexpr int kAssignThreads = 256;
+
+template <bool SCATTER>
+__global__ void __launch_bounds__(kAssignThreads) assign_kernel(
+    const int32_t *__restrict__ expert, const int32_t *__restrict__ tile_off, const int32_t *__restrict__ counts,
+    int64_t T, int N, int C, int tiles, int32_t *__restrict__ slot, int32_t *__restrict__ slot_token,
+    const uint4 *__restrict__ x, uint4 *__restrict__ xbuf, int x_words, float4 *__restrict__ y_zero, int y_words) {
+    static_assert(kTileT == 64, "assignment assumes two ranking warps per tile");
     __shared__ int32_t first_warp_count[256];
+    __shared__ int32_t tile_slot[kTileT];
+    __shared__ int32_t tile_expert[kTileT];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x;
     if (tile < tiles) {
-        const int64_t t = (int64_t)tile * kTileT + tid;
-        const bool valid = t < T;
-        const int e = valid ? expert[t] : -1 - lane;  // distinct keys for absent tokens
-        for (int i = tid; i < N; i += kTileT) first_warp_count[i] = 0;
-        const unsigned same = __match_any_sync(0xffffffffu, e);
-        int rank = __popc(same & (unsigned)lanemask_lt());
+        for (int i = tid; i < N; i += kAssignThreads) first_warp_count[i] = 0;
         __syncthreads();
-        if (warp == 0 && valid && rank == 0) first_warp_count[e] = __popc(same);
+        int e = -1, rank = 0;
+        bool valid = false;
+        int64_t t = 0;
+        unsigned same = 0;
+        if (warp < 2) {
+            t = (int64_t)tile * kTileT + tid;
+            valid = t < T;
+            e = valid ? expert[t] : -1 - lane;  // distinct keys for absent tokens
+            same = __match_any_sync(0xffffffffu, e);
+            rank = __popc(same & (unsigned)lanemask_lt());
+            if (warp == 0 && valid && rank == 0) first_warp_count[e] = __popc(same);
+        }
         __syncthreads();
-        if (valid) {
-            if (warp == 1) rank += first_warp_count[e];
-            const int s = tile_off[(int64_t)e * tiles + tile] + rank;
-            if (s < C) {
-                slot[t] = s;
-                slot_token[(int64_t)e * C + s] = (int32_t)t;
-            } else {
-                slot[t] = -1;
+        if (warp < 2) {
+            int s_out = -2;  // -2: no token here
+            if (valid) {
+                if (warp == 1) rank += first_warp_count[e];
+                const int s = tile_off[(int64_t)e * tiles + tile] + rank;
+                if (s < C) {
+                    slot[t] = s;
+                    slot_token[(int64_t)e * C + s] = (int32_t)t;
+                    s_out = s;
+                } else {
+                    slot[t] = -1;
+                    s_out = -1;
+                }
+            }
+            tile_slot[tid] = s_out;
+            tile_expert[tid] = e;
+        }
+        if (SCATTER) {
+            __syncthreads();
+            for (int r = warp; r < kTileT; r += kAssignThreads / 32) {
+                const int s = tile_slot[r];
+                const int64_t tr = (int64_t)tile * kTileT + r;
+                if (s >= 0) {
+                    const uint4 *src = x + tr * x_words;
+                    uint4 *dst = xbuf + ((int64_t)tile_expert[r] * C + s) * x_words;
+                    int w = lane;
+                    for (; w + 96 < x_words; w += 128) {
+                        const uint4 a = __ldcs(src + w), b = __ldcs(src + w + 32), c = __ldcs(src + w + 64),
+                                    d4 = __ldcs(src + w + 96);
+                        dst[w] = a;
+                        dst[w + 32] = b;
+                        dst[w + 64] = c;
+                        dst[w + 96] = d4;
+                    }
+                    for (; w < x_words; w += 32) dst[w] = __ldcs(src + w);
+                } else if (s == -1 && y_zero) {
+                    float4 *dst = y_zero + tr * y_words;
+                    for (int w = lane; w < y_words; w += 32) __stcs(dst + w, make_float4(0.f, 0.f, 0.f, 0.f));
+                }
             }
         }
     }
     const int64_t total = (int64_t)N * C;
-    for (int64_t i = (int64_t)blockIdx.x * kTileT + tid; i < total; i += (int64_t)gridDim.x * kTileT) {
+    for (int64_t i = (int64_t)blockIdx.x * kAssignThreads + tid; i < total; i += (int64_t)gridDim.x * kAssignThreads) {
         const int e = (int)(i / C);
         const int s = (int)(i % C);
         if (s >= min(counts[e], C)) slot_token[i] = -1;
@@ -452,7 +508,8 @@ cudaError_t launch_router_warp(const switch_dims_t &dims, const XT *x, const flo
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_WARP, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
-                                                         ws.hist, ws.psum, ws.ticket);
+                                                         ws.hist, ws.psum, ws.ticket,
+                                                         static_cast<DeviceStatus *>(ws.status));
     err = cudaGetLastError();
     launch_end(stream);
     return err;
@@ -469,7 +526,8 @@ cudaError_t launch_router_tiled(const switch_dims_t &dims, const XT *x, const fl
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_TILED, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
-                                                         ws.hist, ws.psum, ws.ticket);
+                                                         ws.hist, ws.psum, ws.ticket,
+                                                         static_cast<DeviceStatus *>(ws.status));
     err = cudaGetLastError();
     launch_end(stream);
     return err;
@@ -498,7 +556,7 @@ cudaError_t launch_router(const switch_dims_t &dims, const XT *x, const float *w
 
 cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
                          int32_t *expert, float *gate, int32_t *slot, int32_t *counts, int32_t *slot_token,
-                         float *aux, const Workspace &ws, cudaStream_t stream) {
+                         float *aux, const Workspace &ws, cudaStream_t stream, void *xbuf_scatter, float *y_zero) {
     cudaError_t err = cudaSuccess;
     const int N = dims.num_experts, C = dims.capacity;
     if (ws.tiles > 0) {
@@ -508,8 +566,9 @@ cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *
                   : launch_router<float>(dims, static_cast<const float *>(x), w_r, bias, expert, gate, ws, stream);
         if (err != cudaSuccess) return err;
     } else {
-        // No router launch to reset the scan ticket: do it here.
+        // No router launch to reset the scan ticket and the status word.
         err = cudaMemsetAsync(ws.ticket, 0, sizeof(uint32_t), stream);
+        if (err == cudaSuccess) err = cudaMemsetAsync(ws.status, 0, sizeof(DeviceStatus), stream);
         if (err != cudaSuccess) return err;
     }
     launch_begin(K_SCAN, stream);
@@ -518,11 +577,21 @@ cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *
     err = cudaGetLastError();
     launch_end(stream);
     if (err != cudaSuccess) return err;
-    const int64_t fill_blocks = ((int64_t)N * C + kTileT * 16 - 1) / (kTileT * 16);
+    const int64_t fill_blocks = ((int64_t)N * C + kAssignThreads * 4 - 1) / (kAssignThreads * 4);
     const int64_t grid = ws.tiles > fill_blocks ? ws.tiles : fill_blocks;
-    launch_begin(K_ASSIGN, stream);
-    assign_kernel<<<(unsigned)grid, kTileT, 0, stream>>>(expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles,
-                                                         slot, slot_token);
+    const int x_words = (int)((int64_t)dims.d_model * (dims.dtype == SWITCH_BF16 ? 2 : 4) / 16);
+    if (xbuf_scatter) {
+        launch_begin(K_ASSIGN_SCATTER, stream);
+        assign_kernel<true><<<(unsigned)grid, kAssignThreads, 0, stream>>>(
+            expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token,
+            static_cast<const uint4 *>(x), static_cast<uint4 *>(xbuf_scatter), x_words,
+            reinterpret_cast<float4 *>(y_zero), dims.d_model / 4);
+    } else {
+        launch_begin(K_ASSIGN, stream);
+        assign_kernel<false><<<(unsigned)grid, kAssignThreads, 0, stream>>>(
+            expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token, nullptr, nullptr, 0,
+            nullptr, 0);
+    }
     err = cudaGetLastError();
     launch_end(stream);
     return err;

@@ -105,8 +105,8 @@ def test_entry_points_compose_to_layer(orc):
     slot_token = torch.empty(N * C, dtype=torch.int32, device="cuda")
     aux = torch.empty(1, dtype=torch.float32, device="cuda")
     xbuf = torch.empty(N * C * dm, dtype=torch.bfloat16, device="cuda")
-    ybuf = torch.empty(N * C * dm, dtype=torch.bfloat16, device="cuda")
-    y = torch.empty_like(dev["x"])
+    ybuf = torch.empty(N * C * dm, dtype=torch.float32, device="cuda")
+    y = torch.empty(T, dm, dtype=torch.float32, device="cuda")
     sm.switch_route(d, dev["x"], dev["w_r"], None, expert, gate, slot, counts, slot_token, aux, ws)
     sm.switch_dispatch(d, dev["x"], slot_token, counts, xbuf)
     sm.switch_expert_ffn(d, xbuf, dev["w_in"], dev["w_out"], counts, ybuf, ws)
@@ -114,7 +114,7 @@ def test_entry_points_compose_to_layer(orc):
     assert sm.switch_check(ws) == 0
     assert torch.equal(expert, ref["expert"]) and torch.equal(slot, ref["slot"])
     assert torch.equal(counts, ref["counts"]) and torch.equal(aux, ref["aux"])
-    assert torch.equal(y.view(torch.int16), ref["y"].view(torch.int16))
+    assert torch.equal(y.view(torch.int32), ref["y"].view(torch.int32))
     # dispatch wrote exactly the kept tokens' rows
     kept = torch.clamp(counts, max=C).cpu().numpy()
     st = slot_token.view(N, C).cpu().numpy()
@@ -134,13 +134,17 @@ def test_deterministic_bytes(orc):
     b = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, logit_bias=dev["bias"])
     for k in ("expert", "gate", "slot", "counts", "aux"):
         assert torch.equal(a[k], b[k]), k
-    assert torch.equal(a["y"].view(torch.int16), b["y"].view(torch.int16))
+    assert torch.equal(a["y"].view(torch.int32), b["y"].view(torch.int32))
 
 
 # ---------------------------------------------------------------------------
 # edge cases
 # ---------------------------------------------------------------------------
-def _random_inputs(rng, T, d, F, N, dtype, w_scale=1.0, bias=True):
+def _random_inputs(rng, T, d, F, N, dtype, w_scale=0.1, bias=True):
+    """Shapes of the edge cases with the workloads' value recipe: router
+    weights at 0.1 / sqrt(d) (near-uniform gates), experts at 1 / sqrt(fan_in).
+    (With 10x larger router weights the gates become heavy-tailed, max|y|
+    reaches ~14 RMS and the bf16 rounding of H alone exceeds 2e-2 x RMS.)"""
     x = rng.standard_normal((T, d)).astype(np.float32)
     w_r = (rng.standard_normal((N, d)) * w_scale / np.sqrt(d)).astype(np.float32)
     b = (rng.standard_normal(N) * 0.2).astype(np.float32) if bias else None
@@ -233,7 +237,7 @@ def test_outputs_stay_in_bounds(orc):
         big = torch.full((n + 2 * pad,), -7, dtype=dtype, device="cuda")
         return big, big[pad:pad + n]
 
-    yb, y = guarded(T * d, torch.int16)
+    yb, y = guarded(T * d, torch.int32)
     eb, e = guarded(T, torch.int32)
     gb, gt = guarded(T, torch.float32)
     sb, s = guarded(T, torch.int32)
@@ -251,7 +255,7 @@ def test_outputs_stay_in_bounds(orc):
     g = dict(expert=e.cpu().numpy(), gate=gt.cpu().numpy(), slot=s.cpu().numpy(), counts=c.cpu().numpy(),
              aux=a.cpu().numpy()[0])
     rep = check_routing(o, g, orc, N, C, T, check_slot_token=False)
-    yy = y.view(torch.bfloat16).view(T, d).float().cpu().numpy().astype(np.float64)
+    yy = y.view(torch.float32).view(T, d).cpu().numpy().astype(np.float64)
     check_outputs(yy, np.arange(T), o, rep, orc, inp["x"], inp["w_in"], inp["w_out"], g["expert"], False)
 
 
@@ -261,7 +265,7 @@ def test_errors_leave_outputs_untouched():
     w_r = torch.randn(N, d, device="cuda")
     w_in = torch.randn(N, F, d, device="cuda").bfloat16()
     w_out = torch.randn(N, d, F, device="cuda").bfloat16()
-    y = torch.full((T, d), 3.0, device="cuda").bfloat16()
+    y = torch.full((T, d), 3.0, device="cuda")
     dims = sm.dims(T, d, F, N, C, sm.SWITCH_BF16)
     ws_small = torch.empty(64, dtype=torch.uint8, device="cuda")
     counts = torch.full((N,), 9, dtype=torch.int32, device="cuda")
@@ -286,8 +290,8 @@ def test_tracer_and_launch_counter():
     trace = sm.trace_read()
     sm.trace_stop()
     names = [n for n, _ in trace]
-    assert names == ["router_warp", "capacity_scan", "slot_assign", "dispatch", "ffn_tc_gemm1_relu",
-                     "ffn_tc_gemm2", "combine"]
+    assert names == ["router_warp", "capacity_scan", "slot_assign_scatter", "ffn_tc_gemm1_relu",
+                     "ffn_tc_gemm2_gated_scatter"]
     assert all(ms >= 0 for _, ms in trace)
     assert sm.launch_count() - before == len(names)
     assert sm.switch_check(out["workspace"]) == 0
@@ -348,3 +352,26 @@ def test_full_size(orc, name, record_property):
 def test_full_size_bigexpert_capacity_sweep(orc, record_property):
     wl = synth.WORKLOADS["bigexpert64"]
     _full_size(orc, wl, list(wl.sweep), record_property)
+
+
+@pytest.mark.parametrize("entry", ["layer_fwd", "route", "expert_ffn"])
+def test_uninitialised_workspace_reports_ok(entry):
+    """The workspace may arrive full of stale bytes: every call that can
+    report a device status starts by clearing it."""
+    wl = synth.WORKLOADS["base8"]
+    T = 700
+    inp = synth.inputs(wl, T=T)
+    dev = {k: to_device(v) for k, v in inp.items()}
+    C = synth_capacity(wl, T)
+    d = sm.layer_dims(dev["x"], dev["w_in"], capacity=C)
+    ws = torch.full((sm.switch_workspace_size(d),), 0x5A, dtype=torch.uint8, device="cuda")
+    if entry == "layer_fwd":
+        sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, ws=ws)
+    elif entry == "route":
+        sm.route(dev["x"], dev["w_r"], capacity=C, d_ff=wl.d_ff, ws=ws)
+    else:
+        counts = torch.zeros(wl.num_experts, dtype=torch.int32, device="cuda")
+        xbuf = torch.zeros(wl.num_experts * C * wl.d_model, dtype=torch.bfloat16, device="cuda")
+        ybuf = torch.zeros(wl.num_experts * C * wl.d_model, dtype=torch.float32, device="cuda")
+        sm.switch_expert_ffn(d, xbuf, dev["w_in"], dev["w_out"], counts, ybuf, ws)
+    assert sm.switch_check(ws) == 0
