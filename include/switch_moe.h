@@ -59,7 +59,8 @@ typedef enum {
     SWITCH_ERR_WORKSPACE = 5,      /* workspace smaller than switch_workspace_size() */
     SWITCH_ERR_UNSUPPORTED = 6,    /* valid request this build cannot run (e.g. no sm_100 device) */
     SWITCH_ERR_CUDA = 7,           /* a CUDA runtime call or kernel launch failed */
-    SWITCH_ERR_DEVICE_TIMEOUT = 8  /* a kernel gave up a bounded wait (reported by switch_check) */
+    SWITCH_ERR_DEVICE_TIMEOUT = 8, /* a kernel gave up a bounded wait (reported by switch_check) */
+    SWITCH_ERR_TOO_LARGE = 9       /* switch_route_noalloc: the group needs more scratch than its static buffer */
 } switch_status_t;
 
 /* Storage type of the input activations (x, xbuf) and of the expert weights
@@ -171,6 +172,34 @@ switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const
                                  const float *logit_bias, const void *w_in, const void *w_out, void *y,
                                  int32_t *expert, float *gate, int32_t *slot, int32_t *counts, float *aux,
                                  void *workspace, size_t workspace_bytes, switch_stream_t stream);
+
+/* Routing without a workspace, for callers that cannot allocate device
+ * memory at the point where they route tokens: code running under a host
+ * framework that owns every device allocation and forbids new ones while it
+ * executes (an inference engine's plugin, a server that reserves all of its
+ * device memory up front), or code with no allocator at hand.  The sources
+ * have no counterpart of this entry point; it exists for those callers only.
+ *
+ * Same arguments (minus the workspace) and the same outputs, bit for bit, as
+ * switch_route.  Its scratch is one static device array of
+ * SWITCH_NOALLOC_SCRATCH_BYTES inside this library, which every GPU that
+ * loads the library holds until the process exits; it allocates and frees
+ * nothing.  A call needs about 12 * N * ceil(T / 64) + 8 * N bytes of it
+ * (plus under 2 KiB of alignment padding), so the 4 MiB array holds, for
+ * example, T = 131072 tokens with up to 128 experts; a larger group returns
+ * SWITCH_ERR_TOO_LARGE before anything runs.
+ *
+ * The first call on each device looks up the array's device address with
+ * that device current; make that first call before any stream capture.
+ * Every call shares the one array and leaves its contents behind (the next
+ * call clears what must start at zero), so calls whose kernels may overlap
+ * on the GPU (on different streams, or from several host threads) race and
+ * must not be issued; calls on one stream are fine.  The status word used by
+ * switch_check lives in the array too and cannot be read by the caller. */
+#define SWITCH_NOALLOC_SCRATCH_BYTES (4u << 20)
+switch_status_t switch_route_noalloc(const switch_dims_t *dims, const void *x, const float *w_r,
+                                     const float *logit_bias, int32_t *expert, float *gate, int32_t *slot,
+                                     int32_t *counts, int32_t *slot_token, float *aux, switch_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the device status word kept in
  * `workspace`.  switch_route, switch_expert_ffn and switch_layer_fwd clear

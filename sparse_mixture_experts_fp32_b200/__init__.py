@@ -32,9 +32,11 @@ SWITCH_FLAG_SIMT_ROUTER = 2
 STATUS = {
     0: "SWITCH_OK", 1: "SWITCH_ERR_NULL", 2: "SWITCH_ERR_SHAPE", 3: "SWITCH_ERR_DTYPE", 4: "SWITCH_ERR_ALIGN",
     5: "SWITCH_ERR_WORKSPACE", 6: "SWITCH_ERR_UNSUPPORTED", 7: "SWITCH_ERR_CUDA", 8: "SWITCH_ERR_DEVICE_TIMEOUT",
+    9: "SWITCH_ERR_TOO_LARGE",
 }
 
-EXPORTED = ("switch_capacity", "switch_workspace_size", "switch_route", "switch_dispatch", "switch_expert_ffn",
+EXPORTED = ("switch_capacity", "switch_workspace_size", "switch_route", "switch_route_noalloc", "switch_dispatch",
+            "switch_expert_ffn",
             "switch_combine", "switch_layer_fwd", "switch_check", "switch_status_string", "switch_launch_count",
             "switch_trace_start", "switch_trace_read", "switch_trace_stop", "switch_kernel_name")
 
@@ -73,6 +75,7 @@ def lib() -> ctypes.CDLL:
         "switch_capacity": (ctypes.c_int64, [ctypes.c_int64, ctypes.c_int32, ctypes.c_double]),
         "switch_workspace_size": (I, [D, ctypes.POINTER(ctypes.c_size_t)]),
         "switch_route": (I, [D, P, P, P, P, P, P, P, P, P, P, S, P]),
+        "switch_route_noalloc": (I, [D, P, P, P, P, P, P, P, P, P, P]),
         "switch_dispatch": (I, [D, P, P, P, P, P]),
         "switch_expert_ffn": (I, [D, P, P, P, P, P, P, S, P]),
         "switch_combine": (I, [D, P, P, P, P, P, P]),
@@ -162,6 +165,15 @@ def switch_route(d, x, w_r, logit_bias, expert, gate, slot, counts, slot_token, 
                            _ptr(slot), _ptr(counts), _ptr(slot_token), _ptr(aux), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream, workspace)),
         "switch_route")
+
+
+def switch_route_noalloc(d, x, w_r, logit_bias, expert, gate, slot, counts, slot_token, aux, stream=None):
+    """switch_route without a workspace: for callers that cannot allocate
+    device memory where they route (the scratch is a static array inside the
+    library; calls that overlap on the GPU race)."""
+    _ok(lib().switch_route_noalloc(ctypes.byref(d), _ptr(x), _ptr(w_r), _ptr(logit_bias), _ptr(expert), _ptr(gate),
+                                   _ptr(slot), _ptr(counts), _ptr(slot_token), _ptr(aux), _stream(stream, counts)),
+        "switch_route_noalloc")
 
 
 def switch_dispatch(d, x, slot_token, counts, xbuf, stream=None):

@@ -132,6 +132,8 @@ switch_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SWITCH_OK :
 
 size_t workspace_bytes(const switch_dims_t &dims) { return layout(dims).total; }
 
+size_t route_scratch_bytes(const switch_dims_t &dims) { return layout(dims).slot_token; }
+
 Workspace carve_workspace(const switch_dims_t &dims, void *base) {
     const Sections s = layout(dims);
     uint8_t *b = static_cast<uint8_t *>(base);
@@ -315,6 +317,7 @@ const char *switch_status_string(switch_status_t status) {
         case SWITCH_ERR_UNSUPPORTED: return "unsupported on this device (needs sm_100)";
         case SWITCH_ERR_CUDA: return "CUDA error";
         case SWITCH_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+        case SWITCH_ERR_TOO_LARGE: return "needs more scratch than the library's static buffer holds";
     }
     return "unknown status";
 }

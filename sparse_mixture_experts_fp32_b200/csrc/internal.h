@@ -44,6 +44,9 @@ struct Workspace {
 };
 
 size_t workspace_bytes(const switch_dims_t &dims);
+// Bytes at the start of the workspace layout that the routing step uses
+// (status word, ticket, per-tile counts / sums / offsets, probability totals).
+size_t route_scratch_bytes(const switch_dims_t &dims);
 Workspace carve_workspace(const switch_dims_t &dims, void *base);
 
 // Launch bookkeeping (tracing + launch counter).
