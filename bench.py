@@ -152,9 +152,13 @@ def kernel_work(wl, C, counts):
     K = int(kept.sum())
     E_nz = int((kept > 0).sum())
     tiles = -(-T // 64)
+    router_bytes = T * d * s + N * d * 4 + 8 * T + 8 * N * tiles
     return {
-        "router_warp": ("hbm", T * d * s + N * d * 4 + 8 * T + 8 * N * tiles),
-        "router_tiled": ("hbm", T * d * s + N * d * 4 + 8 * T + 8 * N * tiles),
+        "router_warp": ("hbm", router_bytes),
+        "router_tiled": ("hbm", router_bytes),
+        "router_staged": ("hbm", router_bytes),
+        "router_tc": ("hbm", T * d * s + 3 * N * d * 2 + 8 * T + 8 * N * tiles),
+        "router_weight_split": ("hbm", N * d * 4 + 3 * N * d * 2),
         "capacity_scan": ("hbm", 8 * N * tiles + 4 * N * tiles + 12 * N),
         "slot_assign_scatter": ("hbm", 4 * T + 4 * T + 4 * N * tiles + 4 * N * C + 2 * K * d * s + (T - K) * d * 4),
         "ffn_tc_gemm1_relu": ("tensor", 2.0 * K * d * F),
@@ -378,7 +382,7 @@ def traffic_from_profiles(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if it is current."""
     for p in sorted((ROOT / "profiles").glob("*.md")):
         text = p.read_text()
-        m = re.search(rf"^traffic\[{re.escape(kernel)}@{re.escape(workload)}\]:\s*([0-9.eE+]+)\s+bytes"
+        m = re.search(rf"^\s*traffic\[{re.escape(kernel)}@{re.escape(workload)}\]:\s*([0-9.eE+]+)\s+bytes"
                       rf"\s+source_sha=(\w+)", text, flags=re.M)
         if m and m.group(2) == source_sha():
             return float(m.group(1))

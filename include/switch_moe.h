@@ -80,7 +80,10 @@ enum {
     SWITCH_FLAG_SIMT_FFN = 1,
     /* Compute router logits on CUDA cores (FFMA) even where a tensor-core
      * router exists. */
-    SWITCH_FLAG_SIMT_ROUTER = 2
+    SWITCH_FLAG_SIMT_ROUTER = 2,
+    /* Run each expert GEMM tile on one SM (cta_group::1, 128-row tiles)
+     * instead of on a pair of SMs (cta_group::2, 256-row tiles). */
+    SWITCH_FLAG_GEMM_1CTA = 4
 };
 
 typedef struct {
@@ -184,10 +187,10 @@ switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const
  * switch_route.  Its scratch is one static device array of
  * SWITCH_NOALLOC_SCRATCH_BYTES inside this library, which every GPU that
  * loads the library holds until the process exits; it allocates and frees
- * nothing.  A call needs about 12 * N * ceil(T / 64) + 8 * N bytes of it
- * (plus under 2 KiB of alignment padding), so the 4 MiB array holds, for
- * example, T = 131072 tokens with up to 128 experts; a larger group returns
- * SWITCH_ERR_TOO_LARGE before anything runs.
+ * nothing.  A call needs about 12 * N * ceil(T / 64) + 8 * N + 6 * N * d
+ * bytes of it (plus under 2 KiB of alignment padding), so the 4 MiB array
+ * holds, for example, T = 131072 tokens with 128 experts and d_model = 1024;
+ * a larger group returns SWITCH_ERR_TOO_LARGE before anything runs.
  *
  * The first call on each device looks up the array's device address with
  * that device current; make that first call before any stream capture.

@@ -28,6 +28,7 @@ SWITCH_F32 = 0
 SWITCH_BF16 = 1
 SWITCH_FLAG_SIMT_FFN = 1
 SWITCH_FLAG_SIMT_ROUTER = 2
+SWITCH_FLAG_GEMM_1CTA = 4
 
 STATUS = {
     0: "SWITCH_OK", 1: "SWITCH_ERR_NULL", 2: "SWITCH_ERR_SHAPE", 3: "SWITCH_ERR_DTYPE", 4: "SWITCH_ERR_ALIGN",

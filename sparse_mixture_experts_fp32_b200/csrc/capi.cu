@@ -25,7 +25,7 @@ size_t elem_size(const switch_dims_t &d) { return d.dtype == SWITCH_BF16 ? 2 : 4
 int64_t tiles_of(const switch_dims_t &d) { return (d.T + kTileT - 1) / kTileT; }
 
 struct Sections {
-    size_t status, ticket, hist, psum, tile_off, prob_total, slot_token, xbuf, ybuf, hidden, total;
+    size_t status, ticket, hist, psum, tile_off, prob_total, w_split, slot_token, xbuf, ybuf, hidden, total;
 };
 
 Sections layout(const switch_dims_t &d) {
@@ -43,6 +43,7 @@ Sections layout(const switch_dims_t &d) {
     s.psum = take(N * tiles * 4);
     s.tile_off = take(N * tiles * 4);
     s.prob_total = take(N * 8);
+    s.w_split = take(3 * N * (size_t)d.d_model * 2);
     s.slot_token = take(N * C * 4);
     s.xbuf = take(N * C * (size_t)d.d_model * elem_size(d));
     s.ybuf = take(N * C * (size_t)d.d_model * sizeof(float));
@@ -144,6 +145,7 @@ Workspace carve_workspace(const switch_dims_t &dims, void *base) {
     w.psum = reinterpret_cast<float *>(b + s.psum);
     w.tile_off = reinterpret_cast<int32_t *>(b + s.tile_off);
     w.prob_total = reinterpret_cast<double *>(b + s.prob_total);
+    w.w_split = b + s.w_split;
     w.slot_token = reinterpret_cast<int32_t *>(b + s.slot_token);
     w.xbuf = b + s.xbuf;
     w.ybuf = reinterpret_cast<float *>(b + s.ybuf);
@@ -378,6 +380,9 @@ const char *switch_kernel_name(int32_t id) {
         case K_COMBINE: return "combine";
         case K_FFN_TC_GEMM2_GATED: return "ffn_tc_gemm2_gated_scatter";
         case K_ASSIGN_SCATTER: return "slot_assign_scatter";
+        case K_ROUTER_STAGED: return "router_staged";
+        case K_ROUTER_TC: return "router_tc";
+        case K_ROUTER_SPLIT: return "router_weight_split";
     }
     return "?";
 }

@@ -31,6 +31,8 @@
 // TMA loads and MMAs in flight, frees TMEM and returns.
 #include <cuda.h>
 
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -67,6 +69,49 @@ __device__ __forceinline__ void locate_tile(const int32_t *tile_start, int E, in
 
 enum Epilogue { kEpiHiddenRelu = 0, kEpiExpertOut = 1, kEpiGatedScatter = 2 };
 
+// Epilogue for one thread = one accumulator row (`row` of expert e's rows),
+// BN columns starting at column tile n: tcgen05.ld 32 columns at a time, then
+// the epilogue selected by EPI, for rows below the kept count only.
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_rows(uint32_t t_row, int e, int row, int kept, int C, int n, int Nout,
+                                              void *__restrict__ out, const int32_t *__restrict__ slot_token,
+                                              const float *__restrict__ gate) {
+    const bool row_ok = row < kept;
+    // destination row of this thread (a token row for the gated scatter)
+    int64_t out_row = (int64_t)e * C + row;
+    float g = 1.f;
+    if (EPI == kEpiGatedScatter && row_ok) {
+        out_row = slot_token[(int64_t)e * C + row];
+        g = gate[out_row];
+    }
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
+        tmem_ld_wait();
+        const int col0 = n * BN + c;
+        if (row_ok && col0 < Nout) {
+            if (EPI == kEpiHiddenRelu) {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + out_row * Nout + col0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float v[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i] = fmaxf(__uint_as_float(r[8 * q + i]), 0.f);
+                    dst[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                        pack_bf16x2(v[6], v[7]));
+                }
+            } else {
+                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + out_row * Nout + col0);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    dst[q] = make_float4(g * __uint_as_float(r[4 * q + 0]), g * __uint_as_float(r[4 * q + 1]),
+                                         g * __uint_as_float(r[4 * q + 2]), g * __uint_as_float(r[4 * q + 3]));
+            }
+        }
+    }
+}
+
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_grouped_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -93,10 +138,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Tile list: expert e owns tiles [tile_start[e], tile_start[e+1]), laid
     // out m-major with the BN-wide column tiles innermost.
     if (warp == 0) {
+        int kept_of[8];  // E <= 256: every count is loaded before the scan starts
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = 32 * j + lane;
+            kept_of[j] = e < E ? min(counts[e], C) : 0;
+        }
         int running = 0;
-        for (int e0 = 0; e0 < E; e0 += 32) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e0 = 32 * j;
+            if (e0 >= E) break;
             const int e = e0 + lane;
-            const int kept = e < E ? min(counts[e], C) : 0;
+            const int kept = kept_of[j];
             const int mine = (kept + BM - 1) / BM * n_tiles_n;
             int incl = mine;
 #pragma unroll
@@ -216,43 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             locate_tile(tile_start, E, n_tiles_n, tile, e, m, n);
             if (!mbar_wait(&acc_full[acc], acc_phase, status, 5)) break;
             tc_fence_after();
-            const int kept = min(counts[e], C);
             const int row = m * BM + row_in_tile;
-            const bool row_ok = row < kept;
-            // destination row of this thread (a token row for the gated scatter)
-            int64_t out_row = (int64_t)e * C + row;
-            float g = 1.f;
-            if (EPI == kEpiGatedScatter && row_ok) {
-                out_row = slot_token[(int64_t)e * C + row];
-                g = gate[out_row];
-            }
-            const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-#pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
-                tmem_ld_wait();
-                const int col0 = n * BN + c;
-                if (row_ok && col0 < Nout) {
-                    if (EPI == kEpiHiddenRelu) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + out_row * Nout + col0);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float v[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) v[i] = fmaxf(__uint_as_float(r[8 * q + i]), 0.f);
-                            dst[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                                pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-                        }
-                    } else {
-                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + out_row * Nout + col0);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            dst[q] = make_float4(g * __uint_as_float(r[4 * q + 0]), g * __uint_as_float(r[4 * q + 1]),
-                                                 g * __uint_as_float(r[4 * q + 2]), g * __uint_as_float(r[4 * q + 3]));
-                    }
-                }
-            }
+            epilogue_rows<BN, EPI>(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN), e, row,
+                                   min(counts[e], C), C, n, Nout, out, slot_token, gate);
             tc_fence_before();
             mbar_arrive(&acc_empty[acc]);
             if (++acc == 2) {
@@ -267,6 +287,300 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// Epilogue through the async proxy, one warp = 32 consecutive rows
+// (row_base .. row_base + 31, thread = row), `stage` = this warp's shared
+// staging buffer (4.5 KB, 1024-byte aligned):
+//   kEpiHiddenRelu  64 columns at a time: ReLU + bf16 into a 32 x 128-byte
+//                   box in the 128-byte swizzled layout (conflict-free
+//                   writes), then one TMA tensor store of the box into H.
+//                   Rows in [kept, C) receive values of rows that are never
+//                   read downstream; rows >= C are clipped by the tensor map.
+//   kEpiExpertOut / kEpiGatedScatter  32 fp32 columns at a time: each thread
+//                   writes its row (144-byte pitch: conflict-free) and
+//                   issues one 128-byte bulk copy to its destination row.
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_base, int kept, int C, int n, int Nout,
+                                               void *__restrict__ out, const void *tmap_out,
+                                               const int32_t *__restrict__ slot_token,
+                                               const float *__restrict__ gate, uint8_t *stage) {
+    const int lane = threadIdx.x & 31;
+    const int row = row_base + lane;
+    const bool row_ok = row < kept;
+    if (EPI == kEpiHiddenRelu) {
+        const bool any_row = row_base < kept;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 64) {
+            uint32_t r0[32], r1[32];
+            tmem_ld_32x32b_x32(t_row + (uint32_t)c, r0);
+            tmem_ld_32x32b_x32(t_row + (uint32_t)(c + 32), r1);
+            tmem_ld_wait();
+            if (lane == 0) bulk_wait_read_all();  // the previous box has left the buffer
+            __syncwarp();
+            uint8_t *rowp = stage + lane * 128;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t *src = q < 4 ? &r0[8 * q] : &r1[8 * (q - 4)];
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = fmaxf(__uint_as_float(src[i]), 0.f);
+                *reinterpret_cast<uint4 *>(rowp + ((q ^ (lane & 7)) << 4)) =
+                    make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                               pack_bf16x2(v[6], v[7]));
+            }
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0 && any_row && n * BN + c < Nout) {
+                tma_store_3d(tmap_out, stage, n * BN + c, row_base, e);
+                bulk_commit();
+            }
+        }
+        if (lane == 0) bulk_wait_read_all();
+    } else {
+        float g = 1.f;
+        float *dst_row = nullptr;
+        if (row_ok) {
+            int64_t out_row = (int64_t)e * C + row;
+            if (EPI == kEpiGatedScatter) {
+                out_row = slot_token[(int64_t)e * C + row];
+                g = gate[out_row];
+            }
+            dst_row = static_cast<float *>(out) + out_row * Nout;
+        }
+        uint8_t *rowp = stage + lane * 144;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
+            tmem_ld_wait();
+            const int col0 = n * BN + c;
+            if (row_ok && col0 < Nout) {
+                bulk_wait_read_all();  // this thread's previous row copy has left the buffer
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    *reinterpret_cast<float4 *>(rowp + 16 * q) =
+                        make_float4(g * __uint_as_float(r[4 * q + 0]), g * __uint_as_float(r[4 * q + 1]),
+                                    g * __uint_as_float(r[4 * q + 2]), g * __uint_as_float(r[4 * q + 3]));
+                fence_proxy_async_shared();
+                bulk_store(dst_row + col0, rowp, 128);
+                bulk_commit();
+            }
+        }
+        bulk_wait_read_all();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Pair (2-CTA) version: a cluster of two CTAs on two SMs computes 256-row x
+// BN-column tiles with tcgen05.mma.cta_group::2 (M = 256).  Each CTA loads
+// its own 128 rows of A and half of the BN rows of B, so a ring stage is
+// (16 + BN/8) KB instead of (16 + BN/4) KB: twice the lookahead in the same
+// shared memory, and a third less L2 traffic per flop.
+//   both CTAs, warp 0   TMA loads into their own shared memory, counted on
+//                       the leader's (rank 0) "full" barrier
+//   leader, warp 1      issues the pair MMAs; commits free the ring slot in
+//                       both CTAs and publish the accumulator to both
+//   both CTAs, warps 2-5  epilogue of their own 128 rows, then one arrival
+//                       each on the leader's "accumulator empty" barrier
+// Barrier addresses of the other CTA come from mapa; nothing is multicast.
+// ---------------------------------------------------------------------------
+template <int BN, int STAGES>
+struct PairLayout {
+    static constexpr size_t a_bytes = (size_t)BM * BK * 2;
+    static constexpr size_t b_bytes = (size_t)(BN / 2) * BK * 2;
+    static constexpr size_t ring = STAGES * (a_bytes + b_bytes);
+    static constexpr size_t stage_bytes = 5120;  // per epilogue warp (4.5 KB used), keeps 1024-byte alignment
+    static constexpr size_t staging = 4 * stage_bytes;
+    static constexpr size_t barriers = (2 * STAGES + 2 + 2 + 1) * 8 + 16;
+    static size_t bytes(int experts) { return 1024 + ring + staging + barriers + (size_t)(experts + 1) * 4; }
+};
+
+template <int BN, int STAGES, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                         const __grid_constant__ CUtensorMap tmap_out, void *__restrict__ out,
+                         const int32_t *__restrict__ counts, int E, int C, int K, int Nout,
+                         const int32_t *__restrict__ slot_token, const float *__restrict__ gate,
+                         DeviceStatus *status) {
+    using L = PairLayout<BN, STAGES>;
+    constexpr int BMP = 2 * BM;  // rows of a pair tile
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;
+    uint8_t *sB = sA + STAGES * L::a_bytes;
+    uint8_t *staging = base + L::ring;  // 1024-aligned: the ring is a multiple of 1024 bytes
+    uint64_t *full = reinterpret_cast<uint64_t *>(staging + L::staging);
+    uint64_t *empty = full + STAGES;
+    uint64_t *acc_full = empty + STAGES;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *drain = acc_empty + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    int32_t *tile_start = reinterpret_cast<int32_t *>(tmem_holder + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    const int n_tiles_n = (Nout + BN - 1) / BN;
+    const int k_blocks = K / BK;
+    constexpr uint32_t kTmemCols = 2 * BN;
+
+    if (warp == 0) {
+        int kept_of[8];  // E <= 256: every count is loaded before the scan starts
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = 32 * j + lane;
+            kept_of[j] = e < E ? min(counts[e], C) : 0;
+        }
+        int running = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e0 = 32 * j;
+            if (e0 >= E) break;
+            const int e = e0 + lane;
+            const int kept = kept_of[j];
+            const int mine = (kept + BMP - 1) / BMP * n_tiles_n;
+            int incl = mine;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += u;
+            }
+            if (e < E) tile_start[e] = running + incl - mine;
+            running += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) tile_start[E] = running;
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], 1);
+            }
+            for (int a = 0; a < 2; ++a) {
+                mbar_init(&acc_full[a], 1);
+                mbar_init(&acc_empty[a], 2 * kEpilogueThreads);
+            }
+            mbar_init(drain, 1);
+            fence_barrier_init();
+        }
+        __syncwarp();
+        tmem_alloc_pair(tmem_holder, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised before anyone signals them
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    const int total_tiles = tile_start[E];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tmap_a);
+            prefetch_tmap(&tmap_b);
+            uint32_t issued = 0, parity_of = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+                int e, m, n;
+                locate_tile(tile_start, E, n_tiles_n, tile, e, m, n);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, status, 21)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * (L::a_bytes + L::b_bytes)));
+                    const uint32_t leader_full = map_to_rank(&full[stage], 0);
+                    tma_load_3d_pair(sA + stage * L::a_bytes, &tmap_a, leader_full, kb * BK,
+                                     m * BMP + (int)rank * BM, e);
+                    tma_load_3d_pair(sB + stage * L::b_bytes, &tmap_b, leader_full, kb * BK,
+                                     n * BN + (int)rank * (BN / 2), e);
+                    issued |= 1u << stage;
+                    parity_of = (parity_of & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // Wind-down (leader): every load counted on its barriers has landed.
+            if (rank == 0)
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued & (1u << s)) mbar_wait(&full[s], (parity_of >> s) & 1u, status, 26);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(BMP, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, status, 22)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, status, 23)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t a_desc = smem_desc_sw128(sA + stage * L::a_bytes);
+                    const uint64_t b_desc = smem_desc_sw128(sB + stage * L::b_bytes);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        tc_mma_bf16_pair(d_tmem, a_desc + (uint64_t)(2 * k), b_desc + (uint64_t)(2 * k), idesc,
+                                         (kb | k) != 0 ? 1u : 0u);
+                    tc_commit_pair(smem_u32(&empty[stage]));
+                    tc_commit_pair(map_to_rank(&empty[stage], 1));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit_pair(smem_u32(&acc_full[acc]));
+                tc_commit_pair(map_to_rank(&acc_full[acc], 1));
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            tc_commit_pair(smem_u32(drain));
+            mbar_wait(drain, 0, status, 24);
+        }
+    } else {
+        const int quarter = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = pair; tile < total_tiles; tile += n_pairs) {
+            int e, m, n;
+            locate_tile(tile_start, E, n_tiles_n, tile, e, m, n);
+            if (!mbar_wait(&acc_full[acc], acc_phase, status, 25)) break;
+            tc_fence_after();
+            const int row_base = m * BMP + (int)rank * BM + quarter * 32;
+            epilogue_async<BN, EPI>(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN), e,
+                                    row_base, min(counts[e], C), C, n, Nout, out, &tmap_out, slot_token, gate,
+                                    staging + (warp - 2) * L::stage_bytes);
+            tc_fence_before();
+            mbar_arrive_cluster(map_to_rank(&acc_empty[acc], 0));
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    if (warp >= 2) bulk_wait_all();  // this thread's stores have completed
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // no CTA leaves while its peer may still use its shared memory or barriers
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 }
 
@@ -323,6 +637,28 @@ cudaError_t launch_gemm(int32_t kernel_id, const void *a, const void *b, void *o
     return err;
 }
 
+template <int BN, int STAGES, int EPI>
+cudaError_t launch_gemm_pair(int32_t kernel_id, const void *a, const void *b, void *out, const int32_t *counts, int E,
+                             int C, int K, int Nout, int64_t T, const int32_t *slot_token, const float *gate,
+                             DeviceStatus *status, cudaStream_t stream) {
+    CUtensorMap ta, tb, tout;
+    if (!make_tmap(&ta, a, E, C, K, BM) || !make_tmap(&tb, b, E, Nout, K, BN / 2)) return cudaErrorInvalidValue;
+    memset(&tout, 0, sizeof tout);
+    if (EPI == kEpiHiddenRelu && !make_tmap(&tout, out, E, C, Nout, 32)) return cudaErrorInvalidValue;
+    const size_t smem = PairLayout<BN, STAGES>::bytes(E);
+    auto kern = tc_grouped_gemm_pair<BN, STAGES, EPI>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    const int64_t m_tiles = std::min<int64_t>((int64_t)E * ((C + 2 * BM - 1) / (2 * BM)), (T + 2 * BM - 1) / (2 * BM) + E);
+    const int64_t tiles = m_tiles * ((Nout + BN - 1) / BN);
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / 2, tiles));
+    launch_begin(kernel_id, stream);
+    kern<<<2 * pairs, kThreads, smem, stream>>>(ta, tb, tout, out, counts, E, C, K, Nout, slot_token, gate, status);
+    err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
+
 }  // namespace
 
 cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
@@ -330,14 +666,26 @@ cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const voi
                           const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts, C = dims.capacity, d = dims.d_model, F = dims.d_ff;
     DeviceStatus *st = static_cast<DeviceStatus *>(ws.status);
-    cudaError_t err = launch_gemm<256, 4, kEpiHiddenRelu>(K_FFN_TC_GEMM1, xbuf, w_in, ws.hidden, counts, N, C, d, F,
-                                                          dims.T, nullptr, nullptr, st, stream);
+    if (dims.flags & SWITCH_FLAG_GEMM_1CTA) {
+        cudaError_t err = launch_gemm<256, 4, kEpiHiddenRelu>(K_FFN_TC_GEMM1, xbuf, w_in, ws.hidden, counts, N, C, d,
+                                                              F, dims.T, nullptr, nullptr, st, stream);
+        if (err != cudaSuccess) return err;
+        if (y)
+            return launch_gemm<128, 6, kEpiGatedScatter>(K_FFN_TC_GEMM2_GATED, ws.hidden, w_out, y, counts, N, C, F,
+                                                         d, dims.T, slot_token, gate, st, stream);
+        return launch_gemm<128, 6, kEpiExpertOut>(K_FFN_TC_GEMM2, ws.hidden, w_out, ybuf, counts, N, C, F, d,
+                                                  dims.T, nullptr, nullptr, st, stream);
+    }
+    cudaError_t err = launch_gemm_pair<256, 6, kEpiHiddenRelu>(K_FFN_TC_GEMM1, xbuf, w_in, ws.hidden, counts, N, C,
+                                                               d, F, dims.T, nullptr, nullptr, st, stream);
     if (err != cudaSuccess) return err;
+    // N = 256 MMAs for both GEMMs: with N = 128 the pair MMAs reached about
+    // half the tensor throughput of N = 256 on B200.
     if (y)
-        return launch_gemm<128, 6, kEpiGatedScatter>(K_FFN_TC_GEMM2_GATED, ws.hidden, w_out, y, counts, N, C, F, d,
-                                                     dims.T, slot_token, gate, st, stream);
-    return launch_gemm<128, 6, kEpiExpertOut>(K_FFN_TC_GEMM2, ws.hidden, w_out, ybuf, counts, N, C, F, d, dims.T,
-                                              nullptr, nullptr, st, stream);
+        return launch_gemm_pair<256, 6, kEpiGatedScatter>(K_FFN_TC_GEMM2_GATED, ws.hidden, w_out, y, counts, N, C,
+                                                          F, d, dims.T, slot_token, gate, st, stream);
+    return launch_gemm_pair<256, 6, kEpiExpertOut>(K_FFN_TC_GEMM2, ws.hidden, w_out, ybuf, counts, N, C, F, d,
+                                                   dims.T, nullptr, nullptr, st, stream);
 }
 
 }  // namespace switchmoe

@@ -27,6 +27,9 @@ enum KernelId : int32_t {
     K_COMBINE = 10,
     K_FFN_TC_GEMM2_GATED = 11,
     K_ASSIGN_SCATTER = 12,
+    K_ROUTER_STAGED = 13,
+    K_ROUTER_TC = 14,
+    K_ROUTER_SPLIT = 15,
 };
 
 struct Workspace {
@@ -36,6 +39,7 @@ struct Workspace {
     float *psum;         // [N][tiles] sum of p_i over each tile
     int32_t *tile_off;   // [N][tiles] exclusive prefix of hist over tiles
     double *prob_total;  // [N] sum of p_i over all tokens
+    void *w_split;       // [3][N][d] bf16 terms of W_r (tensor-core router)
     int32_t *slot_token; // [N*C] (layer_fwd only)
     void *xbuf;          // [N][C][d] (layer_fwd only)
     float *ybuf;         // [N][C][d] float32 (layer_fwd only)
@@ -65,6 +69,11 @@ cudaError_t launch_dispatch(const switch_dims_t &dims, const void *x, const int3
                             const int32_t *counts, void *xbuf, cudaStream_t stream);
 cudaError_t launch_combine(const switch_dims_t &dims, const float *ybuf, const int32_t *expert,
                            const int32_t *slot, const float *gate, float *y, cudaStream_t stream);
+// Tensor-core router (bf16 x, 32 < N <= 128): writes expert, gate and the
+// per-tile counts / probability sums like the CUDA-core routers.
+bool router_tc_supported(const switch_dims_t &dims);
+cudaError_t launch_router_tc(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
+                             int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream);
 // Expert FFN; ybuf is float32 [N][C][d].
 cudaError_t launch_ffn_simt(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
                             const int32_t *counts, float *ybuf, const Workspace &ws, cudaStream_t stream);

@@ -21,18 +21,23 @@ constexpr int kThreads = 256;
 constexpr int kRowsPerBlock = kThreads / 32;
 constexpr int kUnroll = 4;
 
-// Row copy of `words` 16-byte words by one warp.
+// Row copy of `words` 16-byte words by one warp: kUnroll loads per lane are
+// in flight before the first store.
 __device__ __forceinline__ void warp_copy_row16(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int words) {
     const int lane = threadIdx.x & 31;
-    int w = lane;
-    for (; w + 32 * (kUnroll - 1) < words; w += 32 * kUnroll) {
+    for (int w0 = 0; w0 < words; w0 += 32 * kUnroll) {
         uint4 v[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) v[u] = __ldcs(src + w + 32 * u);
+        for (int u = 0; u < kUnroll; ++u) {
+            const int w = w0 + lane + 32 * u;
+            if (w < words) v[u] = __ldcs(src + w);
+        }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) dst[w + 32 * u] = v[u];
+        for (int u = 0; u < kUnroll; ++u) {
+            const int w = w0 + lane + 32 * u;
+            if (w < words) dst[w] = v[u];
+        }
     }
-    for (; w < words; w += 32) dst[w] = __ldcs(src + w);
 }
 
 __global__ void __launch_bounds__(kThreads) dispatch_kernel16(const uint4 *__restrict__ x,
@@ -77,18 +82,18 @@ __global__ void __launch_bounds__(kThreads) combine_kernel_vec(const float4 *__r
     }
     const float g = gate[t];
     const float4 *src = ybuf + ((int64_t)expert[t] * C + s) * words;
-    int w = lane;
-    for (; w + 32 * (kUnroll - 1) < words; w += 32 * kUnroll) {
+    for (int w0 = 0; w0 < words; w0 += 32 * kUnroll) {
         float4 v[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) v[u] = __ldcs(src + w + 32 * u);
+        for (int u = 0; u < kUnroll; ++u) {
+            const int w = w0 + lane + 32 * u;
+            if (w < words) v[u] = __ldcs(src + w);
+        }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-            __stcs(dst + w + 32 * u, make_float4(g * v[u].x, g * v[u].y, g * v[u].z, g * v[u].w));
-    }
-    for (; w < words; w += 32) {
-        const float4 v = __ldcs(src + w);
-        __stcs(dst + w, make_float4(g * v.x, g * v.y, g * v.z, g * v.w));
+        for (int u = 0; u < kUnroll; ++u) {
+            const int w = w0 + lane + 32 * u;
+            if (w < words) __stcs(dst + w, make_float4(g * v[u].x, g * v[u].y, g * v[u].z, g * v[u].w));
+        }
     }
 }
 

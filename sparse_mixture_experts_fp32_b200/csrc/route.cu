@@ -118,6 +118,16 @@ struct XLoad<__nv_bfloat16> {
         }
     }
     static __device__ __forceinline__ float one(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+    // the same 16-byte vector read through a generic pointer (shared memory)
+    static __device__ __forceinline__ void vec_generic(const __nv_bfloat16 *p, float (&o)[V]) {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(p);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            o[2 * i] = __uint_as_float(w[i] << 16);
+            o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
 };
 template <>
 struct XLoad<float> {
@@ -130,6 +140,13 @@ struct XLoad<float> {
         o[3] = raw.w;
     }
     static __device__ __forceinline__ float one(const float *p) { return *p; }
+    static __device__ __forceinline__ void vec_generic(const float *p, float (&o)[V]) {
+        const float4 raw = *reinterpret_cast<const float4 *>(p);
+        o[0] = raw.x;
+        o[1] = raw.y;
+        o[2] = raw.z;
+        o[3] = raw.w;
+    }
 };
 
 // ---------------------------------------------------------------------------
@@ -231,6 +248,160 @@ __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restr
     }
     __syncthreads();
     publish_tile(psum_w, hist_w, N, tiles, tile, hist, psum);
+}
+
+// ---------------------------------------------------------------------------
+// Router for N <= 32 with the whole 64-token tile of x staged in shared
+// memory.  One bulk copy per row (rows padded by 64 bytes so that the reads
+// below are free of bank conflicts) completes on one of four mbarriers, one
+// per 16-token chunk, so the first warps start while later rows still land.
+// Four threads share a token: thread (token, part) accumulates all N partial
+// dot products over the 16-byte x vectors j = part, part + 4, ... against
+// W_r held as [d/V][V][NP] (+4 floats of padding per j).  Two shuffles then
+// give each of the four the token's full logits, so the softmax, argmax and
+// gate need no further exchange.  Sum of p over the tile: shuffles over the
+// warp's 8 tokens, then a fixed-order sum over the 8 warps (deterministic).
+// ---------------------------------------------------------------------------
+template <typename XT>
+struct Staged {
+    static constexpr int V = XLoad<XT>::V;
+    static __host__ __device__ int64_t xpitch(int d) { return (int64_t)d * sizeof(XT) + 64; }
+    static __host__ __device__ int64_t wpitch(int NP) { return (int64_t)V * NP + 4; }  // floats per 16-byte x vector of W_r
+    static size_t smem(int d, int NP) {
+        return (size_t)(kTileT * xpitch(d)) + (size_t)((d / V) * wpitch(NP)) * 4 + (size_t)(kWarps * NP) * 4 +
+               (size_t)NP * 4 + 4 * 8 + 16;
+    }
+};
+
+template <typename XT, int NP>
+__global__ void __launch_bounds__(kThreads, 1)
+    router_staged_kernel(const XT *__restrict__ x, const float *__restrict__ w_r, const float *__restrict__ bias,
+                         int64_t T, int d, int N, int tiles, int32_t *__restrict__ expert, float *__restrict__ gate,
+                         int32_t *__restrict__ hist, float *__restrict__ psum, uint32_t *ticket,
+                         DeviceStatus *status) {
+    using S = Staged<XT>;
+    constexpr int V = S::V;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int64_t xpitch = S::xpitch(d);
+    const int64_t wpitch = S::wpitch(NP);
+    unsigned char *xs = smem_raw;
+    float *wsm = reinterpret_cast<float *>(smem_raw + kTileT * xpitch);
+    float *psum_w = wsm + (d / V) * wpitch;
+    int32_t *hist_s = reinterpret_cast<int32_t *>(psum_w + kWarps * NP);
+    uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(hist_s + NP) + 15) & ~uintptr_t(15));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tile = blockIdx.x;
+    const int64_t t0 = (int64_t)tile * kTileT;
+    const int n_tok = (int)(T - t0 < kTileT ? T - t0 : kTileT);
+    const uint32_t row_bytes = (uint32_t)(d * sizeof(XT));
+
+    if (tid == 0) {
+        if (tile == 0) reset_call_state(ticket, status);
+        for (int c = 0; c < 4; ++c) mbar_init(&bar[c], 1);
+        fence_barrier_init();
+        for (int c = 0; c < 4; ++c) {
+            const int rows = max(0, min(16, n_tok - 16 * c));
+            if (rows > 0) mbar_arrive_expect_tx(&bar[c], (uint32_t)rows * row_bytes);
+        }
+    }
+    __syncthreads();  // barriers initialised before any copy signals them
+    if (tid < n_tok) bulk_load(xs + tid * xpitch, x + (t0 + tid) * d, row_bytes, &bar[tid >> 4]);
+    // W_r (row-major [N][d], read coalesced) -> [d/V][V][NP] with padding,
+    // while the rows of x are on their way.  Batches of 8 loads per thread
+    // are in flight before their stores.
+    for (int i0 = 0; i0 < NP * d; i0 += 8 * kThreads) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kThreads + tid;
+            v[u] = (i < N * d) ? w_r[i] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kThreads + tid;
+            if (i < NP * d) {
+                const int e = i / d, k = i % d;
+                wsm[(k / V) * wpitch + (k % V) * NP + e] = v[u];
+            }
+        }
+    }
+    for (int i = tid; i < kWarps * NP; i += kThreads) psum_w[i] = 0.f;
+    for (int i = tid; i < NP; i += kThreads) hist_s[i] = 0;
+    __syncthreads();
+
+    const int tl = tid >> 2, part = tid & 3;
+    const bool valid = tl < n_tok;
+    float acc[NP];
+#pragma unroll
+    for (int e = 0; e < NP; ++e) acc[e] = 0.f;
+    if (valid && mbar_wait(&bar[tl >> 4], 0, status, 10)) {
+        const unsigned char *xrow = xs + tl * xpitch;
+        for (int j = part; j < d / V; j += 4) {
+            float xv[V];
+            XLoad<XT>::vec_generic(reinterpret_cast<const XT *>(xrow + (int64_t)j * 16), xv);  // shared memory
+            const float *wj = wsm + j * wpitch;
+#pragma unroll
+            for (int u = 0; u < V; ++u) {
+#pragma unroll
+                for (int q = 0; q < NP / 4; ++q) {
+                    const float4 w4 = *reinterpret_cast<const float4 *>(wj + u * NP + 4 * q);
+                    acc[4 * q + 0] = fmaf(xv[u], w4.x, acc[4 * q + 0]);
+                    acc[4 * q + 1] = fmaf(xv[u], w4.y, acc[4 * q + 1]);
+                    acc[4 * q + 2] = fmaf(xv[u], w4.z, acc[4 * q + 2]);
+                    acc[4 * q + 3] = fmaf(xv[u], w4.w, acc[4 * q + 3]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 1);
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 2);
+    }
+    float m = -FLT_MAX;
+    int arg = 0;
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+        if (e < N) {
+            acc[e] += bias ? bias[e] : 0.f;
+            if (acc[e] > m) {  // strict: the lowest index wins a tie
+                m = acc[e];
+                arg = e;
+            }
+        }
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+        acc[e] = e < N ? expf(acc[e] - m) : 0.f;
+        s += acc[e];
+    }
+#pragma unroll
+    for (int e = 0; e < NP; ++e) acc[e] = valid ? acc[e] / s : 0.f;  // p_e
+    if (valid && part == 0) {
+        const int64_t t = t0 + tl;
+        expert[t] = arg;
+        gate[t] = 1.0f / s;  // p at the argmax: exp(0) / s
+        atomicAdd(&hist_s[arg], 1);
+    }
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 4);
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int e = 0; e < NP; ++e) psum_w[warp * NP + e] = acc[e];
+    }
+    __syncthreads();
+    for (int i = tid; i < N; i += kThreads) {
+        float p = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) p += psum_w[w * NP + i];
+        hist[(int64_t)i * tiles + tile] = hist_s[i];
+        psum[(int64_t)i * tiles + tile] = p;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -392,23 +563,30 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t *__res
         run += h[i];
     }
 
-    // The last expert block to finish forms the aux loss, in fixed expert order.
+    // The last expert block to finish forms the aux loss: one f_i * P_i per
+    // thread (all loads in parallel), then a fixed-order tree over threads.
     __threadfence();
     __syncthreads();
     if (tid == 0) is_last = atomicAdd(ticket, 1u) == (uint32_t)(N - 1);
     __syncthreads();
-    if (is_last && tid == 0) {
+    if (is_last) {
         __threadfence();
-        double total = 0.0;
-        if (T > 0) {
-            for (int i = 0; i < N; ++i) {
-                const double f = (double)((volatile int32_t *)counts)[i] / (double)T;
-                const double P = ((volatile double *)prob_total)[i] / (double)T;
-                total += f * P;
-            }
+        double term = 0.0;
+        if (T > 0 && tid < N) {
+            const double f = (double)__ldcg(counts + tid) / (double)T;
+            const double P = __ldcg(prob_total + tid) / (double)T;
+            term = f * P;
         }
-        *aux = (float)((double)N * total);
-        *ticket = 0u;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) term += __shfl_xor_sync(0xffffffffu, term, off);
+        if (lane == 0) warp_p[warp] = term;
+        __syncthreads();
+        if (tid == 0) {
+            double total = 0.0;
+            for (int w = 0; w < kScanThreads / 32; ++w) total += warp_p[w];
+            *aux = (float)((double)N * total);
+            *ticket = 0u;
+        }
     }
 }
 
@@ -467,25 +645,43 @@ __global__ void __launch_bounds__(kAssignThreads) assign_kernel(
         }
         if (SCATTER) {
             __syncthreads();
-            for (int r = warp; r < kTileT; r += kAssignThreads / 32) {
-                const int s = tile_slot[r];
-                const int64_t tr = (int64_t)tile * kTileT + r;
-                if (s >= 0) {
-                    const uint4 *src = x + tr * x_words;
-                    uint4 *dst = xbuf + ((int64_t)tile_expert[r] * C + s) * x_words;
-                    int w = lane;
-                    for (; w + 96 < x_words; w += 128) {
-                        const uint4 a = __ldcs(src + w), b = __ldcs(src + w + 32), c = __ldcs(src + w + 64),
-                                    d4 = __ldcs(src + w + 96);
-                        dst[w] = a;
-                        dst[w + 32] = b;
-                        dst[w + 64] = c;
-                        dst[w + 96] = d4;
+            // Each warp moves rows warp, warp + 8, ...: all loads of a group of
+            // four rows are in flight before the first store.
+            constexpr int kRows = 4, kWords = 4;  // per lane: 4 rows x 4 x 16 bytes
+            for (int r0 = warp; r0 < kTileT; r0 += (kAssignThreads / 32) * kRows) {
+                for (int w0 = 0; w0 < x_words; w0 += 32 * kWords) {
+                    uint4 v[kRows][kWords];
+#pragma unroll
+                    for (int i = 0; i < kRows; ++i) {
+                        const int r = r0 + i * (kAssignThreads / 32);
+                        const int s = r < kTileT ? tile_slot[r] : -2;
+                        const uint4 *src = x + ((int64_t)tile * kTileT + r) * x_words;
+#pragma unroll
+                        for (int u = 0; u < kWords; ++u) {
+                            const int w = w0 + lane + 32 * u;
+                            if (s >= 0 && w < x_words) v[i][u] = __ldcs(src + w);
+                        }
                     }
-                    for (; w < x_words; w += 32) dst[w] = __ldcs(src + w);
-                } else if (s == -1 && y_zero) {
-                    float4 *dst = y_zero + tr * y_words;
-                    for (int w = lane; w < y_words; w += 32) __stcs(dst + w, make_float4(0.f, 0.f, 0.f, 0.f));
+#pragma unroll
+                    for (int i = 0; i < kRows; ++i) {
+                        const int r = r0 + i * (kAssignThreads / 32);
+                        const int s = r < kTileT ? tile_slot[r] : -2;
+                        if (s < 0) continue;
+                        uint4 *dst = xbuf + ((int64_t)tile_expert[r] * C + s) * x_words;
+#pragma unroll
+                        for (int u = 0; u < kWords; ++u) {
+                            const int w = w0 + lane + 32 * u;
+                            if (w < x_words) dst[w] = v[i][u];
+                        }
+                    }
+                }
+                if (y_zero) {
+                    for (int i = 0; i < kRows; ++i) {
+                        const int r = r0 + i * (kAssignThreads / 32);
+                        if (r >= kTileT || tile_slot[r] != -1) continue;
+                        float4 *dst = y_zero + ((int64_t)tile * kTileT + r) * y_words;
+                        for (int w = lane; w < y_words; w += 32) __stcs(dst + w, make_float4(0.f, 0.f, 0.f, 0.f));
+                    }
                 }
             }
         }
@@ -515,6 +711,23 @@ cudaError_t launch_router_warp(const switch_dims_t &dims, const XT *x, const flo
     return err;
 }
 
+template <typename XT, int NP>
+cudaError_t launch_router_staged(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
+                                 int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
+    const int N = dims.num_experts, d = dims.d_model;
+    const size_t smem = Staged<XT>::smem(d, NP);
+    auto kern = router_staged_kernel<XT, NP>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    launch_begin(K_ROUTER_STAGED, stream);
+    kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
+                                                         ws.hist, ws.psum, ws.ticket,
+                                                         static_cast<DeviceStatus *>(ws.status));
+    err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
+
 template <typename XT, int EC>
 cudaError_t launch_router_tiled(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
                                 int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
@@ -535,12 +748,21 @@ cudaError_t launch_router_tiled(const switch_dims_t &dims, const XT *x, const fl
 
 // Largest d for which the warp router keeps W_r in shared memory.
 constexpr size_t kWarpRouterSmemLimit = 160 * 1024;
+// Shared memory the staged router may use (x tile + W_r + partials).
+constexpr size_t kStagedSmemLimit = 200 * 1024;
 
 template <typename XT>
 cudaError_t launch_router(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
                           int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts;
     const int NP = N <= 8 ? 8 : N <= 16 ? 16 : 32;
+    const bool staged = N <= 32 && ((int64_t)dims.d_model * (int64_t)sizeof(XT)) % 16 == 0 &&
+                        Staged<XT>::smem(dims.d_model, NP) <= kStagedSmemLimit;
+    if (staged) {
+        if (NP == 8) return launch_router_staged<XT, 8>(dims, x, w_r, bias, expert, gate, ws, stream);
+        if (NP == 16) return launch_router_staged<XT, 16>(dims, x, w_r, bias, expert, gate, ws, stream);
+        return launch_router_staged<XT, 32>(dims, x, w_r, bias, expert, gate, ws, stream);
+    }
     const bool fits = N <= 32 && (size_t)dims.d_model * NP * sizeof(float) + 2048 * 8 <= kWarpRouterSmemLimit;
     if (fits) {
         if (NP == 8) return launch_router_warp<XT, 8>(dims, x, w_r, bias, expert, gate, ws, stream);
@@ -559,7 +781,10 @@ cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *
                          float *aux, const Workspace &ws, cudaStream_t stream, void *xbuf_scatter, float *y_zero) {
     cudaError_t err = cudaSuccess;
     const int N = dims.num_experts, C = dims.capacity;
-    if (ws.tiles > 0) {
+    if (ws.tiles > 0 && router_tc_supported(dims)) {
+        err = launch_router_tc(dims, x, w_r, bias, expert, gate, ws, stream);
+        if (err != cudaSuccess) return err;
+    } else if (ws.tiles > 0) {
         err = dims.dtype == SWITCH_BF16
                   ? launch_router<__nv_bfloat16>(dims, static_cast<const __nv_bfloat16 *>(x), w_r, bias, expert,
                                                  gate, ws, stream)

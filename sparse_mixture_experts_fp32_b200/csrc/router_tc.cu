@@ -1,0 +1,394 @@
+// Router on tcgen05 tensor cores, for bfloat16 activations and 32 < N <= 128
+// experts (sm_100a).
+//
+// The router computes in float32 (kasblo "Switch Transformerとは？" section
+// "Routerだけfloat32で計算するSelective Precision"; logits h = W_r . x,
+// llm-papers-study "精读 06 | Switch Transformers" §3.1).  x is bfloat16, so
+// it is exact as an MMA operand.  W_r (float32) is split into three bfloat16
+// terms, hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid), whose sum
+// is w exactly for every w of normal magnitude.  Three kind::f16 MMAs per
+// K-step add x . hi, x . mid and x . lo into one float32 accumulator in
+// tensor memory: every product is exact, only the order of the float32
+// additions differs from a CUDA-core dot product.
+//
+// Tile = 128 tokens (MMA M) x BN experts (MMA N, the experts padded to 64 or
+// 128; padding rows of W_r are zero-filled by TMA and ignored).  One CTA per
+// SM, persistent over token tiles:
+//   warp 0     TMA: 128 x 64 tile of x and the three 64-wide slices of W_r
+//   warp 1     TMEM allocation; one lane issues the MMAs
+//   warps 2-5  epilogue, one thread per token: tcgen05.ld of its row, max
+//              and argmax (lowest index on ties), sum of exp, gate = 1/sum,
+//              p_i; per-64-token-tile expert counts and sums of p_i
+//              (deterministic: a fixed shuffle tree, then a fixed warp order)
+#include <cuda.h>
+
+#include <algorithm>
+#include <float.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace switchmoe {
+namespace {
+
+constexpr int RM = 128;  // tokens per tile
+constexpr int RK = 64;   // K per ring stage (one 128-byte swizzle row of bf16)
+constexpr int kTerms = 3;
+constexpr int kThreads = 192;
+
+// W_r float32 [N][d] -> three bfloat16 terms [3][N][d].
+__global__ void split_router_weight(const float *__restrict__ w, __nv_bfloat16 *__restrict__ out, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = w[i];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        const float r1 = v - __bfloat162float(hi);
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(mid);
+        out[i] = hi;
+        out[n + i] = mid;
+        out[2 * n + i] = __float2bfloat16_rn(r2);
+    }
+}
+
+template <int BN, int STAGES>
+struct RouterLayout {
+    static constexpr size_t a_bytes = (size_t)RM * RK * 2;
+    static constexpr size_t b_term_bytes = (size_t)BN * RK * 2;
+    static constexpr size_t b_bytes = kTerms * b_term_bytes;
+    static constexpr size_t ring = STAGES * (a_bytes + b_bytes);
+    static constexpr size_t barriers = (2 * STAGES + 2 + 2 + 1) * 8 + 16;
+    static constexpr size_t epi = (size_t)BN * 4 /*bias*/ + 4 * BN * 4 /*psum per warp*/ + 2 * BN * 4 /*counts*/;
+    static constexpr size_t bytes = 1024 + ring + barriers + epi;
+};
+
+// Sum v[i] over the 32 lanes for every i; lane l ends with the total of index l.
+__device__ __forceinline__ float reduce_scatter32(float (&v)[32]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {
+        const int off = 16 >> step;
+        const int half = 16 >> step;
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (i < half) {
+                const float send = upper ? v[i] : v[i + half];
+                const float keep = upper ? v[i + half] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            }
+        }
+    }
+    return v[0];
+}
+
+__device__ __forceinline__ void named_barrier_epilogue() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, uint64_t *bar, int32_t c0, int32_t c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                     const float *__restrict__ bias, int64_t T, int d, int N, int tiles64,
+                     int32_t *__restrict__ expert, float *__restrict__ gate, int32_t *__restrict__ hist,
+                     float *__restrict__ psum, uint32_t *ticket, DeviceStatus *status) {
+    using L = RouterLayout<BN, STAGES>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;
+    uint8_t *sB = sA + STAGES * L::a_bytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(base + L::ring);
+    uint64_t *empty = full + STAGES;
+    uint64_t *acc_full = empty + STAGES;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *drain = acc_empty + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    float *bias_s = reinterpret_cast<float *>(tmem_holder + 4);
+    float *psum_w = bias_s + BN;                                  // [4][BN]
+    int32_t *hist_s = reinterpret_cast<int32_t *>(psum_w + 4 * BN);  // [2][BN]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m_tiles = (int)((T + RM - 1) / RM);
+    const int k_blocks = (d + RK - 1) / RK;
+    constexpr uint32_t kTmemCols = 2 * BN;
+
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *ticket = 0u;
+        status->code = 0;
+        status->where = 0;
+        status->block = 0;
+        status->reserved = 0;
+    }
+    if (warp == 1) {
+        if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], 1);
+            }
+            for (int a = 0; a < 2; ++a) {
+                mbar_init(&acc_full[a], 1);
+                mbar_init(&acc_empty[a], 128);
+            }
+            mbar_init(drain, 1);
+            fence_barrier_init();
+        }
+        __syncwarp();
+        tmem_alloc(tmem_holder, kTmemCols);
+        tmem_relinquish();
+    } else if (warp >= 2) {
+        const int et = threadIdx.x - 64;
+        for (int i = et; i < BN; i += 128) bias_s[i] = (bias && i < N) ? bias[i] : 0.f;
+        for (int i = et; i < 2 * BN; i += 128) hist_s[i] = 0;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tmap_x);
+            prefetch_tmap(&tmap_w);
+            uint32_t issued = 0, parity_of = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < m_tiles; tile += gridDim.x) {
+                // x streams from HBM: pull this CTA's next token tile into L2 now
+                const int next = tile + (int)gridDim.x;
+                if (next < m_tiles)
+                    for (int kb = 0; kb < k_blocks; ++kb) tma_prefetch_l2_2d(&tmap_x, kb * RK, next * RM);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, status, 31)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(L::a_bytes + L::b_bytes));
+                    tma_load_2d(sA + stage * L::a_bytes, &tmap_x, &full[stage], kb * RK, tile * RM);
+#pragma unroll
+                    for (int term = 0; term < kTerms; ++term)
+                        tma_load_3d(sB + stage * L::b_bytes + term * L::b_term_bytes, &tmap_w, &full[stage], kb * RK,
+                                    0, term);
+                    issued |= 1u << stage;
+                    parity_of = (parity_of & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            for (int s = 0; s < STAGES; ++s)
+                if (issued & (1u << s)) mbar_wait(&full[s], (parity_of >> s) & 1u, status, 36);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(RM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < m_tiles; tile += gridDim.x) {
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, status, 32)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, status, 33)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t a_desc = smem_desc_sw128(sA + stage * L::a_bytes);
+#pragma unroll
+                    for (int k = 0; k < RK / 16; ++k) {
+#pragma unroll
+                        for (int term = 0; term < kTerms; ++term) {
+                            const uint64_t b_desc =
+                                smem_desc_sw128(sB + stage * L::b_bytes + term * L::b_term_bytes);
+                            tc_mma_bf16(d_tmem, a_desc + (uint64_t)(2 * k), b_desc + (uint64_t)(2 * k), idesc,
+                                        (kb | k | term) != 0 ? 1u : 0u);
+                        }
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&acc_full[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            tc_commit(drain);
+            mbar_wait(drain, 0, status, 34);
+        }
+    } else {
+        const int q = warp & 3;  // TMEM lane quarter: tokens 32q .. 32q+31 of the tile
+        const int et = threadIdx.x - 64;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < m_tiles; tile += gridDim.x) {
+            if (!mbar_wait(&acc_full[acc], acc_phase, status, 35)) break;
+            tc_fence_after();
+            const int64_t t = (int64_t)tile * RM + q * 32 + lane;
+            const bool valid = t < T;
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+            uint32_t r[32];
+            float m = -FLT_MAX;
+            int arg = 0;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 32) {
+                tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float h = __uint_as_float(r[j]) + bias_s[c + j];
+                    if (c + j < N && h > m) {  // strict: the lowest index wins a tie
+                        m = h;
+                        arg = c + j;
+                    }
+                }
+            }
+            float s = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 32) {
+                tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (c + j < N) s += expf(__uint_as_float(r[j]) + bias_s[c + j] - m);
+            }
+            const float inv_s = 1.0f / s;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 32) {
+                tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
+                tmem_ld_wait();
+                float p[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    p[j] = (valid && c + j < N) ? expf(__uint_as_float(r[j]) + bias_s[c + j] - m) * inv_s : 0.f;
+                const float col_sum = reduce_scatter32(p);  // this warp's 32 tokens, column c + lane
+                psum_w[q * BN + c + lane] = col_sum;
+            }
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);  // the accumulator may be reused now
+            if (valid) {
+                expert[t] = arg;
+                gate[t] = inv_s;  // p at the argmax: exp(0) / s
+                atomicAdd(&hist_s[(q >> 1) * BN + arg], 1);
+            }
+            named_barrier_epilogue();
+            for (int i = et; i < N; i += 128) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int t64 = 2 * tile + half;
+                    if (t64 < tiles64) {
+                        hist[(int64_t)i * tiles64 + t64] = hist_s[half * BN + i];
+                        psum[(int64_t)i * tiles64 + t64] = psum_w[(2 * half) * BN + i] + psum_w[(2 * half + 1) * BN + i];
+                    }
+                    hist_s[half * BN + i] = 0;
+                }
+            }
+            named_barrier_epilogue();
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_bn(const switch_dims_t &dims, const __nv_bfloat16 *x, const float *bias, int32_t *expert,
+                      float *gate, const Workspace &ws, cudaStream_t stream) {
+    const int N = dims.num_experts, d = dims.d_model;
+    const int64_t T = dims.T;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    CUtensorMap tx, tw;
+    const cuuint32_t estr[3] = {1, 1, 1};
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)T};
+        const cuuint64_t gstr[1] = {(cuuint64_t)d * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)RK, (cuuint32_t)RM};
+        if (fn(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(x), gdim, gstr, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const cuuint64_t gdim[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)kTerms};
+        const cuuint64_t gstr[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+        const cuuint32_t box[3] = {(cuuint32_t)RK, (cuuint32_t)BN, 1};
+        if (fn(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ws.w_split, gdim, gstr, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    auto kern = router_tc_kernel<BN, STAGES>;
+    const size_t smem = RouterLayout<BN, STAGES>::bytes;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    const int64_t m_tiles = (T + RM - 1) / RM;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count(), m_tiles));
+    launch_begin(K_ROUTER_TC, stream);
+    kern<<<grid, kThreads, smem, stream>>>(tx, tw, bias, T, d, N, (int)ws.tiles, expert, gate, ws.hist, ws.psum,
+                                           ws.ticket, static_cast<DeviceStatus *>(ws.status));
+    err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
+
+}  // namespace
+
+bool router_tc_supported(const switch_dims_t &dims) {
+    return dims.dtype == SWITCH_BF16 && dims.num_experts > 32 && dims.num_experts <= 128 && dims.T > 0 &&
+           !(dims.flags & SWITCH_FLAG_SIMT_ROUTER);
+}
+
+cudaError_t launch_router_tc(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
+                             int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
+    const int64_t n = (int64_t)dims.num_experts * dims.d_model;
+    launch_begin(K_ROUTER_SPLIT, stream);
+    split_router_weight<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, stream>>>(
+        w_r, static_cast<__nv_bfloat16 *>(ws.w_split), n);
+    cudaError_t err = cudaGetLastError();
+    launch_end(stream);
+    if (err != cudaSuccess) return err;
+    const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+    if (dims.num_experts <= 64) return launch_bn<64, 4>(dims, xb, bias, expert, gate, ws, stream);
+    return launch_bn<128, 3>(dims, xb, bias, expert, gate, ws, stream);
+}
+
+}  // namespace switchmoe

@@ -290,7 +290,7 @@ def test_tracer_and_launch_counter():
     trace = sm.trace_read()
     sm.trace_stop()
     names = [n for n, _ in trace]
-    assert names == ["router_warp", "capacity_scan", "slot_assign_scatter", "ffn_tc_gemm1_relu",
+    assert names == ["router_staged", "capacity_scan", "slot_assign_scatter", "ffn_tc_gemm1_relu",
                      "ffn_tc_gemm2_gated_scatter"]
     assert all(ms >= 0 for _, ms in trace)
     assert sm.launch_count() - before == len(names)
