@@ -163,6 +163,7 @@ def kernel_work(wl, C, counts):
         "slot_assign_scatter": ("hbm", 4 * T + 4 * T + 4 * N * tiles + 4 * N * C + 2 * K * d * s + (T - K) * d * 4),
         "ffn_tc_gemm1_relu": ("tensor", 2.0 * K * d * F),
         "ffn_tc_gemm2_gated_scatter": ("tensor", 2.0 * K * F * d),
+        "ffn_tc_fused": ("tensor", 4.0 * K * d * F),
         "ffn_simt_gemm1_relu": ("alu", 2.0 * K * d * F),
         "ffn_simt_gemm2": ("alu", 2.0 * K * F * d),
         "combine": ("hbm", T * d * 4 + K * d * 4 + 12 * T),
@@ -194,8 +195,10 @@ def run_gpu(args):
     wl = synth.WORKLOADS[args.workload]
     if args.capacity_factor is not None:
         wl = wl.with_capacity_factor(args.capacity_factor)
-    seed = rank_seed(wl, rank)
-    inp = synth.inputs(wl, seed=None) if rank == 0 else dict(synth.inputs(wl), x=synth.activations(wl, seed=seed))
+    # experts and router are shared by all ranks; every rank routes its own tokens
+    w_in_np, w_out_np = synth.all_expert_weights(wl)
+    inp = dict(x=synth.activations(wl, seed=rank_seed(wl, rank)), w_r=synth.router_weight(wl),
+               bias=synth.router_bias(wl), w_in=w_in_np, w_out=w_out_np)
     C = sm.switch_capacity(wl.T, wl.num_experts, wl.capacity_factor)
 
     x = to_dev(inp["x"], device)
@@ -244,7 +247,6 @@ def run_gpu(args):
     sampler = ClockSampler(local) if rank == 0 else None
     if sampler:
         time.sleep(0.3)
-    sm.trace_start(K * 8)
     launches0 = sm.launch_count()
     if world > 1:
         dist.barrier()
@@ -260,8 +262,6 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     launches = sm.launch_count() - launches0
-    trace = sm.trace_read(K * 8)
-    sm.trace_stop()
     clocks = sampler.summary(t_wall0, t_wall1) if sampler else None
     if sampler:
         sampler.stop()
@@ -271,6 +271,21 @@ def run_gpu(args):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = max_over_ranks(sum(step_ms), world, device)
     ms_per_step = total_ms / K
+
+    # the same K steps again with the library's per-launch tracer on: per-kernel
+    # durations for the roofline (events between kernels serialise them, so
+    # these steps are timed separately from the headline ones)
+    sm.trace_start(K * 8)
+    traced_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        flush.fill_(float(i))
+        traced_ev[i][0].record(stream)
+        step()
+        traced_ev[i][1].record(stream)
+    torch.cuda.synchronize(device)
+    trace = sm.trace_read(K * 8)
+    sm.trace_stop()
+    traced_ms_per_step = sum(a.elapsed_time(b) for a, b in traced_ev) / K
 
     # per-kernel averages from the library's tracer (same steps)
     per_kernel: dict[str, list[float]] = {}
@@ -309,6 +324,36 @@ def run_gpu(args):
     # e2e through the public API with pinned host buffers
     e2e = run_e2e(args, sm, wl, inp, C, device, world)
 
+    # capacity-factor sweep on the same tokens and weights (--sweep)
+    sweep = []
+    if args.sweep and wl.sweep:
+        for c in wl.sweep:
+            Cc = sm.switch_capacity(T, N, c)
+            dc = sm.layer_dims(x, w_in, capacity=Cc)
+            wsc = sm.workspace(dc, device)
+            outc = sm.layer_fwd(x, w_r, w_in, w_out, capacity=Cc, logit_bias=bias, ws=wsc)
+            for _ in range(args.warmup):
+                flush.fill_(1.0)
+                sm.layer_fwd(x, w_r, w_in, w_out, capacity=Cc, logit_bias=bias, ws=wsc, out=outc)
+            torch.cuda.synchronize(device)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+            for i in range(K):
+                flush.fill_(float(i))
+                evs[i][0].record(stream)
+                sm.layer_fwd(x, w_r, w_in, w_out, capacity=Cc, logit_bias=bias, ws=wsc, out=outc)
+                evs[i][1].record(stream)
+            torch.cuda.synchronize(device)
+            if sm.switch_check(wsc) != 0:
+                raise RuntimeError("device status after the sweep steps")
+            msc = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, device) / K
+            kept = int(np.minimum(outc["counts"].cpu().numpy(), Cc).sum())
+            sweep.append({"capacity_factor": c, "capacity": Cc, "ms_per_step": round(msc, 5),
+                          "value": round(world * T / (msc * 1e-3), 1), "kept_tokens": kept,
+                          "drop_fraction": round(1 - kept / T, 6),
+                          "expert_flops_per_step": 4.0 * kept * d * wl.d_ff})
+            del wsc, outc
+            torch.cuda.empty_cache()
+
     result = None
     if rank == 0:
         value = world * T / (ms_per_step * 1e-3)
@@ -326,10 +371,13 @@ def run_gpu(args):
             "roofline": roofline,
             "kernels": kernels,
             "gpu_launches": int(launches),
+            "traced_ms_per_step": round(traced_ms_per_step, 5),
             "e2e": e2e,
             "clocks": clocks,
             "wall_s_timed_region": round(t_wall1 - t_wall0, 4),
         }
+        if sweep:
+            result["sweep"] = sweep
         if not args.no_cpu_baseline and world == 1:
             result["cpu_baseline"] = cpu_baseline(wl, inp, C, budget_s=args.cpu_budget)
     if world > 1:
@@ -339,43 +387,71 @@ def run_gpu(args):
 
 
 def run_e2e(args, sm, wl, inp, C, device, world):
-    """Same metric through sm.layer_fwd with host-resident inputs and outputs."""
+    """Same metric through sm.layer_fwd with host-resident inputs and outputs.
+
+    Every step copies its x from pinned host memory to the device, runs the
+    layer and copies y, aux and counts back to pinned host memory.  The three
+    parts run on their own streams with two sets of device buffers, so step
+    i's output copy, step i+1's layer and step i+2's input copy overlap, as a
+    caller streaming batches would run them; the time is from the first input
+    copy to the last output copy."""
     import torch
     T, d, N = wl.T, wl.d_model, wl.num_experts
     tdt = torch.bfloat16 if wl.dtype == synth.BF16 else torch.float32
     x_host = to_dev(inp["x"], "cpu").pin_memory()
-    x_dev = torch.empty(T, d, dtype=tdt, device=device)
     w = {k: to_dev(inp[k], device) for k in ("w_r", "bias", "w_in", "w_out")}
-    y_host = torch.empty(T, d, dtype=torch.float32).pin_memory()
-    aux_host = torch.empty(1, dtype=torch.float32).pin_memory()
-    counts_host = torch.empty(N, dtype=torch.int32).pin_memory()
-    out = None
+    x_dev = [torch.empty(T, d, dtype=tdt, device=device) for _ in range(2)]
+    y_host = [torch.empty(T, d, dtype=torch.float32).pin_memory() for _ in range(2)]
+    aux_host = [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(2)]
+    counts_host = [torch.empty(N, dtype=torch.int32).pin_memory() for _ in range(2)]
+    s_in, s_cmp, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    cmp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+    outs = [None, None]
     ws = None
     steps = max(3, min(args.steps, args.e2e_steps))
 
-    def one():
-        nonlocal out, ws
-        x_dev.copy_(x_host, non_blocking=True)
-        out = sm.layer_fwd(x_dev, w["w_r"], w["w_in"], w["w_out"], capacity=C, logit_bias=w["bias"], ws=ws,
-                           out=out)
-        ws = out["workspace"]
-        y_host.copy_(out["y"], non_blocking=True)
-        aux_host.copy_(out["aux"], non_blocking=True)
-        counts_host.copy_(out["counts"], non_blocking=True)
+    def one(i):
+        nonlocal ws
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(cmp_done[b])  # the layer of step i-2 has read x_dev[b]
+            x_dev[b].copy_(x_host, non_blocking=True)
+            in_done[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(in_done[b])
+            if i >= 2:
+                s_cmp.wait_event(out_done[b])  # y of step i-2 has left outs[b]
+            outs[b] = sm.layer_fwd(x_dev[b], w["w_r"], w["w_in"], w["w_out"], capacity=C, logit_bias=w["bias"],
+                                   ws=ws, out=outs[b], stream=s_cmp)
+            ws = outs[b]["workspace"]
+            cmp_done[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(cmp_done[b])
+            y_host[b].copy_(outs[b]["y"], non_blocking=True)
+            aux_host[b].copy_(outs[b]["aux"], non_blocking=True)
+            counts_host[b].copy_(outs[b]["counts"], non_blocking=True)
+            out_done[b].record(s_out)
 
-    for _ in range(3):
-        one()
+    for i in range(4):
+        one(i)
     torch.cuda.synchronize(device)
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(steps):
-        one()
-    e.record()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    for i in range(steps):
+        one(i + 4)
+    end.record(s_out)
     torch.cuda.synchronize(device)
-    ms = max_over_ranks(s.elapsed_time(e) / steps, world, device)
+    ms = max_over_ranks(start.elapsed_time(end) / steps, world, device)
+    status = sm.switch_check(ws)
+    if status != 0:
+        raise sm.SwitchError(status, "device status after the e2e steps")
     return {"value": round(world * T / (ms * 1e-3), 1), "unit": UNIT, "ms_per_step": round(ms, 5),
             "steps": steps, "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
-            "d2h_bytes_per_step": int(y_host.numel() * 4 + 4 + N * 4)}
+            "d2h_bytes_per_step": int(y_host[0].numel() * 4 + 4 + N * 4),
+            "overlap": "input copy, layer and output copy on three streams, two buffer sets"}
 
 
 def traffic_from_profiles(kernel: str, workload: str):
@@ -464,6 +540,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle FFN time for cpu_baseline")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="also time every capacity factor of the workload's sweep")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -83,7 +83,10 @@ enum {
     SWITCH_FLAG_SIMT_ROUTER = 2,
     /* Run each expert GEMM tile on one SM (cta_group::1, 128-row tiles)
      * instead of on a pair of SMs (cta_group::2, 256-row tiles). */
-    SWITCH_FLAG_GEMM_1CTA = 4
+    SWITCH_FLAG_GEMM_1CTA = 4,
+    /* In switch_layer_fwd, launch the two expert GEMMs one after the other
+     * instead of as one persistent kernel. */
+    SWITCH_FLAG_FFN_TWO_LAUNCHES = 8
 };
 
 typedef struct {
@@ -211,6 +214,15 @@ switch_status_t switch_route_noalloc(const switch_dims_t *dims, const void *x, c
  * Returns SWITCH_OK, SWITCH_ERR_DEVICE_TIMEOUT, or SWITCH_ERR_CUDA if the
  * stream reports an error. */
 switch_status_t switch_check(void *workspace, size_t workspace_bytes, switch_stream_t stream);
+
+/* Self-test of the device-side failure detection.  Launches one block that
+ * waits, with the same bounded wait the library's kernels use, on an mbarrier
+ * that nothing completes.  After about one second the wait gives up, records
+ * SWITCH_ERR_DEVICE_TIMEOUT in the workspace status word and the kernel exits
+ * normally (no trap, no fault): switch_check() then returns
+ * SWITCH_ERR_DEVICE_TIMEOUT and the CUDA context stays usable.  Needs at
+ * least 16 bytes of workspace. */
+switch_status_t switch_selftest_wait_timeout(void *workspace, size_t workspace_bytes, switch_stream_t stream);
 
 /* Static description of a status code. */
 const char *switch_status_string(switch_status_t status);

@@ -29,6 +29,7 @@ SWITCH_BF16 = 1
 SWITCH_FLAG_SIMT_FFN = 1
 SWITCH_FLAG_SIMT_ROUTER = 2
 SWITCH_FLAG_GEMM_1CTA = 4
+SWITCH_FLAG_FFN_TWO_LAUNCHES = 8
 
 STATUS = {
     0: "SWITCH_OK", 1: "SWITCH_ERR_NULL", 2: "SWITCH_ERR_SHAPE", 3: "SWITCH_ERR_DTYPE", 4: "SWITCH_ERR_ALIGN",
@@ -38,7 +39,8 @@ STATUS = {
 
 EXPORTED = ("switch_capacity", "switch_workspace_size", "switch_route", "switch_route_noalloc", "switch_dispatch",
             "switch_expert_ffn",
-            "switch_combine", "switch_layer_fwd", "switch_check", "switch_status_string", "switch_launch_count",
+            "switch_combine", "switch_layer_fwd", "switch_check", "switch_selftest_wait_timeout", "switch_status_string",
+            "switch_launch_count",
             "switch_trace_start", "switch_trace_read", "switch_trace_stop", "switch_kernel_name")
 
 
@@ -82,6 +84,7 @@ def lib() -> ctypes.CDLL:
         "switch_combine": (I, [D, P, P, P, P, P, P]),
         "switch_layer_fwd": (I, [D, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
         "switch_check": (I, [P, S, P]),
+        "switch_selftest_wait_timeout": (I, [P, S, P]),
         "switch_status_string": (ctypes.c_char_p, [I]),
         "switch_launch_count": (ctypes.c_int64, []),
         "switch_trace_start": (I, [ctypes.c_int32]),
@@ -204,6 +207,13 @@ def switch_check(workspace, stream=None) -> int:
     """Synchronise and return the device status code (0 = ok); does not raise."""
     return int(lib().switch_check(_ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream, workspace)))
+
+
+def selftest_wait_timeout(workspace, stream=None) -> None:
+    """Launch the bounded-wait self-test; switch_check(workspace) afterwards
+    reports SWITCH_ERR_DEVICE_TIMEOUT (8)."""
+    _ok(lib().switch_selftest_wait_timeout(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                           _stream(stream, workspace)), "switch_selftest_wait_timeout")
 
 
 def launch_count() -> int:

@@ -25,7 +25,7 @@ size_t elem_size(const switch_dims_t &d) { return d.dtype == SWITCH_BF16 ? 2 : 4
 int64_t tiles_of(const switch_dims_t &d) { return (d.T + kTileT - 1) / kTileT; }
 
 struct Sections {
-    size_t status, ticket, hist, psum, tile_off, prob_total, w_split, slot_token, xbuf, ybuf, hidden, total;
+    size_t status, ticket, hist, psum, tile_off, prob_total, w_split, slot_token, xbuf, ybuf, hidden, done, total;
 };
 
 Sections layout(const switch_dims_t &d) {
@@ -48,6 +48,7 @@ Sections layout(const switch_dims_t &d) {
     s.xbuf = take(N * C * (size_t)d.d_model * elem_size(d));
     s.ybuf = take(N * C * (size_t)d.d_model * sizeof(float));
     s.hidden = take(N * C * (size_t)d.d_ff * elem_size(d));
+    s.done = take((N * ((C + 255) / 256) + 1) * sizeof(int32_t));  // + the fused FFN's tile claim counter
     s.total = off;
     return s;
 }
@@ -129,6 +130,19 @@ switch_status_t check_device() {
 
 switch_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SWITCH_OK : SWITCH_ERR_CUDA; }
 
+// One thread waits on an mbarrier whose phase never completes; the bounded
+// wait gives up and records the timeout (tag 99), then the block exits.
+__global__ void selftest_wait_kernel(DeviceStatus *status) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+        status->code = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, status, 99);
+}
+
 }  // namespace
 
 size_t workspace_bytes(const switch_dims_t &dims) { return layout(dims).total; }
@@ -150,6 +164,7 @@ Workspace carve_workspace(const switch_dims_t &dims, void *base) {
     w.xbuf = b + s.xbuf;
     w.ybuf = reinterpret_cast<float *>(b + s.ybuf);
     w.hidden = b + s.hidden;
+    w.done = reinterpret_cast<int32_t *>(b + s.done);
     w.tiles = tiles_of(dims);
     return w;
 }
@@ -282,7 +297,7 @@ switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const
         // route + scatter-dispatch (zeroing dropped rows of y), GEMM1, GEMM2 with
         // the gate and the token-order scatter fused into its epilogue
         err = launch_route(*dims, x, w_r, logit_bias, expert, gate, slot, counts, ws.slot_token, aux, ws, st,
-                           ws.xbuf, yf);
+                           ws.xbuf, yf, ws.done, (int64_t)dims->num_experts * ((dims->capacity + 255) / 256) + 1);
         if (err == cudaSuccess)
             err = launch_ffn_tc(*dims, ws.xbuf, w_in, w_out, counts, nullptr, ws.slot_token, gate, yf, ws, st);
     } else {
@@ -306,6 +321,20 @@ switch_status_t switch_check(void *workspace, size_t workspace_bytes_given, swit
     if (cudaMemsetAsync(workspace, 0, sizeof host, st) != cudaSuccess) return SWITCH_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return SWITCH_ERR_CUDA;
     return host.code == 0 ? SWITCH_OK : (switch_status_t)host.code;
+}
+
+switch_status_t switch_selftest_wait_timeout(void *workspace, size_t workspace_bytes_given, switch_stream_t stream) {
+    if (!workspace) return SWITCH_ERR_NULL;
+    if (!aligned16(workspace)) return SWITCH_ERR_ALIGN;
+    if (workspace_bytes_given < sizeof(DeviceStatus)) return SWITCH_ERR_WORKSPACE;
+    switch_status_t s = check_device();
+    if (s != SWITCH_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    launch_begin(K_SELFTEST_WAIT, st);
+    selftest_wait_kernel<<<1, 32, 0, st>>>(static_cast<DeviceStatus *>(workspace));
+    const cudaError_t err = cudaGetLastError();
+    launch_end(st);
+    return from_cuda(err);
 }
 
 const char *switch_status_string(switch_status_t status) {
@@ -383,6 +412,8 @@ const char *switch_kernel_name(int32_t id) {
         case K_ROUTER_STAGED: return "router_staged";
         case K_ROUTER_TC: return "router_tc";
         case K_ROUTER_SPLIT: return "router_weight_split";
+        case K_SELFTEST_WAIT: return "selftest_wait_timeout";
+        case K_FFN_TC_FUSED: return "ffn_tc_fused";
     }
     return "?";
 }

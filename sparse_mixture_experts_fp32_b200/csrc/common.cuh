@@ -37,6 +37,16 @@ __device__ __forceinline__ uint64_t global_ns() {
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// serialization attribute may start while its predecessor on the stream
+// still runs; it must execute pdl_wait() before touching any global memory
+// the predecessor writes or reads.  Without the attribute pdl_wait() returns
+// at once.  pdl_launch_dependents() lets the successor start its prologue.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // Shared-memory addresses, mbarriers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -215,6 +225,39 @@ __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bu
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
+// Cross-CTA dependency counters in global memory
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *p) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_add_gpu(int32_t *p, int32_t v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Order this thread's global accesses of the generic proxy with those of the
+// async proxy (TMA loads and stores).
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Wait (bounded, about kWaitLimitNs) until *p >= target; false on timeout.
+__device__ __forceinline__ bool wait_counter_geq(const int32_t *p, int32_t target, DeviceStatus *st, int32_t where) {
+    if (ld_acquire_gpu(p) >= target) return true;
+    const uint64_t start = global_ns();
+    while (ld_acquire_gpu(p) < target) {
+        __nanosleep(64);
+        if (global_ns() - start > kWaitLimitNs) {
+            report_status(st, SWITCH_ERR_DEVICE_TIMEOUT, where);
+            return false;
+        }
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------------
 // Thread-block clusters of two CTAs (a "pair") and the cta_group::2 forms.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -237,6 +280,39 @@ __device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
 // Arrive on an mbarrier given by a shared::cluster address (possibly another CTA's).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Phase wait with acquire at cluster scope: for barriers that another CTA of
+// the cluster arrives on after writing data the waiter then reads (or after
+// reading data the waiter then overwrites).  Bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, DeviceStatus *st, int32_t where) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t start = global_ns();
+    uint32_t spins = 0;
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if ((++spins & 255u) == 0u && global_ns() - start > kWaitLimitNs) {
+            report_status(st, SWITCH_ERR_DEVICE_TIMEOUT, where);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Store one 32-bit word to a shared::cluster address (another CTA's shared memory).
+__device__ __forceinline__ void st_cluster_s32(uint32_t cluster_addr, int32_t v) {
+    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 // TMA 3-D load into this CTA's shared memory whose completion (transaction

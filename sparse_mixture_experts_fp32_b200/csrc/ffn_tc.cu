@@ -426,6 +426,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int k_blocks = K / BK;
     constexpr uint32_t kTmemCols = 2 * BN;
 
+    if (warp == 1) {
+        if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], 1);
+            }
+            for (int a = 0; a < 2; ++a) {
+                mbar_init(&acc_full[a], 1);
+                mbar_init(&acc_empty[a], 2 * kEpilogueThreads);
+            }
+            mbar_init(drain, 1);
+            fence_barrier_init();
+        }
+        __syncwarp();
+        tmem_alloc_pair(tmem_holder, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised before anyone signals them
+    tc_fence_after();
+    pdl_wait();  // counts, the A operand and the epilogue's inputs come from earlier kernels
+    pdl_launch_dependents();
     if (warp == 0) {
         int kept_of[8];  // E <= 256: every count is loaded before the scan starts
 #pragma unroll
@@ -451,27 +474,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             running += __shfl_sync(0xffffffffu, incl, 31);
         }
         if (lane == 0) tile_start[E] = running;
-    } else if (warp == 1) {
-        if (lane == 0) {
-            for (int s = 0; s < STAGES; ++s) {
-                mbar_init(&full[s], 1);
-                mbar_init(&empty[s], 1);
-            }
-            for (int a = 0; a < 2; ++a) {
-                mbar_init(&acc_full[a], 1);
-                mbar_init(&acc_empty[a], 2 * kEpilogueThreads);
-            }
-            mbar_init(drain, 1);
-            fence_barrier_init();
-        }
-        __syncwarp();
-        tmem_alloc_pair(tmem_holder, kTmemCols);
-        tmem_relinquish_pair();
     }
-    tc_fence_before();
     __syncthreads();
-    cluster_sync();  // both CTAs' barriers are initialised before anyone signals them
-    tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int total_tiles = tile_start[E];
 
@@ -585,6 +589,308 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Both expert GEMMs in one persistent launch on SM pairs (256 x 256 tiles).
+// The tile list holds every GEMM1 tile (expert e, 256-row block m, H column
+// block n) and then every GEMM2 tile (e, m, y column block).  Pairs claim
+// tiles in list order from a per-call counter (the leader's producer thread
+// takes the next index and hands it, through a 4-deep queue in shared
+// memory, to its MMA thread, its epilogue warps and the peer CTA).  A GEMM2
+// tile reads the H rows of its row block, written by the n1 = F / 256 GEMM1
+// tiles of (e, m): each of the pair's 8 epilogue warps adds 1 to done[e, m]
+// once its H boxes have fully landed (TMA store completion, then a release
+// add), and both producers of the GEMM2 tile wait (bounded) for done[e, m]
+// = 8 * n1 before loading H.  Every GEMM1 tile is claimed before any GEMM2
+// tile, and only by a running pair whose earlier tiles are GEMM1 tiles too,
+// so each wait is on work that is already in progress: no assumption about
+// how many pairs are resident at once.  The tail of GEMM1 overlaps the start
+// of GEMM2, and the GEMM2 tiles, too few for one even wave on their own,
+// share the waves with GEMM1.
+// ---------------------------------------------------------------------------
+constexpr int kFusedBN = 256;
+constexpr int kTileQ = 4;                // tile-index queue depth
+constexpr int kTileConsumers = 1 + 1 + 8;  // leader MMA thread, peer producer, 8 epilogue warps
+
+template <int STAGES>
+struct FusedLayout {
+    using L = PairLayout<kFusedBN, STAGES>;
+    // PairLayout (ring, staging, barriers, start1[E+1]) + tile queue + start2[E+1]
+    static size_t bytes(int experts) {
+        return L::bytes(experts) + 2 * kTileQ * 8 + kTileQ * 4 + (size_t)(experts + 1) * 4;
+    }
+};
+
+template <int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    tc_ffn_fused_pair(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w1,
+                      const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w2,
+                      const __grid_constant__ CUtensorMap tm_hstore, float *__restrict__ y,
+                      const int32_t *__restrict__ counts, int E, int C, int d, int F,
+                      const int32_t *__restrict__ slot_token, const float *__restrict__ gate,
+                      int32_t *__restrict__ done, int MT, DeviceStatus *status) {
+    constexpr int BN = kFusedBN;
+    using L = PairLayout<BN, STAGES>;
+    constexpr int BMP = 2 * BM;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;
+    uint8_t *sB = sA + STAGES * L::a_bytes;
+    uint8_t *staging = base + L::ring;
+    uint64_t *full = reinterpret_cast<uint64_t *>(staging + L::staging);
+    uint64_t *empty = full + STAGES;
+    uint64_t *acc_full = empty + STAGES;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *drain = acc_empty + 2;
+    uint64_t *tq_full = drain + 1;          // [kTileQ] tile index written (both CTAs)
+    uint64_t *tq_empty = tq_full + kTileQ;  // [kTileQ] tile index read by all (leader's)
+    int32_t *tq = reinterpret_cast<int32_t *>(tq_empty + kTileQ);  // [kTileQ] tile index, -1 = no more
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tq + kTileQ);
+    int32_t *start1 = reinterpret_cast<int32_t *>(tmem_holder + 4);  // [E+1] GEMM1 tiles per expert
+    int32_t *start2 = start1 + (E + 1);                              // [E+1] GEMM2 tiles per expert
+    int32_t *ticket = done + (int64_t)E * MT;                        // tile claim counter of this call
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int n1 = (F + BN - 1) / BN, n2 = (d + BN - 1) / BN;
+    const int kb1 = d / BK, kb2 = F / BK;
+    const int32_t need = 8 * n1;  // arrivals on done[e, m] once H of the row block is complete
+    constexpr uint32_t kTmemCols = 2 * BN;
+
+    if (warp == 1) {
+        if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], 1);
+            }
+            for (int a = 0; a < 2; ++a) {
+                mbar_init(&acc_full[a], 1);
+                mbar_init(&acc_empty[a], 2 * kEpilogueThreads);
+            }
+            mbar_init(drain, 1);
+            for (int j = 0; j < kTileQ; ++j) {
+                mbar_init(&tq_full[j], 1);
+                mbar_init(&tq_empty[j], kTileConsumers);
+            }
+            fence_barrier_init();
+        }
+        __syncwarp();
+        tmem_alloc_pair(tmem_holder, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    tc_fence_after();
+    pdl_wait();
+    pdl_launch_dependents();
+    if (warp == 0) {
+        int kept_of[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = 32 * j + lane;
+            kept_of[j] = e < E ? min(counts[e], C) : 0;
+        }
+        int run1 = 0, run2 = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e0 = 32 * j;
+            if (e0 >= E) break;
+            const int e = e0 + lane;
+            const int mt = (kept_of[j] + BMP - 1) / BMP;
+            int i1 = mt * n1, i2 = mt * n2;
+            const int m1 = i1, m2 = i2;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int u1 = __shfl_up_sync(0xffffffffu, i1, off);
+                const int u2 = __shfl_up_sync(0xffffffffu, i2, off);
+                if (lane >= off) {
+                    i1 += u1;
+                    i2 += u2;
+                }
+            }
+            if (e < E) {
+                start1[e] = run1 + i1 - m1;
+                start2[e] = run2 + i2 - m2;
+            }
+            run1 += __shfl_sync(0xffffffffu, i1, 31);
+            run2 += __shfl_sync(0xffffffffu, i2, 31);
+        }
+        if (lane == 0) {
+            start1[E] = run1;
+            start2[E] = run2;
+        }
+    }
+    __syncthreads();
+    const uint32_t tmem_base = *tmem_holder;
+    const int total1 = start1[E];
+    const int total = total1 + start2[E];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tm_x);
+            prefetch_tmap(&tm_w1);
+            prefetch_tmap(&tm_h);
+            prefetch_tmap(&tm_w2);
+            uint32_t issued = 0, parity_of = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int it = 0; ok; ++it) {
+                const int j = it % kTileQ;
+                const uint32_t qph = (uint32_t)(it / kTileQ) & 1u;
+                int tile;
+                if (rank == 0) {  // claim the next tile and hand its index to everyone
+                    if (!mbar_wait_cluster(&tq_empty[j], qph ^ 1u, status, 48)) break;
+                    tile = atomicAdd(ticket, 1);
+                    if (tile >= total) tile = -1;
+                    tq[j] = tile;
+                    st_cluster_s32(map_to_rank(&tq[j], 1), tile);
+                    mbar_arrive(&tq_full[j]);
+                    mbar_arrive_cluster(map_to_rank(&tq_full[j], 1));
+                } else {
+                    if (!mbar_wait_cluster(&tq_full[j], qph, status, 49)) break;
+                    tile = tq[j];
+                    mbar_arrive_cluster(map_to_rank(&tq_empty[j], 0));
+                }
+                if (tile < 0) break;
+                const bool second = tile >= total1;
+                int e, m, n;
+                if (second) locate_tile(start2, E, n2, tile - total1, e, m, n);
+                else locate_tile(start1, E, n1, tile, e, m, n);
+                if (second) {
+                    if (!wait_counter_geq(done + e * MT + m, need, status, 47)) break;
+                    fence_proxy_async_global();  // H, written through the async proxy, before our TMA reads
+                }
+                const void *ta = second ? (const void *)&tm_h : (const void *)&tm_x;
+                const void *tb = second ? (const void *)&tm_w2 : (const void *)&tm_w1;
+                const int kbs = second ? kb2 : kb1;
+                for (int kb = 0; kb < kbs; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, status, 41)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * (L::a_bytes + L::b_bytes)));
+                    const uint32_t leader_full = map_to_rank(&full[stage], 0);
+                    tma_load_3d_pair(sA + stage * L::a_bytes, ta, leader_full, kb * BK, m * BMP + (int)rank * BM, e);
+                    tma_load_3d_pair(sB + stage * L::b_bytes, tb, leader_full, kb * BK, n * BN + (int)rank * (BN / 2),
+                                     e);
+                    issued |= 1u << stage;
+                    parity_of = (parity_of & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (rank == 0)
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued & (1u << s)) mbar_wait(&full[s], (parity_of >> s) & 1u, status, 46);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(BMP, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int it = 0;; ++it) {
+                const int j = it % kTileQ;
+                if (!mbar_wait(&tq_full[j], (uint32_t)(it / kTileQ) & 1u, status, 50)) break;
+                const int tile = tq[j];
+                mbar_arrive(&tq_empty[j]);
+                if (tile < 0) break;
+                const int kbs = tile >= total1 ? kb2 : kb1;
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, status, 42)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                bool ok = true;
+                for (int kb = 0; kb < kbs; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, status, 43)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t a_desc = smem_desc_sw128(sA + stage * L::a_bytes);
+                    const uint64_t b_desc = smem_desc_sw128(sB + stage * L::b_bytes);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        tc_mma_bf16_pair(d_tmem, a_desc + (uint64_t)(2 * k), b_desc + (uint64_t)(2 * k), idesc,
+                                         (kb | k) != 0 ? 1u : 0u);
+                    tc_commit_pair(smem_u32(&empty[stage]));
+                    tc_commit_pair(map_to_rank(&empty[stage], 1));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit_pair(smem_u32(&acc_full[acc]));
+                tc_commit_pair(map_to_rank(&acc_full[acc], 1));
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            tc_commit_pair(smem_u32(drain));
+            mbar_wait(drain, 0, status, 44);
+        }
+    } else {
+        const int quarter = warp & 3;
+        uint8_t *my_stage = staging + (warp - 2) * L::stage_bytes;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int it = 0;; ++it) {
+            const int j = it % kTileQ;
+            const uint32_t qph = (uint32_t)(it / kTileQ) & 1u;
+            const bool got = rank == 0 ? mbar_wait(&tq_full[j], qph, status, 51)
+                                       : mbar_wait_cluster(&tq_full[j], qph, status, 52);
+            if (!got) break;
+            const int tile = tq[j];
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(&tq_empty[j]);
+                else mbar_arrive_cluster(map_to_rank(&tq_empty[j], 0));
+            }
+            if (tile < 0) break;
+            const bool second = tile >= total1;
+            int e, m, n;
+            if (second) locate_tile(start2, E, n2, tile - total1, e, m, n);
+            else locate_tile(start1, E, n1, tile, e, m, n);
+            if (!mbar_wait(&acc_full[acc], acc_phase, status, 45)) break;
+            tc_fence_after();
+            const int row_base = m * BMP + (int)rank * BM + quarter * 32;
+            const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+            if (second)
+                epilogue_async<BN, kEpiGatedScatter>(t_row, e, row_base, min(counts[e], C), C, n, d, y, nullptr,
+                                                     slot_token, gate, my_stage);
+            else
+                epilogue_async<BN, kEpiHiddenRelu>(t_row, e, row_base, min(counts[e], C), C, n, F, nullptr,
+                                                   &tm_hstore, slot_token, gate, my_stage);
+            tc_fence_before();
+            mbar_arrive_cluster(map_to_rank(&acc_empty[acc], 0));
+            if (!second && lane == 0) {
+                bulk_wait_all();             // this warp's H boxes are in global memory
+                fence_proxy_async_global();  // ... ordered before the release below
+                red_release_add_gpu(done + e * MT + m, 1);
+            }
+            __syncwarp();
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    if (warp >= 2) bulk_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Host side: tensor maps and launches
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -653,8 +959,37 @@ cudaError_t launch_gemm_pair(int32_t kernel_id, const void *a, const void *b, vo
     const int64_t tiles = m_tiles * ((Nout + BN - 1) / BN);
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / 2, tiles));
     launch_begin(kernel_id, stream);
-    kern<<<2 * pairs, kThreads, smem, stream>>>(ta, tb, tout, out, counts, E, C, K, Nout, slot_token, gate, status);
-    err = cudaGetLastError();
+    err = launch_kernel(kern, dim3(2 * pairs), dim3(kThreads), smem, stream, true, ta, tb, tout, out, counts, E, C, K,
+                        Nout, slot_token, gate, status);
+    launch_end(stream);
+    return err;
+}
+
+template <int STAGES>
+cudaError_t launch_ffn_fused(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
+                             const int32_t *counts, const int32_t *slot_token, const float *gate, float *y,
+                             const Workspace &ws, bool zero_done, cudaStream_t stream) {
+    const int E = dims.num_experts, C = dims.capacity, d = dims.d_model, F = dims.d_ff;
+    const size_t smem = FusedLayout<STAGES>::bytes(E);
+    auto kern = tc_ffn_fused_pair<STAGES>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    CUtensorMap tx, tw1, th, tw2, ths;
+    if (!make_tmap(&tx, xbuf, E, C, d, BM) || !make_tmap(&tw1, w_in, E, F, d, kFusedBN / 2) ||
+        !make_tmap(&th, ws.hidden, E, C, F, BM) || !make_tmap(&tw2, w_out, E, d, F, kFusedBN / 2) ||
+        !make_tmap(&ths, ws.hidden, E, C, F, 32))
+        return cudaErrorInvalidValue;
+    const int MT = (C + 2 * BM - 1) / (2 * BM);
+    if (zero_done) {  // counters and the tile claim counter after them
+        err = cudaMemsetAsync(ws.done, 0, ((size_t)E * MT + 1) * sizeof(int32_t), stream);
+        if (err != cudaSuccess) return err;
+    }
+    const int64_t m_tiles = std::min<int64_t>((int64_t)E * MT, (dims.T + 2 * BM - 1) / (2 * BM) + E);
+    const int64_t tiles = m_tiles * (((F + kFusedBN - 1) / kFusedBN) + ((d + kFusedBN - 1) / kFusedBN));
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / 2, tiles));
+    launch_begin(K_FFN_TC_FUSED, stream);
+    err = launch_kernel(kern, dim3(2 * pairs), dim3(kThreads), smem, stream, !zero_done, tx, tw1, th, tw2, ths, y,
+                        counts, E, C, d, F, slot_token, gate, ws.done, MT, static_cast<DeviceStatus *>(ws.status));
     launch_end(stream);
     return err;
 }
@@ -666,6 +1001,11 @@ cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const voi
                           const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts, C = dims.capacity, d = dims.d_model, F = dims.d_ff;
     DeviceStatus *st = static_cast<DeviceStatus *>(ws.status);
+    if (y && !(dims.flags & (SWITCH_FLAG_GEMM_1CTA | SWITCH_FLAG_FFN_TWO_LAUNCHES))) {
+        // both GEMMs in one launch; the dependency counters were zeroed by the
+        // slot assignment of this call
+        return launch_ffn_fused<6>(dims, xbuf, w_in, w_out, counts, slot_token, gate, y, ws, false, stream);
+    }
     if (dims.flags & SWITCH_FLAG_GEMM_1CTA) {
         cudaError_t err = launch_gemm<256, 4, kEpiHiddenRelu>(K_FFN_TC_GEMM1, xbuf, w_in, ws.hidden, counts, N, C, d,
                                                               F, dims.T, nullptr, nullptr, st, stream);

@@ -30,6 +30,8 @@ enum KernelId : int32_t {
     K_ROUTER_STAGED = 13,
     K_ROUTER_TC = 14,
     K_ROUTER_SPLIT = 15,
+    K_SELFTEST_WAIT = 16,
+    K_FFN_TC_FUSED = 17,
 };
 
 struct Workspace {
@@ -44,6 +46,7 @@ struct Workspace {
     void *xbuf;          // [N][C][d] (layer_fwd only)
     float *ybuf;         // [N][C][d] float32 (layer_fwd only)
     void *hidden;        // [N][C][F] expert hidden activations
+    int32_t *done;       // [N][ceil(C/256)] GEMM1 completion counters of the fused FFN, then its tile counter
     int64_t tiles;
 };
 
@@ -64,12 +67,12 @@ void launch_end(cudaStream_t stream);
 cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
                          int32_t *expert, float *gate, int32_t *slot, int32_t *counts, int32_t *slot_token,
                          float *aux, const Workspace &ws, cudaStream_t stream, void *xbuf_scatter = nullptr,
-                         float *y_zero = nullptr);
+                         float *y_zero = nullptr, int32_t *done_zero = nullptr, int64_t n_done = 0);
 cudaError_t launch_dispatch(const switch_dims_t &dims, const void *x, const int32_t *slot_token,
                             const int32_t *counts, void *xbuf, cudaStream_t stream);
 cudaError_t launch_combine(const switch_dims_t &dims, const float *ybuf, const int32_t *expert,
                            const int32_t *slot, const float *gate, float *y, cudaStream_t stream);
-// Tensor-core router (bf16 x, 32 < N <= 128): writes expert, gate and the
+// Tensor-core router (bf16 x, N <= 128): writes expert, gate and the
 // per-tile counts / probability sums like the CUDA-core routers.
 bool router_tc_supported(const switch_dims_t &dims);
 cudaError_t launch_router_tc(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
@@ -85,5 +88,23 @@ cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const voi
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
+
+// Kernel launch; with `pdl` the kernel may begin while its predecessor on the
+// stream finishes (it must pdl_wait() before using the predecessor's data).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
+                          Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 }  // namespace switchmoe

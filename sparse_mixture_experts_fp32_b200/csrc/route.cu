@@ -252,24 +252,32 @@ __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restr
 
 // ---------------------------------------------------------------------------
 // Router for N <= 32 with the whole 64-token tile of x staged in shared
-// memory.  One bulk copy per row (rows padded by 64 bytes so that the reads
-// below are free of bank conflicts) completes on one of four mbarriers, one
-// per 16-token chunk, so the first warps start while later rows still land.
-// Four threads share a token: thread (token, part) accumulates all N partial
-// dot products over the 16-byte x vectors j = part, part + 4, ... against
-// W_r held as [d/V][V][NP] (+4 floats of padding per j).  Two shuffles then
-// give each of the four the token's full logits, so the softmax, argmax and
-// gate need no further exchange.  Sum of p over the tile: shuffles over the
-// warp's 8 tokens, then a fixed-order sum over the 8 warps (deterministic).
+// memory.  One bulk copy per 16-token chunk (the rows are contiguous) completes
+// on the chunk's mbarrier, so the first warps start while later rows still land;
+// W_r is loaded meanwhile as [d/V][V][NP] (+4 floats of padding per j).
+// A register-blocked skinny GEMM: thread (group, part) accumulates 4 tokens
+// x NP experts over the 16-byte x vectors j = part, part + 16, ..., so each
+// W_r value read from shared memory serves four tokens; four shuffles sum the
+// 16 parts.  Softmax, argmax and gate per token in registers; the tile's sum
+// of p is formed in fixed token order (deterministic).
 // ---------------------------------------------------------------------------
 template <typename XT>
 struct Staged {
     static constexpr int V = XLoad<XT>::V;
-    static __host__ __device__ int64_t xpitch(int d) { return (int64_t)d * sizeof(XT) + 64; }
+    static __host__ __device__ int64_t xpitch(int d) { return (int64_t)d * sizeof(XT); }
     static __host__ __device__ int64_t wpitch(int NP) { return (int64_t)V * NP + 4; }  // floats per 16-byte x vector of W_r
-    static size_t smem(int d, int NP) {
-        return (size_t)(kTileT * xpitch(d)) + (size_t)((d / V) * wpitch(NP)) * 4 + (size_t)(kWarps * NP) * 4 +
-               (size_t)NP * 4 + 4 * 8 + 16;
+    // The x tile region is reused for the per-token probabilities at the end.
+    static __host__ __device__ int64_t x_region(int d, int NP) {
+        const int64_t a = kTileT * xpitch(d), b = (int64_t)kTileT * NP * 4;
+        return ((a > b ? a : b) + 15) / 16 * 16;
+    }
+    // smem layout: x tile | W_r as [d/V][V][NP] | per-warp sums | counts | 5 mbarriers | raw W_r (optional)
+    static size_t smem_base(int d, int NP) {
+        return (size_t)x_region(d, NP) + (size_t)((d / V) * wpitch(NP)) * 4 + (size_t)(kWarps * NP) * 4 +
+               (size_t)NP * 4 + 5 * 8 + 16;
+    }
+    static size_t smem(int d, int NP, int N, bool raw) {
+        return smem_base(d, NP) + (raw ? (size_t)N * d * 4 + 16 : 0);
     }
 };
 
@@ -278,50 +286,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     router_staged_kernel(const XT *__restrict__ x, const float *__restrict__ w_r, const float *__restrict__ bias,
                          int64_t T, int d, int N, int tiles, int32_t *__restrict__ expert, float *__restrict__ gate,
                          int32_t *__restrict__ hist, float *__restrict__ psum, uint32_t *ticket,
-                         DeviceStatus *status) {
+                         DeviceStatus *status, int raw_w) {
     using S = Staged<XT>;
     constexpr int V = S::V;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int64_t xpitch = S::xpitch(d);
     const int64_t wpitch = S::wpitch(NP);
     unsigned char *xs = smem_raw;
-    float *wsm = reinterpret_cast<float *>(smem_raw + kTileT * xpitch);
+    float *wsm = reinterpret_cast<float *>(smem_raw + S::x_region(d, NP));
     float *psum_w = wsm + (d / V) * wpitch;
     int32_t *hist_s = reinterpret_cast<int32_t *>(psum_w + kWarps * NP);
     uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(hist_s + NP) + 15) & ~uintptr_t(15));
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float *w_raw = reinterpret_cast<float *>(bar + 5) + 2;  // 16-byte aligned: bar is, and 5 * 8 + 8 = 48
+    const int tid = threadIdx.x;
     const int tile = blockIdx.x;
     const int64_t t0 = (int64_t)tile * kTileT;
     const int n_tok = (int)(T - t0 < kTileT ? T - t0 : kTileT);
     const uint32_t row_bytes = (uint32_t)(d * sizeof(XT));
 
+    pdl_launch_dependents();
+    const uint32_t w_bytes = (uint32_t)(N * d * 4);
     if (tid == 0) {
         if (tile == 0) reset_call_state(ticket, status);
-        for (int c = 0; c < 4; ++c) mbar_init(&bar[c], 1);
+        for (int c = 0; c < 5; ++c) mbar_init(&bar[c], 1);
         fence_barrier_init();
         for (int c = 0; c < 4; ++c) {
             const int rows = max(0, min(16, n_tok - 16 * c));
             if (rows > 0) mbar_arrive_expect_tx(&bar[c], (uint32_t)rows * row_bytes);
         }
+        if (raw_w) mbar_arrive_expect_tx(&bar[4], w_bytes);
     }
     __syncthreads();  // barriers initialised before any copy signals them
-    if (tid < n_tok) bulk_load(xs + tid * xpitch, x + (t0 + tid) * d, row_bytes, &bar[tid >> 4]);
-    // W_r (row-major [N][d], read coalesced) -> [d/V][V][NP] with padding,
-    // while the rows of x are on their way.  Batches of 8 loads per thread
-    // are in flight before their stores.
-    for (int i0 = 0; i0 < NP * d; i0 += 8 * kThreads) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * kThreads + tid;
-            v[u] = (i < N * d) ? w_r[i] : 0.f;
+    if (tid < 4) {    // rows are contiguous: one bulk copy per 16-row chunk
+        const int rows = max(0, min(16, n_tok - 16 * tid));
+        if (rows > 0)
+            bulk_load(xs + 16 * tid * xpitch, x + (t0 + 16 * tid) * d, (uint32_t)rows * row_bytes, &bar[tid]);
+    } else if (tid == 4 && raw_w) {
+        bulk_load(w_raw, w_r, w_bytes, &bar[4]);  // W_r [N][d] as stored
+    }
+    // W_r -> [d/V][V][NP] with padding, while the rows of x are on their way
+    if (raw_w) {
+        mbar_wait(&bar[4], 0, status, 11);
+        for (int i = tid; i < NP * d; i += kThreads) {
+            const int e = i / d, k = i - e * d;
+            float v = 0.f;
+            if (e < N) v = w_raw[i];  // padding experts e >= N read nothing
+            wsm[(k / V) * wpitch + (k % V) * NP + e] = v;
         }
+    } else {
+        for (int k0 = 0; k0 < d; k0 += kThreads) {
+            const int k = k0 + tid;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * kThreads + tid;
-            if (i < NP * d) {
-                const int e = i / d, k = i % d;
-                wsm[(k / V) * wpitch + (k % V) * NP + e] = v[u];
+            for (int e0 = 0; e0 < NP; e0 += 8) {
+                float v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = (k < d && e0 + u < N) ? w_r[(int64_t)(e0 + u) * d + k] : 0.f;
+                if (k < d) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) wsm[(k / V) * wpitch + (k % V) * NP + e0 + u] = v[u];
+                }
             }
         }
     }
@@ -329,78 +352,106 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = tid; i < NP; i += kThreads) hist_s[i] = 0;
     __syncthreads();
 
-    const int tl = tid >> 2, part = tid & 3;
-    const bool valid = tl < n_tok;
-    float acc[NP];
+    // Thread (group g, part p): tokens 4g .. 4g+3 of the tile, 16-byte x
+    // vectors j = p, p + 16, ... of their rows; 4 x NP accumulators.  Each
+    // W_r value read from shared memory feeds four tokens.
+    constexpr int TM = 4, PARTS = 16;
+    const int part = tid & (PARTS - 1), group = tid / PARTS;  // 16 groups x 4 tokens = 64 tokens
+    float acc[TM][NP];
 #pragma unroll
-    for (int e = 0; e < NP; ++e) acc[e] = 0.f;
-    if (valid && mbar_wait(&bar[tl >> 4], 0, status, 10)) {
-        const unsigned char *xrow = xs + tl * xpitch;
-        for (int j = part; j < d / V; j += 4) {
-            float xv[V];
-            XLoad<XT>::vec_generic(reinterpret_cast<const XT *>(xrow + (int64_t)j * 16), xv);  // shared memory
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int e = 0; e < NP; ++e) acc[i][e] = 0.f;
+    const int tok0 = group * TM;
+    bool ready = tok0 < n_tok;
+    if (ready) ready = mbar_wait(&bar[tok0 >> 4], 0, status, 10);  // the 4 tokens share one 16-row chunk
+    if (ready) {
+        for (int j = part; j < d / V; j += PARTS) {
+            float xv[TM][V];
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+                XLoad<XT>::vec_generic(reinterpret_cast<const XT *>(xs + (tok0 + i) * xpitch + (int64_t)j * 16),
+                                       xv[i]);  // shared memory (rows past n_tok hold stale data, never used)
             const float *wj = wsm + j * wpitch;
 #pragma unroll
             for (int u = 0; u < V; ++u) {
 #pragma unroll
                 for (int q = 0; q < NP / 4; ++q) {
                     const float4 w4 = *reinterpret_cast<const float4 *>(wj + u * NP + 4 * q);
-                    acc[4 * q + 0] = fmaf(xv[u], w4.x, acc[4 * q + 0]);
-                    acc[4 * q + 1] = fmaf(xv[u], w4.y, acc[4 * q + 1]);
-                    acc[4 * q + 2] = fmaf(xv[u], w4.z, acc[4 * q + 2]);
-                    acc[4 * q + 3] = fmaf(xv[u], w4.w, acc[4 * q + 3]);
+#pragma unroll
+                    for (int i = 0; i < TM; ++i) {
+                        acc[i][4 * q + 0] = fmaf(xv[i][u], w4.x, acc[i][4 * q + 0]);
+                        acc[i][4 * q + 1] = fmaf(xv[i][u], w4.y, acc[i][4 * q + 1]);
+                        acc[i][4 * q + 2] = fmaf(xv[i][u], w4.z, acc[i][4 * q + 2]);
+                        acc[i][4 * q + 3] = fmaf(xv[i][u], w4.w, acc[i][4 * q + 3]);
+                    }
                 }
             }
         }
     }
+    // sum over the 16 parts (lanes of one half-warp): every lane of the group
+    // ends with the full logits of the group's 4 tokens
 #pragma unroll
-    for (int e = 0; e < NP; ++e) {
-        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 1);
-        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 2);
-    }
-    float m = -FLT_MAX;
-    int arg = 0;
+    for (int i = 0; i < TM; ++i)
 #pragma unroll
-    for (int e = 0; e < NP; ++e) {
-        if (e < N) {
-            acc[e] += bias ? bias[e] : 0.f;
-            if (acc[e] > m) {  // strict: the lowest index wins a tie
-                m = acc[e];
-                arg = e;
+        for (int e = 0; e < NP; ++e) {
+            acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], 1);
+            acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], 2);
+            acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], 4);
+            acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], 8);
+        }
+    // lanes with part < TM finish token tok0 + part
+    float *ptile = reinterpret_cast<float *>(xs);  // [64][NP] per-token p, reusing the x tile
+    __syncthreads();                               // every read of the x tile is done
+    if (part < TM) {
+        const int tl = tok0 + part;
+        const bool valid = tl < n_tok;
+        float h[NP];
+#pragma unroll
+        for (int e = 0; e < NP; ++e) {
+            float v = acc[0][e];
+#pragma unroll
+            for (int i = 1; i < TM; ++i) v = (part == i) ? acc[i][e] : v;
+            h[e] = v;
+        }
+        float m = -FLT_MAX;
+        int arg = 0;
+#pragma unroll
+        for (int e = 0; e < NP; ++e) {
+            if (e < N) {
+                h[e] += bias ? bias[e] : 0.f;
+                if (h[e] > m) {  // strict: the lowest index wins a tie
+                    m = h[e];
+                    arg = e;
+                }
             }
         }
-    }
-    float s = 0.f;
+        float s = 0.f;
 #pragma unroll
-    for (int e = 0; e < NP; ++e) {
-        acc[e] = e < N ? expf(acc[e] - m) : 0.f;
-        s += acc[e];
-    }
+        for (int e = 0; e < NP; ++e) {
+            h[e] = e < N ? expf(h[e] - m) : 0.f;
+            s += h[e];
+        }
 #pragma unroll
-    for (int e = 0; e < NP; ++e) acc[e] = valid ? acc[e] / s : 0.f;  // p_e
-    if (valid && part == 0) {
-        const int64_t t = t0 + tl;
-        expert[t] = arg;
-        gate[t] = 1.0f / s;  // p at the argmax: exp(0) / s
-        atomicAdd(&hist_s[arg], 1);
-    }
-#pragma unroll
-    for (int e = 0; e < NP; ++e) {
-        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 4);
-        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
-        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
-    }
-    if (lane == 0) {
-#pragma unroll
-        for (int e = 0; e < NP; ++e) psum_w[warp * NP + e] = acc[e];
+        for (int e = 0; e < NP; ++e) ptile[tl * NP + e] = valid ? h[e] / s : 0.f;  // p_e
+        if (valid) {
+            const int64_t t = t0 + tl;
+            expert[t] = arg;
+            gate[t] = 1.0f / s;  // p at the argmax: exp(0) / s
+            atomicAdd(&hist_s[arg], 1);
+        }
     }
     __syncthreads();
+    // tile sums of p: four interleaved partial sums, combined in fixed order (deterministic)
     for (int i = tid; i < N; i += kThreads) {
-        float p = 0.f;
+        float p4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int tl = 0; tl < kTileT; tl += 4) {
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) p += psum_w[w * NP + i];
+            for (int u = 0; u < 4; ++u) p4[u] += ptile[(tl + u) * NP + i];
+        }
         hist[(int64_t)i * tiles + tile] = hist_s[i];
-        psum[(int64_t)i * tiles + tile] = p;
+        psum[(int64_t)i * tiles + tile] = (p4[0] + p4[1]) + (p4[2] + p4[3]);
     }
 }
 
@@ -514,6 +565,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t *__res
     __shared__ int32_t warp_cnt[kScanThreads / 32];
     __shared__ double warp_p[kScanThreads / 32];
     __shared__ bool is_last;
+    pdl_wait();
+    pdl_launch_dependents();
     const int e = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int chunk = (tiles + kScanThreads - 1) / kScanThreads;
@@ -603,11 +656,14 @@ template <bool SCATTER>
 __global__ void __launch_bounds__(kAssignThreads) assign_kernel(
     const int32_t *__restrict__ expert, const int32_t *__restrict__ tile_off, const int32_t *__restrict__ counts,
     int64_t T, int N, int C, int tiles, int32_t *__restrict__ slot, int32_t *__restrict__ slot_token,
-    const uint4 *__restrict__ x, uint4 *__restrict__ xbuf, int x_words, float4 *__restrict__ y_zero, int y_words) {
+    const uint4 *__restrict__ x, uint4 *__restrict__ xbuf, int x_words, float4 *__restrict__ y_zero, int y_words,
+    int32_t *__restrict__ done_zero, int64_t n_done) {
     static_assert(kTileT == 64, "assignment assumes two ranking warps per tile");
     __shared__ int32_t first_warp_count[256];
     __shared__ int32_t tile_slot[kTileT];
     __shared__ int32_t tile_expert[kTileT];
+    pdl_wait();
+    pdl_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x;
     if (tile < tiles) {
@@ -686,6 +742,8 @@ __global__ void __launch_bounds__(kAssignThreads) assign_kernel(
             }
         }
     }
+    for (int64_t i = (int64_t)blockIdx.x * kAssignThreads + tid; i < n_done; i += (int64_t)gridDim.x * kAssignThreads)
+        done_zero[i] = 0;  // completion counters of the fused expert FFN that follows
     const int64_t total = (int64_t)N * C;
     for (int64_t i = (int64_t)blockIdx.x * kAssignThreads + tid; i < total; i += (int64_t)gridDim.x * kAssignThreads) {
         const int e = (int)(i / C);
@@ -711,18 +769,22 @@ cudaError_t launch_router_warp(const switch_dims_t &dims, const XT *x, const flo
     return err;
 }
 
+// Shared memory the staged router may use (x tile + W_r + partials).
+constexpr size_t kStagedSmemLimit = 200 * 1024;
+
 template <typename XT, int NP>
 cudaError_t launch_router_staged(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
                                  int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts, d = dims.d_model;
-    const size_t smem = Staged<XT>::smem(d, NP);
+    const bool raw = ((int64_t)N * d * 4) % 16 == 0 && Staged<XT>::smem(d, NP, N, true) <= kStagedSmemLimit;
+    const size_t smem = Staged<XT>::smem(d, NP, N, raw);
     auto kern = router_staged_kernel<XT, NP>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_STAGED, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
                                                          ws.hist, ws.psum, ws.ticket,
-                                                         static_cast<DeviceStatus *>(ws.status));
+                                                         static_cast<DeviceStatus *>(ws.status), raw ? 1 : 0);
     err = cudaGetLastError();
     launch_end(stream);
     return err;
@@ -748,16 +810,13 @@ cudaError_t launch_router_tiled(const switch_dims_t &dims, const XT *x, const fl
 
 // Largest d for which the warp router keeps W_r in shared memory.
 constexpr size_t kWarpRouterSmemLimit = 160 * 1024;
-// Shared memory the staged router may use (x tile + W_r + partials).
-constexpr size_t kStagedSmemLimit = 200 * 1024;
-
 template <typename XT>
 cudaError_t launch_router(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
                           int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts;
     const int NP = N <= 8 ? 8 : N <= 16 ? 16 : 32;
     const bool staged = N <= 32 && ((int64_t)dims.d_model * (int64_t)sizeof(XT)) % 16 == 0 &&
-                        Staged<XT>::smem(dims.d_model, NP) <= kStagedSmemLimit;
+                        Staged<XT>::smem(dims.d_model, NP, N, false) <= kStagedSmemLimit;
     if (staged) {
         if (NP == 8) return launch_router_staged<XT, 8>(dims, x, w_r, bias, expert, gate, ws, stream);
         if (NP == 16) return launch_router_staged<XT, 16>(dims, x, w_r, bias, expert, gate, ws, stream);
@@ -778,7 +837,8 @@ cudaError_t launch_router(const switch_dims_t &dims, const XT *x, const float *w
 
 cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
                          int32_t *expert, float *gate, int32_t *slot, int32_t *counts, int32_t *slot_token,
-                         float *aux, const Workspace &ws, cudaStream_t stream, void *xbuf_scatter, float *y_zero) {
+                         float *aux, const Workspace &ws, cudaStream_t stream, void *xbuf_scatter, float *y_zero,
+                         int32_t *done_zero, int64_t n_done) {
     cudaError_t err = cudaSuccess;
     const int N = dims.num_experts, C = dims.capacity;
     if (ws.tiles > 0 && router_tc_supported(dims)) {
@@ -797,9 +857,8 @@ cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *
         if (err != cudaSuccess) return err;
     }
     launch_begin(K_SCAN, stream);
-    scan_kernel<<<N, kScanThreads, 0, stream>>>(ws.hist, ws.psum, (int)ws.tiles, N, dims.T, ws.tile_off, counts,
-                                                ws.prob_total, aux, ws.ticket);
-    err = cudaGetLastError();
+    err = launch_kernel(scan_kernel, dim3(N), dim3(kScanThreads), 0, stream, ws.tiles > 0, ws.hist, ws.psum,
+                        (int)ws.tiles, N, dims.T, ws.tile_off, counts, ws.prob_total, aux, ws.ticket);
     launch_end(stream);
     if (err != cudaSuccess) return err;
     const int64_t fill_blocks = ((int64_t)N * C + kAssignThreads * 4 - 1) / (kAssignThreads * 4);
@@ -807,17 +866,16 @@ cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *
     const int x_words = (int)((int64_t)dims.d_model * (dims.dtype == SWITCH_BF16 ? 2 : 4) / 16);
     if (xbuf_scatter) {
         launch_begin(K_ASSIGN_SCATTER, stream);
-        assign_kernel<true><<<(unsigned)grid, kAssignThreads, 0, stream>>>(
-            expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token,
-            static_cast<const uint4 *>(x), static_cast<uint4 *>(xbuf_scatter), x_words,
-            reinterpret_cast<float4 *>(y_zero), dims.d_model / 4);
+        err = launch_kernel(assign_kernel<true>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true, expert,
+                            ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token,
+                            static_cast<const uint4 *>(x), static_cast<uint4 *>(xbuf_scatter), x_words,
+                            reinterpret_cast<float4 *>(y_zero), dims.d_model / 4, done_zero, n_done);
     } else {
         launch_begin(K_ASSIGN, stream);
-        assign_kernel<false><<<(unsigned)grid, kAssignThreads, 0, stream>>>(
-            expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token, nullptr, nullptr, 0,
-            nullptr, 0);
+        err = launch_kernel(assign_kernel<false>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
+                            expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token,
+                            (const uint4 *)nullptr, (uint4 *)nullptr, 0, (float4 *)nullptr, 0, done_zero, n_done);
     }
-    err = cudaGetLastError();
     launch_end(stream);
     return err;
 }

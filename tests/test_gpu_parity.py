@@ -74,6 +74,35 @@ def test_layer_small_simt_ffn(orc, name, T):
     full_check(orc, synth.WORKLOADS[name], T, flags=sm.SWITCH_FLAG_SIMT_FFN)
 
 
+@pytest.mark.parametrize("name,T", [("base8", 1000), ("base128_skew", 3000), ("large128", 700)])
+def test_layer_small_simt_router(orc, name, T):
+    # the CUDA-core routers (staged for N <= 32, tiled above) instead of the tensor-core one
+    full_check(orc, synth.WORKLOADS[name], T, flags=sm.SWITCH_FLAG_SIMT_ROUTER)
+
+
+@pytest.mark.parametrize("name,T", [("base8", 3000), ("large128", 2500), ("bigexpert64", 400)])
+def test_fused_ffn_matches_two_launches(name, T):
+    """One persistent launch for both expert GEMMs gives the same bytes as two launches."""
+    wl = synth.WORKLOADS[name]
+    C = synth_capacity(wl, T)
+    inp = synth.inputs(wl, T=T, experts=range(min(wl.num_experts, 16)))
+    dev = {k: to_device(v) for k, v in inp.items()}
+    a = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, logit_bias=dev["bias"])
+    b = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, logit_bias=dev["bias"],
+                     flags=sm.SWITCH_FLAG_FFN_TWO_LAUNCHES)
+    assert sm.switch_check(a["workspace"]) == 0 and sm.switch_check(b["workspace"]) == 0
+    assert torch.equal(a["y"].view(torch.int32), b["y"].view(torch.int32))
+
+
+def test_layer_small_two_launches(orc):
+    full_check(orc, synth.WORKLOADS["base8"], 1000, flags=sm.SWITCH_FLAG_FFN_TWO_LAUNCHES)
+
+
+def test_layer_small_gemm_1cta(orc):
+    # the one-SM (cta_group::1) expert GEMMs instead of the SM-pair ones
+    full_check(orc, synth.WORKLOADS["large128"], 900, flags=sm.SWITCH_FLAG_GEMM_1CTA)
+
+
 def test_route_entry_point_slot_token(orc):
     wl = synth.WORKLOADS["base128_skew"]
     T = 5000
@@ -290,8 +319,7 @@ def test_tracer_and_launch_counter():
     trace = sm.trace_read()
     sm.trace_stop()
     names = [n for n, _ in trace]
-    assert names == ["router_staged", "capacity_scan", "slot_assign_scatter", "ffn_tc_gemm1_relu",
-                     "ffn_tc_gemm2_gated_scatter"]
+    assert names == ["router_staged", "capacity_scan", "slot_assign_scatter", "ffn_tc_fused"]
     assert all(ms >= 0 for _, ms in trace)
     assert sm.launch_count() - before == len(names)
     assert sm.switch_check(out["workspace"]) == 0
