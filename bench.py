@@ -455,21 +455,38 @@ def run_e2e(args, sm, wl, inp, C, device, world):
 
 
 def traffic_from_profiles(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if it is current."""
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's
+    sources are unchanged since the counters were taken."""
+    want = source_sha(kernel)
     for p in sorted((ROOT / "profiles").glob("*.md")):
         text = p.read_text()
         m = re.search(rf"^\s*traffic\[{re.escape(kernel)}@{re.escape(workload)}\]:\s*([0-9.eE+]+)\s+bytes"
                       rf"\s+source_sha=(\w+)", text, flags=re.M)
-        if m and m.group(2) == source_sha():
+        if m and m.group(2) == want:
             return float(m.group(1))
     return None
 
 
-def source_sha() -> str:
+# The source file of each traced kernel; its hash, with the shared headers,
+# identifies the kernel as built.
+KERNEL_SOURCE = {
+    "router_warp": "route.cu", "router_tiled": "route.cu", "router_staged": "route.cu",
+    "capacity_scan": "route.cu", "slot_assign": "route.cu", "slot_assign_scatter": "route.cu",
+    "router_weight_split": "router_tc.cu", "router_tc": "router_tc.cu",
+    "dispatch": "move.cu", "combine": "move.cu",
+}
+
+
+def source_sha(kernel: str) -> str:
     import hashlib
+    csrc = ROOT / "sparse_mixture_experts_fp32_b200" / "csrc"
+    src = KERNEL_SOURCE.get(kernel)
+    if src is None and kernel.startswith(("ffn_tc", "ffn_simt")):
+        src = "ffn_tc.cu" if kernel.startswith("ffn_tc") else "ffn_simt.cu"
+    files = ["common.cuh", "internal.h"] + ([src] if src else sorted(p.name for p in csrc.glob("*.cu")))
     h = hashlib.sha1()
-    for f in sorted((ROOT / "sparse_mixture_experts_fp32_b200" / "csrc").glob("*")):
-        h.update(f.read_bytes())
+    for f in files:
+        h.update((csrc / f).read_bytes())
     return h.hexdigest()[:12]
 
 
