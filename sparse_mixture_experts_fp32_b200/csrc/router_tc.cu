@@ -11,15 +11,25 @@
 // tensor memory: every product is exact, only the order of the float32
 // additions differs from a CUDA-core dot product.
 //
-// Tile = 128 tokens (MMA M) x BN experts (MMA N, the experts padded to 32, 64
-// or 128; padding rows of W_r are zero-filled by TMA and ignored).  One CTA per
-// SM, persistent over token tiles:
-//   warp 0     TMA: 128 x 64 tile of x and the three 64-wide slices of W_r
-//   warp 1     TMEM allocation; one lane issues the MMAs
-//   warps 2-5  epilogue, one thread per token: tcgen05.ld of its row, max
-//              and argmax (lowest index on ties), sum of exp, gate = 1/sum,
-//              p_i; per-64-token-tile expert counts and sums of p_i
-//              (deterministic: a fixed shuffle tree, then a fixed warp order)
+// Tile = 256 tokens (MMA M, a pair of CTAs on two SMs with
+// tcgen05.mma.cta_group::2, 128 tokens each) x BN experts (MMA N, the experts
+// padded to 64 or 128; padding rows of W_r are zero-filled by TMA and
+// ignored).  Each CTA loads its own 128 rows of x and half of the BN rows of
+// every W_r term, so a token tile costs each SM half the W_r traffic of a
+// one-SM tile.  Persistent over token tiles, one CTA per SM:
+//   warp 0     TMA: 128 x 64 slice of x and the three 64-wide half-slices
+//              of W_r, counted on the leader's (rank 0) barrier
+//   warp 1     TMEM allocation; one lane of the leader issues the MMAs
+//   warps 2-9  epilogue of the CTA's 128 tokens, two warps per token: each
+//              reads half of the token's logits from TMEM (warp w may only
+//              reach TMEM lanes 32 (w % 4) .. +31, so warps w and w + 4 share
+//              a lane quarter and split the columns); max and argmax (lowest
+//              index on ties), sum of exp and the two halves combined through
+//              shared memory; gate = 1/sum, p_i; per-64-token-tile expert
+//              counts and sums of p_i (deterministic: a fixed shuffle tree,
+//              then a fixed warp order).  Two warps per SM sub-partition hide
+//              the latency of this per-token chain.
+// Barrier addresses of the other CTA come from mapa; nothing is multicast.
 #include <cuda.h>
 
 #include <algorithm>
@@ -31,10 +41,11 @@
 namespace switchmoe {
 namespace {
 
-constexpr int RM = 128;  // tokens per tile
+constexpr int RM = 128;  // tokens per CTA (a pair tile is 2 * RM)
 constexpr int RK = 64;   // K per ring stage (one 128-byte swizzle row of bf16)
 constexpr int kTerms = 3;
-constexpr int kThreads = 192;
+constexpr int kEpiThreads = 256;             // warps 2-9
+constexpr int kThreads = 64 + kEpiThreads;
 
 // W_r float32 [N][d] -> three bfloat16 terms [3][N][d].
 __global__ void split_router_weight(const float *__restrict__ w, __nv_bfloat16 *__restrict__ out, int64_t n) {
@@ -54,11 +65,13 @@ __global__ void split_router_weight(const float *__restrict__ w, __nv_bfloat16 *
 template <int BN, int STAGES>
 struct RouterLayout {
     static constexpr size_t a_bytes = (size_t)RM * RK * 2;
-    static constexpr size_t b_term_bytes = (size_t)BN * RK * 2;
+    static constexpr size_t b_term_bytes = (size_t)(BN / 2) * RK * 2;  // this CTA's half of the experts
     static constexpr size_t b_bytes = kTerms * b_term_bytes;
     static constexpr size_t ring = STAGES * (a_bytes + b_bytes);
     static constexpr size_t barriers = (2 * STAGES + 2 + 2 + 1) * 8 + 16;
-    static constexpr size_t epi = (size_t)BN * 4 /*bias*/ + 4 * BN * 4 /*psum per warp*/ + 2 * BN * 4 /*counts*/;
+    // bias, per-quarter sums of p and per-64-token counts (both double-buffered by tile parity),
+    // and the exchange of per-half max, argmax and sum between the two warps of a token
+    static constexpr size_t epi = (size_t)BN * 4 + 2 * 4 * BN * 4 + 2 * 2 * BN * 4 + 3 * 2 * RM * 4;
     static constexpr size_t bytes = 1024 + ring + barriers + epi;
 };
 
@@ -82,23 +95,27 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32]) {
     return v[0];
 }
 
-__device__ __forceinline__ void named_barrier_epilogue() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void named_barrier_epilogue() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-__device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, uint64_t *bar, int32_t c0, int32_t c1) {
+// 2-D TMA load into this CTA's shared memory, counted on the mbarrier at
+// `bar_cluster_addr` (the leader's).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const void *tmap, uint32_t bar_cluster_addr,
+                                                 int32_t c0, int32_t c1) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster_addr), "r"(c0), "r"(c1)
         : "memory");
 }
 
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const float *__restrict__ bias, int64_t T, int d, int N, int tiles64,
                      int32_t *__restrict__ expert, float *__restrict__ gate, int32_t *__restrict__ hist,
                      float *__restrict__ psum, uint32_t *ticket, DeviceStatus *status) {
     using L = RouterLayout<BN, STAGES>;
+    constexpr int PM = 2 * RM;  // tokens per pair tile
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
@@ -110,16 +127,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *drain = acc_empty + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     float *bias_s = reinterpret_cast<float *>(tmem_holder + 4);
-    float *psum_w = bias_s + BN;                                  // [4][BN]
-    int32_t *hist_s = reinterpret_cast<int32_t *>(psum_w + 4 * BN);  // [2][BN]
+    float *psum_w = bias_s + BN;                                     // [2 parity][4 quarters][BN]
+    int32_t *hist_s = reinterpret_cast<int32_t *>(psum_w + 8 * BN);  // [2 parity][2 halves][BN]
+    float *x_max = reinterpret_cast<float *>(hist_s + 4 * BN);       // [2 column halves][RM]
+    int32_t *x_arg = reinterpret_cast<int32_t *>(x_max + 2 * RM);    // [2][RM]
+    float *x_sum = reinterpret_cast<float *>(x_arg + 2 * RM);        // [2][RM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m_tiles = (int)((T + RM - 1) / RM);
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    const int m_tiles = (int)((T + PM - 1) / PM);
     const int k_blocks = (d + RK - 1) / RK;
     constexpr uint32_t kTmemCols = 2 * BN;
 
-    pdl_wait();  // the split terms of W_r come from the previous kernel
-    pdl_launch_dependents();
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *ticket = 0u;
         status->code = 0;
@@ -135,22 +155,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int a = 0; a < 2; ++a) {
                 mbar_init(&acc_full[a], 1);
-                mbar_init(&acc_empty[a], 128);
+                mbar_init(&acc_empty[a], 2 * kEpiThreads);
             }
             mbar_init(drain, 1);
             fence_barrier_init();
         }
         __syncwarp();
-        tmem_alloc(tmem_holder, kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_holder, kTmemCols);
+        tmem_relinquish_pair();
     } else if (warp >= 2) {
         const int et = threadIdx.x - 64;
-        for (int i = et; i < BN; i += 128) bias_s[i] = (bias && i < N) ? bias[i] : 0.f;
-        for (int i = et; i < 2 * BN; i += 128) hist_s[i] = 0;
+        for (int i = et; i < BN; i += kEpiThreads) bias_s[i] = (bias && i < N) ? bias[i] : 0.f;
+        for (int i = et; i < 4 * BN; i += kEpiThreads) hist_s[i] = 0;
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised before anyone signals them
     tc_fence_after();
+    pdl_wait();  // the split terms of W_r come from the previous kernel
+    pdl_launch_dependents();
     const uint32_t tmem_base = *tmem_holder;
 
     if (warp == 0) {
@@ -161,22 +184,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < m_tiles; tile += gridDim.x) {
-                // x streams from HBM: pull this CTA's next token tile into L2 now
-                const int next = tile + (int)gridDim.x;
+            const int my_rows = (int)rank * RM;
+            for (int tile = pair; ok && tile < m_tiles; tile += n_pairs) {
+                // x streams from HBM: pull this CTA's rows of the pair's next tile into L2 now
+                const int next = tile + n_pairs;
                 if (next < m_tiles)
-                    for (int kb = 0; kb < k_blocks; ++kb) tma_prefetch_l2_2d(&tmap_x, kb * RK, next * RM);
+                    for (int kb = 0; kb < k_blocks; ++kb) tma_prefetch_l2_2d(&tmap_x, kb * RK, next * PM + my_rows);
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, status, 31)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(L::a_bytes + L::b_bytes));
-                    tma_load_2d(sA + stage * L::a_bytes, &tmap_x, &full[stage], kb * RK, tile * RM);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * (L::a_bytes + L::b_bytes)));
+                    const uint32_t leader_full = map_to_rank(&full[stage], 0);
+                    tma_load_2d_pair(sA + stage * L::a_bytes, &tmap_x, leader_full, kb * RK, tile * PM + my_rows);
 #pragma unroll
                     for (int term = 0; term < kTerms; ++term)
-                        tma_load_3d(sB + stage * L::b_bytes + term * L::b_term_bytes, &tmap_w, &full[stage], kb * RK,
-                                    0, term);
+                        tma_load_3d_pair(sB + stage * L::b_bytes + term * L::b_term_bytes, &tmap_w, leader_full,
+                                         kb * RK, (int)rank * (BN / 2), term);
                     issued |= 1u << stage;
                     parity_of = (parity_of & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -185,18 +210,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            for (int s = 0; s < STAGES; ++s)
-                if (issued & (1u << s)) mbar_wait(&full[s], (parity_of >> s) & 1u, status, 36);
+            if (rank == 0)
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued & (1u << s)) mbar_wait(&full[s], (parity_of >> s) & 1u, status, 36);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(RM, BN);
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(PM, BN);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < m_tiles; tile += gridDim.x) {
+            for (int tile = pair; ok && tile < m_tiles; tile += n_pairs) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, status, 32)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -213,91 +239,112 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int term = 0; term < kTerms; ++term) {
                             const uint64_t b_desc =
                                 smem_desc_sw128(sB + stage * L::b_bytes + term * L::b_term_bytes);
-                            tc_mma_bf16(d_tmem, a_desc + (uint64_t)(2 * k), b_desc + (uint64_t)(2 * k), idesc,
-                                        (kb | k | term) != 0 ? 1u : 0u);
+                            tc_mma_bf16_pair(d_tmem, a_desc + (uint64_t)(2 * k), b_desc + (uint64_t)(2 * k), idesc,
+                                             (kb | k | term) != 0 ? 1u : 0u);
                         }
                     }
-                    tc_commit(&empty[stage]);
+                    tc_commit_pair(smem_u32(&empty[stage]));
+                    tc_commit_pair(map_to_rank(&empty[stage], 1));
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit(&acc_full[acc]);
+                tc_commit_pair(smem_u32(&acc_full[acc]));
+                tc_commit_pair(map_to_rank(&acc_full[acc], 1));
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
                 }
             }
-            tc_commit(drain);
+            tc_commit_pair(smem_u32(drain));
             mbar_wait(drain, 0, status, 34);
         }
     } else {
-        const int q = warp & 3;  // TMEM lane quarter: tokens 32q .. 32q+31 of the tile
+        constexpr int CW = BN / 2;           // columns per warp
+        const int q = warp & 3;              // TMEM lane quarter: tokens 32q .. 32q+31 of this CTA's rows
+        const int half = (warp - 2) >> 2;    // which half of the columns
+        const int col0 = half * CW;
+        const int tok = q * 32 + lane;       // token within this CTA's 128 rows
         const int et = threadIdx.x - 64;
+        const uint32_t acc_empty_leader0 = map_to_rank(&acc_empty[0], 0);
+        const uint32_t acc_empty_leader1 = map_to_rank(&acc_empty[1], 0);
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < m_tiles; tile += gridDim.x) {
+        int par = 0;
+        for (int tile = pair; tile < m_tiles; tile += n_pairs) {
             if (!mbar_wait(&acc_full[acc], acc_phase, status, 35)) break;
             tc_fence_after();
-            const int64_t t = (int64_t)tile * RM + q * 32 + lane;
+            const int64_t row0 = (int64_t)tile * PM + (int64_t)rank * RM;  // this CTA's first token
+            const int64_t t = row0 + tok;
             const bool valid = t < T;
-            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            // the whole row of BN logits in registers: one pass over TMEM
-            float h[BN];
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + col0);
+            float h[CW];
 #pragma unroll
-            for (int c = 0; c < BN; c += 32) {
+            for (int c = 0; c < CW; c += 32) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) h[c + j] = __uint_as_float(r[j]) + bias_s[c + j];
+                for (int j = 0; j < 32; ++j) h[c + j] = __uint_as_float(r[j]) + bias_s[col0 + c + j];
             }
+            tc_fence_before();
+            mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);  // columns in registers: reusable
             float m = -FLT_MAX;
-            int arg = 0;
+            int arg = col0;
 #pragma unroll
-            for (int j = 0; j < BN; ++j) {
-                if (j < N && h[j] > m) {  // strict: the lowest index wins a tie
+            for (int j = 0; j < CW; ++j) {
+                if (col0 + j < N && h[j] > m) {  // strict: the lowest index wins a tie
                     m = h[j];
-                    arg = j;
+                    arg = col0 + j;
                 }
             }
-            float s = 0.f;
+            x_max[half * RM + tok] = m;
+            x_arg[half * RM + tok] = arg;
+            named_barrier_epilogue();
+            const float m_lo = x_max[tok], m_hi = x_max[RM + tok];
+            const float mx = m_hi > m_lo ? m_hi : m_lo;  // ties keep the lower half: lowest index
+            const int amax = m_hi > m_lo ? x_arg[RM + tok] : x_arg[tok];
+            float s_part = 0.f;
 #pragma unroll
-            for (int j = 0; j < BN; ++j) {
-                h[j] = j < N ? expf(h[j] - m) : 0.f;
-                s += h[j];
+            for (int j = 0; j < CW; ++j) {
+                h[j] = col0 + j < N ? expf(h[j] - mx) : 0.f;
+                s_part += h[j];
             }
-            const float inv_s = 1.0f / s;
+            x_sum[half * RM + tok] = s_part;
+            named_barrier_epilogue();
+            const float inv_s = 1.0f / (x_sum[tok] + x_sum[RM + tok]);
+            float *psum_p = psum_w + par * 4 * BN;
+            int32_t *hist_p = hist_s + par * 2 * BN;
 #pragma unroll
-            for (int c = 0; c < BN; c += 32) {
+            for (int c = 0; c < CW; c += 32) {
                 float p[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) p[j] = valid ? h[c + j] * inv_s : 0.f;
-                const float col_sum = reduce_scatter32(p);  // this warp's 32 tokens, column c + lane
-                psum_w[q * BN + c + lane] = col_sum;
+                const float col_sum = reduce_scatter32(p);  // this warp's 32 tokens, column col0 + c + lane
+                psum_p[q * BN + col0 + c + lane] = col_sum;
             }
-            tc_fence_before();
-            mbar_arrive(&acc_empty[acc]);  // the accumulator may be reused now
-            if (valid) {
-                expert[t] = arg;
+            if (valid && half == 0) {
+                expert[t] = amax;
                 gate[t] = inv_s;  // p at the argmax: exp(0) / s
-                atomicAdd(&hist_s[(q >> 1) * BN + arg], 1);
+                atomicAdd(&hist_p[(q >> 1) * BN + amax], 1);
             }
             named_barrier_epilogue();
-            for (int i = et; i < N; i += 128) {
+            // the buffers of this parity are next written two tiles later, after two more barriers
+            const int t64_0 = (int)(row0 / 64);
+            for (int i = et; i < N; i += kEpiThreads) {
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int t64 = 2 * tile + half;
+                for (int h64 = 0; h64 < 2; ++h64) {
+                    const int t64 = t64_0 + h64;
                     if (t64 < tiles64) {
-                        hist[(int64_t)i * tiles64 + t64] = hist_s[half * BN + i];
-                        psum[(int64_t)i * tiles64 + t64] = psum_w[(2 * half) * BN + i] + psum_w[(2 * half + 1) * BN + i];
+                        hist[(int64_t)i * tiles64 + t64] = hist_p[h64 * BN + i];
+                        psum[(int64_t)i * tiles64 + t64] = psum_p[(2 * h64) * BN + i] + psum_p[(2 * h64 + 1) * BN + i];
                     }
-                    hist_s[half * BN + i] = 0;
+                    hist_p[h64 * BN + i] = 0;
                 }
             }
-            named_barrier_epilogue();
+            par ^= 1;
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
@@ -307,9 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 }
 
@@ -350,7 +398,7 @@ cudaError_t launch_bn(const switch_dims_t &dims, const __nv_bfloat16 *x, const f
     {
         const cuuint64_t gdim[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)kTerms};
         const cuuint64_t gstr[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
-        const cuuint32_t box[3] = {(cuuint32_t)RK, (cuuint32_t)BN, 1};
+        const cuuint32_t box[3] = {(cuuint32_t)RK, (cuuint32_t)(BN / 2), 1};
         if (fn(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ws.w_split, gdim, gstr, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -360,10 +408,10 @@ cudaError_t launch_bn(const switch_dims_t &dims, const __nv_bfloat16 *x, const f
     const size_t smem = RouterLayout<BN, STAGES>::bytes;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    const int64_t m_tiles = (T + RM - 1) / RM;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count(), m_tiles));
+    const int64_t m_tiles = (T + 2 * RM - 1) / (2 * RM);
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / 2, m_tiles));
     launch_begin(K_ROUTER_TC, stream);
-    err = launch_kernel(kern, dim3(grid), dim3(kThreads), smem, stream, true, tx, tw, bias, T, d, N, (int)ws.tiles,
+    err = launch_kernel(kern, dim3(2 * pairs), dim3(kThreads), smem, stream, true, tx, tw, bias, T, d, N, (int)ws.tiles,
                         expert, gate, ws.hist, ws.psum, ws.ticket, static_cast<DeviceStatus *>(ws.status));
     launch_end(stream);
     return err;
@@ -388,9 +436,8 @@ cudaError_t launch_router_tc(const switch_dims_t &dims, const void *x, const flo
     launch_end(stream);
     if (err != cudaSuccess) return err;
     const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
-    if (dims.num_experts <= 32) return launch_bn<32, 6>(dims, xb, bias, expert, gate, ws, stream);
-    if (dims.num_experts <= 64) return launch_bn<64, 4>(dims, xb, bias, expert, gate, ws, stream);
-    return launch_bn<128, 3>(dims, xb, bias, expert, gate, ws, stream);
+    if (dims.num_experts <= 64) return launch_bn<64, 7>(dims, xb, bias, expert, gate, ws, stream);
+    return launch_bn<128, 5>(dims, xb, bias, expert, gate, ws, stream);
 }
 
 }  // namespace switchmoe
