@@ -12,13 +12,18 @@
 // additions differs from a CUDA-core dot product.
 //
 // Tile = 256 tokens (MMA M, a pair of CTAs on two SMs with
-// tcgen05.mma.cta_group::2, 128 tokens each) x BN experts (MMA N, the experts
-// padded to 64 or 128; padding rows of W_r are zero-filled by TMA and
-// ignored).  Each CTA loads its own 128 rows of x and half of the BN rows of
-// every W_r term, so a token tile costs each SM half the W_r traffic of a
-// one-SM tile.  Persistent over token tiles, one CTA per SM:
-//   warp 0     TMA: 128 x 64 slice of x and the three 64-wide half-slices
-//              of W_r, counted on the leader's (rank 0) barrier
+// tcgen05.mma.cta_group::2, 128 tokens each) x BN experts (the experts padded
+// to 64 or 128; padding rows of W_r are zero-filled by TMA and ignored).  Per
+// 16-wide K step two MMAs: one with N = 2 BN against hi and mid stacked (the
+// leader's shared memory holds the hi rows, the peer's the mid rows), which
+// writes x . hi to accumulator columns [0, BN) and x . mid to [BN, 2 BN), and
+// one with N = BN against lo (each CTA holds half of its rows), added into
+// columns [0, BN).  The epilogue adds the two column blocks.  Two MMAs
+// instead of three: on B200 a pair MMA with N = 128 took about as long as one
+// with N = 256.  Persistent over token tiles, one CTA per SM:
+//   warp 0     TMA: 128 x 64 slice of x, this CTA's term of the stacked
+//              operand and half of lo, counted on the leader's (rank 0)
+//              barrier
 //   warp 1     TMEM allocation; one lane of the leader issues the MMAs
 //   warps 2-9  epilogue of the CTA's 128 tokens, two warps per token: each
 //              reads half of the token's logits from TMEM (warp w may only
@@ -65,8 +70,10 @@ __global__ void split_router_weight(const float *__restrict__ w, __nv_bfloat16 *
 template <int BN, int STAGES>
 struct RouterLayout {
     static constexpr size_t a_bytes = (size_t)RM * RK * 2;
-    static constexpr size_t b_term_bytes = (size_t)(BN / 2) * RK * 2;  // this CTA's half of the experts
-    static constexpr size_t b_bytes = kTerms * b_term_bytes;
+    static constexpr size_t b_half_bytes = (size_t)(BN / 2) * RK * 2;  // BN/2 rows of one term
+    // this CTA's rows: all BN rows of its stacked term (hi or mid), then BN/2 rows of lo
+    static constexpr size_t b_stack_bytes = 2 * b_half_bytes;
+    static constexpr size_t b_bytes = kTerms * b_half_bytes;
     static constexpr size_t ring = STAGES * (a_bytes + b_bytes);
     static constexpr size_t barriers = (2 * STAGES + 2 + 2 + 1) * 8 + 16;
     // bias, per-quarter sums of p and per-64-token counts (both double-buffered by tile parity),
@@ -138,7 +145,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
     const int m_tiles = (int)((T + PM - 1) / PM);
     const int k_blocks = (d + RK - 1) / RK;
-    constexpr uint32_t kTmemCols = 2 * BN;
+    constexpr uint32_t kAccCols = 2 * BN;  // x . (hi + lo) in [0, BN), x . mid in [BN, 2 BN)
+    constexpr uint32_t kTmemCols = 2 * kAccCols;
 
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *ticket = 0u;
@@ -198,10 +206,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * (L::a_bytes + L::b_bytes)));
                     const uint32_t leader_full = map_to_rank(&full[stage], 0);
                     tma_load_2d_pair(sA + stage * L::a_bytes, &tmap_x, leader_full, kb * RK, tile * PM + my_rows);
-#pragma unroll
-                    for (int term = 0; term < kTerms; ++term)
-                        tma_load_3d_pair(sB + stage * L::b_bytes + term * L::b_term_bytes, &tmap_w, leader_full,
-                                         kb * RK, (int)rank * (BN / 2), term);
+                    uint8_t *b_stage = sB + stage * L::b_bytes;
+                    tma_load_3d_pair(b_stage, &tmap_w, leader_full, kb * RK, 0, (int)rank);  // hi or mid
+                    tma_load_3d_pair(b_stage + L::b_half_bytes, &tmap_w, leader_full, kb * RK, BN / 2, (int)rank);
+                    tma_load_3d_pair(b_stage + L::b_stack_bytes, &tmap_w, leader_full, kb * RK,
+                                     (int)rank * (BN / 2), 2);  // lo
                     issued |= 1u << stage;
                     parity_of = (parity_of & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -216,7 +225,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(PM, BN);
+            constexpr uint32_t idesc_stack = idesc_bf16_f32(PM, 2 * BN);
+            constexpr uint32_t idesc_lo = idesc_bf16_f32(PM, BN);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -225,7 +235,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int tile = pair; ok && tile < m_tiles; tile += n_pairs) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, status, 32)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait(&full[stage], phase, status, 33)) {
                         ok = false;
@@ -233,15 +243,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint64_t a_desc = smem_desc_sw128(sA + stage * L::a_bytes);
+                    const uint64_t b_stack = smem_desc_sw128(sB + stage * L::b_bytes);
+                    const uint64_t b_lo = smem_desc_sw128(sB + stage * L::b_bytes + L::b_stack_bytes);
 #pragma unroll
                     for (int k = 0; k < RK / 16; ++k) {
-#pragma unroll
-                        for (int term = 0; term < kTerms; ++term) {
-                            const uint64_t b_desc =
-                                smem_desc_sw128(sB + stage * L::b_bytes + term * L::b_term_bytes);
-                            tc_mma_bf16_pair(d_tmem, a_desc + (uint64_t)(2 * k), b_desc + (uint64_t)(2 * k), idesc,
-                                             (kb | k | term) != 0 ? 1u : 0u);
-                        }
+                        tc_mma_bf16_pair(d_tmem, a_desc + (uint64_t)(2 * k), b_stack + (uint64_t)(2 * k),
+                                         idesc_stack, (kb | k) != 0 ? 1u : 0u);
+                        tc_mma_bf16_pair(d_tmem, a_desc + (uint64_t)(2 * k), b_lo + (uint64_t)(2 * k), idesc_lo,
+                                         1u);
                     }
                     tc_commit_pair(smem_u32(&empty[stage]));
                     tc_commit_pair(map_to_rank(&empty[stage], 1));
@@ -279,15 +288,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int64_t row0 = (int64_t)tile * PM + (int64_t)rank * RM;  // this CTA's first token
             const int64_t t = row0 + tok;
             const bool valid = t < T;
-            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + col0);
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols + col0);
             float h[CW];
 #pragma unroll
             for (int c = 0; c < CW; c += 32) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
+                uint32_t r[32], r2[32];
+                tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);             // x . (hi + lo)
+                tmem_ld_32x32b_x32(t_row + (uint32_t)(BN + c), r2);     // x . mid
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) h[c + j] = __uint_as_float(r[j]) + bias_s[col0 + c + j];
+                for (int j = 0; j < 32; ++j)
+                    h[c + j] = (__uint_as_float(r[j]) + __uint_as_float(r2[j])) + bias_s[col0 + c + j];
             }
             tc_fence_before();
             mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);  // columns in registers: reusable
