@@ -86,7 +86,13 @@ enum {
     SWITCH_FLAG_GEMM_1CTA = 4,
     /* In switch_layer_fwd, launch the two expert GEMMs one after the other
      * instead of as one persistent kernel. */
-    SWITCH_FLAG_FFN_TWO_LAUNCHES = 8
+    SWITCH_FLAG_FFN_TWO_LAUNCHES = 8,
+    /* Always run the capacity scan as its own kernel.  By default, when the
+     * per-tile expert histogram is small, each slot-assignment block sums the
+     * counts it needs itself and the scan kernel is skipped; both give the
+     * same slots and counts (aux may differ in the last bits: its fp64 sums
+     * run in another fixed order). */
+    SWITCH_FLAG_SEPARATE_SCAN = 16
 };
 
 typedef struct {

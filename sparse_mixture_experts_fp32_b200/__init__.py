@@ -30,6 +30,7 @@ SWITCH_FLAG_SIMT_FFN = 1
 SWITCH_FLAG_SIMT_ROUTER = 2
 SWITCH_FLAG_GEMM_1CTA = 4
 SWITCH_FLAG_FFN_TWO_LAUNCHES = 8
+SWITCH_FLAG_SEPARATE_SCAN = 16
 
 STATUS = {
     0: "SWITCH_OK", 1: "SWITCH_ERR_NULL", 2: "SWITCH_ERR_SHAPE", 3: "SWITCH_ERR_DTYPE", 4: "SWITCH_ERR_ALIGN",

@@ -363,6 +363,19 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster_addr) {
                  : "memory");
 }
 
+// One commit that arrives on the mbarrier at the same shared-memory offset in
+// both CTAs of the pair (ctaMask 0b11) once the MMAs issued so far are done.
+// This is an mbarrier arrive sent to both CTAs, not a data load.  Saves an
+// instruction and a mapa per ring stage in the MMA thread against two
+// separate commits.
+__device__ __forceinline__ void tc_commit_both(const uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((uint16_t)0x3)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA
 // with 128-byte swizzling: rows of 128 bytes, 8-row swizzle atoms of 1024
 // bytes stacked at a 1024-byte stride.  The tile base must be 1024-aligned.

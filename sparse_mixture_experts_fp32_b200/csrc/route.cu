@@ -651,21 +651,82 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t *__res
 // Every block also clears a share of the empty slots of slot_token.
 // ---------------------------------------------------------------------------
 constexpr int kAssignThreads = 256;
+constexpr int64_t kFusedScanLoads = int64_t(1) << 22;  // histogram loads of all assignment blocks together
 
-template <bool SCATTER>
+// Per-expert sums over the tile histograms for one block: the tiles before
+// `tile` (the block's first slot per expert) and all tiles (the counts).
+// Integer sums: exact in any order.  Used when the whole histogram is small,
+// in place of the separate scan kernel.
+__device__ __forceinline__ void block_tile_sums(const int32_t *__restrict__ hist, int tiles, int N, int tile,
+                                                int32_t *s_off, int32_t *s_cnt) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = warp; e < N; e += kAssignThreads / 32) {
+        int32_t pre = 0, tot = 0;
+        for (int i = lane; i < tiles; i += 32) {
+            const int32_t h = hist[(int64_t)e * tiles + i];
+            tot += h;
+            pre += i < tile ? h : 0;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            pre += __shfl_xor_sync(0xffffffffu, pre, off);
+            tot += __shfl_xor_sync(0xffffffffu, tot, off);
+        }
+        if (lane == 0) {
+            s_off[e] = pre;
+            s_cnt[e] = tot;
+        }
+    }
+}
+
+// SCAN: the block forms its own first slots and the counts from the tile
+// histograms (small histograms only), and block 0 writes counts, the Σp
+// totals and aux; otherwise they come from scan_kernel.
+template <bool SCATTER, bool SCAN>
 __global__ void __launch_bounds__(kAssignThreads) assign_kernel(
-    const int32_t *__restrict__ expert, const int32_t *__restrict__ tile_off, const int32_t *__restrict__ counts,
+    const int32_t *__restrict__ expert, const int32_t *__restrict__ tile_off, int32_t *__restrict__ counts,
     int64_t T, int N, int C, int tiles, int32_t *__restrict__ slot, int32_t *__restrict__ slot_token,
     const uint4 *__restrict__ x, uint4 *__restrict__ xbuf, int x_words, float4 *__restrict__ y_zero, int y_words,
-    int32_t *__restrict__ done_zero, int64_t n_done) {
+    int32_t *__restrict__ done_zero, int64_t n_done, const int32_t *__restrict__ hist, const float *__restrict__ psum,
+    double *__restrict__ prob_total, float *__restrict__ aux) {
     static_assert(kTileT == 64, "assignment assumes two ranking warps per tile");
     __shared__ int32_t first_warp_count[256];
     __shared__ int32_t tile_slot[kTileT];
     __shared__ int32_t tile_expert[kTileT];
+    __shared__ int32_t s_off[SCAN ? 256 : 1], s_cnt[SCAN ? 256 : 1];
+    __shared__ double s_p[SCAN ? 256 : 1];
     pdl_wait();
     pdl_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x;
+    if (SCAN) {
+        block_tile_sums(hist, tiles, N, tile, s_off, s_cnt);
+        if (blockIdx.x == 0) {
+            // Σp per expert (fp64, lane-strided partial sums, then a fixed xor tree)
+            for (int e = warp; e < N; e += kAssignThreads / 32) {
+                double p = 0.0;
+                for (int i = lane; i < tiles; i += 32) p += (double)psum[(int64_t)e * tiles + i];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
+                if (lane == 0) s_p[e] = p;
+            }
+        }
+        __syncthreads();
+        if (blockIdx.x == 0) {
+            for (int e = tid; e < N; e += kAssignThreads) {
+                counts[e] = s_cnt[e];
+                prob_total[e] = s_p[e];
+            }
+            if (warp == 0) {  // aux = N * sum_i f_i P_i, one term per lane, then a fixed xor tree
+                double term = 0.0;
+                if (T > 0)
+                    for (int e = lane; e < N; e += 32) term += ((double)s_cnt[e] / (double)T) * (s_p[e] / (double)T);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) term += __shfl_xor_sync(0xffffffffu, term, off);
+                if (lane == 0) *aux = (float)((double)N * term);
+            }
+        }
+    }
     if (tile < tiles) {
         for (int i = tid; i < N; i += kAssignThreads) first_warp_count[i] = 0;
         __syncthreads();
@@ -686,7 +747,7 @@ __global__ void __launch_bounds__(kAssignThreads) assign_kernel(
             int s_out = -2;  // -2: no token here
             if (valid) {
                 if (warp == 1) rank += first_warp_count[e];
-                const int s = tile_off[(int64_t)e * tiles + tile] + rank;
+                const int s = (SCAN ? s_off[e] : tile_off[(int64_t)e * tiles + tile]) + rank;
                 if (s < C) {
                     slot[t] = s;
                     slot_token[(int64_t)e * C + s] = (int32_t)t;
@@ -748,7 +809,7 @@ __global__ void __launch_bounds__(kAssignThreads) assign_kernel(
     for (int64_t i = (int64_t)blockIdx.x * kAssignThreads + tid; i < total; i += (int64_t)gridDim.x * kAssignThreads) {
         const int e = (int)(i / C);
         const int s = (int)(i % C);
-        if (s >= min(counts[e], C)) slot_token[i] = -1;
+        if (s >= min(SCAN ? s_cnt[e] : counts[e], C)) slot_token[i] = -1;
     }
 }
 
@@ -856,26 +917,45 @@ cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *
         if (err == cudaSuccess) err = cudaMemsetAsync(ws.status, 0, sizeof(DeviceStatus), stream);
         if (err != cudaSuccess) return err;
     }
-    launch_begin(K_SCAN, stream);
-    err = launch_kernel(scan_kernel, dim3(N), dim3(kScanThreads), 0, stream, ws.tiles > 0, ws.hist, ws.psum,
-                        (int)ws.tiles, N, dims.T, ws.tile_off, counts, ws.prob_total, aux, ws.ticket);
-    launch_end(stream);
-    if (err != cudaSuccess) return err;
     const int64_t fill_blocks = ((int64_t)N * C + kAssignThreads * 4 - 1) / (kAssignThreads * 4);
     const int64_t grid = ws.tiles > fill_blocks ? ws.tiles : fill_blocks;
-    const int x_words = (int)((int64_t)dims.d_model * (dims.dtype == SWITCH_BF16 ? 2 : 4) / 16);
-    if (xbuf_scatter) {
-        launch_begin(K_ASSIGN_SCATTER, stream);
-        err = launch_kernel(assign_kernel<true>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true, expert,
-                            ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token,
-                            static_cast<const uint4 *>(x), static_cast<uint4 *>(xbuf_scatter), x_words,
-                            reinterpret_cast<float4 *>(y_zero), dims.d_model / 4, done_zero, n_done);
-    } else {
-        launch_begin(K_ASSIGN, stream);
-        err = launch_kernel(assign_kernel<false>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
-                            expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token,
-                            (const uint4 *)nullptr, (uint4 *)nullptr, 0, (float4 *)nullptr, 0, done_zero, n_done);
+    // Small histograms: every assignment block sums the tile counts it needs
+    // itself (at most kFusedScanLoads loads over the whole grid), saving the
+    // scan kernel's launch and its round trip through memory.
+    const bool fused_scan = ws.tiles > 0 && (int64_t)N * ws.tiles * grid <= kFusedScanLoads &&
+                            !(dims.flags & SWITCH_FLAG_SEPARATE_SCAN);
+    if (!fused_scan) {
+        launch_begin(K_SCAN, stream);
+        err = launch_kernel(scan_kernel, dim3(N), dim3(kScanThreads), 0, stream, ws.tiles > 0, ws.hist, ws.psum,
+                            (int)ws.tiles, N, dims.T, ws.tile_off, counts, ws.prob_total, aux, ws.ticket);
+        launch_end(stream);
+        if (err != cudaSuccess) return err;
     }
+    const int x_words = (int)((int64_t)dims.d_model * (dims.dtype == SWITCH_BF16 ? 2 : 4) / 16);
+    const uint4 *xs = static_cast<const uint4 *>(x);
+    uint4 *xb = static_cast<uint4 *>(xbuf_scatter);
+    float4 *yz = reinterpret_cast<float4 *>(y_zero);
+    const int y_words = dims.d_model / 4;
+    const int32_t kid = xbuf_scatter ? K_ASSIGN_SCATTER : K_ASSIGN;
+    launch_begin(kid, stream);
+    if (xbuf_scatter && fused_scan)
+        err = launch_kernel(assign_kernel<true, true>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
+                            expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token, xs, xb,
+                            x_words, yz, y_words, done_zero, n_done, ws.hist, ws.psum, ws.prob_total, aux);
+    else if (xbuf_scatter)
+        err = launch_kernel(assign_kernel<true, false>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
+                            expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token, xs, xb,
+                            x_words, yz, y_words, done_zero, n_done, ws.hist, ws.psum, ws.prob_total, aux);
+    else if (fused_scan)
+        err = launch_kernel(assign_kernel<false, true>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
+                            expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token,
+                            (const uint4 *)nullptr, (uint4 *)nullptr, 0, (float4 *)nullptr, 0, done_zero, n_done,
+                            ws.hist, ws.psum, ws.prob_total, aux);
+    else
+        err = launch_kernel(assign_kernel<false, false>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
+                            expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token,
+                            (const uint4 *)nullptr, (uint4 *)nullptr, 0, (float4 *)nullptr, 0, done_zero, n_done,
+                            ws.hist, ws.psum, ws.prob_total, aux);
     launch_end(stream);
     return err;
 }

@@ -252,16 +252,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         tc_mma_bf16_pair(d_tmem, a_desc + (uint64_t)(2 * k), b_lo + (uint64_t)(2 * k), idesc_lo,
                                          1u);
                     }
-                    tc_commit_pair(smem_u32(&empty[stage]));
-                    tc_commit_pair(map_to_rank(&empty[stage], 1));
+                    tc_commit_both(&empty[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit_pair(smem_u32(&acc_full[acc]));
-                tc_commit_pair(map_to_rank(&acc_full[acc], 1));
+                tc_commit_both(&acc_full[acc]);
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
