@@ -48,7 +48,7 @@ Sections layout(const switch_dims_t &d) {
     s.xbuf = take(N * C * (size_t)d.d_model * elem_size(d));
     s.ybuf = take(N * C * (size_t)d.d_model * sizeof(float));
     s.hidden = take(N * C * (size_t)d.d_ff * elem_size(d));
-    s.done = take((N * ((C + 255) / 256) + 1) * sizeof(int32_t));  // + the fused FFN's tile claim counter
+    s.done = take(fused_counter_ints(N, C, d.d_model) * sizeof(int32_t));  // the fused FFN's counters
     s.total = off;
     return s;
 }
@@ -297,7 +297,7 @@ switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const
         // route + scatter-dispatch (zeroing dropped rows of y), GEMM1, GEMM2 with
         // the gate and the token-order scatter fused into its epilogue
         err = launch_route(*dims, x, w_r, logit_bias, expert, gate, slot, counts, ws.slot_token, aux, ws, st,
-                           ws.xbuf, yf, ws.done, (int64_t)dims->num_experts * ((dims->capacity + 255) / 256) + 1);
+                           ws.xbuf, yf, ws.done, fused_counter_ints(dims->num_experts, dims->capacity, dims->d_model));
         if (err == cudaSuccess)
             err = launch_ffn_tc(*dims, ws.xbuf, w_in, w_out, counts, nullptr, ws.slot_token, gate, yf, ws, st);
     } else {

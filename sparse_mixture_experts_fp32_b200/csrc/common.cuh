@@ -119,13 +119,6 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gmem_src, 
         : "memory");
 }
 
-// Prefetch a tile of a 2-D tensor into L2 (no shared memory, no completion).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const void *tmap, int32_t c0, int32_t c1) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
-                 "r"(c0), "r"(c1)
-                 : "memory");
-}
-
 __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
@@ -211,6 +204,16 @@ __device__ __forceinline__ void tma_store_3d(const void *tmap, const void *smem_
 // Contiguous bulk copy shared -> global (16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void bulk_store(void *gmem_dst, const void *smem_src, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                     reinterpret_cast<uint64_t>(gmem_dst)),
+                 "r"(smem_u32(smem_src)), "r"(bytes)
+                 : "memory");
+}
+
+// Bulk add of fp32 values from shared memory onto global memory (an element-wise
+// reduction performed at the destination; addresses 16-byte aligned, size a
+// multiple of 16).
+__device__ __forceinline__ void bulk_add_f32(float *gmem_dst, const void *smem_src, uint32_t bytes) {
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
                      reinterpret_cast<uint64_t>(gmem_dst)),
                  "r"(smem_u32(smem_src)), "r"(bytes)
                  : "memory");

@@ -300,12 +300,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 //                   read downstream; rows >= C are clipped by the tensor map.
 //   kEpiExpertOut / kEpiGatedScatter  32 fp32 columns at a time: each thread
 //                   writes its row (144-byte pitch: conflict-free) and
-//                   issues one 128-byte bulk copy to its destination row.
+//                   issues one 128-byte bulk copy to its destination row
+//                   (with `add`, a bulk fp32 add onto the destination).
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_base, int kept, int C, int n, int Nout,
                                                void *__restrict__ out, const void *tmap_out,
                                                const int32_t *__restrict__ slot_token,
-                                               const float *__restrict__ gate, uint8_t *stage) {
+                                               const float *__restrict__ gate, uint8_t *stage, bool add = false) {
     const int lane = threadIdx.x & 31;
     const int row = row_base + lane;
     const bool row_ok = row < kept;
@@ -364,7 +365,8 @@ __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_ba
                         make_float4(g * __uint_as_float(r[4 * q + 0]), g * __uint_as_float(r[4 * q + 1]),
                                     g * __uint_as_float(r[4 * q + 2]), g * __uint_as_float(r[4 * q + 3]));
                 fence_proxy_async_shared();
-                bulk_store(dst_row + col0, rowp, 128);
+                if (add) bulk_add_f32(dst_row + col0, rowp, 128);
+                else bulk_store(dst_row + col0, rowp, 128);
                 bulk_commit();
             }
         }
@@ -603,6 +605,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // how many pairs are resident at once.  The tail of GEMM1 overlaps the start
 // of GEMM2, and the GEMM2 tiles, too few for one even wave on their own,
 // share the waves with GEMM1.
+// With split = 2 (chosen by the host when GEMM2 has few tiles) every GEMM2
+// tile is cut in two halves of K = F: all first halves come before all
+// second halves in the list.  A first half stores gate * acc into y and then
+// releases y_done[e, m, n] (8 arrivals, as above); the second half waits for
+// that count and adds its gate * acc onto y with bulk fp32 adds.  Every y
+// element is then y0 + y1 with y0 written first: deterministic, and the
+// short second halves fill the last wave.
 // ---------------------------------------------------------------------------
 constexpr int kFusedBN = 256;
 constexpr int kTileQ = 4;                // tile-index queue depth
@@ -624,7 +633,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_hstore, float *__restrict__ y,
                       const int32_t *__restrict__ counts, int E, int C, int d, int F,
                       const int32_t *__restrict__ slot_token, const float *__restrict__ gate,
-                      int32_t *__restrict__ done, int MT, DeviceStatus *status) {
+                      int32_t *__restrict__ done, int MT, int split, DeviceStatus *status) {
     constexpr int BN = kFusedBN;
     using L = PairLayout<BN, STAGES>;
     constexpr int BMP = 2 * BM;
@@ -645,11 +654,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int32_t *start1 = reinterpret_cast<int32_t *>(tmem_holder + 4);  // [E+1] GEMM1 tiles per expert
     int32_t *start2 = start1 + (E + 1);                              // [E+1] GEMM2 tiles per expert
     int32_t *ticket = done + (int64_t)E * MT;                        // tile claim counter of this call
+    int32_t *y_done = ticket + 1;                                    // [E][MT][n2] first halves stored (split 2)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const int n1 = (F + BN - 1) / BN, n2 = (d + BN - 1) / BN;
-    const int kb1 = d / BK, kb2 = F / BK;
+    const int kb1 = d / BK, kb2 = F / BK / split;  // K blocks of a GEMM1 tile and of a GEMM2 tile (or half)
     const int32_t need = 8 * n1;  // arrivals on done[e, m] once H of the row block is complete
     constexpr uint32_t kTmemCols = 2 * BN;
 
@@ -720,7 +730,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncthreads();
     const uint32_t tmem_base = *tmem_holder;
     const int total1 = start1[E];
-    const int total = total1 + start2[E];
+    const int total2 = start2[E];  // GEMM2 tiles per K half
+    const int total = total1 + split * total2;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -751,9 +762,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 if (tile < 0) break;
                 const bool second = tile >= total1;
-                int e, m, n;
-                if (second) locate_tile(start2, E, n2, tile - total1, e, m, n);
-                else locate_tile(start1, E, n1, tile, e, m, n);
+                int e, m, n, ks = 0;
+                if (second) {
+                    ks = (tile - total1) / total2;
+                    locate_tile(start2, E, n2, tile - total1 - ks * total2, e, m, n);
+                } else {
+                    locate_tile(start1, E, n1, tile, e, m, n);
+                }
+                const int k0 = ks * kb2;  // first K block of this tile
                 if (second) {
                     if (!wait_counter_geq(done + e * MT + m, need, status, 47)) break;
                     fence_proxy_async_global();  // H, written through the async proxy, before our TMA reads
@@ -761,6 +777,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const void *ta = second ? (const void *)&tm_h : (const void *)&tm_x;
                 const void *tb = second ? (const void *)&tm_w2 : (const void *)&tm_w1;
                 const int kbs = second ? kb2 : kb1;
+                const int a_row = m * BMP + (int)rank * BM, b_row = n * BN + (int)rank * (BN / 2);
                 for (int kb = 0; kb < kbs; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, status, 41)) {
                         ok = false;
@@ -768,9 +785,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * (L::a_bytes + L::b_bytes)));
                     const uint32_t leader_full = map_to_rank(&full[stage], 0);
-                    tma_load_3d_pair(sA + stage * L::a_bytes, ta, leader_full, kb * BK, m * BMP + (int)rank * BM, e);
-                    tma_load_3d_pair(sB + stage * L::b_bytes, tb, leader_full, kb * BK, n * BN + (int)rank * (BN / 2),
-                                     e);
+                    tma_load_3d_pair(sA + stage * L::a_bytes, ta, leader_full, (k0 + kb) * BK, a_row, e);
+                    tma_load_3d_pair(sB + stage * L::b_bytes, tb, leader_full, (k0 + kb) * BK, b_row, e);
                     issued |= 1u << stage;
                     parity_of = (parity_of & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -848,25 +864,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             if (tile < 0) break;
             const bool second = tile >= total1;
-            int e, m, n;
-            if (second) locate_tile(start2, E, n2, tile - total1, e, m, n);
-            else locate_tile(start1, E, n1, tile, e, m, n);
+            int e, m, n, ks = 0;
+            if (second) {
+                ks = (tile - total1) / total2;
+                locate_tile(start2, E, n2, tile - total1 - ks * total2, e, m, n);
+            } else {
+                locate_tile(start1, E, n1, tile, e, m, n);
+            }
+            int32_t *ydone = y_done + ((int64_t)e * MT + m) * n2 + n;
+            if (ks == 1) {  // the first half of this tile has stored y
+                bool okw = true;
+                if (lane == 0) {
+                    okw = wait_counter_geq(ydone, 8, status, 53);
+                    fence_proxy_async_global();  // ... before our async-proxy adds
+                }
+                if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+            }
             if (!mbar_wait(&acc_full[acc], acc_phase, status, 45)) break;
             tc_fence_after();
             const int row_base = m * BMP + (int)rank * BM + quarter * 32;
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
             if (second)
                 epilogue_async<BN, kEpiGatedScatter>(t_row, e, row_base, min(counts[e], C), C, n, d, y, nullptr,
-                                                     slot_token, gate, my_stage);
+                                                     slot_token, gate, my_stage, ks == 1);
             else
                 epilogue_async<BN, kEpiHiddenRelu>(t_row, e, row_base, min(counts[e], C), C, n, F, nullptr,
                                                    &tm_hstore, slot_token, gate, my_stage);
             tc_fence_before();
             mbar_arrive_cluster(map_to_rank(&acc_empty[acc], 0));
-            if (!second && lane == 0) {
-                bulk_wait_all();             // this warp's H boxes are in global memory
+            if (lane == 0 && (!second || (split == 2 && ks == 0))) {
+                bulk_wait_all();             // this warp's H boxes (or y rows) are in global memory
                 fence_proxy_async_global();  // ... ordered before the release below
-                red_release_add_gpu(done + e * MT + m, 1);
+                red_release_add_gpu(second ? ydone : done + e * MT + m, 1);
             }
             __syncwarp();
             if (++acc == 2) {
@@ -976,16 +1005,23 @@ cudaError_t launch_ffn_fused(const switch_dims_t &dims, const void *xbuf, const 
         !make_tmap(&ths, ws.hidden, E, C, F, 32))
         return cudaErrorInvalidValue;
     const int MT = (C + 2 * BM - 1) / (2 * BM);
-    if (zero_done) {  // counters and the tile claim counter after them
-        err = cudaMemsetAsync(ws.done, 0, ((size_t)E * MT + 1) * sizeof(int32_t), stream);
+    const int n2 = (d + kFusedBN - 1) / kFusedBN;
+    if (zero_done) {  // counters, the tile claim counter and the y_done counters
+        err = cudaMemsetAsync(ws.done, 0, fused_counter_ints(E, C, d) * sizeof(int32_t), stream);
         if (err != cudaSuccess) return err;
     }
     const int64_t m_tiles = std::min<int64_t>((int64_t)E * MT, (dims.T + 2 * BM - 1) / (2 * BM) + E);
-    const int64_t tiles = m_tiles * (((F + kFusedBN - 1) / kFusedBN) + ((d + kFusedBN - 1) / kFusedBN));
-    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / 2, tiles));
+    const int64_t tiles2 = m_tiles * n2;
+    const int max_pairs = device_sm_count() / 2;
+    // Split GEMM2 tiles over K when they are too few for two even waves: the
+    // halves fill the last wave.  Needs an even number of K blocks.
+    const int split = (tiles2 < 2 * (int64_t)max_pairs && (F / BK) % 2 == 0) ? 2 : 1;
+    const int64_t tiles = m_tiles * ((F + kFusedBN - 1) / kFusedBN) + split * tiles2;
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(max_pairs, tiles));
     launch_begin(K_FFN_TC_FUSED, stream);
     err = launch_kernel(kern, dim3(2 * pairs), dim3(kThreads), smem, stream, !zero_done, tx, tw1, th, tw2, ths, y,
-                        counts, E, C, d, F, slot_token, gate, ws.done, MT, static_cast<DeviceStatus *>(ws.status));
+                        counts, E, C, d, F, slot_token, gate, ws.done, MT, split,
+                        static_cast<DeviceStatus *>(ws.status));
     launch_end(stream);
     return err;
 }

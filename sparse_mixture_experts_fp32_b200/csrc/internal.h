@@ -46,11 +46,17 @@ struct Workspace {
     void *xbuf;          // [N][C][d] (layer_fwd only)
     float *ybuf;         // [N][C][d] float32 (layer_fwd only)
     void *hidden;        // [N][C][F] expert hidden activations
-    int32_t *done;       // [N][ceil(C/256)] GEMM1 completion counters of the fused FFN, then its tile counter
+    int32_t *done;       // fused FFN: [N][ceil(C/256)] GEMM1 completion counters, the tile claim counter,
+                         // [N][ceil(C/256)][ceil(d/256)] GEMM2 first-half counters (fused_counter_ints)
     int64_t tiles;
 };
 
 size_t workspace_bytes(const switch_dims_t &dims);
+// int32 counters the fused expert FFN keeps in Workspace::done.
+inline int64_t fused_counter_ints(int64_t N, int64_t C, int64_t d) {
+    const int64_t MT = (C + 255) / 256;
+    return N * MT + 1 + N * MT * ((d + 255) / 256);
+}
 // Bytes at the start of the workspace layout that the routing step uses
 // (status word, ticket, per-tile counts / sums / offsets, probability totals).
 size_t route_scratch_bytes(const switch_dims_t &dims);

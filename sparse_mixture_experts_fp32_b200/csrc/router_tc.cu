@@ -18,23 +18,26 @@
 // leader's shared memory holds the hi rows, the peer's the mid rows), which
 // writes x . hi to accumulator columns [0, BN) and x . mid to [BN, 2 BN), and
 // one with N = BN against lo (each CTA holds half of its rows), added into
-// columns [0, BN).  The epilogue adds the two column blocks.  Two MMAs
-// instead of three: on B200 a pair MMA with N = 128 took about as long as one
-// with N = 256.  Persistent over token tiles, one CTA per SM:
+// columns [0, BN).  The epilogue adds the two column blocks.  The tensor
+// work is the same as three N = BN MMAs (an N = 256 pair MMA takes 128 cycles,
+// an N = 128 one 64 on B200); the MMA thread issues two instructions per K
+// step instead of three.  Persistent over token tiles, one CTA per SM:
 //   warp 0     TMA: 128 x 64 slice of x, this CTA's term of the stacked
 //              operand and half of lo, counted on the leader's (rank 0)
 //              barrier
 //   warp 1     TMEM allocation; one lane of the leader issues the MMAs
-//   warps 2-9  epilogue of the CTA's 128 tokens, two warps per token: each
-//              reads half of the token's logits from TMEM (warp w may only
-//              reach TMEM lanes 32 (w % 4) .. +31, so warps w and w + 4 share
-//              a lane quarter and split the columns); max and argmax (lowest
-//              index on ties), sum of exp and the two halves combined through
-//              shared memory; gate = 1/sum, p_i; per-64-token-tile expert
-//              counts and sums of p_i (deterministic: a fixed shuffle tree,
-//              then a fixed warp order).  Two warps per SM sub-partition hide
-//              the latency of this per-token chain.
+//   warps 2 .. 2 + 4G - 1 (G = BN / 32)  epilogue of the CTA's 128 tokens,
+//              one warp per TMEM lane quarter (warp w may only reach TMEM lanes
+//              32 (w % 4) .. +31) and 32-expert column group: max and argmax
+//              (lowest index on ties) and the sum of exp per group, combined
+//              across the G groups through shared memory; gate = 1/sum, p_i;
+//              per-64-token-tile expert counts and sums of p_i
+//              (deterministic: a fixed shuffle tree, then a fixed warp order).
+//              Several warps per SM sub-partition hide the latency of this
+//              per-token chain.
 // Barrier addresses of the other CTA come from mapa; nothing is multicast.
+// (An L2 prefetch of the next token tile of x, issued at the start of each
+// tile, made the kernel slower on B200, as it did for the expert GEMMs.)
 #include <cuda.h>
 
 #include <algorithm>
@@ -49,8 +52,14 @@ namespace {
 constexpr int RM = 128;  // tokens per CTA (a pair tile is 2 * RM)
 constexpr int RK = 64;   // K per ring stage (one 128-byte swizzle row of bf16)
 constexpr int kTerms = 3;
-constexpr int kEpiThreads = 256;             // warps 2-9
-constexpr int kThreads = 64 + kEpiThreads;
+// Epilogue: G = BN / 32 column groups of 32 experts; four warps (one per TMEM
+// lane quarter) per group.
+template <int BN>
+struct RouterThreads {
+    static constexpr int kGroups = BN / 32;
+    static constexpr int kEpi = 128 * kGroups;  // warps 2 .. 2 + 4G - 1
+    static constexpr int kAll = 64 + kEpi;
+};
 
 // W_r float32 [N][d] -> three bfloat16 terms [3][N][d].
 __global__ void split_router_weight(const float *__restrict__ w, __nv_bfloat16 *__restrict__ out, int64_t n) {
@@ -77,8 +86,8 @@ struct RouterLayout {
     static constexpr size_t ring = STAGES * (a_bytes + b_bytes);
     static constexpr size_t barriers = (2 * STAGES + 2 + 2 + 1) * 8 + 16;
     // bias, per-quarter sums of p and per-64-token counts (both double-buffered by tile parity),
-    // and the exchange of per-half max, argmax and sum between the two warps of a token
-    static constexpr size_t epi = (size_t)BN * 4 + 2 * 4 * BN * 4 + 2 * 2 * BN * 4 + 3 * 2 * RM * 4;
+    // and the exchange of per-group max, argmax and sum between the warps of a token
+    static constexpr size_t epi = (size_t)BN * 4 + 2 * 4 * BN * 4 + 2 * 2 * BN * 4 + 3 * (BN / 32) * RM * 4;
     static constexpr size_t bytes = 1024 + ring + barriers + epi;
 };
 
@@ -102,7 +111,10 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32]) {
     return v[0];
 }
 
-__device__ __forceinline__ void named_barrier_epilogue() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+template <int NT>
+__device__ __forceinline__ void named_barrier_epilogue() {
+    asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+}
 
 // 2-D TMA load into this CTA's shared memory, counted on the mbarrier at
 // `bar_cluster_addr` (the leader's).  No multicast.
@@ -116,13 +128,15 @@ __device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const void *tma
 }
 
 template <int BN, int STAGES>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::kAll, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const float *__restrict__ bias, int64_t T, int d, int N, int tiles64,
                      int32_t *__restrict__ expert, float *__restrict__ gate, int32_t *__restrict__ hist,
                      float *__restrict__ psum, uint32_t *ticket, DeviceStatus *status) {
     using L = RouterLayout<BN, STAGES>;
     constexpr int PM = 2 * RM;  // tokens per pair tile
+    constexpr int G = RouterThreads<BN>::kGroups;
+    constexpr int kEpiThreads = RouterThreads<BN>::kEpi;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
@@ -136,9 +150,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     float *bias_s = reinterpret_cast<float *>(tmem_holder + 4);
     float *psum_w = bias_s + BN;                                     // [2 parity][4 quarters][BN]
     int32_t *hist_s = reinterpret_cast<int32_t *>(psum_w + 8 * BN);  // [2 parity][2 halves][BN]
-    float *x_max = reinterpret_cast<float *>(hist_s + 4 * BN);       // [2 column halves][RM]
-    int32_t *x_arg = reinterpret_cast<int32_t *>(x_max + 2 * RM);    // [2][RM]
-    float *x_sum = reinterpret_cast<float *>(x_arg + 2 * RM);        // [2][RM]
+    float *x_max = reinterpret_cast<float *>(hist_s + 4 * BN);       // [G column groups][RM]
+    int32_t *x_arg = reinterpret_cast<int32_t *>(x_max + G * RM);    // [G][RM]
+    float *x_sum = reinterpret_cast<float *>(x_arg + G * RM);        // [G][RM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -194,10 +208,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             bool ok = true;
             const int my_rows = (int)rank * RM;
             for (int tile = pair; ok && tile < m_tiles; tile += n_pairs) {
-                // x streams from HBM: pull this CTA's rows of the pair's next tile into L2 now
-                const int next = tile + n_pairs;
-                if (next < m_tiles)
-                    for (int kb = 0; kb < k_blocks; ++kb) tma_prefetch_l2_2d(&tmap_x, kb * RK, next * PM + my_rows);
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, status, 31)) {
                         ok = false;
@@ -269,10 +279,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_wait(drain, 0, status, 34);
         }
     } else {
-        constexpr int CW = BN / 2;           // columns per warp
+        constexpr int CW = 32;               // columns per warp
         const int q = warp & 3;              // TMEM lane quarter: tokens 32q .. 32q+31 of this CTA's rows
-        const int half = (warp - 2) >> 2;    // which half of the columns
-        const int col0 = half * CW;
+        const int grp = (warp - 2) >> 2;     // column group: experts 32 grp .. 32 grp + 31
+        const int col0 = grp * CW;
         const int tok = q * 32 + lane;       // token within this CTA's 128 rows
         const int et = threadIdx.x - 64;
         const uint32_t acc_empty_leader0 = map_to_rank(&acc_empty[0], 0);
@@ -288,58 +298,82 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const bool valid = t < T;
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols + col0);
             float h[CW];
-#pragma unroll
-            for (int c = 0; c < CW; c += 32) {
+            {
                 uint32_t r[32], r2[32];
-                tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);             // x . (hi + lo)
-                tmem_ld_32x32b_x32(t_row + (uint32_t)(BN + c), r2);     // x . mid
+                tmem_ld_32x32b_x32(t_row, r);                       // x . (hi + lo)
+                tmem_ld_32x32b_x32(t_row + (uint32_t)BN, r2);       // x . mid
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    h[c + j] = (__uint_as_float(r[j]) + __uint_as_float(r2[j])) + bias_s[col0 + c + j];
+                for (int j = 0; j < 32; ++j) h[j] = (__uint_as_float(r[j]) + __uint_as_float(r2[j])) + bias_s[col0 + j];
             }
             tc_fence_before();
             mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);  // columns in registers: reusable
-            float m = -FLT_MAX;
-            int arg = col0;
+            // four interleaved max / argmax chains (j = u mod 4), then merged with
+            // ties going to the lowest index, as a single left-to-right scan would
+            float m4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
+            int a4[4] = {col0, col0 + 1, col0 + 2, col0 + 3};
 #pragma unroll
-            for (int j = 0; j < CW; ++j) {
-                if (col0 + j < N && h[j] > m) {  // strict: the lowest index wins a tie
-                    m = h[j];
-                    arg = col0 + j;
+            for (int j = 0; j < CW; j += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (col0 + j + u < N && h[j + u] > m4[u]) {  // strict: the lowest index of the chain wins
+                        m4[u] = h[j + u];
+                        a4[u] = col0 + j + u;
+                    }
                 }
             }
-            x_max[half * RM + tok] = m;
-            x_arg[half * RM + tok] = arg;
-            named_barrier_epilogue();
-            const float m_lo = x_max[tok], m_hi = x_max[RM + tok];
-            const float mx = m_hi > m_lo ? m_hi : m_lo;  // ties keep the lower half: lowest index
-            const int amax = m_hi > m_lo ? x_arg[RM + tok] : x_arg[tok];
-            float s_part = 0.f;
+            float m = m4[0];
+            int arg = a4[0];
 #pragma unroll
-            for (int j = 0; j < CW; ++j) {
-                h[j] = col0 + j < N ? expf(h[j] - mx) : 0.f;
-                s_part += h[j];
+            for (int u = 1; u < 4; ++u) {
+                if (m4[u] > m || (m4[u] == m && a4[u] < arg)) {
+                    m = m4[u];
+                    arg = a4[u];
+                }
             }
-            x_sum[half * RM + tok] = s_part;
-            named_barrier_epilogue();
-            const float inv_s = 1.0f / (x_sum[tok] + x_sum[RM + tok]);
+            x_max[grp * RM + tok] = m;
+            x_arg[grp * RM + tok] = arg;
+            named_barrier_epilogue<kEpiThreads>();
+            float mx = x_max[tok];
+            int amax = x_arg[tok];
+#pragma unroll
+            for (int g = 1; g < G; ++g) {  // groups in column order; strict: ties keep the lower index
+                const float v = x_max[g * RM + tok];
+                if (v > mx) {
+                    mx = v;
+                    amax = x_arg[g * RM + tok];
+                }
+            }
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};  // four interleaved partial sums, merged in fixed order
+#pragma unroll
+            for (int j = 0; j < CW; j += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    h[j + u] = col0 + j + u < N ? expf(h[j + u] - mx) : 0.f;
+                    s4[u] += h[j + u];
+                }
+            }
+            x_sum[grp * RM + tok] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            named_barrier_epilogue<kEpiThreads>();
+            float s_all = x_sum[tok];
+#pragma unroll
+            for (int g = 1; g < G; ++g) s_all += x_sum[g * RM + tok];
+            const float inv_s = 1.0f / s_all;
             float *psum_p = psum_w + par * 4 * BN;
             int32_t *hist_p = hist_s + par * 2 * BN;
-#pragma unroll
-            for (int c = 0; c < CW; c += 32) {
+            {
                 float p[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) p[j] = valid ? h[c + j] * inv_s : 0.f;
-                const float col_sum = reduce_scatter32(p);  // this warp's 32 tokens, column col0 + c + lane
-                psum_p[q * BN + col0 + c + lane] = col_sum;
+                for (int j = 0; j < 32; ++j) p[j] = valid ? h[j] * inv_s : 0.f;
+                const float col_sum = reduce_scatter32(p);  // this warp's 32 tokens, column col0 + lane
+                psum_p[q * BN + col0 + lane] = col_sum;
             }
-            if (valid && half == 0) {
+            if (valid && grp == 0) {
                 expert[t] = amax;
                 gate[t] = inv_s;  // p at the argmax: exp(0) / s
                 atomicAdd(&hist_p[(q >> 1) * BN + amax], 1);
             }
-            named_barrier_epilogue();
+            named_barrier_epilogue<kEpiThreads>();
             // the buffers of this parity are next written two tiles later, after two more barriers
             const int t64_0 = (int)(row0 / 64);
             for (int i = et; i < N; i += kEpiThreads) {
@@ -420,7 +454,8 @@ cudaError_t launch_bn(const switch_dims_t &dims, const __nv_bfloat16 *x, const f
     const int64_t m_tiles = (T + 2 * RM - 1) / (2 * RM);
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / 2, m_tiles));
     launch_begin(K_ROUTER_TC, stream);
-    err = launch_kernel(kern, dim3(2 * pairs), dim3(kThreads), smem, stream, true, tx, tw, bias, T, d, N, (int)ws.tiles,
+    err = launch_kernel(kern, dim3(2 * pairs), dim3(RouterThreads<BN>::kAll), smem, stream, true, tx, tw, bias, T, d,
+                        N, (int)ws.tiles,
                         expert, gate, ws.hist, ws.psum, ws.ticket, static_cast<DeviceStatus *>(ws.status));
     launch_end(stream);
     return err;

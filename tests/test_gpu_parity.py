@@ -82,7 +82,9 @@ def test_layer_small_simt_router(orc, name, T):
 
 @pytest.mark.parametrize("name,T", [("base8", 3000), ("large128", 2500), ("bigexpert64", 400)])
 def test_fused_ffn_matches_two_launches(name, T):
-    """One persistent launch for both expert GEMMs gives the same bytes as two launches."""
+    """One persistent launch for both expert GEMMs agrees with two launches.  Where the fused
+    kernel splits GEMM2 tiles over K (few GEMM2 tiles), y = g*acc0 + g*acc1 instead of
+    g*(acc0 + acc1): the two differ by fp32 rounding only."""
     wl = synth.WORKLOADS[name]
     C = synth_capacity(wl, T)
     inp = synth.inputs(wl, T=T, experts=range(min(wl.num_experts, 16)))
@@ -91,7 +93,12 @@ def test_fused_ffn_matches_two_launches(name, T):
     b = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, logit_bias=dev["bias"],
                      flags=sm.SWITCH_FLAG_FFN_TWO_LAUNCHES)
     assert sm.switch_check(a["workspace"]) == 0 and sm.switch_check(b["workspace"]) == 0
-    assert torch.equal(a["y"].view(torch.int32), b["y"].view(torch.int32))
+    ya, yb = a["y"].double(), b["y"].double()
+    rms = float(yb.pow(2).mean().sqrt())
+    # rounding of the two partial sums (F/2 products each, which may partly cancel) and of the
+    # two gate products: measured 1.3e-5 * RMS on Base-8; the parity bar itself is 2e-2 * RMS
+    assert float((ya - yb).abs().max()) <= 1e-4 * rms
+    assert torch.equal((a["y"] == 0).all(dim=1), (b["y"] == 0).all(dim=1))  # the same rows are zero (dropped)
 
 
 @pytest.mark.parametrize("name,T", [("tiny_fp32", 64), ("base8", 3000), ("base128_skew", 2000)])
@@ -136,13 +143,17 @@ def test_route_entry_point_slot_token(orc):
 
 
 def test_entry_points_compose_to_layer(orc):
-    """route -> dispatch -> expert_ffn -> combine gives the same bytes as layer_fwd."""
+    """route -> dispatch -> expert_ffn -> combine gives the same bytes as layer_fwd with the two
+    expert GEMMs launched one after the other, and agrees with the default layer_fwd (whose fused
+    FFN may split GEMM2 over K) to fp32 rounding."""
     wl = synth.WORKLOADS["base8"]
     T = 2000
     C = synth_capacity(wl, T)
     inp = synth.inputs(wl, T=T)
     dev = {k: to_device(v) for k, v in inp.items()}
-    ref = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C)
+    ref = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C,
+                       flags=sm.SWITCH_FLAG_FFN_TWO_LAUNCHES)
+    fused = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C)
     d = sm.layer_dims(dev["x"], dev["w_in"], capacity=C)
     ws = sm.workspace(d, "cuda")
     N, dm = wl.num_experts, wl.d_model
@@ -163,6 +174,8 @@ def test_entry_points_compose_to_layer(orc):
     assert torch.equal(expert, ref["expert"]) and torch.equal(slot, ref["slot"])
     assert torch.equal(counts, ref["counts"]) and torch.equal(aux, ref["aux"])
     assert torch.equal(y.view(torch.int32), ref["y"].view(torch.int32))
+    rms = float(ref["y"].double().pow(2).mean().sqrt())
+    assert float((fused["y"].double() - y.double()).abs().max()) <= 1e-4 * rms
     # dispatch wrote exactly the kept tokens' rows
     kept = torch.clamp(counts, max=C).cpu().numpy()
     st = slot_token.view(N, C).cpu().numpy()
@@ -173,11 +186,12 @@ def test_entry_points_compose_to_layer(orc):
                                dev["x"][torch.from_numpy(st[e, :kept[e]]).long().cuda()].cpu().view(torch.int16))
 
 
-def test_deterministic_bytes(orc):
-    wl = synth.WORKLOADS["base128_skew"]
-    inp = synth.inputs(wl, T=6000, experts=range(8))
+@pytest.mark.parametrize("name,T", [("base128_skew", 6000), ("base8", 3000)])
+def test_deterministic_bytes(orc, name, T):
+    wl = synth.WORKLOADS[name]
+    inp = synth.inputs(wl, T=T, experts=range(8))
     dev = {k: to_device(v) for k, v in inp.items()}
-    C = synth_capacity(wl, 6000)
+    C = synth_capacity(wl, T)
     a = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, logit_bias=dev["bias"])
     b = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, logit_bias=dev["bias"])
     for k in ("expert", "gate", "slot", "counts", "aux"):
