@@ -605,15 +605,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // how many pairs are resident at once.  The tail of GEMM1 overlaps the start
 // of GEMM2, and the GEMM2 tiles, too few for one even wave on their own,
 // share the waves with GEMM1.
-// With split = 2 (chosen by the host when GEMM2 has few tiles) every GEMM2
-// tile is cut in two halves of K = F: all first halves come before all
-// second halves in the list.  A first half stores gate * acc into y and then
-// releases y_done[e, m, n] (8 arrivals, as above); the second half waits for
-// that count and adds its gate * acc onto y with bulk fp32 adds.  Every y
-// element is then y0 + y1 with y0 written first: deterministic, and the
-// short second halves fill the last wave.
+// When GEMM2 has fewer tiles than two waves, every GEMM2 tile is cut into S
+// parts (S = 2 or 4) along K = F, the part count picked on the device from
+// the real tile counts (fused_split).  All parts ks = 0 come first in the
+// list, then all parts ks = 1, and so on.  Part 0 stores gate * acc into y;
+// part ks > 0 waits until y_done[e, m, n] reaches 8 ks (parts 0 .. ks-1 are
+// in y) and adds its gate * acc with bulk fp32 adds, then releases 8 more.
+// Every y element is ((y0 + y1) + y2) + ... in that order: deterministic.
+// The short parts fill the last wave; the chain of adds costs one epilogue
+// per part.
 // ---------------------------------------------------------------------------
 constexpr int kFusedBN = 256;
+
+// Parts per GEMM2 tile: 1, 2 or 4, for GEMM2 with fewer tiles than two waves
+// only (the adds cost y traffic).  Picks the S that minimises a rough time
+// for the GEMM2 waves in K blocks: waves * (K blocks per part) plus about six
+// K blocks of epilogue per extra part in the chain of adds.  Every CTA
+// computes the same value from the same counts.
+__device__ __forceinline__ int fused_split(int tiles2, int kb_total, int pairs) {
+    if (tiles2 <= 0 || tiles2 >= 2 * pairs) return 1;
+    int best = 1, best_cost = ((tiles2 + pairs - 1) / pairs) * kb_total;
+    for (int s = 2; s <= 4; s *= 2) {
+        if (kb_total % s != 0 || kb_total / s < 8) break;
+        const int cost = ((s * tiles2 + pairs - 1) / pairs) * (kb_total / s) + 6 * (s - 1);
+        if (cost < best_cost) {
+            best = s;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
 constexpr int kTileQ = 4;                // tile-index queue depth
 constexpr int kTileConsumers = 1 + 1 + 8;  // leader MMA thread, peer producer, 8 epilogue warps
 
@@ -633,7 +654,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_hstore, float *__restrict__ y,
                       const int32_t *__restrict__ counts, int E, int C, int d, int F,
                       const int32_t *__restrict__ slot_token, const float *__restrict__ gate,
-                      int32_t *__restrict__ done, int MT, int split, DeviceStatus *status) {
+                      int32_t *__restrict__ done, int MT, DeviceStatus *status) {
     constexpr int BN = kFusedBN;
     using L = PairLayout<BN, STAGES>;
     constexpr int BMP = 2 * BM;
@@ -654,12 +675,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int32_t *start1 = reinterpret_cast<int32_t *>(tmem_holder + 4);  // [E+1] GEMM1 tiles per expert
     int32_t *start2 = start1 + (E + 1);                              // [E+1] GEMM2 tiles per expert
     int32_t *ticket = done + (int64_t)E * MT;                        // tile claim counter of this call
-    int32_t *y_done = ticket + 1;                                    // [E][MT][n2] first halves stored (split 2)
+    int32_t *y_done = ticket + 1;                                    // [E][MT][n2] GEMM2 parts stored in y
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const int n1 = (F + BN - 1) / BN, n2 = (d + BN - 1) / BN;
-    const int kb1 = d / BK, kb2 = F / BK / split;  // K blocks of a GEMM1 tile and of a GEMM2 tile (or half)
+    const int kb1 = d / BK;  // K blocks of a GEMM1 tile
     const int32_t need = 8 * n1;  // arrivals on done[e, m] once H of the row block is complete
     constexpr uint32_t kTmemCols = 2 * BN;
 
@@ -730,7 +751,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncthreads();
     const uint32_t tmem_base = *tmem_holder;
     const int total1 = start1[E];
-    const int total2 = start2[E];  // GEMM2 tiles per K half
+    const int total2 = start2[E];  // GEMM2 output tiles
+    const int split = fused_split(total2, F / BK, (int)(gridDim.x >> 1));
+    const int kb2 = F / BK / split;  // K blocks of a GEMM2 part
     const int total = total1 + split * total2;
 
     if (warp == 0) {
@@ -872,10 +895,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 locate_tile(start1, E, n1, tile, e, m, n);
             }
             int32_t *ydone = y_done + ((int64_t)e * MT + m) * n2 + n;
-            if (ks == 1) {  // the first half of this tile has stored y
+            if (ks > 0) {  // parts 0 .. ks-1 of this output tile are in y
                 bool okw = true;
                 if (lane == 0) {
-                    okw = wait_counter_geq(ydone, 8, status, 53);
+                    okw = wait_counter_geq(ydone, 8 * ks, status, 53);
                     fence_proxy_async_global();  // ... before our async-proxy adds
                 }
                 if (!__shfl_sync(0xffffffffu, okw, 0)) break;
@@ -886,13 +909,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
             if (second)
                 epilogue_async<BN, kEpiGatedScatter>(t_row, e, row_base, min(counts[e], C), C, n, d, y, nullptr,
-                                                     slot_token, gate, my_stage, ks == 1);
+                                                     slot_token, gate, my_stage, ks > 0);
             else
                 epilogue_async<BN, kEpiHiddenRelu>(t_row, e, row_base, min(counts[e], C), C, n, F, nullptr,
                                                    &tm_hstore, slot_token, gate, my_stage);
             tc_fence_before();
             mbar_arrive_cluster(map_to_rank(&acc_empty[acc], 0));
-            if (lane == 0 && (!second || (split == 2 && ks == 0))) {
+            if (lane == 0 && (!second || ks < split - 1)) {
                 bulk_wait_all();             // this warp's H boxes (or y rows) are in global memory
                 fence_proxy_async_global();  // ... ordered before the release below
                 red_release_add_gpu(second ? ydone : done + e * MT + m, 1);
@@ -1013,15 +1036,12 @@ cudaError_t launch_ffn_fused(const switch_dims_t &dims, const void *xbuf, const 
     const int64_t m_tiles = std::min<int64_t>((int64_t)E * MT, (dims.T + 2 * BM - 1) / (2 * BM) + E);
     const int64_t tiles2 = m_tiles * n2;
     const int max_pairs = device_sm_count() / 2;
-    // Split GEMM2 tiles over K when they are too few for two even waves: the
-    // halves fill the last wave.  Needs an even number of K blocks.
-    const int split = (tiles2 < 2 * (int64_t)max_pairs && (F / BK) % 2 == 0) ? 2 : 1;
-    const int64_t tiles = m_tiles * ((F + kFusedBN - 1) / kFusedBN) + split * tiles2;
+    // upper bound on the tile count (GEMM2 tiles may be cut into up to 4 parts on the device)
+    const int64_t tiles = m_tiles * ((F + kFusedBN - 1) / kFusedBN) + 4 * tiles2;
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(max_pairs, tiles));
     launch_begin(K_FFN_TC_FUSED, stream);
     err = launch_kernel(kern, dim3(2 * pairs), dim3(kThreads), smem, stream, !zero_done, tx, tw1, th, tw2, ths, y,
-                        counts, E, C, d, F, slot_token, gate, ws.done, MT, split,
-                        static_cast<DeviceStatus *>(ws.status));
+                        counts, E, C, d, F, slot_token, gate, ws.done, MT, static_cast<DeviceStatus *>(ws.status));
     launch_end(stream);
     return err;
 }

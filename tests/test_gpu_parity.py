@@ -94,7 +94,8 @@ def test_fused_ffn_matches_two_launches(name, T):
                      flags=sm.SWITCH_FLAG_FFN_TWO_LAUNCHES)
     assert sm.switch_check(a["workspace"]) == 0 and sm.switch_check(b["workspace"]) == 0
     ya, yb = a["y"].double(), b["y"].double()
-    rms = float(yb.pow(2).mean().sqrt())
+    kept = ~(b["y"] == 0).all(dim=1)  # rows of kept tokens (dropped rows are zero in both)
+    rms = float(yb[kept].pow(2).mean().sqrt())
     # rounding of the two partial sums (F/2 products each, which may partly cancel) and of the
     # two gate products: measured 1.3e-5 * RMS on Base-8; the parity bar itself is 2e-2 * RMS
     assert float((ya - yb).abs().max()) <= 1e-4 * rms
