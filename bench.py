@@ -319,7 +319,9 @@ def run_gpu(args):
         k = kernels[dominant]
         roofline = {"kernel": dominant, "bound": k["bound"], "achieved": k["achieved"], "peak": k["peak"],
                     "unit": k["unit"], "frac": k["frac"], "traffic": traffic_from_profiles(dominant, wl.name),
-                    "peak_source": f"{peak_src} ({'burst bf16 matmul' if k['bound'] == 'tensor' else 'copy bandwidth'})"}
+                    "peak_source": (f"{peak_src} (burst bf16 matmul)" if k["bound"] == "tensor" else
+                                    f"{peak_src} (copy bandwidth)" if k["bound"] == "hbm" else
+                                    "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz (FFMA issue rate)")}
 
     # e2e through the public API with pinned host buffers
     e2e = run_e2e(args, sm, wl, inp, C, device, world)

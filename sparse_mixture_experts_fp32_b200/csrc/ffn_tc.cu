@@ -1071,8 +1071,10 @@ cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const voi
     cudaError_t err = launch_gemm_pair<256, 6, kEpiHiddenRelu>(K_FFN_TC_GEMM1, xbuf, w_in, ws.hidden, counts, N, C,
                                                                d, F, dims.T, nullptr, nullptr, st, stream);
     if (err != cudaSuccess) return err;
-    // N = 256 MMAs for both GEMMs: with N = 128 the pair MMAs reached about
-    // half the tensor throughput of N = 256 on B200.
+    // 256-column tiles for both GEMMs: a 128-column GEMM2 tile re-reads its
+    // A rows (H) for half the output, doubling the operand traffic per flop,
+    // and ran about half as fast on B200 (the MMAs themselves take 64 cycles
+    // for N = 128 against 128 for N = 256: the same rate per flop).
     if (y)
         return launch_gemm_pair<256, 6, kEpiGatedScatter>(K_FFN_TC_GEMM2_GATED, ws.hidden, w_out, y, counts, N, C,
                                                           F, d, dims.T, slot_token, gate, st, stream);
