@@ -1,0 +1,53 @@
+"""Host-side pieces of bench.py: the kernel work table and the lookup of DRAM
+traffic in committed ncu summaries (no GPU needed)."""
+import shutil
+import sys
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parents[1]
+sys.path.insert(0, str(ROOT))
+import bench  # noqa: E402
+from sparse_mixture_experts_fp32_b200 import synth  # noqa: E402
+
+
+def test_kernel_work_base8():
+    wl = synth.WORKLOADS["base8"]
+    C = 1280
+    counts = np.full(wl.num_experts, wl.T // wl.num_experts, dtype=np.int64)
+    work = bench.kernel_work(wl, C, counts)
+    K = wl.T  # nothing dropped with equal counts below C
+    assert work["ffn_tc_fused"] == ("tensor", 4.0 * K * wl.d_model * wl.d_ff)
+    assert work["_meta"][1]["K"] == K
+    # the router reads x once (bf16), W_r, and writes expert + gate per token plus per-tile partials
+    tiles = -(-wl.T // 64)
+    assert work["router_staged"][1] == wl.T * wl.d_model * 2 + wl.num_experts * wl.d_model * 4 + 8 * wl.T + \
+        8 * wl.num_experts * tiles
+
+
+def _fake_tree(tmp_path):
+    """A copy of the sources and an empty profiles folder under tmp_path."""
+    csrc = tmp_path / "sparse_mixture_experts_fp32_b200" / "csrc"
+    shutil.copytree(ROOT / "sparse_mixture_experts_fp32_b200" / "csrc", csrc,
+                    ignore=shutil.ignore_patterns("_build", "*.o"))
+    (tmp_path / "profiles").mkdir()
+    return csrc
+
+
+def test_traffic_lines_follow_the_kernel_source(tmp_path, monkeypatch):
+    csrc = _fake_tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", tmp_path)
+    sha = bench.source_sha("router_tc")
+    other = bench.source_sha("ffn_tc_fused")
+    assert sha != other  # keyed by the kernel's own source file
+    (tmp_path / "profiles" / "k.md").write_text(
+        f"    traffic[router_tc@base128_skew]: 1234 bytes source_sha={sha}\n"
+        f"    traffic[ffn_tc_fused@base128_skew]: 99 bytes source_sha=000000000000\n")
+    assert bench.traffic_from_profiles("router_tc", "base128_skew") == 1234.0
+    assert bench.traffic_from_profiles("router_tc", "base8") is None          # other workload
+    assert bench.traffic_from_profiles("ffn_tc_fused", "base128_skew") is None  # stale hash
+    # editing the router's source invalidates only the router's line
+    (csrc / "router_tc.cu").write_text((csrc / "router_tc.cu").read_text() + "\n// edit\n")
+    assert bench.traffic_from_profiles("router_tc", "base128_skew") is None
+    assert bench.source_sha("ffn_tc_fused") == other
