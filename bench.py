@@ -3,8 +3,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 One step is one switch_layer_fwd over one batch of synthetic tokens (router,
-capacity scan, slot assignment with dispatch, both expert GEMMs, gated
-combine), inputs already resident in HBM.  Each step is timed with CUDA events
+capacity scan, slot assignment with dispatch, both expert GEMMs with the gated
+combine in the second one's epilogue; the scan runs inside the assignment
+kernel when the per-tile histogram is small), inputs already resident in HBM.  Each step is timed with CUDA events
 on the launching stream; an L2 flush (a 512 MiB write) runs between steps,
 outside the events.  With --gpus N (under torchrun) every rank runs its own
 batch (independent token groups, replicated experts: weak scaling, no
