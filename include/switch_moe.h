@@ -26,8 +26,8 @@
  *    aligned, unless marked otherwise.  The library never allocates, frees or
  *    synchronises, except switch_check() (which synchronises the stream).
  *  - Streams: every compute call is asynchronous on `stream` (a cudaStream_t;
- *    NULL means the legacy default stream) and launches only kernels of this
- *    library on it.
+ *    NULL means the legacy default stream) and enqueues only kernels of this
+ *    library, plus a few small cudaMemsetAsync calls on the workspace, on it.
  *  - Errors: argument errors are detected on the host before anything is
  *    launched and leave every output untouched.  A failed launch returns
  *    SWITCH_ERR_CUDA.  A kernel that gives up a bounded wait records
@@ -178,8 +178,13 @@ switch_status_t switch_combine(const switch_dims_t *dims, const void *ybuf, cons
  * the [N, C, d] buffers and slot_token kept in the workspace.  Arguments as
  * above; y [T, d] float32 is the layer output WITHOUT the residual.  On the
  * bfloat16 tensor-core path the dispatch is fused into the slot assignment
- * and the combine into the second expert GEMM; the result is bit-identical
- * to calling the four steps one by one. */
+ * and both expert GEMMs run in one persistent kernel with the combine in the
+ * second GEMM's epilogue.  With SWITCH_FLAG_FFN_TWO_LAUNCHES the result is
+ * bit-identical to calling the four steps one by one.  By default, when the
+ * second GEMM has few tiles, its tiles are split along d_ff and their parts
+ * added into y in a fixed order: routing, counts and aux are unchanged and y
+ * differs from the four-step result by float32 rounding only.  Either way
+ * identical inputs give identical bytes. */
 switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const float *w_r,
                                  const float *logit_bias, const void *w_in, const void *w_out, void *y,
                                  int32_t *expert, float *gate, int32_t *slot, int32_t *counts, float *aux,
