@@ -5,18 +5,28 @@
 One step is one switch_layer_fwd over one batch of synthetic tokens (router,
 capacity scan, slot assignment with dispatch, both expert GEMMs with the gated
 combine in the second one's epilogue; the scan runs inside the assignment
-kernel when the per-tile histogram is small), inputs already resident in HBM.  Each step is timed with CUDA events
-on the launching stream; an L2 flush (a 512 MiB write) runs between steps,
-outside the events.  With --gpus N (under torchrun) every rank runs its own
-batch (independent token groups, replicated experts: weak scaling, no
-collective on the data path); time = max over ranks.
+kernel when the per-tile histogram is small), inputs already resident in HBM.
+The default workload is the largest one, the Switch-Large-shaped layer
+(T = 131072, d_model = 1024, d_ff = 4096, 128 experts, c = 1.25).  Each step is
+timed with CUDA events on the launching stream; an L2 flush (a 512 MiB write)
+runs between steps, outside the events.  With --gpus N (under torchrun) every
+rank runs its own batch (independent token groups, replicated experts: weak
+scaling, no collective on the data path); time = max over ranks.
 
 The JSON line also carries:
   roofline      the dominant kernel's achieved rate from per-launch CUDA
                 events (the library's tracer) against the measured peak
+                (burst, and sustained for tensor-core kernels)
+  kernels       every kernel's time, share and fraction of its roofline; for
+                the kernels that write the float32 output, also the fraction
+                with those rows counted at the activation dtype
   e2e           the same metric through the public API with pinned host
                 buffers: x copied in and y/aux/counts copied out every step
-  cpu_baseline  the fp64 oracle on the host cores over a bounded sample
+  entry_points  switch_dispatch and switch_combine called on their own
+  sweep         the large-expert layer at every capacity factor of its sweep
+                (drop fraction and tokens/s per c)
+  cpu_baseline  the fp64 oracle on all host cores and on one core, over a
+                bounded sample
   clocks        nvidia-smi samples taken during the timed region
 --impl reference times the oracle as the reference arm.
 """
@@ -42,7 +52,8 @@ from sparse_mixture_experts_fp32_b200 import synth  # noqa: E402
 
 METRIC = "Switch-layer fwd tokens/s on 1 B200; expert GEMM % bf16 peak; route/scatter GB/s"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "base8"
+DEFAULT_WORKLOAD = "large128"
+SWEEP_WORKLOAD = "bigexpert64"
 L2_FLUSH_BYTES = 512 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -79,6 +90,17 @@ def max_over_ranks(value: float, world: int, device) -> float:
     t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def workload_of(args):
+    """The named workload, with the optional capacity factor and token count
+    overrides (a reduced token count serves small profiler captures)."""
+    wl = synth.WORKLOADS[args.workload]
+    if args.capacity_factor is not None:
+        wl = wl.with_capacity_factor(args.capacity_factor)
+    if args.tokens is not None:
+        wl = wl.with_tokens(args.tokens)
+    return wl
 
 
 def rank_seed(wl, rank: int) -> int:
@@ -146,7 +168,13 @@ class ClockSampler:
 # algorithmic work per kernel launch
 # ---------------------------------------------------------------------------
 def kernel_work(wl, C, counts):
-    """Algorithmic bytes (HBM) or flops per launch of each kernel of one step."""
+    """Algorithmic work per launch of each kernel of one step: (bound, amount,
+    amount with every activation-sized tensor counted at the activation dtype).
+
+    The layer writes y (and zero rows of dropped tokens) in float32; the third
+    figure counts those bytes at the activation dtype instead (T*d*s for the
+    output), which is the algorithmic byte count of the combine and the
+    dispatch as the layer's step table states them."""
     T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.num_experts
     s = 2 if wl.dtype == synth.BF16 else 4
     kept = np.minimum(counts, C)
@@ -154,22 +182,54 @@ def kernel_work(wl, C, counts):
     E_nz = int((kept > 0).sum())
     tiles = -(-T // 64)
     router_bytes = T * d * s + N * d * 4 + 8 * T + 8 * N * tiles
+    assign_common = 4 * T + 4 * T + 4 * N * tiles + 4 * N * C + 2 * K * d * s
     return {
-        "router_warp": ("hbm", router_bytes),
-        "router_tiled": ("hbm", router_bytes),
-        "router_staged": ("hbm", router_bytes),
-        "router_tc": ("hbm", T * d * s + 3 * N * d * 2 + 8 * T + 8 * N * tiles),
-        "router_weight_split": ("hbm", N * d * 4 + 3 * N * d * 2),
-        "capacity_scan": ("hbm", 8 * N * tiles + 4 * N * tiles + 12 * N),
-        "slot_assign_scatter": ("hbm", 4 * T + 4 * T + 4 * N * tiles + 4 * N * C + 2 * K * d * s + (T - K) * d * 4),
-        "ffn_tc_gemm1_relu": ("tensor", 2.0 * K * d * F),
-        "ffn_tc_gemm2_gated_scatter": ("tensor", 2.0 * K * F * d),
-        "ffn_tc_fused": ("tensor", 4.0 * K * d * F),
-        "ffn_simt_gemm1_relu": ("alu", 2.0 * K * d * F),
-        "ffn_simt_gemm2": ("alu", 2.0 * K * F * d),
-        "combine": ("hbm", T * d * 4 + K * d * 4 + 12 * T),
-        "_meta": ("", dict(K=K, E_nz=E_nz, gemm_weight_bytes=2 * E_nz * d * F * s)),
+        "router_warp": ("hbm", router_bytes, None),
+        "router_tiled": ("hbm", router_bytes, None),
+        "router_staged": ("hbm", router_bytes, None),
+        "router_tc": ("hbm", T * d * s + 3 * N * d * 2 + 8 * T + 8 * N * tiles, None),
+        "router_weight_split": ("hbm", N * d * 4 + 3 * N * d * 2, None),
+        "capacity_scan": ("hbm", 8 * N * tiles + 4 * N * tiles + 12 * N, None),
+        "slot_assign_scatter": ("hbm", assign_common + (T - K) * d * 4, assign_common + (T - K) * d * s),
+        "ffn_tc_gemm1_relu": ("tensor", 2.0 * K * d * F, None),
+        "ffn_tc_gemm2_gated_scatter": ("tensor", 2.0 * K * F * d, None),
+        "ffn_tc_fused": ("tensor", 4.0 * K * d * F, None),
+        "ffn_simt_gemm1_relu": ("alu", 2.0 * K * d * F, None),
+        "ffn_simt_gemm2": ("alu", 2.0 * K * F * d, None),
+        "combine": ("hbm", T * d * 4 + K * d * 4 + 12 * T, T * d * s + K * d * s + 12 * T),
+        "dispatch": ("hbm", 2 * K * d * s + 4 * N * C + 4 * N, None),
+        "_meta": ("", dict(K=K, E_nz=E_nz, gemm_weight_bytes=2 * E_nz * d * F * s), None),
     }
+
+
+def kernel_entry(kind, amount, amount_act, avg_ms, launches, peaks):
+    """One kernel's achieved rate against the measured peaks."""
+    entry = {"launches": launches, "avg_ms": round(avg_ms, 5), "share": None}
+    sec = avg_ms * 1e-3
+    if kind == "hbm":
+        entry.update(bound="hbm", achieved=amount / sec / 1e9, peak=peaks["hbm_gbs"], unit="GB/s")
+    elif kind == "tensor":
+        entry.update(bound="tensor", achieved=amount / sec / 1e12, peak=peaks["bf16_tflops"], unit="TFLOP/s")
+    elif kind == "alu":
+        entry.update(bound="alu", achieved=amount / sec / 1e12, peak=74.4, unit="TFLOP/s")
+    if "achieved" in entry:
+        entry["frac"] = round(entry["achieved"] / entry["peak"], 4)
+        entry["achieved"] = round(entry["achieved"], 2)
+        if kind == "tensor" and "bf16_tflops_sustained" in peaks:
+            entry["frac_sustained"] = round(entry["achieved"] / peaks["bf16_tflops_sustained"], 4)
+        if amount_act is not None:
+            # the same kernel with the float32 output rows counted at the activation dtype
+            entry["achieved_act_dtype"] = round(amount_act / sec / 1e9, 2)
+            entry["frac_act_dtype"] = round(amount_act / sec / 1e9 / entry["peak"], 4)
+    return entry
+
+
+DOMINANT_WORK_TEXT = {
+    "ffn_tc_fused": "4*K*d_model*d_ff (K = kept tokens; both expert GEMMs)",
+    "router_tc": "T*d*s + 6*N*d + 8*T + 8*N*ceil(T/64)",
+    "router_staged": "T*d*s + 4*N*d + 8*T + 8*N*ceil(T/64)",
+    "slot_assign_scatter": "8*T + 4*N*ceil(T/64) + 4*N*C + 2*K*d*s + 4*(T-K)*d",
+}
 
 
 # ---------------------------------------------------------------------------
@@ -193,9 +253,7 @@ def run_gpu(args):
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     dist = init_dist(world, "nccl")
-    wl = synth.WORKLOADS[args.workload]
-    if args.capacity_factor is not None:
-        wl = wl.with_capacity_factor(args.capacity_factor)
+    wl = workload_of(args)
     # experts and router are shared by all ranks; every rank routes its own tokens
     w_in_np, w_out_np = synth.all_expert_weights(wl)
     inp = dict(x=synth.activations(wl, seed=rank_seed(wl, rank)), w_r=synth.router_weight(wl),
@@ -297,20 +355,8 @@ def run_gpu(args):
     peaks, peak_src = load_peaks()
     kernels = {}
     for name, times in per_kernel.items():
-        avg = statistics.mean(times)
-        kind, amount = work.get(name, ("?", 0))
-        entry = {"launches": len(times), "avg_ms": round(avg, 5), "share": None}
-        if kind == "hbm":
-            entry.update(bound="hbm", achieved=amount / (avg * 1e-3) / 1e9, peak=peaks["hbm_gbs"], unit="GB/s")
-        elif kind == "tensor":
-            entry.update(bound="tensor", achieved=amount / (avg * 1e-3) / 1e12, peak=peaks["bf16_tflops"],
-                         unit="TFLOP/s")
-        elif kind == "alu":
-            entry.update(bound="alu", achieved=amount / (avg * 1e-3) / 1e12, peak=74.4, unit="TFLOP/s")
-        if "achieved" in entry:
-            entry["achieved"] = round(entry["achieved"], 2)
-            entry["frac"] = round(entry["achieved"] / entry["peak"], 4)
-        kernels[name] = entry
+        kind, amount, amount_act = work.get(name, ("?", 0, None))
+        kernels[name] = kernel_entry(kind, amount, amount_act, statistics.mean(times), len(times), peaks)
     tot = sum(k["avg_ms"] * k["launches"] for k in kernels.values())
     for k in kernels.values():
         k["share"] = round(k["avg_ms"] * k["launches"] / tot, 4) if tot else None
@@ -320,42 +366,25 @@ def run_gpu(args):
         k = kernels[dominant]
         roofline = {"kernel": dominant, "bound": k["bound"], "achieved": k["achieved"], "peak": k["peak"],
                     "unit": k["unit"], "frac": k["frac"], "traffic": traffic_from_profiles(dominant, wl.name),
+                    "units_per_launch": ("flops" if k["bound"] in ("tensor", "alu") else "bytes") + " = " +
+                                        DOMINANT_WORK_TEXT.get(dominant, "see kernel_work"),
                     "peak_source": (f"{peak_src} (burst bf16 matmul)" if k["bound"] == "tensor" else
                                     f"{peak_src} (copy bandwidth)" if k["bound"] == "hbm" else
                                     "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz (FFMA issue rate)")}
+        if "frac_sustained" in k:
+            roofline["frac_sustained"] = k["frac_sustained"]
+            roofline["peak_sustained"] = peaks.get("bf16_tflops_sustained")
+        if clocks and clocks.get("sm_mhz"):
+            roofline["sm_mhz_median"] = clocks["sm_mhz"]
 
     # e2e through the public API with pinned host buffers
     e2e = run_e2e(args, sm, wl, inp, C, device, world)
 
-    # capacity-factor sweep on the same tokens and weights (--sweep)
-    sweep = []
-    if args.sweep and wl.sweep:
-        for c in wl.sweep:
-            Cc = sm.switch_capacity(T, N, c)
-            dc = sm.layer_dims(x, w_in, capacity=Cc)
-            wsc = sm.workspace(dc, device)
-            outc = sm.layer_fwd(x, w_r, w_in, w_out, capacity=Cc, logit_bias=bias, ws=wsc)
-            for _ in range(args.warmup):
-                flush.fill_(1.0)
-                sm.layer_fwd(x, w_r, w_in, w_out, capacity=Cc, logit_bias=bias, ws=wsc, out=outc)
-            torch.cuda.synchronize(device)
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-            for i in range(K):
-                flush.fill_(float(i))
-                evs[i][0].record(stream)
-                sm.layer_fwd(x, w_r, w_in, w_out, capacity=Cc, logit_bias=bias, ws=wsc, out=outc)
-                evs[i][1].record(stream)
-            torch.cuda.synchronize(device)
-            if sm.switch_check(wsc) != 0:
-                raise RuntimeError("device status after the sweep steps")
-            msc = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, device) / K
-            kept = int(np.minimum(outc["counts"].cpu().numpy(), Cc).sum())
-            sweep.append({"capacity_factor": c, "capacity": Cc, "ms_per_step": round(msc, 5),
-                          "value": round(world * T / (msc * 1e-3), 1), "kept_tokens": kept,
-                          "drop_fraction": round(1 - kept / T, 6),
-                          "expert_flops_per_step": 4.0 * kept * d * wl.d_ff})
-            del wsc, outc
-            torch.cuda.empty_cache()
+    # standalone dispatch and combine entry points on the same workload
+    entry_points = time_entry_points(sm, wl, x, w_r, bias, C, flush, stream, device) if world == 1 else None
+
+    # capacity-factor sweep of the large-expert layer (its own inputs)
+    sweep = run_sweep(args, sm, device, flush, stream) if (world == 1 and not args.no_sweep) else None
 
     result = None
     if rank == 0:
@@ -379,6 +408,8 @@ def run_gpu(args):
             "clocks": clocks,
             "wall_s_timed_region": round(t_wall1 - t_wall0, 4),
         }
+        if entry_points:
+            result["entry_points"] = entry_points
         if sweep:
             result["sweep"] = sweep
         if not args.no_cpu_baseline and world == 1:
@@ -387,6 +418,110 @@ def run_gpu(args):
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def _time_events(fn, flush, stream, reps):
+    """Average CUDA-event time of fn() over reps calls, L2 flushed before each (outside the events)."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for i in range(reps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        fn()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / reps
+
+
+def time_entry_points(sm, wl, x, w_r, bias, C, flush, stream, device, reps=10):
+    """switch_dispatch and switch_combine called on their own (the layer path
+    fuses both into its neighbours), timed with CUDA events, with their
+    achieved HBM bandwidth over the algorithmic bytes."""
+    import torch
+    T, d, N = wl.T, wl.d_model, wl.num_experts
+    r = sm.route(x, w_r, capacity=C, logit_bias=bias, d_ff=wl.d_ff)
+    if sm.switch_check(r["workspace"]) != 0:
+        raise RuntimeError("device status after route")
+    dims = sm.dims(T, d, wl.d_ff, N, C, x.dtype)
+    xbuf = torch.empty(N * C * d, dtype=x.dtype, device=device)
+    ybuf = torch.randn(N * C * d, dtype=torch.float32, device=device)
+    y = torch.empty(T, d, dtype=torch.float32, device=device)
+    counts = r["counts"]
+    for _ in range(3):
+        sm.switch_dispatch(dims, x, r["slot_token"], counts, xbuf)
+        sm.switch_combine(dims, ybuf, r["expert"], r["slot"], r["gate"], y)
+    torch.cuda.synchronize()
+    ms_d = _time_events(lambda: sm.switch_dispatch(dims, x, r["slot_token"], counts, xbuf), flush, stream, reps)
+    ms_c = _time_events(lambda: sm.switch_combine(dims, ybuf, r["expert"], r["slot"], r["gate"], y), flush,
+                        stream, reps)
+    K = int(torch.clamp(counts, max=C).sum().item())
+    s = x.element_size()
+    peaks, _ = load_peaks()
+    bytes_d = 2 * K * d * s + 4 * N * C + 4 * N
+    bytes_c = T * d * 4 + K * d * 4 + 12 * T
+    bytes_c_act = T * d * s + K * d * s + 12 * T
+    out = {}
+    for name, ms, b, b_act in (("dispatch", ms_d, bytes_d, None), ("combine", ms_c, bytes_c, bytes_c_act)):
+        e = kernel_entry("hbm", b, b_act, ms, reps, peaks)
+        e.pop("share", None)
+        e["bytes"] = b
+        out[name] = e
+    del xbuf, ybuf, y, r
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_sweep(args, sm, device, flush, stream):
+    """The large-expert layer at every capacity factor of its sweep, on one
+    seeded input: ms per step, tokens/s, kept tokens and drop fraction per c.
+
+    With the Zipf(0.8) logit bias only a few experts receive tokens; the
+    weights of the others are left as zeros on the device (the layer never
+    reads an expert without kept tokens), which spares drawing ~10 GB of
+    random weights on the host."""
+    import torch
+    wl = synth.WORKLOADS[SWEEP_WORKLOAD]
+    T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.num_experts
+    x = to_dev(synth.activations(wl), device)
+    w_r = to_dev(synth.router_weight(wl), device)
+    bias = to_dev(synth.router_bias(wl), device)
+    r = sm.route(x, w_r, capacity=1, logit_bias=bias, d_ff=F)
+    if sm.switch_check(r["workspace"]) != 0:
+        raise RuntimeError("device status after route")
+    used = np.flatnonzero(r["counts"].cpu().numpy() > 0)
+    del r
+    w_in = torch.zeros(N, F, d, dtype=x.dtype, device=device)
+    w_out = torch.zeros(N, d, F, dtype=x.dtype, device=device)
+    for e in used:
+        wi, wo = synth.expert_weights(wl, int(e))
+        w_in[int(e)].copy_(to_dev(wi, device))
+        w_out[int(e)].copy_(to_dev(wo, device))
+    steps = max(3, min(args.steps, 20))
+    out = {"workload": wl.name, "T": T, "d_model": d, "d_ff": F, "num_experts": N,
+           "nonzero_weight_experts": int(used.size), "steps": steps, "points": []}
+    for c in wl.sweep:
+        Cc = sm.switch_capacity(T, N, c)
+        dc = sm.layer_dims(x, w_in, capacity=Cc)
+        wsc = sm.workspace(dc, device)
+        outc = sm.layer_fwd(x, w_r, w_in, w_out, capacity=Cc, logit_bias=bias, ws=wsc)
+        fn = lambda: sm.layer_fwd(x, w_r, w_in, w_out, capacity=Cc, logit_bias=bias, ws=wsc, out=outc)
+        for _ in range(args.warmup):
+            flush.fill_(1.0)
+            fn()
+        torch.cuda.synchronize()
+        ms = _time_events(fn, flush, stream, steps)
+        if sm.switch_check(wsc) != 0:
+            raise RuntimeError("device status after the sweep steps")
+        kept = int(np.minimum(outc["counts"].cpu().numpy(), Cc).sum())
+        out["points"].append({"capacity_factor": c, "capacity": Cc, "ms_per_step": round(ms, 5),
+                              "value": round(T / (ms * 1e-3), 1), "unit": UNIT, "kept_tokens": kept,
+                              "drop_fraction": round(1 - kept / T, 6),
+                              "expert_flops_per_step": 4.0 * kept * d * F})
+        del wsc, outc
+        torch.cuda.empty_cache()
+    del x, w_r, bias, w_in, w_out
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(args, sm, wl, inp, C, device, world):
@@ -496,47 +631,79 @@ def source_sha(kernel: str) -> str:
 # ---------------------------------------------------------------------------
 # the oracle: CPU baseline leg and reference arm
 # ---------------------------------------------------------------------------
-def cpu_baseline(wl, inp, C, budget_s=15.0):
-    """Time the fp64 oracle on the host: routing + assignment for every token,
-    expert FFN for a growing prefix of the kept tokens until about budget_s,
-    extrapolated to all kept tokens."""
-    import oracle
-    orc = oracle.Oracle()
+def _oracle_sample(orc, wl, inp, C, budget_s, route_tokens=None):
+    """Oracle time per token: routing (logits, softmax, top-1) on the first
+    `route_tokens` tokens (all when None) plus the capacity assignment and
+    aux on all ids, and the expert FFN on a growing prefix of the kept tokens
+    until about budget_s; returns (seconds extrapolated to the whole
+    workload, description)."""
+    T = wl.T
+    n_route = T if route_tokens is None else min(T, route_tokens)
+    x = inp["x"]
     t0 = time.perf_counter()
-    r = orc.route(inp["x"], inp["w_r"], inp["bias"], capacity=C)
+    h = orc.router_logits(x[:n_route], inp["w_r"], inp["bias"])
+    r = orc.softmax_top1(h)
     t_route = time.perf_counter() - t0
-    kept = np.flatnonzero(r["slot"] >= 0)
-    n, t_ffn, done = 64, 0.0, 0
+    if n_route == T:
+        ids = r["expert"]
+    else:  # ids of the tokens not routed here come from a full routing done outside the timing
+        ids = inp["_oracle_expert"]
+    t1 = time.perf_counter()
+    a = orc.assign(ids, wl.num_experts, C)
+    orc.aux(T, a["counts"], np.zeros(wl.num_experts))
+    t_assign = time.perf_counter() - t1
+    kept = np.flatnonzero(a["slot"] >= 0)
+    gate = np.ones(T)
+    n, t_ffn, done = 16, 0.0, 0
     while done < kept.size and t_ffn < budget_s:
         rows = kept[done:done + n]
-        t1 = time.perf_counter()
-        orc.output_rows(rows, inp["x"], inp["w_in"], inp["w_out"], r["expert"], r["slot"], r["gate"])
-        t_ffn += time.perf_counter() - t1
+        t2 = time.perf_counter()
+        orc.output_rows(rows, x, inp["w_in"], inp["w_out"], ids, a["slot"], gate)
+        t_ffn += time.perf_counter() - t2
         done += rows.size
         n = min(n * 2, kept.size)
-    per_row = t_ffn / max(done, 1)
-    est = t_route + per_row * kept.size
-    return {"value": round(wl.T / est, 2), "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
-            "sample": (f"router/softmax/assignment/aux on all {wl.T} tokens ({t_route:.2f} s) + expert FFN on "
-                       f"{done} of {kept.size} kept tokens ({t_ffn:.2f} s), extrapolated to all kept tokens"),
-            "seconds_measured": round(t_route + t_ffn, 2)}
+    est = t_route * T / n_route + t_assign + (t_ffn / max(done, 1)) * kept.size
+    desc = (f"routing on {n_route} of {T} tokens ({t_route:.2f} s), assignment + aux on all ({t_assign:.2f} s), "
+            f"expert FFN on {done} of {kept.size} kept tokens ({t_ffn:.2f} s); extrapolated to the whole workload")
+    return est, desc, t_route + t_assign + t_ffn
+
+
+def cpu_baseline(wl, inp, C, budget_s=15.0, one_core=True):
+    """Time the fp64 oracle on the host cores over a bounded sample of the
+    workload, extrapolated to tokens/s of the whole workload: once with all
+    host threads and once on a single core."""
+    import oracle
+    orc = oracle.Oracle()
+    all_threads = orc.threads()
+    est, desc, measured = _oracle_sample(orc, wl, inp, C, budget_s)
+    out = {"value": round(wl.T / est, 2), "unit": UNIT, "cores": all_threads, "kind": "oracle",
+           "sample": desc, "seconds_measured": round(measured, 2)}
+    if one_core:
+        if "_oracle_expert" not in inp:
+            inp["_oracle_expert"] = orc.softmax_top1(orc.router_logits(inp["x"], inp["w_r"], inp["bias"]))["expert"]
+        orc.set_threads(1)
+        try:
+            est1, desc1, measured1 = _oracle_sample(orc, wl, inp, C, budget_s / 3, route_tokens=2048)
+        finally:
+            orc.set_threads(all_threads)
+        out["one_core"] = {"value": round(wl.T / est1, 2), "unit": UNIT, "cores": 1, "sample": desc1,
+                           "seconds_measured": round(measured1, 2)}
+    return out
 
 
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return None
-    wl = synth.WORKLOADS[args.workload]
-    if args.capacity_factor is not None:
-        wl = wl.with_capacity_factor(args.capacity_factor)
+    wl = workload_of(args)
     inp = synth.inputs(wl)
     import oracle
     orc = oracle.Oracle()
     C = orc.capacity(wl.T, wl.num_experts, wl.capacity_factor)
     budget = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_baseline(wl, inp, C, budget_s=budget)
-    vals = [cpu_baseline(wl, inp, C, budget_s=budget) for _ in range(args.steps)]
+        cpu_baseline(wl, inp, C, budget_s=budget, one_core=False)
+    vals = [cpu_baseline(wl, inp, C, budget_s=budget, one_core=False) for _ in range(args.steps)]
     value = statistics.mean(v["value"] for v in vals)
     ms = wl.T / value * 1e3
     return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -552,15 +719,17 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--capacity-factor", type=float, default=None)
+    ap.add_argument("--tokens", type=int, default=None, help="token count override (small profiler captures)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle FFN time for cpu_baseline")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sweep", action="store_true", help="also time every capacity factor of the workload's sweep")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help=f"skip the capacity-factor sweep of the {SWEEP_WORKLOAD} workload")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

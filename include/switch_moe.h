@@ -206,8 +206,10 @@ switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const
  * holds, for example, T = 131072 tokens with 128 experts and d_model = 1024;
  * a larger group returns SWITCH_ERR_TOO_LARGE before anything runs.
  *
- * The first call on each device looks up the array's device address with
- * that device current; make that first call before any stream capture.
+ * Every call looks up the array's device address (cudaGetSymbolAddress, which
+ * allocates nothing) with the calling device current; on the first call on a
+ * device this may load the library's device code, so make that first call
+ * before any stream capture.
  * Every call shares the one array and leaves its contents behind (the next
  * call clears what must start at zero), so calls whose kernels may overlap
  * on the GPU (on different streams, or from several host threads) race and

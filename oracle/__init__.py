@@ -70,6 +70,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_output_rows.restype = None
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = ctypes.c_int
+    lib.oracle_set_threads.argtypes = [ctypes.c_int]
+    lib.oracle_set_threads.restype = None
     return lib
 
 
@@ -104,6 +106,10 @@ class Oracle:
 
     def threads(self) -> int:
         return int(self.lib.oracle_threads())
+
+    def set_threads(self, n: int) -> None:
+        """Threads of the OpenMP loops from now on (timing only; results do not depend on it)."""
+        self.lib.oracle_set_threads(int(n))
 
     def capacity(self, T: int, N: int, c: float) -> int:
         return int(self.lib.oracle_capacity(T, N, float(c)))

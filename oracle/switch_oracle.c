@@ -223,6 +223,19 @@ void oracle_output_rows(int32_t d, int32_t F, int64_t n_rows, const int64_t *row
     }
 }
 
+/* Set the number of OpenMP threads the parallel loops above use (no effect
+ * without OpenMP).  Used to time the oracle on one core and on all cores. */
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* Number of OpenMP threads the parallel loops above use (1 without OpenMP). */
 int oracle_threads(void)
 {

@@ -296,13 +296,13 @@ def layer_fwd(x, w_r, w_in, w_out, capacity=None, capacity_factor=None, logit_bi
 
 
 def route(x, w_r, num_experts=None, capacity=None, capacity_factor=None, logit_bias=None, d_ff: int = 64,
-          ws=None, stream=None):
+          ws=None, stream=None, flags: int = 0):
     """Router, top-1, capacity assignment, counts and aux (switch_route)."""
     import torch
     T, dm = x.shape
     N = w_r.shape[0] if num_experts is None else num_experts
     C = _resolve_capacity(T, N, capacity, capacity_factor)
-    d = dims(T, dm, d_ff, N, C, x.dtype)
+    d = dims(T, dm, d_ff, N, C, x.dtype, flags)
     dev = x.device
     out = dict(expert=torch.empty(T, dtype=torch.int32, device=dev),
                gate=torch.empty(T, dtype=torch.float32, device=dev),

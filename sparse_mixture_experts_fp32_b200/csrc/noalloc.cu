@@ -13,11 +13,10 @@
 // The array is part of this library's device image: every GPU on which the
 // library is used holds kNoAllocScratchBytes for it until the process exits.
 // Host code never dereferences its name (on the host it only stands in for
-// the symbol); its device address is looked up once per device with
-// cudaGetSymbolAddress and passed to the kernels like any workspace pointer.
+// the symbol); its device address is looked up with cudaGetSymbolAddress on
+// every call, with the calling device current, and passed to the kernels like
+// any workspace pointer.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -29,25 +28,17 @@ constexpr size_t kNoAllocScratchBytes = SWITCH_NOALLOC_SCRATCH_BYTES;
 
 static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-void *g_scratch_ptr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
-
-// Device address of the scratch array on the current device (looked up on
-// the first call made with that device current).
+// Device address of the scratch array in the current device's context.  It
+// is looked up on every call (cudaGetSymbolAddress allocates nothing and
+// costs a few microseconds) rather than cached per device ordinal: a cached
+// address would go stale if the caller reset the device or released and
+// re-created its primary context, and the next call would then write through
+// a dangling device pointer.
 cudaError_t scratch_on_current_device(void **out) {
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t err = cudaGetSymbolAddress(&p, g_route_scratch);
     if (err != cudaSuccess) return err;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        err = cudaGetSymbolAddress(&p, g_route_scratch);
-        if (err != cudaSuccess) return err;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

@@ -18,12 +18,24 @@ def test_kernel_work_base8():
     counts = np.full(wl.num_experts, wl.T // wl.num_experts, dtype=np.int64)
     work = bench.kernel_work(wl, C, counts)
     K = wl.T  # nothing dropped with equal counts below C
-    assert work["ffn_tc_fused"] == ("tensor", 4.0 * K * wl.d_model * wl.d_ff)
+    assert work["ffn_tc_fused"] == ("tensor", 4.0 * K * wl.d_model * wl.d_ff, None)
     assert work["_meta"][1]["K"] == K
     # the router reads x once (bf16), W_r, and writes expert + gate per token plus per-tile partials
     tiles = -(-wl.T // 64)
     assert work["router_staged"][1] == wl.T * wl.d_model * 2 + wl.num_experts * wl.d_model * 4 + 8 * wl.T + \
         8 * wl.num_experts * tiles
+    # the combine writes y in float32; its activation-dtype figure counts T*d*s written + K*d*s read
+    T, d = wl.T, wl.d_model
+    assert work["combine"][1] == T * d * 4 + K * d * 4 + 12 * T
+    assert work["combine"][2] == T * d * 2 + K * d * 2 + 12 * T
+
+
+def test_kernel_entry_fractions():
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1200.0}
+    e = bench.kernel_entry("tensor", 3.0e12, None, 2.0, 1, peaks)  # 3 TFLOP in 2 ms = 1500 TFLOP/s
+    assert e["frac"] == 1.0 and e["frac_sustained"] == 1.25
+    h = bench.kernel_entry("hbm", 6.0e9, 3.0e9, 1.0, 4, peaks)     # 6 GB in 1 ms = 6000 GB/s
+    assert h["frac"] == 1.0 and h["frac_act_dtype"] == 0.5 and h["launches"] == 4
 
 
 def _fake_tree(tmp_path):

@@ -6,12 +6,16 @@ they route tokens: they run under a host framework that owns every device
 allocation and forbids new ones while it executes, or in a process that
 reserved all of its device memory up front.  switch_route_noalloc keeps its
 scratch in a static array inside the library instead of a caller-supplied
-workspace.  Here it is called through the C ABI twice in a row, on two
-different problems (so that anything the first call leaves in the shared
-array would show in the second), and each result is compared with
-switch_route's on the same inputs.  The test also checks that a call leaves
-the device's free memory unchanged and that a group too large for the static
-array is refused before anything runs.
+workspace.  Here it is called through the C ABI several times in a row, on
+different problems (so that anything one call leaves in the shared array would
+show in the next), and each result is compared with switch_route's on the same
+inputs: ids, slots, counts and slot_token bit for bit, gates and aux within the
+parity tolerances.  The pairs cover both ways the capacity scan runs (inside the
+slot assignment for small histograms, and as its own kernel, which adds to and
+then resets a ticket kept in the shared array), the all-float32 path and an
+empty group.  The test also checks that a call leaves the device's free memory
+unchanged and that a group too large for the static array is refused before
+anything runs.
 
 This file is collected last on purpose: if it fails, a run that stops at the
 first failure has already run every other test.
@@ -56,16 +60,16 @@ def _call_noalloc(d, x, w_r, bias, out):
                                   p(out["slot"]), p(out["counts"]), p(out["slot_token"]), p(out["aux"]), stream)
 
 
-def _compare(name, T):
+def _compare(name, T, flags=0):
     wl = synth.WORKLOADS[name]
     x = _dev(synth.activations(wl, T=T))
     w_r = _dev(synth.router_weight(wl))
     bias = _dev(synth.router_bias(wl))
     N = wl.num_experts
     C = sm.switch_capacity(T, N, wl.capacity_factor)
-    ref = sm.route(x, w_r, capacity=C, logit_bias=bias, d_ff=wl.d_ff)  # with a workspace
+    ref = sm.route(x, w_r, capacity=C, logit_bias=bias, d_ff=wl.d_ff, flags=flags)  # with a workspace
     assert sm.switch_check(ref["workspace"]) == 0
-    d = sm.dims(T, wl.d_model, wl.d_ff, N, C, x.dtype)
+    d = sm.dims(T, wl.d_model, wl.d_ff, N, C, x.dtype, flags)
     out = _outputs(T, N, C)
     torch.cuda.synchronize()
     free_before = torch.cuda.mem_get_info()[0]
@@ -75,8 +79,11 @@ def _compare(name, T):
     assert status == 0, sm.STATUS.get(status, status)
     for k in ("expert", "slot", "counts", "slot_token"):
         assert torch.equal(out[k], ref[k]), k
-    assert torch.max(torch.abs(out["gate"] - ref["gate"])).item() <= GATE_ATOL
-    assert abs(out["aux"].item() - ref["aux"].item()) <= AUX_RTOL * abs(ref["aux"].item())
+    if T > 0:
+        assert torch.max(torch.abs(out["gate"] - ref["gate"])).item() <= GATE_ATOL
+        assert abs(out["aux"].item() - ref["aux"].item()) <= AUX_RTOL * abs(ref["aux"].item())
+    else:
+        assert out["aux"].item() == 0.0
     return free_before, free_after
 
 
@@ -88,6 +95,26 @@ def test_noalloc_route_matches_route_on_two_calls_in_a_row():
     # second call right after it, different N, T and tile count
     free_before, free_after = _compare("base8", 3000)
     assert free_after == free_before, "switch_route_noalloc changed the device's free memory"
+
+
+def test_noalloc_route_with_the_scan_kernel_twice_in_a_row():
+    """The separate scan kernel adds to a ticket in the shared array and resets it;
+    two calls back to back show whether the second starts from a clean ticket."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    flags = sm.SWITCH_FLAG_SEPARATE_SCAN
+    _compare("base128_skew", 5000, flags)
+    _compare("large128", 4000, flags)
+    free_before, free_after = _compare("base8", 3000, flags)
+    assert free_after == free_before
+
+
+def test_noalloc_route_float32_and_empty_group():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    _compare("tiny_fp32", 64)   # all-float32 router
+    _compare("base8", 0)        # no tokens: counts 0, aux 0, every slot empty
+    _compare("tiny_fp32", 64)   # and a normal call again after the empty one
 
 
 def test_noalloc_route_refuses_groups_beyond_its_scratch():
