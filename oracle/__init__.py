@@ -70,6 +70,12 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_output_rows.restype = None
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = ctypes.c_int
+    lib.oracle_softmax_top2.argtypes = [I64, I32, P, P, P, P, P, P]
+    lib.oracle_softmax_top2.restype = None
+    lib.oracle_assign_top2.argtypes = [I64, I32, I64, P, P, P, P, P]
+    lib.oracle_assign_top2.restype = None
+    lib.oracle_output_rows_top2.argtypes = [I32, I32, I64, P, P, ctypes.c_int, P, P, ctypes.c_int, P, P, P, P]
+    lib.oracle_output_rows_top2.restype = None
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_set_threads.restype = None
     return lib
@@ -186,6 +192,78 @@ class Oracle:
                                     _ptr(w_out), dtype_code(w_in), _ptr(expert), _ptr(slot), _ptr(gate),
                                     _ptr(y))
         return y
+
+    # ---- top-2 routing (the classic mixture-of-experts variant) ----------
+    def softmax_top2(self, h: np.ndarray, want_probs: bool = False) -> dict:
+        h = np.ascontiguousarray(h, dtype=np.float64)
+        T, N = h.shape
+        if N < 2:
+            raise ValueError("top-2 routing needs at least two experts")
+        expert = np.empty((T, 2), dtype=np.int32)
+        gate = np.empty((T, 2), dtype=np.float64)
+        margin = np.empty((T, 2), dtype=np.float64)
+        prob_sum = np.empty(N, dtype=np.float64)
+        probs = np.empty((T, N), dtype=np.float64) if want_probs else None
+        self.lib.oracle_softmax_top2(T, N, _ptr(h), _ptr(expert), _ptr(gate), _ptr(margin), _ptr(prob_sum),
+                                     _ptr(probs))
+        out = dict(expert=expert, gate=gate, margin=margin, prob_sum=prob_sum)
+        if want_probs:
+            out["probs"] = probs
+        return out
+
+    def assign_top2(self, expert: np.ndarray, N: int, C: int) -> dict:
+        expert = np.ascontiguousarray(expert, dtype=np.int32)
+        T = expert.shape[0]
+        assert expert.shape == (T, 2)
+        slot = np.empty((T, 2), dtype=np.int32)
+        counts = np.empty(N, dtype=np.int32)
+        counts_first = np.empty(N, dtype=np.int32)
+        slot_token = np.empty(N * C, dtype=np.int32)
+        self.lib.oracle_assign_top2(T, N, C, _ptr(expert), _ptr(slot), _ptr(counts), _ptr(counts_first),
+                                    _ptr(slot_token))
+        return dict(slot=slot, counts=counts, counts_first=counts_first, slot_token=slot_token.reshape(N, C))
+
+    def route_top2(self, x, w_r, bias=None, capacity: int | None = None, capacity_factor: float | None = None,
+                   want_probs: bool = False) -> dict:
+        """Router, top-2, capacity assignment and aux loss for all tokens."""
+        T = x.shape[0]
+        N = w_r.shape[0]
+        if capacity is None:
+            capacity = self.capacity(T, N, capacity_factor)
+        h = self.router_logits(x, w_r, bias)
+        r = self.softmax_top2(h, want_probs=want_probs)
+        a = self.assign_top2(r["expert"], N, capacity)
+        r.update(a)
+        r["logits"] = h
+        r["capacity"] = capacity
+        r["aux"] = self.aux(T, a["counts_first"], r["prob_sum"])
+        return r
+
+    def output_rows_top2(self, rows, x, w_in, w_out, expert, slot, gate) -> np.ndarray:
+        """Top-2 layer output rows (fp64) for the given token indices."""
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        x = np.ascontiguousarray(x)
+        T, d = x.shape
+        N, F, d2 = w_in.shape
+        assert d2 == d and w_out.shape == (N, d, F)
+        assert w_in.flags.c_contiguous and w_out.flags.c_contiguous and w_in.dtype == w_out.dtype
+        expert = np.ascontiguousarray(expert, dtype=np.int32)
+        slot = np.ascontiguousarray(slot, dtype=np.int32)
+        gate = np.ascontiguousarray(gate, dtype=np.float64)
+        assert expert.shape == (T, 2) and slot.shape == (T, 2) and gate.shape == (T, 2)
+        y = np.empty((rows.shape[0], d), dtype=np.float64)
+        self.lib.oracle_output_rows_top2(d, F, rows.shape[0], _ptr(rows), _ptr(x), dtype_code(x), _ptr(w_in),
+                                         _ptr(w_out), dtype_code(w_in), _ptr(expert), _ptr(slot), _ptr(gate),
+                                         _ptr(y))
+        return y
+
+    def layer_fwd_top2(self, x, w_r, w_in, w_out, bias=None, capacity=None, capacity_factor=None,
+                       want_probs: bool = False) -> dict:
+        """The whole top-2 layer for every token."""
+        r = self.route_top2(x, w_r, bias, capacity, capacity_factor, want_probs=want_probs)
+        rows = np.arange(x.shape[0], dtype=np.int64)
+        r["y"] = self.output_rows_top2(rows, x, w_in, w_out, r["expert"], r["slot"], r["gate"])
+        return r
 
     def expert_row(self, x_row, w_in_e, w_out_e, gate: float) -> np.ndarray:
         x_row = np.ascontiguousarray(x_row)

@@ -223,6 +223,140 @@ void oracle_output_rows(int32_t d, int32_t F, int64_t n_rows, const int64_t *row
     }
 }
 
+/* ------------------------------------------------------------------------
+ * Top-2 routing: the classic mixture-of-experts layer that the Switch layer
+ * simplifies (Incredible.AI "Switch Transformer - Scaling to Trillion
+ * Parameter Models", section "Mixture of Experts Routing"; llm-papers-study
+ * "精读 06 | Switch Transformers" §3.1): softmax over the N logits, the k = 2
+ * largest probabilities select the experts, and the output is the sum of the
+ * selected experts' outputs, each weighted by its own probability (no
+ * renormalisation over the selected pair):  y = sum_{i in top-2} p_i(x) E_i(x).
+ *
+ * Readings where the sources are silent:
+ *   - ties: the first choice is the lowest index attaining the largest
+ *     logit, the second the lowest index attaining the largest logit among
+ *     the other experts;
+ *   - capacity applies to (token, choice) assignments: each expert keeps its
+ *     first C assignments in the order "every first choice in token order,
+ *     then every second choice in token order", so that first choices get
+ *     exactly the slots of top-1 routing;
+ *   - the aux loss keeps its definition, f_i counting the tokens whose argmax
+ *     (first choice) is expert i (llm-papers-study §3.3).
+ * ------------------------------------------------------------------------ */
+
+/* Softmax and top-2 for every row of h[T,N] (N >= 2).
+ *   expert2[2t], expert2[2t+1] = first and second choice of token t
+ *   gate2[2t],   gate2[2t+1]   = their probabilities p[t, choice]
+ *   margin2[2t]   = largest logit minus the second largest (first choice gap)
+ *   margin2[2t+1] = second largest minus the third largest (+inf when N == 2)
+ *   prob_sum[i]   = sum over t of p[t,i], in token order
+ *   probs (optional, [T,N]) receives every p[t,i]. */
+void oracle_softmax_top2(int64_t T, int32_t N, const double *h, int32_t *expert2, double *gate2,
+                         double *margin2, double *prob_sum, double *probs)
+{
+    double *p = probs ? probs : (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * (size_t)N);
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const double *row = h + t * (int64_t)N;
+        int32_t first = 0;
+        for (int32_t i = 1; i < N; ++i)
+            if (row[i] > row[first])
+                first = i;
+        int32_t second = -1;
+        for (int32_t i = 0; i < N; ++i)
+            if (i != first && (second < 0 || row[i] > row[second]))
+                second = i;
+        double third = -INFINITY;
+        for (int32_t i = 0; i < N; ++i)
+            if (i != first && i != second && row[i] > third)
+                third = row[i];
+        double m = row[first];
+        double denom = 0.0;
+        for (int32_t j = 0; j < N; ++j)
+            denom += exp(row[j] - m);
+        for (int32_t j = 0; j < N; ++j)
+            p[t * (int64_t)N + j] = exp(row[j] - m) / denom;
+        expert2[2 * t] = first;
+        expert2[2 * t + 1] = second;
+        gate2[2 * t] = p[t * (int64_t)N + first];
+        gate2[2 * t + 1] = p[t * (int64_t)N + second];
+        margin2[2 * t] = row[first] - row[second];
+        margin2[2 * t + 1] = (N == 2) ? INFINITY : row[second] - third;
+    }
+    for (int32_t i = 0; i < N; ++i)
+        prob_sum[i] = 0.0;
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t i = 0; i < N; ++i)
+            prob_sum[i] += p[t * (int64_t)N + i];
+    if (!probs)
+        free(p);
+}
+
+/* Capacity assignment of top-2 choices.  Assignments are taken in the order
+ * (t = 0, first), (t = 1, first), ..., (t = T-1, first), (t = 0, second), ...,
+ * (t = T-1, second); each takes the next slot of its expert, or is dropped
+ * (slot -1) when the expert already holds C assignments.
+ *   counts[i]       = assignments routed to expert i over both choices,
+ *                     before capacity
+ *   counts_first[i] = tokens whose first choice is expert i
+ *   slot2[2t+c]     = slot of choice c of token t, or -1
+ *   slot_token[i*C+s] = the token holding slot s of expert i, -1 if empty. */
+void oracle_assign_top2(int64_t T, int32_t N, int64_t C, const int32_t *expert2, int32_t *slot2,
+                        int32_t *counts, int32_t *counts_first, int32_t *slot_token)
+{
+    for (int32_t i = 0; i < N; ++i) {
+        counts[i] = 0;
+        counts_first[i] = 0;
+    }
+    for (int64_t s = 0; s < (int64_t)N * C; ++s)
+        slot_token[s] = -1;
+    for (int c = 0; c < 2; ++c) {
+        for (int64_t t = 0; t < T; ++t) {
+            int32_t e = expert2[2 * t + c];
+            int32_t position = counts[e];
+            counts[e] = position + 1;
+            if (c == 0)
+                counts_first[e] += 1;
+            if (position < C) {
+                slot2[2 * t + c] = position;
+                slot_token[(int64_t)e * C + position] = (int32_t)t;
+            } else {
+                slot2[2 * t + c] = -1;
+            }
+        }
+    }
+}
+
+/* Top-2 layer outputs for a list of tokens: row r of y is
+ *   sum over the kept choices c of token rows[r] of gate2[2t+c] * E_{expert2[2t+c]}(x_t),
+ * first choice first, all in double; an all-zero row when both were dropped. */
+void oracle_output_rows_top2(int32_t d, int32_t F, int64_t n_rows, const int64_t *rows, const void *x,
+                             int x_dtype, const void *w_in, const void *w_out, int w_dtype,
+                             const int32_t *expert2, const int32_t *slot2, const double *gate2, double *y)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        int64_t t = rows[r];
+        double *out = y + r * (int64_t)d;
+        double *part = (double *)malloc(sizeof(double) * (size_t)d);
+        for (int32_t k = 0; k < d; ++k)
+            out[k] = 0.0;
+        size_t esize = (w_dtype == ORACLE_BF16) ? 2 : 4;
+        const char *x_t = (const char *)x + (size_t)t * (size_t)d * (x_dtype == ORACLE_BF16 ? 2 : 4);
+        for (int c = 0; c < 2; ++c) {
+            if (slot2[2 * t + c] < 0)
+                continue;
+            int64_t e = expert2[2 * t + c];
+            const char *win_e = (const char *)w_in + (size_t)e * (size_t)F * (size_t)d * esize;
+            const char *wout_e = (const char *)w_out + (size_t)e * (size_t)d * (size_t)F * esize;
+            oracle_expert_row(d, F, x_t, x_dtype, win_e, wout_e, w_dtype, gate2[2 * t + c], part);
+            for (int32_t k = 0; k < d; ++k)
+                out[k] += part[k];
+        }
+        free(part);
+    }
+}
+
 /* Set the number of OpenMP threads the parallel loops above use (no effect
  * without OpenMP).  Used to time the oracle on one core and on all cores. */
 void oracle_set_threads(int n)

@@ -346,4 +346,187 @@ def pin_expert_weight_layout(o):
     assert r["y"][0].tolist() == [3.0, 0.0, 0.0]
 
 
+# --------------------------------------------------------------------------
+# Top-2 routing (the classic mixture-of-experts variant)
+# --------------------------------------------------------------------------
+
+def _logits_of_probs(p):
+    """Logits whose softmax is the given row (a zero probability becomes a logit whose exponential is 0)."""
+    p = np.asarray(p, dtype=np.float64)
+    return np.where(p > 0, np.log(np.where(p > 0, p, 1.0)), -1000.0)
+
+
+def _top2_priority_definition(first, second, N, C):
+    """Set definition of the top-2 capacity step: the assignments (t, first_t) for
+    every t in token order, then (t, second_t) for every t; each expert keeps its
+    first C assignments of that list."""
+    T = len(first)
+    order = [(t, 0, first[t]) for t in range(T)] + [(t, 1, second[t]) for t in range(T)]
+    slot = np.full((T, 2), -1, dtype=np.int64)
+    holders = {e: [] for e in range(N)}
+    for t, c, e in order:
+        if len(holders[e]) < C:
+            slot[t, c] = len(holders[e])
+        holders[e].append(t)
+    counts = [len(holders[e]) for e in range(N)]
+    kept = {e: holders[e][:C] for e in range(N)}
+    return slot, counts, kept
+
+
+def pin_top2_p1_softmax_table(o):
+    g = golden("p1_top2_table.json")
+    h = _logits_of_probs(g["probs"])
+    r = o.softmax_top2(h, want_probs=True)
+    assert r["expert"][:, 0].tolist() == g["ours_first"]
+    assert r["expert"][:, 1].tolist() == g["ours_second"]
+    assert np.allclose(r["gate"], g["ours_gates"], rtol=0, atol=1e-15)
+    a = o.assign_top2(r["expert"], 4, g["capacity"])
+    assert a["slot"].tolist() == g["ours_slots"]
+    assert a["counts"].tolist() == g["ours_counts"]
+    assert a["counts_first"].tolist() == g["ours_counts_first"]
+    assert abs(o.aux(5, a["counts_first"], r["prob_sum"]) - g["derived_aux"]) < 1e-12
+
+
+def pin_top2_lps_hospital(o):
+    # Three experts with W_in = I and W_out = s_i I, so E_i(x) = s_i ReLU(x) tells
+    # the experts apart; logits ln p on one token give y = (0.6 s_0 + 0.3 s_1) ReLU(x).
+    g = golden("lps_top2_hospital.json")
+    p = np.array(g["probs"])
+    d = 3
+    x = np.array([[1.0, 2.0, -1.0]], dtype=np.float32)
+    scales = [1.0, 10.0, 100.0]
+    eye = np.eye(d, dtype=np.float32)
+    w_in = np.stack([eye] * 3)
+    w_out = np.stack([np.float32(s) * eye for s in scales])
+    # x has d = 3 features; W_r maps them to ln p: W_r[i] = ln(p_i) * e_0 / x[0]
+    w_r = np.zeros((3, d), dtype=np.float32)
+    w_r[:, 0] = np.log(p).astype(np.float32)
+    r = o.layer_fwd_top2(x, w_r, w_in, w_out, capacity=1)
+    assert r["expert"][0].tolist() == g["selected"]
+    assert np.allclose(r["gate"][0], g["weights"], atol=1e-7)
+    w0, w1 = r["gate"][0]
+    relu = np.maximum(x[0].astype(np.float64), 0.0)
+    assert np.allclose(r["y"][0], (w0 * scales[0] + w1 * scales[1]) * relu, rtol=1e-15, atol=0)
+    assert abs(r["y"][0][1] - 2.0 * (0.6 * 1.0 + 0.3 * 10.0)) < 1e-5
+
+
+def pin_top2_matches_argsort(o):
+    # Top-2 against numpy's stable descending sort (ties keep index order), the
+    # gates against scipy's softmax, the margins against the sorted logits.
+    rng = np.random.default_rng(20)
+    h = rng.standard_normal((80, 6)) * 2.0
+    h[:5] = np.round(h[:5])  # some exact ties
+    h[5] = [1.0, 1.0, 1.0, 0.0, 1.0, 0.0]
+    r = o.softmax_top2(h, want_probs=True)
+    order = np.argsort(-h, axis=1, kind="stable")
+    assert np.array_equal(r["expert"], order[:, :2])
+    ref = scipy.special.softmax(h, axis=1)
+    assert np.allclose(r["gate"], np.take_along_axis(ref, order[:, :2], axis=1), rtol=1e-13, atol=1e-15)
+    srt = -np.sort(-h, axis=1)
+    assert np.allclose(r["margin"][:, 0], srt[:, 0] - srt[:, 1], rtol=0, atol=1e-15)
+    assert np.allclose(r["margin"][:, 1], srt[:, 1] - srt[:, 2], rtol=0, atol=1e-15)
+    assert np.allclose(r["prob_sum"], ref.sum(axis=0), rtol=1e-13)
+
+
+def pin_top2_first_choice_is_top1(o):
+    # First choices, their gates, margins and slots are those of top-1 routing
+    # (first choices rank before every second choice), and aux is unchanged.
+    rng = np.random.default_rng(21)
+    x, w_r, bias, _, _ = _random_problem(rng, 200, 10, 4, 5)
+    for C in (7, 30, 200):
+        a = o.route(x, w_r, bias, capacity=C)
+        b = o.route_top2(x, w_r, bias, capacity=C)
+        assert np.array_equal(b["expert"][:, 0], a["expert"])
+        assert np.array_equal(b["gate"][:, 0], a["gate"])
+        assert np.array_equal(b["margin"][:, 0], a["margin"])
+        assert np.array_equal(b["slot"][:, 0], a["slot"])
+        assert np.array_equal(b["counts_first"], a["counts"])
+        assert b["aux"] == a["aux"]
+
+
+def pin_top2_brute_force_assignment(o):
+    # Every (first, second) choice with first != second for every token, every
+    # capacity, against the set definition of the priority order.
+    for T, N in [(4, 3), (3, 4)]:
+        pairs = [(a, b) for a in range(N) for b in range(N) if a != b]
+        for combo in itertools.product(pairs, repeat=T):
+            expert = np.array(combo, dtype=np.int32)
+            first, second = [c[0] for c in combo], [c[1] for c in combo]
+            for C in range(1, 2 * T + 1):
+                a = o.assign_top2(expert, N, C)
+                slot, counts, kept = _top2_priority_definition(first, second, N, C)
+                assert a["slot"].tolist() == slot.tolist(), (combo, C)
+                assert a["counts"].tolist() == counts
+                assert a["counts_first"].tolist() == np.bincount(first, minlength=N).tolist()
+                for e in range(N):
+                    assert a["slot_token"][e].tolist() == kept[e] + [-1] * (C - len(kept[e]))
+
+
+def pin_top2_dense_masked_formulation(o):
+    # numpy: every expert on every token, the two largest probabilities (stable
+    # sort), the priority-list capacity, then the probability-weighted sum.
+    for seed, (T, d, F, N, C) in enumerate([(40, 8, 16, 4, 12), (30, 6, 10, 3, 9), (25, 4, 8, 5, 50)]):
+        rng = np.random.default_rng(120 + seed)
+        x, w_r, bias, w_in, w_out = _random_problem(rng, T, d, F, N)
+        r = o.layer_fwd_top2(x, w_r, w_in, w_out, bias=bias, capacity=C)
+        x64 = x.astype(np.float64)
+        h = x64 @ w_r.astype(np.float64).T + bias.astype(np.float64)
+        p = scipy.special.softmax(h, axis=1)
+        order = np.argsort(-h, axis=1, kind="stable")[:, :2]
+        slot, _, _ = _top2_priority_definition(order[:, 0].tolist(), order[:, 1].tolist(), N, C)
+        every = np.stack([np.maximum(x64 @ w_in[i].astype(np.float64).T, 0) @ w_out[i].astype(np.float64).T
+                          for i in range(N)])
+        y = np.zeros((T, d))
+        for t in range(T):
+            for c in range(2):
+                if slot[t, c] >= 0:
+                    e = order[t, c]
+                    y[t] += p[t, e] * every[e, t]
+        assert np.array_equal(r["expert"], order)
+        assert np.array_equal(r["slot"], slot)
+        assert np.allclose(r["y"], y, rtol=1e-12, atol=1e-13), np.abs(r["y"] - y).max()
+        f = np.bincount(order[:, 0], minlength=N) / T
+        assert abs(r["aux"] - N * np.dot(f, p.mean(axis=0))) < 1e-12
+
+
+def pin_top2_two_experts_dense_mixture(o):
+    # N = 2 and C = T: every token uses both experts and nothing is dropped, so
+    # the layer is the full softmax mixture p_0 E_0(x) + p_1 E_1(x) (closed form).
+    rng = np.random.default_rng(22)
+    T, d, F = 24, 6, 9
+    x, w_r, bias, w_in, w_out = _random_problem(rng, T, d, F, 2)
+    r = o.layer_fwd_top2(x, w_r, w_in, w_out, bias=bias, capacity=T)
+    x64 = x.astype(np.float64)
+    p = scipy.special.softmax(x64 @ w_r.astype(np.float64).T + bias.astype(np.float64), axis=1)
+    mix = sum(p[:, [i]] * (np.maximum(x64 @ w_in[i].astype(np.float64).T, 0) @ w_out[i].astype(np.float64).T)
+              for i in range(2))
+    assert np.all(r["slot"] >= 0)
+    assert r["counts"].tolist() == [T, T]
+    assert np.allclose(r["y"], mix, rtol=1e-12, atol=1e-13)
+    assert np.all(np.isinf(r["margin"][:, 1]))
+
+
+def pin_top2_invariants(o):
+    rng = np.random.default_rng(23)
+    T, d, F, N = 300, 12, 20, 7
+    x, w_r, bias, w_in, w_out = _random_problem(rng, T, d, F, N)
+    r = o.layer_fwd_top2(x, w_r, w_in, w_out, bias=bias, capacity_factor=1.5, want_probs=True)
+    C = r["capacity"]
+    assert C == 65
+    assert int(r["counts"].sum()) == 2 * T and int(r["counts_first"].sum()) == T
+    assert np.all(r["expert"][:, 0] != r["expert"][:, 1])
+    assert np.all(r["gate"][:, 0] >= r["gate"][:, 1]) and np.all(r["gate"].sum(axis=1) <= 1.0 + 1e-15)
+    assert np.all(r["margin"] >= 0)
+    kept = np.minimum(r["counts"], C)
+    for e in range(N):
+        mask = (r["expert"] == e) & (r["slot"] >= 0)
+        assert int(mask.sum()) == kept[e]
+        assert sorted(r["slot"][mask].tolist()) == list(range(kept[e]))
+        for t, c in zip(*np.nonzero(mask)):
+            assert r["slot_token"][e][r["slot"][t, c]] == t
+        assert np.all(r["slot_token"][e][kept[e]:] == -1)
+    both_dropped = (r["slot"] < 0).all(axis=1)
+    assert np.all(r["y"][both_dropped] == 0.0)
+
+
 PINS = {name: fn for name, fn in sorted(globals().items()) if name.startswith("pin_") and callable(fn)}

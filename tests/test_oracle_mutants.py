@@ -47,6 +47,28 @@ MUTANTS = {
     "ffn_w_in_transposed": ("load_elem(w_in, w_dtype, (int64_t)j * d + k)", "load_elem(w_in, w_dtype, (int64_t)k * F + j)"),
     "ffn_gate_missing": ("y_row[k] = gate * acc;", "y_row[k] = acc;"),
     "dropped_token_not_zeroed": ("if (slot[t] < 0) {", "if (slot[t] < -1) {"),
+    # top-2: second choice on ties goes to the highest index; may repeat the first choice
+    "top2_second_ties_last": ("if (i != first && (second < 0 || row[i] > row[second]))",
+                              "if (i != first && (second < 0 || row[i] >= row[second]))"),
+    "top2_second_may_be_first": ("if (i != first && (second < 0 || row[i] > row[second]))",
+                                 "if ((second < 0 || row[i] > row[second]))"),
+    # top-2 gates renormalised over the selected pair
+    "top2_gate_renormalised": ("gate2[2 * t] = p[t * (int64_t)N + first];",
+                               "gate2[2 * t] = p[t * (int64_t)N + first] / (p[t * (int64_t)N + first] + "
+                               "p[t * (int64_t)N + second]);"),
+    "top2_margin_second_wrong": ("margin2[2 * t + 1] = (N == 2) ? INFINITY : row[second] - third;",
+                                 "margin2[2 * t + 1] = (N == 2) ? INFINITY : row[first] - third;"),
+    "top2_softmax_denominator_missing_term": ("for (int32_t j = 0; j < N; ++j)\n            denom += exp(row[j] - m);",
+                                              "for (int32_t j = 1; j < N; ++j)\n            denom += exp(row[j] - m);"),
+    # top-2 capacity: token-major priority instead of first choices first
+    "top2_token_major_priority": ("for (int c = 0; c < 2; ++c) {\n        for (int64_t t = 0; t < T; ++t) {",
+                                  "for (int64_t t = 0; t < T; ++t) {\n        for (int c = 0; c < 2; ++c) {"),
+    # aux fed with the counts of both choices
+    "top2_first_counts_both_choices": ("if (c == 0)\n                counts_first[e] += 1;",
+                                       "counts_first[e] += 1;"),
+    # top-2 output: second choice never added
+    "top2_output_first_only": ("for (int c = 0; c < 2; ++c) {\n            if (slot2[2 * t + c] < 0)",
+                               "for (int c = 0; c < 1; ++c) {\n            if (slot2[2 * t + c] < 0)"),
     # bf16 loads: wrong half of the 32-bit pattern
     "bf16_wrong_shift": ("uint32_t wide = (uint32_t)bits << 16;", "uint32_t wide = (uint32_t)bits << 15;"),
 }
