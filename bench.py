@@ -22,6 +22,7 @@ The JSON line also carries:
                 with those rows counted at the activation dtype
   e2e           the same metric through the public API with pinned host
                 buffers: x copied in and y/aux/counts copied out every step
+  top2          the top-2 variant (switch_layer_fwd_top2) on the same tensors
   entry_points  switch_dispatch and switch_combine called on their own
   sweep         the large-expert layer at every capacity factor of its sweep
                 (drop fraction and tokens/s per c)
@@ -265,7 +266,7 @@ def run_gpu(args):
     bias = to_dev(inp["bias"], device)
     w_in = to_dev(inp["w_in"], device)
     w_out = to_dev(inp["w_out"], device)
-    dims = sm.layer_dims(x, w_in, capacity=C)
+    dims = sm.layer_dims(x, w_in, capacity=C, flags=args.flags)
     ws = sm.workspace(dims, device)
     T, d, N = wl.T, wl.d_model, wl.num_experts
     out = dict(y=torch.empty(T, d, dtype=torch.float32, device=device),
@@ -380,6 +381,10 @@ def run_gpu(args):
     # e2e through the public API with pinned host buffers
     e2e = run_e2e(args, sm, wl, inp, C, device, world)
 
+    # the top-2 variant of the layer on the same tokens and weights
+    top2 = time_top2(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, device) \
+        if (world == 1 and not args.no_top2 and wl.num_experts >= 2) else None
+
     # standalone dispatch and combine entry points on the same workload
     entry_points = time_entry_points(sm, wl, x, w_r, bias, C, flush, stream, device) if world == 1 else None
 
@@ -399,7 +404,8 @@ def run_gpu(args):
                        "experts": wl.dtype, "kept_tokens": meta["K"], "nonempty_experts": meta["E_nz"],
                        "drop_fraction": round(1 - meta["K"] / T, 6),
                        "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the events)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       **({"flags": args.flags} if args.flags else {})},
             "roofline": roofline,
             "kernels": kernels,
             "gpu_launches": int(launches),
@@ -408,6 +414,8 @@ def run_gpu(args):
             "clocks": clocks,
             "wall_s_timed_region": round(t_wall1 - t_wall0, 4),
         }
+        if top2:
+            result["top2"] = top2
         if entry_points:
             result["entry_points"] = entry_points
         if sweep:
@@ -431,6 +439,59 @@ def _time_events(fn, flush, stream, reps):
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     return sum(a.elapsed_time(b) for a, b in evs) / reps
+
+
+def time_top2(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, device):
+    """The top-2 layer (switch_layer_fwd_top2) on the workload's tensors: ms per
+    step, tokens/s and each kernel's fraction of its roofline."""
+    import torch
+    T = wl.T
+    out = sm.layer_fwd_top2(x, w_r, w_in, w_out, capacity=C, logit_bias=bias)
+    ws = out["workspace"]
+    fn = lambda: sm.layer_fwd_top2(x, w_r, w_in, w_out, capacity=C, logit_bias=bias, ws=ws, out=out)
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        fn()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 20))
+    ms = _time_events(fn, flush, stream, steps)
+    sm.trace_start(steps * 8)
+    _time_events(fn, flush, stream, steps)
+    trace = sm.trace_read(steps * 8)
+    sm.trace_stop()
+    if sm.switch_check(ws) != 0:
+        raise RuntimeError("device status after the top-2 steps")
+    counts = out["counts"].cpu().numpy()
+    kept = np.minimum(counts, C)
+    K = int(kept.sum())
+    s = x.element_size()
+    d, F, N = wl.d_model, wl.d_ff, wl.num_experts
+    tiles = -(-T // 64)
+    work = {
+        "router_tc": ("hbm", T * d * s + 3 * N * d * 2 + 16 * T + 12 * N * tiles, None),
+        "router_staged": ("hbm", T * d * s + 4 * N * d + 16 * T + 12 * N * tiles, None),
+        "router_tiled": ("hbm", T * d * s + 4 * N * d + 16 * T + 12 * N * tiles, None),
+        "router_weight_split": ("hbm", N * d * 4 + 3 * N * d * 2, None),
+        "capacity_scan": ("hbm", 20 * N * tiles + 12 * N, None),
+        "slot_assign_scatter": ("hbm", 16 * T + 8 * N * tiles + 4 * N * C + 2 * K * d * s, None),
+        "ffn_tc_gemm1_relu": ("tensor", 2.0 * K * d * F, None),
+        "ffn_tc_gemm2": ("tensor", 2.0 * K * F * d, None),
+        "combine_top2": ("hbm", T * d * 4 + K * d * 4 + 24 * T, T * d * s + K * d * s + 24 * T),
+    }
+    peaks, _ = load_peaks()
+    per_kernel: dict[str, list[float]] = {}
+    for name, kms in trace:
+        per_kernel.setdefault(name, []).append(kms)
+    kernels = {}
+    for name, times in per_kernel.items():
+        kind, amount, amount_act = work.get(name, ("?", 0, None))
+        kernels[name] = kernel_entry(kind, amount, amount_act, statistics.mean(times), len(times) // steps, peaks)
+    result = {"ms_per_step": round(ms, 5), "value": round(T / (ms * 1e-3), 1), "unit": UNIT, "steps": steps,
+              "capacity": C, "kept_assignments": K, "dropped_assignments": int(2 * T - K),
+              "expert_flops_per_step": 4.0 * K * d * F, "kernels": kernels}
+    del out, ws
+    torch.cuda.empty_cache()
+    return result
 
 
 def time_entry_points(sm, wl, x, w_r, bias, C, flush, stream, device, reps=10):
@@ -724,10 +785,12 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--capacity-factor", type=float, default=None)
     ap.add_argument("--tokens", type=int, default=None, help="token count override (small profiler captures)")
+    ap.add_argument("--flags", type=int, default=0, help="SWITCH_FLAG_* bits for the timed layer (diagnostic paths)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle FFN time for cpu_baseline")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-top2", action="store_true", help="skip timing the top-2 variant of the layer")
     ap.add_argument("--no-sweep", action="store_true",
                     help=f"skip the capacity-factor sweep of the {SWEEP_WORKLOAD} workload")
     args = ap.parse_args(argv)

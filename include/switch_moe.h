@@ -190,6 +190,57 @@ switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const
                                  int32_t *expert, float *gate, int32_t *slot, int32_t *counts, float *aux,
                                  void *workspace, size_t workspace_bytes, switch_stream_t stream);
 
+/* ---- top-2 routing ------------------------------------------------------
+ * The classic mixture-of-experts layer that Switch routing simplifies
+ * (Incredible.AI "Switch Transformer - Scaling to Trillion Parameter Models",
+ * section "Mixture of Experts Routing"; llm-papers-study "精读 06 | Switch
+ * Transformers" §3.1, y = sum over the top-K experts of p_i(x) E_i(x), with
+ * K = 2): the two largest softmax probabilities select two experts, and each
+ * selected expert's output is weighted by its own probability (no
+ * renormalisation over the pair).  Requires N >= 2.  Readings where the
+ * sources are silent:
+ *  - the first choice is the lowest index of the largest logit, the second
+ *    the lowest index of the largest logit among the other experts;
+ *  - capacity C applies to (token, choice) assignments; every first choice
+ *    (in token order) ranks before every second choice (in token order), so
+ *    first choices get exactly the slots of top-1 routing;
+ *  - the aux loss keeps its definition: f_i counts first choices only.
+ * Per-token arrays are [T][2]: element 2t is the first choice of token t,
+ * element 2t + 1 its second choice.  The workspace is the one of
+ * switch_workspace_size(dims). */
+
+/* Router, top-2, capacity assignment, counts and aux.
+ *   expert [T][2] int32, gate [T][2] float32 (p of each choice),
+ *   slot [T][2] int32 (-1 = that choice was dropped),
+ *   counts [N] int32: (token, choice) assignments per expert over both
+ *   choices, before capacity; slot_token [N * C] int32 (-1 = empty);
+ *   aux [1] float32 = N * sum_i (first choices of i / T) * (mean_t p_i).
+ * Errors as switch_route, plus SWITCH_ERR_SHAPE when N < 2.  Deterministic. */
+switch_status_t switch_route_top2(const switch_dims_t *dims, const void *x, const float *w_r,
+                                  const float *logit_bias, int32_t *expert, float *gate, int32_t *slot,
+                                  int32_t *counts, int32_t *slot_token, float *aux, void *workspace,
+                                  size_t workspace_bytes, switch_stream_t stream);
+
+/* Top-2 combine:  y[t, :] = sum over the kept choices c of token t of
+ *   gate[2t+c] * ybuf[expert[2t+c], slot[2t+c], :]
+ * in float32, the first choice's product first, then the second's added
+ * (each product and the sum rounded to float32); an all-zero row when both
+ * choices were dropped.  ybuf [N, C, d] float32 -> y [T, d] float32.
+ * (switch_dispatch and switch_expert_ffn serve top-2 routing unchanged: they
+ * work from slot_token and counts.) */
+switch_status_t switch_combine_top2(const switch_dims_t *dims, const void *ybuf, const int32_t *expert,
+                                    const int32_t *slot, const float *gate, void *y, switch_stream_t stream);
+
+/* The whole top-2 layer: switch_route_top2 (with both choices' rows of x
+ * copied into the workspace's per-expert buffers by the slot assignment), the
+ * expert FFN into the workspace's float32 ybuf, then switch_combine_top2.
+ * Arguments as switch_layer_fwd, with expert, gate and slot of shape [T][2].
+ * Identical inputs give identical bytes. */
+switch_status_t switch_layer_fwd_top2(const switch_dims_t *dims, const void *x, const float *w_r,
+                                      const float *logit_bias, const void *w_in, const void *w_out, void *y,
+                                      int32_t *expert, float *gate, int32_t *slot, int32_t *counts, float *aux,
+                                      void *workspace, size_t workspace_bytes, switch_stream_t stream);
+
 /* Routing without a workspace, for callers that cannot allocate device
  * memory at the point where they route tokens: code running under a host
  * framework that owns every device allocation and forbids new ones while it

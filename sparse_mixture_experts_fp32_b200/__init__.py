@@ -40,7 +40,8 @@ STATUS = {
 
 EXPORTED = ("switch_capacity", "switch_workspace_size", "switch_route", "switch_route_noalloc", "switch_dispatch",
             "switch_expert_ffn",
-            "switch_combine", "switch_layer_fwd", "switch_check", "switch_selftest_wait_timeout", "switch_status_string",
+            "switch_combine", "switch_layer_fwd", "switch_route_top2", "switch_combine_top2", "switch_layer_fwd_top2",
+            "switch_check", "switch_selftest_wait_timeout", "switch_status_string",
             "switch_launch_count",
             "switch_trace_start", "switch_trace_read", "switch_trace_stop", "switch_kernel_name")
 
@@ -84,6 +85,9 @@ def lib() -> ctypes.CDLL:
         "switch_expert_ffn": (I, [D, P, P, P, P, P, P, S, P]),
         "switch_combine": (I, [D, P, P, P, P, P, P]),
         "switch_layer_fwd": (I, [D, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
+        "switch_route_top2": (I, [D, P, P, P, P, P, P, P, P, P, P, S, P]),
+        "switch_combine_top2": (I, [D, P, P, P, P, P, P]),
+        "switch_layer_fwd_top2": (I, [D, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
         "switch_check": (I, [P, S, P]),
         "switch_selftest_wait_timeout": (I, [P, S, P]),
         "switch_status_string": (ctypes.c_char_p, [I]),
@@ -204,6 +208,26 @@ def switch_layer_fwd(d, x, w_r, logit_bias, w_in, w_out, y, expert, gate, slot, 
                                _stream(stream, workspace)), "switch_layer_fwd")
 
 
+def switch_route_top2(d, x, w_r, logit_bias, expert, gate, slot, counts, slot_token, aux, workspace, stream=None):
+    _ok(lib().switch_route_top2(ctypes.byref(d), _ptr(x), _ptr(w_r), _ptr(logit_bias), _ptr(expert), _ptr(gate),
+                                _ptr(slot), _ptr(counts), _ptr(slot_token), _ptr(aux), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream, workspace)),
+        "switch_route_top2")
+
+
+def switch_combine_top2(d, ybuf, expert, slot, gate, y, stream=None):
+    _ok(lib().switch_combine_top2(ctypes.byref(d), _ptr(ybuf), _ptr(expert), _ptr(slot), _ptr(gate), _ptr(y),
+                                  _stream(stream, ybuf)), "switch_combine_top2")
+
+
+def switch_layer_fwd_top2(d, x, w_r, logit_bias, w_in, w_out, y, expert, gate, slot, counts, aux, workspace,
+                          stream=None):
+    _ok(lib().switch_layer_fwd_top2(ctypes.byref(d), _ptr(x), _ptr(w_r), _ptr(logit_bias), _ptr(w_in), _ptr(w_out),
+                                    _ptr(y), _ptr(expert), _ptr(gate), _ptr(slot), _ptr(counts), _ptr(aux),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream, workspace)), "switch_layer_fwd_top2")
+
+
 def switch_check(workspace, stream=None) -> int:
     """Synchronise and return the device status code (0 = ok); does not raise."""
     return int(lib().switch_check(_ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -314,6 +338,53 @@ def route(x, w_r, num_experts=None, capacity=None, capacity_factor=None, logit_b
         ws = workspace(d, dev)
     switch_route(d, x, w_r, logit_bias, out["expert"], out["gate"], out["slot"], out["counts"], out["slot_token"],
                  out["aux"], ws, stream)
+    out["capacity"] = C
+    out["workspace"] = ws
+    return out
+
+
+def layer_fwd_top2(x, w_r, w_in, w_out, capacity=None, capacity_factor=None, logit_bias=None, flags: int = 0,
+                   ws=None, out=None, stream=None):
+    """The top-2 mixture-of-experts layer forward pass.  Returns a dict with
+    y [T, d] float32, aux, expert / gate / slot [T, 2], counts [N]."""
+    import torch
+    d = layer_dims(x, w_in, capacity, capacity_factor, flags)
+    T, dev = x.shape[0], x.device
+    if out is None:
+        out = dict(y=torch.empty(x.shape, dtype=torch.float32, device=dev),
+                   expert=torch.empty(T, 2, dtype=torch.int32, device=dev),
+                   gate=torch.empty(T, 2, dtype=torch.float32, device=dev),
+                   slot=torch.empty(T, 2, dtype=torch.int32, device=dev),
+                   counts=torch.empty(d.num_experts, dtype=torch.int32, device=dev),
+                   aux=torch.empty(1, dtype=torch.float32, device=dev))
+    if ws is None:
+        ws = workspace(d, dev)
+    switch_layer_fwd_top2(d, x, w_r, logit_bias, w_in, w_out, out["y"], out["expert"], out["gate"], out["slot"],
+                          out["counts"], out["aux"], ws, stream)
+    out["capacity"] = d.capacity
+    out["workspace"] = ws
+    return out
+
+
+def route_top2(x, w_r, capacity=None, capacity_factor=None, logit_bias=None, d_ff: int = 64, ws=None, stream=None,
+               flags: int = 0):
+    """Router, top-2, capacity assignment, counts and aux (switch_route_top2)."""
+    import torch
+    T, dm = x.shape
+    N = w_r.shape[0]
+    C = _resolve_capacity(T, N, capacity, capacity_factor)
+    d = dims(T, dm, d_ff, N, C, x.dtype, flags)
+    dev = x.device
+    out = dict(expert=torch.empty(T, 2, dtype=torch.int32, device=dev),
+               gate=torch.empty(T, 2, dtype=torch.float32, device=dev),
+               slot=torch.empty(T, 2, dtype=torch.int32, device=dev),
+               counts=torch.empty(N, dtype=torch.int32, device=dev),
+               slot_token=torch.empty(N * C, dtype=torch.int32, device=dev),
+               aux=torch.empty(1, dtype=torch.float32, device=dev))
+    if ws is None:
+        ws = workspace(d, dev)
+    switch_route_top2(d, x, w_r, logit_bias, out["expert"], out["gate"], out["slot"], out["counts"],
+                      out["slot_token"], out["aux"], ws, stream)
     out["capacity"] = C
     out["workspace"] = ws
     return out

@@ -25,7 +25,8 @@ size_t elem_size(const switch_dims_t &d) { return d.dtype == SWITCH_BF16 ? 2 : 4
 int64_t tiles_of(const switch_dims_t &d) { return (d.T + kTileT - 1) / kTileT; }
 
 struct Sections {
-    size_t status, ticket, hist, psum, tile_off, prob_total, w_split, slot_token, xbuf, ybuf, hidden, done, total;
+    size_t status, ticket, hist, psum, tile_off, prob_total, w_split, slot_token, xbuf, ybuf, hidden, done, hist2,
+        tile_off2, counts_first, total;
 };
 
 Sections layout(const switch_dims_t &d) {
@@ -49,6 +50,10 @@ Sections layout(const switch_dims_t &d) {
     s.ybuf = take(N * C * (size_t)d.d_model * sizeof(float));
     s.hidden = take(N * C * (size_t)d.d_ff * elem_size(d));
     s.done = take(fused_counter_ints(N, C, d.d_model) * sizeof(int32_t));  // the fused FFN's counters
+    // top-2 routing only; after everything top-1 routing uses
+    s.hist2 = take(N * tiles * 4);
+    s.tile_off2 = take(N * tiles * 4);
+    s.counts_first = take(N * 4);
     s.total = off;
     return s;
 }
@@ -165,6 +170,9 @@ Workspace carve_workspace(const switch_dims_t &dims, void *base) {
     w.ybuf = reinterpret_cast<float *>(b + s.ybuf);
     w.hidden = b + s.hidden;
     w.done = reinterpret_cast<int32_t *>(b + s.done);
+    w.hist2 = reinterpret_cast<int32_t *>(b + s.hist2);
+    w.tile_off2 = reinterpret_cast<int32_t *>(b + s.tile_off2);
+    w.counts_first = reinterpret_cast<int32_t *>(b + s.counts_first);
     w.tiles = tiles_of(dims);
     return w;
 }
@@ -310,6 +318,74 @@ switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const
     return from_cuda(err);
 }
 
+switch_status_t switch_route_top2(const switch_dims_t *dims, const void *x, const float *w_r,
+                                  const float *logit_bias, int32_t *expert, float *gate, int32_t *slot,
+                                  int32_t *counts, int32_t *slot_token, float *aux, void *workspace,
+                                  size_t workspace_bytes_given, switch_stream_t stream) {
+    switch_status_t s = check_dims(dims);
+    if (s != SWITCH_OK) return s;
+    if (dims->num_experts < 2) return SWITCH_ERR_SHAPE;
+    const bool has_tokens = dims->T > 0;
+    s = check_ptrs({w_r, counts, slot_token, aux, workspace,
+                    has_tokens ? x : w_r, has_tokens ? (const void *)expert : w_r,
+                    has_tokens ? (const void *)gate : w_r, has_tokens ? (const void *)slot : w_r},
+                   {logit_bias, x, expert, gate, slot});
+    if (s != SWITCH_OK) return s;
+    if (workspace_bytes_given < workspace_bytes(*dims)) return SWITCH_ERR_WORKSPACE;
+    if ((s = check_device()) != SWITCH_OK) return s;
+    const Workspace ws = carve_workspace(*dims, workspace);
+    return from_cuda(launch_route(*dims, x, w_r, logit_bias, expert, gate, slot, counts, slot_token, aux, ws,
+                                  reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr, 0, true));
+}
+
+switch_status_t switch_combine_top2(const switch_dims_t *dims, const void *ybuf, const int32_t *expert,
+                                    const int32_t *slot, const float *gate, void *y, switch_stream_t stream) {
+    switch_status_t s = check_dims(dims);
+    if (s != SWITCH_OK) return s;
+    if (dims->num_experts < 2) return SWITCH_ERR_SHAPE;
+    if (dims->T > 0) {
+        s = check_ptrs({ybuf, expert, slot, gate, y}, {});
+        if (s != SWITCH_OK) return s;
+    }
+    if ((s = check_device()) != SWITCH_OK) return s;
+    return from_cuda(launch_combine_top2(*dims, static_cast<const float *>(ybuf), expert, slot, gate,
+                                         static_cast<float *>(y), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+switch_status_t switch_layer_fwd_top2(const switch_dims_t *dims, const void *x, const float *w_r,
+                                      const float *logit_bias, const void *w_in, const void *w_out, void *y,
+                                      int32_t *expert, float *gate, int32_t *slot, int32_t *counts, float *aux,
+                                      void *workspace, size_t workspace_bytes_given, switch_stream_t stream) {
+    switch_status_t s = check_dims(dims);
+    if (s != SWITCH_OK) return s;
+    if (dims->num_experts < 2) return SWITCH_ERR_SHAPE;
+    const bool has_tokens = dims->T > 0;
+    s = check_ptrs({w_r, w_in, w_out, counts, aux, workspace, has_tokens ? x : w_r, has_tokens ? y : w_r,
+                    has_tokens ? (const void *)expert : w_r, has_tokens ? (const void *)gate : w_r,
+                    has_tokens ? (const void *)slot : w_r},
+                   {logit_bias, x, y, expert, gate, slot});
+    if (s != SWITCH_OK) return s;
+    if (workspace_bytes_given < workspace_bytes(*dims)) return SWITCH_ERR_WORKSPACE;
+    if ((s = check_device()) != SWITCH_OK) return s;
+    const Workspace ws = carve_workspace(*dims, workspace);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool tensor_cores = dims->dtype == SWITCH_BF16 && !(dims->flags & SWITCH_FLAG_SIMT_FFN);
+    const bool rows16 = ((int64_t)dims->d_model * (int64_t)elem_size(*dims)) % 16 == 0;
+    // route (+ scatter-dispatch of both choices), expert FFN into ybuf, top-2 combine
+    cudaError_t err = launch_route(*dims, x, w_r, logit_bias, expert, gate, slot, counts, ws.slot_token, aux, ws, st,
+                                   rows16 ? ws.xbuf : nullptr, nullptr, nullptr, 0, true);
+    if (err == cudaSuccess && !rows16) err = launch_dispatch(*dims, x, ws.slot_token, counts, ws.xbuf, st);
+    // the expert GEMMs see up to 2T kept rows (their grid is sized from that bound)
+    switch_dims_t rows = *dims;
+    rows.T = 2 * dims->T;
+    if (err == cudaSuccess)
+        err = tensor_cores ? launch_ffn_tc(rows, ws.xbuf, w_in, w_out, counts, ws.ybuf, nullptr, nullptr, nullptr, ws,
+                                           st)
+                           : launch_ffn_simt(rows, ws.xbuf, w_in, w_out, counts, ws.ybuf, ws, st);
+    if (err == cudaSuccess) err = launch_combine_top2(*dims, ws.ybuf, expert, slot, gate, static_cast<float *>(y), st);
+    return from_cuda(err);
+}
+
 switch_status_t switch_check(void *workspace, size_t workspace_bytes_given, switch_stream_t stream) {
     if (!workspace) return SWITCH_ERR_NULL;
     if (workspace_bytes_given < sizeof(DeviceStatus)) return SWITCH_ERR_WORKSPACE;
@@ -414,6 +490,7 @@ const char *switch_kernel_name(int32_t id) {
         case K_ROUTER_SPLIT: return "router_weight_split";
         case K_SELFTEST_WAIT: return "selftest_wait_timeout";
         case K_FFN_TC_FUSED: return "ffn_tc_fused";
+        case K_COMBINE_TOP2: return "combine_top2";
     }
     return "?";
 }

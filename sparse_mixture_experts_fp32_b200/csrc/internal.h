@@ -32,6 +32,7 @@ enum KernelId : int32_t {
     K_ROUTER_SPLIT = 15,
     K_SELFTEST_WAIT = 16,
     K_FFN_TC_FUSED = 17,
+    K_COMBINE_TOP2 = 18,
 };
 
 struct Workspace {
@@ -48,6 +49,9 @@ struct Workspace {
     void *hidden;        // [N][C][F] expert hidden activations
     int32_t *done;       // fused FFN: [N][ceil(C/256)] GEMM1 completion counters, the tile claim counter,
                          // [N][ceil(C/256)][ceil(d/256)] GEMM2 first-half counters (fused_counter_ints)
+    int32_t *hist2;      // top-2: [N][tiles] second choices of each expert in each tile
+    int32_t *tile_off2;  // top-2: [N][tiles] first slot of each tile's second choices
+    int32_t *counts_first;  // top-2: [N] first choices per expert (the aux loss's f)
     int64_t tiles;
 };
 
@@ -70,19 +74,27 @@ void launch_end(cudaStream_t stream);
 // With `x_scatter` set, the slot assignment also copies every kept token's
 // row of x into xbuf[expert, slot] (scatter form of the dispatch) and, with
 // `y_zero` set, writes the zero output row of every dropped token.
+// With `top2`, expert, gate and slot are [T][2] (first and second choice of
+// each token) and the scan always runs as its own kernel.
 cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
                          int32_t *expert, float *gate, int32_t *slot, int32_t *counts, int32_t *slot_token,
                          float *aux, const Workspace &ws, cudaStream_t stream, void *xbuf_scatter = nullptr,
-                         float *y_zero = nullptr, int32_t *done_zero = nullptr, int64_t n_done = 0);
+                         float *y_zero = nullptr, int32_t *done_zero = nullptr, int64_t n_done = 0,
+                         bool top2 = false);
 cudaError_t launch_dispatch(const switch_dims_t &dims, const void *x, const int32_t *slot_token,
                             const int32_t *counts, void *xbuf, cudaStream_t stream);
 cudaError_t launch_combine(const switch_dims_t &dims, const float *ybuf, const int32_t *expert,
                            const int32_t *slot, const float *gate, float *y, cudaStream_t stream);
+// Top-2 combine: y[t] = gate[2t] ybuf[expert[2t], slot[2t]] + gate[2t+1] ybuf[expert[2t+1], slot[2t+1]]
+// over the kept choices (0 when both were dropped).
+cudaError_t launch_combine_top2(const switch_dims_t &dims, const float *ybuf, const int32_t *expert,
+                                const int32_t *slot, const float *gate, float *y, cudaStream_t stream);
 // Tensor-core router (bf16 x, N <= 128): writes expert, gate and the
 // per-tile counts / probability sums like the CUDA-core routers.
 bool router_tc_supported(const switch_dims_t &dims);
 cudaError_t launch_router_tc(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
-                             int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream);
+                             int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream,
+                             bool top2 = false);
 // Expert FFN; ybuf is float32 [N][C][d].
 cudaError_t launch_ffn_simt(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
                             const int32_t *counts, float *ybuf, const Workspace &ws, cudaStream_t stream);

@@ -117,7 +117,62 @@ __global__ void __launch_bounds__(kThreads) combine_kernel_scalar(const float *_
     for (int k = lane; k < d; k += 32) dst[k] = g * src[k];
 }
 
+// Top-2: y[t] = g0 * ybuf[e0, s0] + g1 * ybuf[e1, s1] over the kept choices,
+// the first choice's product first (float32; 0 when both were dropped).
+template <bool VEC>
+__global__ void __launch_bounds__(kThreads) combine_top2_kernel(const float *__restrict__ ybuf,
+                                                               const int32_t *__restrict__ expert2,
+                                                               const int32_t *__restrict__ slot2,
+                                                               const float *__restrict__ gate2, int64_t T, int C,
+                                                               int d, float *__restrict__ y) {
+    const int64_t t = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const int lane = threadIdx.x & 31;
+    const int s0 = slot2[2 * t], s1 = slot2[2 * t + 1];
+    const float g0 = s0 >= 0 ? gate2[2 * t] : 0.f, g1 = s1 >= 0 ? gate2[2 * t + 1] : 0.f;
+    const float *src0 = s0 >= 0 ? ybuf + ((int64_t)expert2[2 * t] * C + s0) * d : nullptr;
+    const float *src1 = s1 >= 0 ? ybuf + ((int64_t)expert2[2 * t + 1] * C + s1) * d : nullptr;
+    if (VEC) {
+        const int words = d / 4;
+        float4 *dst = reinterpret_cast<float4 *>(y + t * d);
+        for (int w = lane; w < words; w += 32) {
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+            if (src0) a = __ldcs(reinterpret_cast<const float4 *>(src0) + w);
+            if (src1) b = __ldcs(reinterpret_cast<const float4 *>(src1) + w);
+            float4 o;
+            o.x = __fadd_rn(__fmul_rn(g0, a.x), __fmul_rn(g1, b.x));
+            o.y = __fadd_rn(__fmul_rn(g0, a.y), __fmul_rn(g1, b.y));
+            o.z = __fadd_rn(__fmul_rn(g0, a.z), __fmul_rn(g1, b.z));
+            o.w = __fadd_rn(__fmul_rn(g0, a.w), __fmul_rn(g1, b.w));
+            __stcs(dst + w, o);
+        }
+    } else {
+        float *dst = y + t * d;
+        for (int k = lane; k < d; k += 32) {
+            const float a = src0 ? src0[k] : 0.f, b = src1 ? src1[k] : 0.f;
+            dst[k] = __fadd_rn(__fmul_rn(g0, a), __fmul_rn(g1, b));
+        }
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_combine_top2(const switch_dims_t &dims, const float *ybuf, const int32_t *expert,
+                                const int32_t *slot, const float *gate, float *y, cudaStream_t stream) {
+    const int64_t T = dims.T;
+    if (T == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((T + kRowsPerBlock - 1) / kRowsPerBlock);
+    launch_begin(K_COMBINE_TOP2, stream);
+    if (dims.d_model % 4 == 0)
+        combine_top2_kernel<true><<<grid, kThreads, 0, stream>>>(ybuf, expert, slot, gate, T, dims.capacity,
+                                                                 dims.d_model, y);
+    else
+        combine_top2_kernel<false><<<grid, kThreads, 0, stream>>>(ybuf, expert, slot, gate, T, dims.capacity,
+                                                                  dims.d_model, y);
+    cudaError_t err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
 
 cudaError_t launch_dispatch(const switch_dims_t &dims, const void *x, const int32_t *slot_token,
                             const int32_t *counts, void *xbuf, cudaStream_t stream) {

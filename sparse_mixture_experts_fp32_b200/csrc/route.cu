@@ -30,20 +30,25 @@ __device__ __forceinline__ int lanemask_lt() {
     return m;
 }
 
-// Per-token softmax / top-1 bookkeeping, done by one warp.  Each lane holds
-// up to J logits: value v[j] for expert idx[j] (idx < 0: not held).  Every
-// expert is held by exactly one "owner" lane (own[j] true); other lanes may
-// hold copies, which take part in the max but not in the sums.
-template <int J>
+// Per-token softmax / top-1 (or top-2) bookkeeping, done by one warp.  Each
+// lane holds up to J logits: value v[j] for expert idx[j] (idx < 0: not held).
+// Every expert is held by exactly one "owner" lane (own[j] true); other lanes
+// may hold copies, which take part in the max but not in the sums.  With
+// TOP2 the warp also finds the second choice (the largest logit among the
+// other experts, lowest index on ties) and writes both choices of token t to
+// expert[2t], expert[2t+1] and their probabilities to gate[2t], gate[2t+1].
+__device__ __forceinline__ bool better(float v, int i, float m, int a) { return v > m || (v == m && i < a); }
+
+template <int J, bool TOP2>
 __device__ __forceinline__ void token_epilogue(const float (&v)[J], const int (&idx)[J], const bool (&own)[J],
-                                               int64_t t, float *warp_psum, int32_t *warp_hist, int32_t *expert,
-                                               float *gate) {
+                                               int64_t t, float *warp_psum, int32_t *warp_hist,
+                                               int32_t *warp_hist2, int32_t *expert, float *gate) {
     const int lane = threadIdx.x & 31;
     float m = -FLT_MAX;
     int arg = 0x7fffffff;
 #pragma unroll
     for (int j = 0; j < J; ++j) {
-        if (idx[j] >= 0 && (v[j] > m || (v[j] == m && idx[j] < arg))) {
+        if (idx[j] >= 0 && better(v[j], idx[j], m, arg)) {
             m = v[j];
             arg = idx[j];
         }
@@ -52,10 +57,32 @@ __device__ __forceinline__ void token_epilogue(const float (&v)[J], const int (&
     for (int off = 16; off > 0; off >>= 1) {
         const float om = __shfl_xor_sync(0xffffffffu, m, off);
         const int oa = __shfl_xor_sync(0xffffffffu, arg, off);
-        if (om > m || (om == m && oa < arg)) {
+        if (better(om, oa, m, arg)) {
             m = om;
             arg = oa;
         }
+    }
+    if (arg == 0x7fffffff) arg = 0;  // no comparable logit (NaN inputs): keep every index in range
+    float m2 = -FLT_MAX;
+    int arg2 = 0x7fffffff;
+    if (TOP2) {
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            if (idx[j] >= 0 && idx[j] != arg && better(v[j], idx[j], m2, arg2)) {
+                m2 = v[j];
+                arg2 = idx[j];
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float om = __shfl_xor_sync(0xffffffffu, m2, off);
+            const int oa = __shfl_xor_sync(0xffffffffu, arg2, off);
+            if (better(om, oa, m2, arg2)) {
+                m2 = om;
+                arg2 = oa;
+            }
+        }
+        if (arg2 == 0x7fffffff) arg2 = arg == 0 ? 1 : 0;
     }
     float ex[J];
     float s = 0.f;
@@ -71,24 +98,35 @@ __device__ __forceinline__ void token_epilogue(const float (&v)[J], const int (&
         if (idx[j] >= 0 && own[j]) warp_psum[idx[j]] += ex[j] / s;
     if (lane == 0) {
         warp_hist[arg] += 1;
-        expert[t] = arg;
-        gate[t] = 1.0f / s;  // p at the argmax: exp(0) / s
+        if (TOP2) {
+            warp_hist2[arg2] += 1;
+            expert[2 * t] = arg;
+            expert[2 * t + 1] = arg2;
+            gate[2 * t] = 1.0f / s;  // p at the argmax: exp(0) / s
+            gate[2 * t + 1] = expf(m2 - m) / s;
+        } else {
+            expert[t] = arg;
+            gate[t] = 1.0f / s;  // p at the argmax: exp(0) / s
+        }
     }
 }
 
 // Sum the per-warp partials of a tile in fixed warp order and publish them
-// expert-major ([N][tiles]) for the scan.
-__device__ __forceinline__ void publish_tile(const float *psum_w, const int32_t *hist_w, int N, int tiles,
-                                             int tile, int32_t *hist, float *psum) {
+// expert-major ([N][tiles]) for the scan (with hist2: second-choice counts too).
+__device__ __forceinline__ void publish_tile(const float *psum_w, const int32_t *hist_w, const int32_t *hist2_w,
+                                             int N, int tiles, int tile, int32_t *hist, int32_t *hist2,
+                                             float *psum) {
     for (int i = threadIdx.x; i < N; i += kThreads) {
-        int32_t c = 0;
+        int32_t c = 0, c2 = 0;
         float p = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
             c += hist_w[w * N + i];
+            if (hist2) c2 += hist2_w[w * N + i];
             p += psum_w[w * N + i];
         }
         hist[(int64_t)i * tiles + tile] = c;
+        if (hist2) hist2[(int64_t)i * tiles + tile] = c2;
         psum[(int64_t)i * tiles + tile] = p;
     }
 }
@@ -155,17 +193,19 @@ struct XLoad<float> {
 // NP partial dot products over its share of d; a halving exchange then
 // leaves lane L with the full logit of expert L >> (5 - log2 NP).
 // ---------------------------------------------------------------------------
-template <typename XT, int NP>
+template <typename XT, int NP, bool TOP2>
 __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restrict__ x, const float *__restrict__ w_r,
                                                                const float *__restrict__ bias, int64_t T, int d,
                                                                int N, int tiles, int32_t *__restrict__ expert,
                                                                float *__restrict__ gate, int32_t *__restrict__ hist,
+                                                               int32_t *__restrict__ hist2,
                                                                float *__restrict__ psum, uint32_t *ticket,
                                                                DeviceStatus *status) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *wsm = reinterpret_cast<float *>(smem_raw);  // [d][NP]
     float *psum_w = wsm + (size_t)d * NP;               // [kWarps][N]
     int32_t *hist_w = reinterpret_cast<int32_t *>(psum_w + kWarps * N);
+    int32_t *hist2_w = hist_w + kWarps * N;             // [kWarps][N] second choices (TOP2)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x;
 
@@ -177,6 +217,7 @@ __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restr
     for (int i = tid; i < kWarps * N; i += kThreads) {
         psum_w[i] = 0.f;
         hist_w[i] = 0;
+        if (TOP2) hist2_w[i] = 0;
     }
     __syncthreads();
 
@@ -244,10 +285,11 @@ __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restr
         float v[1] = {acc[0] + my_bias};
         int idx[1] = {valid_e ? my_e : -1};
         bool own[1] = {(lane & ((1 << SHIFT) - 1)) == 0};
-        token_epilogue<1>(v, idx, own, t, psum_w + warp * N, hist_w + warp * N, expert, gate);
+        token_epilogue<1, TOP2>(v, idx, own, t, psum_w + warp * N, hist_w + warp * N, hist2_w + warp * N, expert,
+                                gate);
     }
     __syncthreads();
-    publish_tile(psum_w, hist_w, N, tiles, tile, hist, psum);
+    publish_tile(psum_w, hist_w, hist2_w, N, tiles, tile, hist, TOP2 ? hist2 : nullptr, psum);
 }
 
 // ---------------------------------------------------------------------------
@@ -271,22 +313,23 @@ struct Staged {
         const int64_t a = kTileT * xpitch(d), b = (int64_t)kTileT * NP * 4;
         return ((a > b ? a : b) + 15) / 16 * 16;
     }
-    // smem layout: x tile | W_r as [d/V][V][NP] | per-warp sums | counts | 5 mbarriers | raw W_r (optional)
+    // smem layout: x tile | W_r as [d/V][V][NP] | per-warp sums | counts | second-choice counts |
+    // 5 mbarriers | raw W_r (optional)
     static size_t smem_base(int d, int NP) {
         return (size_t)x_region(d, NP) + (size_t)((d / V) * wpitch(NP)) * 4 + (size_t)(kWarps * NP) * 4 +
-               (size_t)NP * 4 + 5 * 8 + 16;
+               2 * (size_t)NP * 4 + 5 * 8 + 16;
     }
     static size_t smem(int d, int NP, int N, bool raw) {
         return smem_base(d, NP) + (raw ? (size_t)N * d * 4 + 16 : 0);
     }
 };
 
-template <typename XT, int NP>
+template <typename XT, int NP, bool TOP2>
 __global__ void __launch_bounds__(kThreads, 1)
     router_staged_kernel(const XT *__restrict__ x, const float *__restrict__ w_r, const float *__restrict__ bias,
                          int64_t T, int d, int N, int tiles, int32_t *__restrict__ expert, float *__restrict__ gate,
-                         int32_t *__restrict__ hist, float *__restrict__ psum, uint32_t *ticket,
-                         DeviceStatus *status, int raw_w) {
+                         int32_t *__restrict__ hist, int32_t *__restrict__ hist2, float *__restrict__ psum,
+                         uint32_t *ticket, DeviceStatus *status, int raw_w) {
     using S = Staged<XT>;
     constexpr int V = S::V;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -296,7 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *wsm = reinterpret_cast<float *>(smem_raw + S::x_region(d, NP));
     float *psum_w = wsm + (d / V) * wpitch;
     int32_t *hist_s = reinterpret_cast<int32_t *>(psum_w + kWarps * NP);
-    uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(hist_s + NP) + 15) & ~uintptr_t(15));
+    int32_t *hist2_s = hist_s + NP;  // second choices (TOP2)
+    uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(hist2_s + NP) + 15) & ~uintptr_t(15));
     float *w_raw = reinterpret_cast<float *>(bar + 5) + 2;  // 16-byte aligned: bar is, and 5 * 8 + 8 = 48
     const int tid = threadIdx.x;
     const int tile = blockIdx.x;
@@ -349,7 +393,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     for (int i = tid; i < kWarps * NP; i += kThreads) psum_w[i] = 0.f;
-    for (int i = tid; i < NP; i += kThreads) hist_s[i] = 0;
+    for (int i = tid; i < NP; i += kThreads) {
+        hist_s[i] = 0;
+        hist2_s[i] = 0;
+    }
     __syncthreads();
 
     // Thread (group g, part p): tokens 4g .. 4g+3 of the tile, 16-byte x
@@ -414,18 +461,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 1; i < TM; ++i) v = (part == i) ? acc[i][e] : v;
             h[e] = v;
         }
-        float m = -FLT_MAX;
-        int arg = 0;
 #pragma unroll
-        for (int e = 0; e < NP; ++e) {
+        for (int e = 0; e < NP; ++e)
+            if (e < N) h[e] += bias ? bias[e] : 0.f;
+        float m = h[0], m2 = -FLT_MAX;
+        int arg = 0, arg2 = -1;
+#pragma unroll
+        for (int e = 1; e < NP; ++e) {
             if (e < N) {
-                h[e] += bias ? bias[e] : 0.f;
                 if (h[e] > m) {  // strict: the lowest index wins a tie
+                    if (TOP2) {  // the previous leader is now the best of the others
+                        m2 = m;
+                        arg2 = arg;
+                    }
                     m = h[e];
                     arg = e;
+                } else if (TOP2 && (arg2 < 0 || h[e] > m2)) {  // strict: lowest index among the others
+                    m2 = h[e];
+                    arg2 = e;
                 }
             }
         }
+        if (TOP2 && arg2 < 0) arg2 = arg == 0 ? 1 : 0;  // N == 1 only, which top-2 routing rejects
         float s = 0.f;
 #pragma unroll
         for (int e = 0; e < NP; ++e) {
@@ -436,8 +493,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < NP; ++e) ptile[tl * NP + e] = valid ? h[e] / s : 0.f;  // p_e
         if (valid) {
             const int64_t t = t0 + tl;
-            expert[t] = arg;
-            gate[t] = 1.0f / s;  // p at the argmax: exp(0) / s
+            if (TOP2) {
+                expert[2 * t] = arg;
+                expert[2 * t + 1] = arg2;
+                gate[2 * t] = 1.0f / s;
+                gate[2 * t + 1] = expf(m2 - m) / s;
+                atomicAdd(&hist2_s[arg2], 1);
+            } else {
+                expert[t] = arg;
+                gate[t] = 1.0f / s;  // p at the argmax: exp(0) / s
+            }
             atomicAdd(&hist_s[arg], 1);
         }
     }
@@ -451,6 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int u = 0; u < 4; ++u) p4[u] += ptile[(tl + u) * NP + i];
         }
         hist[(int64_t)i * tiles + tile] = hist_s[i];
+        if (TOP2) hist2[(int64_t)i * tiles + tile] = hist2_s[i];
         psum[(int64_t)i * tiles + tile] = (p4[0] + p4[1]) + (p4[2] + p4[3]);
     }
 }
@@ -462,11 +528,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 constexpr int kKC = 32;
 
-template <typename XT, int EC>
+template <typename XT, int EC, bool TOP2>
 __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__restrict__ x, const float *__restrict__ w_r,
                                                                 const float *__restrict__ bias, int64_t T, int d,
                                                                 int N, int tiles, int32_t *__restrict__ expert,
                                                                 float *__restrict__ gate, int32_t *__restrict__ hist,
+                                                                int32_t *__restrict__ hist2,
                                                                 float *__restrict__ psum, uint32_t *ticket,
                                                                 DeviceStatus *status) {
     constexpr int TE = EC / 16;  // experts per thread
@@ -478,6 +545,7 @@ __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__rest
     float *logits = ws + kKC * EC;                     // [kTileT][NL]
     float *psum_w = logits + kTileT * NL;              // [kWarps][N]
     int32_t *hist_w = reinterpret_cast<int32_t *>(psum_w + kWarps * N);
+    int32_t *hist2_w = hist_w + kWarps * N;            // [kWarps][N] second choices (TOP2)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tx = tid % 16, ty = tid / 16;
     const int tile = blockIdx.x;
@@ -487,6 +555,7 @@ __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__rest
     for (int i = tid; i < kWarps * N; i += kThreads) {
         psum_w[i] = 0.f;
         hist_w[i] = 0;
+        if (TOP2) hist2_w[i] = 0;
     }
 
     for (int e0 = 0; e0 < N; e0 += EC) {
@@ -546,10 +615,11 @@ __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__rest
             own[j] = true;
             v[j] = e < N ? logits[r * NL + e] + (bias ? bias[e] : 0.f) : 0.f;
         }
-        token_epilogue<J>(v, idx, own, t, psum_w + warp * N, hist_w + warp * N, expert, gate);
+        token_epilogue<J, TOP2>(v, idx, own, t, psum_w + warp * N, hist_w + warp * N, hist2_w + warp * N, expert,
+                                gate);
     }
     __syncthreads();
-    publish_tile(psum_w, hist_w, N, tiles, tile, hist, psum);
+    publish_tile(psum_w, hist_w, hist2_w, N, tiles, tile, hist, TOP2 ? hist2 : nullptr, psum);
 }
 
 // ---------------------------------------------------------------------------
@@ -557,12 +627,60 @@ __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__rest
 // ---------------------------------------------------------------------------
 constexpr int kScanThreads = 1024;
 
+// Exclusive prefix over tiles of one expert's row of tile counts, starting at
+// `base`: thread tid owns tiles [begin, end).  Returns the row total.
+__device__ __forceinline__ int32_t scan_row(const int32_t *__restrict__ h, int tiles, int32_t base,
+                                            int32_t *__restrict__ off, int32_t *warp_cnt) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int chunk = (tiles + kScanThreads - 1) / kScanThreads;
+    const int begin = min(tiles, tid * chunk), end = min(tiles, begin + chunk);
+    int32_t mine = 0;
+    for (int i = begin; i < end; ++i) mine += h[i];
+    int32_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    __syncthreads();  // warp_cnt may still be read from a previous row
+    if (lane == 31) warp_cnt[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int32_t c = warp_cnt[lane];
+        int32_t ci = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t u = __shfl_up_sync(0xffffffffu, ci, o);
+            if (lane >= o) ci += u;
+        }
+        warp_cnt[lane] = ci - c;  // exclusive prefix of warp totals
+        if (lane == 31) warp_cnt[32] = ci;
+    }
+    __syncthreads();
+    int32_t run = base + warp_cnt[warp] + incl - mine;
+    for (int i = begin; i < end; ++i) {
+        off[i] = run;
+        run += h[i];
+    }
+    return warp_cnt[32];
+}
+
+// Scan: one block per expert.  Top-1: tile_off = exclusive prefix of the tile
+// counts.  Top-2 (hist2 set): first choices take the slots first, so
+// tile_off = prefix of the first-choice counts and tile_off2 = (all first
+// choices of the expert) + prefix of the second-choice counts; counts = both
+// totals, counts_first = the first-choice total (the aux loss counts argmax
+// choices only).
+template <bool TOP2>
 __global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t *__restrict__ hist,
+                                                            const int32_t *__restrict__ hist2,
                                                             const float *__restrict__ psum, int tiles, int N,
                                                             int64_t T, int32_t *__restrict__ tile_off,
-                                                            int32_t *__restrict__ counts, double *prob_total,
+                                                            int32_t *__restrict__ tile_off2,
+                                                            int32_t *__restrict__ counts,
+                                                            int32_t *__restrict__ counts_first, double *prob_total,
                                                             float *aux, uint32_t *ticket) {
-    __shared__ int32_t warp_cnt[kScanThreads / 32];
+    __shared__ int32_t warp_cnt[33];
     __shared__ double warp_p[kScanThreads / 32];
     __shared__ bool is_last;
     pdl_wait();
@@ -571,49 +689,24 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t *__res
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int chunk = (tiles + kScanThreads - 1) / kScanThreads;
     const int begin = min(tiles, tid * chunk), end = min(tiles, begin + chunk);
-    const int32_t *h = hist + (int64_t)e * tiles;
     const float *ps = psum + (int64_t)e * tiles;
 
-    int32_t mine = 0;
     double pmine = 0.0;
-    for (int i = begin; i < end; ++i) {
-        mine += h[i];
-        pmine += (double)ps[i];
-    }
-    // inclusive warp scan of the chunk totals
-    int32_t incl = mine;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int32_t u = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += u;
-    }
+    for (int i = begin; i < end; ++i) pmine += (double)ps[i];
     double pw = pmine;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) pw += __shfl_xor_sync(0xffffffffu, pw, off);
-    if (lane == 31) warp_cnt[warp] = incl;
     if (lane == 0) warp_p[warp] = pw;
-    __syncthreads();
-    if (warp == 0) {
-        int32_t c = warp_cnt[lane];
-        int32_t ci = c;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int32_t u = __shfl_up_sync(0xffffffffu, ci, off);
-            if (lane >= off) ci += u;
-        }
-        warp_cnt[lane] = ci - c;  // exclusive prefix of warp totals
-        if (lane == 31) counts[e] = ci;
-        if (lane == 0) {
-            double p = 0.0;
-            for (int w = 0; w < kScanThreads / 32; ++w) p += warp_p[w];
-            prob_total[e] = p;
-        }
-    }
-    __syncthreads();
-    int32_t run = warp_cnt[warp] + incl - mine;
-    for (int i = begin; i < end; ++i) {
-        tile_off[(int64_t)e * tiles + i] = run;
-        run += h[i];
+    const int32_t total1 = scan_row(hist + (int64_t)e * tiles, tiles, 0, tile_off + (int64_t)e * tiles, warp_cnt);
+    int32_t total = total1;
+    if (TOP2)
+        total += scan_row(hist2 + (int64_t)e * tiles, tiles, total1, tile_off2 + (int64_t)e * tiles, warp_cnt);
+    if (tid == 0) {
+        counts[e] = total;
+        if (TOP2) counts_first[e] = total1;
+        double p = 0.0;
+        for (int w = 0; w < kScanThreads / 32; ++w) p += warp_p[w];
+        prob_total[e] = p;
     }
 
     // The last expert block to finish forms the aux loss: one f_i * P_i per
@@ -626,18 +719,19 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t *__res
         __threadfence();
         double term = 0.0;
         if (T > 0 && tid < N) {
-            const double f = (double)__ldcg(counts + tid) / (double)T;
+            const double f = (double)__ldcg((TOP2 ? counts_first : counts) + tid) / (double)T;
             const double P = __ldcg(prob_total + tid) / (double)T;
             term = f * P;
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) term += __shfl_xor_sync(0xffffffffu, term, off);
+        __syncthreads();  // every warp has read warp_p above
         if (lane == 0) warp_p[warp] = term;
         __syncthreads();
         if (tid == 0) {
-            double total = 0.0;
-            for (int w = 0; w < kScanThreads / 32; ++w) total += warp_p[w];
-            *aux = (float)((double)N * total);
+            double total_aux = 0.0;
+            for (int w = 0; w < kScanThreads / 32; ++w) total_aux += warp_p[w];
+            *aux = (float)((double)N * total_aux);
             *ticket = 0u;
         }
     }
@@ -813,17 +907,93 @@ __global__ void __launch_bounds__(kAssignThreads) assign_kernel(
     }
 }
 
-template <typename XT, int NP>
+// Top-2 assignment: block `tile` ranks the tile's first choices (warps 0-1)
+// and second choices (warps 2-3) within their experts, in token order.  A
+// first choice takes slot tile_off[e][tile] + rank, a second choice
+// tile_off2[e][tile] + rank (tile_off2 starts after all first choices of the
+// expert); kept iff the slot is below C.  With SCATTER all eight warps then
+// copy x[t] to xbuf[e, slot] for every kept (token, choice).  Every block
+// also clears a share of the empty slots of slot_token.
+template <bool SCATTER>
+__global__ void __launch_bounds__(kAssignThreads) assign_top2_kernel(
+    const int32_t *__restrict__ expert2, const int32_t *__restrict__ tile_off, const int32_t *__restrict__ tile_off2,
+    const int32_t *__restrict__ counts, int64_t T, int N, int C, int tiles, int32_t *__restrict__ slot2,
+    int32_t *__restrict__ slot_token, const uint4 *__restrict__ x, uint4 *__restrict__ xbuf, int x_words) {
+    static_assert(kTileT == 64, "top-2 assignment assumes 64-token tiles");
+    __shared__ int32_t first_warp_count[2][256];
+    __shared__ int32_t tile_slot[2 * kTileT];    // [choice][token of the tile]
+    __shared__ int32_t tile_expert[2 * kTileT];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tile = blockIdx.x;
+    if (tile < tiles) {
+        for (int i = tid; i < 2 * 256; i += kAssignThreads) (&first_warp_count[0][0])[i] = 0;
+        __syncthreads();
+        const int c = warp >> 1;         // warps 0-1: first choices, 2-3: second choices
+        const int half = warp & 1;       // tokens 0-31 or 32-63 of the tile
+        int e = -1, rank = 0;
+        bool valid = false;
+        int64_t t = 0;
+        unsigned same = 0;
+        if (warp < 4) {
+            t = (int64_t)tile * kTileT + half * 32 + lane;
+            valid = t < T;
+            e = valid ? expert2[2 * t + c] : -1 - lane;  // distinct keys for absent tokens
+            same = __match_any_sync(0xffffffffu, e);
+            rank = __popc(same & (unsigned)lanemask_lt());
+            if (half == 0 && valid && rank == 0) first_warp_count[c][e] = __popc(same);
+        }
+        __syncthreads();
+        if (warp < 4) {
+            int s_out = -2;  // -2: no token here
+            if (valid) {
+                if (half == 1) rank += first_warp_count[c][e];
+                const int s = (c == 0 ? tile_off : tile_off2)[(int64_t)e * tiles + tile] + rank;
+                if (s < C) {
+                    slot2[2 * t + c] = s;
+                    slot_token[(int64_t)e * C + s] = (int32_t)t;
+                    s_out = s;
+                } else {
+                    slot2[2 * t + c] = -1;
+                    s_out = -1;
+                }
+            }
+            tile_slot[c * kTileT + half * 32 + lane] = s_out;
+            tile_expert[c * kTileT + half * 32 + lane] = e;
+        }
+        if (SCATTER) {
+            __syncthreads();
+            // 128 (token, choice) entries; warp w copies entries w, w + 8, ...
+            for (int j = warp; j < 2 * kTileT; j += kAssignThreads / 32) {
+                const int s = tile_slot[j];
+                if (s < 0) continue;
+                const int r = j & (kTileT - 1);
+                const uint4 *src = x + ((int64_t)tile * kTileT + r) * x_words;
+                uint4 *dst = xbuf + ((int64_t)tile_expert[j] * C + s) * x_words;
+                for (int w = lane; w < x_words; w += 32) dst[w] = __ldg(src + w);
+            }
+        }
+    }
+    const int64_t total = (int64_t)N * C;
+    for (int64_t i = (int64_t)blockIdx.x * kAssignThreads + tid; i < total; i += (int64_t)gridDim.x * kAssignThreads) {
+        const int e = (int)(i / C);
+        const int s = (int)(i % C);
+        if (s >= min(counts[e], C)) slot_token[i] = -1;
+    }
+}
+
+template <typename XT, int NP, bool TOP2>
 cudaError_t launch_router_warp(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
                                int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts, d = dims.d_model;
-    const size_t smem = (size_t)d * NP * sizeof(float) + (size_t)kWarps * N * (sizeof(float) + sizeof(int32_t));
-    auto kern = router_warp_kernel<XT, NP>;
+    const size_t smem = (size_t)d * NP * sizeof(float) + (size_t)kWarps * N * (sizeof(float) + 2 * sizeof(int32_t));
+    auto kern = router_warp_kernel<XT, NP, TOP2>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_WARP, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
-                                                         ws.hist, ws.psum, ws.ticket,
+                                                         ws.hist, ws.hist2, ws.psum, ws.ticket,
                                                          static_cast<DeviceStatus *>(ws.status));
     err = cudaGetLastError();
     launch_end(stream);
@@ -833,36 +1003,36 @@ cudaError_t launch_router_warp(const switch_dims_t &dims, const XT *x, const flo
 // Shared memory the staged router may use (x tile + W_r + partials).
 constexpr size_t kStagedSmemLimit = 200 * 1024;
 
-template <typename XT, int NP>
+template <typename XT, int NP, bool TOP2>
 cudaError_t launch_router_staged(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
                                  int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts, d = dims.d_model;
     const bool raw = ((int64_t)N * d * 4) % 16 == 0 && Staged<XT>::smem(d, NP, N, true) <= kStagedSmemLimit;
     const size_t smem = Staged<XT>::smem(d, NP, N, raw);
-    auto kern = router_staged_kernel<XT, NP>;
+    auto kern = router_staged_kernel<XT, NP, TOP2>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_STAGED, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
-                                                         ws.hist, ws.psum, ws.ticket,
+                                                         ws.hist, ws.hist2, ws.psum, ws.ticket,
                                                          static_cast<DeviceStatus *>(ws.status), raw ? 1 : 0);
     err = cudaGetLastError();
     launch_end(stream);
     return err;
 }
 
-template <typename XT, int EC>
+template <typename XT, int EC, bool TOP2>
 cudaError_t launch_router_tiled(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
                                 int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts, d = dims.d_model;
     const size_t smem = (size_t)(kKC * kTileT + kKC * EC + kTileT * (N + 1)) * sizeof(float) +
-                        (size_t)kWarps * N * (sizeof(float) + sizeof(int32_t));
-    auto kern = router_tiled_kernel<XT, EC>;
+                        (size_t)kWarps * N * (sizeof(float) + 2 * sizeof(int32_t));
+    auto kern = router_tiled_kernel<XT, EC, TOP2>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_TILED, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
-                                                         ws.hist, ws.psum, ws.ticket,
+                                                         ws.hist, ws.hist2, ws.psum, ws.ticket,
                                                          static_cast<DeviceStatus *>(ws.status));
     err = cudaGetLastError();
     launch_end(stream);
@@ -871,7 +1041,7 @@ cudaError_t launch_router_tiled(const switch_dims_t &dims, const XT *x, const fl
 
 // Largest d for which the warp router keeps W_r in shared memory.
 constexpr size_t kWarpRouterSmemLimit = 160 * 1024;
-template <typename XT>
+template <typename XT, bool TOP2>
 cudaError_t launch_router(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
                           int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts;
@@ -879,19 +1049,28 @@ cudaError_t launch_router(const switch_dims_t &dims, const XT *x, const float *w
     const bool staged = N <= 32 && ((int64_t)dims.d_model * (int64_t)sizeof(XT)) % 16 == 0 &&
                         Staged<XT>::smem(dims.d_model, NP, N, false) <= kStagedSmemLimit;
     if (staged) {
-        if (NP == 8) return launch_router_staged<XT, 8>(dims, x, w_r, bias, expert, gate, ws, stream);
-        if (NP == 16) return launch_router_staged<XT, 16>(dims, x, w_r, bias, expert, gate, ws, stream);
-        return launch_router_staged<XT, 32>(dims, x, w_r, bias, expert, gate, ws, stream);
+        if (NP == 8) return launch_router_staged<XT, 8, TOP2>(dims, x, w_r, bias, expert, gate, ws, stream);
+        if (NP == 16) return launch_router_staged<XT, 16, TOP2>(dims, x, w_r, bias, expert, gate, ws, stream);
+        return launch_router_staged<XT, 32, TOP2>(dims, x, w_r, bias, expert, gate, ws, stream);
     }
     const bool fits = N <= 32 && (size_t)dims.d_model * NP * sizeof(float) + 2048 * 8 <= kWarpRouterSmemLimit;
     if (fits) {
-        if (NP == 8) return launch_router_warp<XT, 8>(dims, x, w_r, bias, expert, gate, ws, stream);
-        if (NP == 16) return launch_router_warp<XT, 16>(dims, x, w_r, bias, expert, gate, ws, stream);
-        return launch_router_warp<XT, 32>(dims, x, w_r, bias, expert, gate, ws, stream);
+        if (NP == 8) return launch_router_warp<XT, 8, TOP2>(dims, x, w_r, bias, expert, gate, ws, stream);
+        if (NP == 16) return launch_router_warp<XT, 16, TOP2>(dims, x, w_r, bias, expert, gate, ws, stream);
+        return launch_router_warp<XT, 32, TOP2>(dims, x, w_r, bias, expert, gate, ws, stream);
     }
-    if (N <= 32) return launch_router_tiled<XT, 32>(dims, x, w_r, bias, expert, gate, ws, stream);
-    if (N <= 64) return launch_router_tiled<XT, 64>(dims, x, w_r, bias, expert, gate, ws, stream);
-    return launch_router_tiled<XT, 128>(dims, x, w_r, bias, expert, gate, ws, stream);
+    if (N <= 32) return launch_router_tiled<XT, 32, TOP2>(dims, x, w_r, bias, expert, gate, ws, stream);
+    if (N <= 64) return launch_router_tiled<XT, 64, TOP2>(dims, x, w_r, bias, expert, gate, ws, stream);
+    return launch_router_tiled<XT, 128, TOP2>(dims, x, w_r, bias, expert, gate, ws, stream);
+}
+
+template <bool TOP2>
+cudaError_t launch_any_router(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
+                              int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
+    return dims.dtype == SWITCH_BF16
+               ? launch_router<__nv_bfloat16, TOP2>(dims, static_cast<const __nv_bfloat16 *>(x), w_r, bias, expert,
+                                                    gate, ws, stream)
+               : launch_router<float, TOP2>(dims, static_cast<const float *>(x), w_r, bias, expert, gate, ws, stream);
 }
 
 }  // namespace
@@ -899,17 +1078,15 @@ cudaError_t launch_router(const switch_dims_t &dims, const XT *x, const float *w
 cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
                          int32_t *expert, float *gate, int32_t *slot, int32_t *counts, int32_t *slot_token,
                          float *aux, const Workspace &ws, cudaStream_t stream, void *xbuf_scatter, float *y_zero,
-                         int32_t *done_zero, int64_t n_done) {
+                         int32_t *done_zero, int64_t n_done, bool top2) {
     cudaError_t err = cudaSuccess;
     const int N = dims.num_experts, C = dims.capacity;
     if (ws.tiles > 0 && router_tc_supported(dims)) {
-        err = launch_router_tc(dims, x, w_r, bias, expert, gate, ws, stream);
+        err = launch_router_tc(dims, x, w_r, bias, expert, gate, ws, stream, top2);
         if (err != cudaSuccess) return err;
     } else if (ws.tiles > 0) {
-        err = dims.dtype == SWITCH_BF16
-                  ? launch_router<__nv_bfloat16>(dims, static_cast<const __nv_bfloat16 *>(x), w_r, bias, expert,
-                                                 gate, ws, stream)
-                  : launch_router<float>(dims, static_cast<const float *>(x), w_r, bias, expert, gate, ws, stream);
+        err = top2 ? launch_any_router<true>(dims, x, w_r, bias, expert, gate, ws, stream)
+                   : launch_any_router<false>(dims, x, w_r, bias, expert, gate, ws, stream);
         if (err != cudaSuccess) return err;
     } else {
         // No router launch to reset the scan ticket and the status word.
@@ -919,6 +1096,29 @@ cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *
     }
     const int64_t fill_blocks = ((int64_t)N * C + kAssignThreads * 4 - 1) / (kAssignThreads * 4);
     const int64_t grid = ws.tiles > fill_blocks ? ws.tiles : fill_blocks;
+    const int x_words = (int)((int64_t)dims.d_model * (dims.dtype == SWITCH_BF16 ? 2 : 4) / 16);
+    const uint4 *xs = static_cast<const uint4 *>(x);
+    uint4 *xb = static_cast<uint4 *>(xbuf_scatter);
+    if (top2) {
+        // top-2: the scan kernel always runs (two prefixes per expert)
+        launch_begin(K_SCAN, stream);
+        err = launch_kernel(scan_kernel<true>, dim3(N), dim3(kScanThreads), 0, stream, ws.tiles > 0, ws.hist,
+                            ws.hist2, ws.psum, (int)ws.tiles, N, dims.T, ws.tile_off, ws.tile_off2, counts,
+                            ws.counts_first, ws.prob_total, aux, ws.ticket);
+        launch_end(stream);
+        if (err != cudaSuccess) return err;
+        launch_begin(xbuf_scatter ? K_ASSIGN_SCATTER : K_ASSIGN, stream);
+        if (xbuf_scatter)
+            err = launch_kernel(assign_top2_kernel<true>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
+                                expert, ws.tile_off, ws.tile_off2, counts, dims.T, N, C, (int)ws.tiles, slot,
+                                slot_token, xs, xb, x_words);
+        else
+            err = launch_kernel(assign_top2_kernel<false>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream,
+                                true, expert, ws.tile_off, ws.tile_off2, counts, dims.T, N, C, (int)ws.tiles, slot,
+                                slot_token, (const uint4 *)nullptr, (uint4 *)nullptr, 0);
+        launch_end(stream);
+        return err;
+    }
     // Small histograms: every assignment block sums the tile counts it needs
     // itself (at most kFusedScanLoads loads over the whole grid), saving the
     // scan kernel's launch and its round trip through memory.
@@ -926,14 +1126,12 @@ cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *
                             !(dims.flags & SWITCH_FLAG_SEPARATE_SCAN);
     if (!fused_scan) {
         launch_begin(K_SCAN, stream);
-        err = launch_kernel(scan_kernel, dim3(N), dim3(kScanThreads), 0, stream, ws.tiles > 0, ws.hist, ws.psum,
-                            (int)ws.tiles, N, dims.T, ws.tile_off, counts, ws.prob_total, aux, ws.ticket);
+        err = launch_kernel(scan_kernel<false>, dim3(N), dim3(kScanThreads), 0, stream, ws.tiles > 0, ws.hist,
+                            (const int32_t *)nullptr, ws.psum, (int)ws.tiles, N, dims.T, ws.tile_off,
+                            (int32_t *)nullptr, counts, (int32_t *)nullptr, ws.prob_total, aux, ws.ticket);
         launch_end(stream);
         if (err != cudaSuccess) return err;
     }
-    const int x_words = (int)((int64_t)dims.d_model * (dims.dtype == SWITCH_BF16 ? 2 : 4) / 16);
-    const uint4 *xs = static_cast<const uint4 *>(x);
-    uint4 *xb = static_cast<uint4 *>(xbuf_scatter);
     float4 *yz = reinterpret_cast<float4 *>(y_zero);
     const int y_words = dims.d_model / 4;
     const int32_t kid = xbuf_scatter ? K_ASSIGN_SCATTER : K_ASSIGN;

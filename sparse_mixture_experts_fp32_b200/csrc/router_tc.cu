@@ -76,7 +76,7 @@ __global__ void split_router_weight(const float *__restrict__ w, __nv_bfloat16 *
     }
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool TOP2 = false>
 struct RouterLayout {
     static constexpr size_t a_bytes = (size_t)RM * RK * 2;
     static constexpr size_t b_half_bytes = (size_t)(BN / 2) * RK * 2;  // BN/2 rows of one term
@@ -88,7 +88,9 @@ struct RouterLayout {
     // bias, per-quarter sums of p and per-64-token counts (both double-buffered by tile parity),
     // and the exchange of per-group max, argmax and sum between the warps of a token
     static constexpr size_t epi = (size_t)BN * 4 + 2 * 4 * BN * 4 + 2 * 2 * BN * 4 + 3 * (BN / 32) * RM * 4;
-    static constexpr size_t bytes = 1024 + ring + barriers + epi;
+    // top-2: second-choice counts and the exchange of each group's second best
+    static constexpr size_t epi2 = TOP2 ? 2 * 2 * BN * 4 + 2 * (BN / 32) * RM * 4 : 0;
+    static constexpr size_t bytes = 1024 + ring + barriers + epi + epi2;
 };
 
 // Sum v[i] over the 32 lanes for every i; lane l ends with the total of index l.
@@ -127,13 +129,28 @@ __device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const void *tma
         : "memory");
 }
 
-template <int BN, int STAGES>
+// Top-2 bookkeeping: keep the best two (value, index) pairs, larger value
+// first, lower index first among equal values, whatever the insertion order.
+__device__ __forceinline__ bool better_pair(float v, int i, float m, int a) { return v > m || (v == m && i < a); }
+__device__ __forceinline__ void insert_top2(float v, int i, float &m1, int &a1, float &m2, int &a2) {
+    if (better_pair(v, i, m1, a1)) {
+        m2 = m1;
+        a2 = a1;
+        m1 = v;
+        a1 = i;
+    } else if (better_pair(v, i, m2, a2)) {
+        m2 = v;
+        a2 = i;
+    }
+}
+
+template <int BN, int STAGES, bool TOP2>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::kAll, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const float *__restrict__ bias, int64_t T, int d, int N, int tiles64,
                      int32_t *__restrict__ expert, float *__restrict__ gate, int32_t *__restrict__ hist,
-                     float *__restrict__ psum, uint32_t *ticket, DeviceStatus *status) {
-    using L = RouterLayout<BN, STAGES>;
+                     int32_t *__restrict__ hist2, float *__restrict__ psum, uint32_t *ticket, DeviceStatus *status) {
+    using L = RouterLayout<BN, STAGES, TOP2>;
     constexpr int PM = 2 * RM;  // tokens per pair tile
     constexpr int G = RouterThreads<BN>::kGroups;
     constexpr int kEpiThreads = RouterThreads<BN>::kEpi;
@@ -153,6 +170,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
     float *x_max = reinterpret_cast<float *>(hist_s + 4 * BN);       // [G column groups][RM]
     int32_t *x_arg = reinterpret_cast<int32_t *>(x_max + G * RM);    // [G][RM]
     float *x_sum = reinterpret_cast<float *>(x_arg + G * RM);        // [G][RM]
+    // top-2 only (inside epi2): second-choice counts and each group's second best
+    int32_t *hist2_s = reinterpret_cast<int32_t *>(x_sum + G * RM);  // [2 parity][2 halves][BN]
+    float *x_max2 = reinterpret_cast<float *>(hist2_s + 4 * BN);     // [G][RM]
+    int32_t *x_arg2 = reinterpret_cast<int32_t *>(x_max2 + G * RM);  // [G][RM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -188,7 +209,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
     } else if (warp >= 2) {
         const int et = threadIdx.x - 64;
         for (int i = et; i < BN; i += kEpiThreads) bias_s[i] = (bias && i < N) ? bias[i] : 0.f;
-        for (int i = et; i < 4 * BN; i += kEpiThreads) hist_s[i] = 0;
+        for (int i = et; i < 4 * BN; i += kEpiThreads) {
+            hist_s[i] = 0;
+            if (TOP2) hist2_s[i] = 0;
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -308,6 +332,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
             }
             tc_fence_before();
             mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);  // columns in registers: reusable
+            float mx, mx2 = -FLT_MAX;
+            int amax, amax2 = 0x7fffffff;
+            if (TOP2) {
+                // best two of this group's 32 columns, then of all groups
+                float m1 = -FLT_MAX, m2 = -FLT_MAX;
+                int a1 = 0x7fffffff, a2 = 0x7fffffff;
+#pragma unroll
+                for (int j = 0; j < CW; ++j)
+                    if (col0 + j < N) insert_top2(h[j], col0 + j, m1, a1, m2, a2);
+                x_max[grp * RM + tok] = m1;
+                x_arg[grp * RM + tok] = a1;
+                x_max2[grp * RM + tok] = m2;
+                x_arg2[grp * RM + tok] = a2;
+                named_barrier_epilogue<kEpiThreads>();
+                m1 = x_max[tok];
+                a1 = x_arg[tok];
+                m2 = x_max2[tok];
+                a2 = x_arg2[tok];
+#pragma unroll
+                for (int g = 1; g < G; ++g) {
+                    insert_top2(x_max[g * RM + tok], x_arg[g * RM + tok], m1, a1, m2, a2);
+                    insert_top2(x_max2[g * RM + tok], x_arg2[g * RM + tok], m1, a1, m2, a2);
+                }
+                if (a1 == 0x7fffffff) a1 = 0;  // no comparable logit (NaN inputs): keep indices in range
+                if (a2 == 0x7fffffff) a2 = a1 == 0 ? 1 : 0;
+                mx = m1;
+                amax = a1;
+                mx2 = m2;
+                amax2 = a2;
+            } else {
             // four interleaved max / argmax chains (j = u mod 4), then merged with
             // ties going to the lowest index, as a single left-to-right scan would
             float m4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
@@ -334,8 +388,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
             x_max[grp * RM + tok] = m;
             x_arg[grp * RM + tok] = arg;
             named_barrier_epilogue<kEpiThreads>();
-            float mx = x_max[tok];
-            int amax = x_arg[tok];
+            mx = x_max[tok];
+            amax = x_arg[tok];
 #pragma unroll
             for (int g = 1; g < G; ++g) {  // groups in column order; strict: ties keep the lower index
                 const float v = x_max[g * RM + tok];
@@ -343,6 +397,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
                     mx = v;
                     amax = x_arg[g * RM + tok];
                 }
+            }
             }
             // __expf (hardware exp2 of a scaled argument): arguments are <= 0 here
             // and its relative error, a few 1e-6 over the range that matters, moves
@@ -373,8 +428,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
                 psum_p[q * BN + col0 + lane] = col_sum;
             }
             if (valid && grp == 0) {
-                expert[t] = amax;
-                gate[t] = inv_s;  // p at the argmax: exp(0) / s
+                if (TOP2) {
+                    expert[2 * t] = amax;
+                    expert[2 * t + 1] = amax2;
+                    gate[2 * t] = inv_s;
+                    gate[2 * t + 1] = __expf(mx2 - mx) * inv_s;
+                    atomicAdd(&hist2_s[par * 2 * BN + (q >> 1) * BN + amax2], 1);
+                } else {
+                    expert[t] = amax;
+                    gate[t] = inv_s;  // p at the argmax: exp(0) / s
+                }
                 atomicAdd(&hist_p[(q >> 1) * BN + amax], 1);
             }
             named_barrier_epilogue<kEpiThreads>();
@@ -387,8 +450,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
                     if (t64 < tiles64) {
                         hist[(int64_t)i * tiles64 + t64] = hist_p[h64 * BN + i];
                         psum[(int64_t)i * tiles64 + t64] = psum_p[(2 * h64) * BN + i] + psum_p[(2 * h64 + 1) * BN + i];
+                        if (TOP2) hist2[(int64_t)i * tiles64 + t64] = hist2_s[par * 2 * BN + h64 * BN + i];
                     }
                     hist_p[h64 * BN + i] = 0;
+                    if (TOP2) hist2_s[par * 2 * BN + h64 * BN + i] = 0;
                 }
             }
             par ^= 1;
@@ -424,7 +489,7 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool TOP2>
 cudaError_t launch_bn(const switch_dims_t &dims, const __nv_bfloat16 *x, const float *bias, int32_t *expert,
                       float *gate, const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts, d = dims.d_model;
@@ -451,16 +516,16 @@ cudaError_t launch_bn(const switch_dims_t &dims, const __nv_bfloat16 *x, const f
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    auto kern = router_tc_kernel<BN, STAGES>;
-    const size_t smem = RouterLayout<BN, STAGES>::bytes;
+    auto kern = router_tc_kernel<BN, STAGES, TOP2>;
+    const size_t smem = RouterLayout<BN, STAGES, TOP2>::bytes;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     const int64_t m_tiles = (T + 2 * RM - 1) / (2 * RM);
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / 2, m_tiles));
     launch_begin(K_ROUTER_TC, stream);
     err = launch_kernel(kern, dim3(2 * pairs), dim3(RouterThreads<BN>::kAll), smem, stream, true, tx, tw, bias, T, d,
-                        N, (int)ws.tiles,
-                        expert, gate, ws.hist, ws.psum, ws.ticket, static_cast<DeviceStatus *>(ws.status));
+                        N, (int)ws.tiles, expert, gate, ws.hist, ws.hist2, ws.psum, ws.ticket,
+                        static_cast<DeviceStatus *>(ws.status));
     launch_end(stream);
     return err;
 }
@@ -475,7 +540,7 @@ bool router_tc_supported(const switch_dims_t &dims) {
 }
 
 cudaError_t launch_router_tc(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
-                             int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
+                             int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream, bool top2) {
     const int64_t n = (int64_t)dims.num_experts * dims.d_model;
     launch_begin(K_ROUTER_SPLIT, stream);
     split_router_weight<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, stream>>>(
@@ -484,8 +549,12 @@ cudaError_t launch_router_tc(const switch_dims_t &dims, const void *x, const flo
     launch_end(stream);
     if (err != cudaSuccess) return err;
     const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
-    if (dims.num_experts <= 64) return launch_bn<64, 7>(dims, xb, bias, expert, gate, ws, stream);
-    return launch_bn<128, 5>(dims, xb, bias, expert, gate, ws, stream);
+    if (top2) {
+        if (dims.num_experts <= 64) return launch_bn<64, 7, true>(dims, xb, bias, expert, gate, ws, stream);
+        return launch_bn<128, 5, true>(dims, xb, bias, expert, gate, ws, stream);
+    }
+    if (dims.num_experts <= 64) return launch_bn<64, 7, false>(dims, xb, bias, expert, gate, ws, stream);
+    return launch_bn<128, 5, false>(dims, xb, bias, expert, gate, ws, stream);
 }
 
 }  // namespace switchmoe

@@ -112,3 +112,64 @@ def workload_inputs(wl: synth.Workload, T=None, oracle_route_first=None, orc=Non
     used = np.flatnonzero(np.minimum(o["counts"], C) > 0)
     inp["w_in"], inp["w_out"] = synth.all_expert_weights(wl, experts=used)
     return inp, o
+
+
+# ---------------------------------------------------------------------------
+# top-2 routing
+# ---------------------------------------------------------------------------
+def check_routing_top2(o: dict, g: dict, orc: oracle_mod.Oracle, N: int, C: int, T: int,
+                       check_slot_token=True) -> Report:
+    """o: oracle route_top2() result (with probs); g: numpy copies of the GPU outputs ([T, 2] per token).
+
+    A token whose first-choice margin is <= MARGIN may swap its two choices, and
+    one whose second-choice margin is <= MARGIN may pick another second choice;
+    every other token's two ids must equal the oracle's.  The capacity step is
+    then checked bit for bit on the GPU's own ids."""
+    rep = Report()
+    near1 = o["margin"][:, 0] <= MARGIN
+    near2 = o["margin"][:, 1] <= MARGIN
+    far = ~(near1 | near2)
+    diff = (g["expert"] != o["expert"]).any(axis=1)
+    mism = np.flatnonzero(diff & far)
+    assert mism.size == 0, f"{mism.size} top-2 ids differ on tokens with margins > {MARGIN}: {mism[:10]}"
+    rep["near_ties"] = int((~far).sum())
+    rep["flips"] = int((diff & ~far).sum())
+    a = orc.assign_top2(g["expert"], N, C)
+    assert np.array_equal(g["counts"], a["counts"]), "counts differ from the oracle's count of the GPU ids"
+    bad = np.flatnonzero((g["slot"] != a["slot"]).any(axis=1))
+    assert bad.size == 0, f"{bad.size} tokens' slots differ from the oracle's assignment of the GPU ids: {bad[:10]}"
+    if check_slot_token:
+        assert np.array_equal(g["slot_token"].reshape(N, C), a["slot_token"]), "slot_token differs"
+    if rep["flips"] == 0:
+        assert np.array_equal(g["slot"], o["slot"]) and np.array_equal(g["counts"], o["counts"])
+    if T > 0:
+        aux_ref = orc.aux(T, a["counts_first"], o["prob_sum"])
+        rel = abs(float(g["aux"]) - aux_ref) / abs(aux_ref)
+        assert rel <= AUX_RTOL, f"aux {float(g['aux'])} vs {aux_ref} (rel {rel:.3e})"
+        rep["aux_rel_err"] = rel
+        p_at = np.take_along_axis(o["probs"], g["expert"].astype(np.int64), axis=1)
+        gerr = float(np.abs(g["gate"].astype(np.float64) - p_at).max())
+        assert gerr <= GATE_ATOL, f"gate error {gerr}"
+        rep["gate_max_err"] = gerr
+    rep["assign"] = a
+    rep["dropped_choices"] = int((a["slot"] < 0).sum())
+    return rep
+
+
+def check_outputs_top2(y_gpu: np.ndarray, rows: np.ndarray, o: dict, rep: Report, orc, x, w_in, w_out, g_expert,
+                       fp32: bool) -> None:
+    """GPU output rows against the oracle's top-2 outputs computed with the GPU's ids."""
+    slot = rep["assign"]["slot"]
+    gate = np.take_along_axis(o["probs"], g_expert.astype(np.int64), axis=1)
+    ref = orc.output_rows_top2(rows, x, w_in, w_out, g_expert, slot, gate)
+    kept = (slot[rows] >= 0).any(axis=1)
+    if (~kept).any():
+        assert np.all(y_gpu[~kept] == 0.0), "a token with both choices dropped has a nonzero output row"
+    if kept.any():
+        rms = float(np.sqrt(np.mean(ref[kept] ** 2)))
+        err = float(np.abs(y_gpu[kept] - ref[kept]).max())
+        tol = (TOL_F32 if fp32 else TOL_BF16) * rms
+        rep["y_rms"] = rms
+        rep["y_max_abs_err"] = err
+        rep["y_err_over_rms"] = err / rms if rms > 0 else 0.0
+        assert err <= tol, f"max-abs output error {err:.4e} > {tol:.4e} (RMS {rms:.4e})"

@@ -28,7 +28,8 @@ def declared_functions():
 
 def test_header_declares_the_five_entry_points():
     names = declared_functions()
-    for n in ("switch_route", "switch_dispatch", "switch_expert_ffn", "switch_combine", "switch_layer_fwd"):
+    for n in ("switch_route", "switch_dispatch", "switch_expert_ffn", "switch_combine", "switch_layer_fwd",
+              "switch_route_top2", "switch_combine_top2", "switch_layer_fwd_top2"):
         assert n in names
 
 
@@ -105,6 +106,14 @@ def test_validation_errors_before_any_device_work(L):
     bad = sm.dims(64, 96, 64, 4, 16, sm.SWITCH_BF16)
     assert L.switch_layer_fwd(ctypes.byref(bad), a, a, None, a, a, a, a, a, a, a, a, a, 1 << 30, None) == 2
     assert L.switch_check(None, 0, None) == 1
+    # top-2 routing needs two experts; the same checks as the top-1 calls otherwise
+    one = sm.dims(64, 64, 64, 1, 16, sm.SWITCH_BF16)
+    assert L.switch_route_top2(ctypes.byref(one), a, a, None, a, a, a, a, a, a, a, 1 << 30, None) == 2
+    assert L.switch_layer_fwd_top2(ctypes.byref(one), a, a, None, a, a, a, a, a, a, a, a, a, 1 << 30, None) == 2
+    assert L.switch_combine_top2(ctypes.byref(one), a, a, a, a, a, None) == 2
+    assert L.switch_route_top2(ctypes.byref(d), a, a, None, a, a, a, a, a, a, a, 16, None) == 5
+    assert L.switch_layer_fwd_top2(ctypes.byref(d), a, None, None, a, a, a, a, a, a, a, a, a, 1 << 30, None) == 1
+    assert L.switch_combine_top2(ctypes.byref(d), a, a, a + 4, a, a, None) == 4
 
 
 def test_status_strings_and_kernel_names(L):
