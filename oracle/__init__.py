@@ -76,6 +76,9 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_assign_top2.restype = None
     lib.oracle_output_rows_top2.argtypes = [I32, I32, I64, P, P, ctypes.c_int, P, P, ctypes.c_int, P, P, P, P]
     lib.oracle_output_rows_top2.restype = None
+    lib.oracle_layer_bwd.argtypes = [I64, I32, I32, I32, I64, P, ctypes.c_int, P, P, P, P, ctypes.c_int, P, D,
+                                     P, P, P, P, P]
+    lib.oracle_layer_bwd.restype = None
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_set_threads.restype = None
     return lib
@@ -264,6 +267,30 @@ class Oracle:
         rows = np.arange(x.shape[0], dtype=np.int64)
         r["y"] = self.output_rows_top2(rows, x, w_in, w_out, r["expert"], r["slot"], r["gate"])
         return r
+
+    def layer_bwd(self, x, w_r, w_in, w_out, dy, g_aux: float = 0.0, bias=None, capacity=None,
+                  capacity_factor=None) -> dict:
+        """Gradients of sum(y * dy) + g_aux * aux with respect to x, W_r, the
+        logit bias, W_in and W_out (fp64), for the top-1 layer."""
+        x = np.ascontiguousarray(x)
+        T, d = x.shape
+        N, F, d2 = w_in.shape
+        assert d2 == d and w_out.shape == (N, d, F) and w_in.dtype == w_out.dtype
+        w_r = np.ascontiguousarray(w_r, dtype=np.float32)
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+        w_in = np.ascontiguousarray(w_in)
+        w_out = np.ascontiguousarray(w_out)
+        dy = np.ascontiguousarray(dy, dtype=np.float64)
+        assert dy.shape == (T, d)
+        if capacity is None:
+            capacity = self.capacity(T, N, capacity_factor)
+        out = dict(dx=np.empty((T, d)), dw_r=np.empty((N, d)), dbias=np.empty(N) if b is not None else None,
+                   dw_in=np.empty((N, F, d)), dw_out=np.empty((N, d, F)))
+        self.lib.oracle_layer_bwd(T, d, F, N, capacity, _ptr(x), dtype_code(x), _ptr(w_r), _ptr(b), _ptr(w_in),
+                                  _ptr(w_out), dtype_code(w_in), _ptr(dy), float(g_aux), _ptr(out["dx"]),
+                                  _ptr(out["dw_r"]), _ptr(out["dbias"]), _ptr(out["dw_in"]), _ptr(out["dw_out"]))
+        out["capacity"] = capacity
+        return out
 
     def expert_row(self, x_row, w_in_e, w_out_e, gate: float) -> np.ndarray:
         x_row = np.ascontiguousarray(x_row)

@@ -357,6 +357,168 @@ void oracle_output_rows_top2(int32_t d, int32_t F, int64_t n_rows, const int64_t
     }
 }
 
+/* ------------------------------------------------------------------------
+ * Backward pass of the top-1 layer.  The forward's loss enters as the
+ * upstream gradient dy[T,d] of the layer output y and a scalar g_aux, the
+ * upstream gradient of aux (the training loss adds alpha * aux, so g_aux is
+ * alpha).  The argmax and the capacity assignment are piecewise constant and
+ * pass no gradient; the gradient reaches the router through the selected
+ * probability p_{i*}(x) that scales the expert output (kasblo "Switch
+ * Transformerとは？", section "argmaxは離散なのに、Routerはなぜ学習できるのか")
+ * and, for the aux loss, through P_i only, f_i being a count
+ * (llm-papers-study "精读 06 | Switch Transformers" §3.3).  With z = W_in x,
+ * u = ReLU(z), o = W_out u and y = p_{i*} o for a kept token:
+ *   g_gate = dy . o,   do = p_{i*} dy
+ *   dW_out[i*] += do u^T,   du = W_out[i*]^T do,   dz = du (z > 0), 0 elsewhere
+ *   dW_in[i*]  += dz x^T,   dx += W_in[i*]^T dz
+ *   dp_i = [i = i*] g_gate + g_aux N f_i / T      (g_gate = 0 for a dropped token)
+ *   dh_i = p_i (dp_i - sum_j p_j dp_j)             (softmax backward)
+ *   dW_r += dh x^T,   db += dh,   dx += W_r^T dh
+ * All in double; gradients of weights are summed over tokens in token order.
+ * ------------------------------------------------------------------------ */
+void oracle_layer_bwd(int64_t T, int32_t d, int32_t F, int32_t N, int64_t C, const void *x, int x_dtype,
+                      const float *w_r, const float *bias, const void *w_in, const void *w_out, int w_dtype,
+                      const double *dy, double g_aux, double *dx, double *dw_r, double *dbias, double *dw_in,
+                      double *dw_out)
+{
+    int64_t Tn = T > 0 ? T : 1;
+    double *h = (double *)malloc(sizeof(double) * (size_t)Tn * (size_t)N);
+    double *p = (double *)malloc(sizeof(double) * (size_t)Tn * (size_t)N);
+    int32_t *expert = (int32_t *)malloc(sizeof(int32_t) * (size_t)Tn);
+    double *gate = (double *)malloc(sizeof(double) * (size_t)Tn);
+    double *margin = (double *)malloc(sizeof(double) * (size_t)Tn);
+    double *prob_sum = (double *)malloc(sizeof(double) * (size_t)N);
+    int32_t *slot = (int32_t *)malloc(sizeof(int32_t) * (size_t)Tn);
+    int32_t *counts = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+    int32_t *slot_token = (int32_t *)malloc(sizeof(int32_t) * (size_t)((int64_t)N * C > 0 ? (int64_t)N * C : 1));
+    double *g_gate = (double *)calloc((size_t)Tn, sizeof(double));
+
+    /* forward routing, exactly as the forward pass defines it */
+    oracle_router_logits(T, d, N, x, x_dtype, w_r, bias, h);
+    oracle_softmax_top1(T, N, h, expert, gate, margin, prob_sum, p);
+    oracle_assign(T, N, C, expert, slot, counts, slot_token);
+
+    for (int64_t i = 0; i < T * (int64_t)d; ++i)
+        dx[i] = 0.0;
+    for (int64_t i = 0; i < (int64_t)N * d; ++i)
+        dw_r[i] = 0.0;
+    if (dbias)
+        for (int32_t i = 0; i < N; ++i)
+            dbias[i] = 0.0;
+    for (int64_t i = 0; i < (int64_t)N * F * d; ++i) {
+        dw_in[i] = 0.0;
+        dw_out[i] = 0.0;
+    }
+
+    size_t esize = (w_dtype == ORACLE_BF16) ? 2 : 4;
+    /* expert path: one expert per thread, its tokens in token order */
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int32_t e = 0; e < N; ++e) {
+        const char *win_e = (const char *)w_in + (size_t)e * (size_t)F * (size_t)d * esize;
+        const char *wout_e = (const char *)w_out + (size_t)e * (size_t)d * (size_t)F * esize;
+        double *dwin_e = dw_in + (int64_t)e * F * d;
+        double *dwout_e = dw_out + (int64_t)e * d * F;
+        double *xt = (double *)malloc(sizeof(double) * (size_t)d);
+        double *z = (double *)malloc(sizeof(double) * (size_t)F);
+        double *u = (double *)malloc(sizeof(double) * (size_t)F);
+        double *o = (double *)malloc(sizeof(double) * (size_t)d);
+        double *dout = (double *)malloc(sizeof(double) * (size_t)d);
+        double *dz = (double *)malloc(sizeof(double) * (size_t)F);
+        for (int64_t t = 0; t < T; ++t) {
+            if (expert[t] != e || slot[t] < 0)
+                continue;
+            for (int32_t k = 0; k < d; ++k)
+                xt[k] = load_elem(x, x_dtype, t * (int64_t)d + k);
+            for (int32_t j = 0; j < F; ++j) {
+                double acc = 0.0;
+                for (int32_t k = 0; k < d; ++k)
+                    acc += load_elem(win_e, w_dtype, (int64_t)j * d + k) * xt[k];
+                z[j] = acc;
+                u[j] = acc > 0.0 ? acc : 0.0;
+            }
+            double gg = 0.0;
+            for (int32_t k = 0; k < d; ++k) {
+                double acc = 0.0;
+                for (int32_t j = 0; j < F; ++j)
+                    acc += load_elem(wout_e, w_dtype, (int64_t)k * F + j) * u[j];
+                o[k] = acc;
+                gg += dy[t * (int64_t)d + k] * acc;
+                dout[k] = gate[t] * dy[t * (int64_t)d + k];
+            }
+            g_gate[t] = gg;
+            for (int32_t k = 0; k < d; ++k)
+                for (int32_t j = 0; j < F; ++j)
+                    dwout_e[(int64_t)k * F + j] += dout[k] * u[j];
+            for (int32_t j = 0; j < F; ++j) {
+                double acc = 0.0;
+                for (int32_t k = 0; k < d; ++k)
+                    acc += load_elem(wout_e, w_dtype, (int64_t)k * F + j) * dout[k];
+                dz[j] = z[j] > 0.0 ? acc : 0.0;
+            }
+            for (int32_t j = 0; j < F; ++j)
+                for (int32_t k = 0; k < d; ++k)
+                    dwin_e[(int64_t)j * d + k] += dz[j] * xt[k];
+            for (int32_t k = 0; k < d; ++k) {
+                double acc = 0.0;
+                for (int32_t j = 0; j < F; ++j)
+                    acc += load_elem(win_e, w_dtype, (int64_t)j * d + k) * dz[j];
+                dx[t * (int64_t)d + k] += acc;
+            }
+        }
+        free(xt);
+        free(z);
+        free(u);
+        free(o);
+        free(dout);
+        free(dz);
+    }
+
+    /* router: softmax backward per token, then dh into dx, dW_r and db */
+    double *dh = (double *)malloc(sizeof(double) * (size_t)Tn * (size_t)N);
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const double *pt = p + t * (int64_t)N;
+        double *dht = dh + t * (int64_t)N;
+        double dot = 0.0;
+        for (int32_t i = 0; i < N; ++i) {
+            double dp = g_aux * (double)N * ((double)counts[i] / (double)T) / (double)T;
+            if (i == expert[t])
+                dp += g_gate[t];
+            dht[i] = dp;
+            dot += pt[i] * dp;
+        }
+        for (int32_t i = 0; i < N; ++i)
+            dht[i] = pt[i] * (dht[i] - dot);
+        for (int32_t k = 0; k < d; ++k) {
+            double router_part = 0.0;
+            for (int32_t i = 0; i < N; ++i)
+                router_part += (double)w_r[(int64_t)i * d + k] * dht[i];
+            dx[t * (int64_t)d + k] += router_part;
+        }
+    }
+#pragma omp parallel for schedule(static)
+    for (int32_t i = 0; i < N; ++i) {
+        for (int64_t t = 0; t < T; ++t) {
+            double g = dh[t * (int64_t)N + i];
+            for (int32_t k = 0; k < d; ++k)
+                dw_r[(int64_t)i * d + k] += g * load_elem(x, x_dtype, t * (int64_t)d + k);
+            if (dbias)
+                dbias[i] += g;
+        }
+    }
+    free(dh);
+    free(h);
+    free(p);
+    free(expert);
+    free(gate);
+    free(margin);
+    free(prob_sum);
+    free(slot);
+    free(counts);
+    free(slot_token);
+    free(g_gate);
+}
+
 /* Set the number of OpenMP threads the parallel loops above use (no effect
  * without OpenMP).  Used to time the oracle on one core and on all cores. */
 void oracle_set_threads(int n)

@@ -529,4 +529,148 @@ def pin_top2_invariants(o):
     assert np.all(r["y"][both_dropped] == 0.0)
 
 
+# --------------------------------------------------------------------------
+# Backward pass (gradients of sum(y * dy) + g_aux * aux)
+# --------------------------------------------------------------------------
+
+def _layer_loss(o, x, w_r, bias, w_in, w_out, C, dy, g_aux):
+    r = o.layer_fwd(x, w_r, w_in, w_out, bias=bias, capacity=C)
+    return float(np.sum(r["y"] * dy) + g_aux * r["aux"]), r["expert"], r["slot"]
+
+
+def _stable_problem(T, d, F, N, C, seed0):
+    """A float32 problem whose routing and ReLU pattern survive small perturbations:
+    top-2 logit margins >= 0.05 and |pre-activation| >= 0.05 on every kept token."""
+    for seed in range(seed0, seed0 + 500):
+        rng = np.random.default_rng(seed)
+        x, w_r, bias, w_in, w_out = _random_problem(rng, T, d, F, N)
+        w_r *= 3.0
+        x64 = x.astype(np.float64)
+        h = x64 @ w_r.astype(np.float64).T + bias
+        srt = np.sort(h, axis=1)
+        if N > 1 and (srt[:, -1] - srt[:, -2]).min() < 0.05:
+            continue
+        ids = np.argmax(h, axis=1)
+        z = np.einsum("tk,tjk->tj", x64, w_in[ids].astype(np.float64))
+        if np.abs(z).min() < 0.05:
+            continue
+        counts = np.bincount(ids, minlength=N)
+        if N > 1 and (counts <= C).all():
+            continue  # want some dropped tokens
+        return x, w_r, bias, w_in, w_out
+    raise AssertionError("no stable problem found")
+
+
+def pin_bwd_finite_differences(o):
+    # Central differences of the forward oracle's loss, one float32 element at a
+    # time (the perturbation is the exact float32 step taken); routing and the
+    # ReLU pattern stay fixed under the step, so the loss is smooth there.
+    T, d, F, N, C = 7, 4, 5, 3, 2
+    x, w_r, bias, w_in, w_out = _stable_problem(T, d, F, N, C, 300)
+    rng = np.random.default_rng(31)
+    dy = rng.standard_normal((T, d))
+    g_aux = 0.7
+    g = o.layer_bwd(x, w_r, w_in, w_out, dy, g_aux, bias=bias, capacity=C)
+    _, ids0, slot0 = _layer_loss(o, x, w_r, bias, w_in, w_out, C, dy, g_aux)
+    assert (slot0 < 0).any() and (slot0 >= 0).any()
+    params = {"x": (x, "dx"), "w_r": (w_r, "dw_r"), "bias": (bias, "dbias"), "w_in": (w_in, "dw_in"),
+              "w_out": (w_out, "dw_out")}
+    for name, (arr, gname) in params.items():
+        flat = arr.reshape(-1)
+        num = np.zeros(flat.size)
+        for i in range(flat.size):
+            v = flat[i]
+            steps = []
+            for sgn in (1.0, -1.0):
+                flat[i] = np.float32(v + sgn * np.float32(2.0 ** -11) * max(1.0, abs(float(v))))
+                steps.append((float(flat[i]) - float(v),
+                              _layer_loss(o, x, w_r, bias, w_in, w_out, C, dy, g_aux)))
+                flat[i] = v
+            (dp, (lp, ip, sp)), (dm, (lm, im, sm_)) = steps
+            assert np.array_equal(ip, ids0) and np.array_equal(im, ids0), (name, i)
+            assert np.array_equal(sp, slot0) and np.array_equal(sm_, slot0), (name, i)
+            num[i] = (lp - lm) / (dp - dm)
+        ana = g[gname].reshape(-1)
+        scale = max(1.0, float(np.abs(ana).max()))
+        assert np.allclose(num, ana, rtol=2e-5, atol=2e-5 * scale), (name, np.abs(num - ana).max())
+
+
+def pin_bwd_matches_torch_autograd(o):
+    # A dense formulation in torch (every expert on every token, masks from the
+    # argmax and the first-C rule, gate = selected probability, f held constant),
+    # differentiated by torch.autograd in float64.
+    import torch
+    for seed, (T, d, F, N, C, g_aux) in enumerate([(40, 8, 12, 4, 8, 0.3), (25, 6, 10, 3, 25, 0.0),
+                                                   (30, 5, 7, 5, 3, 1.5)]):
+        rng = np.random.default_rng(140 + seed)
+        x, w_r, bias, w_in, w_out = _random_problem(rng, T, d, F, N)
+        dy = rng.standard_normal((T, d))
+        g = o.layer_bwd(x, w_r, w_in, w_out, dy, g_aux, bias=bias, capacity=C)
+        tx, twr, tb = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (x, w_r, bias))
+        twi, two = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (w_in, w_out))
+        h = tx @ twr.T + tb
+        p = torch.softmax(h, dim=1)
+        ids = torch.argmax(h, dim=1)
+        keep = torch.zeros(T, dtype=torch.float64)
+        seen = [0] * N
+        for t in range(T):
+            e = int(ids[t])
+            keep[t] = 1.0 if seen[e] < C else 0.0
+            seen[e] += 1
+        z = torch.einsum("tk,ejk->etj", tx, twi)
+        out = torch.einsum("etj,ekj->etk", torch.relu(z), two)
+        o_sel = out[ids, torch.arange(T)]
+        gate = p[torch.arange(T), ids]
+        y = keep[:, None] * gate[:, None] * o_sel
+        f = torch.tensor(np.bincount(ids.numpy(), minlength=N) / T, dtype=torch.float64)
+        aux = N * torch.sum(f * p.mean(dim=0))
+        loss = torch.sum(y * torch.tensor(dy)) + g_aux * aux
+        loss.backward()
+        for name, tg in (("dx", tx), ("dw_r", twr), ("dbias", tb), ("dw_in", twi), ("dw_out", two)):
+            assert np.allclose(g[name], tg.grad.numpy(), rtol=1e-11, atol=1e-12), (name, seed)
+
+
+def pin_bwd_single_expert(o):
+    # N = 1: p = 1 identically, so the router gets no gradient (even from aux),
+    # and dx is the dense FFN's backward (numpy closed form).
+    rng = np.random.default_rng(32)
+    T, d, F = 12, 6, 9
+    x, w_r, bias, w_in, w_out = _random_problem(rng, T, d, F, 1)
+    dy = rng.standard_normal((T, d))
+    g = o.layer_bwd(x, w_r, w_in, w_out, dy, 2.0, bias=bias, capacity=T)
+    assert np.all(g["dw_r"] == 0.0) and np.all(g["dbias"] == 0.0)
+    x64, wi, wo = x.astype(np.float64), w_in[0].astype(np.float64), w_out[0].astype(np.float64)
+    z = x64 @ wi.T
+    du = dy @ wo
+    dz = du * (z > 0)
+    assert np.allclose(g["dx"], dz @ wi, rtol=1e-12, atol=1e-13)
+    assert np.allclose(g["dw_out"][0], dy.T @ np.maximum(z, 0), rtol=1e-12, atol=1e-13)
+    assert np.allclose(g["dw_in"][0], dz.T @ x64, rtol=1e-12, atol=1e-13)
+
+
+def pin_bwd_aux_only_and_dropped(o):
+    # dy = 0: the expert weights get no gradient and the router gradient is the
+    # aux term alone, dh_i = p_i (c_i - sum_j p_j c_j) with c_i = g_aux N f_i / T.
+    # With g_aux = 0 a dropped token gets no gradient at all.
+    rng = np.random.default_rng(33)
+    T, d, F, N, C = 30, 6, 8, 4, 5
+    x, w_r, bias, w_in, w_out = _random_problem(rng, T, d, F, N)
+    g = o.layer_bwd(x, w_r, w_in, w_out, np.zeros((T, d)), 1.3, bias=bias, capacity=C)
+    assert np.all(g["dw_in"] == 0.0) and np.all(g["dw_out"] == 0.0)
+    x64 = x.astype(np.float64)
+    h = x64 @ w_r.astype(np.float64).T + bias
+    p = scipy.special.softmax(h, axis=1)
+    f = np.bincount(np.argmax(h, axis=1), minlength=N) / T
+    c = 1.3 * N * f / T
+    dh = p * (c - (p * c).sum(axis=1, keepdims=True))
+    assert np.allclose(g["dw_r"], dh.T @ x64, rtol=1e-12, atol=1e-14)
+    assert np.allclose(g["dbias"], dh.sum(axis=0), rtol=1e-12, atol=1e-14)
+    assert np.allclose(g["dx"], dh @ w_r.astype(np.float64), rtol=1e-12, atol=1e-14)
+    dy = rng.standard_normal((T, d))
+    g0 = o.layer_bwd(x, w_r, w_in, w_out, dy, 0.0, bias=bias, capacity=C)
+    slot = o.route(x, w_r, bias, capacity=C)["slot"]
+    assert (slot < 0).any()
+    assert np.all(g0["dx"][slot < 0] == 0.0)
+
+
 PINS = {name: fn for name, fn in sorted(globals().items()) if name.startswith("pin_") and callable(fn)}

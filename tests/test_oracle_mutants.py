@@ -69,6 +69,20 @@ MUTANTS = {
     # top-2 output: second choice never added
     "top2_output_first_only": ("for (int c = 0; c < 2; ++c) {\n            if (slot2[2 * t + c] < 0)",
                                "for (int c = 0; c < 1; ++c) {\n            if (slot2[2 * t + c] < 0)"),
+    # backward: ReLU mask dropped; gate missing from the expert-output gradient
+    "bwd_relu_mask_dropped": ("dz[j] = z[j] > 0.0 ? acc : 0.0;", "dz[j] = acc;"),
+    "bwd_gate_missing": ("dout[k] = gate[t] * dy[t * (int64_t)d + k];", "dout[k] = dy[t * (int64_t)d + k];"),
+    # softmax backward with the wrong sign of the centring term
+    "bwd_softmax_sign": ("dht[i] = pt[i] * (dht[i] - dot);", "dht[i] = pt[i] * (dht[i] + dot);"),
+    "bwd_aux_missing_N": ("double dp = g_aux * (double)N * ((double)counts[i] / (double)T) / (double)T;",
+                          "double dp = g_aux * ((double)counts[i] / (double)T) / (double)T;"),
+    # dropped tokens still back-propagate through the expert
+    "bwd_dropped_tokens_pass": ("if (expert[t] != e || slot[t] < 0)\n                continue;",
+                                "if (expert[t] != e)\n                continue;"),
+    "bwd_dw_out_transposed": ("dwout_e[(int64_t)k * F + j] += dout[k] * u[j];",
+                              "dwout_e[(int64_t)j * d + k] += dout[k] * u[j];"),
+    "bwd_router_dx_missing": ("dx[t * (int64_t)d + k] += router_part;", "dx[t * (int64_t)d + k] += 0.0 * router_part;"),
+    "bwd_gate_grad_uses_dy_only": ("gg += dy[t * (int64_t)d + k] * acc;", "gg += dy[t * (int64_t)d + k];"),
     # bf16 loads: wrong half of the 32-bit pattern
     "bf16_wrong_shift": ("uint32_t wide = (uint32_t)bits << 16;", "uint32_t wide = (uint32_t)bits << 15;"),
 }
