@@ -434,7 +434,7 @@ void oracle_layer_bwd(int64_t T, int32_t d, int32_t F, int32_t N, int64_t C, con
                 for (int32_t k = 0; k < d; ++k)
                     acc += load_elem(win_e, w_dtype, (int64_t)j * d + k) * xt[k];
                 z[j] = acc;
-                u[j] = acc > 0.0 ? acc : 0.0;
+                u[j] = z[j] > 0.0 ? z[j] : 0.0;
             }
             double gg = 0.0;
             for (int32_t k = 0; k < d; ++k) {
@@ -492,7 +492,7 @@ void oracle_layer_bwd(int64_t T, int32_t d, int32_t F, int32_t N, int64_t C, con
         for (int32_t k = 0; k < d; ++k) {
             double router_part = 0.0;
             for (int32_t i = 0; i < N; ++i)
-                router_part += (double)w_r[(int64_t)i * d + k] * dht[i];
+                router_part += dht[i] * w_r[(int64_t)i * d + k]; /* float -> double, exact */
             dx[t * (int64_t)d + k] += router_part;
         }
     }

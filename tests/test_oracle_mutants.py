@@ -71,6 +71,7 @@ MUTANTS = {
                                "for (int c = 0; c < 1; ++c) {\n            if (slot2[2 * t + c] < 0)"),
     # backward: ReLU mask dropped; gate missing from the expert-output gradient
     "bwd_relu_mask_dropped": ("dz[j] = z[j] > 0.0 ? acc : 0.0;", "dz[j] = acc;"),
+    "bwd_forward_relu_dropped": ("u[j] = z[j] > 0.0 ? z[j] : 0.0;", "u[j] = z[j];"),
     "bwd_gate_missing": ("dout[k] = gate[t] * dy[t * (int64_t)d + k];", "dout[k] = dy[t * (int64_t)d + k];"),
     # softmax backward with the wrong sign of the centring term
     "bwd_softmax_sign": ("dht[i] = pt[i] * (dht[i] - dot);", "dht[i] = pt[i] * (dht[i] + dot);"),
@@ -81,6 +82,8 @@ MUTANTS = {
                                 "if (expert[t] != e)\n                continue;"),
     "bwd_dw_out_transposed": ("dwout_e[(int64_t)k * F + j] += dout[k] * u[j];",
                               "dwout_e[(int64_t)j * d + k] += dout[k] * u[j];"),
+    "bwd_router_dx_transposed_weight": ("router_part += dht[i] * w_r[(int64_t)i * d + k];",
+                                        "router_part += dht[i] * w_r[(int64_t)k * N + i];"),
     "bwd_router_dx_missing": ("dx[t * (int64_t)d + k] += router_part;", "dx[t * (int64_t)d + k] += 0.0 * router_part;"),
     "bwd_gate_grad_uses_dy_only": ("gg += dy[t * (int64_t)d + k] * acc;", "gg += dy[t * (int64_t)d + k];"),
     # bf16 loads: wrong half of the 32-bit pattern
