@@ -92,7 +92,13 @@ enum {
      * counts it needs itself and the scan kernel is skipped; both give the
      * same slots and counts (aux may differ in the last bits: its fp64 sums
      * run in another fixed order). */
-    SWITCH_FLAG_SEPARATE_SCAN = 16
+    SWITCH_FLAG_SEPARATE_SCAN = 16,
+    /* Training: switch_layer_fwd keeps what the backward pass needs in the
+     * workspace (the router probabilities, the dispatched tokens, the hidden
+     * activations and the ungated expert outputs) and runs the two expert
+     * GEMMs and the combine as separate launches; switch_workspace_size grows
+     * accordingly.  switch_layer_bwd requires it.  bfloat16 experts only. */
+    SWITCH_FLAG_TRAINING = 32
 };
 
 typedef struct {
@@ -240,6 +246,33 @@ switch_status_t switch_layer_fwd_top2(const switch_dims_t *dims, const void *x, 
                                       const float *logit_bias, const void *w_in, const void *w_out, void *y,
                                       int32_t *expert, float *gate, int32_t *slot, int32_t *counts, float *aux,
                                       void *workspace, size_t workspace_bytes, switch_stream_t stream);
+
+/* Backward pass of the layer (top-1), after a switch_layer_fwd call made with
+ * SWITCH_FLAG_TRAINING in the same dims and the same workspace (whose
+ * contents that call left behind are its input here).  The loss is
+ * L = sum(y * dy) + g_aux * aux; the argmax and the capacity assignment pass no
+ * gradient: the router learns through the selected probability p_i*(x) that
+ * scales the expert output (kasblo "Switch Transformerとは？", section
+ * "argmaxは離散なのに、Routerはなぜ学習できるのか") and, for the aux loss,
+ * through P_i only, f_i being a count (llm-papers-study §3.3).
+ *   x, w_r, w_in, w_out       the forward's inputs; expert, gate, slot, counts
+ *                             the forward's outputs (as it wrote them)
+ *   dy [T, d] float32         upstream gradient of y
+ *   g_aux                     upstream gradient of aux (the loss weight alpha)
+ * Outputs (float32, all written): dx [T, d]; dw_r [N, d]; dbias [N] (the
+ * gradient of the logit bias; NULL to skip); dw_in [N, F, d]; dw_out [N, d, F]
+ * (zero for experts without kept tokens).  A dropped token's dx is the router
+ * part only.  The expert GEMMs run on tcgen05 tensor cores with bfloat16
+ * operands (gate * dy and the pre-activation gradient rounded to bfloat16) and
+ * float32 accumulation; the router part runs in float32.  Deterministic.
+ * Errors: SWITCH_ERR_UNSUPPORTED without SWITCH_FLAG_TRAINING, for float32
+ * experts or with SWITCH_FLAG_SIMT_FFN / SWITCH_FLAG_GEMM_1CTA; SWITCH_ERR_SHAPE
+ * for a non-finite g_aux; otherwise as switch_layer_fwd. */
+switch_status_t switch_layer_bwd(const switch_dims_t *dims, const void *x, const float *w_r, const void *w_in,
+                                 const void *w_out, const int32_t *expert, const float *gate, const int32_t *slot,
+                                 const int32_t *counts, const float *dy, float g_aux, float *dx, float *dw_r,
+                                 float *dbias, float *dw_in, float *dw_out, void *workspace, size_t workspace_bytes,
+                                 switch_stream_t stream);
 
 /* Routing without a workspace, for callers that cannot allocate device
  * memory at the point where they route tokens: code running under a host

@@ -31,6 +31,7 @@ SWITCH_FLAG_SIMT_ROUTER = 2
 SWITCH_FLAG_GEMM_1CTA = 4
 SWITCH_FLAG_FFN_TWO_LAUNCHES = 8
 SWITCH_FLAG_SEPARATE_SCAN = 16
+SWITCH_FLAG_TRAINING = 32
 
 STATUS = {
     0: "SWITCH_OK", 1: "SWITCH_ERR_NULL", 2: "SWITCH_ERR_SHAPE", 3: "SWITCH_ERR_DTYPE", 4: "SWITCH_ERR_ALIGN",
@@ -41,6 +42,7 @@ STATUS = {
 EXPORTED = ("switch_capacity", "switch_workspace_size", "switch_route", "switch_route_noalloc", "switch_dispatch",
             "switch_expert_ffn",
             "switch_combine", "switch_layer_fwd", "switch_route_top2", "switch_combine_top2", "switch_layer_fwd_top2",
+            "switch_layer_bwd",
             "switch_check", "switch_selftest_wait_timeout", "switch_status_string",
             "switch_launch_count",
             "switch_trace_start", "switch_trace_read", "switch_trace_stop", "switch_kernel_name")
@@ -88,6 +90,7 @@ def lib() -> ctypes.CDLL:
         "switch_route_top2": (I, [D, P, P, P, P, P, P, P, P, P, P, S, P]),
         "switch_combine_top2": (I, [D, P, P, P, P, P, P]),
         "switch_layer_fwd_top2": (I, [D, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
+        "switch_layer_bwd": (I, [D, P, P, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, P, P, S, P]),
         "switch_check": (I, [P, S, P]),
         "switch_selftest_wait_timeout": (I, [P, S, P]),
         "switch_status_string": (ctypes.c_char_p, [I]),
@@ -228,6 +231,15 @@ def switch_layer_fwd_top2(d, x, w_r, logit_bias, w_in, w_out, y, expert, gate, s
                                     _stream(stream, workspace)), "switch_layer_fwd_top2")
 
 
+def switch_layer_bwd(d, x, w_r, w_in, w_out, expert, gate, slot, counts, dy, g_aux, dx, dw_r, dbias, dw_in, dw_out,
+                     workspace, stream=None):
+    _ok(lib().switch_layer_bwd(ctypes.byref(d), _ptr(x), _ptr(w_r), _ptr(w_in), _ptr(w_out), _ptr(expert),
+                               _ptr(gate), _ptr(slot), _ptr(counts), _ptr(dy), float(g_aux), _ptr(dx), _ptr(dw_r),
+                               _ptr(dbias), _ptr(dw_in), _ptr(dw_out), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream, workspace)),
+        "switch_layer_bwd")
+
+
 def switch_check(workspace, stream=None) -> int:
     """Synchronise and return the device status code (0 = ok); does not raise."""
     return int(lib().switch_check(_ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -315,6 +327,7 @@ def layer_fwd(x, w_r, w_in, w_out, capacity=None, capacity_factor=None, logit_bi
     switch_layer_fwd(d, x, w_r, logit_bias, w_in, w_out, out["y"], out["expert"], out["gate"], out["slot"],
                      out["counts"], out["aux"], ws, stream)
     out["capacity"] = d.capacity
+    out["flags"] = d.flags
     out["workspace"] = ws
     return out
 
@@ -387,4 +400,23 @@ def route_top2(x, w_r, capacity=None, capacity_factor=None, logit_bias=None, d_f
                       out["slot_token"], out["aux"], ws, stream)
     out["capacity"] = C
     out["workspace"] = ws
+    return out
+
+
+def layer_bwd(fwd: dict, x, w_r, w_in, w_out, dy, g_aux: float = 0.0, logit_bias=None, stream=None):
+    """Gradients of sum(y * dy) + g_aux * aux after ``layer_fwd(..., flags=SWITCH_FLAG_TRAINING)``
+    (whose result dict, with its workspace, is ``fwd``).  Returns dx, dw_r, dbias
+    (None without a logit bias), dw_in, dw_out, all float32."""
+    import torch
+    T, dm = x.shape
+    N, F, _ = w_in.shape
+    dev = x.device
+    d = layer_dims(x, w_in, capacity=fwd["capacity"], flags=fwd.get("flags", SWITCH_FLAG_TRAINING))
+    out = dict(dx=torch.empty(T, dm, dtype=torch.float32, device=dev),
+               dw_r=torch.empty(N, dm, dtype=torch.float32, device=dev),
+               dbias=torch.empty(N, dtype=torch.float32, device=dev) if logit_bias is not None else None,
+               dw_in=torch.empty(N, F, dm, dtype=torch.float32, device=dev),
+               dw_out=torch.empty(N, dm, F, dtype=torch.float32, device=dev))
+    switch_layer_bwd(d, x, w_r, w_in, w_out, fwd["expert"], fwd["gate"], fwd["slot"], fwd["counts"], dy, g_aux,
+                     out["dx"], out["dw_r"], out["dbias"], out["dw_in"], out["dw_out"], fwd["workspace"], stream)
     return out

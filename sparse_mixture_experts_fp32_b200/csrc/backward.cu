@@ -1,0 +1,348 @@
+// Backward pass of the Switch layer (top-1, bfloat16 experts), sm_100a.
+//
+// Given the upstream gradient dy [T, d] of the layer output y and the scalar
+// upstream gradient g_aux of the aux loss, computes dx, dW_r, d(logit bias),
+// dW_in and dW_out.  The argmax and the capacity assignment pass no gradient:
+// the router learns through the selected probability p_i*(x) that scales the
+// expert output (kasblo "Switch Transformerとは？", section "argmaxは離散なの
+// に、Routerはなぜ学習できるのか"), and through P_i in the aux loss, f_i being
+// a count (llm-papers-study "精读 06 | Switch Transformers" §3.3).  With
+// z = W_in x, u = ReLU(z), o = W_out u, y = p_i* o for a kept token:
+//   g_gate = dy . o                      dE = p_i* dy          (bwd_token_kernel)
+//   dp_i = [i = i*] g_gate + g_aux N f_i / T,  dh = p (dp - p . dp)
+//   dZ = (dE W_out[i*]) masked by z > 0  (tcgen05 GEMM, epilogue kEpiReluGrad)
+//   dx = dh W_r + dZ W_in[i*]            (router_dx_kernel, then a tcgen05 GEMM
+//                                         whose epilogue adds into dx rows)
+//   dW_out[i] = sum over kept tokens of dE u^T   (tcgen05 GEMM over K = tokens)
+//   dW_in[i]  = sum over kept tokens of dZ x^T   (tcgen05 GEMM over K = tokens)
+//   dW_r = sum_t dh x^T, d bias = sum_t dh        (router_dw_kernel + fixed-order reduce)
+// The expert GEMMs are the forward's grouped "A . B^T" kernel with both
+// operands K-major: the weights and the per-expert activation buffers are
+// first transposed in HBM (batched 64 x 64 tile transposes; rows past an
+// expert's kept tokens become zeros, so the weight-gradient GEMMs only see
+// kept tokens).  Every reduction runs in a fixed order: identical inputs give
+// identical bytes.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace switchmoe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+// One warp per token: the gate gradient g_gate = dy . o (o = the forward's
+// ungated expert output), dE[e, s] = bf16(gate * dy) for a kept token, then
+// the softmax backward over the N probabilities kept by the forward.
+__global__ void __launch_bounds__(kThreads) bwd_token_kernel(const float *__restrict__ dy, const float *__restrict__ ybuf,
+                                                            const int32_t *__restrict__ expert,
+                                                            const int32_t *__restrict__ slot,
+                                                            const float *__restrict__ gate,
+                                                            const float *__restrict__ probs,
+                                                            const int32_t *__restrict__ counts, int64_t T, int d,
+                                                            int N, int C, float g_aux, __nv_bfloat16 *__restrict__ dE,
+                                                            float *__restrict__ dh) {
+    const int64_t t = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const int lane = threadIdx.x & 31;
+    const int s = slot[t], e = expert[t];
+    float g = 0.f;
+    if (s >= 0) {
+        const float gt = gate[t];
+        const float4 *o = reinterpret_cast<const float4 *>(ybuf + ((int64_t)e * C + s) * d);
+        const float4 *dyt = reinterpret_cast<const float4 *>(dy + t * d);
+        uint2 *de = reinterpret_cast<uint2 *>(dE + ((int64_t)e * C + s) * d);
+        float acc = 0.f;
+        for (int w = lane; w < d / 4; w += 32) {
+            const float4 a = __ldg(dyt + w), b = __ldg(o + w);
+            acc = fmaf(a.x, b.x, acc);
+            acc = fmaf(a.y, b.y, acc);
+            acc = fmaf(a.z, b.z, acc);
+            acc = fmaf(a.w, b.w, acc);
+            de[w] = make_uint2(pack_bf16x2(gt * a.x, gt * a.y), pack_bf16x2(gt * a.z, gt * a.w));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        g = acc;
+    }
+    const float *pt = probs + t * N;
+    const float c_aux = g_aux * (float)N / ((float)T * (float)T);
+    float dot = 0.f;
+    for (int i = lane; i < N; i += 32) {
+        const float dp = (i == e ? g : 0.f) + c_aux * (float)counts[i];
+        dot = fmaf(pt[i], dp, dot);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    for (int i = lane; i < N; i += 32) {
+        const float dp = (i == e ? g : 0.f) + c_aux * (float)counts[i];
+        dh[t * N + i] = pt[i] * (dp - dot);
+    }
+}
+
+// Batched transpose of bf16 matrices: in [B][R][Cc] -> out [B][Cc][Rp].
+// Rows r >= valid(b) of the input (valid = min(counts[b], cap) when counts is
+// given, else R) and the padding rows up to Rp become zeros.  64 x 64 tiles,
+// 32-bit (two-element) accesses on both sides.
+constexpr int kTT = 64;
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t *__restrict__ in, uint16_t *__restrict__ out,
+                                                            int R, int Cc, int Rp, const int32_t *__restrict__ counts,
+                                                            int cap) {
+    __shared__ uint16_t tile[kTT][kTT + 2];
+    const int b = blockIdx.z;
+    const int c0 = blockIdx.x * kTT, r0 = blockIdx.y * kTT;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    const int valid = counts ? min(min(counts[b], cap), R) : R;
+    const uint16_t *src = in + (int64_t)b * R * Cc;
+    uint16_t *dst = out + (int64_t)b * Cc * Rp;
+#pragma unroll
+    for (int j = 0; j < kTT / 8; ++j) {
+        const int r = r0 + ty + 8 * j;
+        const int c = c0 + 2 * tx;
+        uint32_t v = 0u;
+        if (r < valid && c + 1 < Cc) v = *reinterpret_cast<const uint32_t *>(src + (int64_t)r * Cc + c);
+        else if (r < valid && c < Cc) v = src[(int64_t)r * Cc + c];
+        tile[ty + 8 * j][2 * tx] = (uint16_t)(v & 0xffffu);
+        tile[ty + 8 * j][2 * tx + 1] = (uint16_t)(v >> 16);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kTT / 8; ++j) {
+        const int c = c0 + ty + 8 * j;  // output row
+        const int r = r0 + 2 * tx;      // output columns r, r + 1
+        if (c < Cc && r + 1 < Rp) {
+            const uint32_t v = (uint32_t)tile[2 * tx][ty + 8 * j] | ((uint32_t)tile[2 * tx + 1][ty + 8 * j] << 16);
+            *reinterpret_cast<uint32_t *>(dst + (int64_t)c * Rp + r) = v;
+        } else if (c < Cc && r < Rp) {
+            dst[(int64_t)c * Rp + r] = tile[2 * tx][ty + 8 * j];
+        }
+    }
+}
+
+// dx[t, :] = sum_i dh[t, i] W_r[i, :]  (overwrites dx; the expert part is
+// added afterwards).  Block: 32 tokens x 128 columns; thread: 4 tokens x 4
+// columns; experts in chunks of 32 through shared memory.
+constexpr int kDxTok = 32, kDxCol = 128, kDxI = 32;
+__global__ void __launch_bounds__(256) router_dx_kernel(const float *__restrict__ dh, const float *__restrict__ w_r,
+                                                       int64_t T, int N, int d, float *__restrict__ dx) {
+    __shared__ float s_dh[kDxI][kDxTok + 1];
+    __shared__ __align__(16) float s_w[kDxI][kDxCol];
+    const int64_t t0 = (int64_t)blockIdx.y * kDxTok;
+    const int k0 = blockIdx.x * kDxCol;
+    const int tid = threadIdx.x;
+    const int tc = tid & 31;   // columns k0 + 4 tc .. + 3
+    const int tt = tid >> 5;   // tokens t0 + tt + 8 j, j < 4
+    float acc[4][4] = {};
+    for (int i0 = 0; i0 < N; i0 += kDxI) {
+        __syncthreads();
+        for (int q = tid; q < kDxI * kDxTok; q += 256) {
+            const int ii = q % kDxI, tl = q / kDxI;
+            const int64_t t = t0 + tl;
+            s_dh[ii][tl] = (t < T && i0 + ii < N) ? dh[t * N + i0 + ii] : 0.f;
+        }
+        for (int q = tid; q < kDxI * kDxCol; q += 256) {
+            const int ii = q / kDxCol, kk = q % kDxCol;
+            s_w[ii][kk] = (i0 + ii < N && k0 + kk < d) ? w_r[(int64_t)(i0 + ii) * d + k0 + kk] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int ii = 0; ii < kDxI; ++ii) {
+            const float4 w = *reinterpret_cast<const float4 *>(&s_w[ii][4 * tc]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float a = s_dh[ii][tt + 8 * j];
+                acc[j][0] = fmaf(a, w.x, acc[j][0]);
+                acc[j][1] = fmaf(a, w.y, acc[j][1]);
+                acc[j][2] = fmaf(a, w.z, acc[j][2]);
+                acc[j][3] = fmaf(a, w.w, acc[j][3]);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int64_t t = t0 + tt + 8 * j;
+        const int k = k0 + 4 * tc;
+        if (t < T && k < d)  // d % 64 == 0 on this path: the four columns are in range together
+            *reinterpret_cast<float4 *>(dx + t * d + k) = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+    }
+}
+
+// Partial sums of dW_r and d bias over chunks of tokens:
+//   part_w[chunk][i][k] = sum_{t in chunk} dh[t, i] x[t, k],  part_b[chunk][i] = sum dh[t, i]
+// Block: 64 experts x 128 columns of one chunk; thread: 4 experts x 8 columns.
+constexpr int kDwI = 64, kDwCol = 128, kDwTok = 32;
+__global__ void __launch_bounds__(256) router_dw_kernel(const float *__restrict__ dh, const uint16_t *__restrict__ x,
+                                                       int64_t T, int N, int d, int64_t chunk_tokens,
+                                                       float *__restrict__ part_w, float *__restrict__ part_b) {
+    __shared__ float s_dh[kDwTok][kDwI + 1];
+    __shared__ __align__(16) float s_x[kDwTok][kDwCol];
+    const int k0 = blockIdx.x * kDwCol, i0 = blockIdx.y * kDwI;
+    const int chunk = blockIdx.z;
+    const int64_t tbeg = (int64_t)chunk * chunk_tokens;
+    const int64_t tend = min(T, tbeg + chunk_tokens);
+    const int tid = threadIdx.x;
+    const int tk = tid & 15;   // columns k0 + 8 tk .. + 7
+    const int ti = tid >> 4;   // experts i0 + ti + 16 j, j < 4
+    float acc[4][8] = {};
+    float accb4[4] = {0.f, 0.f, 0.f, 0.f};  // threads with tk == 0: d bias of experts i0 + ti + 16 j
+    for (int64_t tb = tbeg; tb < tend; tb += kDwTok) {
+        __syncthreads();
+        for (int q = tid; q < kDwTok * kDwI; q += 256) {
+            const int ii = q % kDwI, tl = q / kDwI;
+            const int64_t t = tb + tl;
+            s_dh[tl][ii] = (t < tend && i0 + ii < N) ? dh[t * N + i0 + ii] : 0.f;
+        }
+        for (int q = tid; q < kDwTok * kDwCol / 2; q += 256) {
+            const int tl = q / (kDwCol / 2), kk = 2 * (q % (kDwCol / 2));
+            const int64_t t = tb + tl;
+            uint32_t v = 0u;
+            if (t < tend && k0 + kk < d) v = *reinterpret_cast<const uint32_t *>(x + t * d + k0 + kk);
+            s_x[tl][kk] = __uint_as_float(v << 16);
+            s_x[tl][kk + 1] = __uint_as_float(v & 0xffff0000u);
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int tl = 0; tl < kDwTok; ++tl) {
+            const float4 xa = *reinterpret_cast<const float4 *>(&s_x[tl][8 * tk]);
+            const float4 xb = *reinterpret_cast<const float4 *>(&s_x[tl][8 * tk + 4]);
+            const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float a = s_dh[tl][ti + 16 * j];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[j][c] = fmaf(a, xv[c], acc[j][c]);
+                if (tk == 0) accb4[j] += a;
+            }
+        }
+    }
+    float *pw = part_w + (int64_t)chunk * N * d;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int i = i0 + ti + 16 * j;
+        const int k = k0 + 8 * tk;
+        if (i < N && k < d) {
+            float4 *dst = reinterpret_cast<float4 *>(pw + (int64_t)i * d + k);
+            dst[0] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+            dst[1] = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
+        }
+        if (tk == 0 && blockIdx.x == 0 && i < N) part_b[(int64_t)chunk * N + i] = accb4[j];
+    }
+}
+
+// Sum the chunk partials in chunk order: out[j] = sum_c part[c][j].
+__global__ void reduce_chunks_kernel(const float *__restrict__ part, int chunks, int64_t n, float *__restrict__ out) {
+    for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n; j += (int64_t)gridDim.x * blockDim.x) {
+        float acc = 0.f;
+        for (int c = 0; c < chunks; ++c) acc += part[(int64_t)c * n + j];
+        out[j] = acc;
+    }
+}
+
+int64_t round_up64(int64_t v) { return (v + 63) / 64 * 64; }
+
+cudaError_t launch_transpose(int32_t kernel_id, const void *in, void *out, int B, int R, int Cc, int Rp,
+                             const int32_t *counts, int cap, cudaStream_t stream) {
+    const dim3 grid((unsigned)((Cc + kTT - 1) / kTT), (unsigned)((Rp + kTT - 1) / kTT), (unsigned)B);
+    launch_begin(kernel_id, stream);
+    transpose_bf16_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(in), static_cast<uint16_t *>(out),
+                                                    R, Cc, Rp, counts, cap);
+    cudaError_t err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
+
+}  // namespace
+
+// Chunks of tokens for the dW_r partial sums (enough blocks to fill the GPU,
+// each chunk long enough that the partials stay small).
+int64_t router_dw_chunks(int64_t T) {
+    const int64_t c = (T + 2047) / 2048;
+    return c < 1 ? 1 : (c > 64 ? 64 : c);
+}
+
+cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const float *w_r, const void *w_in,
+                             const void *w_out, const int32_t *expert, const float *gate, const int32_t *slot,
+                             const int32_t *counts, const float *dy, float g_aux, float *dx, float *dw_r, float *dbias,
+                             float *dw_in, float *dw_out, const Workspace &ws, cudaStream_t stream) {
+    const int64_t T = dims.T;
+    const int N = dims.num_experts, C = dims.capacity, d = dims.d_model, F = dims.d_ff;
+    const int64_t Cp = round_up64(C);
+    DeviceStatus *st = static_cast<DeviceStatus *>(ws.status);
+    cudaError_t err = cudaMemsetAsync(ws.status, 0, sizeof(DeviceStatus), stream);
+    // weight gradients of experts without kept tokens are zero; the GEMMs write the others
+    if (err == cudaSuccess) err = cudaMemsetAsync(dw_in, 0, (size_t)N * F * d * sizeof(float), stream);
+    if (err == cudaSuccess) err = cudaMemsetAsync(dw_out, 0, (size_t)N * d * F * sizeof(float), stream);
+    if (err != cudaSuccess) return err;
+    if (T == 0) {
+        err = cudaMemsetAsync(dw_r, 0, (size_t)N * d * sizeof(float), stream);
+        if (err == cudaSuccess && dbias) err = cudaMemsetAsync(dbias, 0, (size_t)N * sizeof(float), stream);
+        return err;
+    }
+    // 1. gate gradients, dE and the softmax backward
+    launch_begin(K_BWD_TOKEN, stream);
+    bwd_token_kernel<<<(unsigned)((T + kWarps - 1) / kWarps), kThreads, 0, stream>>>(
+        dy, ws.ybuf, expert, slot, gate, ws.probs, counts, T, d, N, C, g_aux,
+        static_cast<__nv_bfloat16 *>(ws.grad_e), ws.dh);
+    err = cudaGetLastError();
+    launch_end(stream);
+    if (err != cudaSuccess) return err;
+    // 2. transposed weights: W_out^T [N][F][d], W_in^T [N][d][F]
+    if ((err = launch_transpose(K_BWD_TRANSPOSE, w_out, ws.w_out_t, N, d, F, d, nullptr, 0, stream)) != cudaSuccess)
+        return err;
+    if ((err = launch_transpose(K_BWD_TRANSPOSE, w_in, ws.w_in_t, N, F, d, F, nullptr, 0, stream)) != cudaSuccess)
+        return err;
+    // 3. dZ = (dE W_out) masked by the forward's ReLU: [N][C][F] bf16
+    err = launch_ffn_tc_bwd_dz(dims, ws.grad_e, ws.w_out_t, counts, ws.grad_z, ws.hidden, st, stream);
+    if (err != cudaSuccess) return err;
+    // 4. dx = dh W_r (all rows), then + dZ W_in for kept rows
+    {
+        const dim3 grid((unsigned)((d + kDxCol - 1) / kDxCol), (unsigned)((T + kDxTok - 1) / kDxTok));
+        launch_begin(K_BWD_ROUTER_DX, stream);
+        router_dx_kernel<<<grid, 256, 0, stream>>>(ws.dh, w_r, T, N, d, dx);
+        err = cudaGetLastError();
+        launch_end(stream);
+        if (err != cudaSuccess) return err;
+    }
+    err = launch_ffn_tc_bwd_dx(dims, ws.grad_z, ws.w_in_t, counts, ws.slot_token, dx, st, stream);
+    if (err != cudaSuccess) return err;
+    // 5. transposed activations (rows past each expert's kept tokens zeroed)
+    if ((err = launch_transpose(K_BWD_TRANSPOSE, ws.grad_e, ws.grad_e_t, N, C, d, (int)Cp, counts, C, stream)) !=
+        cudaSuccess)
+        return err;
+    if ((err = launch_transpose(K_BWD_TRANSPOSE, ws.hidden, ws.hidden_t, N, C, F, (int)Cp, counts, C, stream)) !=
+        cudaSuccess)
+        return err;
+    if ((err = launch_transpose(K_BWD_TRANSPOSE, ws.xbuf, ws.xbuf_t, N, C, d, (int)Cp, counts, C, stream)) !=
+        cudaSuccess)
+        return err;
+    if ((err = launch_transpose(K_BWD_TRANSPOSE, ws.grad_z, ws.grad_z_t, N, C, F, (int)Cp, counts, C, stream)) !=
+        cudaSuccess)
+        return err;
+    // 6. dW_out = dE^T H, dW_in = dZ^T x over each expert's kept tokens
+    err = launch_ffn_tc_bwd_dw(dims, ws.grad_e_t, ws.hidden_t, counts, d, F, (int)Cp, dw_out, st, stream);
+    if (err != cudaSuccess) return err;
+    err = launch_ffn_tc_bwd_dw(dims, ws.grad_z_t, ws.xbuf_t, counts, F, d, (int)Cp, dw_in, st, stream);
+    if (err != cudaSuccess) return err;
+    // 7. dW_r and d bias: chunk partials, then a fixed-order sum
+    {
+        const int64_t chunks = router_dw_chunks(T);
+        const int64_t chunk_tokens = (T + chunks - 1) / chunks;
+        const dim3 grid((unsigned)((d + kDwCol - 1) / kDwCol), (unsigned)((N + kDwI - 1) / kDwI), (unsigned)chunks);
+        launch_begin(K_BWD_ROUTER_DW, stream);
+        router_dw_kernel<<<grid, 256, 0, stream>>>(ws.dh, static_cast<const uint16_t *>(x), T, N, d, chunk_tokens,
+                                                   ws.dw_part, ws.db_part);
+        err = cudaGetLastError();
+        launch_end(stream);
+        if (err != cudaSuccess) return err;
+        launch_begin(K_BWD_REDUCE, stream);
+        reduce_chunks_kernel<<<256, 256, 0, stream>>>(ws.dw_part, (int)chunks, (int64_t)N * d, dw_r);
+        if (dbias) reduce_chunks_kernel<<<1, 256, 0, stream>>>(ws.db_part, (int)chunks, (int64_t)N, dbias);
+        err = cudaGetLastError();
+        launch_end(stream);
+    }
+    return err;
+}
+
+}  // namespace switchmoe

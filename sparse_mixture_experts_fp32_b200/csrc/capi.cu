@@ -26,7 +26,8 @@ int64_t tiles_of(const switch_dims_t &d) { return (d.T + kTileT - 1) / kTileT; }
 
 struct Sections {
     size_t status, ticket, hist, psum, tile_off, prob_total, w_split, slot_token, xbuf, ybuf, hidden, done, hist2,
-        tile_off2, counts_first, total;
+        tile_off2, counts_first, probs, dh, grad_e, grad_z, w_out_t, w_in_t, grad_e_t, hidden_t, xbuf_t, grad_z_t,
+        dw_part, db_part, total;
 };
 
 Sections layout(const switch_dims_t &d) {
@@ -54,6 +55,22 @@ Sections layout(const switch_dims_t &d) {
     s.hist2 = take(N * tiles * 4);
     s.tile_off2 = take(N * tiles * 4);
     s.counts_first = take(N * 4);
+    if (d.flags & SWITCH_FLAG_TRAINING) {  // kept by the training forward, used by the backward pass
+        const size_t T = (size_t)d.T, dm = (size_t)d.d_model, F = (size_t)d.d_ff, es = elem_size(d);
+        const size_t Cp = (C + 63) / 64 * 64, chunks = (size_t)router_dw_chunks(d.T);
+        s.probs = take(T * N * 4);
+        s.dh = take(T * N * 4);
+        s.grad_e = take(N * C * dm * es);
+        s.grad_z = take(N * C * F * es);
+        s.w_out_t = take(N * F * dm * es);
+        s.w_in_t = take(N * dm * F * es);
+        s.grad_e_t = take(N * dm * Cp * es);
+        s.hidden_t = take(N * F * Cp * es);
+        s.xbuf_t = take(N * dm * Cp * es);
+        s.grad_z_t = take(N * F * Cp * es);
+        s.dw_part = take(chunks * N * dm * 4);
+        s.db_part = take(chunks * N * 4);
+    }
     s.total = off;
     return s;
 }
@@ -173,6 +190,20 @@ Workspace carve_workspace(const switch_dims_t &dims, void *base) {
     w.hist2 = reinterpret_cast<int32_t *>(b + s.hist2);
     w.tile_off2 = reinterpret_cast<int32_t *>(b + s.tile_off2);
     w.counts_first = reinterpret_cast<int32_t *>(b + s.counts_first);
+    const bool training = (dims.flags & SWITCH_FLAG_TRAINING) != 0;
+    auto at = [&](size_t o) -> void * { return training ? (void *)(b + o) : nullptr; };
+    w.probs = static_cast<float *>(at(s.probs));
+    w.dh = static_cast<float *>(at(s.dh));
+    w.grad_e = at(s.grad_e);
+    w.grad_z = at(s.grad_z);
+    w.w_out_t = at(s.w_out_t);
+    w.w_in_t = at(s.w_in_t);
+    w.grad_e_t = at(s.grad_e_t);
+    w.hidden_t = at(s.hidden_t);
+    w.xbuf_t = at(s.xbuf_t);
+    w.grad_z_t = at(s.grad_z_t);
+    w.dw_part = static_cast<float *>(at(s.dw_part));
+    w.db_part = static_cast<float *>(at(s.db_part));
     w.tiles = tiles_of(dims);
     return w;
 }
@@ -301,7 +332,16 @@ switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const
     const bool tensor_cores = dims->dtype == SWITCH_BF16 && !(dims->flags & SWITCH_FLAG_SIMT_FFN);
     const bool rows16 = ((int64_t)dims->d_model * (int64_t)elem_size(*dims)) % 16 == 0;
     cudaError_t err;
-    if (tensor_cores) {
+    if (dims->flags & SWITCH_FLAG_TRAINING) {
+        // training forward: keeps the router probabilities, xbuf, H and the ungated
+        // expert output ybuf in the workspace for switch_layer_bwd
+        if (!tensor_cores) return SWITCH_ERR_UNSUPPORTED;
+        err = launch_route(*dims, x, w_r, logit_bias, expert, gate, slot, counts, ws.slot_token, aux, ws, st,
+                           ws.xbuf, nullptr);
+        if (err == cudaSuccess)
+            err = launch_ffn_tc(*dims, ws.xbuf, w_in, w_out, counts, ws.ybuf, nullptr, nullptr, nullptr, ws, st);
+        if (err == cudaSuccess) err = launch_combine(*dims, ws.ybuf, expert, slot, gate, yf, st);
+    } else if (tensor_cores) {
         // route + scatter-dispatch (zeroing dropped rows of y), GEMM1, GEMM2 with
         // the gate and the token-order scatter fused into its epilogue
         err = launch_route(*dims, x, w_r, logit_bias, expert, gate, slot, counts, ws.slot_token, aux, ws, st,
@@ -384,6 +424,31 @@ switch_status_t switch_layer_fwd_top2(const switch_dims_t *dims, const void *x, 
                            : launch_ffn_simt(rows, ws.xbuf, w_in, w_out, counts, ws.ybuf, ws, st);
     if (err == cudaSuccess) err = launch_combine_top2(*dims, ws.ybuf, expert, slot, gate, static_cast<float *>(y), st);
     return from_cuda(err);
+}
+
+switch_status_t switch_layer_bwd(const switch_dims_t *dims, const void *x, const float *w_r, const void *w_in,
+                                 const void *w_out, const int32_t *expert, const float *gate, const int32_t *slot,
+                                 const int32_t *counts, const float *dy, float g_aux, float *dx, float *dw_r,
+                                 float *dbias, float *dw_in, float *dw_out, void *workspace,
+                                 size_t workspace_bytes_given, switch_stream_t stream) {
+    switch_status_t s = check_dims(dims);
+    if (s != SWITCH_OK) return s;
+    if (!(dims->flags & SWITCH_FLAG_TRAINING)) return SWITCH_ERR_UNSUPPORTED;
+    if (dims->dtype != SWITCH_BF16 || (dims->flags & (SWITCH_FLAG_SIMT_FFN | SWITCH_FLAG_GEMM_1CTA)))
+        return SWITCH_ERR_UNSUPPORTED;
+    const bool has_tokens = dims->T > 0;
+    s = check_ptrs({w_r, w_in, w_out, counts, dw_r, dw_in, dw_out, workspace, has_tokens ? x : w_r,
+                    has_tokens ? (const void *)expert : w_r, has_tokens ? (const void *)gate : w_r,
+                    has_tokens ? (const void *)slot : w_r, has_tokens ? (const void *)dy : w_r,
+                    has_tokens ? (const void *)dx : w_r},
+                   {x, expert, gate, slot, dy, dx, dbias});
+    if (s != SWITCH_OK) return s;
+    if (!std::isfinite(g_aux)) return SWITCH_ERR_SHAPE;
+    if (workspace_bytes_given < workspace_bytes(*dims)) return SWITCH_ERR_WORKSPACE;
+    if ((s = check_device()) != SWITCH_OK) return s;
+    const Workspace ws = carve_workspace(*dims, workspace);
+    return from_cuda(launch_layer_bwd(*dims, x, w_r, w_in, w_out, expert, gate, slot, counts, dy, g_aux, dx, dw_r,
+                                      dbias, dw_in, dw_out, ws, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 switch_status_t switch_check(void *workspace, size_t workspace_bytes_given, switch_stream_t stream) {
@@ -491,6 +556,14 @@ const char *switch_kernel_name(int32_t id) {
         case K_SELFTEST_WAIT: return "selftest_wait_timeout";
         case K_FFN_TC_FUSED: return "ffn_tc_fused";
         case K_COMBINE_TOP2: return "combine_top2";
+        case K_BWD_TOKEN: return "bwd_gate_softmax";
+        case K_BWD_TRANSPOSE: return "bwd_transpose";
+        case K_BWD_GEMM_DZ: return "bwd_tc_gemm_dz";
+        case K_BWD_GEMM_DX: return "bwd_tc_gemm_dx";
+        case K_BWD_GEMM_DW: return "bwd_tc_gemm_dw";
+        case K_BWD_ROUTER_DX: return "bwd_router_dx";
+        case K_BWD_ROUTER_DW: return "bwd_router_dw";
+        case K_BWD_REDUCE: return "bwd_reduce";
     }
     return "?";
 }

@@ -67,7 +67,13 @@ __device__ __forceinline__ void locate_tile(const int32_t *tile_start, int E, in
     n = local % n_tiles_n;
 }
 
-enum Epilogue { kEpiHiddenRelu = 0, kEpiExpertOut = 1, kEpiGatedScatter = 2 };
+enum Epilogue {
+    kEpiHiddenRelu = 0,    // H = bf16(ReLU(acc))
+    kEpiExpertOut = 1,     // fp32 rows out[e * out_rows + row]
+    kEpiGatedScatter = 2,  // y[slot_token] = gate * acc (with `add`: += )
+    kEpiReluGrad = 3,      // backward: dZ = bf16(acc) where the forward's H > 0, else 0
+    kEpiScatterAdd = 4     // backward: dx[slot_token] += acc
+};
 
 // Epilogue for one thread = one accumulator row (`row` of expert e's rows),
 // BN columns starting at column tile n: tcgen05.ld 32 columns at a time, then
@@ -306,11 +312,12 @@ template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_base, int kept, int C, int n, int Nout,
                                                void *__restrict__ out, const void *tmap_out,
                                                const int32_t *__restrict__ slot_token,
-                                               const float *__restrict__ gate, uint8_t *stage, bool add = false) {
+                                               const float *__restrict__ gate, uint8_t *stage, bool add = false,
+                                               int out_rows = 0, const uint16_t *__restrict__ mask_h = nullptr) {
     const int lane = threadIdx.x & 31;
     const int row = row_base + lane;
     const bool row_ok = row < kept;
-    if (EPI == kEpiHiddenRelu) {
+    if (EPI == kEpiHiddenRelu || EPI == kEpiReluGrad) {
         const bool any_row = row_base < kept;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 64) {
@@ -321,12 +328,31 @@ __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_ba
             if (lane == 0) bulk_wait_read_all();  // the previous box has left the buffer
             __syncwarp();
             uint8_t *rowp = stage + lane * 128;
+            uint4 hm[8];  // kEpiReluGrad: the forward's H at these 64 columns (its sign is the ReLU mask)
+            if (EPI == kEpiReluGrad) {
+                const int col = n * BN + c;
+                const bool ld = row_ok && col < Nout;
+                const uint4 *hp = reinterpret_cast<const uint4 *>(mask_h + ((int64_t)e * C + row) * Nout + col);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) hm[q] = ld ? __ldg(hp + q) : make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const uint32_t *src = q < 4 ? &r0[8 * q] : &r1[8 * (q - 4)];
                 float v[8];
+                if (EPI == kEpiReluGrad) {
+                    const uint32_t w[4] = {hm[q].x, hm[q].y, hm[q].z, hm[q].w};
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = fmaxf(__uint_as_float(src[i]), 0.f);
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t hb = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xffffu);
+                        // H = bf16(ReLU(z)) > 0 exactly where z > 0 (but for z below the smallest bf16 subnormal)
+                        const bool pos = hb != 0u && (hb & 0x8000u) == 0u;
+                        v[i] = pos ? __uint_as_float(src[i]) : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i] = fmaxf(__uint_as_float(src[i]), 0.f);
+                }
                 *reinterpret_cast<uint4 *>(rowp + ((q ^ (lane & 7)) << 4)) =
                     make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                                pack_bf16x2(v[6], v[7]));
@@ -343,13 +369,14 @@ __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_ba
         float g = 1.f;
         float *dst_row = nullptr;
         if (row_ok) {
-            int64_t out_row = (int64_t)e * C + row;
-            if (EPI == kEpiGatedScatter) {
+            int64_t out_row = (int64_t)e * (out_rows > 0 ? out_rows : C) + row;
+            if (EPI == kEpiGatedScatter || EPI == kEpiScatterAdd) {
                 out_row = slot_token[(int64_t)e * C + row];
-                g = gate[out_row];
+                if (EPI == kEpiGatedScatter) g = gate[out_row];
             }
             dst_row = static_cast<float *>(out) + out_row * Nout;
         }
+        if (EPI == kEpiScatterAdd) add = true;
         uint8_t *rowp = stage + lane * 144;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -399,13 +426,29 @@ struct PairLayout {
     static size_t bytes(int experts) { return 1024 + ring + staging + barriers + (size_t)(experts + 1) * 4; }
 };
 
+// Per-expert shape of a grouped GEMM.  Forward: the rows of expert e are its
+// kept tokens (min(counts[e], C)) and K is fixed.  Weight gradients of the
+// backward pass: every expert with kept tokens has `rows_fixed` output rows
+// (d_model or d_ff), no rows otherwise, and K runs over its kept tokens only
+// (k_per_expert: ceil(kept / 64) K blocks; the operands are zero past them).
+struct GroupShape {
+    int rows_fixed;    // 0: rows = kept tokens
+    int k_per_expert;  // 0: K / BK blocks for every tile
+    int out_rows;      // kEpiExpertOut: rows of each expert's block of `out` (0: C)
+    const uint16_t *mask_h;  // kEpiReluGrad: the forward's H [E][C][Nout]
+};
+
+__device__ __forceinline__ int group_rows(const GroupShape &g, int kept) {
+    return g.rows_fixed > 0 ? (kept > 0 ? g.rows_fixed : 0) : kept;
+}
+
 template <int BN, int STAGES, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                          const __grid_constant__ CUtensorMap tmap_out, void *__restrict__ out,
                          const int32_t *__restrict__ counts, int E, int C, int K, int Nout,
                          const int32_t *__restrict__ slot_token, const float *__restrict__ gate,
-                         DeviceStatus *status) {
+                         DeviceStatus *status, const GroupShape shape) {
     using L = PairLayout<BN, STAGES>;
     constexpr int BMP = 2 * BM;  // rows of a pair tile
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -456,7 +499,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = 32 * j + lane;
-            kept_of[j] = e < E ? min(counts[e], C) : 0;
+            kept_of[j] = e < E ? group_rows(shape, min(counts[e], C)) : 0;
         }
         int running = 0;
 #pragma unroll
@@ -492,7 +535,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
                 int e, m, n;
                 locate_tile(tile_start, E, n_tiles_n, tile, e, m, n);
-                for (int kb = 0; kb < k_blocks; ++kb) {
+                const int kbs = shape.k_per_expert ? (min(counts[e], C) + BK - 1) / BK : k_blocks;
+                for (int kb = 0; kb < kbs; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, status, 21)) {
                         ok = false;
                         break;
@@ -525,10 +569,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+                int kbs = k_blocks;
+                if (shape.k_per_expert) {
+                    int e, m, n;
+                    locate_tile(tile_start, E, n_tiles_n, tile, e, m, n);
+                    kbs = (min(counts[e], C) + BK - 1) / BK;
+                }
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, status, 22)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < k_blocks; ++kb) {
+                for (int kb = 0; kb < kbs; ++kb) {
                     if (!mbar_wait(&full[stage], phase, status, 23)) {
                         ok = false;
                         break;
@@ -567,8 +617,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int row_base = m * BMP + (int)rank * BM + quarter * 32;
             epilogue_async<BN, EPI>(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN), e,
-                                    row_base, min(counts[e], C), C, n, Nout, out, &tmap_out, slot_token, gate,
-                                    staging + (warp - 2) * L::stage_bytes);
+                                    row_base, group_rows(shape, min(counts[e], C)), C, n, Nout, out, &tmap_out,
+                                    slot_token, gate, staging + (warp - 2) * L::stage_bytes, false, shape.out_rows,
+                                    shape.mask_h);
             tc_fence_before();
             mbar_arrive_cluster(map_to_rank(&acc_empty[acc], 0));
             if (++acc == 2) {
@@ -991,24 +1042,32 @@ cudaError_t launch_gemm(int32_t kernel_id, const void *a, const void *b, void *o
     return err;
 }
 
+// A [E][a_rows][K] and B [E][Nout][K] (bf16, K contiguous); a_rows = C unless
+// the shape has fixed rows (then A holds rows_fixed rows per expert and K is
+// the padded token count).
 template <int BN, int STAGES, int EPI>
 cudaError_t launch_gemm_pair(int32_t kernel_id, const void *a, const void *b, void *out, const int32_t *counts, int E,
                              int C, int K, int Nout, int64_t T, const int32_t *slot_token, const float *gate,
-                             DeviceStatus *status, cudaStream_t stream) {
+                             DeviceStatus *status, cudaStream_t stream, GroupShape shape = GroupShape{0, 0, 0, nullptr}) {
+    const int a_rows = shape.rows_fixed > 0 ? shape.rows_fixed : C;
     CUtensorMap ta, tb, tout;
-    if (!make_tmap(&ta, a, E, C, K, BM) || !make_tmap(&tb, b, E, Nout, K, BN / 2)) return cudaErrorInvalidValue;
+    if (!make_tmap(&ta, a, E, a_rows, K, BM) || !make_tmap(&tb, b, E, Nout, K, BN / 2)) return cudaErrorInvalidValue;
     memset(&tout, 0, sizeof tout);
-    if (EPI == kEpiHiddenRelu && !make_tmap(&tout, out, E, C, Nout, 32)) return cudaErrorInvalidValue;
+    if ((EPI == kEpiHiddenRelu || EPI == kEpiReluGrad) && !make_tmap(&tout, out, E, C, Nout, 32))
+        return cudaErrorInvalidValue;
     const size_t smem = PairLayout<BN, STAGES>::bytes(E);
     auto kern = tc_grouped_gemm_pair<BN, STAGES, EPI>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    const int64_t m_tiles = std::min<int64_t>((int64_t)E * ((C + 2 * BM - 1) / (2 * BM)), (T + 2 * BM - 1) / (2 * BM) + E);
+    const int64_t m_tiles =
+        shape.rows_fixed > 0
+            ? (int64_t)E * ((shape.rows_fixed + 2 * BM - 1) / (2 * BM))
+            : std::min<int64_t>((int64_t)E * ((C + 2 * BM - 1) / (2 * BM)), (T + 2 * BM - 1) / (2 * BM) + E);
     const int64_t tiles = m_tiles * ((Nout + BN - 1) / BN);
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / 2, tiles));
     launch_begin(kernel_id, stream);
     err = launch_kernel(kern, dim3(2 * pairs), dim3(kThreads), smem, stream, true, ta, tb, tout, out, counts, E, C, K,
-                        Nout, slot_token, gate, status);
+                        Nout, slot_token, gate, status, shape);
     launch_end(stream);
     return err;
 }
@@ -1047,6 +1106,36 @@ cudaError_t launch_ffn_fused(const switch_dims_t &dims, const void *xbuf, const 
 }
 
 }  // namespace
+
+// Backward GEMMs (SM pairs, 256 x 256 tiles, the forward's kernel).
+// dZ [N][C][F] = bf16((dE W_out) where H > 0): A = dE [N][C][d], B = W_out^T [N][F][d].
+cudaError_t launch_ffn_tc_bwd_dz(const switch_dims_t &dims, const void *grad_e, const void *w_out_t,
+                                 const int32_t *counts, void *grad_z, const void *hidden, DeviceStatus *st,
+                                 cudaStream_t stream) {
+    return launch_gemm_pair<256, 6, kEpiReluGrad>(K_BWD_GEMM_DZ, grad_e, w_out_t, grad_z, counts, dims.num_experts,
+                                                  dims.capacity, dims.d_model, dims.d_ff, dims.T, nullptr, nullptr,
+                                                  st, stream,
+                                                  GroupShape{0, 0, 0, static_cast<const uint16_t *>(hidden)});
+}
+
+// dx[slot_token] += dZ W_in: A = dZ [N][C][F], B = W_in^T [N][d][F].
+cudaError_t launch_ffn_tc_bwd_dx(const switch_dims_t &dims, const void *grad_z, const void *w_in_t,
+                                 const int32_t *counts, const int32_t *slot_token, float *dx, DeviceStatus *st,
+                                 cudaStream_t stream) {
+    return launch_gemm_pair<256, 6, kEpiScatterAdd>(K_BWD_GEMM_DX, grad_z, w_in_t, dx, counts, dims.num_experts,
+                                                    dims.capacity, dims.d_ff, dims.d_model, dims.T, slot_token,
+                                                    nullptr, st, stream);
+}
+
+// Weight gradient out [N][rows][nout] (fp32) = A^T-free form A . B^T over each
+// expert's kept tokens: A [N][rows][Kp], B [N][nout][Kp] (token-contiguous,
+// zero past the kept tokens).
+cudaError_t launch_ffn_tc_bwd_dw(const switch_dims_t &dims, const void *a_t, const void *b_t, const int32_t *counts,
+                                 int rows, int nout, int Kp, float *out, DeviceStatus *st, cudaStream_t stream) {
+    return launch_gemm_pair<256, 6, kEpiExpertOut>(K_BWD_GEMM_DW, a_t, b_t, out, counts, dims.num_experts,
+                                                   dims.capacity, Kp, nout, dims.T, nullptr, nullptr, st, stream,
+                                                   GroupShape{rows, 1, rows, nullptr});
+}
 
 cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
                           const int32_t *counts, void *ybuf, const int32_t *slot_token, const float *gate, float *y,

@@ -33,6 +33,14 @@ enum KernelId : int32_t {
     K_SELFTEST_WAIT = 16,
     K_FFN_TC_FUSED = 17,
     K_COMBINE_TOP2 = 18,
+    K_BWD_TOKEN = 19,
+    K_BWD_TRANSPOSE = 20,
+    K_BWD_GEMM_DZ = 21,
+    K_BWD_GEMM_DX = 22,
+    K_BWD_GEMM_DW = 23,
+    K_BWD_ROUTER_DX = 24,
+    K_BWD_ROUTER_DW = 25,
+    K_BWD_REDUCE = 26,
 };
 
 struct Workspace {
@@ -52,6 +60,19 @@ struct Workspace {
     int32_t *hist2;      // top-2: [N][tiles] second choices of each expert in each tile
     int32_t *tile_off2;  // top-2: [N][tiles] first slot of each tile's second choices
     int32_t *counts_first;  // top-2: [N] first choices per expert (the aux loss's f)
+    float *probs;        // training: [T][N] router probabilities kept for the backward pass (else null)
+    // training only (SWITCH_FLAG_TRAINING): backward-pass buffers
+    float *dh;           // [T][N] gradient of the router logits
+    void *grad_e;        // [N][C][d] bf16 gate * dy in expert order
+    void *grad_z;        // [N][C][F] bf16 gradient of the pre-activations
+    void *w_out_t;       // [N][F][d] bf16 W_out transposed
+    void *w_in_t;        // [N][d][F] bf16 W_in transposed
+    void *grad_e_t;      // [N][d][Cp] bf16 (Cp = C rounded up to 64; zero past the kept tokens)
+    void *hidden_t;      // [N][F][Cp] bf16
+    void *xbuf_t;        // [N][d][Cp] bf16
+    void *grad_z_t;      // [N][F][Cp] bf16
+    float *dw_part;      // [chunks][N][d] partial sums of dW_r
+    float *db_part;      // [chunks][N] partial sums of d bias
     int64_t tiles;
 };
 
@@ -103,6 +124,21 @@ cudaError_t launch_ffn_simt(const switch_dims_t &dims, const void *xbuf, const v
 cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
                           const int32_t *counts, void *ybuf, const int32_t *slot_token, const float *gate, float *y,
                           const Workspace &ws, cudaStream_t stream);
+
+// Backward pass (bfloat16 experts; the workspace of a SWITCH_FLAG_TRAINING forward).
+int64_t router_dw_chunks(int64_t T);
+cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const float *w_r, const void *w_in,
+                             const void *w_out, const int32_t *expert, const float *gate, const int32_t *slot,
+                             const int32_t *counts, const float *dy, float g_aux, float *dx, float *dw_r, float *dbias,
+                             float *dw_in, float *dw_out, const Workspace &ws, cudaStream_t stream);
+cudaError_t launch_ffn_tc_bwd_dz(const switch_dims_t &dims, const void *grad_e, const void *w_out_t,
+                                 const int32_t *counts, void *grad_z, const void *hidden, DeviceStatus *st,
+                                 cudaStream_t stream);
+cudaError_t launch_ffn_tc_bwd_dx(const switch_dims_t &dims, const void *grad_z, const void *w_in_t,
+                                 const int32_t *counts, const int32_t *slot_token, float *dx, DeviceStatus *st,
+                                 cudaStream_t stream);
+cudaError_t launch_ffn_tc_bwd_dw(const switch_dims_t &dims, const void *a_t, const void *b_t, const int32_t *counts,
+                                 int rows, int nout, int Kp, float *out, DeviceStatus *st, cudaStream_t stream);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();

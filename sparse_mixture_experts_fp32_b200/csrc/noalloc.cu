@@ -81,8 +81,13 @@ extern "C" switch_status_t switch_route_noalloc(const switch_dims_t *dims, const
     // first block clears the ticket and the status word, and every other
     // section is fully rewritten by the call, so the previous call's
     // contents never leak into this one.
-    const Workspace ws = carve_workspace(*dims, scratch);
-    const cudaError_t err = launch_route(*dims, x, w_r, logit_bias, expert, gate, slot, counts, slot_token, aux, ws,
-                                         reinterpret_cast<cudaStream_t>(stream));
+    // The training flag would make the routers also write the [T][N]
+    // probabilities into a section past the routing scratch; routing here
+    // never keeps them, so the flag is cleared for the carve and the launch.
+    switch_dims_t route_dims = *dims;
+    route_dims.flags &= ~SWITCH_FLAG_TRAINING;
+    const Workspace ws = carve_workspace(route_dims, scratch);
+    const cudaError_t err = launch_route(route_dims, x, w_r, logit_bias, expert, gate, slot, counts, slot_token, aux,
+                                         ws, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? SWITCH_OK : SWITCH_ERR_CUDA;
 }

@@ -42,7 +42,8 @@ __device__ __forceinline__ bool better(float v, int i, float m, int a) { return 
 template <int J, bool TOP2>
 __device__ __forceinline__ void token_epilogue(const float (&v)[J], const int (&idx)[J], const bool (&own)[J],
                                                int64_t t, float *warp_psum, int32_t *warp_hist,
-                                               int32_t *warp_hist2, int32_t *expert, float *gate) {
+                                               int32_t *warp_hist2, int32_t *expert, float *gate, float *probs,
+                                               int N) {
     const int lane = threadIdx.x & 31;
     float m = -FLT_MAX;
     int arg = 0x7fffffff;
@@ -95,7 +96,10 @@ __device__ __forceinline__ void token_epilogue(const float (&v)[J], const int (&
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
 #pragma unroll
     for (int j = 0; j < J; ++j)
-        if (idx[j] >= 0 && own[j]) warp_psum[idx[j]] += ex[j] / s;
+        if (idx[j] >= 0 && own[j]) {
+            warp_psum[idx[j]] += ex[j] / s;
+            if (probs) probs[t * N + idx[j]] = ex[j] / s;  // kept for the backward pass
+        }
     if (lane == 0) {
         warp_hist[arg] += 1;
         if (TOP2) {
@@ -199,8 +203,8 @@ __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restr
                                                                int N, int tiles, int32_t *__restrict__ expert,
                                                                float *__restrict__ gate, int32_t *__restrict__ hist,
                                                                int32_t *__restrict__ hist2,
-                                                               float *__restrict__ psum, uint32_t *ticket,
-                                                               DeviceStatus *status) {
+                                                               float *__restrict__ psum, float *__restrict__ probs,
+                                                               uint32_t *ticket, DeviceStatus *status) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *wsm = reinterpret_cast<float *>(smem_raw);  // [d][NP]
     float *psum_w = wsm + (size_t)d * NP;               // [kWarps][N]
@@ -286,7 +290,7 @@ __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restr
         int idx[1] = {valid_e ? my_e : -1};
         bool own[1] = {(lane & ((1 << SHIFT) - 1)) == 0};
         token_epilogue<1, TOP2>(v, idx, own, t, psum_w + warp * N, hist_w + warp * N, hist2_w + warp * N, expert,
-                                gate);
+                                gate, probs, N);
     }
     __syncthreads();
     publish_tile(psum_w, hist_w, hist2_w, N, tiles, tile, hist, TOP2 ? hist2 : nullptr, psum);
@@ -329,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     router_staged_kernel(const XT *__restrict__ x, const float *__restrict__ w_r, const float *__restrict__ bias,
                          int64_t T, int d, int N, int tiles, int32_t *__restrict__ expert, float *__restrict__ gate,
                          int32_t *__restrict__ hist, int32_t *__restrict__ hist2, float *__restrict__ psum,
-                         uint32_t *ticket, DeviceStatus *status, int raw_w) {
+                         float *__restrict__ probs, uint32_t *ticket, DeviceStatus *status, int raw_w) {
     using S = Staged<XT>;
     constexpr int V = S::V;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -491,6 +495,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int e = 0; e < NP; ++e) ptile[tl * NP + e] = valid ? h[e] / s : 0.f;  // p_e
+        if (probs && valid) {  // kept for the backward pass
+#pragma unroll
+            for (int e = 0; e < NP; ++e)
+                if (e < N) probs[(t0 + tl) * N + e] = h[e] / s;
+        }
         if (valid) {
             const int64_t t = t0 + tl;
             if (TOP2) {
@@ -534,8 +543,8 @@ __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__rest
                                                                 int N, int tiles, int32_t *__restrict__ expert,
                                                                 float *__restrict__ gate, int32_t *__restrict__ hist,
                                                                 int32_t *__restrict__ hist2,
-                                                                float *__restrict__ psum, uint32_t *ticket,
-                                                                DeviceStatus *status) {
+                                                                float *__restrict__ psum, float *__restrict__ probs,
+                                                                uint32_t *ticket, DeviceStatus *status) {
     constexpr int TE = EC / 16;  // experts per thread
     constexpr int TT = 4;        // tokens per thread
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -616,7 +625,7 @@ __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__rest
             v[j] = e < N ? logits[r * NL + e] + (bias ? bias[e] : 0.f) : 0.f;
         }
         token_epilogue<J, TOP2>(v, idx, own, t, psum_w + warp * N, hist_w + warp * N, hist2_w + warp * N, expert,
-                                gate);
+                                gate, probs, N);
     }
     __syncthreads();
     publish_tile(psum_w, hist_w, hist2_w, N, tiles, tile, hist, TOP2 ? hist2 : nullptr, psum);
@@ -993,7 +1002,7 @@ cudaError_t launch_router_warp(const switch_dims_t &dims, const XT *x, const flo
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_WARP, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
-                                                         ws.hist, ws.hist2, ws.psum, ws.ticket,
+                                                         ws.hist, ws.hist2, ws.psum, ws.probs, ws.ticket,
                                                          static_cast<DeviceStatus *>(ws.status));
     err = cudaGetLastError();
     launch_end(stream);
@@ -1014,7 +1023,7 @@ cudaError_t launch_router_staged(const switch_dims_t &dims, const XT *x, const f
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_STAGED, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
-                                                         ws.hist, ws.hist2, ws.psum, ws.ticket,
+                                                         ws.hist, ws.hist2, ws.psum, ws.probs, ws.ticket,
                                                          static_cast<DeviceStatus *>(ws.status), raw ? 1 : 0);
     err = cudaGetLastError();
     launch_end(stream);
@@ -1032,7 +1041,7 @@ cudaError_t launch_router_tiled(const switch_dims_t &dims, const XT *x, const fl
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_TILED, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
-                                                         ws.hist, ws.hist2, ws.psum, ws.ticket,
+                                                         ws.hist, ws.hist2, ws.psum, ws.probs, ws.ticket,
                                                          static_cast<DeviceStatus *>(ws.status));
     err = cudaGetLastError();
     launch_end(stream);

@@ -149,7 +149,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
     router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const float *__restrict__ bias, int64_t T, int d, int N, int tiles64,
                      int32_t *__restrict__ expert, float *__restrict__ gate, int32_t *__restrict__ hist,
-                     int32_t *__restrict__ hist2, float *__restrict__ psum, uint32_t *ticket, DeviceStatus *status) {
+                     int32_t *__restrict__ hist2, float *__restrict__ psum, float *__restrict__ probs,
+                     uint32_t *ticket, DeviceStatus *status) {
     using L = RouterLayout<BN, STAGES, TOP2>;
     constexpr int PM = 2 * RM;  // tokens per pair tile
     constexpr int G = RouterThreads<BN>::kGroups;
@@ -424,6 +425,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
                 float p[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) p[j] = valid ? h[j] * inv_s : 0.f;
+                if (probs && valid) {  // kept for the backward pass
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (col0 + j < N) probs[t * N + col0 + j] = p[j];
+                }
                 const float col_sum = reduce_scatter32(p);  // this warp's 32 tokens, column col0 + lane
                 psum_p[q * BN + col0 + lane] = col_sum;
             }
@@ -524,7 +530,7 @@ cudaError_t launch_bn(const switch_dims_t &dims, const __nv_bfloat16 *x, const f
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / 2, m_tiles));
     launch_begin(K_ROUTER_TC, stream);
     err = launch_kernel(kern, dim3(2 * pairs), dim3(RouterThreads<BN>::kAll), smem, stream, true, tx, tw, bias, T, d,
-                        N, (int)ws.tiles, expert, gate, ws.hist, ws.hist2, ws.psum, ws.ticket,
+                        N, (int)ws.tiles, expert, gate, ws.hist, ws.hist2, ws.psum, ws.probs, ws.ticket,
                         static_cast<DeviceStatus *>(ws.status));
     launch_end(stream);
     return err;
