@@ -313,14 +313,16 @@ __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_ba
                                                void *__restrict__ out, const void *tmap_out,
                                                const int32_t *__restrict__ slot_token,
                                                const float *__restrict__ gate, uint8_t *stage, bool add = false,
-                                               int out_rows = 0, const uint16_t *__restrict__ mask_h = nullptr) {
+                                               int out_rows = 0, const uint16_t *__restrict__ mask_h = nullptr,
+                                               int cols = BN) {
+    // `cols` (a multiple of 64, at most BN): the tile's width; column tile n starts at n * cols
     const int lane = threadIdx.x & 31;
     const int row = row_base + lane;
     const bool row_ok = row < kept;
     if (EPI == kEpiHiddenRelu || EPI == kEpiReluGrad) {
         const bool any_row = row_base < kept;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 64) {
+        for (int c = 0; c < cols; c += 64) {
             uint32_t r0[32], r1[32];
             tmem_ld_32x32b_x32(t_row + (uint32_t)c, r0);
             tmem_ld_32x32b_x32(t_row + (uint32_t)(c + 32), r1);
@@ -330,7 +332,7 @@ __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_ba
             uint8_t *rowp = stage + lane * 128;
             uint4 hm[8];  // kEpiReluGrad: the forward's H at these 64 columns (its sign is the ReLU mask)
             if (EPI == kEpiReluGrad) {
-                const int col = n * BN + c;
+                const int col = n * cols + c;
                 const bool ld = row_ok && col < Nout;
                 const uint4 *hp = reinterpret_cast<const uint4 *>(mask_h + ((int64_t)e * C + row) * Nout + col);
 #pragma unroll
@@ -359,8 +361,8 @@ __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_ba
             }
             fence_proxy_async_shared();
             __syncwarp();
-            if (lane == 0 && any_row && n * BN + c < Nout) {
-                tma_store_3d(tmap_out, stage, n * BN + c, row_base, e);
+            if (lane == 0 && any_row && n * cols + c < Nout) {
+                tma_store_3d(tmap_out, stage, n * cols + c, row_base, e);
                 bulk_commit();
             }
         }
@@ -379,11 +381,11 @@ __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_ba
         if (EPI == kEpiScatterAdd) add = true;
         uint8_t *rowp = stage + lane * 144;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = 0; c < cols; c += 32) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
             tmem_ld_wait();
-            const int col0 = n * BN + c;
+            const int col0 = n * cols + c;
             if (row_ok && col0 < Nout) {
                 bulk_wait_read_all();  // this thread's previous row copy has left the buffer
 #pragma unroll
@@ -702,6 +704,7 @@ template <int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_ffn_fused_pair(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w1,
                       const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w2,
+                      const __grid_constant__ CUtensorMap tm_w1h, const __grid_constant__ CUtensorMap tm_w2h,
                       const __grid_constant__ CUtensorMap tm_hstore, float *__restrict__ y,
                       const int32_t *__restrict__ counts, int E, int C, int d, int F,
                       const int32_t *__restrict__ slot_token, const float *__restrict__ gate,
@@ -730,9 +733,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
-    const int n1 = (F + BN - 1) / BN, n2 = (d + BN - 1) / BN;
     const int kb1 = d / BK;  // K blocks of a GEMM1 tile
-    const int32_t need = 8 * n1;  // arrivals on done[e, m] once H of the row block is complete
     constexpr uint32_t kTmemCols = 2 * BN;
 
     if (warp == 1) {
@@ -764,11 +765,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pdl_launch_dependents();
     if (warp == 0) {
         int kept_of[8];
+        int mt_all = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = 32 * j + lane;
             kept_of[j] = e < E ? min(counts[e], C) : 0;
+            mt_all += (kept_of[j] + BMP - 1) / BMP;
         }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mt_all += __shfl_xor_sync(0xffffffffu, mt_all, off);
+        // Tile width: 256 columns, or 128 when 256-wide GEMM1 tiles cannot give
+        // every pair one (few kept rows, e.g. a skewed routing): twice the tiles,
+        // each half as long.  Every CTA derives the same width from the same counts.
+        const int bw = mt_all * ((F + BN - 1) / BN) < (int)(gridDim.x >> 1) ? BN / 2 : BN;
+        const int n1 = (F + bw - 1) / bw, n2 = (d + bw - 1) / bw;
+        if (lane == 0) tmem_holder[1] = (uint32_t)bw;
         int run1 = 0, run2 = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -801,6 +812,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     const uint32_t tmem_base = *tmem_holder;
+    const int bw = (int)tmem_holder[1];          // tile width (columns) of both GEMMs
+    const int n1 = (F + bw - 1) / bw, n2 = (d + bw - 1) / bw;
+    const int32_t need = 8 * n1;  // arrivals on done[e, m] once H of the row block is complete
+    const uint32_t b_bytes = (uint32_t)(bw / 2) * BK * 2;  // this CTA's rows of a B stage
     const int total1 = start1[E];
     const int total2 = start2[E];  // GEMM2 output tiles
     const int split = fused_split(total2, F / BK, (int)(gridDim.x >> 1));
@@ -810,9 +825,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             prefetch_tmap(&tm_x);
-            prefetch_tmap(&tm_w1);
+            prefetch_tmap(bw == BN ? &tm_w1 : &tm_w1h);
             prefetch_tmap(&tm_h);
-            prefetch_tmap(&tm_w2);
+            prefetch_tmap(bw == BN ? &tm_w2 : &tm_w2h);
             uint32_t issued = 0, parity_of = 0;
             int stage = 0;
             uint32_t phase = 0;
@@ -849,15 +864,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     fence_proxy_async_global();  // H, written through the async proxy, before our TMA reads
                 }
                 const void *ta = second ? (const void *)&tm_h : (const void *)&tm_x;
-                const void *tb = second ? (const void *)&tm_w2 : (const void *)&tm_w1;
+                const void *tb = second ? (bw == BN ? (const void *)&tm_w2 : (const void *)&tm_w2h)
+                                        : (bw == BN ? (const void *)&tm_w1 : (const void *)&tm_w1h);
                 const int kbs = second ? kb2 : kb1;
-                const int a_row = m * BMP + (int)rank * BM, b_row = n * BN + (int)rank * (BN / 2);
+                const int a_row = m * BMP + (int)rank * BM, b_row = n * bw + (int)rank * (bw / 2);
                 for (int kb = 0; kb < kbs; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, status, 41)) {
                         ok = false;
                         break;
                     }
-                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * (L::a_bytes + L::b_bytes)));
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * (L::a_bytes + b_bytes)));
                     const uint32_t leader_full = map_to_rank(&full[stage], 0);
                     tma_load_3d_pair(sA + stage * L::a_bytes, ta, leader_full, (k0 + kb) * BK, a_row, e);
                     tma_load_3d_pair(sB + stage * L::b_bytes, tb, leader_full, (k0 + kb) * BK, b_row, e);
@@ -875,7 +891,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BMP, BN);
+            const uint32_t idesc = idesc_bf16_f32(BMP, bw);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -960,10 +976,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
             if (second)
                 epilogue_async<BN, kEpiGatedScatter>(t_row, e, row_base, min(counts[e], C), C, n, d, y, nullptr,
-                                                     slot_token, gate, my_stage, ks > 0);
+                                                     slot_token, gate, my_stage, ks > 0, 0, nullptr, bw);
             else
                 epilogue_async<BN, kEpiHiddenRelu>(t_row, e, row_base, min(counts[e], C), C, n, F, nullptr,
-                                                   &tm_hstore, slot_token, gate, my_stage);
+                                                   &tm_hstore, slot_token, gate, my_stage, false, 0, nullptr, bw);
             tc_fence_before();
             mbar_arrive_cluster(map_to_rank(&acc_empty[acc], 0));
             if (lane == 0 && (!second || ks < split - 1)) {
@@ -1081,13 +1097,14 @@ cudaError_t launch_ffn_fused(const switch_dims_t &dims, const void *xbuf, const 
     auto kern = tc_ffn_fused_pair<STAGES>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    CUtensorMap tx, tw1, th, tw2, ths;
+    CUtensorMap tx, tw1, th, tw2, tw1h, tw2h, ths;
     if (!make_tmap(&tx, xbuf, E, C, d, BM) || !make_tmap(&tw1, w_in, E, F, d, kFusedBN / 2) ||
         !make_tmap(&th, ws.hidden, E, C, F, BM) || !make_tmap(&tw2, w_out, E, d, F, kFusedBN / 2) ||
+        !make_tmap(&tw1h, w_in, E, F, d, kFusedBN / 4) || !make_tmap(&tw2h, w_out, E, d, F, kFusedBN / 4) ||
         !make_tmap(&ths, ws.hidden, E, C, F, 32))
         return cudaErrorInvalidValue;
     const int MT = (C + 2 * BM - 1) / (2 * BM);
-    const int n2 = (d + kFusedBN - 1) / kFusedBN;
+    const int n2 = (d + kFusedBN / 2 - 1) / (kFusedBN / 2);  // at the narrow tile width
     if (zero_done) {  // counters, the tile claim counter and the y_done counters
         err = cudaMemsetAsync(ws.done, 0, fused_counter_ints(E, C, d) * sizeof(int32_t), stream);
         if (err != cudaSuccess) return err;
@@ -1096,10 +1113,11 @@ cudaError_t launch_ffn_fused(const switch_dims_t &dims, const void *xbuf, const 
     const int64_t tiles2 = m_tiles * n2;
     const int max_pairs = device_sm_count() / 2;
     // upper bound on the tile count (GEMM2 tiles may be cut into up to 4 parts on the device)
-    const int64_t tiles = m_tiles * ((F + kFusedBN - 1) / kFusedBN) + 4 * tiles2;
+    const int64_t tiles = m_tiles * ((F + kFusedBN / 2 - 1) / (kFusedBN / 2)) + 4 * tiles2;
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(max_pairs, tiles));
     launch_begin(K_FFN_TC_FUSED, stream);
-    err = launch_kernel(kern, dim3(2 * pairs), dim3(kThreads), smem, stream, !zero_done, tx, tw1, th, tw2, ths, y,
+    err = launch_kernel(kern, dim3(2 * pairs), dim3(kThreads), smem, stream, !zero_done, tx, tw1, th, tw2, tw1h, tw2h,
+                        ths, y,
                         counts, E, C, d, F, slot_token, gate, ws.done, MT, static_cast<DeviceStatus *>(ws.status));
     launch_end(stream);
     return err;

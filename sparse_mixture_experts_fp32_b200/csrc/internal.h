@@ -77,10 +77,11 @@ struct Workspace {
 };
 
 size_t workspace_bytes(const switch_dims_t &dims);
-// int32 counters the fused expert FFN keeps in Workspace::done.
+// int32 counters the fused expert FFN keeps in Workspace::done (GEMM2 counters
+// for its narrower 128-column tiles, the larger count).
 inline int64_t fused_counter_ints(int64_t N, int64_t C, int64_t d) {
     const int64_t MT = (C + 255) / 256;
-    return N * MT + 1 + N * MT * ((d + 255) / 256);
+    return N * MT + 1 + N * MT * ((d + 127) / 128);
 }
 // Bytes at the start of the workspace layout that the routing step uses
 // (status word, ticket, per-tile counts / sums / offsets, probability totals).

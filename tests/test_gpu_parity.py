@@ -80,11 +80,13 @@ def test_layer_small_simt_router(orc, name, T):
     full_check(orc, synth.WORKLOADS[name], T, flags=sm.SWITCH_FLAG_SIMT_ROUTER)
 
 
-@pytest.mark.parametrize("name,T", [("base8", 3000), ("large128", 2500), ("bigexpert64", 400)])
+@pytest.mark.parametrize("name,T", [("base8", 3000), ("large128", 2500), ("bigexpert64", 400),
+                                    ("base128_skew", 6000)])
 def test_fused_ffn_matches_two_launches(name, T):
     """One persistent launch for both expert GEMMs agrees with two launches.  Where the fused
     kernel splits GEMM2 tiles over K (few GEMM2 tiles), y = g*acc0 + g*acc1 instead of
-    g*(acc0 + acc1): the two differ by fp32 rounding only."""
+    g*(acc0 + acc1): the two differ by fp32 rounding only.  The skewed case (few kept rows)
+    runs the fused kernel's 128-column tiles."""
     wl = synth.WORKLOADS[name]
     C = synth_capacity(wl, T)
     inp = synth.inputs(wl, T=T, experts=range(min(wl.num_experts, 16)))
