@@ -98,7 +98,11 @@ enum {
      * activations and the ungated expert outputs) and runs the two expert
      * GEMMs and the combine as separate launches; switch_workspace_size grows
      * accordingly.  switch_layer_bwd requires it.  bfloat16 experts only. */
-    SWITCH_FLAG_TRAINING = 32
+    SWITCH_FLAG_TRAINING = 32,
+    /* The routing step also sums the entropy of every token's router
+     * distribution per 64-token tile into the workspace, for
+     * switch_router_stats. */
+    SWITCH_FLAG_ROUTER_STATS = 64
 };
 
 typedef struct {
@@ -246,6 +250,22 @@ switch_status_t switch_layer_fwd_top2(const switch_dims_t *dims, const void *x, 
                                       const float *logit_bias, const void *w_in, const void *w_out, void *y,
                                       int32_t *expert, float *gate, int32_t *slot, int32_t *counts, float *aux,
                                       void *workspace, size_t workspace_bytes, switch_stream_t stream);
+
+/* Router statistics that the sources list for monitoring a Switch layer next
+ * to its loss (kasblo "Switch Transformerとは？", end of section "補助負荷分散
+ * lossは何を均等にするのか": tokens per expert, use of capacity, the overflow /
+ * dropped-token rate, the entropy of the router probabilities), for the last
+ * switch_route / switch_layer_fwd (or top-2) call made with the same dims and
+ * workspace.  stats [4] float32 (device):
+ *   stats[0] mean over tokens of -sum_i p_i ln p_i  (NaN unless that call had
+ *            SWITCH_FLAG_ROUTER_STATS in its dims flags, as these dims must)
+ *   stats[1] dropped fraction  sum_i max(0, counts_i - C) / T
+ *   stats[2] capacity utilisation  sum_i min(counts_i, C) / (N C)
+ *   stats[3] busiest expert's load over the uniform load  max_i counts_i N / T
+ * counts [N] as that call wrote them (after a top-2 call: assignments; the
+ * dropped fraction is then per (token, choice) over T).  All 0 when T == 0. */
+switch_status_t switch_router_stats(const switch_dims_t *dims, const int32_t *counts, const void *workspace,
+                                    size_t workspace_bytes, float *stats, switch_stream_t stream);
 
 /* Backward pass of the layer (top-1), after a switch_layer_fwd call made with
  * SWITCH_FLAG_TRAINING in the same dims and the same workspace (whose

@@ -79,6 +79,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_layer_bwd.argtypes = [I64, I32, I32, I32, I64, P, ctypes.c_int, P, P, P, P, ctypes.c_int, P, D,
                                      P, P, P, P, P]
     lib.oracle_layer_bwd.restype = None
+    lib.oracle_router_stats.argtypes = [I64, I32, I64, P, P, P]
+    lib.oracle_router_stats.restype = None
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_set_threads.restype = None
     return lib
@@ -291,6 +293,15 @@ class Oracle:
                                   _ptr(out["dw_r"]), _ptr(out["dbias"]), _ptr(out["dw_in"]), _ptr(out["dw_out"]))
         out["capacity"] = capacity
         return out
+
+    def router_stats(self, probs: np.ndarray, counts: np.ndarray, C: int) -> dict:
+        """Mean router entropy, dropped-token fraction, capacity utilisation, busiest-expert load."""
+        probs = np.ascontiguousarray(probs, dtype=np.float64)
+        counts = np.ascontiguousarray(counts, dtype=np.int32)
+        T, N = probs.shape
+        out = np.empty(4, dtype=np.float64)
+        self.lib.oracle_router_stats(T, N, int(C), _ptr(probs), _ptr(counts), _ptr(out))
+        return dict(entropy=out[0], drop_fraction=out[1], capacity_utilisation=out[2], max_load=out[3])
 
     def expert_row(self, x_row, w_in_e, w_out_e, gate: float) -> np.ndarray:
         x_row = np.ascontiguousarray(x_row)

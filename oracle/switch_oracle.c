@@ -357,6 +357,45 @@ void oracle_output_rows_top2(int32_t d, int32_t F, int64_t n_rows, const int64_t
     }
 }
 
+/* Router statistics that the sources list for monitoring a Switch layer
+ * next to its loss (kasblo "Switch Transformerとは？", end of section "補助
+ * 負荷分散lossは何を均等にするのか": tokens per expert, use of capacity, the
+ * overflow / dropped-token rate, the entropy of the router probabilities):
+ *   out[0] = mean over the T tokens of -sum_i p_i ln p_i   (0 ln 0 = 0)
+ *   out[1] = dropped-token fraction  sum_i max(0, counts_i - C) / T
+ *   out[2] = capacity utilisation    sum_i min(counts_i, C) / (N C)
+ *   out[3] = busiest expert's load over the uniform load, max_i counts_i N / T
+ * probs is [T,N]; every value is 0 when T == 0. */
+void oracle_router_stats(int64_t T, int32_t N, int64_t C, const double *probs, const int32_t *counts, double *out)
+{
+    for (int k = 0; k < 4; ++k)
+        out[k] = 0.0;
+    if (T <= 0)
+        return;
+    double entropy = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+        double h = 0.0;
+        for (int32_t i = 0; i < N; ++i) {
+            double p = probs[t * (int64_t)N + i];
+            if (p > 0.0)
+                h -= p * log(p);
+        }
+        entropy += h;
+    }
+    int64_t dropped = 0, kept = 0, busiest = 0;
+    for (int32_t i = 0; i < N; ++i) {
+        int64_t c = counts[i];
+        dropped += c > C ? c - C : 0;
+        kept += c < C ? c : C;
+        if (c > busiest)
+            busiest = c;
+    }
+    out[0] = entropy / (double)T;
+    out[1] = (double)dropped / (double)T;
+    out[2] = (double)kept / ((double)N * (double)C);
+    out[3] = (double)busiest * (double)N / (double)T;
+}
+
 /* ------------------------------------------------------------------------
  * Backward pass of the top-1 layer.  The forward's loss enters as the
  * upstream gradient dy[T,d] of the layer output y and a scalar g_aux, the

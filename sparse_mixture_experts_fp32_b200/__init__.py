@@ -32,6 +32,7 @@ SWITCH_FLAG_GEMM_1CTA = 4
 SWITCH_FLAG_FFN_TWO_LAUNCHES = 8
 SWITCH_FLAG_SEPARATE_SCAN = 16
 SWITCH_FLAG_TRAINING = 32
+SWITCH_FLAG_ROUTER_STATS = 64
 
 STATUS = {
     0: "SWITCH_OK", 1: "SWITCH_ERR_NULL", 2: "SWITCH_ERR_SHAPE", 3: "SWITCH_ERR_DTYPE", 4: "SWITCH_ERR_ALIGN",
@@ -42,7 +43,7 @@ STATUS = {
 EXPORTED = ("switch_capacity", "switch_workspace_size", "switch_route", "switch_route_noalloc", "switch_dispatch",
             "switch_expert_ffn",
             "switch_combine", "switch_layer_fwd", "switch_route_top2", "switch_combine_top2", "switch_layer_fwd_top2",
-            "switch_layer_bwd",
+            "switch_layer_bwd", "switch_router_stats",
             "switch_check", "switch_selftest_wait_timeout", "switch_status_string",
             "switch_launch_count",
             "switch_trace_start", "switch_trace_read", "switch_trace_stop", "switch_kernel_name")
@@ -91,6 +92,7 @@ def lib() -> ctypes.CDLL:
         "switch_combine_top2": (I, [D, P, P, P, P, P, P]),
         "switch_layer_fwd_top2": (I, [D, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
         "switch_layer_bwd": (I, [D, P, P, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, P, P, S, P]),
+        "switch_router_stats": (I, [D, P, P, S, P, P]),
         "switch_check": (I, [P, S, P]),
         "switch_selftest_wait_timeout": (I, [P, S, P]),
         "switch_status_string": (ctypes.c_char_p, [I]),
@@ -240,6 +242,12 @@ def switch_layer_bwd(d, x, w_r, w_in, w_out, expert, gate, slot, counts, dy, g_a
         "switch_layer_bwd")
 
 
+def switch_router_stats(d, counts, workspace, stats, stream=None):
+    _ok(lib().switch_router_stats(ctypes.byref(d), _ptr(counts), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _ptr(stats),
+                                  _stream(stream, workspace)), "switch_router_stats")
+
+
 def switch_check(workspace, stream=None) -> int:
     """Synchronise and return the device status code (0 = ok); does not raise."""
     return int(lib().switch_check(_ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -352,6 +360,7 @@ def route(x, w_r, num_experts=None, capacity=None, capacity_factor=None, logit_b
     switch_route(d, x, w_r, logit_bias, out["expert"], out["gate"], out["slot"], out["counts"], out["slot_token"],
                  out["aux"], ws, stream)
     out["capacity"] = C
+    out["flags"] = d.flags
     out["workspace"] = ws
     return out
 
@@ -399,6 +408,7 @@ def route_top2(x, w_r, capacity=None, capacity_factor=None, logit_bias=None, d_f
     switch_route_top2(d, x, w_r, logit_bias, out["expert"], out["gate"], out["slot"], out["counts"],
                       out["slot_token"], out["aux"], ws, stream)
     out["capacity"] = C
+    out["flags"] = d.flags
     out["workspace"] = ws
     return out
 
@@ -420,3 +430,14 @@ def layer_bwd(fwd: dict, x, w_r, w_in, w_out, dy, g_aux: float = 0.0, logit_bias
     switch_layer_bwd(d, x, w_r, w_in, w_out, fwd["expert"], fwd["gate"], fwd["slot"], fwd["counts"], dy, g_aux,
                      out["dx"], out["dw_r"], out["dbias"], out["dw_in"], out["dw_out"], fwd["workspace"], stream)
     return out
+
+
+def router_stats(result: dict, T: int, d_model: int, d_ff: int, dtype, stream=None):
+    """Router statistics of a route / layer_fwd result made with SWITCH_FLAG_ROUTER_STATS:
+    a 4-element float32 tensor (mean entropy, dropped fraction, capacity utilisation, busiest load)."""
+    import torch
+    counts = result["counts"]
+    d = dims(T, d_model, d_ff, counts.numel(), result["capacity"], dtype, result.get("flags", SWITCH_FLAG_ROUTER_STATS))
+    stats = torch.empty(4, dtype=torch.float32, device=counts.device)
+    switch_router_stats(d, counts, result["workspace"], stats, stream)
+    return stats

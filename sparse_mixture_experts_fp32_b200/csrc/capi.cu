@@ -26,7 +26,7 @@ int64_t tiles_of(const switch_dims_t &d) { return (d.T + kTileT - 1) / kTileT; }
 
 struct Sections {
     size_t status, ticket, hist, psum, tile_off, prob_total, w_split, slot_token, xbuf, ybuf, hidden, done, hist2,
-        tile_off2, counts_first, probs, dh, grad_e, grad_z, w_out_t, w_in_t, grad_e_t, hidden_t, xbuf_t, grad_z_t,
+        tile_off2, counts_first, ent, probs, dh, grad_e, grad_z, w_out_t, w_in_t, grad_e_t, hidden_t, xbuf_t, grad_z_t,
         dw_part, db_part, total;
 };
 
@@ -55,6 +55,7 @@ Sections layout(const switch_dims_t &d) {
     s.hist2 = take(N * tiles * 4);
     s.tile_off2 = take(N * tiles * 4);
     s.counts_first = take(N * 4);
+    s.ent = take(tiles * 4);
     if (d.flags & SWITCH_FLAG_TRAINING) {  // kept by the training forward, used by the backward pass
         const size_t T = (size_t)d.T, dm = (size_t)d.d_model, F = (size_t)d.d_ff, es = elem_size(d);
         const size_t Cp = (C + 63) / 64 * 64, chunks = (size_t)router_dw_chunks(d.T);
@@ -190,6 +191,7 @@ Workspace carve_workspace(const switch_dims_t &dims, void *base) {
     w.hist2 = reinterpret_cast<int32_t *>(b + s.hist2);
     w.tile_off2 = reinterpret_cast<int32_t *>(b + s.tile_off2);
     w.counts_first = reinterpret_cast<int32_t *>(b + s.counts_first);
+    w.ent = (dims.flags & SWITCH_FLAG_ROUTER_STATS) ? reinterpret_cast<float *>(b + s.ent) : nullptr;
     const bool training = (dims.flags & SWITCH_FLAG_TRAINING) != 0;
     auto at = [&](size_t o) -> void * { return training ? (void *)(b + o) : nullptr; };
     w.probs = static_cast<float *>(at(s.probs));
@@ -426,6 +428,18 @@ switch_status_t switch_layer_fwd_top2(const switch_dims_t *dims, const void *x, 
     return from_cuda(err);
 }
 
+switch_status_t switch_router_stats(const switch_dims_t *dims, const int32_t *counts, const void *workspace,
+                                    size_t workspace_bytes_given, float *stats, switch_stream_t stream) {
+    switch_status_t s = check_dims(dims);
+    if (s != SWITCH_OK) return s;
+    s = check_ptrs({counts, workspace, stats}, {});
+    if (s != SWITCH_OK) return s;
+    if (workspace_bytes_given < workspace_bytes(*dims)) return SWITCH_ERR_WORKSPACE;
+    if ((s = check_device()) != SWITCH_OK) return s;
+    const Workspace ws = carve_workspace(*dims, const_cast<void *>(workspace));
+    return from_cuda(launch_router_stats(*dims, counts, ws, stats, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 switch_status_t switch_layer_bwd(const switch_dims_t *dims, const void *x, const float *w_r, const void *w_in,
                                  const void *w_out, const int32_t *expert, const float *gate, const int32_t *slot,
                                  const int32_t *counts, const float *dy, float g_aux, float *dx, float *dw_r,
@@ -564,6 +578,7 @@ const char *switch_kernel_name(int32_t id) {
         case K_BWD_ROUTER_DX: return "bwd_router_dx";
         case K_BWD_ROUTER_DW: return "bwd_router_dw";
         case K_BWD_REDUCE: return "bwd_reduce";
+        case K_ROUTER_STATS: return "router_stats";
     }
     return "?";
 }

@@ -41,6 +41,7 @@ enum KernelId : int32_t {
     K_BWD_ROUTER_DX = 24,
     K_BWD_ROUTER_DW = 25,
     K_BWD_REDUCE = 26,
+    K_ROUTER_STATS = 27,
 };
 
 struct Workspace {
@@ -60,6 +61,7 @@ struct Workspace {
     int32_t *hist2;      // top-2: [N][tiles] second choices of each expert in each tile
     int32_t *tile_off2;  // top-2: [N][tiles] first slot of each tile's second choices
     int32_t *counts_first;  // top-2: [N] first choices per expert (the aux loss's f)
+    float *ent;          // with SWITCH_FLAG_ROUTER_STATS: [tiles] per-tile sums of the router entropy (else null)
     float *probs;        // training: [T][N] router probabilities kept for the backward pass (else null)
     // training only (SWITCH_FLAG_TRAINING): backward-pass buffers
     float *dh;           // [T][N] gradient of the router logits
@@ -125,6 +127,10 @@ cudaError_t launch_ffn_simt(const switch_dims_t &dims, const void *xbuf, const v
 cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
                           const int32_t *counts, void *ybuf, const int32_t *slot_token, const float *gate, float *y,
                           const Workspace &ws, cudaStream_t stream);
+
+// Router statistics from the per-tile entropy sums a routing call left in the workspace.
+cudaError_t launch_router_stats(const switch_dims_t &dims, const int32_t *counts, const Workspace &ws, float *stats,
+                                cudaStream_t stream);
 
 // Backward pass (bfloat16 experts; the workspace of a SWITCH_FLAG_TRAINING forward).
 int64_t router_dw_chunks(int64_t T);

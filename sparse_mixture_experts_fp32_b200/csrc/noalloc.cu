@@ -81,11 +81,12 @@ extern "C" switch_status_t switch_route_noalloc(const switch_dims_t *dims, const
     // first block clears the ticket and the status word, and every other
     // section is fully rewritten by the call, so the previous call's
     // contents never leak into this one.
-    // The training flag would make the routers also write the [T][N]
-    // probabilities into a section past the routing scratch; routing here
-    // never keeps them, so the flag is cleared for the carve and the launch.
+    // The training and statistics flags would make the routers also write the
+    // [T][N] probabilities or per-tile entropy sums into sections past the
+    // routing scratch; routing here keeps neither, so both flags are cleared
+    // for the carve and the launch.
     switch_dims_t route_dims = *dims;
-    route_dims.flags &= ~SWITCH_FLAG_TRAINING;
+    route_dims.flags &= ~(SWITCH_FLAG_TRAINING | SWITCH_FLAG_ROUTER_STATS);
     const Workspace ws = carve_workspace(route_dims, scratch);
     const cudaError_t err = launch_route(route_dims, x, w_r, logit_bias, expert, gate, slot, counts, slot_token, aux,
                                          ws, reinterpret_cast<cudaStream_t>(stream));

@@ -43,7 +43,7 @@ template <int J, bool TOP2>
 __device__ __forceinline__ void token_epilogue(const float (&v)[J], const int (&idx)[J], const bool (&own)[J],
                                                int64_t t, float *warp_psum, int32_t *warp_hist,
                                                int32_t *warp_hist2, int32_t *expert, float *gate, float *probs,
-                                               int N) {
+                                               int N, float *warp_ent) {
     const int lane = threadIdx.x & 31;
     float m = -FLT_MAX;
     int arg = 0x7fffffff;
@@ -94,6 +94,15 @@ __device__ __forceinline__ void token_epilogue(const float (&v)[J], const int (&
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (warp_ent) {  // entropy -sum p ln p = ln s - sum e (v - m) / s
+        float sv = 0.f;
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+            if (idx[j] >= 0 && own[j]) sv += ex[j] * (v[j] - m);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sv += __shfl_xor_sync(0xffffffffu, sv, off);
+        if (lane == 0) *warp_ent += logf(s) - sv / s;
+    }
 #pragma unroll
     for (int j = 0; j < J; ++j)
         if (idx[j] >= 0 && own[j]) {
@@ -119,7 +128,13 @@ __device__ __forceinline__ void token_epilogue(const float (&v)[J], const int (&
 // expert-major ([N][tiles]) for the scan (with hist2: second-choice counts too).
 __device__ __forceinline__ void publish_tile(const float *psum_w, const int32_t *hist_w, const int32_t *hist2_w,
                                              int N, int tiles, int tile, int32_t *hist, int32_t *hist2,
-                                             float *psum) {
+                                             float *psum, const float *ent_w, float *ent) {
+    if (ent && threadIdx.x == 0) {  // the tile's entropy sum, warps in fixed order
+        float e = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) e += ent_w[w];
+        ent[tile] = e;
+    }
     for (int i = threadIdx.x; i < N; i += kThreads) {
         int32_t c = 0, c2 = 0;
         float p = 0.f;
@@ -204,16 +219,19 @@ __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restr
                                                                float *__restrict__ gate, int32_t *__restrict__ hist,
                                                                int32_t *__restrict__ hist2,
                                                                float *__restrict__ psum, float *__restrict__ probs,
-                                                               uint32_t *ticket, DeviceStatus *status) {
+                                                               float *__restrict__ ent, uint32_t *ticket,
+                                                               DeviceStatus *status) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *wsm = reinterpret_cast<float *>(smem_raw);  // [d][NP]
     float *psum_w = wsm + (size_t)d * NP;               // [kWarps][N]
     int32_t *hist_w = reinterpret_cast<int32_t *>(psum_w + kWarps * N);
     int32_t *hist2_w = hist_w + kWarps * N;             // [kWarps][N] second choices (TOP2)
+    float *ent_w = reinterpret_cast<float *>(hist2_w + kWarps * N);  // [kWarps] entropy sums
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x;
 
     if (tile == 0 && tid == 0) reset_call_state(ticket, status);
+    if (tid < kWarps) ent_w[tid] = 0.f;
     for (int i = tid; i < d * NP; i += kThreads) {
         const int k = i / NP, e = i % NP;
         wsm[i] = e < N ? w_r[(int64_t)e * d + k] : 0.f;
@@ -290,10 +308,10 @@ __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restr
         int idx[1] = {valid_e ? my_e : -1};
         bool own[1] = {(lane & ((1 << SHIFT) - 1)) == 0};
         token_epilogue<1, TOP2>(v, idx, own, t, psum_w + warp * N, hist_w + warp * N, hist2_w + warp * N, expert,
-                                gate, probs, N);
+                                gate, probs, N, ent ? ent_w + warp : nullptr);
     }
     __syncthreads();
-    publish_tile(psum_w, hist_w, hist2_w, N, tiles, tile, hist, TOP2 ? hist2 : nullptr, psum);
+    publish_tile(psum_w, hist_w, hist2_w, N, tiles, tile, hist, TOP2 ? hist2 : nullptr, psum, ent_w, ent);
 }
 
 // ---------------------------------------------------------------------------
@@ -318,10 +336,10 @@ struct Staged {
         return ((a > b ? a : b) + 15) / 16 * 16;
     }
     // smem layout: x tile | W_r as [d/V][V][NP] | per-warp sums | counts | second-choice counts |
-    // 5 mbarriers | raw W_r (optional)
+    // per-token entropies [64] | 5 mbarriers | raw W_r (optional)
     static size_t smem_base(int d, int NP) {
         return (size_t)x_region(d, NP) + (size_t)((d / V) * wpitch(NP)) * 4 + (size_t)(kWarps * NP) * 4 +
-               2 * (size_t)NP * 4 + 5 * 8 + 16;
+               2 * (size_t)NP * 4 + kTileT * 4 + 5 * 8 + 16;
     }
     static size_t smem(int d, int NP, int N, bool raw) {
         return smem_base(d, NP) + (raw ? (size_t)N * d * 4 + 16 : 0);
@@ -333,7 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     router_staged_kernel(const XT *__restrict__ x, const float *__restrict__ w_r, const float *__restrict__ bias,
                          int64_t T, int d, int N, int tiles, int32_t *__restrict__ expert, float *__restrict__ gate,
                          int32_t *__restrict__ hist, int32_t *__restrict__ hist2, float *__restrict__ psum,
-                         float *__restrict__ probs, uint32_t *ticket, DeviceStatus *status, int raw_w) {
+                         float *__restrict__ probs, float *__restrict__ ent, uint32_t *ticket, DeviceStatus *status,
+                         int raw_w) {
     using S = Staged<XT>;
     constexpr int V = S::V;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -344,7 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *psum_w = wsm + (d / V) * wpitch;
     int32_t *hist_s = reinterpret_cast<int32_t *>(psum_w + kWarps * NP);
     int32_t *hist2_s = hist_s + NP;  // second choices (TOP2)
-    uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(hist2_s + NP) + 15) & ~uintptr_t(15));
+    float *ent_tok = reinterpret_cast<float *>(hist2_s + NP);  // [64] per-token entropy (with ent)
+    uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(ent_tok + kTileT) + 15) & ~uintptr_t(15));
     float *w_raw = reinterpret_cast<float *>(bar + 5) + 2;  // 16-byte aligned: bar is, and 5 * 8 + 8 = 48
     const int tid = threadIdx.x;
     const int tile = blockIdx.x;
@@ -487,12 +507,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (TOP2 && arg2 < 0) arg2 = arg == 0 ? 1 : 0;  // N == 1 only, which top-2 routing rejects
-        float s = 0.f;
+        float s = 0.f, sv = 0.f;
 #pragma unroll
         for (int e = 0; e < NP; ++e) {
-            h[e] = e < N ? expf(h[e] - m) : 0.f;
+            const float z = h[e] - m;
+            h[e] = e < N ? expf(z) : 0.f;
             s += h[e];
+            if (e < N) sv += h[e] * z;
         }
+        if (ent) ent_tok[tl] = valid ? logf(s) - sv / s : 0.f;  // -sum p ln p
 #pragma unroll
         for (int e = 0; e < NP; ++e) ptile[tl * NP + e] = valid ? h[e] / s : 0.f;  // p_e
         if (probs && valid) {  // kept for the backward pass
@@ -516,6 +539,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     __syncthreads();
+    if (ent && tid == 0) {  // the tile's entropy sum in token order
+        float e = 0.f;
+        for (int tl = 0; tl < kTileT; ++tl) e += ent_tok[tl];
+        ent[tile] = e;
+    }
     // tile sums of p: four interleaved partial sums, combined in fixed order (deterministic)
     for (int i = tid; i < N; i += kThreads) {
         float p4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -544,7 +572,8 @@ __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__rest
                                                                 float *__restrict__ gate, int32_t *__restrict__ hist,
                                                                 int32_t *__restrict__ hist2,
                                                                 float *__restrict__ psum, float *__restrict__ probs,
-                                                                uint32_t *ticket, DeviceStatus *status) {
+                                                                float *__restrict__ ent, uint32_t *ticket,
+                                                                DeviceStatus *status) {
     constexpr int TE = EC / 16;  // experts per thread
     constexpr int TT = 4;        // tokens per thread
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -555,12 +584,14 @@ __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__rest
     float *psum_w = logits + kTileT * NL;              // [kWarps][N]
     int32_t *hist_w = reinterpret_cast<int32_t *>(psum_w + kWarps * N);
     int32_t *hist2_w = hist_w + kWarps * N;            // [kWarps][N] second choices (TOP2)
+    float *ent_w = reinterpret_cast<float *>(hist2_w + kWarps * N);  // [kWarps] entropy sums
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tx = tid % 16, ty = tid / 16;
     const int tile = blockIdx.x;
     const int64_t t0 = (int64_t)tile * kTileT;
 
     if (tile == 0 && tid == 0) reset_call_state(ticket, status);
+    if (tid < kWarps) ent_w[tid] = 0.f;
     for (int i = tid; i < kWarps * N; i += kThreads) {
         psum_w[i] = 0.f;
         hist_w[i] = 0;
@@ -625,10 +656,10 @@ __global__ void __launch_bounds__(kThreads) router_tiled_kernel(const XT *__rest
             v[j] = e < N ? logits[r * NL + e] + (bias ? bias[e] : 0.f) : 0.f;
         }
         token_epilogue<J, TOP2>(v, idx, own, t, psum_w + warp * N, hist_w + warp * N, hist2_w + warp * N, expert,
-                                gate, probs, N);
+                                gate, probs, N, ent ? ent_w + warp : nullptr);
     }
     __syncthreads();
-    publish_tile(psum_w, hist_w, hist2_w, N, tiles, tile, hist, TOP2 ? hist2 : nullptr, psum);
+    publish_tile(psum_w, hist_w, hist2_w, N, tiles, tile, hist, TOP2 ? hist2 : nullptr, psum, ent_w, ent);
 }
 
 // ---------------------------------------------------------------------------
@@ -996,13 +1027,14 @@ template <typename XT, int NP, bool TOP2>
 cudaError_t launch_router_warp(const switch_dims_t &dims, const XT *x, const float *w_r, const float *bias,
                                int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts, d = dims.d_model;
-    const size_t smem = (size_t)d * NP * sizeof(float) + (size_t)kWarps * N * (sizeof(float) + 2 * sizeof(int32_t));
+    const size_t smem = (size_t)d * NP * sizeof(float) + (size_t)kWarps * N * (sizeof(float) + 2 * sizeof(int32_t)) +
+                        kWarps * sizeof(float);
     auto kern = router_warp_kernel<XT, NP, TOP2>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_WARP, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
-                                                         ws.hist, ws.hist2, ws.psum, ws.probs, ws.ticket,
+                                                         ws.hist, ws.hist2, ws.psum, ws.probs, ws.ent, ws.ticket,
                                                          static_cast<DeviceStatus *>(ws.status));
     err = cudaGetLastError();
     launch_end(stream);
@@ -1023,7 +1055,7 @@ cudaError_t launch_router_staged(const switch_dims_t &dims, const XT *x, const f
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_STAGED, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
-                                                         ws.hist, ws.hist2, ws.psum, ws.probs, ws.ticket,
+                                                         ws.hist, ws.hist2, ws.psum, ws.probs, ws.ent, ws.ticket,
                                                          static_cast<DeviceStatus *>(ws.status), raw ? 1 : 0);
     err = cudaGetLastError();
     launch_end(stream);
@@ -1035,13 +1067,13 @@ cudaError_t launch_router_tiled(const switch_dims_t &dims, const XT *x, const fl
                                 int32_t *expert, float *gate, const Workspace &ws, cudaStream_t stream) {
     const int N = dims.num_experts, d = dims.d_model;
     const size_t smem = (size_t)(kKC * kTileT + kKC * EC + kTileT * (N + 1)) * sizeof(float) +
-                        (size_t)kWarps * N * (sizeof(float) + 2 * sizeof(int32_t));
+                        (size_t)kWarps * N * (sizeof(float) + 2 * sizeof(int32_t)) + kWarps * sizeof(float);
     auto kern = router_tiled_kernel<XT, EC, TOP2>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_TILED, stream);
     kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
-                                                         ws.hist, ws.hist2, ws.psum, ws.probs, ws.ticket,
+                                                         ws.hist, ws.hist2, ws.psum, ws.probs, ws.ent, ws.ticket,
                                                          static_cast<DeviceStatus *>(ws.status));
     err = cudaGetLastError();
     launch_end(stream);
@@ -1082,7 +1114,68 @@ cudaError_t launch_any_router(const switch_dims_t &dims, const void *x, const fl
                : launch_router<float, TOP2>(dims, static_cast<const float *>(x), w_r, bias, expert, gate, ws, stream);
 }
 
+// Router statistics from a routing call's per-tile entropy sums and counts:
+// stats = {mean entropy, dropped fraction, capacity utilisation, busiest load
+// over the uniform load}; fp64 sums in a fixed order.  One block.
+__global__ void __launch_bounds__(256) router_stats_kernel(const float *__restrict__ ent, int tiles,
+                                                          const int32_t *__restrict__ counts, int N, int C,
+                                                          int64_t T, float *__restrict__ stats) {
+    __shared__ double s_ent[kWarps];
+    __shared__ long long s_drop[kWarps], s_kept[kWarps], s_max[kWarps];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    double e = 0.0;
+    if (ent)
+        for (int i = tid; i < tiles; i += 256) e += (double)ent[i];
+    long long drop = 0, kept = 0, mx = 0;
+    for (int i = tid; i < N; i += 256) {
+        const long long c = counts[i];
+        drop += c > C ? c - C : 0;
+        kept += c < C ? c : C;
+        mx = c > mx ? c : mx;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        e += __shfl_xor_sync(0xffffffffu, e, off);
+        drop += __shfl_xor_sync(0xffffffffu, drop, off);
+        kept += __shfl_xor_sync(0xffffffffu, kept, off);
+        const long long o = __shfl_xor_sync(0xffffffffu, mx, off);
+        mx = o > mx ? o : mx;
+    }
+    if (lane == 0) {
+        s_ent[warp] = e;
+        s_drop[warp] = drop;
+        s_kept[warp] = kept;
+        s_max[warp] = mx;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        double et = 0.0;
+        long long dt = 0, kt = 0, mt = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            et += s_ent[w];
+            dt += s_drop[w];
+            kt += s_kept[w];
+            mt = s_max[w] > mt ? s_max[w] : mt;
+        }
+        const bool any = T > 0;
+        stats[0] = !ent ? __int_as_float(0x7fc00000) : any ? (float)(et / (double)T) : 0.f;
+        stats[1] = any ? (float)((double)dt / (double)T) : 0.f;
+        stats[2] = any ? (float)((double)kt / ((double)N * (double)C)) : 0.f;
+        stats[3] = any ? (float)((double)mt * (double)N / (double)T) : 0.f;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_router_stats(const switch_dims_t &dims, const int32_t *counts, const Workspace &ws, float *stats,
+                                cudaStream_t stream) {
+    launch_begin(K_ROUTER_STATS, stream);
+    router_stats_kernel<<<1, 256, 0, stream>>>(ws.ent, (int)ws.tiles, counts, dims.num_experts, dims.capacity,
+                                               dims.T, stats);
+    const cudaError_t err = cudaGetLastError();
+    launch_end(stream);
+    return err;
+}
 
 cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
                          int32_t *expert, float *gate, int32_t *slot, int32_t *counts, int32_t *slot_token,

@@ -87,7 +87,9 @@ struct RouterLayout {
     static constexpr size_t barriers = (2 * STAGES + 2 + 2 + 1) * 8 + 16;
     // bias, per-quarter sums of p and per-64-token counts (both double-buffered by tile parity),
     // and the exchange of per-group max, argmax and sum between the warps of a token
-    static constexpr size_t epi = (size_t)BN * 4 + 2 * 4 * BN * 4 + 2 * 2 * BN * 4 + 3 * (BN / 32) * RM * 4;
+    // (+ the exchange of each group's entropy partial and per-quarter entropy sums, both parities)
+    static constexpr size_t epi =
+        (size_t)BN * 4 + 2 * 4 * BN * 4 + 2 * 2 * BN * 4 + 3 * (BN / 32) * RM * 4 + (BN / 32) * RM * 4 + 2 * 4 * 4;
     // top-2: second-choice counts and the exchange of each group's second best
     static constexpr size_t epi2 = TOP2 ? 2 * 2 * BN * 4 + 2 * (BN / 32) * RM * 4 : 0;
     static constexpr size_t bytes = 1024 + ring + barriers + epi + epi2;
@@ -150,7 +152,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
                      const float *__restrict__ bias, int64_t T, int d, int N, int tiles64,
                      int32_t *__restrict__ expert, float *__restrict__ gate, int32_t *__restrict__ hist,
                      int32_t *__restrict__ hist2, float *__restrict__ psum, float *__restrict__ probs,
-                     uint32_t *ticket, DeviceStatus *status) {
+                     float *__restrict__ ent, uint32_t *ticket, DeviceStatus *status) {
     using L = RouterLayout<BN, STAGES, TOP2>;
     constexpr int PM = 2 * RM;  // tokens per pair tile
     constexpr int G = RouterThreads<BN>::kGroups;
@@ -171,8 +173,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
     float *x_max = reinterpret_cast<float *>(hist_s + 4 * BN);       // [G column groups][RM]
     int32_t *x_arg = reinterpret_cast<int32_t *>(x_max + G * RM);    // [G][RM]
     float *x_sum = reinterpret_cast<float *>(x_arg + G * RM);        // [G][RM]
+    float *x_ent = x_sum + G * RM;                                   // [G][RM] sum of e (h - max), with ent
+    float *ent_q = x_ent + G * RM;                                   // [2 parity][4 quarters] entropy sums
     // top-2 only (inside epi2): second-choice counts and each group's second best
-    int32_t *hist2_s = reinterpret_cast<int32_t *>(x_sum + G * RM);  // [2 parity][2 halves][BN]
+    int32_t *hist2_s = reinterpret_cast<int32_t *>(ent_q + 8);       // [2 parity][2 halves][BN]
     float *x_max2 = reinterpret_cast<float *>(hist2_s + 4 * BN);     // [G][RM]
     int32_t *x_arg2 = reinterpret_cast<int32_t *>(x_max2 + G * RM);  // [G][RM]
 
@@ -405,20 +409,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
             // the gates by well under the 1e-5 parity bound; the full-precision
             // expf made this phase the longest of the epilogue
             float s4[4] = {0.f, 0.f, 0.f, 0.f};  // four interleaved partial sums, merged in fixed order
+            float sv = 0.f;                       // with ent: sum of e (h - max) over this group
 #pragma unroll
             for (int j = 0; j < CW; j += 4) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    h[j + u] = col0 + j + u < N ? __expf(h[j + u] - mx) : 0.f;
+                    const float z = h[j + u] - mx;
+                    h[j + u] = col0 + j + u < N ? __expf(z) : 0.f;
                     s4[u] += h[j + u];
+                    if (ent && col0 + j + u < N) sv += h[j + u] * z;
                 }
             }
             x_sum[grp * RM + tok] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            if (ent) x_ent[grp * RM + tok] = sv;
             named_barrier_epilogue<kEpiThreads>();
             float s_all = x_sum[tok];
 #pragma unroll
             for (int g = 1; g < G; ++g) s_all += x_sum[g * RM + tok];
             const float inv_s = 1.0f / s_all;
+            if (ent && grp == 0) {  // entropy -sum p ln p = ln s - sum e (h - max) / s; summed over the warp's tokens
+                float sv_all = x_ent[tok];
+#pragma unroll
+                for (int g = 1; g < G; ++g) sv_all += x_ent[g * RM + tok];
+                float hq = valid ? __logf(s_all) - sv_all * inv_s : 0.f;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) hq += __shfl_xor_sync(0xffffffffu, hq, off);
+                if (lane == 0) ent_q[par * 4 + q] = hq;
+            }
             float *psum_p = psum_w + par * 4 * BN;
             int32_t *hist_p = hist_s + par * 2 * BN;
             {
@@ -453,6 +470,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RouterThreads<BN>::k
 #pragma unroll
                 for (int h64 = 0; h64 < 2; ++h64) {
                     const int t64 = t64_0 + h64;
+                    if (ent && i == 0 && t64 < tiles64)
+                        ent[t64] = ent_q[par * 4 + 2 * h64] + ent_q[par * 4 + 2 * h64 + 1];
                     if (t64 < tiles64) {
                         hist[(int64_t)i * tiles64 + t64] = hist_p[h64 * BN + i];
                         psum[(int64_t)i * tiles64 + t64] = psum_p[(2 * h64) * BN + i] + psum_p[(2 * h64 + 1) * BN + i];
@@ -530,7 +549,7 @@ cudaError_t launch_bn(const switch_dims_t &dims, const __nv_bfloat16 *x, const f
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(device_sm_count() / 2, m_tiles));
     launch_begin(K_ROUTER_TC, stream);
     err = launch_kernel(kern, dim3(2 * pairs), dim3(RouterThreads<BN>::kAll), smem, stream, true, tx, tw, bias, T, d,
-                        N, (int)ws.tiles, expert, gate, ws.hist, ws.hist2, ws.psum, ws.probs, ws.ticket,
+                        N, (int)ws.tiles, expert, gate, ws.hist, ws.hist2, ws.psum, ws.probs, ws.ent, ws.ticket,
                         static_cast<DeviceStatus *>(ws.status));
     launch_end(stream);
     return err;

@@ -16,6 +16,7 @@ from pathlib import Path
 
 import numpy as np
 import scipy.special
+import scipy.stats
 
 GOLDEN = Path(__file__).resolve().parent / "golden"
 
@@ -527,6 +528,39 @@ def pin_top2_invariants(o):
         assert np.all(r["slot_token"][e][kept[e]:] == -1)
     both_dropped = (r["slot"] < 0).all(axis=1)
     assert np.all(r["y"][both_dropped] == 0.0)
+
+
+# --------------------------------------------------------------------------
+# Router statistics (the monitoring list)
+# --------------------------------------------------------------------------
+
+def pin_router_stats_16tok(o):
+    # The 16-token example: counts [7, 4, 3, 2] at capacity 4 drop 3 of 16 tokens, keep 13 of the
+    # 16 slots, and the busiest expert carries 7 / (16 / 4) = 1.75 times the uniform load.
+    g = golden("overflow_16tok.json")
+    counts = np.array(g["counts"], dtype=np.int32)
+    T, N = int(counts.sum()), len(counts)
+    st = o.router_stats(np.full((T, N), 1.0 / N), counts, g["capacity"])
+    assert st["drop_fraction"] == 3 / 16 and st["capacity_utilisation"] == 13 / 16
+    assert st["max_load"] == 1.75
+    assert abs(st["entropy"] - np.log(N)) < 1e-15  # uniform probabilities: ln N
+
+
+def pin_router_stats_entropy(o):
+    # Entropy against scipy's (natural log), one-hot rows give 0, and the statistics of a routed batch.
+    rng = np.random.default_rng(41)
+    p = scipy.special.softmax(rng.standard_normal((50, 6)) * 2, axis=1)
+    p[:3] = 0.0
+    p[0, 2] = p[1, 0] = p[2, 5] = 1.0
+    counts = np.array([20, 10, 9, 6, 3, 2], dtype=np.int32)
+    st = o.router_stats(p, counts, 8)
+    ref = scipy.stats.entropy(p, axis=1)
+    assert np.all(ref[:3] == 0.0)
+    assert abs(st["entropy"] - ref.mean()) < 1e-14
+    assert st["drop_fraction"] == (12 + 2 + 1) / 50
+    assert st["capacity_utilisation"] == (8 + 8 + 8 + 6 + 3 + 2) / 48
+    assert st["max_load"] == 20 * 6 / 50
+    assert o.router_stats(np.zeros((0, 6)), np.zeros(6, np.int32), 8)["entropy"] == 0.0
 
 
 # --------------------------------------------------------------------------

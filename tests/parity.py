@@ -173,3 +173,84 @@ def check_outputs_top2(y_gpu: np.ndarray, rows: np.ndarray, o: dict, rep: Report
         rep["y_max_abs_err"] = err
         rep["y_err_over_rms"] = err / rms if rms > 0 else 0.0
         assert err <= tol, f"max-abs output error {err:.4e} > {tol:.4e} (RMS {rms:.4e})"
+
+
+# ---------------------------------------------------------------------------
+# backward pass: per-element error bounds derived from the arithmetic
+# ---------------------------------------------------------------------------
+U_BF16 = 2.0 ** -8   # unit roundoff of bfloat16 (8 significant bits, round to nearest)
+U_F32 = 2.0 ** -24   # unit roundoff of float32
+EPS_P = 2.0 ** -18   # relative error of the float32 router probabilities and their sums
+
+
+def _f64(a):
+    return synth.bf16_bits_to_f32(a).astype(np.float64) if a.dtype == np.uint16 else a.astype(np.float64)
+
+
+def backward_error_bounds(inp: dict, C: int, dy: np.ndarray, g_aux: float, route: dict) -> dict:
+    """First-order bounds on |GPU - exact| for every gradient, from the rounding points of the
+    CUDA path: the hidden activations H, gate * dy and the pre-activation gradient dZ enter the
+    expert matmuls as bfloat16 (one rounding each, relative error <= u = 2^-8), every matmul
+    accumulates in float32 (K terms: <= K * 2^-24 relative to the sum of absolute products), and
+    the router's probabilities are float32 (relative error <= 2^-18).  For a dot product of a
+    rounded operand with an exact one the error is at most (u + K 2^-24) times the sum of
+    absolute products; the bounds below chain that through the backward's steps (magnitudes
+    computed in float64 from the inputs and the oracle's routing).  route: oracle route() with probs."""
+    x = _f64(inp["x"])
+    w_in, w_out = _f64(inp["w_in"]), _f64(inp["w_out"])
+    w_r = inp["w_r"].astype(np.float64)
+    T, d = x.shape
+    N, F, _ = w_in.shape
+    p, e_of, slot = route["probs"], route["expert"], route["slot"]
+    gate = p[np.arange(T), e_of]
+    dy = dy.astype(np.float64)
+    g_f, g_d, g_c, g_t, g_n = F * U_F32, d * U_F32, max(C, 1) * U_F32, T * U_F32, N * U_F32
+    b = dict(dx=np.zeros((T, d)), dw_in=np.zeros((N, F, d)), dw_out=np.zeros((N, d, F)))
+    err_g = np.zeros(T)                      # bound on the gate gradient's error
+    for e in range(N):
+        toks = np.flatnonzero((e_of == e) & (slot >= 0))
+        if toks.size == 0:
+            continue
+        xe = x[toks]
+        aw_in, aw_out = np.abs(w_in[e]), np.abs(w_out[e])
+        h = np.maximum(xe @ w_in[e].T, 0.0)
+        ho = h @ aw_out.T                              # |W_out| |H|: magnitude of o's terms
+        err_g[toks] = (U_BF16 + g_f) * (np.abs(dy[toks]) * ho).sum(1) + g_d * np.abs(dy[toks] * (h @ w_out[e].T)).sum(1)
+        de = np.abs(gate[toks, None] * dy[toks])
+        mask = (xe @ w_in[e].T) > 0
+        mz = (de @ aw_out) * mask                      # magnitude of dZ's terms
+        b["dx"][toks] += (2 * U_BF16 + 2 * g_f + 2 * g_d) * (mz @ aw_in)
+        b["dw_out"][e] = (2 * U_BF16 + g_c) * (de.T @ h)
+        b["dw_in"][e] = (2 * U_BF16 + 2 * g_d + g_c) * (mz.T @ np.abs(xe))
+    onehot = np.zeros((T, N))
+    onehot[np.arange(T), e_of] = 1.0
+    g_gate = np.zeros(T)
+    kept = slot >= 0
+    # exact gate gradients, for the magnitude of dp
+    for e in range(N):
+        toks = np.flatnonzero((e_of == e) & kept)
+        if toks.size:
+            o = np.maximum(x[toks] @ w_in[e].T, 0.0) @ w_out[e].T
+            g_gate[toks] = (dy[toks] * o).sum(1)
+    dp = g_aux * N * route["counts"][None, :] / T / T + onehot * g_gate[:, None]
+    dh = p * (dp - (p * dp).sum(1, keepdims=True))
+    err_dh = p * (onehot + gate[:, None]) * err_g[:, None] + \
+        EPS_P * (p * np.abs(dp) + p * (p * np.abs(dp)).sum(1, keepdims=True))
+    b["dx"] += err_dh @ np.abs(w_r) + g_n * (np.abs(dh) @ np.abs(w_r))
+    b["dw_r"] = err_dh.T @ np.abs(x) + g_t * (np.abs(dh).T @ np.abs(x))
+    b["dbias"] = err_dh.sum(0) + g_t * np.abs(dh).sum(0)
+    return b
+
+
+def check_within_bound(name: str, got: np.ndarray, ref: np.ndarray, bound: np.ndarray, report: dict,
+                       slack: float = 2.0) -> None:
+    """|got - ref| <= slack * bound + a float32 floor, element by element; report the worst ratio."""
+    floor = 4 * U_F32 * (np.abs(ref).max() if ref.size else 0.0) + 1e-30
+    err = np.abs(got - ref)
+    ratio = err / (slack * bound + floor)
+    worst = float(ratio.max()) if ratio.size else 0.0
+    report[name] = worst
+    if worst > 1.0:
+        i = np.unravel_index(int(np.argmax(ratio)), ratio.shape)
+        raise AssertionError(f"{name}: error {err[i]:.3e} at {i} exceeds {slack} x bound {bound[i]:.3e} "
+                             f"(got {got[i]:.6e}, exact {ref[i]:.6e})")

@@ -86,6 +86,11 @@ MUTANTS = {
                                         "router_part += dht[i] * w_r[(int64_t)k * N + i];"),
     "bwd_router_dx_missing": ("dx[t * (int64_t)d + k] += router_part;", "dx[t * (int64_t)d + k] += 0.0 * router_part;"),
     "bwd_gate_grad_uses_dy_only": ("gg += dy[t * (int64_t)d + k] * acc;", "gg += dy[t * (int64_t)d + k];"),
+    # router statistics: log base 2; overflow counted on every token; utilisation over T
+    "stats_entropy_log2": ("h -= p * log(p);", "h -= p * log2(p);"),
+    "stats_drop_no_clamp": ("dropped += c > C ? c - C : 0;", "dropped += c - C;"),
+    "stats_utilisation_over_T": ("out[2] = (double)kept / ((double)N * (double)C);",
+                                 "out[2] = (double)kept / (double)T;"),
     # bf16 loads: wrong half of the 32-bit pattern
     "bf16_wrong_shift": ("uint32_t wide = (uint32_t)bits << 16;", "uint32_t wide = (uint32_t)bits << 15;"),
 }
