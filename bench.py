@@ -256,10 +256,25 @@ def run_gpu(args):
     dist = init_dist(world, "nccl")
     wl = workload_of(args)
     # experts and router are shared by all ranks; every rank routes its own tokens
-    w_in_np, w_out_np = synth.all_expert_weights(wl)
     inp = dict(x=synth.activations(wl, seed=rank_seed(wl, rank)), w_r=synth.router_weight(wl),
-               bias=synth.router_bias(wl), w_in=w_in_np, w_out=w_out_np)
+               bias=synth.router_bias(wl))
     C = sm.switch_capacity(wl.T, wl.num_experts, wl.capacity_factor)
+    experts = None
+    if wl.zipf_s is not None:
+        # Skewed routing sends every token to a few experts: draw the weights of the experts
+        # that receive tokens (found by routing on the GPU) and leave the others zero.  The
+        # layer never reads an expert without kept tokens, so the timed work is the same.
+        r = sm.route(to_dev(inp["x"], device), to_dev(inp["w_r"], device), capacity=C,
+                     logit_bias=to_dev(inp["bias"], device), d_ff=wl.d_ff)
+        experts = np.flatnonzero(r["counts"].cpu().numpy() > 0)
+        if world > 1:  # every rank holds the same experts: the union over ranks
+            import torch.distributed as tdist
+            mask = torch.zeros(wl.num_experts, dtype=torch.int32, device=device)
+            mask[torch.from_numpy(experts).to(device)] = 1
+            tdist.all_reduce(mask, op=tdist.ReduceOp.MAX)
+            experts = np.flatnonzero(mask.cpu().numpy() > 0)
+        del r
+    inp["w_in"], inp["w_out"] = synth.all_expert_weights(wl, experts=experts)
 
     x = to_dev(inp["x"], device)
     w_r = to_dev(inp["w_r"], device)
