@@ -23,6 +23,7 @@ The JSON line also carries:
   e2e           the same metric through the public API with pinned host
                 buffers: x copied in and y/aux/counts copied out every step
   top2          the top-2 variant (switch_layer_fwd_top2) on the same tensors
+  backward      a training step (training forward + switch_layer_bwd) on the same tensors
   entry_points  switch_dispatch and switch_combine called on their own
   sweep         the large-expert layer at every capacity factor of its sweep
                 (drop fraction and tokens/s per c)
@@ -400,6 +401,10 @@ def run_gpu(args):
     top2 = time_top2(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, device) \
         if (world == 1 and not args.no_top2 and wl.num_experts >= 2) else None
 
+    # the backward pass (training forward + switch_layer_bwd) on the same tokens and weights
+    backward = time_backward(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, device) \
+        if (world == 1 and not args.no_backward and wl.dtype == synth.BF16) else None
+
     # standalone dispatch and combine entry points on the same workload
     entry_points = time_entry_points(sm, wl, x, w_r, bias, C, flush, stream, device) if world == 1 else None
 
@@ -431,6 +436,8 @@ def run_gpu(args):
         }
         if top2:
             result["top2"] = top2
+        if backward:
+            result["backward"] = backward
         if entry_points:
             result["entry_points"] = entry_points
         if sweep:
@@ -505,6 +512,72 @@ def time_top2(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, device)
               "capacity": C, "kept_assignments": K, "dropped_assignments": int(2 * T - K),
               "expert_flops_per_step": 4.0 * K * d * F, "kernels": kernels}
     del out, ws
+    torch.cuda.empty_cache()
+    return result
+
+
+def time_backward(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, device):
+    """A training step of the layer: the training forward (SWITCH_FLAG_TRAINING) and
+    switch_layer_bwd with a fixed upstream gradient, timed together and per kernel."""
+    import torch
+    T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.num_experts
+    dy = torch.randn(T, d, device=device, generator=torch.Generator(device).manual_seed(7))
+    fwd = sm.layer_fwd(x, w_r, w_in, w_out, capacity=C, logit_bias=bias, flags=sm.SWITCH_FLAG_TRAINING)
+    grads = sm.layer_bwd(fwd, x, w_r, w_in, w_out, dy, 0.01, logit_bias=bias)
+
+    def step():
+        sm.layer_fwd(x, w_r, w_in, w_out, capacity=C, logit_bias=bias, flags=sm.SWITCH_FLAG_TRAINING,
+                     ws=fwd["workspace"], out=fwd)
+        d_ = sm.layer_dims(x, w_in, capacity=C, flags=sm.SWITCH_FLAG_TRAINING)
+        sm.switch_layer_bwd(d_, x, w_r, w_in, w_out, fwd["expert"], fwd["gate"], fwd["slot"], fwd["counts"], dy,
+                            0.01, grads["dx"], grads["dw_r"], grads["dbias"], grads["dw_in"], grads["dw_out"],
+                            fwd["workspace"])
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    ms = _time_events(step, flush, stream, steps)
+    sm.trace_start(steps * 32)
+    _time_events(step, flush, stream, steps)
+    trace = sm.trace_read(steps * 32)
+    sm.trace_stop()
+    if sm.switch_check(fwd["workspace"]) != 0:
+        raise RuntimeError("device status after the backward steps")
+    K = int(np.minimum(fwd["counts"].cpu().numpy(), C).sum())
+    s = x.element_size()
+    Cp = -(-C // 64) * 64
+    per_kernel: dict[str, list[float]] = {}
+    for name, kms in trace:
+        per_kernel.setdefault(name, []).append(kms)
+    transposes = 2 * (2 * N * d * F * s + N * Cp * (2 * d + 2 * F) * s)  # bytes of the six transposes per step
+    work = {
+        "bwd_gate_softmax": ("hbm", 4 * T * d + 4 * K * d + 2 * K * d + 8 * T * N, None),
+        "bwd_tc_gemm_dz": ("tensor", 2.0 * K * d * F, None),
+        "bwd_tc_gemm_dx": ("tensor", 2.0 * K * F * d, None),
+        "bwd_tc_gemm_dw": ("tensor", 2.0 * K * d * F, None),
+        "bwd_router_dx": ("alu", 2.0 * T * N * d, None),
+        "bwd_router_dw": ("alu", 2.0 * T * N * d, None),
+        "ffn_tc_gemm1_relu": ("tensor", 2.0 * K * d * F, None),
+        "ffn_tc_gemm2": ("tensor", 2.0 * K * F * d, None),
+    }
+    peaks, _ = load_peaks()
+    kernels = {}
+    for name, times in per_kernel.items():
+        n_per_step = len(times) // steps
+        if name == "bwd_transpose":
+            kernels[name] = kernel_entry("hbm", transposes / max(n_per_step, 1), None, statistics.mean(times),
+                                         n_per_step, peaks)
+            continue
+        kind, amount, amount_act = work.get(name, ("?", 0, None))
+        kernels[name] = kernel_entry(kind, amount, amount_act, statistics.mean(times), n_per_step, peaks)
+    tot = sum(k["avg_ms"] * k["launches"] for k in kernels.values())
+    for k in kernels.values():
+        k["share"] = round(k["avg_ms"] * k["launches"] / tot, 4) if tot else None
+    result = {"ms_per_step": round(ms, 5), "value": round(T / (ms * 1e-3), 1), "unit": UNIT,
+              "what": "training forward (SWITCH_FLAG_TRAINING) + switch_layer_bwd per step", "steps": steps,
+              "kept_tokens": K, "expert_flops_per_step": 12.0 * K * d * F, "kernels": kernels}
+    del fwd, grads, dy
     torch.cuda.empty_cache()
     return result
 
@@ -806,6 +879,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-top2", action="store_true", help="skip timing the top-2 variant of the layer")
+    ap.add_argument("--no-backward", action="store_true", help="skip timing the backward pass")
     ap.add_argument("--no-sweep", action="store_true",
                     help=f"skip the capacity-factor sweep of the {SWEEP_WORKLOAD} workload")
     args = ap.parse_args(argv)
