@@ -440,3 +440,40 @@ def test_uninitialised_workspace_reports_ok(entry):
         ybuf = torch.zeros(wl.num_experts * C * wl.d_model, dtype=torch.float32, device="cuda")
         sm.switch_expert_ffn(d, xbuf, dev["w_in"], dev["w_out"], counts, ybuf, ws)
     assert sm.switch_check(ws) == 0
+
+
+@pytest.mark.parametrize("d,dt", [(768, torch.bfloat16), (1024, torch.bfloat16), (4096, torch.bfloat16),
+                                  (8192, torch.bfloat16), (96, torch.float32), (33, torch.float32)],
+                         ids=["bf16-768", "bf16-1024", "bf16-4096", "bf16-8192", "f32-96", "f32-33"])
+def test_dispatch_and_combine_match_gathers(d, dt):
+    """switch_dispatch and switch_combine on their own, bit for bit against torch gathers: xbuf rows
+    are copies of x rows; y = gate * ybuf[expert, slot] (one float32 multiply), zero rows for dropped
+    tokens.  Short rows move through shared memory by bulk copies, long ones (and rows that are not a
+    multiple of 16 bytes) through vector loads and stores."""
+    T, N = 3000, 6
+    g = torch.Generator("cuda").manual_seed(d)
+    C = 300  # ~500 tokens per expert: about 40 % dropped
+    x = torch.randn(T, d, device="cuda", generator=g).to(dt)
+    w_r = torch.randn(N, d, device="cuda", generator=g) * 0.01
+    r = sm.route(x, w_r, capacity=C, d_ff=64)
+    assert sm.switch_check(r["workspace"]) == 0
+    dims = sm.dims(T, d, 64, N, C, dt)
+    xbuf = torch.full((N * C, d), 7, dtype=dt, device="cuda")
+    sm.switch_dispatch(dims, x, r["slot_token"], r["counts"], xbuf)
+    st = r["slot_token"].view(N, C)
+    kept = torch.clamp(r["counts"], max=C)
+    for e in range(N):
+        k = int(kept[e])
+        rows = xbuf.view(N, C, d)[e]
+        assert torch.equal(rows[:k], x[st[e, :k].long()]), e
+        assert torch.all(rows[k:] == 7)  # slots past the kept count are not written
+    ybuf = torch.randn(N * C, d, device="cuda", generator=g)
+    y = torch.full((T, d), 5.0, device="cuda")
+    sm.switch_combine(dims, ybuf, r["expert"], r["slot"], r["gate"], y)
+    torch.cuda.synchronize()
+    keep = r["slot"] >= 0
+    assert int((~keep).sum()) > 0
+    idx = (r["expert"].long() * C + r["slot"].long().clamp(min=0))
+    ref = r["gate"][:, None] * ybuf[idx]
+    assert torch.equal(y[keep].view(torch.int32), ref[keep].view(torch.int32))
+    assert torch.all(y[~keep] == 0)
