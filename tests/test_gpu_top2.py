@@ -134,14 +134,20 @@ def test_top2_first_choices_are_top1_routing(orc):
 
 
 def test_top2_entry_points_compose_to_layer():
-    """route_top2 -> dispatch -> expert_ffn -> combine_top2 gives the same bytes as layer_fwd_top2."""
+    """route_top2 -> dispatch -> expert_ffn -> combine_top2 gives the same bytes as layer_fwd_top2 with
+    the two expert GEMMs launched one after the other, and agrees with the default layer_fwd_top2
+    (one persistent launch, which may split its second GEMM over d_ff) to float32 rounding."""
     wl = synth.WORKLOADS["base8"]
     T = 2000
     C = sm.switch_capacity(T, wl.num_experts, 2.0)
     inp = synth.inputs(wl, T=T)
     dev = {k: to_device(v) for k, v in inp.items()}
-    ref = sm.layer_fwd_top2(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C)
-    assert sm.switch_check(ref["workspace"]) == 0
+    ref = sm.layer_fwd_top2(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C,
+                            flags=sm.SWITCH_FLAG_FFN_TWO_LAUNCHES)
+    fused = sm.layer_fwd_top2(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C)
+    assert sm.switch_check(ref["workspace"]) == 0 and sm.switch_check(fused["workspace"]) == 0
+    rms = float(ref["y"].double().pow(2).mean().sqrt())
+    assert float((fused["y"].double() - ref["y"].double()).abs().max()) <= 1e-4 * rms
     d = sm.layer_dims(dev["x"], dev["w_in"], capacity=C)
     ws = sm.workspace(d, "cuda")
     N, dm = wl.num_experts, wl.d_model
