@@ -102,7 +102,11 @@ enum {
     /* The routing step also sums the entropy of every token's router
      * distribution per 64-token tile into the workspace, for
      * switch_router_stats. */
-    SWITCH_FLAG_ROUTER_STATS = 64
+    SWITCH_FLAG_ROUTER_STATS = 64,
+    /* In switch_layer_fwd, run the layer as its separate kernels even where
+     * the single-block path for small float32 layers (T <= 256, N <= 32,
+     * inputs and weights within 160 KB of shared memory) would apply. */
+    SWITCH_FLAG_MULTI_KERNEL = 128
 };
 
 typedef struct {

@@ -84,60 +84,68 @@ __global__ void __launch_bounds__(kThreads) bwd_token_kernel(const float *__rest
 
 // Batched transpose of bf16 matrices: in [B][R][Cc] -> out [B][Cc][Rp].
 // Rows r >= valid(b) of the input (valid = min(counts[b], cap) when counts is
-// given, else R) and the padding rows up to Rp become zeros.  64 x 64 tiles,
-// 32-bit (two-element) accesses on both sides.
+// given, else R) and the padding rows up to Rp become zeros.  64 x 64 tiles
+// through shared memory (rows padded to 33 words), 16-byte global loads and
+// stores on both sides; Cc and Rp are multiples of 8 (checked by the launcher).
 constexpr int kTT = 64;
 __global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t *__restrict__ in, uint16_t *__restrict__ out,
                                                             int R, int Cc, int Rp, const int32_t *__restrict__ counts,
                                                             int cap) {
-    __shared__ uint16_t tile[kTT][kTT + 2];
+    __shared__ uint32_t tile[kTT][kTT / 2 + 1];  // [row][column pair]
     const int b = blockIdx.z;
     const int c0 = blockIdx.x * kTT, r0 = blockIdx.y * kTT;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    const int tid = threadIdx.x;
     const int valid = counts ? min(min(counts[b], cap), R) : R;
     const uint16_t *src = in + (int64_t)b * R * Cc;
     uint16_t *dst = out + (int64_t)b * Cc * Rp;
 #pragma unroll
-    for (int j = 0; j < kTT / 8; ++j) {
-        const int r = r0 + ty + 8 * j;
-        const int c = c0 + 2 * tx;
-        uint32_t v = 0u;
-        if (r < valid && c + 1 < Cc) v = *reinterpret_cast<const uint32_t *>(src + (int64_t)r * Cc + c);
-        else if (r < valid && c < Cc) v = src[(int64_t)r * Cc + c];
-        tile[ty + 8 * j][2 * tx] = (uint16_t)(v & 0xffffu);
-        tile[ty + 8 * j][2 * tx + 1] = (uint16_t)(v >> 16);
+    for (int j = 0; j < 2; ++j) {  // 64 rows x 8 chunks of 8 elements
+        const int idx = tid + 256 * j;
+        const int r = idx >> 3, ch = idx & 7;
+        const int c = c0 + ch * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r0 + r < valid && c < Cc) v = __ldg(reinterpret_cast<const uint4 *>(src + (int64_t)(r0 + r) * Cc + c));
+        tile[r][ch * 4 + 0] = v.x;
+        tile[r][ch * 4 + 1] = v.y;
+        tile[r][ch * 4 + 2] = v.z;
+        tile[r][ch * 4 + 3] = v.w;
     }
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < kTT / 8; ++j) {
-        const int c = c0 + ty + 8 * j;  // output row
-        const int r = r0 + 2 * tx;      // output columns r, r + 1
-        if (c < Cc && r + 1 < Rp) {
-            const uint32_t v = (uint32_t)tile[2 * tx][ty + 8 * j] | ((uint32_t)tile[2 * tx + 1][ty + 8 * j] << 16);
-            *reinterpret_cast<uint32_t *>(dst + (int64_t)c * Rp + r) = v;
-        } else if (c < Cc && r < Rp) {
-            dst[(int64_t)c * Rp + r] = tile[2 * tx][ty + 8 * j];
+    for (int j = 0; j < 2; ++j) {  // 64 output rows x 8 chunks of 8 input rows
+        const int idx = tid + 256 * j;
+        const int c = idx >> 3, rb = idx & 7;
+        if (c0 + c >= Cc || r0 + rb * 8 >= Rp) continue;
+        const int shift = (c & 1) * 16;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t lo = (tile[rb * 8 + 2 * q][c >> 1] >> shift) & 0xffffu;
+            const uint32_t hi = (tile[rb * 8 + 2 * q + 1][c >> 1] >> shift) & 0xffffu;
+            w[q] = lo | (hi << 16);
         }
+        *reinterpret_cast<uint4 *>(dst + (int64_t)(c0 + c) * Rp + r0 + rb * 8) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
 // dx[t, :] = sum_i dh[t, i] W_r[i, :]  (overwrites dx; the expert part is
-// added afterwards).  Block: 32 tokens x 128 columns; thread: 4 tokens x 4
-// columns; experts in chunks of 32 through shared memory.
-constexpr int kDxTok = 32, kDxCol = 128, kDxI = 32;
+// added afterwards).  Block: 64 tokens x 128 columns; thread: 8 tokens x 4
+// columns; experts in chunks of 32 through shared memory, dh stored
+// expert-major so that a thread's 8 tokens are two 16-byte reads.
+constexpr int kDxTok = 64, kDxCol = 128, kDxI = 32, kDxPitch = kDxTok + 8;
 __global__ void __launch_bounds__(256) router_dx_kernel(const float *__restrict__ dh, const float *__restrict__ w_r,
                                                        int64_t T, int N, int d, float *__restrict__ dx) {
-    __shared__ float s_dh[kDxI][kDxTok + 1];
+    __shared__ __align__(16) float s_dh[kDxI][kDxPitch];  // [expert][token]
     __shared__ __align__(16) float s_w[kDxI][kDxCol];
     const int64_t t0 = (int64_t)blockIdx.y * kDxTok;
     const int k0 = blockIdx.x * kDxCol;
     const int tid = threadIdx.x;
     const int tc = tid & 31;   // columns k0 + 4 tc .. + 3
-    const int tt = tid >> 5;   // tokens t0 + tt + 8 j, j < 4
-    float acc[4][4] = {};
+    const int tt = tid >> 5;   // tokens t0 + 8 tt .. + 7
+    float acc[8][4] = {};
     for (int i0 = 0; i0 < N; i0 += kDxI) {
         __syncthreads();
-        for (int q = tid; q < kDxI * kDxTok; q += 256) {
+        for (int q = tid; q < kDxI * kDxTok; q += 256) {  // coalesced along the experts of a token
             const int ii = q % kDxI, tl = q / kDxI;
             const int64_t t = t0 + tl;
             s_dh[ii][tl] = (t < T && i0 + ii < N) ? dh[t * N + i0 + ii] : 0.f;
@@ -147,22 +155,24 @@ __global__ void __launch_bounds__(256) router_dx_kernel(const float *__restrict_
             s_w[ii][kk] = (i0 + ii < N && k0 + kk < d) ? w_r[(int64_t)(i0 + ii) * d + k0 + kk] : 0.f;
         }
         __syncthreads();
-#pragma unroll 8
+#pragma unroll 4
         for (int ii = 0; ii < kDxI; ++ii) {
             const float4 w = *reinterpret_cast<const float4 *>(&s_w[ii][4 * tc]);
+            const float4 a0 = *reinterpret_cast<const float4 *>(&s_dh[ii][8 * tt]);
+            const float4 a1 = *reinterpret_cast<const float4 *>(&s_dh[ii][8 * tt + 4]);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float a = s_dh[ii][tt + 8 * j];
-                acc[j][0] = fmaf(a, w.x, acc[j][0]);
-                acc[j][1] = fmaf(a, w.y, acc[j][1]);
-                acc[j][2] = fmaf(a, w.z, acc[j][2]);
-                acc[j][3] = fmaf(a, w.w, acc[j][3]);
+            for (int j = 0; j < 8; ++j) {
+                acc[j][0] = fmaf(a[j], w.x, acc[j][0]);
+                acc[j][1] = fmaf(a[j], w.y, acc[j][1]);
+                acc[j][2] = fmaf(a[j], w.z, acc[j][2]);
+                acc[j][3] = fmaf(a[j], w.w, acc[j][3]);
             }
         }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int64_t t = t0 + tt + 8 * j;
+    for (int j = 0; j < 8; ++j) {
+        const int64_t t = t0 + 8 * tt + j;
         const int k = k0 + 4 * tc;
         if (t < T && k < d)  // d % 64 == 0 on this path: the four columns are in range together
             *reinterpret_cast<float4 *>(dx + t * d + k) = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
@@ -171,12 +181,13 @@ __global__ void __launch_bounds__(256) router_dx_kernel(const float *__restrict_
 
 // Partial sums of dW_r and d bias over chunks of tokens:
 //   part_w[chunk][i][k] = sum_{t in chunk} dh[t, i] x[t, k],  part_b[chunk][i] = sum dh[t, i]
-// Block: 64 experts x 128 columns of one chunk; thread: 4 experts x 8 columns.
-constexpr int kDwI = 64, kDwCol = 128, kDwTok = 32;
+// Block: 64 experts x 128 columns of one chunk; thread: 4 consecutive experts x
+// 8 columns (three 16-byte shared-memory reads per 32 FMAs).
+constexpr int kDwI = 64, kDwCol = 128, kDwTok = 32, kDwPitch = kDwI + 4;
 __global__ void __launch_bounds__(256) router_dw_kernel(const float *__restrict__ dh, const uint16_t *__restrict__ x,
                                                        int64_t T, int N, int d, int64_t chunk_tokens,
                                                        float *__restrict__ part_w, float *__restrict__ part_b) {
-    __shared__ float s_dh[kDwTok][kDwI + 1];
+    __shared__ __align__(16) float s_dh[kDwTok][kDwPitch];  // [token][expert]
     __shared__ __align__(16) float s_x[kDwTok][kDwCol];
     const int k0 = blockIdx.x * kDwCol, i0 = blockIdx.y * kDwI;
     const int chunk = blockIdx.z;
@@ -184,9 +195,9 @@ __global__ void __launch_bounds__(256) router_dw_kernel(const float *__restrict_
     const int64_t tend = min(T, tbeg + chunk_tokens);
     const int tid = threadIdx.x;
     const int tk = tid & 15;   // columns k0 + 8 tk .. + 7
-    const int ti = tid >> 4;   // experts i0 + ti + 16 j, j < 4
+    const int ti = tid >> 4;   // experts i0 + 4 ti .. + 3
     float acc[4][8] = {};
-    float accb4[4] = {0.f, 0.f, 0.f, 0.f};  // threads with tk == 0: d bias of experts i0 + ti + 16 j
+    float accb[4] = {0.f, 0.f, 0.f, 0.f};  // threads with tk == 0: d bias of their four experts
     for (int64_t tb = tbeg; tb < tend; tb += kDwTok) {
         __syncthreads();
         for (int q = tid; q < kDwTok * kDwI; q += 256) {
@@ -207,27 +218,28 @@ __global__ void __launch_bounds__(256) router_dw_kernel(const float *__restrict_
         for (int tl = 0; tl < kDwTok; ++tl) {
             const float4 xa = *reinterpret_cast<const float4 *>(&s_x[tl][8 * tk]);
             const float4 xb = *reinterpret_cast<const float4 *>(&s_x[tl][8 * tk + 4]);
+            const float4 h4 = *reinterpret_cast<const float4 *>(&s_dh[tl][4 * ti]);
             const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+            const float hv[4] = {h4.x, h4.y, h4.z, h4.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const float a = s_dh[tl][ti + 16 * j];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) acc[j][c] = fmaf(a, xv[c], acc[j][c]);
-                if (tk == 0) accb4[j] += a;
+                for (int c = 0; c < 8; ++c) acc[j][c] = fmaf(hv[j], xv[c], acc[j][c]);
+                if (tk == 0) accb[j] += hv[j];
             }
         }
     }
     float *pw = part_w + (int64_t)chunk * N * d;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const int i = i0 + ti + 16 * j;
+        const int i = i0 + 4 * ti + j;
         const int k = k0 + 8 * tk;
         if (i < N && k < d) {
             float4 *dst = reinterpret_cast<float4 *>(pw + (int64_t)i * d + k);
             dst[0] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
             dst[1] = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
         }
-        if (tk == 0 && blockIdx.x == 0 && i < N) part_b[(int64_t)chunk * N + i] = accb4[j];
+        if (tk == 0 && blockIdx.x == 0 && i < N) part_b[(int64_t)chunk * N + i] = accb[j];
     }
 }
 
@@ -244,6 +256,7 @@ int64_t round_up64(int64_t v) { return (v + 63) / 64 * 64; }
 
 cudaError_t launch_transpose(int32_t kernel_id, const void *in, void *out, int B, int R, int Cc, int Rp,
                              const int32_t *counts, int cap, cudaStream_t stream) {
+    if (Cc % 8 != 0 || Rp % 8 != 0) return cudaErrorInvalidValue;  // 16-byte rows on both sides
     const dim3 grid((unsigned)((Cc + kTT - 1) / kTT), (unsigned)((Rp + kTT - 1) / kTT), (unsigned)B);
     launch_begin(kernel_id, stream);
     transpose_bf16_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(in), static_cast<uint16_t *>(out),

@@ -334,7 +334,9 @@ switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const
     const bool tensor_cores = dims->dtype == SWITCH_BF16 && !(dims->flags & SWITCH_FLAG_SIMT_FFN);
     const bool rows16 = ((int64_t)dims->d_model * (int64_t)elem_size(*dims)) % 16 == 0;
     cudaError_t err;
-    if (dims->flags & SWITCH_FLAG_TRAINING) {
+    if (small_layer_supported(*dims)) {
+        err = launch_small_layer(*dims, x, w_r, logit_bias, w_in, w_out, yf, expert, gate, slot, counts, aux, ws, st);
+    } else if (dims->flags & SWITCH_FLAG_TRAINING) {
         // training forward: keeps the router probabilities, xbuf, H and the ungated
         // expert output ybuf in the workspace for switch_layer_bwd
         if (!tensor_cores) return SWITCH_ERR_UNSUPPORTED;
@@ -581,6 +583,7 @@ const char *switch_kernel_name(int32_t id) {
         case K_BWD_ROUTER_DW: return "bwd_router_dw";
         case K_BWD_REDUCE: return "bwd_reduce";
         case K_ROUTER_STATS: return "router_stats";
+        case K_SMALL_LAYER: return "small_layer";
     }
     return "?";
 }

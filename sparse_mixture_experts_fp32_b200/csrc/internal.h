@@ -42,6 +42,7 @@ enum KernelId : int32_t {
     K_BWD_ROUTER_DW = 25,
     K_BWD_REDUCE = 26,
     K_ROUTER_STATS = 27,
+    K_SMALL_LAYER = 28,
 };
 
 struct Workspace {
@@ -127,6 +128,12 @@ cudaError_t launch_ffn_simt(const switch_dims_t &dims, const void *xbuf, const v
 cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
                           const int32_t *counts, void *ybuf, const int32_t *slot_token, const float *gate, float *y,
                           const Workspace &ws, cudaStream_t stream);
+
+// The whole layer in one block for small float32 layers (switch_layer_fwd's default there).
+bool small_layer_supported(const switch_dims_t &dims);
+cudaError_t launch_small_layer(const switch_dims_t &dims, const void *x, const float *w_r, const float *bias,
+                               const void *w_in, const void *w_out, float *y, int32_t *expert, float *gate,
+                               int32_t *slot, int32_t *counts, float *aux, const Workspace &ws, cudaStream_t stream);
 
 // Router statistics from the per-tile entropy sums a routing call left in the workspace.
 cudaError_t launch_router_stats(const switch_dims_t &dims, const int32_t *counts, const Workspace &ws, float *stats,

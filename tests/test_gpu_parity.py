@@ -477,3 +477,61 @@ def test_dispatch_and_combine_match_gathers(d, dt):
     ref = r["gate"][:, None] * ybuf[idx]
     assert torch.equal(y[keep].view(torch.int32), ref[keep].view(torch.int32))
     assert torch.all(y[~keep] == 0)
+
+
+def test_full_size_large128_every_row(orc, record_property):
+    """The Switch-Large-shaped workload at full size, every output row against the oracle (fp64 on the
+    host cores, about a minute), and the near-tie tokens bounded: with router logits of spread ~0.1
+    about 60 tokens of 131072 have a top-2 margin under 1e-5; any flip must be one of them."""
+    wl = synth.WORKLOADS["large128"]
+    x, w_r = synth.activations(wl), synth.router_weight(wl)
+    T, N = x.shape[0], wl.num_experts
+    C = sm.switch_capacity(T, N, wl.capacity_factor)
+    o = orc.route(x, w_r, None, capacity=C, want_probs=True)
+    w_in, w_out = synth.all_expert_weights(wl)
+    out = sm.layer_fwd(to_device(x), to_device(w_r), to_device(w_in), to_device(w_out), capacity=C)
+    assert sm.switch_check(out["workspace"]) == 0
+    g = {k: out[k].cpu().numpy() for k in ("expert", "gate", "slot", "counts", "aux")}
+    g["aux"] = g["aux"][0]
+    rep = check_routing(o, g, orc, N, C, T, check_slot_token=False)
+    assert rep["near_ties"] <= 400, rep["near_ties"]
+    y = y_to_numpy(out["y"])
+    del out
+    torch.cuda.empty_cache()
+    check_outputs(y, np.arange(T, dtype=np.int64), o, rep, orc, x, w_in, w_out, g["expert"], False)
+    record_property("report", {k: rep.get(k) for k in ("near_ties", "flips", "drops", "aux_rel_err",
+                                                       "y_err_over_rms")})
+
+
+@pytest.mark.parametrize("name,T", [("tiny_fp32", 64), ("tiny_fp32", 256)])
+def test_small_float32_layer_single_launch(orc, name, T):
+    """Small float32 layers run as one kernel: same routing, counts and aux as the multi-kernel
+    path, outputs equal to float32 rounding, both within the float32 bar of the oracle."""
+    wl = synth.WORKLOADS[name]
+    C = synth_capacity(wl, T)
+    inp = synth.inputs(wl, T=T)
+    dev = {k: to_device(v) for k, v in inp.items()}
+    sm.trace_start(16)
+    a = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C)
+    torch.cuda.synchronize()
+    names = [n for n, _ in sm.trace_read()]
+    sm.trace_stop()
+    assert names == ["small_layer"]
+    b = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, flags=sm.SWITCH_FLAG_MULTI_KERNEL)
+    assert sm.switch_check(a["workspace"]) == 0 and sm.switch_check(b["workspace"]) == 0
+    for k in ("expert", "slot", "counts"):
+        assert torch.equal(a[k], b[k]), k
+    assert float((a["gate"] - b["gate"]).abs().max()) <= 1e-6
+    assert abs(float(a["aux"][0]) - float(b["aux"][0])) <= 1e-6 * abs(float(b["aux"][0]))
+    rms = float(b["y"].double().pow(2).mean().sqrt())
+    assert float((a["y"].double() - b["y"].double()).abs().max()) <= 1e-5 * rms
+    full_check(orc, wl, T, flags=sm.SWITCH_FLAG_MULTI_KERNEL)
+
+
+def test_small_path_odd_float32_shapes_multi_kernel(orc):
+    # the multi-kernel float32 path on odd shapes (the default there is the single-block path)
+    inp = _random_inputs(np.random.default_rng(zlib.crc32(b"f32_odd_multi")), 77, 33, 17, 3, "f32")
+    g, y, _ = run_layer(inp, 30, flags=sm.SWITCH_FLAG_MULTI_KERNEL)
+    o = oracle_route(orc, inp, 30)
+    rep = check_routing(o, g, orc, 3, 30, 77, check_slot_token=False)
+    check_outputs(y, np.arange(77), o, rep, orc, inp["x"], inp["w_in"], inp["w_out"], g["expert"], True)
