@@ -190,6 +190,9 @@ def kernel_work(wl, C, counts):
         "router_tiled": ("hbm", router_bytes, None),
         "router_staged": ("hbm", router_bytes, None),
         "router_tc": ("hbm", T * d * s + 3 * N * d * 2 + 8 * T + 8 * N * tiles, None),
+        # the same kernel against its tensor-core work: three exact bf16 terms of W_r per token, the
+        # experts padded to the tile width (64 or 128)
+        "router_tc/tensor": ("tensor", 6.0 * T * d * (64 if N <= 64 else 128), None),
         "router_weight_split": ("hbm", N * d * 4 + 3 * N * d * 2, None),
         "capacity_scan": ("hbm", 8 * N * tiles + 4 * N * tiles + 12 * N, None),
         "slot_assign_scatter": ("hbm", assign_common + (T - K) * d * 4, assign_common + (T - K) * d * s),
@@ -374,6 +377,11 @@ def run_gpu(args):
     for name, times in per_kernel.items():
         kind, amount, amount_act = work.get(name, ("?", 0, None))
         kernels[name] = kernel_entry(kind, amount, amount_act, statistics.mean(times), len(times), peaks)
+        if name + "/tensor" in work:  # a second roofline for the same kernel
+            t_kind, t_amount, _ = work[name + "/tensor"]
+            t = kernel_entry(t_kind, t_amount, None, statistics.mean(times), len(times), peaks)
+            kernels[name]["tensor_achieved_tflops"] = t["achieved"]
+            kernels[name]["frac_tensor"] = t["frac"]
     tot = sum(k["avg_ms"] * k["launches"] for k in kernels.values())
     for k in kernels.values():
         k["share"] = round(k["avg_ms"] * k["launches"] / tot, 4) if tot else None

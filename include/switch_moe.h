@@ -106,7 +106,11 @@ enum {
     /* In switch_layer_fwd, run the layer as its separate kernels even where
      * the single-block path for small float32 layers (T <= 256, N <= 32,
      * inputs and weights within 160 KB of shared memory) would apply. */
-    SWITCH_FLAG_MULTI_KERNEL = 128
+    SWITCH_FLAG_MULTI_KERNEL = 128,
+    /* switch_dispatch and switch_combine move rows of up to ~6 KB through
+     * shared memory by bulk copies (the TMA engine) instead of vector loads
+     * and stores; the results are identical. */
+    SWITCH_FLAG_STAGED_MOVES = 256
 };
 
 typedef struct {

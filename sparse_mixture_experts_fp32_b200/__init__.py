@@ -34,6 +34,7 @@ SWITCH_FLAG_SEPARATE_SCAN = 16
 SWITCH_FLAG_TRAINING = 32
 SWITCH_FLAG_ROUTER_STATS = 64
 SWITCH_FLAG_MULTI_KERNEL = 128
+SWITCH_FLAG_STAGED_MOVES = 256
 
 STATUS = {
     0: "SWITCH_OK", 1: "SWITCH_ERR_NULL", 2: "SWITCH_ERR_SHAPE", 3: "SWITCH_ERR_DTYPE", 4: "SWITCH_ERR_ALIGN",

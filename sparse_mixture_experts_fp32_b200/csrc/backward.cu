@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(256) router_dw_kernel(const float *__restrict_
     const int tk = tid & 15;   // columns k0 + 8 tk .. + 7
     const int ti = tid >> 4;   // experts i0 + 4 ti .. + 3
     float acc[4][8] = {};
-    float accb[4] = {0.f, 0.f, 0.f, 0.f};  // threads with tk == 0: d bias of their four experts
+    float accb[4] = {0.f, 0.f, 0.f, 0.f};  // d bias of the thread's four experts (written by tk == 0)
     for (int64_t tb = tbeg; tb < tend; tb += kDwTok) {
         __syncthreads();
         for (int q = tid; q < kDwTok * kDwI; q += 256) {
@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(256) router_dw_kernel(const float *__restrict_
             for (int j = 0; j < 4; ++j) {
 #pragma unroll
                 for (int c = 0; c < 8; ++c) acc[j][c] = fmaf(hv[j], xv[c], acc[j][c]);
-                if (tk == 0) accb[j] += hv[j];
+                accb[j] += hv[j];  // every thread: no divergent branch in the inner loop
             }
         }
     }

@@ -422,12 +422,12 @@ switch_status_t switch_layer_fwd_top2(const switch_dims_t *dims, const void *x, 
     // the expert GEMMs see up to 2T kept rows (their grid is sized from that bound)
     switch_dims_t rows = *dims;
     rows.T = 2 * dims->T;
-    const bool fused = tensor_cores && !(dims->flags & (SWITCH_FLAG_GEMM_1CTA | SWITCH_FLAG_FFN_TWO_LAUNCHES));
+    // (two launches: with ~2T rows both GEMMs have many tiles, and the persistent
+    // fused kernel measured slower here: 2.13 against 2.04 ms on the Switch-Large shape)
     if (err == cudaSuccess)
-        err = fused ? launch_ffn_tc_fused_ybuf(rows, ws.xbuf, w_in, w_out, counts, ws.ybuf, ws, st)
-              : tensor_cores ? launch_ffn_tc(rows, ws.xbuf, w_in, w_out, counts, ws.ybuf, nullptr, nullptr, nullptr, ws,
-                                             st)
-                             : launch_ffn_simt(rows, ws.xbuf, w_in, w_out, counts, ws.ybuf, ws, st);
+        err = tensor_cores ? launch_ffn_tc(rows, ws.xbuf, w_in, w_out, counts, ws.ybuf, nullptr, nullptr, nullptr, ws,
+                                           st)
+                           : launch_ffn_simt(rows, ws.xbuf, w_in, w_out, counts, ws.ybuf, ws, st);
     if (err == cudaSuccess) err = launch_combine_top2(*dims, ws.ybuf, expert, slot, gate, static_cast<float *>(y), st);
     return from_cuda(err);
 }

@@ -700,10 +700,7 @@ struct FusedLayout {
     }
 };
 
-// TO_YBUF: GEMM2 writes the ungated float32 expert output rows ybuf[e, s]
-// (a K-split part adds onto them) instead of the gated token-order scatter
-// into y; for top-2 routing, whose combine adds two rows per token.
-template <int STAGES, bool TO_YBUF>
+template <int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_ffn_fused_pair(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w1,
                       const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w2,
@@ -977,10 +974,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int row_base = m * BMP + (int)rank * BM + quarter * 32;
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-            if (second && TO_YBUF)
-                epilogue_async<BN, kEpiExpertOut>(t_row, e, row_base, min(counts[e], C), C, n, d, y, nullptr,
-                                                  slot_token, gate, my_stage, ks > 0, 0, nullptr, bw);
-            else if (second)
+            if (second)
                 epilogue_async<BN, kEpiGatedScatter>(t_row, e, row_base, min(counts[e], C), C, n, d, y, nullptr,
                                                      slot_token, gate, my_stage, ks > 0, 0, nullptr, bw);
             else
@@ -1094,13 +1088,13 @@ cudaError_t launch_gemm_pair(int32_t kernel_id, const void *a, const void *b, vo
     return err;
 }
 
-template <int STAGES, bool TO_YBUF>
+template <int STAGES>
 cudaError_t launch_ffn_fused(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
                              const int32_t *counts, const int32_t *slot_token, const float *gate, float *y,
                              const Workspace &ws, bool zero_done, cudaStream_t stream) {
     const int E = dims.num_experts, C = dims.capacity, d = dims.d_model, F = dims.d_ff;
     const size_t smem = FusedLayout<STAGES>::bytes(E);
-    auto kern = tc_ffn_fused_pair<STAGES, TO_YBUF>;
+    auto kern = tc_ffn_fused_pair<STAGES>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     CUtensorMap tx, tw1, th, tw2, tw1h, tw2h, ths;
@@ -1130,13 +1124,6 @@ cudaError_t launch_ffn_fused(const switch_dims_t &dims, const void *xbuf, const 
 }
 
 }  // namespace
-
-// Both expert GEMMs in one persistent launch, GEMM2 writing the ungated
-// float32 rows ybuf[e, s] (top-2 routing); zeroes the kernel's counters first.
-cudaError_t launch_ffn_tc_fused_ybuf(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
-                                     const int32_t *counts, float *ybuf, const Workspace &ws, cudaStream_t stream) {
-    return launch_ffn_fused<6, true>(dims, xbuf, w_in, w_out, counts, nullptr, nullptr, ybuf, ws, true, stream);
-}
 
 // Backward GEMMs (SM pairs, 256 x 256 tiles, the forward's kernel).
 // dZ [N][C][F] = bf16((dE W_out) where H > 0): A = dE [N][C][d], B = W_out^T [N][F][d].
@@ -1176,7 +1163,7 @@ cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const voi
     if (y && !(dims.flags & (SWITCH_FLAG_GEMM_1CTA | SWITCH_FLAG_FFN_TWO_LAUNCHES))) {
         // both GEMMs in one launch; the dependency counters were zeroed by the
         // slot assignment of this call
-        return launch_ffn_fused<6, false>(dims, xbuf, w_in, w_out, counts, slot_token, gate, y, ws, false, stream);
+        return launch_ffn_fused<6>(dims, xbuf, w_in, w_out, counts, slot_token, gate, y, ws, false, stream);
     }
     if (dims.flags & SWITCH_FLAG_GEMM_1CTA) {
         cudaError_t err = launch_gemm<256, 4, kEpiHiddenRelu>(K_FFN_TC_GEMM1, xbuf, w_in, ws.hidden, counts, N, C, d,

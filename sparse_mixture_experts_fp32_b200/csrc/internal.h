@@ -139,10 +139,6 @@ cudaError_t launch_small_layer(const switch_dims_t &dims, const void *x, const f
 cudaError_t launch_router_stats(const switch_dims_t &dims, const int32_t *counts, const Workspace &ws, float *stats,
                                 cudaStream_t stream);
 
-// Both expert GEMMs in one persistent launch writing the ungated ybuf rows (top-2 layer).
-cudaError_t launch_ffn_tc_fused_ybuf(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
-                                     const int32_t *counts, float *ybuf, const Workspace &ws, cudaStream_t stream);
-
 // Backward pass (bfloat16 experts; the workspace of a SWITCH_FLAG_TRAINING forward).
 int64_t router_dw_chunks(int64_t T);
 cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const float *w_r, const void *w_in,

@@ -9,10 +9,12 @@
 //   0 for a dropped token (llm-papers-study "精读 06 | Switch Transformers" §3.2,
 //   y = p_i*(x) E_i*(x); §3.4, dropped tokens skip the expert).
 //
-// Both are pure HBM streams.  Rows up to ~6 KB move through shared memory by
-// bulk copies (the TMA engine); longer rows (and rows that are not a multiple
-// of 16 bytes) use one warp per row with 16-byte (or 4-byte) vector accesses,
-// all of a lane's loads issued before its stores.
+// Both are pure HBM streams: by default one warp per row with 16-byte (or
+// 4-byte) vector accesses, all of a lane's loads issued before its stores.
+// With SWITCH_FLAG_STAGED_MOVES, rows up to ~6 KB move through shared memory
+// by bulk copies (the TMA engine) instead; on B200 that measured 4-6 % slower
+// on the Switch-Large shape (dispatch 98.9 against 94.7 us, combine 194.5
+// against 183.3 us), so the vector kernels stay the default.
 #include <algorithm>
 
 #include "common.cuh"
@@ -67,22 +69,15 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel16(const uint4 *__res
 // buffers it waits until the stores have read them.  The waits are bounded
 // (about a second); these entry points have no status word, so a wait that
 // gives up ends the warp's work after a second bounded wait for its loads.
-// Rounds alternate between two halves of the ring, so one round's loads
-// overlap the previous round's stores.
 // ---------------------------------------------------------------------------
 constexpr int kRingWarps = 4;
-constexpr int kRing = 4;     // rows per round; two rounds' buffers per warp (double buffering)
+constexpr int kRing = 4;
 // Shared memory of one ring block at most (rows up to ~6 KB; longer rows use the LSU kernels).
-constexpr size_t kRingSmemLimit = 200 * 1024;
+constexpr size_t kRingSmemLimit = 100 * 1024;
 
 __host__ __device__ constexpr int ring_stage_bytes(int row_bytes) { return (row_bytes + 127) / 128 * 128; }
 __host__ __device__ constexpr size_t ring_warp_bytes(int row_bytes) {
-    return 128 + (size_t)2 * kRing * ring_stage_bytes(row_bytes);  // barriers (padded to 128), then the buffers
-}
-
-// Wait until all but the most recent bulk group of this thread have read their shared memory.
-__device__ __forceinline__ void bulk_wait_read_all_but_one() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+    return 128 + (size_t)kRing * ring_stage_bytes(row_bytes);  // barriers (padded to 128), then the buffers
 }
 
 __device__ __forceinline__ bool ring_wait(uint64_t *bar, uint32_t parity) {
@@ -92,9 +87,6 @@ __device__ __forceinline__ bool ring_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // xbuf[e, s] = x[slot_token[e*C+s]] for the kept slots of every expert.
-// Round r uses buffer half r & 1: its loads are issued once the stores of
-// round r - 2 (the same half) have read their buffers, so they overlap the
-// stores of round r - 1.  One bulk group per round.
 __global__ void __launch_bounds__(32 * kRingWarps) dispatch_bulk_kernel(const uint8_t *__restrict__ x,
                                                                        const int32_t *__restrict__ slot_token,
                                                                        const int32_t *__restrict__ counts, int N,
@@ -103,21 +95,17 @@ __global__ void __launch_bounds__(32 * kRingWarps) dispatch_bulk_kernel(const ui
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t *base = smem_raw + (size_t)warp * ring_warp_bytes(row_bytes);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(base);  // 2 * kRing barriers
+    uint64_t *bar = reinterpret_cast<uint64_t *>(base);
     uint8_t *buf = base + 128;
     const int stage = ring_stage_bytes(row_bytes);
     if (lane != 0) return;  // one thread per warp drives the copy engine
-    for (int k = 0; k < 2 * kRing; ++k) mbar_init(&bar[k], 1);
+    for (int k = 0; k < kRing; ++k) mbar_init(&bar[k], 1);
     fence_barrier_init();
     const int64_t rows = (int64_t)N * C;
     const int64_t nwarps = (int64_t)gridDim.x * kRingWarps;
     uint32_t phases = 0;
     bool ok = true;
-    int round = 0;
-    for (int64_t first = (int64_t)blockIdx.x * kRingWarps + warp; ok && first < rows;
-         first += nwarps * kRing, ++round) {
-        const int h = (round & 1) * kRing;  // this round's buffers
-        if (round >= 2) bulk_wait_read_all_but_one();
+    for (int64_t first = (int64_t)blockIdx.x * kRingWarps + warp; ok && first < rows; first += nwarps * kRing) {
         int64_t dst[kRing];
         for (int k = 0; k < kRing; ++k) {
             const int64_t row = first + (int64_t)k * nwarps;
@@ -126,27 +114,27 @@ __global__ void __launch_bounds__(32 * kRingWarps) dispatch_bulk_kernel(const ui
             const int e = (int)(row / C), s = (int)(row % C);
             if (s >= min(counts[e], C)) continue;
             const int64_t t = slot_token[row];
-            mbar_arrive_expect_tx(&bar[h + k], (uint32_t)row_bytes);
-            bulk_load(buf + (size_t)(h + k) * stage, x + t * row_bytes, (uint32_t)row_bytes, &bar[h + k]);
+            mbar_arrive_expect_tx(&bar[k], (uint32_t)row_bytes);
+            bulk_load(buf + (size_t)k * stage, x + t * row_bytes, (uint32_t)row_bytes, &bar[k]);
             dst[k] = row;
         }
         for (int k = 0; k < kRing; ++k) {
             if (dst[k] < 0) continue;
-            const bool landed = ring_wait(&bar[h + k], (phases >> (h + k)) & 1u);
-            phases ^= 1u << (h + k);
+            const bool landed = ring_wait(&bar[k], (phases >> k) & 1u);
+            phases ^= 1u << k;
             if (!landed) {
                 ok = false;
                 continue;
             }
-            bulk_store(xbuf + dst[k] * row_bytes, buf + (size_t)(h + k) * stage, (uint32_t)row_bytes);
+            bulk_store(xbuf + dst[k] * row_bytes, buf + (size_t)k * stage, (uint32_t)row_bytes);
+            bulk_commit();
         }
-        bulk_commit();  // one group per round (possibly empty)
+        bulk_wait_read_all();  // the stores have read the buffers: the next round may refill them
     }
     bulk_wait_all();
 }
 
 // y[t] = gate[t] * ybuf[expert[t], slot[t]] (float32, one rounding), or a zero row.
-// Double-buffered rounds as in dispatch_bulk_kernel.
 __global__ void __launch_bounds__(32 * kRingWarps) combine_bulk_kernel(const float *__restrict__ ybuf,
                                                                       const int32_t *__restrict__ expert,
                                                                       const int32_t *__restrict__ slot,
@@ -160,7 +148,7 @@ __global__ void __launch_bounds__(32 * kRingWarps) combine_bulk_kernel(const flo
     uint8_t *buf = base + 128;
     const int stage = ring_stage_bytes(row_bytes);
     if (lane == 0) {
-        for (int k = 0; k < 2 * kRing; ++k) mbar_init(&bar[k], 1);
+        for (int k = 0; k < kRing; ++k) mbar_init(&bar[k], 1);
         fence_barrier_init();
     }
     __syncwarp();
@@ -168,14 +156,7 @@ __global__ void __launch_bounds__(32 * kRingWarps) combine_bulk_kernel(const flo
     const int words = d / 4;
     uint32_t phases = 0;
     bool ok = true;
-    int round = 0;
-    for (int64_t first = (int64_t)blockIdx.x * kRingWarps + warp; ok && first < T;
-         first += nwarps * kRing, ++round) {
-        const int h = (round & 1) * kRing;
-        if (round >= 2) {
-            if (lane == 0) bulk_wait_read_all_but_one();  // round r - 2's stores have read this half
-            __syncwarp();
-        }
+    for (int64_t first = (int64_t)blockIdx.x * kRingWarps + warp; ok && first < T; first += nwarps * kRing) {
         // lane k < kRing reads row k's slot; lane 0 starts the kept rows' loads
         int my_slot = -2;  // -2: past T
         const int64_t my_t = first + (int64_t)lane * nwarps;
@@ -188,18 +169,18 @@ __global__ void __launch_bounds__(32 * kRingWarps) combine_bulk_kernel(const flo
             for (int k = 0; k < kRing; ++k) {
                 if (s_of[k] < 0) continue;
                 const int64_t t = first + (int64_t)k * nwarps;
-                mbar_arrive_expect_tx(&bar[h + k], (uint32_t)row_bytes);
-                bulk_load(buf + (size_t)(h + k) * stage, ybuf + ((int64_t)expert[t] * C + s_of[k]) * d,
-                          (uint32_t)row_bytes, &bar[h + k]);
+                mbar_arrive_expect_tx(&bar[k], (uint32_t)row_bytes);
+                bulk_load(buf + (size_t)k * stage, ybuf + ((int64_t)expert[t] * C + s_of[k]) * d,
+                          (uint32_t)row_bytes, &bar[k]);
             }
         }
         for (int k = 0; k < kRing; ++k) {
             if (s_of[k] == -2) break;
             const int64_t t = first + (int64_t)k * nwarps;
-            float4 *row = reinterpret_cast<float4 *>(buf + (size_t)(h + k) * stage);
+            float4 *row = reinterpret_cast<float4 *>(buf + (size_t)k * stage);
             if (s_of[k] >= 0) {
-                const bool landed = ring_wait(&bar[h + k], (phases >> (h + k)) & 1u);
-                phases ^= 1u << (h + k);
+                const bool landed = ring_wait(&bar[k], (phases >> k) & 1u);
+                phases ^= 1u << k;
                 if (!landed) {
                     ok = false;
                     continue;
@@ -214,9 +195,12 @@ __global__ void __launch_bounds__(32 * kRingWarps) combine_bulk_kernel(const flo
             }
             fence_proxy_async_shared();  // the lanes' shared-memory writes, before the bulk store reads them
             __syncwarp();
-            if (lane == 0) bulk_store(y + t * d, row, (uint32_t)row_bytes);
+            if (lane == 0) {
+                bulk_store(y + t * d, row, (uint32_t)row_bytes);
+                bulk_commit();
+            }
         }
-        if (lane == 0) bulk_commit();  // one group per round (possibly empty)
+        if (lane == 0) bulk_wait_read_all();
         __syncwarp();
     }
     if (lane == 0) bulk_wait_all();
@@ -353,7 +337,7 @@ cudaError_t launch_dispatch(const switch_dims_t &dims, const void *x, const int3
     if (dims.T == 0) return cudaSuccess;
     const size_t ring_smem = kRingWarps * ring_warp_bytes((int)row_bytes);
     launch_begin(K_DISPATCH, stream);
-    if (row_bytes % 16 == 0 && ring_smem <= kRingSmemLimit) {
+    if ((dims.flags & SWITCH_FLAG_STAGED_MOVES) && row_bytes % 16 == 0 && ring_smem <= kRingSmemLimit) {
         cudaError_t err = cudaFuncSetAttribute(dispatch_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)ring_smem);
         if (err != cudaSuccess) {
@@ -384,7 +368,7 @@ cudaError_t launch_combine(const switch_dims_t &dims, const float *ybuf, const i
     const unsigned grid = (unsigned)((T + kRowsPerBlock - 1) / kRowsPerBlock);
     const size_t ring_smem = kRingWarps * ring_warp_bytes(dims.d_model * 4);
     launch_begin(K_COMBINE, stream);
-    if (dims.d_model % 4 == 0 && ring_smem <= kRingSmemLimit) {
+    if ((dims.flags & SWITCH_FLAG_STAGED_MOVES) && dims.d_model % 4 == 0 && ring_smem <= kRingSmemLimit) {
         cudaError_t err = cudaFuncSetAttribute(combine_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)ring_smem);
         if (err != cudaSuccess) {

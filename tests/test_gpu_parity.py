@@ -445,11 +445,13 @@ def test_uninitialised_workspace_reports_ok(entry):
 @pytest.mark.parametrize("d,dt", [(768, torch.bfloat16), (1024, torch.bfloat16), (4096, torch.bfloat16),
                                   (8192, torch.bfloat16), (96, torch.float32), (33, torch.float32)],
                          ids=["bf16-768", "bf16-1024", "bf16-4096", "bf16-8192", "f32-96", "f32-33"])
-def test_dispatch_and_combine_match_gathers(d, dt):
+@pytest.mark.parametrize("flags", [0, sm.SWITCH_FLAG_STAGED_MOVES], ids=["vector", "staged"])
+def test_dispatch_and_combine_match_gathers(d, dt, flags):
     """switch_dispatch and switch_combine on their own, bit for bit against torch gathers: xbuf rows
     are copies of x rows; y = gate * ybuf[expert, slot] (one float32 multiply), zero rows for dropped
-    tokens.  Short rows move through shared memory by bulk copies, long ones (and rows that are not a
-    multiple of 16 bytes) through vector loads and stores."""
+    tokens.  By default rows move through vector loads and stores; with SWITCH_FLAG_STAGED_MOVES short
+    rows move through shared memory by bulk copies (long ones, and rows that are not a multiple of 16
+    bytes, through vector accesses either way)."""
     T, N = 3000, 6
     g = torch.Generator("cuda").manual_seed(d)
     C = 300  # ~500 tokens per expert: about 40 % dropped
@@ -457,7 +459,7 @@ def test_dispatch_and_combine_match_gathers(d, dt):
     w_r = torch.randn(N, d, device="cuda", generator=g) * 0.01
     r = sm.route(x, w_r, capacity=C, d_ff=64)
     assert sm.switch_check(r["workspace"]) == 0
-    dims = sm.dims(T, d, 64, N, C, dt)
+    dims = sm.dims(T, d, 64, N, C, dt, flags)
     xbuf = torch.full((N * C, d), 7, dtype=dt, device="cuda")
     sm.switch_dispatch(dims, x, r["slot_token"], r["counts"], xbuf)
     st = r["slot_token"].view(N, C)
