@@ -72,7 +72,8 @@ enum Epilogue {
     kEpiExpertOut = 1,     // fp32 rows out[e * out_rows + row]
     kEpiGatedScatter = 2,  // y[slot_token] = gate * acc (with `add`: += )
     kEpiReluGrad = 3,      // backward: dZ = bf16(acc) where the forward's H > 0, else 0
-    kEpiScatterAdd = 4     // backward: dx[slot_token] += acc
+    kEpiScatterAdd = 4,    // backward: dx[slot_token] += acc
+    kEpiWeightGrad = 5     // backward weight gradients: fp32 rows out[e * out_rows + row] by TMA box stores
 };
 
 // Epilogue for one thread = one accumulator row (`row` of expert e's rows),
@@ -308,6 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 //                   writes its row (144-byte pitch: conflict-free) and
 //                   issues one 128-byte bulk copy to its destination row
 //                   (with `add`, a bulk fp32 add onto the destination).
+//   kEpiWeightGrad  32 fp32 columns at a time into a 32 x 128-byte swizzled
+//                   box, one TMA tensor store per box into the fixed-row
+//                   output [E][out_rows][Nout] (rows past out_rows clipped
+//                   by the tensor map).
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_base, int kept, int C, int n, int Nout,
                                                void *__restrict__ out, const void *tmap_out,
@@ -359,6 +364,30 @@ __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_ba
                     make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                                pack_bf16x2(v[6], v[7]));
             }
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0 && any_row && n * cols + c < Nout) {
+                tma_store_3d(tmap_out, stage, n * cols + c, row_base, e);
+                bulk_commit();
+            }
+        }
+        if (lane == 0) bulk_wait_read_all();
+    } else if (EPI == kEpiWeightGrad) {
+        // the warp's 32 rows x 32 fp32 columns per step, 128-byte-swizzled in its staging buffer
+        // (conflict-free writes), then one TMA tensor store of the 32 x 32 box
+        const bool any_row = row_base < kept;
+#pragma unroll 1
+        for (int c = 0; c < cols; c += 32) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
+            tmem_ld_wait();
+            if (lane == 0) bulk_wait_read_all();  // the previous box has left the buffer
+            __syncwarp();
+            uint8_t *rowp = stage + lane * 128;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<uint4 *>(rowp + ((q ^ (lane & 7)) << 4)) =
+                    make_uint4(r[4 * q + 0], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
             fence_proxy_async_shared();
             __syncwarp();
             if (lane == 0 && any_row && n * cols + c < Nout) {
@@ -1037,6 +1066,20 @@ bool make_tmap(CUtensorMap *map, const void *ptr, int E, int rows, int K, int bo
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D fp32 tensor [E][rows][cols] (cols contiguous), box = 32 rows x 32 columns, 128-byte swizzle
+// (the weight-gradient epilogue's store boxes).
+bool make_tmap_f32_box32(CUtensorMap *map, const void *ptr, int E, int rows, int cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)E};
+    const cuuint64_t strides[2] = {(cuuint64_t)cols * 4, (cuuint64_t)rows * cols * 4};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN, int STAGES, int EPI>
 cudaError_t launch_gemm(int32_t kernel_id, const void *a, const void *b, void *out, const int32_t *counts, int E,
                         int C, int K, int Nout, int64_t T, const int32_t *slot_token, const float *gate,
@@ -1070,6 +1113,8 @@ cudaError_t launch_gemm_pair(int32_t kernel_id, const void *a, const void *b, vo
     if (!make_tmap(&ta, a, E, a_rows, K, BM) || !make_tmap(&tb, b, E, Nout, K, BN / 2)) return cudaErrorInvalidValue;
     memset(&tout, 0, sizeof tout);
     if ((EPI == kEpiHiddenRelu || EPI == kEpiReluGrad) && !make_tmap(&tout, out, E, C, Nout, 32))
+        return cudaErrorInvalidValue;
+    if (EPI == kEpiWeightGrad && (shape.rows_fixed <= 0 || !make_tmap_f32_box32(&tout, out, E, shape.rows_fixed, Nout)))
         return cudaErrorInvalidValue;
     const size_t smem = PairLayout<BN, STAGES>::bytes(E);
     auto kern = tc_grouped_gemm_pair<BN, STAGES, EPI>;
@@ -1150,7 +1195,7 @@ cudaError_t launch_ffn_tc_bwd_dx(const switch_dims_t &dims, const void *grad_z, 
 // zero past the kept tokens).
 cudaError_t launch_ffn_tc_bwd_dw(const switch_dims_t &dims, const void *a_t, const void *b_t, const int32_t *counts,
                                  int rows, int nout, int Kp, float *out, DeviceStatus *st, cudaStream_t stream) {
-    return launch_gemm_pair<256, 6, kEpiExpertOut>(K_BWD_GEMM_DW, a_t, b_t, out, counts, dims.num_experts,
+    return launch_gemm_pair<256, 6, kEpiWeightGrad>(K_BWD_GEMM_DW, a_t, b_t, out, counts, dims.num_experts,
                                                    dims.capacity, Kp, nout, dims.T, nullptr, nullptr, st, stream,
                                                    GroupShape{rows, 1, rows, nullptr});
 }
