@@ -558,7 +558,13 @@ def time_backward(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, dev
     per_kernel: dict[str, list[float]] = {}
     for name, kms in trace:
         per_kernel.setdefault(name, []).append(kms)
-    transposes = 2 * (2 * N * d * F * s + N * Cp * (2 * d + 2 * F) * s)  # bytes of the six transposes per step
+    Np = -(-N // 64) * 64
+    Tc = max(256, -(-(-(-T // 64)) // 128) * 128)                       # tokens per dW_r chunk
+    chunks = -(-T // Tc)
+    # bytes of the transposes per step: two weights, four activation buffers, x in chunks of tokens
+    transposes = 2 * (2 * N * d * F * s + N * Cp * (2 * d + 2 * F) * s) + T * d * s + chunks * Tc * d * s
+    # the router operand splits: dh -> [T][6 Np] and W_r -> [d][6 Np] (dx), dh -> [3N][chunk tokens] (dW_r)
+    splits = (4 * T * N + 2 * T * 6 * Np) + (4 * N * d + 2 * d * 6 * Np) + (4 * T * N + 2 * 3 * N * chunks * Tc)
     work = {
         "bwd_gate_softmax": ("hbm", 4 * T * d + 4 * K * d + 2 * K * d + 8 * T * N, None),
         "bwd_tc_gemm_dz": ("tensor", 2.0 * K * d * F, None),
@@ -566,6 +572,9 @@ def time_backward(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, dev
         "bwd_tc_gemm_dw": ("tensor", 2.0 * K * d * F, None),
         "bwd_router_dx": ("alu", 2.0 * T * N * d, None),
         "bwd_router_dw": ("alu", 2.0 * T * N * d, None),
+        # bf16 MMA flops executed on the exact splits: six term pairs (dx), three dh terms (dW_r)
+        "bwd_router_tc_dx": ("tensor", 2.0 * T * d * 6 * N, None),
+        "bwd_router_tc_dw": ("tensor", 2.0 * T * d * 3 * N, None),
         "ffn_tc_gemm1_relu": ("tensor", 2.0 * K * d * F, None),
         "ffn_tc_gemm2": ("tensor", 2.0 * K * F * d, None),
     }
@@ -573,8 +582,9 @@ def time_backward(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, dev
     kernels = {}
     for name, times in per_kernel.items():
         n_per_step = len(times) // steps
-        if name == "bwd_transpose":
-            kernels[name] = kernel_entry("hbm", transposes / max(n_per_step, 1), None, statistics.mean(times),
+        if name in ("bwd_transpose", "bwd_router_split"):
+            total = transposes if name == "bwd_transpose" else splits
+            kernels[name] = kernel_entry("hbm", total / max(n_per_step, 1), None, statistics.mean(times),
                                          n_per_step, peaks)
             continue
         kind, amount, amount_act = work.get(name, ("?", 0, None))

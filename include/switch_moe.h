@@ -292,7 +292,12 @@ switch_status_t switch_router_stats(const switch_dims_t *dims, const int32_t *co
  * (zero for experts without kept tokens).  A dropped token's dx is the router
  * part only.  The expert GEMMs run on tcgen05 tensor cores with bfloat16
  * operands (gate * dy and the pre-activation gradient rounded to bfloat16) and
- * float32 accumulation; the router part runs in float32.  Deterministic.
+ * float32 accumulation.  The router products (dh W_r into dx, dh^T x into
+ * dw_r) run on the tensor cores too, over exact three-term bfloat16 splits of
+ * their float32 operands with float32 accumulation (the three smallest term
+ * pairs of dh W_r, below 2^-23 of |dh| |W_r| together, are left out); with
+ * SWITCH_FLAG_SIMT_ROUTER in dims.flags (for the forward too) they run as
+ * float32 FMA kernels instead.  Deterministic.
  * Errors: SWITCH_ERR_UNSUPPORTED without SWITCH_FLAG_TRAINING, for float32
  * experts or with SWITCH_FLAG_SIMT_FFN / SWITCH_FLAG_GEMM_1CTA; SWITCH_ERR_SHAPE
  * for a non-finite g_aux; otherwise as switch_layer_fwd. */

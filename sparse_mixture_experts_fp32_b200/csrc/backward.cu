@@ -11,11 +11,15 @@
 //   g_gate = dy . o                      dE = p_i* dy          (bwd_token_kernel)
 //   dp_i = [i = i*] g_gate + g_aux N f_i / T,  dh = p (dp - p . dp)
 //   dZ = (dE W_out[i*]) masked by z > 0  (tcgen05 GEMM, epilogue kEpiReluGrad)
-//   dx = dh W_r + dZ W_in[i*]            (router_dx_kernel, then a tcgen05 GEMM
-//                                         whose epilogue adds into dx rows)
+//   dx = dh W_r + dZ W_in[i*]            (tcgen05 GEMM on exact bf16 splits of dh
+//                                         and W_r, then a tcgen05 GEMM whose
+//                                         epilogue adds into dx rows)
 //   dW_out[i] = sum over kept tokens of dE u^T   (tcgen05 GEMM over K = tokens)
 //   dW_in[i]  = sum over kept tokens of dZ x^T   (tcgen05 GEMM over K = tokens)
-//   dW_r = sum_t dh x^T, d bias = sum_t dh        (router_dw_kernel + fixed-order reduce)
+//   dW_r = sum_t dh x^T, d bias = sum_t dh        (tcgen05 GEMM per chunk of tokens
+//                                         on the split dh, + fixed-order reduce)
+// With SWITCH_FLAG_SIMT_ROUTER the two router products run as float32 FMA
+// kernels instead (router_dx_kernel, router_dw_kernel).
 // The expert GEMMs are the forward's grouped "A . B^T" kernel with both
 // operands K-major: the weights and the per-expert activation buffers are
 // first transposed in HBM (batched 64 x 64 tile transposes; rows past an
@@ -23,6 +27,8 @@
 // kept tokens).  Every reduction runs in a fixed order: identical inputs give
 // identical bytes.
 #include <cuda.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
@@ -252,6 +258,139 @@ __global__ void reduce_chunks_kernel(const float *__restrict__ part, int chunks,
     }
 }
 
+// ---------------------------------------------------------------------------
+// Router backward on the tensor cores.  Both router products are dense
+// float32 contractions (dx += dh W_r over the N experts, dW_r = dh^T x over
+// the tokens); they run as bf16 tcgen05 GEMMs on exact three-term splits of
+// their float32 operands (split_bf16x3; x is bf16 already):
+//   dx:   sum over the six term pairs (dh_a, W_b) with a + b <= 2 of
+//         dh_a W_b, laid side by side along K (K = 6 Np, Np = N rounded up
+//         to 64, zero columns past N).  The three dropped pairs are below
+//         2^-23 of |dh| |W_r| together.
+//   dW_r: the three dh terms stacked as rows (M = 3N) against x^T, per chunk
+//         of Tc tokens (the chunks are the GEMM's groups, K = Tc), then a
+//         fixed-order sum over terms and chunks.
+// Products of bf16 terms are exact in float32; the tensor cores accumulate
+// in float32.
+// ---------------------------------------------------------------------------
+constexpr int kDxPairs = 6;
+__device__ __forceinline__ int dx_dh_term(int p) { return p < 3 ? 0 : (p < 5 ? 1 : 2); }  // 0 0 0 1 1 2
+__device__ __forceinline__ int dx_w_term(int p) { return p < 3 ? p : (p < 5 ? p - 3 : 0); }  // 0 1 2 0 1 0
+
+// A operand of the dx product: a[t][p * Np + i] = term dx_dh_term(p) of dh[t, i]
+// (zero for i >= N).  One thread per 8 experts of a token.
+__global__ void __launch_bounds__(256) router_dx_a_kernel(const float *__restrict__ dh, int64_t T, int N, int Np,
+                                                         uint16_t *__restrict__ a) {
+    const int oct = Np / 8;
+    const int64_t total = T * oct;
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total;
+         q += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = q / oct;
+        const int i0 = (int)(q % oct) * 8;
+        uint16_t sp[8][3];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) split_bf16x3(i0 + j < N ? dh[t * N + i0 + j] : 0.f, sp[j]);
+        uint16_t *row = a + t * (int64_t)(kDxPairs * Np) + i0;
+#pragma unroll
+        for (int p = 0; p < kDxPairs; ++p) {
+            const int m = dx_dh_term(p);
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w[j] = (uint32_t)sp[2 * j][m] | ((uint32_t)sp[2 * j + 1][m] << 16);
+            *reinterpret_cast<uint4 *>(row + p * Np) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
+// B operand of the dx product: b[k][p * Np + i] = term dx_w_term(p) of W_r[i, k]
+// (zero for i >= N); also the token count of every dW_r chunk and a 1 at
+// chunk_counts[chunks] (the single group of the dx GEMM).
+__global__ void __launch_bounds__(256) router_dx_b_kernel(const float *__restrict__ w_r, int N, int d, int Np,
+                                                         uint16_t *__restrict__ b, int64_t T, int64_t chunk_tokens,
+                                                         int chunks, int32_t *__restrict__ chunk_counts) {
+    const int oct = Np / 8;
+    const int64_t total = (int64_t)d * oct;
+    const int64_t first = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (int64_t c = first; c <= chunks; c += (int64_t)gridDim.x * blockDim.x)
+        chunk_counts[c] = c < chunks ? (int32_t)min(chunk_tokens, T - c * chunk_tokens) : 1;
+    for (int64_t q = first; q < total; q += (int64_t)gridDim.x * blockDim.x) {
+        const int k = (int)(q / oct);
+        const int i0 = (int)(q % oct) * 8;
+        uint16_t sp[8][3];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) split_bf16x3(i0 + j < N ? w_r[(int64_t)(i0 + j) * d + k] : 0.f, sp[j]);
+        uint16_t *row = b + (int64_t)k * (kDxPairs * Np) + i0;
+#pragma unroll
+        for (int p = 0; p < kDxPairs; ++p) {
+            const int m = dx_w_term(p);
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w[j] = (uint32_t)sp[2 * j][m] | ((uint32_t)sp[2 * j + 1][m] << 16);
+            *reinterpret_cast<uint4 *>(row + p * Np) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
+// A operand of the dW_r product, transposed per chunk of Tc tokens:
+// a[c][m * N + i][tl] = term m of dh[c Tc + tl, i] (zero past T), and the
+// chunk's d bias partial db_part[c][i] = sum over its tokens of dh[t, i] in
+// token order.  Block: one chunk x 32 experts, 128-token tiles through shared
+// memory; lane = expert, each thread writes 16 tokens (32 bytes) of one term.
+constexpr int kDwtTok = 128;
+__global__ void __launch_bounds__(256) router_dw_a_kernel(const float *__restrict__ dh, int64_t T, int N,
+                                                         int64_t chunk_tokens, uint16_t *__restrict__ a,
+                                                         float *__restrict__ db_part) {
+    __shared__ float s[kDwtTok][33];
+    const int c = blockIdx.x, i0 = blockIdx.y * 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t tbeg = (int64_t)c * chunk_tokens;
+    float acc_b = 0.f;
+    for (int64_t tl0 = 0; tl0 < chunk_tokens; tl0 += kDwtTok) {
+        __syncthreads();
+        for (int q = tid; q < kDwtTok * 32; q += 256) {
+            const int tl = q >> 5, ii = q & 31;
+            const int64_t t = tbeg + tl0 + tl;
+            s[tl][ii] = (t < T && tl0 + tl < chunk_tokens && i0 + ii < N) ? dh[t * N + i0 + ii] : 0.f;
+        }
+        __syncthreads();
+        if (warp == 0)
+            for (int tl = 0; tl < kDwtTok; ++tl) acc_b += s[tl][lane];
+        const int i = i0 + lane;
+        if (i < N) {
+            for (int combo = warp; combo < 3 * (kDwtTok / 16); combo += 8) {
+                const int m = combo / (kDwtTok / 16), q = combo % (kDwtTok / 16);
+                uint32_t w[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint16_t lo[3], hi[3];
+                    split_bf16x3(s[16 * q + 2 * j][lane], lo);
+                    split_bf16x3(s[16 * q + 2 * j + 1][lane], hi);
+                    w[j] = (uint32_t)lo[m] | ((uint32_t)hi[m] << 16);
+                }
+                uint4 *dst = reinterpret_cast<uint4 *>(a + (((int64_t)c * 3 * N + (int64_t)m * N + i) * chunk_tokens +
+                                                            tl0 + 16 * q));
+                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+        }
+    }
+    if (warp == 0 && i0 + lane < N) db_part[(int64_t)c * N + i0 + lane] = acc_b;
+}
+
+// dW_r[i][k] = sum over chunks c, in order, of (part[c][2N + i][k] + part[c][N + i][k]) + part[c][i][k].
+__global__ void router_dw_reduce_kernel(const float *__restrict__ part, int chunks, int N, int d,
+                                        float *__restrict__ dw_r) {
+    const int64_t n = (int64_t)N * d, term = (int64_t)N * d;
+    for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n; j += (int64_t)gridDim.x * blockDim.x) {
+        float acc = 0.f;
+        for (int c = 0; c < chunks; ++c) {
+            const float *pc = part + (int64_t)c * 3 * term;
+            acc += (pc[2 * term + j] + pc[term + j]) + pc[j];
+        }
+        dw_r[j] = acc;
+    }
+}
+
 int64_t round_up64(int64_t v) { return (v + 63) / 64 * 64; }
 
 cudaError_t launch_transpose(int32_t kernel_id, const void *in, void *out, int B, int R, int Cc, int Rp,
@@ -274,6 +413,18 @@ int64_t router_dw_chunks(int64_t T) {
     const int64_t c = (T + 2047) / 2048;
     return c < 1 ? 1 : (c > 64 ? 64 : c);
 }
+
+// Tokens per chunk of the tensor-core dW_r product: a multiple of 128, at
+// least 256, and at most 64 chunks.
+int64_t router_tc_chunk_tokens(int64_t T) {
+    int64_t tc = ((T + 63) / 64 + 127) / 128 * 128;
+    return tc < 256 ? 256 : tc;
+}
+int64_t router_tc_chunks(int64_t T) {
+    const int64_t tc = router_tc_chunk_tokens(T);
+    return T > 0 ? (T + tc - 1) / tc : 1;
+}
+int router_tc_np(int N) { return (N + 63) / 64 * 64; }
 
 cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const float *w_r, const void *w_in,
                              const void *w_out, const int32_t *expert, const float *gate, const int32_t *slot,
@@ -310,12 +461,32 @@ cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const flo
     err = launch_ffn_tc_bwd_dz(dims, ws.grad_e, ws.w_out_t, counts, ws.grad_z, ws.hidden, st, stream);
     if (err != cudaSuccess) return err;
     // 4. dx = dh W_r (all rows), then + dZ W_in for kept rows
-    {
+    const bool simt_router = (dims.flags & SWITCH_FLAG_SIMT_ROUTER) != 0;
+    const int Np = router_tc_np(N);
+    const int64_t Tc = router_tc_chunk_tokens(T), chunks_tc = router_tc_chunks(T);
+    if (simt_router) {
         const dim3 grid((unsigned)((d + kDxCol - 1) / kDxCol), (unsigned)((T + kDxTok - 1) / kDxTok));
         launch_begin(K_BWD_ROUTER_DX, stream);
         router_dx_kernel<<<grid, 256, 0, stream>>>(ws.dh, w_r, T, N, d, dx);
         err = cudaGetLastError();
         launch_end(stream);
+        if (err != cudaSuccess) return err;
+    } else {
+        const int sms = device_sm_count();
+        launch_begin(K_BWD_ROUTER_SPLIT, stream);
+        router_dx_a_kernel<<<(unsigned)std::min<int64_t>((T * (Np / 8) + 255) / 256, 16 * sms), 256, 0, stream>>>(
+            ws.dh, T, N, Np, static_cast<uint16_t *>(ws.rdx_a));
+        err = cudaGetLastError();
+        launch_end(stream);
+        if (err != cudaSuccess) return err;
+        launch_begin(K_BWD_ROUTER_SPLIT, stream);
+        router_dx_b_kernel<<<(unsigned)(((int64_t)d * (Np / 8) + 255) / 256), 256, 0, stream>>>(
+            w_r, N, d, Np, static_cast<uint16_t *>(ws.rdx_b), T, Tc, (int)chunks_tc, ws.chunk_counts);
+        err = cudaGetLastError();
+        launch_end(stream);
+        if (err != cudaSuccess) return err;
+        err = launch_router_tc_bwd_dx(ws.rdx_a, ws.rdx_b, ws.chunk_counts + chunks_tc, T, d, kDxPairs * Np, dx, st,
+                                      stream);
         if (err != cudaSuccess) return err;
     }
     err = launch_ffn_tc_bwd_dx(dims, ws.grad_z, ws.w_in_t, counts, ws.slot_token, dx, st, stream);
@@ -339,7 +510,30 @@ cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const flo
     err = launch_ffn_tc_bwd_dw(dims, ws.grad_z_t, ws.xbuf_t, counts, F, d, (int)Cp, dw_in, st, stream);
     if (err != cudaSuccess) return err;
     // 7. dW_r and d bias: chunk partials, then a fixed-order sum
-    {
+    if (!simt_router) {
+        launch_begin(K_BWD_ROUTER_SPLIT, stream);
+        router_dw_a_kernel<<<dim3((unsigned)chunks_tc, (unsigned)((N + 31) / 32)), 256, 0, stream>>>(
+            ws.dh, T, N, Tc, static_cast<uint16_t *>(ws.rdw_a), ws.db_part);
+        err = cudaGetLastError();
+        launch_end(stream);
+        if (err != cudaSuccess) return err;
+        if ((err = launch_transpose(K_BWD_TRANSPOSE, x, ws.x_t, (int)chunks_tc, (int)Tc, d, (int)Tc, ws.chunk_counts,
+                                    (int)Tc, stream)) != cudaSuccess)
+            return err;
+        err = launch_router_tc_bwd_dw(ws.rdw_a, ws.x_t, ws.chunk_counts, (int)chunks_tc, 3 * N, (int)Tc, d, T,
+                                      ws.dw_part, st, stream);
+        if (err != cudaSuccess) return err;
+        launch_begin(K_BWD_REDUCE, stream);
+        router_dw_reduce_kernel<<<256, 256, 0, stream>>>(ws.dw_part, (int)chunks_tc, N, d, dw_r);
+        err = cudaGetLastError();
+        launch_end(stream);
+        if (err == cudaSuccess && dbias) {
+            launch_begin(K_BWD_REDUCE, stream);
+            reduce_chunks_kernel<<<1, 256, 0, stream>>>(ws.db_part, (int)chunks_tc, (int64_t)N, dbias);
+            err = cudaGetLastError();
+            launch_end(stream);
+        }
+    } else {
         const int64_t chunks = router_dw_chunks(T);
         const int64_t chunk_tokens = (T + chunks - 1) / chunks;
         const dim3 grid((unsigned)((d + kDwCol - 1) / kDwCol), (unsigned)((N + kDwI - 1) / kDwI), (unsigned)chunks);
@@ -351,9 +545,14 @@ cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const flo
         if (err != cudaSuccess) return err;
         launch_begin(K_BWD_REDUCE, stream);
         reduce_chunks_kernel<<<256, 256, 0, stream>>>(ws.dw_part, (int)chunks, (int64_t)N * d, dw_r);
-        if (dbias) reduce_chunks_kernel<<<1, 256, 0, stream>>>(ws.db_part, (int)chunks, (int64_t)N, dbias);
         err = cudaGetLastError();
         launch_end(stream);
+        if (err == cudaSuccess && dbias) {
+            launch_begin(K_BWD_REDUCE, stream);
+            reduce_chunks_kernel<<<1, 256, 0, stream>>>(ws.db_part, (int)chunks, (int64_t)N, dbias);
+            err = cudaGetLastError();
+            launch_end(stream);
+        }
     }
     return err;
 }

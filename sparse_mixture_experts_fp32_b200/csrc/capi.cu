@@ -27,7 +27,7 @@ int64_t tiles_of(const switch_dims_t &d) { return (d.T + kTileT - 1) / kTileT; }
 struct Sections {
     size_t status, ticket, hist, psum, tile_off, prob_total, w_split, slot_token, xbuf, ybuf, hidden, done, hist2,
         tile_off2, counts_first, ent, probs, dh, grad_e, grad_z, w_out_t, w_in_t, grad_e_t, hidden_t, xbuf_t, grad_z_t,
-        dw_part, db_part, total;
+        dw_part, db_part, rdx_a, rdx_b, rdw_a, x_t, chunk_counts, total;
 };
 
 Sections layout(const switch_dims_t &d) {
@@ -69,8 +69,20 @@ Sections layout(const switch_dims_t &d) {
         s.hidden_t = take(N * F * Cp * es);
         s.xbuf_t = take(N * dm * Cp * es);
         s.grad_z_t = take(N * F * Cp * es);
-        s.dw_part = take(chunks * N * dm * 4);
-        s.db_part = take(chunks * N * 4);
+        if (d.flags & SWITCH_FLAG_SIMT_ROUTER) {  // float32 FMA router products
+            s.dw_part = take(chunks * N * dm * 4);
+            s.db_part = take(chunks * N * 4);
+        } else {  // tensor-core router products on split operands
+            const size_t Np = (size_t)router_tc_np((int)N), Tc = (size_t)router_tc_chunk_tokens(d.T),
+                         ch = (size_t)router_tc_chunks(d.T);
+            s.dw_part = take(ch * 3 * N * dm * 4);
+            s.db_part = take(ch * N * 4);
+            s.rdx_a = take(T * 6 * Np * 2);
+            s.rdx_b = take(dm * 6 * Np * 2);
+            s.rdw_a = take(ch * 3 * N * Tc * 2);
+            s.x_t = take(ch * dm * Tc * 2);
+            s.chunk_counts = take((ch + 1) * 4);
+        }
     }
     s.total = off;
     return s;
@@ -206,6 +218,11 @@ Workspace carve_workspace(const switch_dims_t &dims, void *base) {
     w.grad_z_t = at(s.grad_z_t);
     w.dw_part = static_cast<float *>(at(s.dw_part));
     w.db_part = static_cast<float *>(at(s.db_part));
+    w.rdx_a = at(s.rdx_a);
+    w.rdx_b = at(s.rdx_b);
+    w.rdw_a = at(s.rdw_a);
+    w.x_t = at(s.x_t);
+    w.chunk_counts = static_cast<int32_t *>(at(s.chunk_counts));
     w.tiles = tiles_of(dims);
     return w;
 }
@@ -584,6 +601,9 @@ const char *switch_kernel_name(int32_t id) {
         case K_BWD_REDUCE: return "bwd_reduce";
         case K_ROUTER_STATS: return "router_stats";
         case K_SMALL_LAYER: return "small_layer";
+        case K_BWD_ROUTER_SPLIT: return "bwd_router_split";
+        case K_BWD_ROUTER_TC_DX: return "bwd_router_tc_dx";
+        case K_BWD_ROUTER_TC_DW: return "bwd_router_tc_dw";
     }
     return "?";
 }

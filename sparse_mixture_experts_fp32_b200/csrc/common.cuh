@@ -412,6 +412,20 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
+// Exact three-term split of a float32 into bfloat16 bit patterns,
+// v = s[0] + s[1] + s[2]: each term is the round-to-nearest bfloat16 of what
+// the earlier terms left (8 significant bits plus the rounding's sign each,
+// enough for the 24 of a float32; the differences are exact in float32).
+__device__ __forceinline__ void split_bf16x3(float v, uint16_t s[3]) {
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);
+    s[0] = __bfloat16_as_ushort(hi);
+    s[1] = __bfloat16_as_ushort(mid);
+    s[2] = float_to_bf16_bits(r2);
+}
+
 // Two floats -> packed bf16x2 (lo in the low half).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

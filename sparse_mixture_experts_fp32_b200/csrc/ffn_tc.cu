@@ -675,8 +675,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // The tile list holds every GEMM1 tile (expert e, 256-row block m, H column
 // block n) and then every GEMM2 tile (e, m, y column block).  Pairs claim
 // tiles in list order from a per-call counter (the leader's producer thread
-// takes the next index and hands it, through a 4-deep queue in shared
-// memory, to its MMA thread, its epilogue warps and the peer CTA).  A GEMM2
+// takes the next index one tile ahead and hands it, through a 4-deep queue in
+// shared memory, to its MMA thread, its epilogue warps and the peer CTA); a
+// pair works through its claims in claim order, and every wait below is on a
+// tile of lower index, so the lowest unfinished tile can always proceed.  A GEMM2
 // tile reads the H rows of its row block, written by the n1 = F / 256 GEMM1
 // tiles of (e, m): each of the pair's 8 epilogue warps adds 1 to done[e, m]
 // once its H boxes have fully landed (TMA store completion, then a release
@@ -861,14 +863,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            // The leader claims one tile ahead: the claim of the next tile is in
+            // flight while this tile's loads are issued, so the ring does not run
+            // dry for the claim's round trip at every tile boundary.  Tiles are
+            // still processed in claim order, one pair at a time.
+            int pending = rank == 0 ? atomicAdd(ticket, 1) : -1;
             for (int it = 0; ok; ++it) {
                 const int j = it % kTileQ;
                 const uint32_t qph = (uint32_t)(it / kTileQ) & 1u;
                 int tile;
-                if (rank == 0) {  // claim the next tile and hand its index to everyone
+                if (rank == 0) {  // hand the claimed tile's index to everyone, claim the next
                     if (!mbar_wait_cluster(&tq_empty[j], qph ^ 1u, status, 48)) break;
-                    tile = atomicAdd(ticket, 1);
+                    tile = pending;
                     if (tile >= total) tile = -1;
+                    if (tile >= 0) pending = atomicAdd(ticket, 1);
                     tq[j] = tile;
                     st_cluster_s32(map_to_rank(&tq[j], 1), tile);
                     mbar_arrive(&tq_full[j]);
@@ -1197,6 +1205,26 @@ cudaError_t launch_ffn_tc_bwd_dw(const switch_dims_t &dims, const void *a_t, con
                                  int rows, int nout, int Kp, float *out, DeviceStatus *st, cudaStream_t stream) {
     return launch_gemm_pair<256, 6, kEpiWeightGrad>(K_BWD_GEMM_DW, a_t, b_t, out, counts, dims.num_experts,
                                                    dims.capacity, Kp, nout, dims.T, nullptr, nullptr, st, stream,
+                                                   GroupShape{rows, 1, rows, nullptr});
+}
+
+// Router part of dx (float32 [T][d], overwritten) = A . B^T with A [T][K] the
+// split dh terms and B [d][K] the split W_r terms: one group of T fixed rows
+// (`one` points at a device 1, the group's count).
+cudaError_t launch_router_tc_bwd_dx(const void *a, const void *b, const int32_t *one, int64_t T, int d, int K,
+                                    float *dx, DeviceStatus *st, cudaStream_t stream) {
+    if (T > INT32_MAX) return cudaErrorInvalidValue;
+    return launch_gemm_pair<256, 6, kEpiWeightGrad>(K_BWD_ROUTER_TC_DX, a, b, dx, one, 1, 1, K, d, T, nullptr,
+                                                   nullptr, st, stream, GroupShape{(int)T, 0, (int)T, nullptr});
+}
+
+// dW_r partials part [chunks][rows][d] (float32): per chunk c, A [rows][Tc]
+// (split dh terms) . B [d][Tc] (x^T) over the chunk's chunk_counts[c] tokens.
+cudaError_t launch_router_tc_bwd_dw(const void *a, const void *b, const int32_t *chunk_counts, int chunks, int rows,
+                                    int chunk_tokens, int d, int64_t T, float *part, DeviceStatus *st,
+                                    cudaStream_t stream) {
+    return launch_gemm_pair<256, 6, kEpiWeightGrad>(K_BWD_ROUTER_TC_DW, a, b, part, chunk_counts, chunks,
+                                                   chunk_tokens, chunk_tokens, d, T, nullptr, nullptr, st, stream,
                                                    GroupShape{rows, 1, rows, nullptr});
 }
 

@@ -43,6 +43,9 @@ enum KernelId : int32_t {
     K_BWD_REDUCE = 26,
     K_ROUTER_STATS = 27,
     K_SMALL_LAYER = 28,
+    K_BWD_ROUTER_SPLIT = 29,
+    K_BWD_ROUTER_TC_DX = 30,
+    K_BWD_ROUTER_TC_DW = 31,
 };
 
 struct Workspace {
@@ -76,6 +79,11 @@ struct Workspace {
     void *grad_z_t;      // [N][F][Cp] bf16
     float *dw_part;      // [chunks][N][d] partial sums of dW_r
     float *db_part;      // [chunks][N] partial sums of d bias
+    void *rdx_a;         // [T][6 Np] bf16 split dh terms (tensor-core router dx)
+    void *rdx_b;         // [d][6 Np] bf16 split W_r terms (tensor-core router dx)
+    void *rdw_a;         // [chunks][3N][Tc] bf16 split dh terms, token-contiguous (tensor-core dW_r)
+    void *x_t;           // [chunks][d][Tc] bf16 x, token-contiguous (tensor-core dW_r)
+    int32_t *chunk_counts;  // [chunks + 1] tokens of each dW_r chunk, then a 1
     int64_t tiles;
 };
 
@@ -141,6 +149,14 @@ cudaError_t launch_router_stats(const switch_dims_t &dims, const int32_t *counts
 
 // Backward pass (bfloat16 experts; the workspace of a SWITCH_FLAG_TRAINING forward).
 int64_t router_dw_chunks(int64_t T);
+int64_t router_tc_chunk_tokens(int64_t T);
+int64_t router_tc_chunks(int64_t T);
+int router_tc_np(int N);
+cudaError_t launch_router_tc_bwd_dx(const void *a, const void *b, const int32_t *one, int64_t T, int d, int K,
+                                    float *dx, DeviceStatus *st, cudaStream_t stream);
+cudaError_t launch_router_tc_bwd_dw(const void *a, const void *b, const int32_t *chunk_counts, int chunks, int rows,
+                                    int chunk_tokens, int d, int64_t T, float *part, DeviceStatus *st,
+                                    cudaStream_t stream);
 cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const float *w_r, const void *w_in,
                              const void *w_out, const int32_t *expert, const float *gate, const int32_t *slot,
                              const int32_t *counts, const float *dy, float g_aux, float *dx, float *dw_r, float *dbias,

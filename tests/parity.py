@@ -195,7 +195,14 @@ def backward_error_bounds(inp: dict, C: int, dy: np.ndarray, g_aux: float, route
     the router's probabilities are float32 (relative error <= 2^-18).  For a dot product of a
     rounded operand with an exact one the error is at most (u + K 2^-24) times the sum of
     absolute products; the bounds below chain that through the backward's steps (magnitudes
-    computed in float64 from the inputs and the oracle's routing).  route: oracle route() with probs."""
+    computed in float64 from the inputs and the oracle's routing).
+    The router products run on the tensor cores over exact three-term bfloat16 splits of their
+    float32 operands (products exact; float32 accumulation taken as <= 2^-23 per addition, which
+    also covers truncating adders): dx's router part sums 6N split products (the three dropped
+    term pairs add <= 2^-23 of |dh| |W_r|), so (12N + 3) 2^-24; dW_r sums <= Tc <= T products per
+    chunk and term, then three terms and <= 64 chunks in float32, so (2T + 67) 2^-24; d bias is a
+    float32 sum in token order per chunk, then over the chunks, so (T + 64) 2^-24.  These also
+    bound the float32 FMA router kernels (N 2^-24 and T 2^-24).  route: oracle route() with probs."""
     x = _f64(inp["x"])
     w_in, w_out = _f64(inp["w_in"]), _f64(inp["w_out"])
     w_r = inp["w_r"].astype(np.float64)
@@ -204,7 +211,7 @@ def backward_error_bounds(inp: dict, C: int, dy: np.ndarray, g_aux: float, route
     p, e_of, slot = route["probs"], route["expert"], route["slot"]
     gate = p[np.arange(T), e_of]
     dy = dy.astype(np.float64)
-    g_f, g_d, g_c, g_t, g_n = F * U_F32, d * U_F32, max(C, 1) * U_F32, T * U_F32, N * U_F32
+    g_f, g_d, g_c = F * U_F32, d * U_F32, max(C, 1) * U_F32
     b = dict(dx=np.zeros((T, d)), dw_in=np.zeros((N, F, d)), dw_out=np.zeros((N, d, F)))
     err_g = np.zeros(T)                      # bound on the gate gradient's error
     for e in range(N):
@@ -236,9 +243,10 @@ def backward_error_bounds(inp: dict, C: int, dy: np.ndarray, g_aux: float, route
     dh = p * (dp - (p * dp).sum(1, keepdims=True))
     err_dh = p * (onehot + gate[:, None]) * err_g[:, None] + \
         EPS_P * (p * np.abs(dp) + p * (p * np.abs(dp)).sum(1, keepdims=True))
-    b["dx"] += err_dh @ np.abs(w_r) + g_n * (np.abs(dh) @ np.abs(w_r))
-    b["dw_r"] = err_dh.T @ np.abs(x) + g_t * (np.abs(dh).T @ np.abs(x))
-    b["dbias"] = err_dh.sum(0) + g_t * np.abs(dh).sum(0)
+    g_rdx, g_rdw, g_db = (12 * N + 3) * U_F32, (2 * T + 67) * U_F32, (T + 64) * U_F32
+    b["dx"] += err_dh @ np.abs(w_r) + g_rdx * (np.abs(dh) @ np.abs(w_r))
+    b["dw_r"] = err_dh.T @ np.abs(x) + g_rdw * (np.abs(dh).T @ np.abs(x))
+    b["dbias"] = err_dh.sum(0) + g_db * np.abs(dh).sum(0)
     return b
 
 

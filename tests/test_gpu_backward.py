@@ -4,7 +4,9 @@ fp64 backward oracle, element by element.
 The loss is L = sum(y * dy) + g_aux * aux with a seeded upstream gradient dy.
 The expert GEMMs take bfloat16 operands (the hidden activations H, gate * dy
 and the pre-activation gradient dZ, each rounded once) and accumulate in
-float32; the router part runs in float32.  The tolerance is derived from that
+float32; the router products run on the tensor cores over exact three-term
+bfloat16 splits of their float32 operands (or, with SWITCH_FLAG_SIMT_ROUTER,
+as float32 FMA kernels).  The tolerance is derived from that
 arithmetic, element by element: every gradient must lie within twice the
 first-order floating-point error bound of its computation (for each dot
 product, the unit roundoffs of its rounded operands plus K float32 roundings,
@@ -37,13 +39,13 @@ def lib():
     return sm.lib()
 
 
-def run_backward(orc, inp, C, g_aux, seed, check_bias=True):
+def run_backward(orc, inp, C, g_aux, seed, check_bias=True, flags=0):
     T, d = inp["x"].shape
     rng = np.random.default_rng(seed)
     dy = rng.standard_normal((T, d)).astype(np.float32)
     dev = {k: to_device(v) for k, v in inp.items()}
     fwd = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, logit_bias=dev["bias"],
-                       flags=sm.SWITCH_FLAG_TRAINING)
+                       flags=sm.SWITCH_FLAG_TRAINING | flags)
     g = sm.layer_bwd(fwd, dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], torch.from_numpy(dy).cuda(), g_aux,
                      logit_bias=dev["bias"])
     assert sm.switch_check(fwd["workspace"]) == 0
@@ -98,6 +100,8 @@ EDGE = [
     ("capacity_one", 400, 64, 128, 6, 1, 0.0),
     ("aux_only_weight", 500, 64, 64, 4, 200, 3.0),
     ("many_experts", 2000, 64, 128, 70, 40, 0.01),
+    # tensor-core dW_r over 61 chunks of 1152 tokens (ragged last chunk), dx over 274 row tiles
+    ("many_token_chunks", 70000, 64, 64, 70, 1300, 0.01),
 ]
 
 
@@ -108,6 +112,24 @@ def test_backward_edge_cases(orc, case):
     rep, fwd, g = run_backward(orc, inp, C, g_aux, 7)
     if N == 1:  # one expert: p = 1 identically, no router gradient at all
         assert torch.all(g["dw_r"] == 0) and torch.all(g["dbias"] == 0)
+
+
+@pytest.mark.parametrize("name,T", [("base128_skew", 3000), ("base8", 600)])
+def test_backward_simt_router(orc, name, T):
+    """The float32 FMA router products (SWITCH_FLAG_SIMT_ROUTER) against the oracle, and against the
+    tensor-core router products on the same inputs: both within their bounds, the expert-path
+    gradients identical (the flag changes only the router's kernels)."""
+    wl = synth.WORKLOADS[name]
+    C = sm.switch_capacity(T, wl.num_experts, wl.capacity_factor)
+    x = synth.activations(wl, T=T)
+    w_r, bias = synth.router_weight(wl), synth.router_bias(wl)
+    used = np.flatnonzero(np.minimum(orc.route(x, w_r, bias, capacity=C)["counts"], C) > 0)
+    w_in, w_out = synth.all_expert_weights(wl, experts=used)
+    inp = dict(x=x, w_r=w_r, bias=bias, w_in=w_in, w_out=w_out)
+    _, _, g_simt = run_backward(orc, inp, C, 0.01, 5, flags=sm.SWITCH_FLAG_SIMT_ROUTER)
+    _, _, g_tc = run_backward(orc, inp, C, 0.01, 5)
+    for k in ("dw_in", "dw_out"):
+        assert torch.equal(g_simt[k], g_tc[k]), k
 
 
 def exact_problem(rng, T=400, d=128, F=192, N=4):
