@@ -554,15 +554,17 @@ def time_backward(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, dev
         raise RuntimeError("device status after the backward steps")
     K = int(np.minimum(fwd["counts"].cpu().numpy(), C).sum())
     s = x.element_size()
-    Cp = -(-C // 64) * 64
     per_kernel: dict[str, list[float]] = {}
     for name, kms in trace:
         per_kernel.setdefault(name, []).append(kms)
     Np = -(-N // 64) * 64
     Tc = max(256, -(-(-(-T // 64)) // 128) * 128)                       # tokens per dW_r chunk
     chunks = -(-T // Tc)
-    # bytes of the transposes per step: two weights, four activation buffers, x in chunks of tokens
-    transposes = 2 * (2 * N * d * F * s + N * Cp * (2 * d + 2 * F) * s) + T * d * s + chunks * Tc * d * s
+    # bytes of the one transpose per step: x, in chunks of tokens (read T rows, write whole chunks)
+    transposes = T * d * s + chunks * Tc * d * s
+    kept_e = np.minimum(fwd["counts"].cpu().numpy().astype(np.int64), C)
+    tails = np.where(kept_e > 0, np.minimum(C, -(-kept_e // 64) * 64) - kept_e, 0)
+    zero_tails = int(tails.sum()) * (2 * d + 2 * F) * s  # rows zeroed in dE, xbuf, H and dZ
     # the router operand splits: dh -> [T][6 Np] and W_r -> [d][6 Np] (dx), dh -> [3N][chunk tokens] (dW_r)
     splits = (4 * T * N + 2 * T * 6 * Np) + (4 * N * d + 2 * d * 6 * Np) + (4 * T * N + 2 * 3 * N * chunks * Tc)
     work = {
@@ -582,8 +584,8 @@ def time_backward(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, dev
     kernels = {}
     for name, times in per_kernel.items():
         n_per_step = len(times) // steps
-        if name in ("bwd_transpose", "bwd_router_split"):
-            total = transposes if name == "bwd_transpose" else splits
+        if name in ("bwd_transpose", "bwd_router_split", "bwd_zero_tails"):
+            total = {"bwd_transpose": transposes, "bwd_router_split": splits, "bwd_zero_tails": zero_tails}[name]
             kernels[name] = kernel_entry("hbm", total / max(n_per_step, 1), None, statistics.mean(times),
                                          n_per_step, peaks)
             continue

@@ -20,12 +20,15 @@
 //                                         on the split dh, + fixed-order reduce)
 // With SWITCH_FLAG_SIMT_ROUTER the two router products run as float32 FMA
 // kernels instead (router_dx_kernel, router_dw_kernel).
-// The expert GEMMs are the forward's grouped "A . B^T" kernel with both
-// operands K-major: the weights and the per-expert activation buffers are
-// first transposed in HBM (batched 64 x 64 tile transposes; rows past an
-// expert's kept tokens become zeros, so the weight-gradient GEMMs only see
-// kept tokens).  Every reduction runs in a fixed order: identical inputs give
-// identical bytes.
+// The expert GEMMs are the forward's grouped "A . B^T" pair kernel reading
+// the weights and the per-expert activation buffers where they lie, as
+// MN-major operands where the contraction runs along their rows (W_out and
+// W_in for dZ and dx; dE, H, dZ and xbuf along the tokens for the weight
+// gradients), so nothing is transposed in HBM; rows past an expert's kept
+// tokens up to the next multiple of 64 are zeroed first, so the
+// weight-gradient GEMMs only see kept tokens.  The one transpose left is x
+// per chunk of tokens for the tensor-core dW_r.  Every reduction runs in a
+// fixed order: identical inputs give identical bytes.
 #include <cuda.h>
 
 #include <algorithm>
@@ -391,7 +394,28 @@ __global__ void router_dw_reduce_kernel(const float *__restrict__ part, int chun
     }
 }
 
-int64_t round_up64(int64_t v) { return (v + 63) / 64 * 64; }
+// The weight-gradient GEMMs read the token-indexed buffers dE, H, dZ and
+// xbuf along K = tokens in blocks of 64: block (expert e, row r) zeroes row
+// kept_e + r of each of them when that row lies below both C and kept_e
+// rounded up to 64 (those rows hold values of no token).
+__global__ void __launch_bounds__(256) zero_tails_kernel(const int32_t *__restrict__ counts, int C, int d, int F,
+                                                        uint16_t *__restrict__ grad_e, uint16_t *__restrict__ xbuf,
+                                                        uint16_t *__restrict__ hidden, uint16_t *__restrict__ grad_z) {
+    const int e = blockIdx.x;
+    const int kept = min(counts[e], C);
+    const int row = kept + (int)blockIdx.y;
+    if (kept == 0 || row >= C || row >= (kept + 63) / 64 * 64) return;
+    const int64_t r = (int64_t)e * C + row;
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int w = threadIdx.x; w < d / 8; w += blockDim.x) {
+        reinterpret_cast<uint4 *>(grad_e + r * d)[w] = z;
+        reinterpret_cast<uint4 *>(xbuf + r * d)[w] = z;
+    }
+    for (int w = threadIdx.x; w < F / 8; w += blockDim.x) {
+        reinterpret_cast<uint4 *>(hidden + r * F)[w] = z;
+        reinterpret_cast<uint4 *>(grad_z + r * F)[w] = z;
+    }
+}
 
 cudaError_t launch_transpose(int32_t kernel_id, const void *in, void *out, int B, int R, int Cc, int Rp,
                              const int32_t *counts, int cap, cudaStream_t stream) {
@@ -432,7 +456,6 @@ cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const flo
                              float *dw_in, float *dw_out, const Workspace &ws, cudaStream_t stream) {
     const int64_t T = dims.T;
     const int N = dims.num_experts, C = dims.capacity, d = dims.d_model, F = dims.d_ff;
-    const int64_t Cp = round_up64(C);
     DeviceStatus *st = static_cast<DeviceStatus *>(ws.status);
     cudaError_t err = cudaMemsetAsync(ws.status, 0, sizeof(DeviceStatus), stream);
     // weight gradients of experts without kept tokens are zero; the GEMMs write the others
@@ -452,13 +475,16 @@ cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const flo
     err = cudaGetLastError();
     launch_end(stream);
     if (err != cudaSuccess) return err;
-    // 2. transposed weights: W_out^T [N][F][d], W_in^T [N][d][F]
-    if ((err = launch_transpose(K_BWD_TRANSPOSE, w_out, ws.w_out_t, N, d, F, d, nullptr, 0, stream)) != cudaSuccess)
-        return err;
-    if ((err = launch_transpose(K_BWD_TRANSPOSE, w_in, ws.w_in_t, N, F, d, F, nullptr, 0, stream)) != cudaSuccess)
-        return err;
-    // 3. dZ = (dE W_out) masked by the forward's ReLU: [N][C][F] bf16
-    err = launch_ffn_tc_bwd_dz(dims, ws.grad_e, ws.w_out_t, counts, ws.grad_z, ws.hidden, st, stream);
+    // 2. dZ = (dE W_out) masked by the forward's ReLU: [N][C][F] bf16 (W_out read as it is stored)
+    err = launch_ffn_tc_bwd_dz(dims, ws.grad_e, w_out, counts, ws.grad_z, ws.hidden, st, stream);
+    if (err != cudaSuccess) return err;
+    // 3. zero rows past each expert's kept tokens up to the next 64 (the dW GEMMs' last K block)
+    launch_begin(K_BWD_ZERO_TAILS, stream);
+    zero_tails_kernel<<<dim3((unsigned)N, 64), 256, 0, stream>>>(
+        counts, C, d, F, static_cast<uint16_t *>(ws.grad_e), static_cast<uint16_t *>(ws.xbuf),
+        static_cast<uint16_t *>(ws.hidden), static_cast<uint16_t *>(ws.grad_z));
+    err = cudaGetLastError();
+    launch_end(stream);
     if (err != cudaSuccess) return err;
     // 4. dx = dh W_r (all rows), then + dZ W_in for kept rows
     const bool simt_router = (dims.flags & SWITCH_FLAG_SIMT_ROUTER) != 0;
@@ -489,27 +515,14 @@ cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const flo
                                       stream);
         if (err != cudaSuccess) return err;
     }
-    err = launch_ffn_tc_bwd_dx(dims, ws.grad_z, ws.w_in_t, counts, ws.slot_token, dx, st, stream);
+    err = launch_ffn_tc_bwd_dx(dims, ws.grad_z, w_in, counts, ws.slot_token, dx, st, stream);
     if (err != cudaSuccess) return err;
-    // 5. transposed activations (rows past each expert's kept tokens zeroed)
-    if ((err = launch_transpose(K_BWD_TRANSPOSE, ws.grad_e, ws.grad_e_t, N, C, d, (int)Cp, counts, C, stream)) !=
-        cudaSuccess)
-        return err;
-    if ((err = launch_transpose(K_BWD_TRANSPOSE, ws.hidden, ws.hidden_t, N, C, F, (int)Cp, counts, C, stream)) !=
-        cudaSuccess)
-        return err;
-    if ((err = launch_transpose(K_BWD_TRANSPOSE, ws.xbuf, ws.xbuf_t, N, C, d, (int)Cp, counts, C, stream)) !=
-        cudaSuccess)
-        return err;
-    if ((err = launch_transpose(K_BWD_TRANSPOSE, ws.grad_z, ws.grad_z_t, N, C, F, (int)Cp, counts, C, stream)) !=
-        cudaSuccess)
-        return err;
-    // 6. dW_out = dE^T H, dW_in = dZ^T x over each expert's kept tokens
-    err = launch_ffn_tc_bwd_dw(dims, ws.grad_e_t, ws.hidden_t, counts, d, F, (int)Cp, dw_out, st, stream);
+    // 5. dW_out = dE^T H, dW_in = dZ^T x over each expert's kept tokens (token-major operands)
+    err = launch_ffn_tc_bwd_dw(dims, ws.grad_e, ws.hidden, counts, d, F, dw_out, st, stream);
     if (err != cudaSuccess) return err;
-    err = launch_ffn_tc_bwd_dw(dims, ws.grad_z_t, ws.xbuf_t, counts, F, d, (int)Cp, dw_in, st, stream);
+    err = launch_ffn_tc_bwd_dw(dims, ws.grad_z, ws.xbuf, counts, F, d, dw_in, st, stream);
     if (err != cudaSuccess) return err;
-    // 7. dW_r and d bias: chunk partials, then a fixed-order sum
+    // 6. dW_r and d bias: chunk partials, then a fixed-order sum
     if (!simt_router) {
         launch_begin(K_BWD_ROUTER_SPLIT, stream);
         router_dw_a_kernel<<<dim3((unsigned)chunks_tc, (unsigned)((N + 31) / 32)), 256, 0, stream>>>(

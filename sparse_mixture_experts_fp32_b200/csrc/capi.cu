@@ -26,7 +26,7 @@ int64_t tiles_of(const switch_dims_t &d) { return (d.T + kTileT - 1) / kTileT; }
 
 struct Sections {
     size_t status, ticket, hist, psum, tile_off, prob_total, w_split, slot_token, xbuf, ybuf, hidden, done, hist2,
-        tile_off2, counts_first, ent, probs, dh, grad_e, grad_z, w_out_t, w_in_t, grad_e_t, hidden_t, xbuf_t, grad_z_t,
+        tile_off2, counts_first, ent, probs, dh, grad_e, grad_z,
         dw_part, db_part, rdx_a, rdx_b, rdw_a, x_t, chunk_counts, total;
 };
 
@@ -58,17 +58,11 @@ Sections layout(const switch_dims_t &d) {
     s.ent = take(tiles * 4);
     if (d.flags & SWITCH_FLAG_TRAINING) {  // kept by the training forward, used by the backward pass
         const size_t T = (size_t)d.T, dm = (size_t)d.d_model, F = (size_t)d.d_ff, es = elem_size(d);
-        const size_t Cp = (C + 63) / 64 * 64, chunks = (size_t)router_dw_chunks(d.T);
+        const size_t chunks = (size_t)router_dw_chunks(d.T);
         s.probs = take(T * N * 4);
         s.dh = take(T * N * 4);
         s.grad_e = take(N * C * dm * es);
         s.grad_z = take(N * C * F * es);
-        s.w_out_t = take(N * F * dm * es);
-        s.w_in_t = take(N * dm * F * es);
-        s.grad_e_t = take(N * dm * Cp * es);
-        s.hidden_t = take(N * F * Cp * es);
-        s.xbuf_t = take(N * dm * Cp * es);
-        s.grad_z_t = take(N * F * Cp * es);
         if (d.flags & SWITCH_FLAG_SIMT_ROUTER) {  // float32 FMA router products
             s.dw_part = take(chunks * N * dm * 4);
             s.db_part = take(chunks * N * 4);
@@ -210,12 +204,6 @@ Workspace carve_workspace(const switch_dims_t &dims, void *base) {
     w.dh = static_cast<float *>(at(s.dh));
     w.grad_e = at(s.grad_e);
     w.grad_z = at(s.grad_z);
-    w.w_out_t = at(s.w_out_t);
-    w.w_in_t = at(s.w_in_t);
-    w.grad_e_t = at(s.grad_e_t);
-    w.hidden_t = at(s.hidden_t);
-    w.xbuf_t = at(s.xbuf_t);
-    w.grad_z_t = at(s.grad_z_t);
     w.dw_part = static_cast<float *>(at(s.dw_part));
     w.db_part = static_cast<float *>(at(s.db_part));
     w.rdx_a = at(s.rdx_a);
@@ -604,6 +592,7 @@ const char *switch_kernel_name(int32_t id) {
         case K_BWD_ROUTER_SPLIT: return "bwd_router_split";
         case K_BWD_ROUTER_TC_DX: return "bwd_router_tc_dx";
         case K_BWD_ROUTER_TC_DW: return "bwd_router_tc_dw";
+        case K_BWD_ZERO_TAILS: return "bwd_zero_tails";
     }
     return "?";
 }

@@ -393,6 +393,22 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(const void *tile) {
     return desc;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile written by TMA
+// with 128-byte swizzling: each 64-element (128-byte) slice of the M (or N)
+// extent holds its K rows at a 128-byte pitch (8-row swizzle atoms of 1024
+// bytes along K), and the slices lie `slice_bytes` apart.  The tile base must
+// be 1024-aligned.  Advancing K by 16 moves the start by two atoms (2048 bytes).
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(const void *tile, uint32_t slice_bytes) {
+    const uint64_t addr = smem_u32(tile);
+    uint64_t desc = 0;
+    desc |= (addr >> 4) & 0x3FFFull;                  // start address
+    desc |= (uint64_t)((slice_bytes >> 4) & 0x3FFFu) << 16;  // leading byte offset: next 64-element MN slice
+    desc |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset: next 8-row group along K
+    desc |= (uint64_t)1 << 46;                        // descriptor version for sm_100
+    desc |= (uint64_t)2 << 61;                        // layout: 128-byte swizzle
+    return desc;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A and B (both K-major) and
 // an fp32 accumulator of shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
@@ -401,6 +417,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            | (1u << 10)                    // B format: bf16
            | ((uint32_t)(N >> 3) << 17)    // N / 8
            | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// The same with A and/or B stored MN-major (M or N contiguous in shared memory).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+    return idesc_bf16_f32(M, N) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
 }
 
 // ---------------------------------------------------------------------------

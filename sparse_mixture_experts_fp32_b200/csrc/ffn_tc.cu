@@ -473,7 +473,13 @@ __device__ __forceinline__ int group_rows(const GroupShape &g, int kept) {
     return g.rows_fixed > 0 ? (kept > 0 ? g.rows_fixed : 0) : kept;
 }
 
-template <int BN, int STAGES, int EPI>
+// Operand storage of the pair GEMM: K-major (K contiguous, the forward's
+// layout) or MN-major (M resp. N contiguous: the backward reads activations
+// and weights in their forward layout, no transposes).  MN-major operands
+// are loaded as two 64-element-wide TMA boxes per CTA and stage.
+enum OperandMajor : int { kMajK = 0, kMajAmn = 1, kMajBmn = 2 };
+
+template <int BN, int STAGES, int EPI, int MAJ = kMajK>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                          const __grid_constant__ CUtensorMap tmap_out, void *__restrict__ out,
@@ -482,6 +488,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                          DeviceStatus *status, const GroupShape shape) {
     using L = PairLayout<BN, STAGES>;
     constexpr int BMP = 2 * BM;  // rows of a pair tile
+    constexpr bool kAmn = (MAJ & kMajAmn) != 0, kBmn = (MAJ & kMajBmn) != 0;
+    static_assert(!kAmn || BM == 128, "MN-major A: two 64-row boxes per CTA");
+    static_assert(!kBmn || BN == 256, "MN-major B: two 64-column boxes per CTA");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
@@ -574,10 +583,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * (L::a_bytes + L::b_bytes)));
                     const uint32_t leader_full = map_to_rank(&full[stage], 0);
-                    tma_load_3d_pair(sA + stage * L::a_bytes, &tmap_a, leader_full, kb * BK,
-                                     m * BMP + (int)rank * BM, e);
-                    tma_load_3d_pair(sB + stage * L::b_bytes, &tmap_b, leader_full, kb * BK,
-                                     n * BN + (int)rank * (BN / 2), e);
+                    const int a_row = m * BMP + (int)rank * BM, b_row = n * BN + (int)rank * (BN / 2);
+                    if (kAmn) {  // A stored [E][K][M]: this CTA's 128 rows as two 64-row slices of 8 KB
+                        tma_load_3d_pair(sA + stage * L::a_bytes, &tmap_a, leader_full, a_row, kb * BK, e);
+                        tma_load_3d_pair(sA + stage * L::a_bytes + L::a_bytes / 2, &tmap_a, leader_full,
+                                         a_row + 64, kb * BK, e);
+                    } else {
+                        tma_load_3d_pair(sA + stage * L::a_bytes, &tmap_a, leader_full, kb * BK, a_row, e);
+                    }
+                    if (kBmn) {  // B stored [E][K][N]: this CTA's 128 columns as two 64-column slices
+                        tma_load_3d_pair(sB + stage * L::b_bytes, &tmap_b, leader_full, b_row, kb * BK, e);
+                        tma_load_3d_pair(sB + stage * L::b_bytes + L::b_bytes / 2, &tmap_b, leader_full,
+                                         b_row + 64, kb * BK, e);
+                    } else {
+                        tma_load_3d_pair(sB + stage * L::b_bytes, &tmap_b, leader_full, kb * BK, b_row, e);
+                    }
                     issued |= 1u << stage;
                     parity_of = (parity_of & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -593,7 +613,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BMP, BN);
+            constexpr uint32_t idesc = idesc_bf16_f32_major(BMP, BN, kAmn, kBmn);
+            // per 16-element K step: +32 bytes inside a K-major row, +2048 bytes (two 8-row
+            // groups) in an MN-major slice; descriptor start addresses count 16-byte units
+            constexpr uint64_t a_step = kAmn ? 128 : 2, b_step = kBmn ? 128 : 2;
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -615,11 +638,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t a_desc = smem_desc_sw128(sA + stage * L::a_bytes);
-                    const uint64_t b_desc = smem_desc_sw128(sB + stage * L::b_bytes);
+                    const uint64_t a_desc = kAmn ? smem_desc_sw128_mn(sA + stage * L::a_bytes, L::a_bytes / 2)
+                                                 : smem_desc_sw128(sA + stage * L::a_bytes);
+                    const uint64_t b_desc = kBmn ? smem_desc_sw128_mn(sB + stage * L::b_bytes, L::b_bytes / 2)
+                                                 : smem_desc_sw128(sB + stage * L::b_bytes);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        tc_mma_bf16_pair(d_tmem, a_desc + (uint64_t)(2 * k), b_desc + (uint64_t)(2 * k), idesc,
+                        tc_mma_bf16_pair(d_tmem, a_desc + a_step * (uint64_t)k, b_desc + b_step * (uint64_t)k, idesc,
                                          (kb | k) != 0 ? 1u : 0u);
                     tc_commit_both(&empty[stage]);
                     if (++stage == STAGES) {
@@ -1109,23 +1134,26 @@ cudaError_t launch_gemm(int32_t kernel_id, const void *a, const void *b, void *o
     return err;
 }
 
-// A [E][a_rows][K] and B [E][Nout][K] (bf16, K contiguous); a_rows = C unless
-// the shape has fixed rows (then A holds rows_fixed rows per expert and K is
-// the padded token count).
-template <int BN, int STAGES, int EPI>
+// A [E][a_rows][K] and B [E][Nout][K] (bf16, K contiguous), or with MAJ
+// MN-major A [E][K][a_rows] and/or B [E][K][Nout]; a_rows = C unless the shape
+// has fixed rows (then A holds rows_fixed rows per expert and K is the token
+// extent of the operands, read up to each expert's kept tokens).
+template <int BN, int STAGES, int EPI, int MAJ = kMajK>
 cudaError_t launch_gemm_pair(int32_t kernel_id, const void *a, const void *b, void *out, const int32_t *counts, int E,
                              int C, int K, int Nout, int64_t T, const int32_t *slot_token, const float *gate,
                              DeviceStatus *status, cudaStream_t stream, GroupShape shape = GroupShape{0, 0, 0, nullptr}) {
     const int a_rows = shape.rows_fixed > 0 ? shape.rows_fixed : C;
     CUtensorMap ta, tb, tout;
-    if (!make_tmap(&ta, a, E, a_rows, K, BM) || !make_tmap(&tb, b, E, Nout, K, BN / 2)) return cudaErrorInvalidValue;
+    const bool ok_a = (MAJ & kMajAmn) ? make_tmap(&ta, a, E, K, a_rows, 64) : make_tmap(&ta, a, E, a_rows, K, BM);
+    const bool ok_b = (MAJ & kMajBmn) ? make_tmap(&tb, b, E, K, Nout, 64) : make_tmap(&tb, b, E, Nout, K, BN / 2);
+    if (!ok_a || !ok_b) return cudaErrorInvalidValue;
     memset(&tout, 0, sizeof tout);
     if ((EPI == kEpiHiddenRelu || EPI == kEpiReluGrad) && !make_tmap(&tout, out, E, C, Nout, 32))
         return cudaErrorInvalidValue;
     if (EPI == kEpiWeightGrad && (shape.rows_fixed <= 0 || !make_tmap_f32_box32(&tout, out, E, shape.rows_fixed, Nout)))
         return cudaErrorInvalidValue;
     const size_t smem = PairLayout<BN, STAGES>::bytes(E);
-    auto kern = tc_grouped_gemm_pair<BN, STAGES, EPI>;
+    auto kern = tc_grouped_gemm_pair<BN, STAGES, EPI, MAJ>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     const int64_t m_tiles =
@@ -1178,34 +1206,37 @@ cudaError_t launch_ffn_fused(const switch_dims_t &dims, const void *xbuf, const 
 
 }  // namespace
 
-// Backward GEMMs (SM pairs, 256 x 256 tiles, the forward's kernel).
-// dZ [N][C][F] = bf16((dE W_out) where H > 0): A = dE [N][C][d], B = W_out^T [N][F][d].
-cudaError_t launch_ffn_tc_bwd_dz(const switch_dims_t &dims, const void *grad_e, const void *w_out_t,
+// Backward GEMMs (SM pairs, 256 x 256 tiles, the forward's kernel; weights and
+// activations read in their forward layout as MN-major operands).
+// dZ [N][C][F] = bf16((dE W_out) where H > 0): A = dE [N][C][d] (K-major),
+// B = W_out [N][d][F] (K = d rows, N = F contiguous).
+cudaError_t launch_ffn_tc_bwd_dz(const switch_dims_t &dims, const void *grad_e, const void *w_out,
                                  const int32_t *counts, void *grad_z, const void *hidden, DeviceStatus *st,
                                  cudaStream_t stream) {
-    return launch_gemm_pair<256, 6, kEpiReluGrad>(K_BWD_GEMM_DZ, grad_e, w_out_t, grad_z, counts, dims.num_experts,
-                                                  dims.capacity, dims.d_model, dims.d_ff, dims.T, nullptr, nullptr,
-                                                  st, stream,
-                                                  GroupShape{0, 0, 0, static_cast<const uint16_t *>(hidden)});
+    return launch_gemm_pair<256, 6, kEpiReluGrad, kMajBmn>(
+        K_BWD_GEMM_DZ, grad_e, w_out, grad_z, counts, dims.num_experts, dims.capacity, dims.d_model, dims.d_ff,
+        dims.T, nullptr, nullptr, st, stream, GroupShape{0, 0, 0, static_cast<const uint16_t *>(hidden)});
 }
 
-// dx[slot_token] += dZ W_in: A = dZ [N][C][F], B = W_in^T [N][d][F].
-cudaError_t launch_ffn_tc_bwd_dx(const switch_dims_t &dims, const void *grad_z, const void *w_in_t,
+// dx[slot_token] += dZ W_in: A = dZ [N][C][F] (K-major), B = W_in [N][F][d]
+// (K = F rows, N = d contiguous).
+cudaError_t launch_ffn_tc_bwd_dx(const switch_dims_t &dims, const void *grad_z, const void *w_in,
                                  const int32_t *counts, const int32_t *slot_token, float *dx, DeviceStatus *st,
                                  cudaStream_t stream) {
-    return launch_gemm_pair<256, 6, kEpiScatterAdd>(K_BWD_GEMM_DX, grad_z, w_in_t, dx, counts, dims.num_experts,
-                                                    dims.capacity, dims.d_ff, dims.d_model, dims.T, slot_token,
-                                                    nullptr, st, stream);
+    return launch_gemm_pair<256, 6, kEpiScatterAdd, kMajBmn>(K_BWD_GEMM_DX, grad_z, w_in, dx, counts,
+                                                             dims.num_experts, dims.capacity, dims.d_ff, dims.d_model,
+                                                             dims.T, slot_token, nullptr, st, stream);
 }
 
-// Weight gradient out [N][rows][nout] (fp32) = A^T-free form A . B^T over each
-// expert's kept tokens: A [N][rows][Kp], B [N][nout][Kp] (token-contiguous,
-// zero past the kept tokens).
-cudaError_t launch_ffn_tc_bwd_dw(const switch_dims_t &dims, const void *a_t, const void *b_t, const int32_t *counts,
-                                 int rows, int nout, int Kp, float *out, DeviceStatus *st, cudaStream_t stream) {
-    return launch_gemm_pair<256, 6, kEpiWeightGrad>(K_BWD_GEMM_DW, a_t, b_t, out, counts, dims.num_experts,
-                                                   dims.capacity, Kp, nout, dims.T, nullptr, nullptr, st, stream,
-                                                   GroupShape{rows, 1, rows, nullptr});
+// Weight gradient out [N][rows][nout] (fp32) = sum over each expert's kept
+// tokens s of a[s] b[s]^T: A [N][C][rows] and B [N][C][nout], both read
+// MN-major (token rows, K = the tokens; rows from the expert's kept count up
+// to the next multiple of 64 must hold zeros, rows past C read as zeros).
+cudaError_t launch_ffn_tc_bwd_dw(const switch_dims_t &dims, const void *a, const void *b, const int32_t *counts,
+                                 int rows, int nout, float *out, DeviceStatus *st, cudaStream_t stream) {
+    return launch_gemm_pair<256, 6, kEpiWeightGrad, kMajAmn | kMajBmn>(
+        K_BWD_GEMM_DW, a, b, out, counts, dims.num_experts, dims.capacity, dims.capacity, nout, dims.T, nullptr,
+        nullptr, st, stream, GroupShape{rows, 1, rows, nullptr});
 }
 
 // Router part of dx (float32 [T][d], overwritten) = A . B^T with A [T][K] the

@@ -46,6 +46,7 @@ enum KernelId : int32_t {
     K_BWD_ROUTER_SPLIT = 29,
     K_BWD_ROUTER_TC_DX = 30,
     K_BWD_ROUTER_TC_DW = 31,
+    K_BWD_ZERO_TAILS = 32,
 };
 
 struct Workspace {
@@ -71,12 +72,6 @@ struct Workspace {
     float *dh;           // [T][N] gradient of the router logits
     void *grad_e;        // [N][C][d] bf16 gate * dy in expert order
     void *grad_z;        // [N][C][F] bf16 gradient of the pre-activations
-    void *w_out_t;       // [N][F][d] bf16 W_out transposed
-    void *w_in_t;        // [N][d][F] bf16 W_in transposed
-    void *grad_e_t;      // [N][d][Cp] bf16 (Cp = C rounded up to 64; zero past the kept tokens)
-    void *hidden_t;      // [N][F][Cp] bf16
-    void *xbuf_t;        // [N][d][Cp] bf16
-    void *grad_z_t;      // [N][F][Cp] bf16
     float *dw_part;      // [chunks][N][d] partial sums of dW_r
     float *db_part;      // [chunks][N] partial sums of d bias
     void *rdx_a;         // [T][6 Np] bf16 split dh terms (tensor-core router dx)
@@ -161,14 +156,14 @@ cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const flo
                              const void *w_out, const int32_t *expert, const float *gate, const int32_t *slot,
                              const int32_t *counts, const float *dy, float g_aux, float *dx, float *dw_r, float *dbias,
                              float *dw_in, float *dw_out, const Workspace &ws, cudaStream_t stream);
-cudaError_t launch_ffn_tc_bwd_dz(const switch_dims_t &dims, const void *grad_e, const void *w_out_t,
+cudaError_t launch_ffn_tc_bwd_dz(const switch_dims_t &dims, const void *grad_e, const void *w_out,
                                  const int32_t *counts, void *grad_z, const void *hidden, DeviceStatus *st,
                                  cudaStream_t stream);
-cudaError_t launch_ffn_tc_bwd_dx(const switch_dims_t &dims, const void *grad_z, const void *w_in_t,
+cudaError_t launch_ffn_tc_bwd_dx(const switch_dims_t &dims, const void *grad_z, const void *w_in,
                                  const int32_t *counts, const int32_t *slot_token, float *dx, DeviceStatus *st,
                                  cudaStream_t stream);
-cudaError_t launch_ffn_tc_bwd_dw(const switch_dims_t &dims, const void *a_t, const void *b_t, const int32_t *counts,
-                                 int rows, int nout, int Kp, float *out, DeviceStatus *st, cudaStream_t stream);
+cudaError_t launch_ffn_tc_bwd_dw(const switch_dims_t &dims, const void *a, const void *b, const int32_t *counts,
+                                 int rows, int nout, float *out, DeviceStatus *st, cudaStream_t stream);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
