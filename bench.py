@@ -560,8 +560,6 @@ def time_backward(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, dev
     Np = -(-N // 64) * 64
     Tc = max(256, -(-(-(-T // 64)) // 128) * 128)                       # tokens per dW_r chunk
     chunks = -(-T // Tc)
-    # bytes of the one transpose per step: x, in chunks of tokens (read T rows, write whole chunks)
-    transposes = T * d * s + chunks * Tc * d * s
     kept_e = np.minimum(fwd["counts"].cpu().numpy().astype(np.int64), C)
     tails = np.where(kept_e > 0, np.minimum(C, -(-kept_e // 64) * 64) - kept_e, 0)
     zero_tails = int(tails.sum()) * (2 * d + 2 * F) * s  # rows zeroed in dE, xbuf, H and dZ
@@ -584,8 +582,8 @@ def time_backward(args, sm, wl, x, w_r, bias, w_in, w_out, C, flush, stream, dev
     kernels = {}
     for name, times in per_kernel.items():
         n_per_step = len(times) // steps
-        if name in ("bwd_transpose", "bwd_router_split", "bwd_zero_tails"):
-            total = {"bwd_transpose": transposes, "bwd_router_split": splits, "bwd_zero_tails": zero_tails}[name]
+        if name in ("bwd_router_split", "bwd_zero_tails"):
+            total = splits if name == "bwd_router_split" else zero_tails
             kernels[name] = kernel_entry("hbm", total / max(n_per_step, 1), None, statistics.mean(times),
                                          n_per_step, peaks)
             continue

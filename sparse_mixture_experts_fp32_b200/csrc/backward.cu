@@ -24,11 +24,11 @@
 // the weights and the per-expert activation buffers where they lie, as
 // MN-major operands where the contraction runs along their rows (W_out and
 // W_in for dZ and dx; dE, H, dZ and xbuf along the tokens for the weight
-// gradients), so nothing is transposed in HBM; rows past an expert's kept
-// tokens up to the next multiple of 64 are zeroed first, so the
-// weight-gradient GEMMs only see kept tokens.  The one transpose left is x
-// per chunk of tokens for the tensor-core dW_r.  Every reduction runs in a
-// fixed order: identical inputs give identical bytes.
+// gradients; x along its tokens for the tensor-core dW_r), so nothing is
+// transposed in HBM; rows past an expert's kept tokens up to the next
+// multiple of 64 are zeroed first, so the weight-gradient GEMMs only see kept
+// tokens.  Every reduction runs in a fixed order: identical inputs give
+// identical bytes.
 #include <cuda.h>
 
 #include <algorithm>
@@ -88,52 +88,6 @@ __global__ void __launch_bounds__(kThreads) bwd_token_kernel(const float *__rest
     for (int i = lane; i < N; i += 32) {
         const float dp = (i == e ? g : 0.f) + c_aux * (float)counts[i];
         dh[t * N + i] = pt[i] * (dp - dot);
-    }
-}
-
-// Batched transpose of bf16 matrices: in [B][R][Cc] -> out [B][Cc][Rp].
-// Rows r >= valid(b) of the input (valid = min(counts[b], cap) when counts is
-// given, else R) and the padding rows up to Rp become zeros.  64 x 64 tiles
-// through shared memory (rows padded to 33 words), 16-byte global loads and
-// stores on both sides; Cc and Rp are multiples of 8 (checked by the launcher).
-constexpr int kTT = 64;
-__global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t *__restrict__ in, uint16_t *__restrict__ out,
-                                                            int R, int Cc, int Rp, const int32_t *__restrict__ counts,
-                                                            int cap) {
-    __shared__ uint32_t tile[kTT][kTT / 2 + 1];  // [row][column pair]
-    const int b = blockIdx.z;
-    const int c0 = blockIdx.x * kTT, r0 = blockIdx.y * kTT;
-    const int tid = threadIdx.x;
-    const int valid = counts ? min(min(counts[b], cap), R) : R;
-    const uint16_t *src = in + (int64_t)b * R * Cc;
-    uint16_t *dst = out + (int64_t)b * Cc * Rp;
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {  // 64 rows x 8 chunks of 8 elements
-        const int idx = tid + 256 * j;
-        const int r = idx >> 3, ch = idx & 7;
-        const int c = c0 + ch * 8;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r0 + r < valid && c < Cc) v = __ldg(reinterpret_cast<const uint4 *>(src + (int64_t)(r0 + r) * Cc + c));
-        tile[r][ch * 4 + 0] = v.x;
-        tile[r][ch * 4 + 1] = v.y;
-        tile[r][ch * 4 + 2] = v.z;
-        tile[r][ch * 4 + 3] = v.w;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {  // 64 output rows x 8 chunks of 8 input rows
-        const int idx = tid + 256 * j;
-        const int c = idx >> 3, rb = idx & 7;
-        if (c0 + c >= Cc || r0 + rb * 8 >= Rp) continue;
-        const int shift = (c & 1) * 16;
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t lo = (tile[rb * 8 + 2 * q][c >> 1] >> shift) & 0xffffu;
-            const uint32_t hi = (tile[rb * 8 + 2 * q + 1][c >> 1] >> shift) & 0xffffu;
-            w[q] = lo | (hi << 16);
-        }
-        *reinterpret_cast<uint4 *>(dst + (int64_t)(c0 + c) * Rp + r0 + rb * 8) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -417,17 +371,6 @@ __global__ void __launch_bounds__(256) zero_tails_kernel(const int32_t *__restri
     }
 }
 
-cudaError_t launch_transpose(int32_t kernel_id, const void *in, void *out, int B, int R, int Cc, int Rp,
-                             const int32_t *counts, int cap, cudaStream_t stream) {
-    if (Cc % 8 != 0 || Rp % 8 != 0) return cudaErrorInvalidValue;  // 16-byte rows on both sides
-    const dim3 grid((unsigned)((Cc + kTT - 1) / kTT), (unsigned)((Rp + kTT - 1) / kTT), (unsigned)B);
-    launch_begin(kernel_id, stream);
-    transpose_bf16_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(in), static_cast<uint16_t *>(out),
-                                                    R, Cc, Rp, counts, cap);
-    cudaError_t err = cudaGetLastError();
-    launch_end(stream);
-    return err;
-}
 
 }  // namespace
 
@@ -530,10 +473,7 @@ cudaError_t launch_layer_bwd(const switch_dims_t &dims, const void *x, const flo
         err = cudaGetLastError();
         launch_end(stream);
         if (err != cudaSuccess) return err;
-        if ((err = launch_transpose(K_BWD_TRANSPOSE, x, ws.x_t, (int)chunks_tc, (int)Tc, d, (int)Tc, ws.chunk_counts,
-                                    (int)Tc, stream)) != cudaSuccess)
-            return err;
-        err = launch_router_tc_bwd_dw(ws.rdw_a, ws.x_t, ws.chunk_counts, (int)chunks_tc, 3 * N, (int)Tc, d, T,
+        err = launch_router_tc_bwd_dw(ws.rdw_a, x, ws.chunk_counts, (int)chunks_tc, 3 * N, (int)Tc, d, T,
                                       ws.dw_part, st, stream);
         if (err != cudaSuccess) return err;
         launch_begin(K_BWD_REDUCE, stream);

@@ -27,7 +27,7 @@ int64_t tiles_of(const switch_dims_t &d) { return (d.T + kTileT - 1) / kTileT; }
 struct Sections {
     size_t status, ticket, hist, psum, tile_off, prob_total, w_split, slot_token, xbuf, ybuf, hidden, done, hist2,
         tile_off2, counts_first, ent, probs, dh, grad_e, grad_z,
-        dw_part, db_part, rdx_a, rdx_b, rdw_a, x_t, chunk_counts, total;
+        dw_part, db_part, rdx_a, rdx_b, rdw_a, chunk_counts, total;
 };
 
 Sections layout(const switch_dims_t &d) {
@@ -74,7 +74,6 @@ Sections layout(const switch_dims_t &d) {
             s.rdx_a = take(T * 6 * Np * 2);
             s.rdx_b = take(dm * 6 * Np * 2);
             s.rdw_a = take(ch * 3 * N * Tc * 2);
-            s.x_t = take(ch * dm * Tc * 2);
             s.chunk_counts = take((ch + 1) * 4);
         }
     }
@@ -209,7 +208,6 @@ Workspace carve_workspace(const switch_dims_t &dims, void *base) {
     w.rdx_a = at(s.rdx_a);
     w.rdx_b = at(s.rdx_b);
     w.rdw_a = at(s.rdw_a);
-    w.x_t = at(s.x_t);
     w.chunk_counts = static_cast<int32_t *>(at(s.chunk_counts));
     w.tiles = tiles_of(dims);
     return w;
@@ -580,7 +578,6 @@ const char *switch_kernel_name(int32_t id) {
         case K_FFN_TC_FUSED: return "ffn_tc_fused";
         case K_COMBINE_TOP2: return "combine_top2";
         case K_BWD_TOKEN: return "bwd_gate_softmax";
-        case K_BWD_TRANSPOSE: return "bwd_transpose";
         case K_BWD_GEMM_DZ: return "bwd_tc_gemm_dz";
         case K_BWD_GEMM_DX: return "bwd_tc_gemm_dx";
         case K_BWD_GEMM_DW: return "bwd_tc_gemm_dw";

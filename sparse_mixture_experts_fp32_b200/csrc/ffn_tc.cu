@@ -467,6 +467,8 @@ struct GroupShape {
     int k_per_expert;  // 0: K / BK blocks for every tile
     int out_rows;      // kEpiExpertOut: rows of each expert's block of `out` (0: C)
     const uint16_t *mask_h;  // kEpiReluGrad: the forward's H [E][C][Nout]
+    int b_k_stride;    // MN-major B only: > 0: B is one [T][Nout] matrix and group e's K rows start at
+                       // row e * b_k_stride (groups = consecutive chunks of its rows)
 };
 
 __device__ __forceinline__ int group_rows(const GroupShape &g, int kept) {
@@ -592,9 +594,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         tma_load_3d_pair(sA + stage * L::a_bytes, &tmap_a, leader_full, kb * BK, a_row, e);
                     }
                     if (kBmn) {  // B stored [E][K][N]: this CTA's 128 columns as two 64-column slices
-                        tma_load_3d_pair(sB + stage * L::b_bytes, &tmap_b, leader_full, b_row, kb * BK, e);
+                        const int bk = shape.b_k_stride > 0 ? e * shape.b_k_stride + kb * BK : kb * BK;
+                        const int bz = shape.b_k_stride > 0 ? 0 : e;
+                        tma_load_3d_pair(sB + stage * L::b_bytes, &tmap_b, leader_full, b_row, bk, bz);
                         tma_load_3d_pair(sB + stage * L::b_bytes + L::b_bytes / 2, &tmap_b, leader_full,
-                                         b_row + 64, kb * BK, e);
+                                         b_row + 64, bk, bz);
                     } else {
                         tma_load_3d_pair(sB + stage * L::b_bytes, &tmap_b, leader_full, kb * BK, b_row, e);
                     }
@@ -1145,7 +1149,10 @@ cudaError_t launch_gemm_pair(int32_t kernel_id, const void *a, const void *b, vo
     const int a_rows = shape.rows_fixed > 0 ? shape.rows_fixed : C;
     CUtensorMap ta, tb, tout;
     const bool ok_a = (MAJ & kMajAmn) ? make_tmap(&ta, a, E, K, a_rows, 64) : make_tmap(&ta, a, E, a_rows, K, BM);
-    const bool ok_b = (MAJ & kMajBmn) ? make_tmap(&tb, b, E, K, Nout, 64) : make_tmap(&tb, b, E, Nout, K, BN / 2);
+    if (shape.b_k_stride > 0 && (!(MAJ & kMajBmn) || T > INT32_MAX)) return cudaErrorInvalidValue;
+    const bool ok_b = !(MAJ & kMajBmn)        ? make_tmap(&tb, b, E, Nout, K, BN / 2)
+                      : shape.b_k_stride > 0 ? make_tmap(&tb, b, 1, (int)T, Nout, 64)  // one [T][Nout] matrix
+                                             : make_tmap(&tb, b, E, K, Nout, 64);
     if (!ok_a || !ok_b) return cudaErrorInvalidValue;
     memset(&tout, 0, sizeof tout);
     if ((EPI == kEpiHiddenRelu || EPI == kEpiReluGrad) && !make_tmap(&tout, out, E, C, Nout, 32))
@@ -1249,14 +1256,16 @@ cudaError_t launch_router_tc_bwd_dx(const void *a, const void *b, const int32_t 
                                                    nullptr, st, stream, GroupShape{(int)T, 0, (int)T, nullptr});
 }
 
-// dW_r partials part [chunks][rows][d] (float32): per chunk c, A [rows][Tc]
-// (split dh terms) . B [d][Tc] (x^T) over the chunk's chunk_counts[c] tokens.
-cudaError_t launch_router_tc_bwd_dw(const void *a, const void *b, const int32_t *chunk_counts, int chunks, int rows,
+// dW_r partials part [chunks][rows][d] (float32): per chunk c of Tc tokens,
+// A [rows][Tc] (split dh terms, token-contiguous) . x[c Tc .. c Tc + Tc)
+// (x [T][d] read as an MN-major B along its token rows; rows past T read as
+// zeros) over the chunk's chunk_counts[c] tokens.
+cudaError_t launch_router_tc_bwd_dw(const void *a, const void *x, const int32_t *chunk_counts, int chunks, int rows,
                                     int chunk_tokens, int d, int64_t T, float *part, DeviceStatus *st,
                                     cudaStream_t stream) {
-    return launch_gemm_pair<256, 6, kEpiWeightGrad>(K_BWD_ROUTER_TC_DW, a, b, part, chunk_counts, chunks,
-                                                   chunk_tokens, chunk_tokens, d, T, nullptr, nullptr, st, stream,
-                                                   GroupShape{rows, 1, rows, nullptr});
+    return launch_gemm_pair<256, 6, kEpiWeightGrad, kMajBmn>(K_BWD_ROUTER_TC_DW, a, x, part, chunk_counts, chunks,
+                                                            chunk_tokens, chunk_tokens, d, T, nullptr, nullptr, st,
+                                                            stream, GroupShape{rows, 1, rows, nullptr, chunk_tokens});
 }
 
 cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,

@@ -34,7 +34,6 @@ enum KernelId : int32_t {
     K_FFN_TC_FUSED = 17,
     K_COMBINE_TOP2 = 18,
     K_BWD_TOKEN = 19,
-    K_BWD_TRANSPOSE = 20,
     K_BWD_GEMM_DZ = 21,
     K_BWD_GEMM_DX = 22,
     K_BWD_GEMM_DW = 23,
@@ -77,7 +76,6 @@ struct Workspace {
     void *rdx_a;         // [T][6 Np] bf16 split dh terms (tensor-core router dx)
     void *rdx_b;         // [d][6 Np] bf16 split W_r terms (tensor-core router dx)
     void *rdw_a;         // [chunks][3N][Tc] bf16 split dh terms, token-contiguous (tensor-core dW_r)
-    void *x_t;           // [chunks][d][Tc] bf16 x, token-contiguous (tensor-core dW_r)
     int32_t *chunk_counts;  // [chunks + 1] tokens of each dW_r chunk, then a 1
     int64_t tiles;
 };

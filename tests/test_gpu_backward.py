@@ -162,8 +162,9 @@ def exact_problem(rng, T=400, d=128, F=192, N=4):
 def test_backward_exact_arithmetic(orc, capacity):
     """With exactly representable operands and sums the GPU's expert-path gradients equal the
     oracle's exactly: the per-expert indexing, the slot-to-token scatter of dx, the ReLU masks, the
-    transposes and the zeroing past each expert's kept tokens are pinned without any tolerance
-    (with capacity 70 some tokens are dropped; theirs and the router's gradients are 0)."""
+    token-major (MN-major) operand reads and the zeroing past each expert's kept tokens are pinned
+    without any tolerance (with capacity 70 some tokens are dropped; theirs and the router's
+    gradients are 0)."""
     inp, dy, ids = exact_problem(np.random.default_rng(21))
     T, d = dy.shape
     dev = {k: to_device(v) for k, v in inp.items()}
