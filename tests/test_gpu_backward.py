@@ -116,9 +116,10 @@ def test_backward_edge_cases(orc, case):
 
 @pytest.mark.parametrize("name,T", [("base128_skew", 3000), ("base8", 600)])
 def test_backward_simt_router(orc, name, T):
-    """The float32 FMA router products (SWITCH_FLAG_SIMT_ROUTER) against the oracle, and against the
-    tensor-core router products on the same inputs: both within their bounds, the expert-path
-    gradients identical (the flag changes only the router's kernels)."""
+    """The float32 FMA router products (SWITCH_FLAG_SIMT_ROUTER) against the oracle, next to the
+    tensor-core router products on the same inputs: both within their bounds.  The flag also selects
+    the forward's float32 FMA router; where that gives the same gates bit for bit (N <= 32 runs the
+    same router either way), the expert-path gradients are identical too."""
     wl = synth.WORKLOADS[name]
     C = sm.switch_capacity(T, wl.num_experts, wl.capacity_factor)
     x = synth.activations(wl, T=T)
@@ -126,10 +127,13 @@ def test_backward_simt_router(orc, name, T):
     used = np.flatnonzero(np.minimum(orc.route(x, w_r, bias, capacity=C)["counts"], C) > 0)
     w_in, w_out = synth.all_expert_weights(wl, experts=used)
     inp = dict(x=x, w_r=w_r, bias=bias, w_in=w_in, w_out=w_out)
-    _, _, g_simt = run_backward(orc, inp, C, 0.01, 5, flags=sm.SWITCH_FLAG_SIMT_ROUTER)
-    _, _, g_tc = run_backward(orc, inp, C, 0.01, 5)
-    for k in ("dw_in", "dw_out"):
-        assert torch.equal(g_simt[k], g_tc[k]), k
+    _, f_simt, g_simt = run_backward(orc, inp, C, 0.01, 5, flags=sm.SWITCH_FLAG_SIMT_ROUTER)
+    _, f_tc, g_tc = run_backward(orc, inp, C, 0.01, 5)
+    if torch.equal(f_simt["gate"], f_tc["gate"]):
+        for k in ("dw_in", "dw_out"):
+            assert torch.equal(g_simt[k], g_tc[k]), k
+    else:
+        assert wl.num_experts > 32
 
 
 def exact_problem(rng, T=400, d=128, F=192, N=4):
