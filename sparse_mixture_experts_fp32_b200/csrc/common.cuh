@@ -227,6 +227,18 @@ __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bu
 // Wait until this thread's committed bulk groups have completed entirely.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Wait until all but this thread's `newest` most recent bulk groups have
+// completed entirely (newest = 0 .. 4; larger values wait for all).
+__device__ __forceinline__ void bulk_wait_all_but(int newest) {
+    switch (newest) {
+        case 1: asm volatile("cp.async.bulk.wait_group 1;" ::: "memory"); break;
+        case 2: asm volatile("cp.async.bulk.wait_group 2;" ::: "memory"); break;
+        case 3: asm volatile("cp.async.bulk.wait_group 3;" ::: "memory"); break;
+        case 4: asm volatile("cp.async.bulk.wait_group 4;" ::: "memory"); break;
+        default: asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); break;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Cross-CTA dependency counters in global memory
 // ---------------------------------------------------------------------------

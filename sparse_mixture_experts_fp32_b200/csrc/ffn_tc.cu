@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 //                   output [E][out_rows][Nout] (rows past out_rows clipped
 //                   by the tensor map).
 template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_base, int kept, int C, int n, int Nout,
+__device__ __forceinline__ int epilogue_async(uint32_t t_row, int e, int row_base, int kept, int C, int n, int Nout,
                                                void *__restrict__ out, const void *tmap_out,
                                                const int32_t *__restrict__ slot_token,
                                                const float *__restrict__ gate, uint8_t *stage, bool add = false,
@@ -324,6 +324,7 @@ __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_ba
     const int lane = threadIdx.x & 31;
     const int row = row_base + lane;
     const bool row_ok = row < kept;
+    int groups = 0;  // bulk groups committed by lane 0 (the box-store epilogues)
     if (EPI == kEpiHiddenRelu || EPI == kEpiReluGrad) {
         const bool any_row = row_base < kept;
 #pragma unroll 1
@@ -369,6 +370,7 @@ __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_ba
             if (lane == 0 && any_row && n * cols + c < Nout) {
                 tma_store_3d(tmap_out, stage, n * cols + c, row_base, e);
                 bulk_commit();
+                ++groups;
             }
         }
         if (lane == 0) bulk_wait_read_all();
@@ -430,6 +432,7 @@ __device__ __forceinline__ void epilogue_async(uint32_t t_row, int e, int row_ba
         }
         bulk_wait_read_all();
     }
+    return groups;
 }
 
 // ---------------------------------------------------------------------------
@@ -1006,6 +1009,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint8_t *my_stage = staging + (warp - 2) * L::stage_bytes;
         int acc = 0;
         uint32_t acc_phase = 0;
+        // Lane 0 releases a GEMM1 tile's H counter one tile late: after the next
+        // GEMM1 tile's boxes are issued it waits for all but those, so the warp
+        // never idles on its own store completions between tiles.  Before a GEMM2
+        // tile (whose loads may wait on that counter) or the end, it releases at once.
+        int32_t *deferred = nullptr;
         for (int it = 0;; ++it) {
             const int j = it % kTileQ;
             const uint32_t qph = (uint32_t)(it / kTileQ) & 1u;
@@ -1017,6 +1025,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (lane == 0) {
                 if (rank == 0) mbar_arrive(&tq_empty[j]);
                 else mbar_arrive_cluster(map_to_rank(&tq_empty[j], 0));
+                if (deferred && (tile < 0 || tile >= total1)) {
+                    bulk_wait_all();
+                    fence_proxy_async_global();
+                    red_release_add_gpu(deferred, 1);
+                    deferred = nullptr;
+                }
             }
             if (tile < 0) break;
             const bool second = tile >= total1;
@@ -1040,18 +1054,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int row_base = m * BMP + (int)rank * BM + quarter * 32;
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+            int groups = 0;
             if (second)
                 epilogue_async<BN, kEpiGatedScatter>(t_row, e, row_base, min(counts[e], C), C, n, d, y, nullptr,
                                                      slot_token, gate, my_stage, ks > 0, 0, nullptr, bw);
             else
-                epilogue_async<BN, kEpiHiddenRelu>(t_row, e, row_base, min(counts[e], C), C, n, F, nullptr,
-                                                   &tm_hstore, slot_token, gate, my_stage, false, 0, nullptr, bw);
+                groups = epilogue_async<BN, kEpiHiddenRelu>(t_row, e, row_base, min(counts[e], C), C, n, F,
+                                                            nullptr, &tm_hstore, slot_token, gate, my_stage, false, 0,
+                                                            nullptr, bw);
             tc_fence_before();
             mbar_arrive_cluster(map_to_rank(&acc_empty[acc], 0));
-            if (lane == 0 && (!second || ks < split - 1)) {
-                bulk_wait_all();             // this warp's H boxes (or y rows) are in global memory
-                fence_proxy_async_global();  // ... ordered before the release below
-                red_release_add_gpu(second ? ydone : done + e * MT + m, 1);
+            if (lane == 0) {
+                if (!second) {
+                    if (deferred) {  // the previous GEMM1 tile's boxes, this tile's may stay in flight
+                        bulk_wait_all_but(groups);
+                        fence_proxy_async_global();  // ... ordered before the release below
+                        red_release_add_gpu(deferred, 1);
+                    }
+                    deferred = done + e * MT + m;
+                } else if (ks < split - 1) {
+                    bulk_wait_all();             // this warp's y rows are in global memory
+                    fence_proxy_async_global();  // ... ordered before the release below
+                    red_release_add_gpu(ydone, 1);
+                }
             }
             __syncwarp();
             if (++acc == 2) {
