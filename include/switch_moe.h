@@ -330,12 +330,22 @@ switch_status_t switch_layer_bwd(const switch_dims_t *dims, const void *x, const
  * Every call shares the one array and leaves its contents behind (the next
  * call clears what must start at zero), so calls whose kernels may overlap
  * on the GPU (on different streams, or from several host threads) race and
- * must not be issued; calls on one stream are fine.  The status word used by
- * switch_check lives in the array too and cannot be read by the caller. */
+ * must not be issued; calls on one stream are fine.  The device status word
+ * lives in the array too: switch_check_noalloc reads it. */
 #define SWITCH_NOALLOC_SCRATCH_BYTES (4u << 20)
 switch_status_t switch_route_noalloc(const switch_dims_t *dims, const void *x, const float *w_r,
                                      const float *logit_bias, int32_t *expert, float *gate, int32_t *slot,
                                      int32_t *counts, int32_t *slot_token, float *aux, switch_stream_t stream);
+
+/* switch_check for switch_route_noalloc: synchronise `stream`, then read and
+ * clear the status word kept in the library's static routing array on the
+ * current device (a bounded wait of the router that gave up leaves
+ * SWITCH_ERR_DEVICE_TIMEOUT there).  Allocates nothing. */
+switch_status_t switch_check_noalloc(switch_stream_t stream);
+
+/* switch_selftest_wait_timeout on the static routing array's status word
+ * (for testing switch_check_noalloc); allocates nothing. */
+switch_status_t switch_selftest_wait_timeout_noalloc(switch_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the device status word kept in
  * `workspace`.  switch_route, switch_expert_ffn and switch_layer_fwd clear

@@ -46,7 +46,8 @@ EXPORTED = ("switch_capacity", "switch_workspace_size", "switch_route", "switch_
             "switch_expert_ffn",
             "switch_combine", "switch_layer_fwd", "switch_route_top2", "switch_combine_top2", "switch_layer_fwd_top2",
             "switch_layer_bwd", "switch_router_stats",
-            "switch_check", "switch_selftest_wait_timeout", "switch_status_string",
+            "switch_check", "switch_selftest_wait_timeout", "switch_check_noalloc",
+            "switch_selftest_wait_timeout_noalloc", "switch_status_string",
             "switch_launch_count",
             "switch_trace_start", "switch_trace_read", "switch_trace_stop", "switch_kernel_name")
 
@@ -97,6 +98,8 @@ def lib() -> ctypes.CDLL:
         "switch_router_stats": (I, [D, P, P, S, P, P]),
         "switch_check": (I, [P, S, P]),
         "switch_selftest_wait_timeout": (I, [P, S, P]),
+        "switch_check_noalloc": (I, [P]),
+        "switch_selftest_wait_timeout_noalloc": (I, [P]),
         "switch_status_string": (ctypes.c_char_p, [I]),
         "switch_launch_count": (ctypes.c_int64, []),
         "switch_trace_start": (I, [ctypes.c_int32]),
@@ -261,6 +264,16 @@ def selftest_wait_timeout(workspace, stream=None) -> None:
     reports SWITCH_ERR_DEVICE_TIMEOUT (8)."""
     _ok(lib().switch_selftest_wait_timeout(_ptr(workspace), workspace.numel() * workspace.element_size(),
                                            _stream(stream, workspace)), "switch_selftest_wait_timeout")
+
+
+def switch_check_noalloc(stream=None) -> int:
+    """switch_check for the static array switch_route_noalloc uses (0 = ok); does not raise."""
+    return int(lib().switch_check_noalloc(_stream(stream)))
+
+
+def selftest_wait_timeout_noalloc(stream=None) -> None:
+    """The bounded-wait self-test on the static routing array's status word."""
+    _ok(lib().switch_selftest_wait_timeout_noalloc(_stream(stream)), "switch_selftest_wait_timeout_noalloc")
 
 
 def launch_count() -> int:

@@ -92,3 +92,15 @@ extern "C" switch_status_t switch_route_noalloc(const switch_dims_t *dims, const
                                          ws, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? SWITCH_OK : SWITCH_ERR_CUDA;
 }
+
+extern "C" switch_status_t switch_check_noalloc(switch_stream_t stream) {
+    void *scratch = nullptr;
+    if (scratch_on_current_device(&scratch) != cudaSuccess) return SWITCH_ERR_CUDA;
+    return switch_check(scratch, kNoAllocScratchBytes, stream);
+}
+
+extern "C" switch_status_t switch_selftest_wait_timeout_noalloc(switch_stream_t stream) {
+    void *scratch = nullptr;
+    if (scratch_on_current_device(&scratch) != cudaSuccess) return SWITCH_ERR_CUDA;
+    return switch_selftest_wait_timeout(scratch, kNoAllocScratchBytes, stream);
+}

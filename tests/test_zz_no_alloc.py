@@ -14,8 +14,10 @@ parity tolerances.  The pairs cover both ways the capacity scan runs (inside the
 slot assignment for small histograms, and as its own kernel, which adds to and
 then resets a ticket kept in the shared array), the all-float32 path and an
 empty group.  The test also checks that a call leaves the device's free memory
-unchanged and that a group too large for the static array is refused before
-anything runs.
+unchanged, that a group too large for the static array is refused before
+anything runs, and that switch_check_noalloc reads (and clears) the status word
+kept in the static array: OK after a routing call, SWITCH_ERR_DEVICE_TIMEOUT
+after the bounded-wait self-test.
 
 This file is collected last on purpose: if it fails, a run that stops at the
 first failure has already run every other test.
@@ -128,3 +130,19 @@ def test_noalloc_route_refuses_groups_beyond_its_scratch():
     assert status == 9  # SWITCH_ERR_TOO_LARGE
     torch.cuda.synchronize()
     assert torch.all(out["counts"] == -7) and torch.all(out["aux"] == -7.0)
+
+
+def test_noalloc_status_word_is_readable():
+    """switch_check_noalloc: OK after a routing call; after the bounded-wait self-test (one block that
+    gives up waiting on an mbarrier nothing completes, after about a second, and exits normally) it
+    reports SWITCH_ERR_DEVICE_TIMEOUT once, clears the word, and routing still matches switch_route."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    _compare("base8", 1000)
+    assert sm.switch_check_noalloc() == 0
+    sm.selftest_wait_timeout_noalloc()
+    assert sm.switch_check_noalloc() == 8  # SWITCH_ERR_DEVICE_TIMEOUT
+    assert sm.switch_check_noalloc() == 0  # read and cleared
+    _compare("base8", 1000)
+    assert sm.switch_check_noalloc() == 0
+
