@@ -221,6 +221,12 @@ __device__ __forceinline__ void bulk_add_f32(float *gmem_dst, const void *smem_s
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
+// out[0..3] += v, one 16-byte float32 reduction in global memory (round to nearest).
+__device__ __forceinline__ void red_add_v4_f32(float *out, float4 v) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
 // Wait until this thread's committed bulk groups have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 

@@ -305,10 +305,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 //                   writes), then one TMA tensor store of the box into H.
 //                   Rows in [kept, C) receive values of rows that are never
 //                   read downstream; rows >= C are clipped by the tensor map.
-//   kEpiExpertOut / kEpiGatedScatter  32 fp32 columns at a time: each thread
-//                   writes its row (144-byte pitch: conflict-free) and
-//                   issues one 128-byte bulk copy to its destination row
-//                   (with `add`, a bulk fp32 add onto the destination).
+//   kEpiExpertOut / kEpiGatedScatter / kEpiScatterAdd  32 fp32 columns at a
+//                   time: each thread writes its row (144-byte pitch:
+//                   conflict-free), then the warp stores the block with
+//                   row-coalesced 16-byte stores (with `add`: 16-byte fp32
+//                   reductions onto the destination), no bulk-copy waits.
 //   kEpiWeightGrad  32 fp32 columns at a time into a 32 x 128-byte swizzled
 //                   box, one TMA tensor store per box into the fixed-row
 //                   output [E][out_rows][Nout] (rows past out_rows clipped
@@ -399,17 +400,25 @@ __device__ __forceinline__ int epilogue_async(uint32_t t_row, int e, int row_bas
         }
         if (lane == 0) bulk_wait_read_all();
     } else {
+        // 32 fp32 columns at a time: each lane writes its row (scaled by its gate) into the
+        // staging buffer (144-byte pitch: conflict-free), then the warp stores the 32 x 128-byte
+        // block row-coalesced: 8 lanes per row, 4 rows per instruction (float4 stores, or float4
+        // reductions with `add`).
         float g = 1.f;
-        float *dst_row = nullptr;
+        int32_t out_row = -1;  // this lane's destination row, -1 past the kept rows
         if (row_ok) {
-            int64_t out_row = (int64_t)e * (out_rows > 0 ? out_rows : C) + row;
+            out_row = (int32_t)((int64_t)e * (out_rows > 0 ? out_rows : C) + row);
             if (EPI == kEpiGatedScatter || EPI == kEpiScatterAdd) {
                 out_row = slot_token[(int64_t)e * C + row];
                 if (EPI == kEpiGatedScatter) g = gate[out_row];
             }
-            dst_row = static_cast<float *>(out) + out_row * Nout;
         }
         if (EPI == kEpiScatterAdd) add = true;
+        const int sub = lane >> 3, q4 = lane & 7;  // store phase: row 4 i + sub, 16-byte column q4
+        int32_t dst[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dst[i] = __shfl_sync(0xffffffffu, out_row, 4 * i + sub);
+        float *outf = static_cast<float *>(out);
         uint8_t *rowp = stage + lane * 144;
 #pragma unroll 1
         for (int c = 0; c < cols; c += 32) {
@@ -417,20 +426,25 @@ __device__ __forceinline__ int epilogue_async(uint32_t t_row, int e, int row_bas
             tmem_ld_32x32b_x32(t_row + (uint32_t)c, r);
             tmem_ld_wait();
             const int col0 = n * cols + c;
-            if (row_ok && col0 < Nout) {
-                bulk_wait_read_all();  // this thread's previous row copy has left the buffer
+            if (col0 < Nout) {  // the same for every lane
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
                     *reinterpret_cast<float4 *>(rowp + 16 * q) =
                         make_float4(g * __uint_as_float(r[4 * q + 0]), g * __uint_as_float(r[4 * q + 1]),
                                     g * __uint_as_float(r[4 * q + 2]), g * __uint_as_float(r[4 * q + 3]));
-                fence_proxy_async_shared();
-                if (add) bulk_add_f32(dst_row + col0, rowp, 128);
-                else bulk_store(dst_row + col0, rowp, 128);
-                bulk_commit();
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 v = *reinterpret_cast<const float4 *>(stage + (4 * i + sub) * 144 + 16 * q4);
+                    if (dst[i] >= 0) {
+                        float *p = outf + (int64_t)dst[i] * Nout + col0 + 4 * q4;
+                        if (add) red_add_v4_f32(p, v);
+                        else *reinterpret_cast<float4 *>(p) = v;
+                    }
+                }
+                __syncwarp();
             }
         }
-        bulk_wait_read_all();
     }
     return groups;
 }
@@ -726,7 +740,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // the real tile counts (fused_split).  All parts ks = 0 come first in the
 // list, then all parts ks = 1, and so on.  Part 0 stores gate * acc into y;
 // part ks > 0 waits until y_done[e, m, n] reaches 8 ks (parts 0 .. ks-1 are
-// in y) and adds its gate * acc with bulk fp32 adds, then releases 8 more.
+// in y) and adds its gate * acc with 16-byte fp32 reductions, then releases 8 more.
 // Every y element is ((y0 + y1) + y2) + ... in that order: deterministic.
 // The short parts fill the last wave; the chain of adds costs one epilogue
 // per part.
@@ -1044,10 +1058,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int32_t *ydone = y_done + ((int64_t)e * MT + m) * n2 + n;
             if (ks > 0) {  // parts 0 .. ks-1 of this output tile are in y
                 bool okw = true;
-                if (lane == 0) {
-                    okw = wait_counter_geq(ydone, 8 * ks, status, 53);
-                    fence_proxy_async_global();  // ... before our async-proxy adds
-                }
+                if (lane == 0) okw = wait_counter_geq(ydone, 8 * ks, status, 53);
+                __syncwarp();  // every lane's adds below come after lane 0's acquire
                 if (!__shfl_sync(0xffffffffu, okw, 0)) break;
             }
             if (!mbar_wait(&acc_full[acc], acc_phase, status, 45)) break;
@@ -1072,9 +1084,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         red_release_add_gpu(deferred, 1);
                     }
                     deferred = done + e * MT + m;
-                } else if (ks < split - 1) {
-                    bulk_wait_all();             // this warp's y rows are in global memory
-                    fence_proxy_async_global();  // ... ordered before the release below
+                }
+            }
+            if (second && ks < split - 1) {
+                __syncwarp();  // every lane's y stores / adds of this part ...
+                if (lane == 0) {
+                    __threadfence();  // ... are visible before the release below
                     red_release_add_gpu(ydone, 1);
                 }
             }
