@@ -851,12 +851,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mt_all += __shfl_xor_sync(0xffffffffu, mt_all, off);
-        // Tile width: 256 columns, or 128 when 256-wide GEMM1 tiles cannot give
-        // every pair one (few kept rows, e.g. a skewed routing): twice the tiles,
-        // each half as long.  Every CTA derives the same width from the same counts.
-        const int bw = mt_all * ((F + BN - 1) / BN) < (int)(gridDim.x >> 1) ? BN / 2 : BN;
-        const int n1 = (F + bw - 1) / bw, n2 = (d + bw - 1) / bw;
-        if (lane == 0) tmem_holder[1] = (uint32_t)bw;
+        // Tile widths, per GEMM: 256 columns, or 128 when few rows are kept (e.g.
+        // a skewed routing): twice the tiles, each half as long.  GEMM1 goes
+        // narrow only when 256-wide tiles would leave more than half the pairs
+        // without one (a narrow tile re-reads its A rows for half the output);
+        // GEMM2, whose tiles wait on H, goes narrow as soon as 256-wide tiles
+        // cannot give every pair one.  Every CTA derives the same widths from
+        // the same counts.
+        const int pairs = (int)(gridDim.x >> 1);
+        const int bw1 = 2 * mt_all * ((F + BN - 1) / BN) <= pairs ? BN / 2 : BN;
+        const int bw2 = mt_all * ((d + BN - 1) / BN) < pairs ? BN / 2 : BN;
+        const int n1 = (F + bw1 - 1) / bw1, n2 = (d + bw2 - 1) / bw2;
+        if (lane == 0) {
+            tmem_holder[1] = (uint32_t)bw1;
+            tmem_holder[2] = (uint32_t)bw2;
+        }
         int run1 = 0, run2 = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -889,10 +898,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     const uint32_t tmem_base = *tmem_holder;
-    const int bw = (int)tmem_holder[1];          // tile width (columns) of both GEMMs
-    const int n1 = (F + bw - 1) / bw, n2 = (d + bw - 1) / bw;
+    const int bw1 = (int)tmem_holder[1], bw2 = (int)tmem_holder[2];  // tile widths (columns) of GEMM1, GEMM2
+    const int n1 = (F + bw1 - 1) / bw1, n2 = (d + bw2 - 1) / bw2;
     const int32_t need = 8 * n1;  // arrivals on done[e, m] once H of the row block is complete
-    const uint32_t b_bytes = (uint32_t)(bw / 2) * BK * 2;  // this CTA's rows of a B stage
     const int total1 = start1[E];
     const int total2 = start2[E];  // GEMM2 output tiles
     const int split = fused_split(total2, F / BK, (int)(gridDim.x >> 1));
@@ -902,9 +910,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             prefetch_tmap(&tm_x);
-            prefetch_tmap(bw == BN ? &tm_w1 : &tm_w1h);
+            prefetch_tmap(bw1 == BN ? &tm_w1 : &tm_w1h);
             prefetch_tmap(&tm_h);
-            prefetch_tmap(bw == BN ? &tm_w2 : &tm_w2h);
+            prefetch_tmap(bw2 == BN ? &tm_w2 : &tm_w2h);
             uint32_t issued = 0, parity_of = 0;
             int stage = 0;
             uint32_t phase = 0;
@@ -947,9 +955,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     fence_proxy_async_global();  // H, written through the async proxy, before our TMA reads
                 }
                 const void *ta = second ? (const void *)&tm_h : (const void *)&tm_x;
-                const void *tb = second ? (bw == BN ? (const void *)&tm_w2 : (const void *)&tm_w2h)
-                                        : (bw == BN ? (const void *)&tm_w1 : (const void *)&tm_w1h);
+                const void *tb = second ? (bw2 == BN ? (const void *)&tm_w2 : (const void *)&tm_w2h)
+                                        : (bw1 == BN ? (const void *)&tm_w1 : (const void *)&tm_w1h);
                 const int kbs = second ? kb2 : kb1;
+                const int bw = second ? bw2 : bw1;
+                const uint32_t b_bytes = (uint32_t)(bw / 2) * BK * 2;  // this CTA's rows of a B stage
                 const int a_row = m * BMP + (int)rank * BM, b_row = n * bw + (int)rank * (bw / 2);
                 for (int kb = 0; kb < kbs; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, status, 41)) {
@@ -974,7 +984,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
-            const uint32_t idesc = idesc_bf16_f32(BMP, bw);
+            const uint32_t idesc1 = idesc_bf16_f32(BMP, bw1), idesc2 = idesc_bf16_f32(BMP, bw2);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -986,6 +996,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 mbar_arrive(&tq_empty[j]);
                 if (tile < 0) break;
                 const int kbs = tile >= total1 ? kb2 : kb1;
+                const uint32_t idesc = tile >= total1 ? idesc2 : idesc1;
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, status, 42)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -1069,11 +1080,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int groups = 0;
             if (second)
                 epilogue_async<BN, kEpiGatedScatter>(t_row, e, row_base, min(counts[e], C), C, n, d, y, nullptr,
-                                                     slot_token, gate, my_stage, ks > 0, 0, nullptr, bw);
+                                                     slot_token, gate, my_stage, ks > 0, 0, nullptr, bw2);
             else
                 groups = epilogue_async<BN, kEpiHiddenRelu>(t_row, e, row_base, min(counts[e], C), C, n, F,
                                                             nullptr, &tm_hstore, slot_token, gate, my_stage, false, 0,
-                                                            nullptr, bw);
+                                                            nullptr, bw1);
             tc_fence_before();
             mbar_arrive_cluster(map_to_rank(&acc_empty[acc], 0));
             if (lane == 0) {
