@@ -169,14 +169,27 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # algorithmic work per kernel launch
 # ---------------------------------------------------------------------------
-def kernel_work(wl, C, counts):
+WIDE_WAVES = 12  # the library's GEMM2 tile waves from which GEMM1 runs as its own launch
+
+
+def ffn_two_launches(wl, C, counts, pairs=74):
+    """Whether a layer call runs GEMM1 as its own launch and the fused kernel does GEMM2 only (else
+    the fused kernel does both and GEMM1's launch, if any, exits without work): the library's own
+    rule, from the same counts (256-row blocks x 256-wide GEMM2 column tiles)."""
+    mt = int(np.sum((np.minimum(counts, C) + 255) // 256))
+    return mt * (-(-wl.d_model // 256)) >= WIDE_WAVES * pairs
+
+
+def kernel_work(wl, C, counts, pairs=74, flags=0):
     """Algorithmic work per launch of each kernel of one step: (bound, amount,
     amount with every activation-sized tensor counted at the activation dtype).
 
     The layer writes y (and zero rows of dropped tokens) in float32; the third
     figure counts those bytes at the activation dtype instead (T*d*s for the
     output), which is the algorithmic byte count of the combine and the
-    dispatch as the layer's step table states them."""
+    dispatch as the layer's step table states them.  Of the fused FFN kernel
+    and the two-launch GEMMs, the ones that exit without work in a layer call
+    (the library decides on the device from the counts) get no work here."""
     T, d, F, N = wl.T, wl.d_model, wl.d_ff, wl.num_experts
     s = 2 if wl.dtype == synth.BF16 else 4
     kept = np.minimum(counts, C)
@@ -204,7 +217,9 @@ def kernel_work(wl, C, counts):
         "combine": ("hbm", T * d * 4 + K * d * 4 + 12 * T, T * d * s + K * d * s + 12 * T),
         "dispatch": ("hbm", 2 * K * d * s + 4 * N * C + 4 * N, None),
         "_meta": ("", dict(K=K, E_nz=E_nz, gemm_weight_bytes=2 * E_nz * d * F * s), None),
-    }
+    } | ({} if flags & 12 else  # SWITCH_FLAG_GEMM_1CTA | SWITCH_FLAG_FFN_TWO_LAUNCHES: no fused kernel
+          {"ffn_tc_fused": ("tensor", 2.0 * K * F * d, None)} if ffn_two_launches(wl, C, counts, pairs) else
+          {"ffn_tc_gemm1_relu": ("?", 0, None)})
 
 
 def kernel_entry(kind, amount, amount_act, avg_ms, launches, peaks):
@@ -230,7 +245,10 @@ def kernel_entry(kind, amount, amount_act, avg_ms, launches, peaks):
 
 
 DOMINANT_WORK_TEXT = {
-    "ffn_tc_fused": "4*K*d_model*d_ff (K = kept tokens; both expert GEMMs)",
+    "ffn_tc_fused": "4*K*d_model*d_ff (K = kept tokens; both expert GEMMs), or 2*K*d_ff*d_model when GEMM1 "
+                    "ran as its own launch (GEMM2 only)",
+    "ffn_tc_gemm1_relu": "2*K*d_model*d_ff (K = kept tokens; the first expert GEMM)",
+    "ffn_tc_gemm2_gated_scatter": "2*K*d_ff*d_model (K = kept tokens; the second expert GEMM)",
     "router_tc": "T*d*s + 6*N*d + 8*T + 8*N*ceil(T/64)",
     "router_staged": "T*d*s + 4*N*d + 8*T + 8*N*ceil(T/64)",
     "slot_assign_scatter": "8*T + 4*N*ceil(T/64) + 4*N*C + 2*K*d*s + 4*(T-K)*d",
@@ -370,7 +388,8 @@ def run_gpu(args):
     per_kernel: dict[str, list[float]] = {}
     for name, ms in trace:
         per_kernel.setdefault(name, []).append(ms)
-    work = kernel_work(wl, C, counts)
+    work = kernel_work(wl, C, counts, torch.cuda.get_device_properties(device).multi_processor_count // 2,
+                       args.flags)
     meta = work.pop("_meta")[1]
     peaks, peak_src = load_peaks()
     kernels = {}

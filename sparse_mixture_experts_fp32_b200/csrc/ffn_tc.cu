@@ -486,6 +486,8 @@ struct GroupShape {
     const uint16_t *mask_h;  // kEpiReluGrad: the forward's H [E][C][Nout]
     int b_k_stride;    // MN-major B only: > 0: B is one [T][Nout] matrix and group e's K rows start at
                        // row e * b_k_stride (groups = consecutive chunks of its rows)
+    int wide_min;      // > 0: run only when (256-row blocks over all groups) * wide_n2 >= wide_min
+    int wide_n2;       //      (the expert FFN's GEMM2 tile count; otherwise the fused kernel runs it)
 };
 
 __device__ __forceinline__ int group_rows(const GroupShape &g, int kept) {
@@ -581,7 +583,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     const uint32_t tmem_base = *tmem_holder;
-    const int total_tiles = tile_start[E];
+    int total_tiles = tile_start[E];
+    if (shape.wide_min > 0 && total_tiles / n_tiles_n * shape.wide_n2 < shape.wide_min)
+        total_tiles = 0;  // few tiles: the fused kernel of this call computes the FFN
 
     if (warp == 0) {
         if (lane == 0) {
@@ -746,6 +750,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // per part.
 // ---------------------------------------------------------------------------
 constexpr int kFusedBN = 256;
+// GEMM2 tile waves (256 x 256 tiles over the SM pairs) from which a layer call
+// runs GEMM1 as its own launch and the fused kernel takes GEMM2 only.
+constexpr int kWideWaves = 12;
 
 // Parts per GEMM2 tile: 1, 2 or 4, for GEMM2 with fewer tiles than two waves
 // only (the adds cost y traffic).  Picks the S that minimises a rough time
@@ -785,7 +792,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_hstore, float *__restrict__ y,
                       const int32_t *__restrict__ counts, int E, int C, int d, int F,
                       const int32_t *__restrict__ slot_token, const float *__restrict__ gate,
-                      int32_t *__restrict__ done, int MT, DeviceStatus *status) {
+                      int32_t *__restrict__ done, int MT, DeviceStatus *status, int wide_min) {
     constexpr int BN = kFusedBN;
     using L = PairLayout<BN, STAGES>;
     constexpr int BMP = 2 * BM;
@@ -901,7 +908,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int bw1 = (int)tmem_holder[1], bw2 = (int)tmem_holder[2];  // tile widths (columns) of GEMM1, GEMM2
     const int n1 = (F + bw1 - 1) / bw1, n2 = (d + bw2 - 1) / bw2;
     const int32_t need = 8 * n1;  // arrivals on done[e, m] once H of the row block is complete
-    const int total1 = start1[E];
+    // Many tiles: GEMM1 ran as its own launch just before this one (measured faster there), so
+    // this launch takes the GEMM2 tiles only and their H is complete before griddepcontrol.wait
+    // returns; every CTA decides alike from the same counts.
+    const bool wide = wide_min > 0 && start1[E] / n1 * ((d + BN - 1) / BN) >= wide_min;
+    const int total1 = wide ? 0 : start1[E];
     const int total2 = start2[E];  // GEMM2 output tiles
     const int split = fused_split(total2, F / BK, (int)(gridDim.x >> 1));
     const int kb2 = F / BK / split;  // K blocks of a GEMM2 part
@@ -950,7 +961,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     locate_tile(start1, E, n1, tile, e, m, n);
                 }
                 const int k0 = ks * kb2;  // first K block of this tile
-                if (second) {
+                if (second && !wide) {
                     if (!wait_counter_geq(done + e * MT + m, need, status, 47)) break;
                     fence_proxy_async_global();  // H, written through the async proxy, before our TMA reads
                 }
@@ -1230,7 +1241,7 @@ cudaError_t launch_gemm_pair(int32_t kernel_id, const void *a, const void *b, vo
 template <int STAGES>
 cudaError_t launch_ffn_fused(const switch_dims_t &dims, const void *xbuf, const void *w_in, const void *w_out,
                              const int32_t *counts, const int32_t *slot_token, const float *gate, float *y,
-                             const Workspace &ws, bool zero_done, cudaStream_t stream) {
+                             const Workspace &ws, bool zero_done, int wide_min, cudaStream_t stream) {
     const int E = dims.num_experts, C = dims.capacity, d = dims.d_model, F = dims.d_ff;
     const size_t smem = FusedLayout<STAGES>::bytes(E);
     auto kern = tc_ffn_fused_pair<STAGES>;
@@ -1256,8 +1267,8 @@ cudaError_t launch_ffn_fused(const switch_dims_t &dims, const void *xbuf, const 
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(max_pairs, tiles));
     launch_begin(K_FFN_TC_FUSED, stream);
     err = launch_kernel(kern, dim3(2 * pairs), dim3(kThreads), smem, stream, !zero_done, tx, tw1, th, tw2, tw1h, tw2h,
-                        ths, y,
-                        counts, E, C, d, F, slot_token, gate, ws.done, MT, static_cast<DeviceStatus *>(ws.status));
+                        ths, y, counts, E, C, d, F, slot_token, gate, ws.done, MT,
+                        static_cast<DeviceStatus *>(ws.status), wide_min);
     launch_end(stream);
     return err;
 }
@@ -1325,9 +1336,25 @@ cudaError_t launch_ffn_tc(const switch_dims_t &dims, const void *xbuf, const voi
     const int N = dims.num_experts, C = dims.capacity, d = dims.d_model, F = dims.d_ff;
     DeviceStatus *st = static_cast<DeviceStatus *>(ws.status);
     if (y && !(dims.flags & (SWITCH_FLAG_GEMM_1CTA | SWITCH_FLAG_FFN_TWO_LAUNCHES))) {
-        // both GEMMs in one launch; the dependency counters were zeroed by the
-        // slot assignment of this call
-        return launch_ffn_fused<6>(dims, xbuf, w_in, w_out, counts, slot_token, gate, y, ws, false, stream);
+        // Both GEMMs in one launch (the dependency counters were zeroed by the
+        // slot assignment of this call).  When GEMM2 may have kWideWaves waves of
+        // 256-wide tiles or more, GEMM1's own launch goes first and the device
+        // counts decide: with that many tiles GEMM1 runs there and the fused
+        // kernel takes GEMM2 only (measured faster: 1.68 against 1.78 ms of
+        // expert GEMMs on the Switch-Large shape); otherwise GEMM1's launch exits
+        // at once and the fused kernel runs both.
+        const int pairs = device_sm_count() / 2;
+        const int n2w = (d + 255) / 256;
+        const int64_t max_mt = std::min<int64_t>((int64_t)N * ((C + 255) / 256), (dims.T + 255) / 256 + N);
+        const int wide_min = kWideWaves * pairs;
+        if (max_mt * n2w < wide_min)
+            return launch_ffn_fused<6>(dims, xbuf, w_in, w_out, counts, slot_token, gate, y, ws, false, 0, stream);
+        const GroupShape gated{0, 0, 0, nullptr, 0, wide_min, n2w};
+        cudaError_t err = launch_gemm_pair<256, 6, kEpiHiddenRelu>(K_FFN_TC_GEMM1, xbuf, w_in, ws.hidden, counts, N,
+                                                                   C, d, F, dims.T, nullptr, nullptr, st, stream,
+                                                                   gated);
+        if (err != cudaSuccess) return err;
+        return launch_ffn_fused<6>(dims, xbuf, w_in, w_out, counts, slot_token, gate, y, ws, false, wide_min, stream);
     }
     if (dims.flags & SWITCH_FLAG_GEMM_1CTA) {
         cudaError_t err = launch_gemm<256, 4, kEpiHiddenRelu>(K_FFN_TC_GEMM1, xbuf, w_in, ws.hidden, counts, N, C, d,

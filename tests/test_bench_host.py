@@ -63,3 +63,24 @@ def test_traffic_lines_follow_the_kernel_source(tmp_path, monkeypatch):
     (csrc / "router_tc.cu").write_text((csrc / "router_tc.cu").read_text() + "\n// edit\n")
     assert bench.traffic_from_profiles("router_tc", "base128_skew") is None
     assert bench.source_sha("ffn_tc_fused") == other
+
+
+def test_ffn_path_rule():
+    """The bench reproduces the library's device-side choice of FFN path from the counts: with at
+    least twelve waves of 256-wide GEMM2 tiles GEMM1 runs as its own launch and the fused kernel
+    does GEMM2 only; otherwise the fused kernel does both and GEMM1's launch (if any) no work."""
+    wl = synth.WORKLOADS["large128"]
+    C = 1280
+    balanced = np.full(wl.num_experts, wl.T // wl.num_experts, dtype=np.int64)
+    assert bench.ffn_two_launches(wl, C, balanced)
+    work = bench.kernel_work(wl, C, balanced)
+    K = int(np.minimum(balanced, C).sum())
+    assert work["ffn_tc_fused"] == ("tensor", 2.0 * K * wl.d_ff * wl.d_model, None)
+    assert work["ffn_tc_gemm1_relu"][0] == "tensor"
+    skewed = np.zeros(wl.num_experts, dtype=np.int64)
+    skewed[:2] = C  # two experts at capacity: 10 row blocks x 4 column tiles = 40 tiles
+    assert not bench.ffn_two_launches(wl, C, skewed)
+    work = bench.kernel_work(wl, C, skewed)
+    assert work["ffn_tc_fused"][0] == "tensor" and work["ffn_tc_gemm1_relu"][0] == "?"
+    # with SWITCH_FLAG_FFN_TWO_LAUNCHES both GEMMs are real launches and there is no fused kernel
+    assert bench.kernel_work(wl, C, skewed, flags=8)["ffn_tc_gemm1_relu"][0] == "tensor"

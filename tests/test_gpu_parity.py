@@ -104,6 +104,54 @@ def test_fused_ffn_matches_two_launches(name, T):
     assert torch.equal((a["y"] == 0).all(dim=1), (b["y"] == 0).all(dim=1))  # the same rows are zero (dropped)
 
 
+@pytest.mark.parametrize("skewed", [False, True], ids=["balanced", "skewed"])
+def test_ffn_path_chosen_on_device(orc, skewed):
+    """Where GEMM2 may have twelve waves of 256-wide tiles or more, a layer call launches GEMM1 on
+    its own and then the fused FFN kernel, and the device counts decide: with that many tiles GEMM1
+    runs there and the fused kernel does GEMM2 only, so y equals that of
+    SWITCH_FLAG_FFN_TWO_LAUNCHES bit for bit (balanced routing: ~540 row blocks x 2 column tiles);
+    otherwise GEMM1's launch exits at once and the fused kernel does both (a bias that sends every
+    token to two experts), within the fused-vs-two-launch rounding bound.  Sampled rows are checked
+    against the oracle in both cases."""
+    rng = np.random.default_rng(17 + skewed)
+    T, d, F, N, c = 131072, 512, 512, 64, 1.25
+    C = sm.switch_capacity(T, N, c)
+    x = synth.to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))
+    w_r = (rng.standard_normal((N, d)) * 0.1 / np.sqrt(d)).astype(np.float32)
+    bias = np.zeros(N, np.float32)
+    if skewed:
+        bias[[3, 41]] = 40.0  # every token's two largest logits are experts 3 and 41
+    w_in = synth.to_bf16_bits((rng.standard_normal((N, F, d)) / np.sqrt(d)).astype(np.float32))
+    w_out = synth.to_bf16_bits((rng.standard_normal((N, d, F)) / np.sqrt(F)).astype(np.float32))
+    dev = {k: to_device(v) for k, v in dict(x=x, w_r=w_r, bias=bias, w_in=w_in, w_out=w_out).items()}
+    sm.trace_start(64)
+    a = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, logit_bias=dev["bias"])
+    torch.cuda.synchronize()
+    names = [n for n, _ in sm.trace_read()]
+    sm.trace_stop()
+    assert names[-2:] == ["ffn_tc_gemm1_relu", "ffn_tc_fused"], names
+    b = sm.layer_fwd(dev["x"], dev["w_r"], dev["w_in"], dev["w_out"], capacity=C, logit_bias=dev["bias"],
+                     flags=sm.SWITCH_FLAG_FFN_TWO_LAUNCHES)
+    assert sm.switch_check(a["workspace"]) == 0 and sm.switch_check(b["workspace"]) == 0
+    counts = a["counts"].cpu().numpy()
+    mt = int(np.sum((np.minimum(counts, C) + 255) // 256))
+    assert (mt * 2 >= 12 * 74) == (not skewed)
+    if skewed:
+        ya, yb = a["y"].double(), b["y"].double()
+        kept = ~(b["y"] == 0).all(dim=1)
+        rms = float(yb[kept].pow(2).mean().sqrt())
+        assert float((ya - yb).abs().max()) <= 1e-4 * rms
+    else:
+        assert torch.equal(a["y"].view(torch.int32), b["y"].view(torch.int32))
+    o = orc.route(x, w_r, bias, capacity=C, want_probs=True)
+    g = {k: a[k].cpu().numpy() for k in ("expert", "gate", "slot", "counts", "aux")}
+    g["aux"] = g["aux"][0]
+    rep = check_routing(o, g, orc, N, C, T, check_slot_token=False)
+    rows = _sample_rows(rep["assign"]["slot"])
+    y_rows = a["y"][torch.from_numpy(rows).cuda()].float().cpu().numpy().astype(np.float64)
+    check_outputs(y_rows, rows, o, rep, orc, x, w_in, w_out, g["expert"], False)
+
+
 @pytest.mark.parametrize("name,T", [("tiny_fp32", 64), ("base8", 3000), ("base128_skew", 2000)])
 def test_fused_scan_matches_scan_kernel(name, T):
     """The assignment kernel's own scan of a small histogram gives the same slots, counts and
