@@ -325,6 +325,11 @@ __global__ void __launch_bounds__(kThreads) router_warp_kernel(const XT *__restr
 // 16 parts.  Softmax, argmax and gate per token in registers; the tile's sum
 // of p is formed in fixed token order (deterministic).
 // ---------------------------------------------------------------------------
+// Threads of the staged router: 16 groups of 4 tokens of a 64-token tile,
+// each group one warp (NP <= 16) or half a warp (NP = 32: 4 x 32 accumulators
+// per thread, which 512 threads' register budget cannot hold).
+__host__ __device__ constexpr int staged_threads(int NP) { return NP <= 16 ? 512 : 256; }
+
 template <typename XT>
 struct Staged {
     static constexpr int V = XLoad<XT>::V;
@@ -335,10 +340,10 @@ struct Staged {
         const int64_t a = kTileT * xpitch(d), b = (int64_t)kTileT * NP * 4;
         return ((a > b ? a : b) + 15) / 16 * 16;
     }
-    // smem layout: x tile | W_r as [d/V][V][NP] | per-warp sums | counts | second-choice counts |
+    // smem layout: x tile | W_r as [d/V][V][NP] | counts | second-choice counts |
     // per-token entropies [64] | 5 mbarriers | raw W_r (optional)
     static size_t smem_base(int d, int NP) {
-        return (size_t)x_region(d, NP) + (size_t)((d / V) * wpitch(NP)) * 4 + (size_t)(kWarps * NP) * 4 +
+        return (size_t)x_region(d, NP) + (size_t)((d / V) * wpitch(NP)) * 4 +
                2 * (size_t)NP * 4 + kTileT * 4 + 5 * 8 + 16;
     }
     static size_t smem(int d, int NP, int N, bool raw) {
@@ -347,7 +352,7 @@ struct Staged {
 };
 
 template <typename XT, int NP, bool TOP2>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(staged_threads(NP), 1)
     router_staged_kernel(const XT *__restrict__ x, const float *__restrict__ w_r, const float *__restrict__ bias,
                          int64_t T, int d, int N, int tiles, int32_t *__restrict__ expert, float *__restrict__ gate,
                          int32_t *__restrict__ hist, int32_t *__restrict__ hist2, float *__restrict__ psum,
@@ -355,13 +360,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                          int raw_w) {
     using S = Staged<XT>;
     constexpr int V = S::V;
+    constexpr int kST = staged_threads(NP);
+    if (blockDim.x != (unsigned)kST) {  // launched with another block size: report it, write nothing
+        if (threadIdx.x == 0) report_status(status, SWITCH_ERR_CUDA, 62);
+        return;
+    }
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int64_t xpitch = S::xpitch(d);
     const int64_t wpitch = S::wpitch(NP);
     unsigned char *xs = smem_raw;
     float *wsm = reinterpret_cast<float *>(smem_raw + S::x_region(d, NP));
-    float *psum_w = wsm + (d / V) * wpitch;
-    int32_t *hist_s = reinterpret_cast<int32_t *>(psum_w + kWarps * NP);
+    int32_t *hist_s = reinterpret_cast<int32_t *>(wsm + (d / V) * wpitch);
     int32_t *hist2_s = hist_s + NP;  // second choices (TOP2)
     float *ent_tok = reinterpret_cast<float *>(hist2_s + NP);  // [64] per-token entropy (with ent)
     uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(ent_tok + kTileT) + 15) & ~uintptr_t(15));
@@ -385,24 +394,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (raw_w) mbar_arrive_expect_tx(&bar[4], w_bytes);
     }
     __syncthreads();  // barriers initialised before any copy signals them
-    if (tid < 4) {    // rows are contiguous: one bulk copy per 16-row chunk
-        const int rows = max(0, min(16, n_tok - 16 * tid));
-        if (rows > 0)
-            bulk_load(xs + 16 * tid * xpitch, x + (t0 + 16 * tid) * d, (uint32_t)rows * row_bytes, &bar[tid]);
-    } else if (tid == 4 && raw_w) {
-        bulk_load(w_raw, w_r, w_bytes, &bar[4]);  // W_r [N][d] as stored
+    if (tid < 32) {  // warp 0: W_r first (every thread needs it), then one bulk copy per row of x
+        if (tid == 0 && raw_w) bulk_load(w_raw, w_r, w_bytes, &bar[4]);  // W_r [N][d] as stored
+        __syncwarp();
+        for (int r = tid; r < n_tok; r += 32)
+            bulk_load(xs + r * xpitch, x + (t0 + r) * d, row_bytes, &bar[r >> 4]);
     }
     // W_r -> [d/V][V][NP] with padding, while the rows of x are on their way
     if (raw_w) {
         mbar_wait(&bar[4], 0, status, 11);
-        for (int i = tid; i < NP * d; i += kThreads) {
+        for (int i = tid; i < NP * d; i += kST) {
             const int e = i / d, k = i - e * d;
             float v = 0.f;
             if (e < N) v = w_raw[i];  // padding experts e >= N read nothing
             wsm[(k / V) * wpitch + (k % V) * NP + e] = v;
         }
     } else {
-        for (int k0 = 0; k0 < d; k0 += kThreads) {
+        for (int k0 = 0; k0 < d; k0 += kST) {
             const int k = k0 + tid;
 #pragma unroll
             for (int e0 = 0; e0 < NP; e0 += 8) {
@@ -416,17 +424,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     }
-    for (int i = tid; i < kWarps * NP; i += kThreads) psum_w[i] = 0.f;
-    for (int i = tid; i < NP; i += kThreads) {
+    for (int i = tid; i < NP; i += kST) {
         hist_s[i] = 0;
         hist2_s[i] = 0;
     }
     __syncthreads();
 
-    // Thread (group g, part p): tokens 4g .. 4g+3 of the tile, 16-byte x
-    // vectors j = p, p + 16, ... of their rows; 4 x NP accumulators.  Each
-    // W_r value read from shared memory feeds four tokens.
-    constexpr int TM = 4, PARTS = 16;
+    // Thread (group g, part p of PARTS = 32 or 16 lanes): tokens 4g .. 4g+3 of
+    // the tile, 16-byte x vectors j = p, p + PARTS, ... of their rows; 4 x NP
+    // accumulators.  Each W_r value read from shared memory feeds four tokens.
+    constexpr int TM = 4, PARTS = kST / 16;
+    static_assert(kST / PARTS * TM == kTileT, "16 groups of 4 tokens");
     const int part = tid & (PARTS - 1), group = tid / PARTS;  // 16 groups x 4 tokens = 64 tokens
     float acc[TM][NP];
 #pragma unroll
@@ -460,8 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     }
-    // sum over the 16 parts (lanes of one half-warp): every lane of the group
-    // ends with the full logits of the group's 4 tokens
+    // sum over the parts (lanes of the group): every lane of the group ends
+    // with the full logits of the group's 4 tokens
 #pragma unroll
     for (int i = 0; i < TM; ++i)
 #pragma unroll
@@ -470,6 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], 2);
             acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], 4);
             acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], 8);
+            if (PARTS == 32) acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], 16);
         }
     // lanes with part < TM finish token tok0 + part
     float *ptile = reinterpret_cast<float *>(xs);  // [64][NP] per-token p, reusing the x tile
@@ -545,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ent[tile] = e;
     }
     // tile sums of p: four interleaved partial sums, combined in fixed order (deterministic)
-    for (int i = tid; i < N; i += kThreads) {
+    for (int i = tid; i < N; i += kST) {
         float p4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
         for (int tl = 0; tl < kTileT; tl += 4) {
@@ -822,7 +831,7 @@ __global__ void __launch_bounds__(kAssignThreads) assign_kernel(
     int64_t T, int N, int C, int tiles, int32_t *__restrict__ slot, int32_t *__restrict__ slot_token,
     const uint4 *__restrict__ x, uint4 *__restrict__ xbuf, int x_words, float4 *__restrict__ y_zero, int y_words,
     int32_t *__restrict__ done_zero, int64_t n_done, const int32_t *__restrict__ hist, const float *__restrict__ psum,
-    double *__restrict__ prob_total, float *__restrict__ aux) {
+    double *__restrict__ prob_total, float *__restrict__ aux, DeviceStatus *status) {
     static_assert(kTileT == 64, "assignment assumes two ranking warps per tile");
     __shared__ int32_t first_warp_count[256];
     __shared__ int32_t tile_slot[kTileT];
@@ -865,20 +874,27 @@ __global__ void __launch_bounds__(kAssignThreads) assign_kernel(
         for (int i = tid; i < N; i += kAssignThreads) first_warp_count[i] = 0;
         __syncthreads();
         int e = -1, rank = 0;
-        bool valid = false;
+        bool valid = false, rejected = false;
         int64_t t = 0;
         unsigned same = 0;
         if (warp < 2) {
             t = (int64_t)tile * kTileT + tid;
             valid = t < T;
             e = valid ? expert[t] : -1 - lane;  // distinct keys for absent tokens
+            if (valid && (unsigned)e >= (unsigned)N) {  // an id no router writes: report it, index
+                report_status(status, SWITCH_ERR_SHAPE, 60);  // nothing, and drop the token
+                valid = false;
+                rejected = true;
+                e = -1 - lane;
+            }
             same = __match_any_sync(0xffffffffu, e);
             rank = __popc(same & (unsigned)lanemask_lt());
             if (warp == 0 && valid && rank == 0) first_warp_count[e] = __popc(same);
         }
         __syncthreads();
         if (warp < 2) {
-            int s_out = -2;  // -2: no token here
+            int s_out = rejected ? -1 : -2;  // -2: no token here; -1: dropped
+            if (rejected) slot[t] = -1;
             if (valid) {
                 if (warp == 1) rank += first_warp_count[e];
                 const int s = (SCAN ? s_off[e] : tile_off[(int64_t)e * tiles + tile]) + rank;
@@ -958,7 +974,8 @@ template <bool SCATTER>
 __global__ void __launch_bounds__(kAssignThreads) assign_top2_kernel(
     const int32_t *__restrict__ expert2, const int32_t *__restrict__ tile_off, const int32_t *__restrict__ tile_off2,
     const int32_t *__restrict__ counts, int64_t T, int N, int C, int tiles, int32_t *__restrict__ slot2,
-    int32_t *__restrict__ slot_token, const uint4 *__restrict__ x, uint4 *__restrict__ xbuf, int x_words) {
+    int32_t *__restrict__ slot_token, const uint4 *__restrict__ x, uint4 *__restrict__ xbuf, int x_words,
+    DeviceStatus *status) {
     static_assert(kTileT == 64, "top-2 assignment assumes 64-token tiles");
     __shared__ int32_t first_warp_count[2][256];
     __shared__ int32_t tile_slot[2 * kTileT];    // [choice][token of the tile]
@@ -973,20 +990,27 @@ __global__ void __launch_bounds__(kAssignThreads) assign_top2_kernel(
         const int c = warp >> 1;         // warps 0-1: first choices, 2-3: second choices
         const int half = warp & 1;       // tokens 0-31 or 32-63 of the tile
         int e = -1, rank = 0;
-        bool valid = false;
+        bool valid = false, rejected = false;
         int64_t t = 0;
         unsigned same = 0;
         if (warp < 4) {
             t = (int64_t)tile * kTileT + half * 32 + lane;
             valid = t < T;
             e = valid ? expert2[2 * t + c] : -1 - lane;  // distinct keys for absent tokens
+            if (valid && (unsigned)e >= (unsigned)N) {  // an id no router writes: report it, index
+                report_status(status, SWITCH_ERR_SHAPE, 61);  // nothing, and drop the choice
+                valid = false;
+                rejected = true;
+                e = -1 - lane;
+            }
             same = __match_any_sync(0xffffffffu, e);
             rank = __popc(same & (unsigned)lanemask_lt());
             if (half == 0 && valid && rank == 0) first_warp_count[c][e] = __popc(same);
         }
         __syncthreads();
         if (warp < 4) {
-            int s_out = -2;  // -2: no token here
+            int s_out = rejected ? -1 : -2;  // -2: no token here; -1: dropped
+            if (rejected) slot2[2 * t + c] = -1;
             if (valid) {
                 if (half == 1) rank += first_warp_count[c][e];
                 const int s = (c == 0 ? tile_off : tile_off2)[(int64_t)e * tiles + tile] + rank;
@@ -1054,7 +1078,7 @@ cudaError_t launch_router_staged(const switch_dims_t &dims, const XT *x, const f
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     launch_begin(K_ROUTER_STAGED, stream);
-    kern<<<(unsigned)ws.tiles, kThreads, smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
+    kern<<<(unsigned)ws.tiles, staged_threads(NP), smem, stream>>>(x, w_r, bias, dims.T, d, N, (int)ws.tiles, expert, gate,
                                                          ws.hist, ws.hist2, ws.psum, ws.probs, ws.ent, ws.ticket,
                                                          static_cast<DeviceStatus *>(ws.status), raw ? 1 : 0);
     err = cudaGetLastError();
@@ -1213,11 +1237,12 @@ cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *
         if (xbuf_scatter)
             err = launch_kernel(assign_top2_kernel<true>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
                                 expert, ws.tile_off, ws.tile_off2, counts, dims.T, N, C, (int)ws.tiles, slot,
-                                slot_token, xs, xb, x_words);
+                                slot_token, xs, xb, x_words, static_cast<DeviceStatus *>(ws.status));
         else
             err = launch_kernel(assign_top2_kernel<false>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream,
                                 true, expert, ws.tile_off, ws.tile_off2, counts, dims.T, N, C, (int)ws.tiles, slot,
-                                slot_token, (const uint4 *)nullptr, (uint4 *)nullptr, 0);
+                                slot_token, (const uint4 *)nullptr, (uint4 *)nullptr, 0,
+                                static_cast<DeviceStatus *>(ws.status));
         launch_end(stream);
         return err;
     }
@@ -1241,21 +1266,25 @@ cudaError_t launch_route(const switch_dims_t &dims, const void *x, const float *
     if (xbuf_scatter && fused_scan)
         err = launch_kernel(assign_kernel<true, true>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
                             expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token, xs, xb,
-                            x_words, yz, y_words, done_zero, n_done, ws.hist, ws.psum, ws.prob_total, aux);
+                            x_words, yz, y_words, done_zero, n_done, ws.hist, ws.psum, ws.prob_total, aux,
+                            static_cast<DeviceStatus *>(ws.status));
     else if (xbuf_scatter)
         err = launch_kernel(assign_kernel<true, false>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
                             expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token, xs, xb,
-                            x_words, yz, y_words, done_zero, n_done, ws.hist, ws.psum, ws.prob_total, aux);
+                            x_words, yz, y_words, done_zero, n_done, ws.hist, ws.psum, ws.prob_total, aux,
+                            static_cast<DeviceStatus *>(ws.status));
     else if (fused_scan)
         err = launch_kernel(assign_kernel<false, true>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
                             expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token,
                             (const uint4 *)nullptr, (uint4 *)nullptr, 0, (float4 *)nullptr, 0, done_zero, n_done,
-                            ws.hist, ws.psum, ws.prob_total, aux);
+                            ws.hist, ws.psum, ws.prob_total, aux,
+                            static_cast<DeviceStatus *>(ws.status));
     else
         err = launch_kernel(assign_kernel<false, false>, dim3((unsigned)grid), dim3(kAssignThreads), 0, stream, true,
                             expert, ws.tile_off, counts, dims.T, N, C, (int)ws.tiles, slot, slot_token,
                             (const uint4 *)nullptr, (uint4 *)nullptr, 0, (float4 *)nullptr, 0, done_zero, n_done,
-                            ws.hist, ws.psum, ws.prob_total, aux);
+                            ws.hist, ws.psum, ws.prob_total, aux,
+                            static_cast<DeviceStatus *>(ws.status));
     launch_end(stream);
     return err;
 }
