@@ -16,17 +16,24 @@ constexpr int kSmallThreads = 256;
 constexpr int kSmallMaxT = 256;
 constexpr int kSmallMaxN = 32;
 
+// Rows in shared memory have odd pitches (d | 1, F | 1 floats), so that the 32
+// lanes of a warp reading one element of 32 different rows hit 32 different
+// banks (with a pitch of 32 or 64 floats they all hit one bank, and the layer
+// ran about 10x slower).
 struct SmallLayout {
+    int pd, pf;  // row pitches (floats) of x / W_r / W_in rows and of W_out rows
     int64_t x, wr, win, wout, h, logit, gate_s, expert_s, slot_s, total;  // float offsets
 };
 __host__ __device__ inline SmallLayout small_layout(int T, int d, int F, int N) {
     SmallLayout L{};
+    L.pd = d | 1;
+    L.pf = F | 1;
     int64_t o = 0;
     auto take = [&](int64_t n) { const int64_t at = o; o += (n + 3) / 4 * 4; return at; };
-    L.x = take((int64_t)T * d);
-    L.wr = take((int64_t)N * d);
-    L.win = take((int64_t)N * F * d);
-    L.wout = take((int64_t)N * d * F);
+    L.x = take((int64_t)T * L.pd);
+    L.wr = take((int64_t)N * L.pd);
+    L.win = take((int64_t)N * F * L.pd);
+    L.wout = take((int64_t)N * d * L.pf);
     L.h = take((int64_t)(kSmallThreads / 32) * F);  // one hidden row per warp
     L.logit = take((int64_t)T * N);                  // logits, then probabilities
     L.gate_s = take(T);
@@ -57,18 +64,19 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         status->block = 0;
         status->reserved = 0;
     }
-    for (int64_t i = tid; i < (int64_t)T * d; i += kSmallThreads) xs[i] = x[i];
-    for (int64_t i = tid; i < (int64_t)N * d; i += kSmallThreads) wrs[i] = w_r[i];
+    const int pd = L.pd, pf = L.pf;
+    for (int64_t i = tid; i < (int64_t)T * d; i += kSmallThreads) xs[i / d * pd + i % d] = x[i];
+    for (int64_t i = tid; i < (int64_t)N * d; i += kSmallThreads) wrs[i / d * pd + i % d] = w_r[i];
     for (int64_t i = tid; i < (int64_t)N * F * d; i += kSmallThreads) {
-        wis[i] = w_in[i];
-        wos[i] = w_out[i];
+        wis[i / d * pd + i % d] = w_in[i];   // row (e, j) of W_in
+        wos[i / F * pf + i % F] = w_out[i];  // row (e, k) of W_out
     }
     __syncthreads();
     // router logits, one (token, expert) pair per thread at a time
     for (int q = tid; q < T * N; q += kSmallThreads) {
         const int t = q / N, i = q % N;
         float acc = 0.f;
-        for (int k = 0; k < d; ++k) acc = fmaf(xs[t * d + k], wrs[i * d + k], acc);
+        for (int k = 0; k < d; ++k) acc = fmaf(xs[t * pd + k], wrs[i * pd + k], acc);
         lg[q] = acc + (bias ? bias[i] : 0.f);
     }
     __syncthreads();
@@ -131,17 +139,17 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
             continue;
         }
         const int e = es[t];
-        const float *wi = wis + (int64_t)e * F * d, *wo = wos + (int64_t)e * d * F, *xt = xs + t * d;
+        const float *wi = wis + (int64_t)e * F * pd, *wo = wos + (int64_t)e * d * pf, *xt = xs + t * pd;
         for (int j = lane; j < F; j += 32) {
             float acc = 0.f;
-            for (int k = 0; k < d; ++k) acc = fmaf(wi[j * d + k], xt[k], acc);
+            for (int k = 0; k < d; ++k) acc = fmaf(wi[j * pd + k], xt[k], acc);
             hrow[j] = fmaxf(acc, 0.f);
         }
         __syncwarp();
         const float g = gs[t];
         for (int k = lane; k < d; k += 32) {
             float acc = 0.f;
-            for (int j = 0; j < F; ++j) acc = fmaf(wo[k * F + j], hrow[j], acc);
+            for (int j = 0; j < F; ++j) acc = fmaf(wo[k * pf + j], hrow[j], acc);
             yt[k] = g * acc;
         }
         __syncwarp();
