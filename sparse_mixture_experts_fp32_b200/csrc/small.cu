@@ -43,6 +43,36 @@ __host__ __device__ inline SmallLayout small_layout(int T, int d, int F, int N) 
     return L;
 }
 
+// Copies an [n / cols][cols] float32 matrix into shared-memory rows of `pitch`
+// floats.  Each thread keeps eight 16-byte loads in flight before it stores
+// them (a load-then-store loop left every load's latency exposed).
+__device__ __forceinline__ void load_rows(float *dst, const float *__restrict__ src, int64_t n, int cols, int pitch) {
+    const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
+    const int64_t n4 = vec ? n / 4 : 0;
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+    for (int64_t base = threadIdx.x; base < n4; base += 8 * kSmallThreads) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int64_t i = base + (int64_t)u * kSmallThreads;
+            if (i < n4) v[u] = __ldg(s4 + i);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int64_t i = base + (int64_t)u * kSmallThreads;
+            if (i < n4) {
+                const float c[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int64_t k = 4 * i + q;
+                    dst[k / cols * pitch + k % cols] = c[q];
+                }
+            }
+        }
+    }
+    for (int64_t k = 4 * n4 + threadIdx.x; k < n; k += kSmallThreads) dst[k / cols * pitch + k % cols] = src[k];
+}
+
 __global__ void __launch_bounds__(kSmallThreads, 1)
     small_layer_kernel(const float *__restrict__ x, const float *__restrict__ w_r, const float *__restrict__ bias,
                        const float *__restrict__ w_in, const float *__restrict__ w_out, int T, int d, int F, int N,
@@ -65,12 +95,10 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         status->reserved = 0;
     }
     const int pd = L.pd, pf = L.pf;
-    for (int64_t i = tid; i < (int64_t)T * d; i += kSmallThreads) xs[i / d * pd + i % d] = x[i];
-    for (int64_t i = tid; i < (int64_t)N * d; i += kSmallThreads) wrs[i / d * pd + i % d] = w_r[i];
-    for (int64_t i = tid; i < (int64_t)N * F * d; i += kSmallThreads) {
-        wis[i / d * pd + i % d] = w_in[i];   // row (e, j) of W_in
-        wos[i / F * pf + i % F] = w_out[i];  // row (e, k) of W_out
-    }
+    load_rows(xs, x, (int64_t)T * d, d, pd);
+    load_rows(wrs, w_r, (int64_t)N * d, d, pd);
+    load_rows(wis, w_in, (int64_t)N * F * d, d, pd);   // rows (e, j) of W_in
+    load_rows(wos, w_out, (int64_t)N * d * F, F, pf);  // rows (e, k) of W_out
     __syncthreads();
     // router logits, one (token, expert) pair per thread at a time
     for (int q = tid; q < T * N; q += kSmallThreads) {
