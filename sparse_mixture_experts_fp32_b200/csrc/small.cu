@@ -46,31 +46,53 @@ __host__ __device__ inline SmallLayout small_layout(int T, int d, int F, int N) 
 // Copies an [n / cols][cols] float32 matrix into shared-memory rows of `pitch`
 // floats.  Each thread keeps eight 16-byte loads in flight before it stores
 // them (a load-then-store loop left every load's latency exposed).
-__device__ __forceinline__ void load_rows(float *dst, const float *__restrict__ src, int64_t n, int cols, int pitch) {
+// (The layer's arrays hold at most 160 KB here, so 32-bit indices suffice: a
+// 64-bit division per element cost more than the loads.)
+__device__ __forceinline__ void load_rows(float *dst, const float *__restrict__ src, int n, int cols, int pitch) {
     const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
-    const int64_t n4 = vec ? n / 4 : 0;
+    const int n4 = vec ? n / 4 : 0;
     const float4 *s4 = reinterpret_cast<const float4 *>(src);
-    for (int64_t base = threadIdx.x; base < n4; base += 8 * kSmallThreads) {
+    for (int base = threadIdx.x; base < n4; base += 8 * kSmallThreads) {
         float4 v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const int64_t i = base + (int64_t)u * kSmallThreads;
+            const int i = base + u * kSmallThreads;
             if (i < n4) v[u] = __ldg(s4 + i);
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const int64_t i = base + (int64_t)u * kSmallThreads;
+            const int i = base + u * kSmallThreads;
             if (i < n4) {
                 const float c[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                int row = (4 * i) / cols, col = 4 * i - row * cols;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const int64_t k = 4 * i + q;
-                    dst[k / cols * pitch + k % cols] = c[q];
+                    dst[row * pitch + col] = c[q];
+                    if (++col == cols) {
+                        col = 0;
+                        ++row;
+                    }
                 }
             }
         }
     }
-    for (int64_t k = 4 * n4 + threadIdx.x; k < n; k += kSmallThreads) dst[k / cols * pitch + k % cols] = src[k];
+    for (int k = 4 * n4 + threadIdx.x; k < n; k += kSmallThreads) dst[k / cols * pitch + k % cols] = src[k];
+}
+
+// sum_k a[k] b[k] over k < n, in four interleaved partial sums (k mod 4) added
+// as (s0 + s1) + (s2 + s3): four independent FMA chains instead of one.
+__device__ __forceinline__ float dot4(const float *a, const float *b, int n) {
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    int k = 0;
+#pragma unroll 4
+    for (; k + 4 <= n; k += 4) {
+        s0 = fmaf(a[k], b[k], s0);
+        s1 = fmaf(a[k + 1], b[k + 1], s1);
+        s2 = fmaf(a[k + 2], b[k + 2], s2);
+        s3 = fmaf(a[k + 3], b[k + 3], s3);
+    }
+    for (; k < n; ++k) s0 = fmaf(a[k], b[k], s0);
+    return (s0 + s1) + (s2 + s3);
 }
 
 __global__ void __launch_bounds__(kSmallThreads, 1)
@@ -95,17 +117,23 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         status->reserved = 0;
     }
     const int pd = L.pd, pf = L.pf;
-    load_rows(xs, x, (int64_t)T * d, d, pd);
-    load_rows(wrs, w_r, (int64_t)N * d, d, pd);
-    load_rows(wis, w_in, (int64_t)N * F * d, d, pd);   // rows (e, j) of W_in
-    load_rows(wos, w_out, (int64_t)N * d * F, F, pf);  // rows (e, k) of W_out
+    // All four arrays start on their way to L2 at once; then they are staged one after the other.
+    if (tid < 4) {
+        const float *src = tid == 0 ? x : tid == 1 ? w_r : tid == 2 ? w_in : w_out;
+        const int n = tid == 0 ? T * d : tid == 1 ? N * d : N * F * d;
+        const uint32_t bytes = (uint32_t)n * 4u & ~15u;
+        if (bytes > 0 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0)
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+    }
+    load_rows(xs, x, T * d, d, pd);
+    load_rows(wrs, w_r, N * d, d, pd);
+    load_rows(wis, w_in, N * F * d, d, pd);   // rows (e, j) of W_in
+    load_rows(wos, w_out, N * d * F, F, pf);  // rows (e, k) of W_out
     __syncthreads();
     // router logits, one (token, expert) pair per thread at a time
     for (int q = tid; q < T * N; q += kSmallThreads) {
         const int t = q / N, i = q % N;
-        float acc = 0.f;
-        for (int k = 0; k < d; ++k) acc = fmaf(xs[t * pd + k], wrs[i * pd + k], acc);
-        lg[q] = acc + (bias ? bias[i] : 0.f);
+        lg[q] = dot4(xs + t * pd, wrs + i * pd, d) + (bias ? bias[i] : 0.f);
     }
     __syncthreads();
     // softmax, argmax (lowest index on ties), gate: one thread per token
@@ -139,17 +167,25 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         ss[t] = s_;
         slot[t] = s_;
     }
-    // counts and the probability sums per expert (token order, fp64), then aux
-    for (int i = tid; i < N; i += kSmallThreads) {
+    // counts and the probability sums per expert (fp64), then aux
+    // (a warp per expert: lane-strided partial sums, then a fixed xor tree)
+    for (int i = warp; i < N; i += kSmallThreads / 32) {
         int c = 0;
         double p = 0.0;
-        for (int t = 0; t < T; ++t) {
+        for (int t = lane; t < T; t += 32) {
             c += es[t] == i;
             p += (double)lg[t * N + i];
         }
-        cnt_s[i] = c;
-        psum_s[i] = p;
-        counts[i] = c;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            c += __shfl_xor_sync(0xffffffffu, c, off);
+            p += __shfl_xor_sync(0xffffffffu, p, off);
+        }
+        if (lane == 0) {
+            cnt_s[i] = c;
+            psum_s[i] = p;
+            counts[i] = c;
+        }
     }
     __syncthreads();
     if (tid == 0) {
@@ -168,18 +204,10 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         }
         const int e = es[t];
         const float *wi = wis + (int64_t)e * F * pd, *wo = wos + (int64_t)e * d * pf, *xt = xs + t * pd;
-        for (int j = lane; j < F; j += 32) {
-            float acc = 0.f;
-            for (int k = 0; k < d; ++k) acc = fmaf(wi[j * pd + k], xt[k], acc);
-            hrow[j] = fmaxf(acc, 0.f);
-        }
+        for (int j = lane; j < F; j += 32) hrow[j] = fmaxf(dot4(wi + j * pd, xt, d), 0.f);
         __syncwarp();
         const float g = gs[t];
-        for (int k = lane; k < d; k += 32) {
-            float acc = 0.f;
-            for (int j = 0; j < F; ++j) acc = fmaf(wo[k * pf + j], hrow[j], acc);
-            yt[k] = g * acc;
-        }
+        for (int k = lane; k < d; k += 32) yt[k] = g * dot4(wo + k * pf, hrow, F);
         __syncwarp();
     }
 }
