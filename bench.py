@@ -50,6 +50,7 @@ import numpy as np
 ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
+import sparse_mixture_experts_fp32_b200 as swm  # noqa: E402  (flag constants; the library loads lazily)
 from sparse_mixture_experts_fp32_b200 import synth  # noqa: E402
 
 METRIC = "Switch-layer fwd tokens/s on 1 B200; expert GEMM % bf16 peak; route/scatter GB/s"
@@ -217,7 +218,7 @@ def kernel_work(wl, C, counts, pairs=74, flags=0):
         "combine": ("hbm", T * d * 4 + K * d * 4 + 12 * T, T * d * s + K * d * s + 12 * T),
         "dispatch": ("hbm", 2 * K * d * s + 4 * N * C + 4 * N, None),
         "_meta": ("", dict(K=K, E_nz=E_nz, gemm_weight_bytes=2 * E_nz * d * F * s), None),
-    } | ({} if flags & 12 else  # SWITCH_FLAG_GEMM_1CTA | SWITCH_FLAG_FFN_TWO_LAUNCHES: no fused kernel
+    } | ({} if flags & (swm.SWITCH_FLAG_GEMM_1CTA | swm.SWITCH_FLAG_FFN_TWO_LAUNCHES) else  # no fused kernel
           {"ffn_tc_fused": ("tensor", 2.0 * K * F * d, None)} if ffn_two_launches(wl, C, counts, pairs) else
           {"ffn_tc_gemm1_relu": ("?", 0, None)})
 
