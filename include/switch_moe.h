@@ -197,12 +197,19 @@ switch_status_t switch_combine(const switch_dims_t *dims, const void *ybuf, cons
  * above; y [T, d] float32 is the layer output WITHOUT the residual.  On the
  * bfloat16 tensor-core path the dispatch is fused into the slot assignment
  * and both expert GEMMs run in one persistent kernel with the combine in the
- * second GEMM's epilogue.  With SWITCH_FLAG_FFN_TWO_LAUNCHES the result is
- * bit-identical to calling the four steps one by one.  By default, when the
- * second GEMM has few tiles, its tiles are split along d_ff and their parts
- * added into y in a fixed order: routing, counts and aux are unchanged and y
- * differs from the four-step result by float32 rounding only.  Either way
- * identical inputs give identical bytes. */
+ * second GEMM's epilogue; when the second GEMM may have many tiles (12 waves
+ * of 256 x 256 tiles over the SM pairs or more, an upper bound from T, N and
+ * C), the first GEMM also gets its own launch, and the device counts decide
+ * which of the two launches runs it.  With SWITCH_FLAG_FFN_TWO_LAUNCHES the
+ * result is bit-identical to calling the four steps one by one, and so is the
+ * default wherever the second GEMM is not split.  By default, when the second
+ * GEMM has few tiles, its tiles are split along d_ff and their parts added
+ * into y in a fixed order: routing, counts and aux are unchanged and y differs
+ * from the four-step result by float32 rounding only.  Small float32 layers
+ * (T <= 256, N <= 32, everything within 160 KB of shared memory) run in one
+ * thread block instead (SWITCH_FLAG_MULTI_KERNEL keeps the separate steps);
+ * there y differs from the four-step result by float32 rounding only.  Either
+ * way identical inputs give identical bytes. */
 switch_status_t switch_layer_fwd(const switch_dims_t *dims, const void *x, const float *w_r,
                                  const float *logit_bias, const void *w_in, const void *w_out, void *y,
                                  int32_t *expert, float *gate, int32_t *slot, int32_t *counts, float *aux,
