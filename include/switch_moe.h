@@ -57,7 +57,7 @@ typedef enum {
     SWITCH_ERR_DTYPE = 3,          /* unknown dtype code */
     SWITCH_ERR_ALIGN = 4,          /* a pointer is not 16-byte aligned */
     SWITCH_ERR_WORKSPACE = 5,      /* workspace smaller than switch_workspace_size() */
-    SWITCH_ERR_UNSUPPORTED = 6,    /* valid request this build cannot run (e.g. no sm_100 device) */
+    SWITCH_ERR_UNSUPPORTED = 6,    /* valid request the library cannot run (e.g. no sm_100 device) */
     SWITCH_ERR_CUDA = 7,           /* a CUDA runtime call or kernel launch failed */
     SWITCH_ERR_DEVICE_TIMEOUT = 8, /* a kernel gave up a bounded wait (reported by switch_check) */
     SWITCH_ERR_TOO_LARGE = 9       /* switch_route_noalloc: the group needs more scratch than its static buffer */

@@ -98,7 +98,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, Device
 }
 
 // ---------------------------------------------------------------------------
-// TMA (no multicast anywhere in this library)
+// TMA (no multicast loads anywhere in this library)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, uint64_t *bar, int32_t c0,
                                             int32_t c1, int32_t c2) {
@@ -338,7 +338,7 @@ __device__ __forceinline__ void st_cluster_s32(uint32_t cluster_addr, int32_t v)
 
 // TMA 3-D load into this CTA's shared memory whose completion (transaction
 // bytes) is counted on the mbarrier at `bar_cluster_addr`, which may belong
-// to the peer CTA of the pair.  No multicast.
+// to the peer CTA of the pair.  No multicast load.
 __device__ __forceinline__ void tma_load_3d_pair(void *smem_dst, const void *tmap, uint32_t bar_cluster_addr,
                                                  int32_t c0, int32_t c1, int32_t c2) {
     asm volatile(

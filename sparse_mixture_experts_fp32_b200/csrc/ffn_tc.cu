@@ -461,7 +461,7 @@ __device__ __forceinline__ int epilogue_async(uint32_t t_row, int e, int row_bas
 //                       both CTAs and publish the accumulator to both
 //   both CTAs, warps 2-5  epilogue of their own 128 rows, then one arrival
 //                       each on the leader's "accumulator empty" barrier
-// Barrier addresses of the other CTA come from mapa; nothing is multicast.
+// Barrier addresses of the other CTA come from mapa; no load is multicast.
 // ---------------------------------------------------------------------------
 template <int BN, int STAGES>
 struct PairLayout {

@@ -35,7 +35,7 @@
 //              (deterministic: a fixed shuffle tree, then a fixed warp order).
 //              Several warps per SM sub-partition hide the latency of this
 //              per-token chain.
-// Barrier addresses of the other CTA come from mapa; nothing is multicast.
+// Barrier addresses of the other CTA come from mapa; no load is multicast.
 // (An L2 prefetch of the next token tile of x, issued at the start of each
 // tile, made the kernel slower on B200, as it did for the expert GEMMs.)
 #include <cuda.h>
@@ -121,7 +121,7 @@ __device__ __forceinline__ void named_barrier_epilogue() {
 }
 
 // 2-D TMA load into this CTA's shared memory, counted on the mbarrier at
-// `bar_cluster_addr` (the leader's).  No multicast.
+// `bar_cluster_addr` (the leader's).  No multicast load.
 __device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const void *tmap, uint32_t bar_cluster_addr,
                                                  int32_t c0, int32_t c1) {
     asm volatile(
