@@ -209,16 +209,6 @@ __device__ __forceinline__ void bulk_store(void *gmem_dst, const void *smem_src,
                  : "memory");
 }
 
-// Bulk add of fp32 values from shared memory onto global memory (an element-wise
-// reduction performed at the destination; addresses 16-byte aligned, size a
-// multiple of 16).
-__device__ __forceinline__ void bulk_add_f32(float *gmem_dst, const void *smem_src, uint32_t bytes) {
-    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                     reinterpret_cast<uint64_t>(gmem_dst)),
-                 "r"(smem_u32(smem_src)), "r"(bytes)
-                 : "memory");
-}
-
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // out[0..3] += v, one 16-byte float32 reduction in global memory (round to nearest).
