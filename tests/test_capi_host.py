@@ -129,3 +129,31 @@ def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
     monkeypatch.setattr(sm, "LIB_PATH", tmp_path / "missing.so")
     with pytest.raises(RuntimeError, match="not built"):
         sm.lib()
+
+
+def test_training_workspace_holds_the_backward_sections(L):
+    """The training forward keeps what the backward reads; the tensor-core router products add
+    their split operands (dh terms [T][6 Np] for dx, [chunks][3N][Tc] for dW_r, W_r terms
+    [d][6 Np], dW_r partials) and the float32 FMA router path (SWITCH_FLAG_SIMT_ROUTER) only its
+    per-chunk partials.  No transposed copies of weights or activations exist any more."""
+    T, d, F, N, C = 131072, 1024, 4096, 128, 1280
+    base = sm.switch_workspace_size(sm.dims(T, d, F, N, C, sm.SWITCH_BF16))
+    train = sm.switch_workspace_size(sm.dims(T, d, F, N, C, sm.SWITCH_BF16, sm.SWITCH_FLAG_TRAINING))
+    simt = sm.switch_workspace_size(sm.dims(T, d, F, N, C, sm.SWITCH_BF16,
+                                            sm.SWITCH_FLAG_TRAINING | sm.SWITCH_FLAG_SIMT_ROUTER))
+    probs_dh = 2 * T * N * 4
+    grads = N * C * (d + F) * 2                      # dE and dZ, bf16
+    Np, Tc = 128, 2048
+    chunks = T // Tc
+    tc_router = T * 6 * Np * 2 + d * 6 * Np * 2 + chunks * 3 * N * Tc * 2 + chunks * 3 * N * d * 4
+    assert train - base >= probs_dh + grads + tc_router
+    # no room for transposed weights (2 N d F bf16 = 2.1 GB) is reserved
+    assert train - base < probs_dh + grads + tc_router + 64 * (1 << 20)
+    assert simt < train
+    assert simt - base >= probs_dh + grads
+
+
+def test_backward_kernel_names(L):
+    names = {29: "bwd_router_split", 30: "bwd_router_tc_dx", 31: "bwd_router_tc_dw", 32: "bwd_zero_tails"}
+    for k, v in names.items():
+        assert L.switch_kernel_name(k).decode() == v
